@@ -1,0 +1,204 @@
+"""CPU oracle for GGUF Q4_K dequantisation and Q4_K GEMV (ctypes front end).
+
+TEST INFRASTRUCTURE. Only `tests/`, `__graft_entry__.smoke()` and the
+`cpu_baseline` / `--impl reference` legs of `bench.py` may import this package.
+The product library (`gguf_quant_dequant_q4k_b200`) never imports, loads or
+calls it, and the two share no code.
+
+The arithmetic lives in `q4k_oracle.c` (plain C, built with gcc); this file only
+compiles it and marshals numpy arrays. The C file's header states what each
+function follows on the pages and the format readings it takes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "q4k_oracle.c")
+LIB = os.path.join(_HERE, "libq4k_oracle.so")
+
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+
+CFLAGS = ["-O2", "-fPIC", "-shared", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+          "-pthread"]
+
+
+def build(src: str = SRC, out: str = LIB, force: bool = False) -> str:
+    """Compile `src` with gcc into the shared library `out` (only if stale)."""
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(src)):
+        return out
+    tmp = out + ".tmp%d" % os.getpid()
+    subprocess.run(["gcc", *CFLAGS, src, "-o", tmp, "-lm"], check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _p(arr: np.ndarray, ptype):
+    return arr.ctypes.data_as(ptype)
+
+
+def _check_shape(w: np.ndarray, n: int, k: int) -> None:
+    if k <= 0 or k % 256 or n <= 0:
+        raise ValueError(f"bad Q4_K shape n={n} k={k}")
+    if w.dtype != np.uint8 or not w.flags.c_contiguous or w.size != n * (k // 256) * 144:
+        raise ValueError("w must be contiguous uint8 of n*(k/256)*144 bytes")
+
+
+def _rows(rows, n: int) -> np.ndarray:
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1)
+    if rows.size and (rows.min() < 0 or rows.max() >= n):
+        raise ValueError("row index out of range")
+    return rows
+
+
+class Oracle:
+    """One loaded copy of the oracle library."""
+
+    def __init__(self, path: str):
+        L = ctypes.CDLL(path)
+        L.q4k_oracle_half_to_double.argtypes = [ctypes.c_uint16]
+        L.q4k_oracle_half_to_double.restype = ctypes.c_double
+        L.q4k_oracle_unpack.argtypes = [_u8p, _u16p, _u16p, _i32p, _i32p, _i32p]
+        L.q4k_oracle_unpack.restype = None
+        L.q4k_oracle_pack.argtypes = [ctypes.c_uint16, ctypes.c_uint16, _i32p, _i32p, _i32p,
+                                      _u8p]
+        L.q4k_oracle_pack.restype = None
+        L.q4k_oracle_dequant_f32.argtypes = [_u8p, ctypes.c_int64, ctypes.c_int64, _f32p]
+        L.q4k_oracle_dequant_f32.restype = None
+        L.q4k_oracle_dequant_rows.argtypes = [_u8p, ctypes.c_int64, _i64p, ctypes.c_int64,
+                                              _f32p]
+        L.q4k_oracle_dequant_rows.restype = None
+        L.q4k_oracle_gemv.argtypes = [_u8p, _f32p, ctypes.c_int32, ctypes.c_int64,
+                                      ctypes.c_int64, _f64p, _f64p, ctypes.c_int32]
+        L.q4k_oracle_gemv.restype = ctypes.c_int
+        L.q4k_oracle_gemv_rows.argtypes = [_u8p, _f32p, ctypes.c_int32, ctypes.c_int64, _i64p,
+                                           ctypes.c_int64, _f64p, _f64p]
+        L.q4k_oracle_gemv_rows.restype = None
+        self.L = L
+        self.path = path
+
+    def half_to_double(self, bits: int) -> float:
+        return self.L.q4k_oracle_half_to_double(int(bits) & 0xFFFF)
+
+    def unpack(self, sb: np.ndarray):
+        """One 144-byte superblock -> (d_bits, dmin_bits, sc[8], m[8], q[256])."""
+        sb = np.ascontiguousarray(sb, dtype=np.uint8).reshape(-1)
+        if sb.size != 144:
+            raise ValueError("a superblock is 144 bytes")
+        d = ctypes.c_uint16()
+        dm = ctypes.c_uint16()
+        sc = np.zeros(8, np.int32)
+        mn = np.zeros(8, np.int32)
+        q = np.zeros(256, np.int32)
+        self.L.q4k_oracle_unpack(_p(sb, _u8p), ctypes.byref(d), ctypes.byref(dm),
+                                 _p(sc, _i32p), _p(mn, _i32p), _p(q, _i32p))
+        return d.value, dm.value, sc, mn, q
+
+    def pack(self, d_bits: int, dmin_bits: int, sc, mn, q) -> np.ndarray:
+        """Integer fields -> one 144-byte superblock (the inverse of `unpack`)."""
+        sc = np.ascontiguousarray(sc, dtype=np.int32)
+        mn = np.ascontiguousarray(mn, dtype=np.int32)
+        q = np.ascontiguousarray(q, dtype=np.int32)
+        out = np.zeros(144, np.uint8)
+        self.L.q4k_oracle_pack(int(d_bits), int(dmin_bits), _p(sc, _i32p), _p(mn, _i32p),
+                               _p(q, _i32p), _p(out, _u8p))
+        return out
+
+    def dequant_f32(self, w: np.ndarray, n: int, k: int) -> np.ndarray:
+        """Dequantised W as an (n, k) float32 array."""
+        w = np.ascontiguousarray(w, dtype=np.uint8).reshape(-1)
+        _check_shape(w, n, k)
+        out = np.empty((n, k), np.float32)
+        self.L.q4k_oracle_dequant_f32(_p(w, _u8p), n, k, _p(out, _f32p))
+        return out
+
+    def dequant_rows(self, w: np.ndarray, n: int, k: int, rows) -> np.ndarray:
+        """Dequantised rows `rows` of W as a (len(rows), k) float32 array."""
+        w = np.ascontiguousarray(w, dtype=np.uint8).reshape(-1)
+        _check_shape(w, n, k)
+        rows = _rows(rows, n)
+        out = np.empty((rows.size, k), np.float32)
+        self.L.q4k_oracle_dequant_rows(_p(w, _u8p), k, _p(rows, _i64p), rows.size,
+                                       _p(out, _f32p))
+        return out
+
+    def gemv(self, w: np.ndarray, x: np.ndarray, n: int, k: int, nthreads: int = 1):
+        """(y, a): y = W x in double, a = sum |w x| per element; both (m, n) float64."""
+        w = np.ascontiguousarray(w, dtype=np.uint8).reshape(-1)
+        _check_shape(w, n, k)
+        x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1, k)
+        m = x.shape[0]
+        y = np.empty((m, n), np.float64)
+        a = np.empty((m, n), np.float64)
+        rc = self.L.q4k_oracle_gemv(_p(w, _u8p), _p(x, _f32p), m, n, k, _p(y, _f64p),
+                                    _p(a, _f64p), int(nthreads))
+        if rc != 0:
+            raise RuntimeError("oracle could not start its threads")
+        return y, a
+
+    def gemv_rows(self, w: np.ndarray, x: np.ndarray, n: int, k: int, rows):
+        """(y, a) for the listed rows only: both (m, len(rows)) float64."""
+        w = np.ascontiguousarray(w, dtype=np.uint8).reshape(-1)
+        _check_shape(w, n, k)
+        x = np.ascontiguousarray(x, dtype=np.float32).reshape(-1, k)
+        rows = _rows(rows, n)
+        m = x.shape[0]
+        y = np.empty((m, rows.size), np.float64)
+        a = np.empty((m, rows.size), np.float64)
+        self.L.q4k_oracle_gemv_rows(_p(w, _u8p), _p(x, _f32p), m, k, _p(rows, _i64p),
+                                    rows.size, _p(y, _f64p), _p(a, _f64p))
+        return y, a
+
+
+_default: Oracle | None = None
+
+
+def default() -> Oracle:
+    """The oracle built from `q4k_oracle.c` in this directory."""
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def half_to_double(bits):
+    return default().half_to_double(bits)
+
+
+def unpack(sb):
+    return default().unpack(sb)
+
+
+def pack(d_bits, dmin_bits, sc, mn, q):
+    return default().pack(d_bits, dmin_bits, sc, mn, q)
+
+
+def dequant_f32(w, n, k):
+    return default().dequant_f32(w, n, k)
+
+
+def dequant_rows(w, n, k, rows):
+    return default().dequant_rows(w, n, k, rows)
+
+
+def gemv(w, x, n, k, nthreads=1):
+    return default().gemv(w, x, n, k, nthreads)
+
+
+def gemv_rows(w, x, n, k, rows):
+    return default().gemv_rows(w, x, n, k, rows)
+
+
+def tolerance(a: np.ndarray) -> np.ndarray:
+    """Per-element GEMV bound |y_gpu - y_ref| <= 1e-4 * sum|w x| + 1e-6."""
+    return 1e-4 * np.asarray(a) + 1e-6
