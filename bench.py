@@ -1,0 +1,438 @@
+"""Benchmark: Q4_K GEMV (m = 1) over the decode N x K sweep on B200.
+
+One step = one q4k_gemv call for each of the 8 decode projections of the
+1.5B / 7B / 8B classes (N x K: 8960x1536, 1536x8960, 1536x1536, 11008x4096,
+4096x11008, 4096x4096, 4096x14336, 128256x4096), inputs already in HBM.
+value = bytes counted per step / device time per step, in GB/s, with
+bytes = N*K/256*144 + 4*m*(K+N) per call.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs the same sweep on its own GPU (replicas:
+the GEMV needs no exchange); value sums the bytes of all ranks over the slowest
+rank's time. `--impl reference` times the CPU oracle instead (rank 0 only).
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import q4k_synth  # noqa: E402
+
+METRIC = ("Q4_K GEMV µs/call & achieved HBM GB/s (% of B200 peak), m=1, "
+          "N×K sweep")
+SWEEP = q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B + q4k_synth.SHAPES_8B
+WORKLOAD = ("Q4_K GEMV m=1 decode sweep, one call per projection: "
+            + ", ".join(f"{n}x{k}" for n, k in SWEEP))
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+GRAPH_STEPS = 10
+
+
+def bytes_counted(n: int, k: int, m: int = 1) -> int:
+    return n * k // 256 * 144 + 4 * m * (k + n)
+
+
+BYTES_PER_STEP = sum(bytes_counted(n, k) for n, k in SWEEP)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest() -> str:
+    """Hash of the CUDA sources, to tell whether committed ncu counters still apply."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gguf_quant_dequant_q4k_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """DRAM bytes per step from the committed ncu summary, if it matches the sources."""
+    path = os.path.join(ROOT, "profiles", "q4k_gemv_sweep_traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_digest") != source_digest():
+        return None
+    return t.get("dram_bytes_per_step")
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid: str | None):
+        self.proc = None
+        self.out = None
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "50"]
+            if gpu_uuid:
+                cmd += ["-i", gpu_uuid]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [v.strip() for v in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def oracle_sample_rows(frac: float):
+    return [(n, k, max(1, int(round(n * frac)))) for n, k in SWEEP]
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    threads = max(1, min(cores, 64))
+    problems = []
+    for n, k in SWEEP:
+        # the same bytes the GPU arm streams, first rows only (a bounded sample)
+        w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS[(n, k)])
+        problems.append((n, k, w, x))
+
+    def step(frac):
+        nbytes = 0
+        for n, k, w, x in problems:
+            rows = max(1, int(round(n * frac)))
+            wrows = w[: rows * (k // 256) * 144]
+            oracle.gemv(wrows, x, rows, k, nthreads=threads)
+            nbytes += bytes_counted(rows, k)
+        return nbytes
+
+    # size the sample so the whole run stays within about two minutes
+    t0 = time.perf_counter()
+    probe = 0.002
+    step(probe)
+    per_frac = (time.perf_counter() - t0) / probe
+    budget = min(2.0, 120.0 / max(1, args.steps + args.warmup))
+    frac = min(1.0, max(1e-4, budget / per_frac))
+    for _ in range(args.warmup):
+        step(frac)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += step(frac)
+    dt = time.perf_counter() - t0
+    value = nbytes / dt / 1e9
+    sample = (f"first {frac:.2%} of the rows of each of the 8 sweep projections per step "
+              f"(CPU oracle, {threads} threads, double accumulation)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "m": 1, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline() -> dict:
+    """The oracle as it stands on this host's cores: one full pass of the sweep."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    threads = max(1, min(cores, 64))
+    nbytes, dt = 0, 0.0
+    for n, k in SWEEP:
+        w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS[(n, k)])
+        t0 = time.perf_counter()
+        oracle.gemv(w, x, n, k, nthreads=threads)
+        dt += time.perf_counter() - t0
+        nbytes += bytes_counted(n, k)
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": "one full pass of the 8-projection sweep (all rows), row-parallel "
+                      f"over {threads} threads, {dt:.2f} s"}
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args) -> None:
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import gguf_quant_dequant_q4k_b200 as q4k
+
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 << 20))
+    stream = torch.cuda.Stream(device=dev)
+
+    # inputs: per projection, enough copies of W that each copy is re-read only
+    # after more than 2 x L2 of other traffic
+    shapes = []
+    for n, k in SWEEP:
+        w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS[(n, k)])
+        wdev = torch.from_numpy(w).to(dev)
+        copies = max(2, -(-2 * l2 // w.nbytes) + 1)
+        ws = [wdev] + [wdev.clone() for _ in range(copies - 1)]
+        xdev = torch.from_numpy(x).to(dev)
+        ydev = torch.empty((1, n), dtype=torch.float32, device=dev)
+        shapes.append({"n": n, "k": k, "ws": ws, "x": xdev, "y": ydev, "x_host": x})
+    torch.cuda.synchronize(dev)
+    plans = [q4k.q4k_gemv_plan_for(1, s["n"], s["k"], props.multi_processor_count)
+             for s in shapes]
+    launches_per_step = sum(p["launches"] for p in plans)
+
+    def sweep(step_index: int):
+        for s in shapes:
+            w = s["ws"][step_index % 2]
+            q4k.q4k_gemv(w, s["x"], s["y"], 1, s["n"], s["k"], stream=stream)
+
+    # CUDA graph of GRAPH_STEPS steps (copies alternate step to step)
+    use_graph = not args.no_graph
+    graph = None
+    if use_graph:
+        with torch.cuda.stream(stream):
+            sweep(0)  # make sure per-device set-up happened outside capture
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for i in range(GRAPH_STEPS):
+                sweep(i)
+
+    def run_steps(count: int):
+        if use_graph:
+            reps = count // GRAPH_STEPS
+            with torch.cuda.stream(stream):
+                for _ in range(reps):
+                    graph.replay()
+            for i in range(count - reps * GRAPH_STEPS):
+                sweep(i)
+        else:
+            for i in range(count):
+                sweep(i)
+
+    # warm-up
+    run_steps(max(args.warmup, 3))
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(str(getattr(props, "uuid", "")) or None) if rank == 0 else None
+    if sampler is not None:
+        time.sleep(0.15)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run_steps(args.steps)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler is not None else None
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * BYTES_PER_STEP * args.steps / (ms * 1e-3) / 1e9
+
+    # per-projection us/call: R back-to-back calls over rotating copies
+    per_shape = []
+    peak, peak_kind = measured_peak()
+    for s, p in zip([] if args.skip_extras else shapes, plans):
+        reps = 200
+        with torch.cuda.stream(stream):
+            for i in range(10):
+                q4k.q4k_gemv(s["ws"][i % len(s["ws"])], s["x"], s["y"], 1, s["n"], s["k"],
+                             stream=stream)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(reps):
+            q4k.q4k_gemv(s["ws"][i % len(s["ws"])], s["x"], s["y"], 1, s["n"], s["k"],
+                         stream=stream)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        us = a0.elapsed_time(a1) * 1e3 / reps
+        b = bytes_counted(s["n"], s["k"])
+        per_shape.append({"n": s["n"], "k": s["k"], "us_per_call": round(us, 3),
+                          "gbs": round(b / us / 1e3, 1), "frac_of_measured": round(b / us / 1e3 / peak, 4),
+                          "frac_of_nominal": round(b / us / 1e3 / NOMINAL_HBM_GBS, 4),
+                          "w_copies": len(s["ws"]), "kernel": p["kernel"], "grid": p["grid"],
+                          "k_splits": p["k_splits"]})
+
+    # end to end through the public API: pinned x -> device, gemv, y -> pinned host
+    e2e_steps = 0 if args.skip_extras else min(args.steps, 500)
+    xs_pinned = [torch.from_numpy(s["x_host"]).pin_memory() for s in shapes]
+    ys_pinned = [torch.empty((1, s["n"]), dtype=torch.float32).pin_memory() for s in shapes]
+    h2d = sum(x.numel() * 4 for x in xs_pinned)
+    d2h = sum(y.numel() * 4 for y in ys_pinned)
+
+    def e2e_step(i):
+        with torch.cuda.stream(stream):
+            for s, xp, yp in zip(shapes, xs_pinned, ys_pinned):
+                s["x"].copy_(xp, non_blocking=True)
+                q4k.q4k_gemv(s["ws"][i % 2], s["x"], s["y"], 1, s["n"], s["k"], stream=stream)
+                yp.copy_(s["y"], non_blocking=True)
+
+    for i in range(3 if e2e_steps else 0):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    b1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = b0.elapsed_time(b1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = (world * BYTES_PER_STEP * e2e_steps / (e2e_ms * 1e-3) / 1e9
+                 if e2e_steps else None)
+
+    if world > 1:
+        dist.barrier()
+        graph = None
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    achieved = BYTES_PER_STEP / (ms_per_step * 1e-3) / 1e9   # per GPU, all launches of a step
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic: seeded Q4_K superblocks (d, dmin fp16 of U[1e-3,2e-2], random "
+                "scale and quant bytes), x ~ N(0,1) f32",
+        "config": {
+            "workload": WORKLOAD, "m": 1, "bytes_per_step": BYTES_PER_STEP,
+            "bytes_rule": "N*K/256*144 + 4*m*(K+N) per call",
+            "l2": f"inputs larger than L2: {BYTES_PER_STEP / 1e6:.0f} MB of Q4_K per step, two "
+                  f"rotating copies of every W, so each copy is re-read after "
+                  f"~{2 * BYTES_PER_STEP / 1e6:.0f} MB (L2 {l2 / 2**20:.0f} MiB)",
+            "launch": (f"CUDA graph of {GRAPH_STEPS} steps, replayed" if use_graph
+                       else "eager launches"),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "per_shape": per_shape,
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
+            "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
+            "traffic": committed_traffic(), "algorithmic_bytes": BYTES_PER_STEP,
+            "per": "one step = the 8 q4k_gemv launches of the sweep",
+            "kernel": "q4k_gemv",
+        },
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "how": "per call: pinned x -> device copy, q4k_gemv, y -> pinned host copy, "
+                       "eager through the ctypes API"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-graph", action="store_true", help="eager launches (for profilers)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shapes", default=None,
+                    help="comma-separated NxK subset of the sweep (profiling runs only)")
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="skip the per-shape and end-to-end passes (profiling runs only)")
+    args = ap.parse_args()
+    if args.steps < 1 or args.warmup < 0:
+        raise SystemExit("--steps must be >= 1 and --warmup >= 0")
+    if args.shapes:
+        global SWEEP, BYTES_PER_STEP, WORKLOAD
+        SWEEP = [tuple(int(v) for v in s.lower().split("x")) for s in args.shapes.split(",")]
+        for sh in SWEEP:
+            if sh not in q4k_synth.SEEDS:
+                raise SystemExit(f"shape {sh} is not one of the sweep's")
+        BYTES_PER_STEP = sum(bytes_counted(n, k) for n, k in SWEEP)
+        WORKLOAD = "subset of the sweep: " + ", ".join(f"{n}x{k}" for n, k in SWEEP)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,135 @@
+"""ctypes binding of libq4k_b200.so: the C ABI of include/q4k.h, same names.
+
+Argument marshalling only: torch tensors (or raw integer device addresses) are
+turned into pointers and the current torch CUDA stream into a cudaStream_t;
+every step of the computation runs in the library's CUDA kernels. There is no
+fallback: if the library is missing this module raises on import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libq4k_b200.so")
+
+Q4K_OK = 0
+Q4K_ERR_NULL = 1
+Q4K_ERR_SHAPE = 2
+Q4K_ERR_ALIGN = 3
+Q4K_ERR_UNSUPPORTED_M = 4
+Q4K_ERR_CUDA = 5
+Q4K_ERR_OVERLAP = 6
+Q4K_QK = 256
+Q4K_BLOCK_BYTES = 144
+Q4K_MAX_M = 8
+Q4K_KERNEL_ROWS = 1
+Q4K_KERNEL_SPLITK = 2
+
+# Every function include/q4k.h declares.
+EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
+           "q4k_last_cuda_error", "q4k_gemv_plan_for")
+
+
+class Q4KError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = f"{what}: {q4k_status_string(status)} (status {status})"
+        if status == Q4K_ERR_CUDA:
+            msg += f", cudaError {q4k_last_cuda_error()}"
+        super().__init__(msg)
+
+
+class q4k_gemv_plan(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int), ("grid", ctypes.c_int), ("block", ctypes.c_int),
+                ("smem_bytes", ctypes.c_int), ("k_splits", ctypes.c_int),
+                ("launches", ctypes.c_int), ("units", ctypes.c_longlong),
+                ("units_per_cta_max", ctypes.c_longlong)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m gguf_quant_dequant_q4k_b200.build` "
+                      "(or __graft_entry__.build()). There is no CPU fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp = ctypes.c_void_p
+_lib.q4k_gemv.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp]
+_lib.q4k_gemv.restype = ctypes.c_int
+_lib.q4k_dequant_f32.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp]
+_lib.q4k_dequant_f32.restype = ctypes.c_int
+_lib.q4k_weight_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
+_lib.q4k_weight_bytes.restype = ctypes.c_size_t
+_lib.q4k_status_string.argtypes = [ctypes.c_int]
+_lib.q4k_status_string.restype = ctypes.c_char_p
+_lib.q4k_last_cuda_error.argtypes = []
+_lib.q4k_last_cuda_error.restype = ctypes.c_int
+_lib.q4k_gemv_plan_for.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.POINTER(q4k_gemv_plan)]
+_lib.q4k_gemv_plan_for.restype = ctypes.c_int
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def q4k_weight_bytes(n: int, k: int) -> int:
+    return _lib.q4k_weight_bytes(int(n), int(k))
+
+
+def q4k_status_string(status: int) -> str:
+    return _lib.q4k_status_string(int(status)).decode()
+
+
+def q4k_last_cuda_error() -> int:
+    return _lib.q4k_last_cuda_error()
+
+
+def q4k_gemv_plan_for(m: int, n: int, k: int, num_sms: int) -> dict:
+    plan = q4k_gemv_plan()
+    st = _lib.q4k_gemv_plan_for(int(m), int(n), int(k), int(num_sms), ctypes.byref(plan))
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_gemv_plan_for")
+    return plan.as_dict()
+
+
+def q4k_gemv_status(w, x, y, m: int, n: int, k: int, stream=None) -> int:
+    """Raw status of the C call (no exception)."""
+    return _lib.q4k_gemv(_ptr(w), _ptr(x), _ptr(y), int(m), int(n), int(k), _stream(stream))
+
+
+def q4k_gemv(w, x, y, m: int, n: int, k: int, stream=None) -> None:
+    """y[m, n] = W[n, k] x[m, k] on `stream` (default: torch's current stream)."""
+    st = q4k_gemv_status(w, x, y, m, n, k, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_gemv")
+
+
+def q4k_dequant_f32_status(w, out, n: int, k: int, stream=None) -> int:
+    return _lib.q4k_dequant_f32(_ptr(w), _ptr(out), int(n), int(k), _stream(stream))
+
+
+def q4k_dequant_f32(w, out, n: int, k: int, stream=None) -> None:
+    """out[n, k] = dequantised W (f32) on `stream` (default: torch's current stream)."""
+    st = q4k_dequant_f32_status(w, out, n, k, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_dequant_f32")

@@ -1,0 +1,133 @@
+// q4k_api.cu -- the extern "C" entry points declared in include/q4k.h:
+// argument validation, status codes and per-device set-up.
+//
+// Validation follows the pages' host wrappers: a null device pointer is
+// refused before launch (`q4k_gemv_indexed_async`, "realizar 0.8.5,
+// src/cuda/executor/q4k_gemv_cached.rs"); K must be a multiple of 256
+// (`batched_q4k_gemv_into`, "realizar 0.8.5, src/cuda/executor/uses.rs") and is
+// refused rather than padded; the byte size N*(K/256)*144 is computed with
+// overflow checks (`validate_block_quant_embedding`, "turbospark-runtime
+// 0.1.0, src/real_forward_dispatch.rs"); more than 8 vectors is refused rather
+// than looped (`encode_gemm_any`, same page); a failed launch returns an error
+// code to the caller (the rc convention of "memra-engine 0.83.1,
+// src/f16_ffi.rs").
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "q4k_internal.h"
+
+namespace q4k {
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+DeviceInfo g_dev[kMaxDevices];
+int g_dev_status[kMaxDevices];
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Weight bytes n*(k/256)*144 in 64 bits; 0 for an invalid shape.
+size_t weight_bytes_checked(int n, int k) {
+    if (n <= 0 || k <= 0 || (k % Q4K_QK) != 0) return 0;
+    return static_cast<size_t>(n) * static_cast<size_t>(k / Q4K_QK) * Q4K_BLOCK_BYTES;
+}
+
+}  // namespace
+
+int cuda_failure(cudaError_t e) {
+    t_last_cuda_error = static_cast<int>(e);
+    return Q4K_ERR_CUDA;
+}
+
+int current_device_info(DeviceInfo* info) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_failure(e);
+    if (dev < 0 || dev >= kMaxDevices) return cuda_failure(cudaErrorInvalidDevice);
+    std::call_once(g_dev_once[dev], [dev] {
+        DeviceInfo d{};
+        cudaError_t e1 = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        cudaError_t e2 = cudaDeviceGetAttribute(&d.max_smem_optin,
+                                                cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        g_dev[dev] = d;
+        g_dev_status[dev] = (e1 != cudaSuccess) ? static_cast<int>(e1)
+                                                : static_cast<int>(e2);
+    });
+    if (g_dev_status[dev] != 0) return cuda_failure(static_cast<cudaError_t>(g_dev_status[dev]));
+    *info = g_dev[dev];
+    return Q4K_OK;
+}
+
+}  // namespace q4k
+
+using namespace q4k;
+
+extern "C" {
+
+size_t q4k_weight_bytes(int n, int k) { return weight_bytes_checked(n, k); }
+
+const char* q4k_status_string(int status) {
+    switch (status) {
+        case Q4K_OK: return "ok";
+        case Q4K_ERR_NULL: return "null pointer argument";
+        case Q4K_ERR_SHAPE: return "invalid shape (need n > 0, k > 0, k % 256 == 0)";
+        case Q4K_ERR_ALIGN: return "misaligned pointer (w, x, out: 16 bytes; y: 4 bytes)";
+        case Q4K_ERR_UNSUPPORTED_M: return "unsupported number of vectors (need 1 <= m <= 8)";
+        case Q4K_ERR_CUDA: return "CUDA runtime error (see q4k_last_cuda_error)";
+        case Q4K_ERR_OVERLAP: return "output overlaps an input";
+        default: return "unknown status";
+    }
+}
+
+int q4k_last_cuda_error(void) { return t_last_cuda_error; }
+
+int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
+    if (plan == nullptr) return Q4K_ERR_NULL;
+    if (weight_bytes_checked(n, k) == 0 || num_sms <= 0) return Q4K_ERR_SHAPE;
+    if (m < 1 || m > Q4K_MAX_M) return Q4K_ERR_UNSUPPORTED_M;
+    return plan_gemv(m, n, k, num_sms, plan);
+}
+
+int q4k_gemv(const void* w, const float* x, float* y, int m, int n, int k,
+             q4k_stream_t stream) {
+    if (w == nullptr || x == nullptr || y == nullptr) return Q4K_ERR_NULL;
+    const size_t wbytes = weight_bytes_checked(n, k);
+    if (wbytes == 0) return Q4K_ERR_SHAPE;
+    if (m < 1 || m > Q4K_MAX_M) return Q4K_ERR_UNSUPPORTED_M;
+    if (!aligned(w, 16) || !aligned(x, 16) || !aligned(y, 4)) return Q4K_ERR_ALIGN;
+    const size_t xbytes = static_cast<size_t>(m) * static_cast<size_t>(k) * sizeof(float);
+    const size_t ybytes = static_cast<size_t>(m) * static_cast<size_t>(n) * sizeof(float);
+    if (overlaps(y, ybytes, w, wbytes) || overlaps(y, ybytes, x, xbytes)) return Q4K_ERR_OVERLAP;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    q4k_gemv_plan plan;
+    st = plan_gemv(m, n, k, dev.sm_count, &plan);
+    if (st != Q4K_OK) return st;
+    return launch_gemv(plan, w, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4k_dequant_f32(const void* w, float* out, int n, int k, q4k_stream_t stream) {
+    if (w == nullptr || out == nullptr) return Q4K_ERR_NULL;
+    const size_t wbytes = weight_bytes_checked(n, k);
+    if (wbytes == 0) return Q4K_ERR_SHAPE;
+    if (!aligned(w, 16) || !aligned(out, 16)) return Q4K_ERR_ALIGN;
+    const size_t obytes = static_cast<size_t>(n) * static_cast<size_t>(k) * sizeof(float);
+    if (overlaps(out, obytes, w, wbytes)) return Q4K_ERR_OVERLAP;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return launch_dequant(w, out, n, k, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,129 @@
+// q4k_gemv.cu -- y = W x for Q4_K W and 1..8 f32 vectors (q4k_gemv).
+//
+// First implementation: one warp per output row (the row-per-warp mapping of
+// the pages' `Q4KGemv`, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs",
+// grid (n,1) x 32 threads), with each decoded weight applied to all m vectors
+// (`BatchedQ4KGemv`, "realizar 0.8.5, src/cuda/executor/uses.rs": dequantise
+// once, multiply by M input vectors).
+//
+// Per step a warp covers 4 superblocks of its row: lane = 8*sb + c, where
+// c = 0..7 selects the 16-byte slice 16c..16c+15 of Q. That slice's byte l
+// carries weight 64g+16h+l (low nibble, sub-block 2g) and weight 64g+32+16h+l
+// (high nibble, sub-block 2g+1), with g = c/2, h = c%2. The warp's 32 quant
+// loads are 4 x 128 contiguous bytes.
+#include "q4k_internal.h"
+#include "q4k_superblock.cuh"
+
+namespace q4k {
+
+namespace {
+
+constexpr int kRowsThreads = 256;
+
+template <int M>
+__global__ void __launch_bounds__(kRowsThreads)
+q4k_gemv_rows_kernel(const uint8_t* __restrict__ w, const float* __restrict__ x,
+                     float* __restrict__ y, int n, int k) {
+    const int nsb = k / kQK;
+    const int lane = threadIdx.x & 31;
+    const int c = lane & 7, sub = lane >> 3, g = c >> 1, h = c & 1;
+    const int warp = (blockIdx.x * kRowsThreads + threadIdx.x) >> 5;
+    const int nwarps = gridDim.x * (kRowsThreads / 32);
+    for (int row = warp; row < n; row += nwarps) {
+        float acc[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) acc[i] = 0.f;
+        const uint8_t* wr = w + static_cast<size_t>(row) * nsb * kBlockBytes;
+        for (int b = sub; b < nsb; b += 4) {
+            const uint8_t* sb = wr + static_cast<size_t>(b) * kBlockBytes;
+            const Header hd = decode_header(ldg_nc_v4(sb));
+            const uint4 qv = ldg_nc_v4(sb + kQsOffset + 16 * c);
+            float dsc0, dm0, dsc1, dm1;
+            subblock_coeffs(hd, 2 * g, dsc0, dm0);
+            subblock_coeffs(hd, 2 * g + 1, dsc1, dm1);
+            const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
+            float wl[16], wh[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const uint32_t byte = (words[e >> 2] >> (8 * (e & 3))) & 0xFFu;
+                wl[e] = weight_value(dsc0, dm0, byte & 15u);
+                wh[e] = weight_value(dsc1, dm1, byte >> 4);
+            }
+            const int k0 = b * kQK + 64 * g + 16 * h;
+#pragma unroll
+            for (int i = 0; i < M; ++i) {
+                const float4* xl = reinterpret_cast<const float4*>(x + static_cast<size_t>(i) * k + k0);
+                const float4* xh = xl + 8;  // +32 floats
+                float s = acc[i];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const float4 a = __ldg(xl + v);
+                    const float4 bq = __ldg(xh + v);
+                    s = fmaf(wl[4 * v + 0], a.x, s);
+                    s = fmaf(wl[4 * v + 1], a.y, s);
+                    s = fmaf(wl[4 * v + 2], a.z, s);
+                    s = fmaf(wl[4 * v + 3], a.w, s);
+                    s = fmaf(wh[4 * v + 0], bq.x, s);
+                    s = fmaf(wh[4 * v + 1], bq.y, s);
+                    s = fmaf(wh[4 * v + 2], bq.z, s);
+                    s = fmaf(wh[4 * v + 3], bq.w, s);
+                }
+                acc[i] = s;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            float s = acc[i];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
+            if (lane == 0) y[static_cast<size_t>(i) * n + row] = s;
+        }
+    }
+}
+
+template <int M>
+void launch_rows(const q4k_gemv_plan& plan, const void* w, const float* x, float* y, int n,
+                 int k, cudaStream_t stream) {
+    q4k_gemv_rows_kernel<M><<<plan.grid, plan.block, 0, stream>>>(
+        static_cast<const uint8_t*>(w), x, y, n, k);
+}
+
+}  // namespace
+
+int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
+    (void)m;
+    (void)k;
+    const int warps_per_cta = kRowsThreads / 32;
+    long long ctas = (static_cast<long long>(n) + warps_per_cta - 1) / warps_per_cta;
+    const long long cap = static_cast<long long>(num_sms) * 8;
+    if (ctas > cap) ctas = cap;
+    const long long warps = ctas * warps_per_cta;
+    plan->kernel = Q4K_KERNEL_ROWS;
+    plan->grid = static_cast<int>(ctas);
+    plan->block = kRowsThreads;
+    plan->smem_bytes = 0;
+    plan->k_splits = 1;
+    plan->launches = 1;
+    plan->units = n;
+    plan->units_per_cta_max = ((n + warps - 1) / warps) * warps_per_cta;
+    return Q4K_OK;
+}
+
+int launch_gemv(const q4k_gemv_plan& plan, const void* w, const float* x, float* y, int m,
+                int n, int k, cudaStream_t stream) {
+    switch (m) {
+        case 1: launch_rows<1>(plan, w, x, y, n, k, stream); break;
+        case 2: launch_rows<2>(plan, w, x, y, n, k, stream); break;
+        case 3: launch_rows<3>(plan, w, x, y, n, k, stream); break;
+        case 4: launch_rows<4>(plan, w, x, y, n, k, stream); break;
+        case 5: launch_rows<5>(plan, w, x, y, n, k, stream); break;
+        case 6: launch_rows<6>(plan, w, x, y, n, k, stream); break;
+        case 7: launch_rows<7>(plan, w, x, y, n, k, stream); break;
+        case 8: launch_rows<8>(plan, w, x, y, n, k, stream); break;
+        default: return Q4K_ERR_UNSUPPORTED_M;
+    }
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+}
+
+}  // namespace q4k

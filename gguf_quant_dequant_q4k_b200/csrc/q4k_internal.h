@@ -1,0 +1,32 @@
+// q4k_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/q4k.h"
+
+namespace q4k {
+
+// Per-device facts the launch planner needs, read once per device.
+struct DeviceInfo {
+    int sm_count;
+    int max_smem_optin;  // largest dynamic shared memory a CTA may opt in to
+};
+
+// Returns Q4K_OK and fills *info for the current device, or Q4K_ERR_CUDA.
+int current_device_info(DeviceInfo* info);
+
+// Records `e` as the calling thread's last CUDA error and returns Q4K_ERR_CUDA.
+int cuda_failure(cudaError_t e);
+
+// Host-only launch planning (no CUDA calls).
+int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan);
+
+// Enqueue the planned kernels. Arguments are already validated.
+int launch_gemv(const q4k_gemv_plan& plan, const void* w, const float* x, float* y, int m,
+                int n, int k, cudaStream_t stream);
+
+int launch_dequant(const void* w, float* out, int n, int k, int num_sms, cudaStream_t stream);
+
+}  // namespace q4k

@@ -1,0 +1,150 @@
+/*
+ * q4k.h -- C ABI of libq4k_b200.so: GGUF Q4_K GEMV and dequantisation on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (y = W x with W stored as Q4_K superblocks, decoded on the fly)
+ * is the one the realizar pages launch as `Q4KGemv`, `TiledQ4KGemv`,
+ * `ChunkedTiledQ4KGemv`, `MwvQ4KGemv` ("realizar 0.8.5,
+ * src/cuda/executor/q4k_gemv_cached.rs": `q4k_gemv_cached`,
+ * `q4k_gemv_indexed_async`) and `BatchedQ4KGemv` for up to 8 vectors
+ * ("realizar 0.8.5, src/cuda/executor/uses.rs": `batched_q4k_gemv_into`).
+ * The dequantisation is the one "memra-engine 0.83.1, src/f16_ffi.rs" declares
+ * as `memra_q4_K_dequant_f16` (Q4_K 144-byte superblocks to a row-major
+ * mirror), here with an f32 target.
+ *
+ * Q4_K superblock (256 weights, 144 bytes; the pages give the size, the field
+ * layout is GGUF's block_q4_K):
+ *     bytes   0..1   d     binary16, little-endian
+ *     bytes   2..3   dmin  binary16, little-endian
+ *     bytes   4..15  S[12] eight 6-bit scales sc_j and eight 6-bit mins m_j
+ *                          (j < 4: sc_j = S[j]&63, m_j = S[j+4]&63;
+ *                           j >= 4: sc_j = (S[j+4]&15) | (S[j-4]>>6)<<4,
+ *                                   m_j  = (S[j+4]>>4) | (S[j]>>6)<<4)
+ *     bytes  16..143 Q[128] byte Q[32g+l] holds weight 64g+l (low nibble) and
+ *                          weight 64g+32+l (high nibble), g = 0..3, l = 0..31
+ *     weight t (sub-block j = t/32): value = d*sc_j*q_t - dmin*m_j
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer is DEVICE memory owned by the caller; the library never
+ *     allocates, frees or keeps a pointer after the call returns.
+ *   - W is row-major by output row: row r is K/256 consecutive superblocks,
+ *     N*(K/256)*144 bytes in all ("weights: N x K/256 Q4_K super-blocks",
+ *     `batched_q4k_gemv_into` doc comment). K must be a positive multiple of
+ *     256; nothing is padded.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream) and the
+ *     call returns without synchronising; no host copy, allocation or JIT
+ *     happens inside a call (the pages sync and copy to the host only in their
+ *     debugging wrappers, and preload modules because compiling during graph
+ *     capture fails).
+ *   - Arguments are validated before anything is enqueued; an invalid call
+ *     returns a status and enqueues nothing (a null weight pointer "poisons
+ *     the CUDA context" if launched, `q4k_gemv_indexed_async`). A status of
+ *     Q4K_ERR_CUDA means the launch itself failed; q4k_last_cuda_error()
+ *     then returns the cudaError_t. Faults during execution surface at the
+ *     caller's next synchronisation, as for any asynchronous CUDA work.
+ *   - Output buffers must not overlap any input (checked: Q4K_ERR_OVERLAP).
+ */
+#ifndef Q4K_H
+#define Q4K_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define Q4K_API __attribute__((visibility("default")))
+#else
+#define Q4K_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *q4k_stream_t;
+
+enum q4k_status {
+    Q4K_OK = 0,
+    Q4K_ERR_NULL = 1,           /* a required pointer is NULL                     */
+    Q4K_ERR_SHAPE = 2,          /* n <= 0, k <= 0, k % 256 != 0, or size overflow  */
+    Q4K_ERR_ALIGN = 3,          /* w or x not 16-byte aligned, y/out not 4-byte    */
+    Q4K_ERR_UNSUPPORTED_M = 4,  /* m outside 1..Q4K_MAX_M                          */
+    Q4K_ERR_CUDA = 5,           /* a CUDA runtime call failed (see last_cuda_error) */
+    Q4K_ERR_OVERLAP = 6         /* an output range overlaps an input range         */
+};
+
+#define Q4K_QK 256          /* weights per superblock */
+#define Q4K_BLOCK_BYTES 144 /* bytes per superblock   */
+#define Q4K_MAX_M 8         /* most vectors per q4k_gemv call */
+
+/*
+ * y = W x for m vectors.
+ *   w  : N*(K/256)*144 bytes of Q4_K superblocks, row-major by output row,
+ *        16-byte aligned.
+ *   x  : m x K float32, row-major (vector i at x + i*K), 16-byte aligned
+ *        ("input: M x K row-major", `batched_q4k_gemv_into`).
+ *   y  : m x N float32, row-major (vector i at y + i*N); fully overwritten,
+ *        never accumulated into ("output: M x N row-major").
+ *   m  : 1..8 vectors. Larger m is refused, not looped (the turbospark page,
+ *        "turbospark-runtime 0.1.0, src/real_forward_dispatch.rs",
+ *        `encode_gemm_any`, refuses rather than silently looping).
+ * Accuracy: per element |y - sum_k w_nk x_ik| <= 1e-4 * sum_k |w_nk x_ik| + 1e-6,
+ * where w_nk is the f32 value d*sc*q - dmin*m; accumulation is in f32.
+ * Weight reads may start before the previous kernel on `stream` has finished
+ * (programmatic dependent launch): x is read and y written only after it has.
+ * W is treated as constant model data: it must not be written by work still
+ * pending on `stream` when this is called.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_gemv(const void *w, const float *x, float *y, int m, int n, int k,
+             q4k_stream_t stream);
+
+/*
+ * out = W dequantised to float32, row-major n x k (out[r*k + t] is weight t of
+ * row r). Each value is d*sc*q - dmin*m rounded once to f32 (the products are
+ * exact in f32), so results are bit-reproducible.
+ *   w  : as for q4k_gemv (16-byte aligned).
+ *   out: n*k floats, 16-byte aligned, must not overlap w.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_dequant_f32(const void *w, float *out, int n, int k, q4k_stream_t stream);
+
+/* Bytes of an n x k Q4_K matrix: n*(k/256)*144; 0 if n <= 0, k <= 0 or
+ * k % 256 != 0 (the size rule the memra `build_q8_f16` and turbospark
+ * `encode_gemv_any` pages check before every Q4_K launch). */
+Q4K_API size_t q4k_weight_bytes(int n, int k);
+
+/* A static, NUL-terminated description of a q4k_status value. */
+Q4K_API const char *q4k_status_string(int status);
+
+/* The cudaError_t behind the most recent Q4K_ERR_CUDA returned on the calling
+ * thread (0 if none). */
+Q4K_API int q4k_last_cuda_error(void);
+
+/*
+ * How q4k_gemv would run a problem on a GPU with `num_sms` SMs (host-only, no
+ * CUDA call). Fills *plan and returns Q4K_OK, or the status q4k_gemv would
+ * return for these sizes.
+ */
+typedef struct q4k_gemv_plan {
+    int kernel;          /* Q4K_KERNEL_* below                                  */
+    int grid;            /* CTAs of the main kernel                             */
+    int block;           /* threads per CTA                                     */
+    int smem_bytes;      /* dynamic shared memory per CTA                       */
+    int k_splits;        /* parts K is cut into (1 = no split)                  */
+    int launches;        /* kernels one call enqueues                           */
+    long long units;     /* work units (row x K-part) shared out among the CTAs */
+    long long units_per_cta_max; /* most units any CTA processes                */
+} q4k_gemv_plan;
+
+enum q4k_kernel {
+    Q4K_KERNEL_ROWS = 1,        /* whole rows per CTA, bulk-copy streamed         */
+    Q4K_KERNEL_SPLITK = 2       /* K split across CTAs + second-stage reduce       */
+};
+
+Q4K_API int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan *plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4K_H */

@@ -1,0 +1,243 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on a B200.
+
+GEMV: |y_gpu - y_ref| <= 1e-4 * sum|w x| + 1e-6 per element (y_ref in double).
+Dequant: bit-exact f32 (NaN compared as NaN: its payload is not part of the
+format's value).
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import q4k_synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+NTHREADS = max(1, len(os.sched_getaffinity(0)))
+
+
+@pytest.fixture(scope="module")
+def q4k():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gguf_quant_dequant_q4k_b200 as lib
+    return lib
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def gpu_gemv(q4k, w, x, n, k, wt=None):
+    x = np.ascontiguousarray(x, np.float32).reshape(-1, k)
+    m = x.shape[0]
+    wt = dev(w) if wt is None else wt
+    xt = dev(x)
+    y = torch.full((m, n), float("nan"), dtype=torch.float32, device="cuda")
+    q4k.q4k_gemv(wt, xt, y, m, n, k)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def gpu_dequant(q4k, w, n, k, wt=None):
+    wt = dev(w) if wt is None else wt
+    out = torch.full((n, k), float("nan"), dtype=torch.float32, device="cuda")
+    q4k.q4k_dequant_f32(wt, out, n, k)
+    torch.cuda.synchronize()
+    return out
+
+
+def assert_gemv_close(y, yref, a, what=""):
+    err = np.abs(y.astype(np.float64) - yref)
+    tol = oracle.tolerance(a)
+    bad = ~(err <= tol)
+    assert not bad.any(), (f"{what}: {bad.sum()} elements out of tolerance; worst "
+                           f"err/tol={np.nanmax(err / tol):.3g}")
+
+
+def assert_bitexact(got, ref, what=""):
+    got = np.asarray(got, np.float32)
+    ref = np.asarray(ref, np.float32)
+    gn, rn = np.isnan(got), np.isnan(ref)
+    assert np.array_equal(gn, rn), f"{what}: NaN positions differ"
+    gb, rb = got[~gn].view(np.uint32), ref[~rn].view(np.uint32)
+    bad = gb != rb
+    assert not bad.any(), f"{what}: {bad.sum()} values differ bitwise"
+
+
+# --------------------------------------------------------------------------- dequant
+
+@pytest.mark.parametrize("n,k", [(1, 256), (3, 768), (33, 256), (256, 1024), (1536, 1536),
+                                 (8960, 1536), (4096, 11008)])
+def test_dequant_bitexact(q4k, n, k):
+    w, _ = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS.get((n, k), 100 + n))
+    got = gpu_dequant(q4k, w, n, k).cpu().numpy()
+    assert_bitexact(got, oracle.dequant_f32(w, n, k), f"{n}x{k}")
+
+
+def test_dequant_raw_random_bytes(q4k):
+    """Every byte random, d and dmin included: subnormals, infinities, NaNs."""
+    n, k = 64, 1024
+    w = q4k_synth.random_bytes(n * (k // 256) * 144, 21)
+    assert_bitexact(gpu_dequant(q4k, w, n, k).cpu().numpy(), oracle.dequant_f32(w, n, k))
+
+
+def test_dequant_lm_head_sampled_rows(q4k):
+    n, k = 128256, 4096
+    w, _ = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS[(n, k)])
+    out = gpu_dequant(q4k, w, n, k)
+    rows = np.unique(np.concatenate([[0, 1, n - 2, n - 1],
+                                     np.random.default_rng(3).integers(0, n, 60)]))
+    got = out[torch.from_numpy(rows).cuda()].cpu().numpy()
+    assert_bitexact(got, oracle.dequant_rows(w, n, k, rows))
+
+
+# --------------------------------------------------------------------------- GEMV, m = 1
+
+CONFIG_SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
+                 + q4k_synth.SHAPES_8B)
+
+
+@pytest.mark.parametrize("n,k", CONFIG_SHAPES)
+def test_gemv_config_shapes(q4k, n, k):
+    w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS[(n, k)])
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k, nthreads=NTHREADS)
+    assert_gemv_close(y, yref, a, f"{n}x{k}")
+
+
+@pytest.mark.parametrize("n,k", [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280),
+                                 (33, 2304), (37, 8960), (129, 256), (1, 14336), (3, 11008),
+                                 (97, 4352), (300, 3840)])
+def test_gemv_ragged_shapes(q4k, n, k):
+    w, x = q4k_synth.q4k_problem(n, k, 1, 1000 + n + k)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(y, yref, a, f"{n}x{k}")
+
+
+# --------------------------------------------------------------------------- GEMV, m > 1
+
+@pytest.mark.parametrize("m", range(1, 9))
+@pytest.mark.parametrize("n,k", [(33, 512), (200, 1792)])
+def test_gemv_every_m_small(q4k, n, k, m):
+    w, x = q4k_synth.q4k_problem(n, k, m, 7 * m + n)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
+
+
+@pytest.mark.parametrize("m", [1, 2, 4, 8])
+@pytest.mark.parametrize("n,k", q4k_synth.SHAPES_MULTIVEC)
+def test_gemv_multivector_shapes(q4k, n, k, m):
+    w, x = q4k_synth.q4k_problem(n, k, m, q4k_synth.SEED_MULTIVEC[(n, k)])
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k, nthreads=NTHREADS)
+    assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
+
+
+def test_gemv_32_layer_sweep_sampled(q4k):
+    """All 224 projections of the 32-layer 8B-class decode sweep, each layer's
+    weights seeded independently; the oracle checks 8 sampled rows of each."""
+    rng = np.random.default_rng(5)
+    for layer in range(32):
+        for proj, (n, k) in enumerate(q4k_synth.LAYER_8B):
+            w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.layer_seed(layer, proj))
+            y = gpu_gemv(q4k, w, x, n, k)
+            assert np.isfinite(y).all()
+            rows = np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, 6)]))
+            yref, a = oracle.gemv_rows(w, x, n, k, rows)
+            assert_gemv_close(y[:, rows], yref, a, f"layer {layer} proj {proj}")
+
+
+# --------------------------------------------------------------------------- special inputs
+
+def test_gemv_zero_vector_gives_exact_zero(q4k):
+    n, k = 300, 4096
+    w, _ = q4k_synth.q4k_problem(n, k, 1, 31)
+    y = gpu_gemv(q4k, w, np.zeros((1, k), np.float32), n, k)
+    assert (y == 0).all()
+
+
+def test_gemv_unit_vectors_give_columns(q4k):
+    n, k = 257, 2048
+    w, _ = q4k_synth.q4k_problem(n, k, 1, 32)
+    deq = oracle.dequant_f32(w, n, k)
+    cols = [0, 31, 32, 63, 64, 255, 256, 1000, 2047]
+    x = np.zeros((len(cols), k), np.float32)
+    for i, c in enumerate(cols[:8]):
+        x[i, c] = 1.0
+    y = gpu_gemv(q4k, w, x[:8], n, k)
+    for i, c in enumerate(cols[:8]):
+        assert_gemv_close(y[i], deq[:, c].astype(np.float64), np.abs(deq[:, c]).astype(np.float64),
+                          f"column {c}")
+
+
+def _cancelling_block():
+    # sc_j = 4, m_j = 60, every q = 15, d = dmin  =>  every weight is exactly 0
+    S = np.array([4, 4, 4, 4, 60 | 0xC0, 60 | 0xC0, 60 | 0xC0, 60 | 0xC0,
+                  0xC4, 0xC4, 0xC4, 0xC4], np.uint8)
+    b = np.zeros(144, np.uint8)
+    b[0:2] = b[2:4] = np.array([0x66, 0x2E], np.uint8)   # binary16 0x2E66, about 0.1
+    b[4:16] = S
+    b[16:] = 0xFF
+    return b
+
+
+def test_gemv_cancelling_blocks(q4k):
+    """Rows whose weights are all exactly 0 by cancellation (d*sc*q == dmin*m):
+    the contract's bound there is the 1e-6 absolute floor."""
+    n, k = 40, 4096
+    w, x = q4k_synth.q4k_problem(n, k, 2, 33)
+    sb = w.reshape(n, k // 256, 144)
+    sb[::3] = _cancelling_block()          # every third row cancels exactly
+    w = sb.reshape(-1)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert (yref[:, ::3] == 0).all()
+    y = gpu_gemv(q4k, w, x * 10, n, k)      # large activations stress the floor
+    yref, a = oracle.gemv(w, x * 10, n, k)
+    assert_gemv_close(y, yref, a, "cancelling")
+
+
+def test_gemv_deterministic(q4k):
+    n, k = 4096, 11008
+    w, x = q4k_synth.q4k_problem(n, k, 3, 34)
+    wt = dev(w)
+    y1 = gpu_gemv(q4k, w, x, n, k, wt=wt)
+    y2 = gpu_gemv(q4k, w, x, n, k, wt=wt)
+    assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+
+
+def test_gemv_offsets_guard_band_and_stream(q4k):
+    """W at a 16-byte (not 256-byte) offset inside a larger buffer, y with guard
+    elements around it, launched on a side stream: only y[0:m*n] changes."""
+    n, k, m = 77, 1536, 3
+    w, x = q4k_synth.q4k_problem(n, k, m, 35)
+    wbuf = torch.zeros(w.size + 64, dtype=torch.uint8, device="cuda")
+    wbuf[16:16 + w.size] = dev(w)
+    xbuf = torch.zeros(m * k + 8, dtype=torch.float32, device="cuda")
+    xbuf[4:4 + m * k] = dev(x.reshape(-1))
+    ybuf = torch.full((m * n + 64,), 7.0, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        q4k.q4k_gemv(wbuf.data_ptr() + 16, xbuf.data_ptr() + 16, ybuf.data_ptr() + 4 * 32,
+                     m, n, k, stream=s)
+    s.synchronize()
+    yb = ybuf.cpu().numpy()
+    assert (yb[:32] == 7.0).all() and (yb[32 + m * n:] == 7.0).all()
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(yb[32:32 + m * n].reshape(m, n), yref, a, "offsets")
+
+
+def test_invalid_arguments_on_gpu_enqueue_nothing(q4k):
+    n, k = 16, 512
+    wt = torch.zeros(q4k.q4k_weight_bytes(n, k), dtype=torch.uint8, device="cuda")
+    xt = torch.zeros(k, dtype=torch.float32, device="cuda")
+    y = torch.full((n,), 3.0, device="cuda")
+    assert q4k.q4k_gemv_status(wt, xt, y, 9, n, k) == q4k.Q4K_ERR_UNSUPPORTED_M
+    assert q4k.q4k_gemv_status(wt.data_ptr() + 8, xt, y, 1, n, k) == q4k.Q4K_ERR_ALIGN
+    assert q4k.q4k_gemv_status(wt, xt, y, 1, n, 500) == q4k.Q4K_ERR_SHAPE
+    torch.cuda.synchronize()
+    assert (y == 3.0).all()
