@@ -278,7 +278,10 @@ def run_ours(args) -> None:
     run_steps(max(args.warmup, 3))
     torch.cuda.synchronize(dev)
 
-    sampler = ClockSampler(str(getattr(props, "uuid", "")) or None) if rank == 0 else None
+    uuid = str(getattr(props, "uuid", "") or "")
+    if uuid and not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+    sampler = ClockSampler(uuid or None) if rank == 0 else None
     if sampler is not None:
         time.sleep(0.15)
     if world > 1:
@@ -324,7 +327,7 @@ def run_ours(args) -> None:
                           "gbs": round(b / us / 1e3, 1), "frac_of_measured": round(b / us / 1e3 / peak, 4),
                           "frac_of_nominal": round(b / us / 1e3 / NOMINAL_HBM_GBS, 4),
                           "w_copies": len(s["ws"]), "kernel": p["kernel"], "grid": p["grid"],
-                          "k_splits": p["k_splits"]})
+                          "teams": p["teams"], "depth": p["depth"]})
 
     # end to end through the public API: pinned x -> device, gemv, y -> pinned host
     e2e_steps = 0 if args.skip_extras else min(args.steps, 500)

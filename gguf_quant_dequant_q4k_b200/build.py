@@ -1,6 +1,7 @@
 """Builds libq4k_b200.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-Usage: python -m gguf_quant_dequant_q4k_b200.build [--force]
+Usage: python gguf_quant_dequant_q4k_b200/build.py [--force] [-v]
+(run it by path: importing the package needs the library this builds)
 """
 from __future__ import annotations
 

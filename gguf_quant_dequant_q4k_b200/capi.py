@@ -23,12 +23,12 @@ Q4K_ERR_OVERLAP = 6
 Q4K_QK = 256
 Q4K_BLOCK_BYTES = 144
 Q4K_MAX_M = 8
-Q4K_KERNEL_ROWS = 1
-Q4K_KERNEL_SPLITK = 2
+Q4K_KERNEL_WARP_ROWS = 1
+Q4K_KERNEL_STREAM = 2
 
 # Every function include/q4k.h declares.
 EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
-           "q4k_last_cuda_error", "q4k_gemv_plan_for")
+           "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags")
 
 
 class Q4KError(RuntimeError):
@@ -42,7 +42,7 @@ class Q4KError(RuntimeError):
 
 class q4k_gemv_plan(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int), ("grid", ctypes.c_int), ("block", ctypes.c_int),
-                ("smem_bytes", ctypes.c_int), ("k_splits", ctypes.c_int),
+                ("smem_bytes", ctypes.c_int), ("teams", ctypes.c_int), ("depth", ctypes.c_int),
                 ("launches", ctypes.c_int), ("units", ctypes.c_longlong),
                 ("units_per_cta_max", ctypes.c_longlong)]
 
@@ -51,7 +51,7 @@ class q4k_gemv_plan(ctypes.Structure):
 
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is not built; run `python -m gguf_quant_dequant_q4k_b200.build` "
+    raise ImportError(f"{LIB_PATH} is not built; run `python gguf_quant_dequant_q4k_b200/build.py` "
                       "(or __graft_entry__.build()). There is no CPU fallback.")
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -69,6 +69,8 @@ _lib.q4k_last_cuda_error.restype = ctypes.c_int
 _lib.q4k_gemv_plan_for.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.POINTER(q4k_gemv_plan)]
 _lib.q4k_gemv_plan_for.restype = ctypes.c_int
+_lib.q4k_device_fault_flags.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+_lib.q4k_device_fault_flags.restype = ctypes.c_int
 
 
 def library() -> ctypes.CDLL:
@@ -110,6 +112,15 @@ def q4k_gemv_plan_for(m: int, n: int, k: int, num_sms: int) -> dict:
     if st != Q4K_OK:
         raise Q4KError(st, "q4k_gemv_plan_for")
     return plan.as_dict()
+
+
+def q4k_device_fault_flags() -> int:
+    """Reads and clears the current device's kernel fault flags (synchronises)."""
+    v = ctypes.c_uint(0)
+    st = _lib.q4k_device_fault_flags(ctypes.byref(v))
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_device_fault_flags")
+    return v.value
 
 
 def q4k_gemv_status(w, x, y, m: int, n: int, k: int, stream=None) -> int:

@@ -17,6 +17,7 @@
 #include <mutex>
 
 #include "q4k_internal.h"
+#include "q4k_stream.h"
 
 namespace q4k {
 
@@ -49,6 +50,8 @@ int cuda_failure(cudaError_t e) {
     return Q4K_ERR_CUDA;
 }
 
+int q4k_last_cuda_error_value() { return t_last_cuda_error; }
+
 int current_device_info(DeviceInfo* info) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -62,6 +65,8 @@ int current_device_info(DeviceInfo* info) {
         g_dev[dev] = d;
         g_dev_status[dev] = (e1 != cudaSuccess) ? static_cast<int>(e1)
                                                 : static_cast<int>(e2);
+        if (g_dev_status[dev] == 0 && stream_set_attributes() != Q4K_OK)
+            g_dev_status[dev] = q4k_last_cuda_error_value();
     });
     if (g_dev_status[dev] != 0) return cuda_failure(static_cast<cudaError_t>(g_dev_status[dev]));
     *info = g_dev[dev];
@@ -91,6 +96,11 @@ const char* q4k_status_string(int status) {
 
 int q4k_last_cuda_error(void) { return t_last_cuda_error; }
 
+int q4k_device_fault_flags(unsigned int* flags) {
+    if (flags == nullptr) return Q4K_ERR_NULL;
+    return read_fault_flags(flags);
+}
+
 int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
     if (plan == nullptr) return Q4K_ERR_NULL;
     if (weight_bytes_checked(n, k) == 0 || num_sms <= 0) return Q4K_ERR_SHAPE;
@@ -111,10 +121,7 @@ int q4k_gemv(const void* w, const float* x, float* y, int m, int n, int k,
     DeviceInfo dev;
     int st = current_device_info(&dev);
     if (st != Q4K_OK) return st;
-    q4k_gemv_plan plan;
-    st = plan_gemv(m, n, k, dev.sm_count, &plan);
-    if (st != Q4K_OK) return st;
-    return launch_gemv(plan, w, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
+    return launch_gemv(dev, w, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int q4k_dequant_f32(const void* w, float* out, int n, int k, q4k_stream_t stream) {

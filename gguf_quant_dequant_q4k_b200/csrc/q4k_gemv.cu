@@ -1,6 +1,6 @@
 // q4k_gemv.cu -- y = W x for Q4_K W and 1..8 f32 vectors (q4k_gemv).
 //
-// First implementation: one warp per output row (the row-per-warp mapping of
+// General path (any K, m <= 8): one warp per output row (the row-per-warp mapping of
 // the pages' `Q4KGemv`, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs",
 // grid (n,1) x 32 threads), with each decoded weight applied to all m vectors
 // (`BatchedQ4KGemv`, "realizar 0.8.5, src/cuda/executor/uses.rs": dequantise
@@ -12,6 +12,7 @@
 // (high nibble, sub-block 2g+1), with g = c/2, h = c%2. The warp's 32 quant
 // loads are 4 x 128 contiguous bytes.
 #include "q4k_internal.h"
+#include "q4k_stream.h"
 #include "q4k_superblock.cuh"
 
 namespace q4k {
@@ -90,27 +91,52 @@ void launch_rows(const q4k_gemv_plan& plan, const void* w, const float* x, float
 
 }  // namespace
 
-int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
-    (void)m;
-    (void)k;
+int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, q4k_gemv_plan* plan,
+                     StreamParams* sp) {
+    StreamParams q{};
+    int grid = 0, block = 0, smem = 0;
+    if (plan_stream(m, n, k, num_sms, max_smem, &q, &grid, &block, &smem)) {
+        plan->kernel = Q4K_KERNEL_STREAM;
+        plan->grid = grid;
+        plan->block = block;
+        plan->smem_bytes = smem;
+        plan->teams = q.teams;
+        plan->depth = q.depth;
+        plan->launches = 1;
+        plan->units = n;
+        plan->units_per_cta_max = q.rows_base + (q.rows_extra > 0 ? 1 : 0);
+        if (sp) *sp = q;
+        return Q4K_OK;
+    }
     const int warps_per_cta = kRowsThreads / 32;
     long long ctas = (static_cast<long long>(n) + warps_per_cta - 1) / warps_per_cta;
     const long long cap = static_cast<long long>(num_sms) * 8;
     if (ctas > cap) ctas = cap;
     const long long warps = ctas * warps_per_cta;
-    plan->kernel = Q4K_KERNEL_ROWS;
+    plan->kernel = Q4K_KERNEL_WARP_ROWS;
     plan->grid = static_cast<int>(ctas);
     plan->block = kRowsThreads;
     plan->smem_bytes = 0;
-    plan->k_splits = 1;
+    plan->teams = 0;
+    plan->depth = 0;
     plan->launches = 1;
     plan->units = n;
     plan->units_per_cta_max = ((n + warps - 1) / warps) * warps_per_cta;
     return Q4K_OK;
 }
 
-int launch_gemv(const q4k_gemv_plan& plan, const void* w, const float* x, float* y, int m,
-                int n, int k, cudaStream_t stream) {
+int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
+    return plan_gemv_device(m, n, k, num_sms, kB200SmemOptin, plan, nullptr);
+}
+
+int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n,
+                int k, cudaStream_t stream) {
+    q4k_gemv_plan plan;
+    StreamParams sp;
+    int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin, &plan, &sp);
+    if (st != Q4K_OK) return st;
+    if (plan.kernel == Q4K_KERNEL_STREAM)
+        return launch_stream(sp, plan.grid, plan.block, plan.smem_bytes, w, x, y, m, stream);
     switch (m) {
         case 1: launch_rows<1>(plan, w, x, y, n, k, stream); break;
         case 2: launch_rows<2>(plan, w, x, y, n, k, stream); break;

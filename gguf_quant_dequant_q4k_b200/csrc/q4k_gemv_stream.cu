@@ -1,0 +1,493 @@
+// q4k_gemv_stream.cu -- the streaming Q4_K GEMV for m = 1, 2 and K <= 32768.
+//
+// What it computes: y[i][r] = sum_k W[r][k] x[i][k] with W in Q4_K, as the
+// pages' `Q4KGemv` / `TiledQ4KGemv` / `ChunkedTiledQ4KGemv` / `MwvQ4KGemv`
+// family ("realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs") and
+// `BatchedQ4KGemv` ("realizar 0.8.5, src/cuda/executor/uses.rs"). The pages'
+// designs stage x in shared memory per CTA (K*4 bytes, capped at 48 KB by
+// `MAX_TILED_K`) and give each CTA 4 output rows; this kernel is laid out for
+// B200 instead:
+//
+// * Work split. One persistent CTA per SM owns a balanced, contiguous range of
+//   whole rows (counts differ by at most one). The CTA's warps form T "teams";
+//   the CTA's superblocks (rows x K/256, contiguous in memory) are cut into T
+//   equal contiguous pieces at superblock granularity, one per team, so every
+//   team streams the same number of bytes. A row cut between two teams is
+//   finished from the teams' partial sums in shared memory, in team order
+//   (deterministic; no atomics, no global workspace).
+// * x-stationary. A team has ceil(K/1024) warps: team lane l owns the 16-byte
+//   quant slice c = l%8 of superblock position b = l/8 of every row, i.e. 32
+//   fixed weights of K (16 low nibbles of sub-block 2g and 16 high nibbles of
+//   sub-block 2g+1, g = c/2). Its 32 x values per vector live in registers for
+//   the whole kernel, so x costs no shared-memory bandwidth per row and there
+//   is no K*4-byte shared-memory ceiling.
+// * Streaming. Each team streams its byte range through a ring of `depth`
+//   shared-memory stages with 1-D bulk async copies (cp.async.bulk, completing
+//   on an mbarrier; no multicast). A stage is up to 4 consecutive row segments
+//   (one contiguous copy). Every weight byte is read from HBM once. The first
+//   `depth` copies are issued before griddepcontrol.wait, so under
+//   programmatic dependent launch they overlap the previous kernel's tail.
+// * Decode. Once per stage the team decodes each superblock header (d, dmin,
+//   12 scale bytes; GGUF get_scale_min_k4 packing) into eight (A_j, B_j)
+//   pairs with A_j = 128*d*sc_j (exact) and B_j = -(A_j + dmin*m_j). A weight
+//   with quant q is then A_j*f + B_j where f = 1 + q/128 is built by one byte
+//   permute into the mantissa of 1.0 (exact): d*sc_j*q - dmin*m_j rounded
+//   once (B_j's own rounding, at most half an ulp of 128*d*sc_j + dmin*m_j, is
+//   the only other error). Weights and dot products use packed f32x2 FMAs.
+// * Reduction. Per stage each lane holds one partial per row segment; a
+//   4-segment transpose-reduce across the warp (5 shuffles) leaves one value
+//   per segment, and the team's warps are summed in shared memory.
+//
+// Synchronisation per stage: wait on the stage's mbarrier (bounded), decode,
+// one named barrier per team; the team leader then refills the stage consumed
+// in the previous iteration and finishes the previous stage's row sums.
+#include <cstdint>
+#include <cuda_fp16.h>
+
+#include "q4k_internal.h"
+#include "q4k_sm100.cuh"
+#include "q4k_stream.h"
+#include "q4k_superblock.cuh"
+
+namespace q4k {
+
+namespace {
+
+// Set by a kernel whose bounded wait on a bulk copy gave up; read and cleared by
+// q4k_device_fault_flags(). Never set in normal operation.
+__device__ unsigned int g_fault_flags = 0;
+
+constexpr int kSeg = kStreamSegRows;  // row segments per stage
+constexpr uint32_t kMagicOne = 0x3F000000u;  // bytes 0,1 = 0x00, byte 3 = 0x3F
+
+// f = 1 + q/128 for the nibble held in byte `sel` of `masked` (whose bytes are
+// 0x80 | q): the byte becomes bits 16..23 of 0x3F8?0000.
+template <int SEL>
+__device__ __forceinline__ float nib_to_f(uint32_t masked) {
+    return __uint_as_float(__byte_perm(masked, kMagicOne, 0x7054 | (SEL << 8)));
+}
+
+struct TeamRange {
+    long long s0, s1;   // superblock range [s0, s1) in flat (row*nsb + b) units
+    long long row0;     // first row touched
+    int nseg;           // rows touched
+    int nstages;
+};
+
+__device__ __forceinline__ TeamRange team_range(const StreamParams& p, int team) {
+    const long long cta = blockIdx.x;
+    const long long rows = p.rows_base + (cta < p.rows_extra ? 1 : 0);
+    const long long row_begin = cta * p.rows_base + (cta < p.rows_extra ? cta : p.rows_extra);
+    const long long S0 = row_begin * p.nsb;
+    const long long L = rows * p.nsb;
+    TeamRange r;
+    r.s0 = S0 + (L * team) / p.teams;
+    r.s1 = S0 + (L * (team + 1)) / p.teams;
+    if (r.s1 > r.s0) {
+        r.row0 = r.s0 / p.nsb;
+        r.nseg = static_cast<int>((r.s1 - 1) / p.nsb - r.row0 + 1);
+        r.nstages = (r.nseg + kSeg - 1) / kSeg;
+    } else {
+        r.row0 = 0;
+        r.nseg = 0;
+        r.nstages = 0;
+    }
+    return r;
+}
+
+__device__ __forceinline__ long long seg_begin(const TeamRange& r, int i, int nsb) {
+    const long long b = (r.row0 + i) * nsb;
+    return b > r.s0 ? b : r.s0;
+}
+
+__device__ __forceinline__ long long seg_end(const TeamRange& r, int i, int nsb) {
+    const long long e = (r.row0 + i + 1) * nsb;
+    return e < r.s1 ? e : r.s1;
+}
+
+// Decode one superblock header into 16 floats: (A_j, B_j), j = 0..7.
+__device__ __forceinline__ void decode_coefs(const uint8_t* sb, float* out) {
+    const uint4 h = *reinterpret_cast<const uint4*>(sb);
+    const Header hd = decode_header(h);
+    const float d128 = hd.d * 128.0f;
+    float c[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t scw = (j < 4) ? hd.sc_lo : hd.sc_hi;
+        const uint32_t mw = (j < 4) ? hd.m_lo : hd.m_hi;
+        const float a = d128 * small_u32_to_f32(byte_of(scw, j & 3));
+        const float dm = hd.dmin * small_u32_to_f32(byte_of(mw, j & 3));
+        c[2 * j] = a;
+        c[2 * j + 1] = -(a + dm);
+    }
+    float4* o = reinterpret_cast<float4*>(out);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) o[v] = make_float4(c[4 * v], c[4 * v + 1], c[4 * v + 2], c[4 * v + 3]);
+}
+
+// Sum over this lane's 32 weights of one row: returns (low-nibble, high-nibble)
+// accumulator pairs added into acc_lo / acc_hi for each vector.
+template <int M>
+__device__ __forceinline__ void dot_item(uint4 q, float4 cf, const float2 (&xlo)[M][8],
+                                         const float2 (&xhi)[M][8], float2 (&acc)[M][2]) {
+    const float2 alo = make_float2(cf.x, cf.x), blo = make_float2(cf.y, cf.y);
+    const float2 ahi = make_float2(cf.z, cf.z), bhi = make_float2(cf.w, cf.w);
+    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+        const uint32_t w = words[wi];
+        const uint32_t lo = (w & 0x0F0F0F0Fu) | 0x80808080u;
+        const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+        const float2 flo0 = make_float2(nib_to_f<0>(lo), nib_to_f<1>(lo));
+        const float2 flo1 = make_float2(nib_to_f<2>(lo), nib_to_f<3>(lo));
+        const float2 fhi0 = make_float2(nib_to_f<0>(hi), nib_to_f<1>(hi));
+        const float2 fhi1 = make_float2(nib_to_f<2>(hi), nib_to_f<3>(hi));
+        const float2 wlo0 = ffma2(alo, flo0, blo);
+        const float2 wlo1 = ffma2(alo, flo1, blo);
+        const float2 whi0 = ffma2(ahi, fhi0, bhi);
+        const float2 whi1 = ffma2(ahi, fhi1, bhi);
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            acc[i][0] = ffma2(wlo0, xlo[i][2 * wi], acc[i][0]);
+            acc[i][0] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][0]);
+            acc[i][1] = ffma2(whi0, xhi[i][2 * wi], acc[i][1]);
+            acc[i][1] = ffma2(whi1, xhi[i][2 * wi + 1], acc[i][1]);
+        }
+    }
+}
+
+// 4 values per lane -> each lane holds the warp sum of value index
+// ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1).
+__device__ __forceinline__ float transpose_reduce4(float s0, float s1, float s2, float s3,
+                                                   int lane) {
+    const bool up = (lane & 16) != 0;
+    float a0 = up ? s2 : s0, a1 = up ? s3 : s1;
+    const float b0 = up ? s0 : s2, b1 = up ? s1 : s3;
+    a0 += __shfl_xor_sync(0xFFFFFFFFu, b0, 16);
+    a1 += __shfl_xor_sync(0xFFFFFFFFu, b1, 16);
+    const bool up8 = (lane & 8) != 0;
+    float k = up8 ? a1 : a0;
+    const float snd = up8 ? a0 : a1;
+    k += __shfl_xor_sync(0xFFFFFFFFu, snd, 8);
+    k += __shfl_xor_sync(0xFFFFFFFFu, k, 4);
+    k += __shfl_xor_sync(0xFFFFFFFFu, k, 2);
+    k += __shfl_xor_sync(0xFFFFFFFFu, k, 1);
+    return k;
+}
+
+template <int M>
+__global__ void __launch_bounds__(stream_max_threads(M), 1)
+q4k_gemv_stream_kernel(const StreamParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int nsb = p.nsb;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int team = warp / p.team_warps;
+    const int wit = warp % p.team_warps;           // warp index in team
+    const int tl = wit * 32 + lane;                 // lane index in team
+    const int team_threads = p.team_warps * 32;
+    const bool leader = (tl == 0);
+
+    uint8_t* ring = smem + static_cast<size_t>(team) * p.depth * p.stage_bytes;
+    float* coef = reinterpret_cast<float*>(smem + p.off_coef) +
+                  static_cast<size_t>(team) * 2 * p.coef_floats;
+    float* red = reinterpret_cast<float*>(smem + p.off_red) +
+                 static_cast<size_t>(team) * 2 * p.team_warps * kSeg * M;
+    float* part = reinterpret_cast<float*>(smem + p.off_part);   // [teams][2][M]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar) +
+                     static_cast<size_t>(team) * p.depth;
+    __shared__ volatile int abort_flag;
+
+    const TeamRange tr = team_range(p, team);
+
+    if (threadIdx.x == 0) abort_flag = 0;
+    if (leader) {
+        for (int s = 0; s < p.depth; ++s) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+        for (int i = 0; i < 2 * M; ++i) part[team * 2 * M + i] = 0.f;
+    }
+    __syncthreads();
+
+    // Prologue: the first `depth` stages of W. Weights are model data that no
+    // preceding kernel writes, so they are fetched before the dependency wait.
+    int issued = 0;     // stages whose copy the leader has issued
+    int waited = 0;     // stages the leader has seen complete
+    if (leader) {
+        const int pre = tr.nstages < p.depth ? tr.nstages : p.depth;
+        issued = pre;
+        for (int s = 0; s < pre; ++s) {
+            const int i0 = s * kSeg;
+            const int i1 = (i0 + kSeg < tr.nseg ? i0 + kSeg : tr.nseg) - 1;
+            const long long b = seg_begin(tr, i0, nsb), e = seg_end(tr, i1, nsb);
+            const uint32_t bytes = static_cast<uint32_t>((e - b) * kBlockBytes);
+            mbar_arrive_expect_tx(&bars[s], bytes);
+            bulk_copy_g2s(ring + static_cast<size_t>(s) * p.stage_bytes, p.w + b * kBlockBytes,
+                          bytes, &bars[s]);
+        }
+    }
+    pdl_launch_dependents();
+    pdl_wait();   // x and y belong to the dependency chain
+
+    // This lane's fixed slice of K and its x values.
+    const bool valid = tl < 8 * nsb;
+    const int bl = tl >> 3, c = tl & 7, g = c >> 1, h = c & 1;
+    float2 xlo[M][8], xhi[M][8];
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) xlo[i][v] = xhi[i][v] = make_float2(0.f, 0.f);
+    }
+    if (valid) {
+        const int k0 = bl * kQK + 64 * g + 16 * h;
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const float4* xl = reinterpret_cast<const float4*>(p.x + static_cast<size_t>(i) * p.k + k0);
+            const float4* xh = xl + 8;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const float4 a = __ldg(xl + v), b = __ldg(xh + v);
+                xlo[i][2 * v] = make_float2(a.x, a.y);
+                xlo[i][2 * v + 1] = make_float2(a.z, a.w);
+                xhi[i][2 * v] = make_float2(b.x, b.y);
+                xhi[i][2 * v + 1] = make_float2(b.z, b.w);
+            }
+        }
+    }
+
+    // Finishes stage `s`'s row segments from red[s % 2] (leader warp, lanes < kSeg*M).
+    auto finish_stage = [&](int s) {
+        if (wit != 0) return;
+        const int u = lane % kSeg, i = lane / kSeg;
+        const int seg = s * kSeg + u;
+        if (i >= M || seg >= tr.nseg) return;
+        const float* rb = red + static_cast<size_t>(s & 1) * p.team_warps * kSeg * M;
+        float tot = 0.f;
+        for (int wi = 0; wi < p.team_warps; ++wi) tot += rb[(wi * M + i) * kSeg + u];
+        const long long row = tr.row0 + seg;
+        const long long b = seg_begin(tr, seg, nsb) - row * nsb;
+        const long long e = seg_end(tr, seg, nsb) - row * nsb;
+        if (b == 0 && e == nsb) {
+            p.y[static_cast<size_t>(i) * p.n + row] = tot;
+        } else {
+            part[(team * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
+        }
+    };
+
+    for (int s = 0; s < tr.nstages; ++s) {
+        const int slot = s % p.depth;
+        const uint8_t* st = ring + static_cast<size_t>(slot) * p.stage_bytes;
+        const int i0 = s * kSeg;
+        const int nseg_s = (tr.nseg - i0) < kSeg ? (tr.nseg - i0) : kSeg;
+        const long long sb0 = seg_begin(tr, i0, nsb);
+        const long long sb1 = seg_end(tr, i0 + nseg_s - 1, nsb);
+        const int nsb_stage = static_cast<int>(sb1 - sb0);
+
+        if (!abort_flag) {
+            if (mbar_wait_bounded(&bars[slot], static_cast<uint32_t>((s / p.depth) & 1),
+                                  &g_fault_flags)) {
+                if (leader) waited = s + 1;
+            } else {
+                abort_flag = 1;
+            }
+        }
+        float* cbuf = coef + static_cast<size_t>(s & 1) * p.coef_floats;
+        for (int i = tl; i < nsb_stage; i += team_threads)
+            decode_coefs(st + static_cast<size_t>(i) * kBlockBytes, cbuf + 16 * i);
+        named_barrier_sync(1 + team, team_threads);
+
+        if (s >= 1) {
+            finish_stage(s - 1);
+            if (leader && !abort_flag) {
+                const int ns = s - 1 + p.depth;
+                if (ns < tr.nstages) {
+                    const int nslot = (s - 1) % p.depth;
+                    const int j0 = ns * kSeg;
+                    const int j1 = (j0 + kSeg < tr.nseg ? j0 + kSeg : tr.nseg) - 1;
+                    const long long b = seg_begin(tr, j0, nsb), e = seg_end(tr, j1, nsb);
+                    const uint32_t bytes = static_cast<uint32_t>((e - b) * kBlockBytes);
+                    mbar_arrive_expect_tx(&bars[nslot], bytes);
+                    bulk_copy_g2s(ring + static_cast<size_t>(nslot) * p.stage_bytes,
+                                  p.w + b * kBlockBytes, bytes, &bars[nslot]);
+                    issued = ns + 1;
+                }
+            }
+        }
+
+        // Branch-free over the stage's (up to) kSeg row segments: a lane whose
+        // superblock is not in a segment computes on superblock 0 of the stage
+        // and the result is discarded by a select.
+        float part_sum[M][kSeg];
+#pragma unroll
+        for (int u = 0; u < kSeg; ++u) {
+            const long long row = tr.row0 + i0 + u;
+            const long long mine = row * nsb + bl;
+            const bool use = valid && u < nseg_s && mine >= seg_begin(tr, i0 + u, nsb) &&
+                             mine < seg_end(tr, i0 + u, nsb);
+            const int idx = use ? static_cast<int>(mine - sb0) : 0;
+            const uint4 q = *reinterpret_cast<const uint4*>(
+                st + static_cast<size_t>(idx) * kBlockBytes + kQsOffset + 16 * c);
+            const float4 cf = *reinterpret_cast<const float4*>(cbuf + 16 * idx + 4 * g);
+            float2 acc[M][2];
+#pragma unroll
+            for (int i = 0; i < M; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+            dot_item<M>(q, cf, xlo, xhi, acc);
+#pragma unroll
+            for (int i = 0; i < M; ++i) {
+                const float v = (acc[i][0].x + acc[i][0].y) + (acc[i][1].x + acc[i][1].y);
+                part_sum[i][u] = use ? v : 0.f;
+            }
+        }
+        float* rb = red + static_cast<size_t>(s & 1) * p.team_warps * kSeg * M;
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const float r = transpose_reduce4(part_sum[i][0], part_sum[i][1], part_sum[i][2],
+                                              part_sum[i][3], lane);
+            if ((lane & 7) == 0) {
+                const int u = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+                rb[(wit * M + i) * kSeg + u] = r;
+            }
+        }
+    }
+    if (tr.nstages > 0) {
+        named_barrier_sync(1 + team, team_threads);
+        finish_stage(tr.nstages - 1);
+    }
+    // After a lost copy, give the copies still in flight a bounded chance to
+    // land before the CTA's shared memory is released.
+    if (leader && abort_flag) {
+        for (int s = waited; s < issued; ++s)
+            mbar_wait_bounded(&bars[s % p.depth], static_cast<uint32_t>((s / p.depth) & 1),
+                              &g_fault_flags);
+    }
+    __syncthreads();
+
+    // Rows cut between teams: the team holding a row's first superblock adds the
+    // partial sums of the following teams that touch the row, in team order.
+    if (leader && tr.nseg > 0) {
+        const long long last = tr.row0 + tr.nseg - 1;
+        const long long lb = seg_begin(tr, tr.nseg - 1, nsb) - last * nsb;
+        const long long le = seg_end(tr, tr.nseg - 1, nsb) - last * nsb;
+        if (lb == 0 && le < nsb) {
+            float tot[M];
+#pragma unroll
+            for (int i = 0; i < M; ++i) tot[i] = part[(team * 2 + 1) * M + i];
+            for (int t2 = team + 1; t2 < p.teams; ++t2) {
+                const TeamRange o = team_range(p, t2);
+                if (o.s0 >= (last + 1) * nsb) break;
+                if (o.s1 <= o.s0) continue;   // a team with an empty range
+#pragma unroll
+                for (int i = 0; i < M; ++i) tot[i] += part[(t2 * 2 + 0) * M + i];
+            }
+#pragma unroll
+            for (int i = 0; i < M; ++i) p.y[static_cast<size_t>(i) * p.n + last] = tot[i];
+        }
+    }
+}
+
+}  // namespace
+
+int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp, int* grid,
+                int* block, int* smem_bytes) {
+    const int nsb = k / kQK;
+    if (m < 1 || m > kStreamMaxM || nsb > kStreamMaxNsb || n < 1) return 0;
+    const int team_warps = (nsb + 3) / 4;               // 8*nsb slices / 32 lanes
+    const int max_warps = stream_max_threads(m) / 32;
+    if (team_warps > max_warps) return 0;
+    int teams = max_warps / team_warps;
+    if (teams < 1) teams = 1;
+    if (teams > kStreamMaxTeams) teams = kStreamMaxTeams;
+    const int ctas = n < num_sms ? n : num_sms;
+    const int stage_bytes = ((kSeg * nsb * kBlockBytes) + 127) / 128 * 128;
+    const int coef_floats = kSeg * nsb * 16;
+    const int fixed_team = 2 * coef_floats * 4 + 2 * team_warps * kSeg * m * 4 + 64;
+    const int budget = (max_smem < kStreamSmemBudget ? max_smem : kStreamSmemBudget) - 1024;
+    int depth = (budget / teams - fixed_team) / stage_bytes;
+    if (depth > kStreamMaxDepth) depth = kStreamMaxDepth;
+    if (depth < 2) {
+        // fewer, deeper teams
+        while (teams > 1 && depth < 2) {
+            --teams;
+            depth = (budget / teams - fixed_team) / stage_bytes;
+        }
+        if (depth < 2) return 0;
+        if (depth > kStreamMaxDepth) depth = kStreamMaxDepth;
+    }
+    StreamParams q{};
+    q.n = n;
+    q.k = k;
+    q.nsb = nsb;
+    q.rows_base = n / ctas;
+    q.rows_extra = n % ctas;
+    q.teams = teams;
+    q.team_warps = team_warps;
+    q.depth = depth;
+    q.stage_bytes = stage_bytes;
+    q.coef_floats = coef_floats;
+    size_t off = static_cast<size_t>(teams) * depth * stage_bytes;
+    q.off_coef = static_cast<int>(off);
+    off += static_cast<size_t>(teams) * 2 * coef_floats * 4;
+    q.off_red = static_cast<int>(off);
+    off += static_cast<size_t>(teams) * 2 * team_warps * kSeg * m * 4;
+    q.off_part = static_cast<int>(off);
+    off += static_cast<size_t>(teams) * 2 * m * 4;
+    off = (off + 15) / 16 * 16;
+    q.off_bar = static_cast<int>(off);
+    off += static_cast<size_t>(teams) * depth * 8;
+    *sp = q;
+    *grid = ctas;
+    *block = teams * team_warps * 32;
+    *smem_bytes = static_cast<int>(off);
+    return 1;
+}
+
+int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, const void* w,
+                  const float* x, float* y, int m, cudaStream_t stream) {
+    StreamParams sp = sp0;
+    sp.w = static_cast<const uint8_t*>(w);
+    sp.x = x;
+    sp.y = y;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (m == 1) {
+        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1>, sp);
+    } else {
+        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2>, sp);
+    }
+    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+}
+
+int stream_set_attributes() {
+    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kStreamSmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
+    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+}
+
+}  // namespace q4k
+
+namespace q4k {
+
+int read_fault_flags(unsigned* flags) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_fault_flags, sizeof(v));
+    if (e != cudaSuccess) return cuda_failure(e);
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_fault_flags, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_failure(e);
+    *flags = v;
+    return Q4K_OK;
+}
+
+}  // namespace q4k

@@ -19,13 +19,18 @@ int current_device_info(DeviceInfo* info);
 
 // Records `e` as the calling thread's last CUDA error and returns Q4K_ERR_CUDA.
 int cuda_failure(cudaError_t e);
+int q4k_last_cuda_error_value();
+
+// Opt-in dynamic shared memory per CTA on B200 (227 KiB), assumed by the
+// host-only planner when no device is queried.
+constexpr int kB200SmemOptin = 232448;
 
 // Host-only launch planning (no CUDA calls).
 int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan);
 
-// Enqueue the planned kernels. Arguments are already validated.
-int launch_gemv(const q4k_gemv_plan& plan, const void* w, const float* x, float* y, int m,
-                int n, int k, cudaStream_t stream);
+// Enqueue the planned kernels on the current device. Arguments are already validated.
+int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n,
+                int k, cudaStream_t stream);
 
 int launch_dequant(const void* w, float* out, int n, int k, int num_sms, cudaStream_t stream);
 

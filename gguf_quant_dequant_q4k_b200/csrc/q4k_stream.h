@@ -1,0 +1,45 @@
+// q4k_stream.h -- host-side interface of the streaming GEMV kernel.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace q4k {
+
+constexpr int kStreamSegRows = 4;       // row segments per ring stage
+constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kernel
+// Threads per CTA (launch bound): 20 warps for one vector (x: 32 registers per
+// lane), 16 warps for two (x: 64 registers per lane).
+constexpr int stream_max_threads(int m) { return m == 1 ? 640 : 512; }
+constexpr int kStreamMaxNsb = 80;       // K <= 20480 (m = 1) / 16384 (m = 2): one team covers K
+constexpr int kStreamMaxTeams = 15;     // named barriers 1..15
+constexpr int kStreamMaxDepth = 8;
+constexpr int kStreamSmemBudget = 200 * 1024;
+
+struct StreamParams {
+    const uint8_t* w;
+    const float* x;
+    float* y;
+    int n, k, nsb;
+    int rows_base, rows_extra;  // CTA c owns rows_base (+1 if c < rows_extra) rows
+    int teams, team_warps, depth;
+    int stage_bytes;            // bytes per ring slot
+    int coef_floats;            // floats per coefficient buffer (two per team)
+    int off_coef, off_red, off_part, off_bar;  // shared-memory offsets (bytes)
+};
+
+// Fills the launch configuration; returns 0 if the streaming kernel does not
+// handle (m, k) or the shared-memory budget cannot hold two stages.
+int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp, int* grid,
+                int* block, int* smem_bytes);
+
+int launch_stream(const StreamParams& sp, int grid, int block, int smem_bytes, const void* w,
+                  const float* x, float* y, int m, cudaStream_t stream);
+
+// Per-device kernel attributes (dynamic shared memory opt-in).
+int stream_set_attributes();
+
+// Reads and clears the device fault flags (synchronises the device).
+int read_fault_flags(unsigned* flags);
+
+}  // namespace q4k

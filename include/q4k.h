@@ -121,24 +121,35 @@ Q4K_API const char *q4k_status_string(int status);
 Q4K_API int q4k_last_cuda_error(void);
 
 /*
- * How q4k_gemv would run a problem on a GPU with `num_sms` SMs (host-only, no
- * CUDA call). Fills *plan and returns Q4K_OK, or the status q4k_gemv would
+ * Reads and clears the calling device's fault flags: bit 0 is set if a bounded
+ * wait inside a kernel on a bulk copy into shared memory gave up (the kernel
+ * then skipped its remaining work and returned; its output is invalid). This
+ * never happens in normal operation. Synchronises the device. Returns a
+ * q4k_status; *flags receives the flags.
+ */
+Q4K_API int q4k_device_fault_flags(unsigned int *flags);
+
+/*
+ * How q4k_gemv would run a problem on a B200 with `num_sms` SMs (host-only,
+ * no CUDA call). Fills *plan and returns Q4K_OK, or the status q4k_gemv would
  * return for these sizes.
  */
 typedef struct q4k_gemv_plan {
     int kernel;          /* Q4K_KERNEL_* below                                  */
-    int grid;            /* CTAs of the main kernel                             */
+    int grid;            /* CTAs                                                */
     int block;           /* threads per CTA                                     */
     int smem_bytes;      /* dynamic shared memory per CTA                       */
-    int k_splits;        /* parts K is cut into (1 = no split)                  */
+    int teams;           /* warp teams per CTA (streaming kernel; else 0)       */
+    int depth;           /* bulk-copy ring stages per team (streaming; else 0)  */
     int launches;        /* kernels one call enqueues                           */
-    long long units;     /* work units (row x K-part) shared out among the CTAs */
-    long long units_per_cta_max; /* most units any CTA processes                */
+    long long units;     /* output rows shared out among the CTAs               */
+    long long units_per_cta_max; /* most rows any CTA owns                      */
 } q4k_gemv_plan;
 
 enum q4k_kernel {
-    Q4K_KERNEL_ROWS = 1,        /* whole rows per CTA, bulk-copy streamed         */
-    Q4K_KERNEL_SPLITK = 2       /* K split across CTAs + second-stage reduce       */
+    Q4K_KERNEL_WARP_ROWS = 1,   /* any K, m <= 8: one warp per row, loads via L1  */
+    Q4K_KERNEL_STREAM = 2       /* m <= 2, K <= 20480: bulk-copy streamed rows,
+                                   x held in registers, balanced per-SM ranges    */
 };
 
 Q4K_API int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan *plan);

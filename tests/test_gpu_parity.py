@@ -110,7 +110,8 @@ def test_gemv_config_shapes(q4k, n, k):
 
 @pytest.mark.parametrize("n,k", [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280),
                                  (33, 2304), (37, 8960), (129, 256), (1, 14336), (3, 11008),
-                                 (97, 4352), (300, 3840)])
+                                 (97, 4352), (300, 3840), (149, 1024), (77, 1536), (40, 4096),
+                                 (147, 20480), (1000, 20480), (64, 20736), (2, 32768)])
 def test_gemv_ragged_shapes(q4k, n, k):
     w, x = q4k_synth.q4k_problem(n, k, 1, 1000 + n + k)
     y = gpu_gemv(q4k, w, x, n, k)
@@ -241,3 +242,16 @@ def test_invalid_arguments_on_gpu_enqueue_nothing(q4k):
     assert q4k.q4k_gemv_status(wt, xt, y, 1, n, 500) == q4k.Q4K_ERR_SHAPE
     torch.cuda.synchronize()
     assert (y == 3.0).all()
+
+
+@pytest.mark.parametrize("n,k", [(149, 1024), (40, 4096), (1000, 20480)])
+def test_gemv_two_vectors_team_split(q4k, n, k):
+    w, x = q4k_synth.q4k_problem(n, k, 2, 40 + n)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(y, yref, a, f"{n}x{k} m=2")
+
+
+def test_no_kernel_fault_flags(q4k):
+    """No bounded wait on a bulk copy gave up during any of the runs above."""
+    assert q4k.q4k_device_fault_flags() == 0

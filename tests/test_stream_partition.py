@@ -1,0 +1,134 @@
+"""Host-side checks of the streaming GEMV kernel's work partition (CPU only).
+
+The kernel cuts each CTA's rows into per-team superblock ranges, the ranges into
+row segments and the segments into ring stages of at most 4 segments. This
+replays that index arithmetic (as the kernel states it) for the launch
+configuration the library plans, and checks: every superblock is streamed by
+exactly one team; each stage is one contiguous copy that fits its ring slot
+and is a multiple of 16 bytes; every row is written exactly once, either by
+the team holding a whole row segment or, for a row cut between teams, by the
+team holding its first superblock, which adds the following teams' partials;
+every lane's superblock index stays inside its stage; shared memory fits.
+"""
+import pytest
+
+import gguf_quant_dequant_q4k_b200 as q4k
+import q4k_synth
+
+SEG = 4
+SM_COUNT = 148
+SMEM_OPTIN = 232448
+
+
+def team_range(cta, team, n, nsb, ctas, teams):
+    base, extra = n // ctas, n % ctas
+    rows = base + (1 if cta < extra else 0)
+    row_begin = cta * base + min(cta, extra)
+    S0, L = row_begin * nsb, rows * nsb
+    s0 = S0 + (L * team) // teams
+    s1 = S0 + (L * (team + 1)) // teams
+    if s1 > s0:
+        row0 = s0 // nsb
+        nseg = (s1 - 1) // nsb - row0 + 1
+    else:
+        row0, nseg = 0, 0
+    return s0, s1, row0, nseg
+
+
+def seg_bounds(s0, s1, row0, i, nsb):
+    return max(s0, (row0 + i) * nsb), min(s1, (row0 + i + 1) * nsb)
+
+
+def check_plan(m, n, k):
+    p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
+    if p["kernel"] != q4k.Q4K_KERNEL_STREAM:
+        return p
+    nsb = k // 256
+    ctas, teams, depth = p["grid"], p["teams"], p["depth"]
+    team_warps = (nsb + 3) // 4
+    assert p["block"] == teams * team_warps * 32
+    assert p["block"] <= (640 if m == 1 else 512)
+    assert 2 <= depth <= 8 and 1 <= teams <= 15
+    stage_bytes = -(-SEG * nsb * 144 // 128) * 128
+    coef_floats = SEG * nsb * 16
+    need = (teams * depth * stage_bytes + teams * 2 * coef_floats * 4
+            + teams * 2 * team_warps * SEG * m * 4 + teams * 2 * m * 4)
+    need = -(-need // 16) * 16 + teams * depth * 8
+    assert p["smem_bytes"] == need and need <= 200 * 1024 <= SMEM_OPTIN - 1024
+    covered = [0] * (n * nsb)
+    writes = [0] * n
+    for cta in range(ctas):
+        ranges = [team_range(cta, t, n, nsb, ctas, teams) for t in range(teams)]
+        for t, (s0, s1, row0, nseg) in enumerate(ranges):
+            for sb in range(s0, s1):
+                covered[sb] += 1
+            nstages = -(-nseg // SEG)
+            for s in range(nstages):
+                i0 = s * SEG
+                nseg_s = min(SEG, nseg - i0)
+                b, _ = seg_bounds(s0, s1, row0, i0, nsb)
+                _, e = seg_bounds(s0, s1, row0, i0 + nseg_s - 1, nsb)
+                nbytes = (e - b) * 144
+                assert 0 < nbytes <= stage_bytes and nbytes % 16 == 0
+                # every lane's superblock in each segment lies inside the stage
+                for u in range(nseg_s):
+                    sb_b, sb_e = seg_bounds(s0, s1, row0, i0 + u, nsb)
+                    assert b <= sb_b < sb_e <= e
+            for i in range(nseg):
+                row = row0 + i
+                sb_b, sb_e = seg_bounds(s0, s1, row0, i, nsb)
+                rb, re = sb_b - row * nsb, sb_e - row * nsb
+                if rb == 0 and re == nsb:
+                    writes[row] += 1
+                elif rb > 0:
+                    assert i == 0, "a contributor partial must be the team's first segment"
+                else:
+                    assert i == nseg - 1, "an owner partial must be the team's last segment"
+            # finishing a row cut between teams
+            if nseg:
+                last = row0 + nseg - 1
+                lb, le = seg_bounds(s0, s1, row0, nseg - 1, nsb)
+                lb, le = lb - last * nsb, le - last * nsb
+                if lb == 0 and le < nsb:
+                    got = le
+                    for t2 in range(t + 1, teams):
+                        o0, o1, _, _ = ranges[t2]
+                        if o0 >= (last + 1) * nsb:
+                            break
+                        if o1 <= o0:
+                            continue
+                        assert o0 == last * nsb + got, "contributors must be contiguous"
+                        got = min(o1, (last + 1) * nsb) - last * nsb
+                    assert got == nsb, "a cut row's partials must cover the whole row"
+                    writes[last] += 1
+    assert all(c == 1 for c in covered), "every superblock streamed exactly once"
+    assert all(w == 1 for w in writes), "every row written exactly once"
+    return p
+
+
+SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
+          + [(4096, 14336), (1024, 4096), (14336, 4096)]
+          + [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280), (33, 2304), (37, 8960),
+             (129, 256), (1, 14336), (3, 11008), (97, 4352), (300, 3840), (149, 1024),
+             (147, 20480), (1000, 20480), (77, 1536), (40, 4096), (200, 1792)])
+
+
+@pytest.mark.parametrize("n,k", SHAPES)
+@pytest.mark.parametrize("m", [1, 2])
+def test_stream_partition(m, n, k):
+    check_plan(m, n, k)
+
+
+def test_lm_head_partition():
+    p = check_plan(1, 128256, 4096)
+    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["grid"] == SM_COUNT
+    assert p["units_per_cta_max"] == -(-128256 // SM_COUNT)
+
+
+def test_kernel_choice():
+    assert q4k.q4k_gemv_plan_for(1, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
+    assert q4k.q4k_gemv_plan_for(2, 4096, 14336, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
+    # outside the streaming kernel's range: the general kernel
+    assert q4k.q4k_gemv_plan_for(3, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    assert q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    assert q4k.q4k_gemv_plan_for(2, 64, 16640, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
