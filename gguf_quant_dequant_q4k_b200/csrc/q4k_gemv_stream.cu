@@ -57,14 +57,22 @@ namespace {
 // q4k_device_fault_flags(). Never set in normal operation.
 __device__ unsigned int g_fault_flags = 0;
 
-constexpr int kSeg = kStreamSegRows;  // row segments per stage
+constexpr int kSeg = kStreamSegRows;         // row segments per stage
 constexpr uint32_t kMagicOne = 0x3F000000u;  // bytes 0,1 = 0x00, byte 3 = 0x3F
+constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
+constexpr int kCoefFloatsPerWarp = kSeg * 4 * 8 * 4;  // [seg][4 positions][8 sub-blocks][A A B B]
 
-// f = 1 + q/128 for the nibble held in byte `sel` of `masked` (whose bytes are
-// 0x80 | q): the byte becomes bits 16..23 of 0x3F8?0000.
+// f = 1 + q/128 for the nibble held in byte SEL of `masked` (bytes 0x80 | q):
+// the byte becomes bits 16..23 of 0x3F800000 + q * 2^16.
 template <int SEL>
 __device__ __forceinline__ float nib_to_f(uint32_t masked) {
     return __uint_as_float(__byte_perm(masked, kMagicOne, 0x7054 | (SEL << 8)));
+}
+
+// 2^23 + (byte SEL of w), exactly.
+template <int SEL>
+__device__ __forceinline__ float byte_2p23(uint32_t w) {
+    return __uint_as_float(__byte_perm(w, kMagic2p23, 0x7650 | SEL));
 }
 
 struct TeamRange {
@@ -105,52 +113,62 @@ __device__ __forceinline__ long long seg_end(const TeamRange& r, int i, int nsb)
     return e < r.s1 ? e : r.s1;
 }
 
-// Decode one superblock header into 16 floats: (A_j, B_j), j = 0..7.
-__device__ __forceinline__ void decode_coefs(const uint8_t* sb, float* out) {
-    const uint4 h = *reinterpret_cast<const uint4*>(sb);
-    const Header hd = decode_header(h);
-    const float d128 = hd.d * 128.0f;
-    float c[16];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        const uint32_t scw = (j < 4) ? hd.sc_lo : hd.sc_hi;
-        const uint32_t mw = (j < 4) ? hd.m_lo : hd.m_hi;
-        const float a = d128 * small_u32_to_f32(byte_of(scw, j & 3));
-        const float dm = hd.dmin * small_u32_to_f32(byte_of(mw, j & 3));
-        c[2 * j] = a;
-        c[2 * j + 1] = -(a + dm);
-    }
-    float4* o = reinterpret_cast<float4*>(out);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) o[v] = make_float4(c[4 * v], c[4 * v + 1], c[4 * v + 2], c[4 * v + 3]);
+// Stage t of a team: flat superblock range [b, e) covering its segments.
+__device__ __forceinline__ void stage_span(const TeamRange& r, int t, int nsb, long long& b,
+                                           long long& e) {
+    const int i0 = t * kSeg;
+    const int i1 = (i0 + kSeg < r.nseg ? i0 + kSeg : r.nseg) - 1;
+    b = seg_begin(r, i0, nsb);
+    e = seg_end(r, i1, nsb);
 }
 
-// Sum over this lane's 32 weights of one row: returns (low-nibble, high-nibble)
-// accumulator pairs added into acc_lo / acc_hi for each vector.
+// Sub-blocks 4*half .. 4*half+3 of one superblock header -> four (A, A, B, B)
+// float4s: A_j = 128*d*sc_j (exact), B_j = -(A_j + dmin*m_j).
+__device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out) {
+    const uint4 h = *reinterpret_cast<const uint4*>(sb);
+    const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu)));
+    const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x >> 16)));
+    // six-bit fields of sub-blocks 4*half .. +3 (GGUF get_scale_min_k4 packing)
+    const uint32_t sc = half ? ((h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u))
+                             : (h.y & 0x3F3F3F3Fu);
+    const uint32_t mm = half ? (((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u))
+                             : (h.z & 0x3F3F3F3Fu);
+    const float d128 = d * 128.0f;
+    // (2^23 + v) * s - 2^23 * s == v * s exactly for the 6-bit v and these s.
+    const float2 sa = make_float2(d128, d128), sb2 = make_float2(-8388608.0f * d128, -8388608.0f * d128);
+    const float2 ma = make_float2(dmin, dmin), mb = make_float2(-8388608.0f * dmin, -8388608.0f * dmin);
+    const float2 a01 = ffma2(sa, make_float2(byte_2p23<0>(sc), byte_2p23<1>(sc)), sb2);
+    const float2 a23 = ffma2(sa, make_float2(byte_2p23<2>(sc), byte_2p23<3>(sc)), sb2);
+    const float2 m01 = ffma2(ma, make_float2(byte_2p23<0>(mm), byte_2p23<1>(mm)), mb);
+    const float2 m23 = ffma2(ma, make_float2(byte_2p23<2>(mm), byte_2p23<3>(mm)), mb);
+    out[0] = make_float4(a01.x, a01.x, -a01.x - m01.x, -a01.x - m01.x);
+    out[1] = make_float4(a01.y, a01.y, -a01.y - m01.y, -a01.y - m01.y);
+    out[2] = make_float4(a23.x, a23.x, -a23.x - m23.x, -a23.x - m23.x);
+    out[3] = make_float4(a23.y, a23.y, -a23.y - m23.y, -a23.y - m23.y);
+}
+
+// This lane's 32 weights of one row against its x registers:
+// acc[i][0] += low-nibble weights * x, acc[i][1] += high-nibble weights * x.
 template <int M>
-__device__ __forceinline__ void dot_item(uint4 q, float4 cf, const float2 (&xlo)[M][8],
+__device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const float2 (&xlo)[M][8],
                                          const float2 (&xhi)[M][8], float2 (&acc)[M][2]) {
-    const float2 alo = make_float2(cf.x, cf.x), blo = make_float2(cf.y, cf.y);
-    const float2 ahi = make_float2(cf.z, cf.z), bhi = make_float2(cf.w, cf.w);
+    const float2 alo = make_float2(clo.x, clo.y), blo = make_float2(clo.z, clo.w);
+    const float2 ahi = make_float2(chi.x, chi.y), bhi = make_float2(chi.z, chi.w);
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
         const uint32_t w = words[wi];
         const uint32_t lo = (w & 0x0F0F0F0Fu) | 0x80808080u;
         const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
-        const float2 flo0 = make_float2(nib_to_f<0>(lo), nib_to_f<1>(lo));
-        const float2 flo1 = make_float2(nib_to_f<2>(lo), nib_to_f<3>(lo));
-        const float2 fhi0 = make_float2(nib_to_f<0>(hi), nib_to_f<1>(hi));
-        const float2 fhi1 = make_float2(nib_to_f<2>(hi), nib_to_f<3>(hi));
-        const float2 wlo0 = ffma2(alo, flo0, blo);
-        const float2 wlo1 = ffma2(alo, flo1, blo);
-        const float2 whi0 = ffma2(ahi, fhi0, bhi);
-        const float2 whi1 = ffma2(ahi, fhi1, bhi);
+        const float2 wlo0 = ffma2(alo, make_float2(nib_to_f<0>(lo), nib_to_f<1>(lo)), blo);
+        const float2 wlo1 = ffma2(alo, make_float2(nib_to_f<2>(lo), nib_to_f<3>(lo)), blo);
+        const float2 whi0 = ffma2(ahi, make_float2(nib_to_f<0>(hi), nib_to_f<1>(hi)), bhi);
+        const float2 whi1 = ffma2(ahi, make_float2(nib_to_f<2>(hi), nib_to_f<3>(hi)), bhi);
 #pragma unroll
         for (int i = 0; i < M; ++i) {
             acc[i][0] = ffma2(wlo0, xlo[i][2 * wi], acc[i][0]);
-            acc[i][0] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][0]);
             acc[i][1] = ffma2(whi0, xhi[i][2 * wi], acc[i][1]);
+            acc[i][0] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][0]);
             acc[i][1] = ffma2(whi1, xhi[i][2 * wi + 1], acc[i][1]);
         }
     }
@@ -175,6 +193,10 @@ __device__ __forceinline__ float transpose_reduce4(float s0, float s1, float s2,
     return k;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 template <int M>
 __global__ void __launch_bounds__(stream_max_threads(M), 1)
 q4k_gemv_stream_kernel(const StreamParams p) {
@@ -185,24 +207,28 @@ q4k_gemv_stream_kernel(const StreamParams p) {
     const int team = warp / p.team_warps;
     const int wit = warp % p.team_warps;           // warp index in team
     const int tl = wit * 32 + lane;                 // lane index in team
-    const int team_threads = p.team_warps * 32;
-    const bool leader = (tl == 0);
+    const bool lead_warp = (wit == 0);
 
     uint8_t* ring = smem + static_cast<size_t>(team) * p.depth * p.stage_bytes;
-    float* coef = reinterpret_cast<float*>(smem + p.off_coef) +
-                  static_cast<size_t>(team) * 2 * p.coef_floats;
+    float* wcoef = reinterpret_cast<float*>(smem + p.off_coef) +
+                   static_cast<size_t>(warp) * kCoefFloatsPerWarp;
+    const int red_stride = p.team_warps * kSeg * M;   // floats per slot
     float* red = reinterpret_cast<float*>(smem + p.off_red) +
-                 static_cast<size_t>(team) * 2 * p.team_warps * kSeg * M;
+                 static_cast<size_t>(team) * p.depth * red_stride;
     float* part = reinterpret_cast<float*>(smem + p.off_part);   // [teams][2][M]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar) +
-                     static_cast<size_t>(team) * p.depth;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar) +
+                     static_cast<size_t>(team) * 2 * p.depth;
+    uint64_t* done = full + p.depth;
     __shared__ volatile int abort_flag;
 
     const TeamRange tr = team_range(p, team);
 
     if (threadIdx.x == 0) abort_flag = 0;
-    if (leader) {
-        for (int s = 0; s < p.depth; ++s) mbar_init(&bars[s], 1);
+    if (lead_warp && lane == 0) {
+        for (int s = 0; s < p.depth; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&done[s], p.team_warps);
+        }
         fence_mbar_init();
         for (int i = 0; i < 2 * M; ++i) part[team * 2 * M + i] = 0.f;
     }
@@ -210,20 +236,18 @@ q4k_gemv_stream_kernel(const StreamParams p) {
 
     // Prologue: the first `depth` stages of W. Weights are model data that no
     // preceding kernel writes, so they are fetched before the dependency wait.
-    int issued = 0;     // stages whose copy the leader has issued
-    int waited = 0;     // stages the leader has seen complete
-    if (leader) {
+    int issued = 0;   // stages whose copy this team's leader lane has issued
+    if (lead_warp && lane == 0) {
         const int pre = tr.nstages < p.depth ? tr.nstages : p.depth;
-        issued = pre;
         for (int s = 0; s < pre; ++s) {
-            const int i0 = s * kSeg;
-            const int i1 = (i0 + kSeg < tr.nseg ? i0 + kSeg : tr.nseg) - 1;
-            const long long b = seg_begin(tr, i0, nsb), e = seg_end(tr, i1, nsb);
+            long long b, e;
+            stage_span(tr, s, nsb, b, e);
             const uint32_t bytes = static_cast<uint32_t>((e - b) * kBlockBytes);
-            mbar_arrive_expect_tx(&bars[s], bytes);
+            mbar_arrive_expect_tx(&full[s], bytes);
             bulk_copy_g2s(ring + static_cast<size_t>(s) * p.stage_bytes, p.w + b * kBlockBytes,
-                          bytes, &bars[s]);
+                          bytes, &full[s]);
         }
+        issued = pre;
     }
     pdl_launch_dependents();
     pdl_wait();   // x and y belong to the dependency chain
@@ -254,90 +278,96 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         }
     }
 
-    // Finishes stage `s`'s row segments from red[s % 2] (leader warp, lanes < kSeg*M).
-    auto finish_stage = [&](int s) {
-        if (wit != 0) return;
+    // Decode lanes: lane -> (segment du, superblock position dpos of this warp's
+    // four, half of the sub-blocks).
+    const int du = lane >> 3, dpos = (lane >> 1) & 3, dhalf = lane & 1;
+    const int dbl = 4 * wit + dpos;
+
+    // The lead warp finishes stage t: waits until every warp of the team has
+    // consumed it, adds the warps' partials, writes y (or a cut row's partial),
+    // and refills the slot with stage t + depth.
+    auto finish_stage = [&](int t, int tslot, uint32_t tphase) {
+        bool ok = !abort_flag;
+        if (ok) ok = mbar_wait_bounded(&done[tslot], tphase, &g_fault_flags);
+        if (!ok) abort_flag = 1;
+        __syncwarp();
         const int u = lane % kSeg, i = lane / kSeg;
-        const int seg = s * kSeg + u;
-        if (i >= M || seg >= tr.nseg) return;
-        const float* rb = red + static_cast<size_t>(s & 1) * p.team_warps * kSeg * M;
-        float tot = 0.f;
-        for (int wi = 0; wi < p.team_warps; ++wi) tot += rb[(wi * M + i) * kSeg + u];
-        const long long row = tr.row0 + seg;
-        const long long b = seg_begin(tr, seg, nsb) - row * nsb;
-        const long long e = seg_end(tr, seg, nsb) - row * nsb;
-        if (b == 0 && e == nsb) {
-            p.y[static_cast<size_t>(i) * p.n + row] = tot;
-        } else {
-            part[(team * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
+        const int seg = t * kSeg + u;
+        if (i < M && seg < tr.nseg) {
+            const float* rb = red + static_cast<size_t>(tslot) * red_stride;
+            float tot = 0.f;
+            for (int wi = 0; wi < p.team_warps; ++wi) tot += rb[(wi * M + i) * kSeg + u];
+            const long long row = tr.row0 + seg;
+            const long long b = seg_begin(tr, seg, nsb) - row * nsb;
+            const long long e = seg_end(tr, seg, nsb) - row * nsb;
+            if (b == 0 && e == nsb) {
+                p.y[static_cast<size_t>(i) * p.n + row] = tot;
+            } else {
+                part[(team * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && !abort_flag && t + p.depth < tr.nstages) {
+            long long b, e;
+            stage_span(tr, t + p.depth, nsb, b, e);
+            const uint32_t bytes = static_cast<uint32_t>((e - b) * kBlockBytes);
+            mbar_arrive_expect_tx(&full[tslot], bytes);
+            bulk_copy_g2s(ring + static_cast<size_t>(tslot) * p.stage_bytes,
+                          p.w + b * kBlockBytes, bytes, &full[tslot]);
+            issued = t + p.depth + 1;
         }
     };
 
+    int slot = 0;
+    uint32_t phase = 0;
+    int prev_slot = 0;
+    uint32_t prev_phase = 0;
+    int consumed = 0;   // stages this warp has seen land
     for (int s = 0; s < tr.nstages; ++s) {
-        const int slot = s % p.depth;
         const uint8_t* st = ring + static_cast<size_t>(slot) * p.stage_bytes;
-        const int i0 = s * kSeg;
-        const int nseg_s = (tr.nseg - i0) < kSeg ? (tr.nseg - i0) : kSeg;
-        const long long sb0 = seg_begin(tr, i0, nsb);
-        const long long sb1 = seg_end(tr, i0 + nseg_s - 1, nsb);
+        long long sb0, sb1;
+        stage_span(tr, s, nsb, sb0, sb1);
         const int nsb_stage = static_cast<int>(sb1 - sb0);
+        // row-relative index of the stage's first superblock
+        const int head = static_cast<int>(sb0 - (tr.row0 + s * kSeg) * nsb);
 
         if (!abort_flag) {
-            if (mbar_wait_bounded(&bars[slot], static_cast<uint32_t>((s / p.depth) & 1),
-                                  &g_fault_flags)) {
-                if (leader) waited = s + 1;
-            } else {
+            if (mbar_wait_bounded(&full[slot], phase, &g_fault_flags))
+                consumed = s + 1;
+            else
                 abort_flag = 1;
-            }
-        }
-        float* cbuf = coef + static_cast<size_t>(s & 1) * p.coef_floats;
-        for (int i = tl; i < nsb_stage; i += team_threads)
-            decode_coefs(st + static_cast<size_t>(i) * kBlockBytes, cbuf + 16 * i);
-        named_barrier_sync(1 + team, team_threads);
-
-        if (s >= 1) {
-            finish_stage(s - 1);
-            if (leader && !abort_flag) {
-                const int ns = s - 1 + p.depth;
-                if (ns < tr.nstages) {
-                    const int nslot = (s - 1) % p.depth;
-                    const int j0 = ns * kSeg;
-                    const int j1 = (j0 + kSeg < tr.nseg ? j0 + kSeg : tr.nseg) - 1;
-                    const long long b = seg_begin(tr, j0, nsb), e = seg_end(tr, j1, nsb);
-                    const uint32_t bytes = static_cast<uint32_t>((e - b) * kBlockBytes);
-                    mbar_arrive_expect_tx(&bars[nslot], bytes);
-                    bulk_copy_g2s(ring + static_cast<size_t>(nslot) * p.stage_bytes,
-                                  p.w + b * kBlockBytes, bytes, &bars[nslot]);
-                    issued = ns + 1;
-                }
-            }
         }
 
-        // Branch-free over the stage's (up to) kSeg row segments: a lane whose
-        // superblock is not in a segment computes on superblock 0 of the stage
-        // and the result is discarded by a select.
+        // Decode this warp's superblock headers of the stage.
+        {
+            const int idx = du * nsb + dbl - head;
+            if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage))
+                decode4(st + static_cast<size_t>(idx) * kBlockBytes, dhalf,
+                        reinterpret_cast<float4*>(wcoef) + (du * 4 + dpos) * 8 + 4 * dhalf);
+        }
+        __syncwarp();
+
         float part_sum[M][kSeg];
 #pragma unroll
         for (int u = 0; u < kSeg; ++u) {
-            const long long row = tr.row0 + i0 + u;
-            const long long mine = row * nsb + bl;
-            const bool use = valid && u < nseg_s && mine >= seg_begin(tr, i0 + u, nsb) &&
-                             mine < seg_end(tr, i0 + u, nsb);
-            const int idx = use ? static_cast<int>(mine - sb0) : 0;
+            const int idx = u * nsb + bl - head;
+            const bool use = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
+            const int sidx = use ? idx : 0;
             const uint4 q = *reinterpret_cast<const uint4*>(
-                st + static_cast<size_t>(idx) * kBlockBytes + kQsOffset + 16 * c);
-            const float4 cf = *reinterpret_cast<const float4*>(cbuf + 16 * idx + 4 * g);
+                st + static_cast<size_t>(sidx) * kBlockBytes + kQsOffset + 16 * c);
+            const float4* cp = reinterpret_cast<const float4*>(wcoef) + (u * 4 + (lane >> 3)) * 8 + 2 * g;
+            const float4 clo = cp[0], chi = cp[1];
             float2 acc[M][2];
 #pragma unroll
             for (int i = 0; i < M; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
-            dot_item<M>(q, cf, xlo, xhi, acc);
+            dot_item<M>(q, clo, chi, xlo, xhi, acc);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
                 const float v = (acc[i][0].x + acc[i][0].y) + (acc[i][1].x + acc[i][1].y);
                 part_sum[i][u] = use ? v : 0.f;
             }
         }
-        float* rb = red + static_cast<size_t>(s & 1) * p.team_warps * kSeg * M;
+        float* rb = red + static_cast<size_t>(slot) * red_stride;
 #pragma unroll
         for (int i = 0; i < M; ++i) {
             const float r = transpose_reduce4(part_sum[i][0], part_sum[i][1], part_sum[i][2],
@@ -347,23 +377,32 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 rb[(wit * M + i) * kSeg + u] = r;
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&done[slot]);
+
+        if (lead_warp && s >= 1) finish_stage(s - 1, prev_slot, prev_phase);
+
+        prev_slot = slot;
+        prev_phase = phase;
+        if (++slot == p.depth) {
+            slot = 0;
+            phase ^= 1u;
+        }
     }
-    if (tr.nstages > 0) {
-        named_barrier_sync(1 + team, team_threads);
-        finish_stage(tr.nstages - 1);
-    }
+    if (lead_warp && tr.nstages > 0) finish_stage(tr.nstages - 1, prev_slot, prev_phase);
+
     // After a lost copy, give the copies still in flight a bounded chance to
     // land before the CTA's shared memory is released.
-    if (leader && abort_flag) {
-        for (int s = waited; s < issued; ++s)
-            mbar_wait_bounded(&bars[s % p.depth], static_cast<uint32_t>((s / p.depth) & 1),
+    if (lead_warp && lane == 0 && abort_flag) {
+        for (int s = consumed; s < issued; ++s)
+            mbar_wait_bounded(&full[s % p.depth], static_cast<uint32_t>((s / p.depth) & 1),
                               &g_fault_flags);
     }
     __syncthreads();
 
     // Rows cut between teams: the team holding a row's first superblock adds the
     // partial sums of the following teams that touch the row, in team order.
-    if (leader && tr.nseg > 0) {
+    if (lead_warp && lane == 0 && tr.nseg > 0) {
         const long long last = tr.row0 + tr.nseg - 1;
         const long long lb = seg_begin(tr, tr.nseg - 1, nsb) - last * nsb;
         const long long le = seg_end(tr, tr.nseg - 1, nsb) - last * nsb;
@@ -394,24 +433,28 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
     const int max_warps = stream_max_threads(m) / 32;
     if (team_warps > max_warps) return 0;
     int teams = max_warps / team_warps;
-    if (teams < 1) teams = 1;
     if (teams > kStreamMaxTeams) teams = kStreamMaxTeams;
     const int ctas = n < num_sms ? n : num_sms;
     const int stage_bytes = ((kSeg * nsb * kBlockBytes) + 127) / 128 * 128;
-    const int coef_floats = kSeg * nsb * 16;
-    const int fixed_team = 2 * coef_floats * 4 + 2 * team_warps * kSeg * m * 4 + 64;
     const int budget = (max_smem < kStreamSmemBudget ? max_smem : kStreamSmemBudget) - 1024;
-    int depth = (budget / teams - fixed_team) / stage_bytes;
-    if (depth > kStreamMaxDepth) depth = kStreamMaxDepth;
-    if (depth < 2) {
-        // fewer, deeper teams
-        while (teams > 1 && depth < 2) {
+    // bytes per team besides its ring: coefficient buffers of its warps, the
+    // per-slot partial sums, its cut-row partials and two barriers per slot
+    auto fixed_team = [&](int depth) {
+        return team_warps * kCoefFloatsPerWarp * 4 + depth * team_warps * kSeg * m * 4 +
+               2 * m * 4 + 2 * depth * 8 + 16;
+    };
+    int depth = kStreamMaxDepth;
+    while (depth >= 2 && teams * (depth * stage_bytes + fixed_team(depth)) > budget) {
+        if (depth > 2) {
+            --depth;
+        } else if (teams > 1) {
             --teams;
-            depth = (budget / teams - fixed_team) / stage_bytes;
+            depth = kStreamMaxDepth;
+        } else {
+            break;
         }
-        if (depth < 2) return 0;
-        if (depth > kStreamMaxDepth) depth = kStreamMaxDepth;
     }
+    if (teams * (depth * stage_bytes + fixed_team(depth)) > budget) return 0;
     StreamParams q{};
     q.n = n;
     q.k = k;
@@ -422,17 +465,16 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
     q.team_warps = team_warps;
     q.depth = depth;
     q.stage_bytes = stage_bytes;
-    q.coef_floats = coef_floats;
     size_t off = static_cast<size_t>(teams) * depth * stage_bytes;
     q.off_coef = static_cast<int>(off);
-    off += static_cast<size_t>(teams) * 2 * coef_floats * 4;
+    off += static_cast<size_t>(teams) * team_warps * kCoefFloatsPerWarp * 4;
     q.off_red = static_cast<int>(off);
-    off += static_cast<size_t>(teams) * 2 * team_warps * kSeg * m * 4;
+    off += static_cast<size_t>(teams) * depth * team_warps * kSeg * m * 4;
     q.off_part = static_cast<int>(off);
     off += static_cast<size_t>(teams) * 2 * m * 4;
     off = (off + 15) / 16 * 16;
     q.off_bar = static_cast<int>(off);
-    off += static_cast<size_t>(teams) * depth * 8;
+    off += static_cast<size_t>(teams) * 2 * depth * 8;
     *sp = q;
     *grid = ctas;
     *block = teams * team_warps * 32;

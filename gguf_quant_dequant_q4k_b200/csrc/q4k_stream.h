@@ -24,7 +24,6 @@ struct StreamParams {
     int rows_base, rows_extra;  // CTA c owns rows_base (+1 if c < rows_extra) rows
     int teams, team_warps, depth;
     int stage_bytes;            // bytes per ring slot
-    int coef_floats;            // floats per coefficient buffer (two per team)
     int off_coef, off_red, off_part, off_bar;  // shared-memory offsets (bytes)
 };
 

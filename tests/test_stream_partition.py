@@ -50,11 +50,11 @@ def check_plan(m, n, k):
     assert p["block"] <= (640 if m == 1 else 512)
     assert 2 <= depth <= 8 and 1 <= teams <= 15
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
-    coef_floats = SEG * nsb * 16
-    need = (teams * depth * stage_bytes + teams * 2 * coef_floats * 4
-            + teams * 2 * team_warps * SEG * m * 4 + teams * 2 * m * 4)
-    need = -(-need // 16) * 16 + teams * depth * 8
-    assert p["smem_bytes"] == need and need <= 200 * 1024 <= SMEM_OPTIN - 1024
+    coef_per_warp = SEG * 4 * 8 * 4 * 4          # [seg][4 positions][8 sub-blocks][A A B B]
+    need = (teams * depth * stage_bytes + teams * team_warps * coef_per_warp
+            + teams * depth * team_warps * SEG * m * 4 + teams * 2 * m * 4)
+    need = -(-need // 16) * 16 + teams * 2 * depth * 8
+    assert p["smem_bytes"] == need and need <= 200 * 1024 - 1024
     covered = [0] * (n * nsb)
     writes = [0] * n
     for cta in range(ctas):
