@@ -147,11 +147,11 @@ __device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out
     out[3] = make_float4(a23.y, a23.y, -a23.y - m23.y, -a23.y - m23.y);
 }
 
-// This lane's 32 weights of one row against its x registers:
-// acc[i][0] += low-nibble weights * x, acc[i][1] += high-nibble weights * x.
+// This lane's 32 weights of one row against its x registers, accumulated in
+// four independent f32x2 chains per vector (acc[i][0..3]).
 template <int M>
 __device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const float2 (&xlo)[M][8],
-                                         const float2 (&xhi)[M][8], float2 (&acc)[M][2]) {
+                                         const float2 (&xhi)[M][8], float2 (&acc)[M][4]) {
     const float2 alo = make_float2(clo.x, clo.y), blo = make_float2(clo.z, clo.w);
     const float2 ahi = make_float2(chi.x, chi.y), bhi = make_float2(chi.z, chi.w);
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
@@ -159,7 +159,7 @@ __device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const 
     for (int wi = 0; wi < 4; ++wi) {
         const uint32_t w = words[wi];
         const uint32_t lo = (w & 0x0F0F0F0Fu) | 0x80808080u;
-        const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+        const uint32_t hi = (__umulhi(w, 1u << 28) & 0x0F0F0F0Fu) | 0x80808080u;  // (w >> 4)
         const float2 wlo0 = ffma2(alo, make_float2(nib_to_f<0>(lo), nib_to_f<1>(lo)), blo);
         const float2 wlo1 = ffma2(alo, make_float2(nib_to_f<2>(lo), nib_to_f<3>(lo)), blo);
         const float2 whi0 = ffma2(ahi, make_float2(nib_to_f<0>(hi), nib_to_f<1>(hi)), bhi);
@@ -168,8 +168,8 @@ __device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const 
         for (int i = 0; i < M; ++i) {
             acc[i][0] = ffma2(wlo0, xlo[i][2 * wi], acc[i][0]);
             acc[i][1] = ffma2(whi0, xhi[i][2 * wi], acc[i][1]);
-            acc[i][0] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][0]);
-            acc[i][1] = ffma2(whi1, xhi[i][2 * wi + 1], acc[i][1]);
+            acc[i][2] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][2]);
+            acc[i][3] = ffma2(whi1, xhi[i][2 * wi + 1], acc[i][3]);
         }
     }
 }
@@ -283,23 +283,32 @@ q4k_gemv_stream_kernel(const StreamParams p) {
     const int du = lane >> 3, dpos = (lane >> 1) & 3, dhalf = lane & 1;
     const int dbl = 4 * wit + dpos;
 
-    // The lead warp finishes stage t: waits until every warp of the team has
-    // consumed it, adds the warps' partials, writes y (or a cut row's partial),
-    // and refills the slot with stage t + depth.
-    auto finish_stage = [&](int t, int tslot, uint32_t tphase) {
+    // Team-relative, 32-bit stage arithmetic: stage t holds rows row0 + 4t ..
+    // +3 clipped to the team's range [0, team_len) (in superblocks from s0);
+    // head0 is the row-relative index of the team's first superblock.
+    const int head0 = static_cast<int>(tr.s0 - tr.row0 * nsb);
+    const int team_len = static_cast<int>(tr.s1 - tr.s0);
+    const int stage_rows_sb = kSeg * nsb;
+    const uint8_t* wteam = p.w + tr.s0 * kBlockBytes;
+
+    // The lead warp finishes stage t (first row start rb_t, team-relative):
+    // waits until every warp of the team has consumed it, adds the warps'
+    // partials, writes y (or a cut row's partial), and refills the slot with
+    // stage t + depth.
+    auto finish_stage = [&](int t, int tslot, uint32_t tphase, int rb_t) {
         bool ok = !abort_flag;
         if (ok) ok = mbar_wait_bounded(&done[tslot], tphase, &g_fault_flags);
         if (!ok) abort_flag = 1;
         __syncwarp();
         const int u = lane % kSeg, i = lane / kSeg;
-        const int seg = t * kSeg + u;
-        if (i < M && seg < tr.nseg) {
-            const float* rb = red + static_cast<size_t>(tslot) * red_stride;
+        if (i < M && t * kSeg + u < tr.nseg) {
+            const float* rbuf = red + static_cast<size_t>(tslot) * red_stride;
             float tot = 0.f;
-            for (int wi = 0; wi < p.team_warps; ++wi) tot += rb[(wi * M + i) * kSeg + u];
-            const long long row = tr.row0 + seg;
-            const long long b = seg_begin(tr, seg, nsb) - row * nsb;
-            const long long e = seg_end(tr, seg, nsb) - row * nsb;
+            for (int wi = 0; wi < p.team_warps; ++wi) tot += rbuf[(wi * M + i) * kSeg + u];
+            const int r0 = rb_t + u * nsb;           // team-relative row start
+            const int b = (r0 > 0 ? r0 : 0) - r0;     // row-relative segment begin
+            const int e = ((r0 + nsb) < team_len ? (r0 + nsb) : team_len) - r0;
+            const long long row = tr.row0 + t * kSeg + u;
             if (b == 0 && e == nsb) {
                 p.y[static_cast<size_t>(i) * p.n + row] = tot;
             } else {
@@ -307,29 +316,36 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             }
         }
         __syncwarp();
-        if (lane == 0 && !abort_flag && t + p.depth < tr.nstages) {
-            long long b, e;
-            stage_span(tr, t + p.depth, nsb, b, e);
-            const uint32_t bytes = static_cast<uint32_t>((e - b) * kBlockBytes);
+        const int tn = t + p.depth;
+        if (lane == 0 && !abort_flag && tn < tr.nstages) {
+            const int rbn = rb_t + p.depth * stage_rows_sb;
+            const int b_rel = rbn > 0 ? rbn : 0;
+            const int e_rel = (rbn + stage_rows_sb) < team_len ? (rbn + stage_rows_sb) : team_len;
+            const uint32_t bytes = static_cast<uint32_t>(e_rel - b_rel) * kBlockBytes;
             mbar_arrive_expect_tx(&full[tslot], bytes);
             bulk_copy_g2s(ring + static_cast<size_t>(tslot) * p.stage_bytes,
-                          p.w + b * kBlockBytes, bytes, &full[tslot]);
-            issued = t + p.depth + 1;
+                          wteam + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &full[tslot]);
+            issued = tn + 1;
         }
     };
+
+    const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c);
+    const float4* lane_coef = reinterpret_cast<const float4*>(wcoef) + (lane >> 3) * 8 + 2 * g;
+    float4* dec_out = reinterpret_cast<float4*>(wcoef) + (du * 4 + dpos) * 8 + 4 * dhalf;
 
     int slot = 0;
     uint32_t phase = 0;
     int prev_slot = 0;
     uint32_t prev_phase = 0;
+    int prev_rb = 0;
     int consumed = 0;   // stages this warp has seen land
-    for (int s = 0; s < tr.nstages; ++s) {
+    int rb = -head0;    // team-relative index of stage t's first row start
+    for (int s = 0; s < tr.nstages; ++s, rb += stage_rows_sb) {
         const uint8_t* st = ring + static_cast<size_t>(slot) * p.stage_bytes;
-        long long sb0, sb1;
-        stage_span(tr, s, nsb, sb0, sb1);
-        const int nsb_stage = static_cast<int>(sb1 - sb0);
-        // row-relative index of the stage's first superblock
-        const int head = static_cast<int>(sb0 - (tr.row0 + s * kSeg) * nsb);
+        const int b_rel = rb > 0 ? rb : 0;
+        const int e_rel = (rb + stage_rows_sb) < team_len ? (rb + stage_rows_sb) : team_len;
+        const int nsb_stage = e_rel - b_rel;
+        const int head = b_rel - rb;   // row-relative index of the stage's first superblock
 
         if (!abort_flag) {
             if (mbar_wait_bounded(&full[slot], phase, &g_fault_flags))
@@ -342,54 +358,57 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         {
             const int idx = du * nsb + dbl - head;
             if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage))
-                decode4(st + static_cast<size_t>(idx) * kBlockBytes, dhalf,
-                        reinterpret_cast<float4*>(wcoef) + (du * 4 + dpos) * 8 + 4 * dhalf);
+                decode4(st + static_cast<size_t>(idx) * kBlockBytes, dhalf, dec_out);
         }
         __syncwarp();
 
+        // Items of the stage's (up to) kSeg row segments, branch-free: a lane
+        // whose superblock is not in a segment computes on superblock 0 and the
+        // result is discarded by a select.
         float part_sum[M][kSeg];
 #pragma unroll
         for (int u = 0; u < kSeg; ++u) {
-            const int idx = u * nsb + bl - head;
+            const int idx = u * nsb - head + bl;
             const bool use = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
-            const int sidx = use ? idx : 0;
-            const uint4 q = *reinterpret_cast<const uint4*>(
-                st + static_cast<size_t>(sidx) * kBlockBytes + kQsOffset + 16 * c);
-            const float4* cp = reinterpret_cast<const float4*>(wcoef) + (u * 4 + (lane >> 3)) * 8 + 2 * g;
-            const float4 clo = cp[0], chi = cp[1];
-            float2 acc[M][2];
+            const int off = use ? (u * nsb - head) * kBlockBytes : -bl * kBlockBytes;
+            const uint4 q = *reinterpret_cast<const uint4*>(st + lane_qoff + off);
+            const float4 clo = lane_coef[u * 32], chi = lane_coef[u * 32 + 1];
+            float2 acc[M][4];
 #pragma unroll
-            for (int i = 0; i < M; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+            for (int i = 0; i < M; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = make_float2(0.f, 0.f);
             dot_item<M>(q, clo, chi, xlo, xhi, acc);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
-                const float v = (acc[i][0].x + acc[i][0].y) + (acc[i][1].x + acc[i][1].y);
-                part_sum[i][u] = use ? v : 0.f;
+                const float2 t01 = __fadd2_rn(acc[i][0], acc[i][1]);
+                const float2 t23 = __fadd2_rn(acc[i][2], acc[i][3]);
+                const float2 t = __fadd2_rn(t01, t23);
+                part_sum[i][u] = use ? (t.x + t.y) : 0.f;
             }
         }
-        float* rb = red + static_cast<size_t>(slot) * red_stride;
+        float* rbuf = red + static_cast<size_t>(slot) * red_stride;
 #pragma unroll
         for (int i = 0; i < M; ++i) {
             const float r = transpose_reduce4(part_sum[i][0], part_sum[i][1], part_sum[i][2],
                                               part_sum[i][3], lane);
             if ((lane & 7) == 0) {
                 const int u = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-                rb[(wit * M + i) * kSeg + u] = r;
+                rbuf[(wit * M + i) * kSeg + u] = r;
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&done[slot]);
 
-        if (lead_warp && s >= 1) finish_stage(s - 1, prev_slot, prev_phase);
+        if (lead_warp && s >= 1) finish_stage(s - 1, prev_slot, prev_phase, prev_rb);
 
         prev_slot = slot;
         prev_phase = phase;
+        prev_rb = rb;
         if (++slot == p.depth) {
             slot = 0;
             phase ^= 1u;
         }
     }
-    if (lead_warp && tr.nstages > 0) finish_stage(tr.nstages - 1, prev_slot, prev_phase);
+    if (lead_warp && tr.nstages > 0) finish_stage(tr.nstages - 1, prev_slot, prev_phase, prev_rb);
 
     // After a lost copy, give the copies still in flight a bounded chance to
     // land before the CTA's shared memory is released.
