@@ -147,8 +147,9 @@ __device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out
     out[3] = make_float4(a23.y, a23.y, -a23.y - m23.y, -a23.y - m23.y);
 }
 
-// This lane's 32 weights of one row against its x registers, accumulated in
-// four independent f32x2 chains per vector (acc[i][0..3]).
+// This lane's 32 weights of one row against its x registers, in four
+// independent f32x2 chains per vector (acc[i][0..3]); the first product
+// initialises each chain.
 template <int M>
 __device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const float2 (&xlo)[M][8],
                                          const float2 (&xhi)[M][8], float2 (&acc)[M][4]) {
@@ -159,17 +160,24 @@ __device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const 
     for (int wi = 0; wi < 4; ++wi) {
         const uint32_t w = words[wi];
         const uint32_t lo = (w & 0x0F0F0F0Fu) | 0x80808080u;
-        const uint32_t hi = (__umulhi(w, 1u << 28) & 0x0F0F0F0Fu) | 0x80808080u;  // (w >> 4)
+        const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
         const float2 wlo0 = ffma2(alo, make_float2(nib_to_f<0>(lo), nib_to_f<1>(lo)), blo);
         const float2 wlo1 = ffma2(alo, make_float2(nib_to_f<2>(lo), nib_to_f<3>(lo)), blo);
         const float2 whi0 = ffma2(ahi, make_float2(nib_to_f<0>(hi), nib_to_f<1>(hi)), bhi);
         const float2 whi1 = ffma2(ahi, make_float2(nib_to_f<2>(hi), nib_to_f<3>(hi)), bhi);
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            acc[i][0] = ffma2(wlo0, xlo[i][2 * wi], acc[i][0]);
-            acc[i][1] = ffma2(whi0, xhi[i][2 * wi], acc[i][1]);
-            acc[i][2] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][2]);
-            acc[i][3] = ffma2(whi1, xhi[i][2 * wi + 1], acc[i][3]);
+            if (wi == 0) {
+                acc[i][0] = __fmul2_rn(wlo0, xlo[i][0]);
+                acc[i][1] = __fmul2_rn(whi0, xhi[i][0]);
+                acc[i][2] = __fmul2_rn(wlo1, xlo[i][1]);
+                acc[i][3] = __fmul2_rn(whi1, xhi[i][1]);
+            } else {
+                acc[i][0] = ffma2(wlo0, xlo[i][2 * wi], acc[i][0]);
+                acc[i][1] = ffma2(whi0, xhi[i][2 * wi], acc[i][1]);
+                acc[i][2] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][2]);
+                acc[i][3] = ffma2(whi1, xhi[i][2 * wi + 1], acc[i][3]);
+            }
         }
     }
 }
@@ -197,247 +205,279 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Per-team view of the kernel's shared memory and work range.
+struct Team {
+    TeamRange tr;
+    int head0;          // row-relative index of the team's first superblock
+    int team_len;       // superblocks in the team's range
+    const uint8_t* w;   // W at the team's first superblock
+    uint8_t* ring;      // depth slots of stage_bytes
+    float* red;         // [depth][team_warps][M][kSeg] warp partials
+    uint64_t* full;     // [depth] stage landed (1 arrival + bytes)
+    uint64_t* done;     // [depth] stage consumed (team_warps arrivals)
+};
+
 template <int M>
-__global__ void __launch_bounds__(stream_max_threads(M), 1)
+__device__ __forceinline__ Team make_team(const StreamParams& p, uint8_t* smem, int team) {
+    Team t;
+    t.tr = team_range(p, team);
+    t.head0 = static_cast<int>(t.tr.s0 - t.tr.row0 * p.nsb);
+    t.team_len = static_cast<int>(t.tr.s1 - t.tr.s0);
+    t.w = p.w + t.tr.s0 * kBlockBytes;
+    t.ring = smem + static_cast<size_t>(team) * p.depth * p.stage_bytes;
+    t.red = reinterpret_cast<float*>(smem + p.off_red) +
+            static_cast<size_t>(team) * p.depth * p.team_warps * kSeg * M;
+    t.full = reinterpret_cast<uint64_t*>(smem + p.off_bar) + static_cast<size_t>(team) * 2 * p.depth;
+    t.done = t.full + p.depth;
+    return t;
+}
+
+// Stage `st` (first row start rb team-relative) -> one bulk copy into `slot`.
+__device__ __forceinline__ void issue_stage(const Team& T, const StreamParams& p, int rb, int slot) {
+    const int span = kSeg * p.nsb;
+    const int b_rel = rb > 0 ? rb : 0;
+    const int e_rel = (rb + span) < T.team_len ? (rb + span) : T.team_len;
+    const uint32_t bytes = static_cast<uint32_t>(e_rel - b_rel) * kBlockBytes;
+    mbar_arrive_expect_tx(&T.full[slot], bytes);
+    bulk_copy_g2s(T.ring + static_cast<size_t>(slot) * p.stage_bytes,
+                  T.w + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &T.full[slot]);
+}
+
+template <int M>
+__global__ void __launch_bounds__(stream_max_threads(M) + 32, 1)
 q4k_gemv_stream_kernel(const StreamParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ volatile int abort_flag;
     const int nsb = p.nsb;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int team = warp / p.team_warps;
-    const int wit = warp % p.team_warps;           // warp index in team
-    const int tl = wit * 32 + lane;                 // lane index in team
-    const bool lead_warp = (wit == 0);
-
-    uint8_t* ring = smem + static_cast<size_t>(team) * p.depth * p.stage_bytes;
-    float* wcoef = reinterpret_cast<float*>(smem + p.off_coef) +
-                   static_cast<size_t>(warp) * kCoefFloatsPerWarp;
-    const int red_stride = p.team_warps * kSeg * M;   // floats per slot
-    float* red = reinterpret_cast<float*>(smem + p.off_red) +
-                 static_cast<size_t>(team) * p.depth * red_stride;
+    const int compute_warps = p.teams * p.team_warps;
     float* part = reinterpret_cast<float*>(smem + p.off_part);   // [teams][2][M]
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bar) +
-                     static_cast<size_t>(team) * 2 * p.depth;
-    uint64_t* done = full + p.depth;
-    __shared__ volatile int abort_flag;
 
-    const TeamRange tr = team_range(p, team);
-
-    if (threadIdx.x == 0) abort_flag = 0;
-    if (lead_warp && lane == 0) {
-        for (int s = 0; s < p.depth; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&done[s], p.team_warps);
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+        for (int t = 0; t < p.teams; ++t) {
+            for (int s = 0; s < p.depth; ++s) {
+                mbar_init(&bars[(2 * t) * p.depth + s], 1);
+                mbar_init(&bars[(2 * t + 1) * p.depth + s], p.team_warps);
+            }
         }
         fence_mbar_init();
-        for (int i = 0; i < 2 * M; ++i) part[team * 2 * M + i] = 0.f;
+        for (int i = 0; i < p.teams * 2 * M; ++i) part[i] = 0.f;
     }
     __syncthreads();
 
-    // Prologue: the first `depth` stages of W. Weights are model data that no
-    // preceding kernel writes, so they are fetched before the dependency wait.
-    int issued = 0;   // stages whose copy this team's leader lane has issued
-    if (lead_warp && lane == 0) {
-        const int pre = tr.nstages < p.depth ? tr.nstages : p.depth;
-        for (int s = 0; s < pre; ++s) {
-            long long b, e;
-            stage_span(tr, s, nsb, b, e);
-            const uint32_t bytes = static_cast<uint32_t>((e - b) * kBlockBytes);
-            mbar_arrive_expect_tx(&full[s], bytes);
-            bulk_copy_g2s(ring + static_cast<size_t>(s) * p.stage_bytes, p.w + b * kBlockBytes,
-                          bytes, &full[s]);
+    if (warp == compute_warps) {
+        // ------------------------------------------------------------ producer
+        // Lane t < teams owns team t's ring: it issues the team's copies, and
+        // as soon as every warp of the team has consumed a stage it adds the
+        // warps' partials into y (or a cut row's partial) and refills the slot.
+        const bool own = lane < p.teams;
+        Team T;
+        int nst = 0;
+        if (own) {
+            T = make_team<M>(p, smem, lane);
+            nst = T.tr.nstages;
+            const int pre = nst < p.depth ? nst : p.depth;
+            for (int s = 0; s < pre; ++s) issue_stage(T, p, s * kSeg * nsb - T.head0, s);
         }
-        issued = pre;
-    }
-    pdl_launch_dependents();
-    pdl_wait();   // x and y belong to the dependency chain
+        pdl_launch_dependents();
+        pdl_wait();
+        int tf = 0, fslot = 0;
+        uint32_t fphase = 0;
+        int rbf = own ? -T.head0 : 0;
+        unsigned idle = 0;
+        for (;;) {
+            const bool active = own && tf < nst && !abort_flag;
+            if (!__any_sync(0xFFFFFFFFu, active)) break;
+            bool progressed = false;
+            if (active && mbar_test_wait(&T.done[fslot], fphase)) {
+                const float* rbuf = T.red + static_cast<size_t>(fslot) * p.team_warps * kSeg * M;
+#pragma unroll
+                for (int u = 0; u < kSeg; ++u) {
+                    if (tf * kSeg + u >= T.tr.nseg) break;
+                    const int r0 = rbf + u * nsb;              // team-relative row start
+                    const int b = (r0 > 0 ? r0 : 0) - r0;      // row-relative segment bounds
+                    const int e = ((r0 + nsb) < T.team_len ? (r0 + nsb) : T.team_len) - r0;
+                    const long long row = T.tr.row0 + tf * kSeg + u;
+#pragma unroll
+                    for (int i = 0; i < M; ++i) {
+                        float tot = 0.f;
+                        for (int wi = 0; wi < p.team_warps; ++wi)
+                            tot += rbuf[(wi * M + i) * kSeg + u];
+                        if (b == 0 && e == nsb)
+                            p.y[static_cast<size_t>(i) * p.n + row] = tot;
+                        else
+                            part[(lane * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
+                    }
+                }
+                if (tf + p.depth < nst) issue_stage(T, p, rbf + p.depth * kSeg * nsb, fslot);
+                ++tf;
+                rbf += kSeg * nsb;
+                if (++fslot == p.depth) {
+                    fslot = 0;
+                    fphase ^= 1u;
+                }
+                progressed = true;
+                idle = 0;
+            } else if (active && ++idle > kSpinLimit) {
+                atomicOr(&g_fault_flags, kFaultCopyTimeout);
+                abort_flag = 1;
+            }
+            if (!__any_sync(0xFFFFFFFFu, progressed)) __nanosleep(32);
+        }
+        // After a lost copy, give the copies still in flight a bounded chance
+        // to land before the CTA's shared memory is released.
+        if (own && abort_flag) {
+            const int first = nst - p.depth > 0 ? nst - p.depth : 0;
+            for (int s = first; s < nst; ++s)
+                mbar_wait_bounded(&T.full[s % p.depth], static_cast<uint32_t>((s / p.depth) & 1),
+                                  &g_fault_flags);
+        }
+    } else {
+        // ------------------------------------------------------------ compute
+        const int team = warp / p.team_warps;
+        const int wit = warp % p.team_warps;
+        const int tl = wit * 32 + lane;
+        const Team T = make_team<M>(p, smem, team);
+        float* wcoef = reinterpret_cast<float*>(smem + p.off_coef) +
+                       static_cast<size_t>(warp) * kCoefFloatsPerWarp;
+        pdl_launch_dependents();
+        pdl_wait();   // x and y belong to the dependency chain
 
-    // This lane's fixed slice of K and its x values.
-    const bool valid = tl < 8 * nsb;
-    const int bl = tl >> 3, c = tl & 7, g = c >> 1, h = c & 1;
-    float2 xlo[M][8], xhi[M][8];
-#pragma unroll
-    for (int i = 0; i < M; ++i) {
-#pragma unroll
-        for (int v = 0; v < 8; ++v) xlo[i][v] = xhi[i][v] = make_float2(0.f, 0.f);
-    }
-    if (valid) {
-        const int k0 = bl * kQK + 64 * g + 16 * h;
+        // This lane's fixed slice of K and its x values.
+        const bool valid = tl < 8 * nsb;
+        const int bl = tl >> 3, c = tl & 7, g = c >> 1, h = c & 1;
+        float2 xlo[M][8], xhi[M][8];
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            const float4* xl = reinterpret_cast<const float4*>(p.x + static_cast<size_t>(i) * p.k + k0);
-            const float4* xh = xl + 8;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float4 a = __ldg(xl + v), b = __ldg(xh + v);
-                xlo[i][2 * v] = make_float2(a.x, a.y);
-                xlo[i][2 * v + 1] = make_float2(a.z, a.w);
-                xhi[i][2 * v] = make_float2(b.x, b.y);
-                xhi[i][2 * v + 1] = make_float2(b.z, b.w);
-            }
+            for (int v = 0; v < 8; ++v) xlo[i][v] = xhi[i][v] = make_float2(0.f, 0.f);
         }
-    }
-
-    // Decode lanes: lane -> (segment du, superblock position dpos of this warp's
-    // four, half of the sub-blocks).
-    const int du = lane >> 3, dpos = (lane >> 1) & 3, dhalf = lane & 1;
-    const int dbl = 4 * wit + dpos;
-
-    // Team-relative, 32-bit stage arithmetic: stage t holds rows row0 + 4t ..
-    // +3 clipped to the team's range [0, team_len) (in superblocks from s0);
-    // head0 is the row-relative index of the team's first superblock.
-    const int head0 = static_cast<int>(tr.s0 - tr.row0 * nsb);
-    const int team_len = static_cast<int>(tr.s1 - tr.s0);
-    const int stage_rows_sb = kSeg * nsb;
-    const uint8_t* wteam = p.w + tr.s0 * kBlockBytes;
-
-    // The lead warp finishes stage t (first row start rb_t, team-relative):
-    // waits until every warp of the team has consumed it, adds the warps'
-    // partials, writes y (or a cut row's partial), and refills the slot with
-    // stage t + depth.
-    auto finish_stage = [&](int t, int tslot, uint32_t tphase, int rb_t) {
-        bool ok = !abort_flag;
-        if (ok) ok = mbar_wait_bounded(&done[tslot], tphase, &g_fault_flags);
-        if (!ok) abort_flag = 1;
-        __syncwarp();
-        const int u = lane % kSeg, i = lane / kSeg;
-        if (i < M && t * kSeg + u < tr.nseg) {
-            const float* rbuf = red + static_cast<size_t>(tslot) * red_stride;
-            float tot = 0.f;
-            for (int wi = 0; wi < p.team_warps; ++wi) tot += rbuf[(wi * M + i) * kSeg + u];
-            const int r0 = rb_t + u * nsb;           // team-relative row start
-            const int b = (r0 > 0 ? r0 : 0) - r0;     // row-relative segment begin
-            const int e = ((r0 + nsb) < team_len ? (r0 + nsb) : team_len) - r0;
-            const long long row = tr.row0 + t * kSeg + u;
-            if (b == 0 && e == nsb) {
-                p.y[static_cast<size_t>(i) * p.n + row] = tot;
-            } else {
-                part[(team * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
-            }
-        }
-        __syncwarp();
-        const int tn = t + p.depth;
-        if (lane == 0 && !abort_flag && tn < tr.nstages) {
-            const int rbn = rb_t + p.depth * stage_rows_sb;
-            const int b_rel = rbn > 0 ? rbn : 0;
-            const int e_rel = (rbn + stage_rows_sb) < team_len ? (rbn + stage_rows_sb) : team_len;
-            const uint32_t bytes = static_cast<uint32_t>(e_rel - b_rel) * kBlockBytes;
-            mbar_arrive_expect_tx(&full[tslot], bytes);
-            bulk_copy_g2s(ring + static_cast<size_t>(tslot) * p.stage_bytes,
-                          wteam + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &full[tslot]);
-            issued = tn + 1;
-        }
-    };
-
-    const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c);
-    const float4* lane_coef = reinterpret_cast<const float4*>(wcoef) + (lane >> 3) * 8 + 2 * g;
-    float4* dec_out = reinterpret_cast<float4*>(wcoef) + (du * 4 + dpos) * 8 + 4 * dhalf;
-
-    int slot = 0;
-    uint32_t phase = 0;
-    int prev_slot = 0;
-    uint32_t prev_phase = 0;
-    int prev_rb = 0;
-    int consumed = 0;   // stages this warp has seen land
-    int rb = -head0;    // team-relative index of stage t's first row start
-    for (int s = 0; s < tr.nstages; ++s, rb += stage_rows_sb) {
-        const uint8_t* st = ring + static_cast<size_t>(slot) * p.stage_bytes;
-        const int b_rel = rb > 0 ? rb : 0;
-        const int e_rel = (rb + stage_rows_sb) < team_len ? (rb + stage_rows_sb) : team_len;
-        const int nsb_stage = e_rel - b_rel;
-        const int head = b_rel - rb;   // row-relative index of the stage's first superblock
-
-        if (!abort_flag) {
-            if (mbar_wait_bounded(&full[slot], phase, &g_fault_flags))
-                consumed = s + 1;
-            else
-                abort_flag = 1;
-        }
-
-        // Decode this warp's superblock headers of the stage.
-        {
-            const int idx = du * nsb + dbl - head;
-            if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage))
-                decode4(st + static_cast<size_t>(idx) * kBlockBytes, dhalf, dec_out);
-        }
-        __syncwarp();
-
-        // Items of the stage's (up to) kSeg row segments, branch-free: a lane
-        // whose superblock is not in a segment computes on superblock 0 and the
-        // result is discarded by a select.
-        float part_sum[M][kSeg];
-#pragma unroll
-        for (int u = 0; u < kSeg; ++u) {
-            const int idx = u * nsb - head + bl;
-            const bool use = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
-            const int off = use ? (u * nsb - head) * kBlockBytes : -bl * kBlockBytes;
-            const uint4 q = *reinterpret_cast<const uint4*>(st + lane_qoff + off);
-            const float4 clo = lane_coef[u * 32], chi = lane_coef[u * 32 + 1];
-            float2 acc[M][4];
-#pragma unroll
-            for (int i = 0; i < M; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = make_float2(0.f, 0.f);
-            dot_item<M>(q, clo, chi, xlo, xhi, acc);
+        if (valid) {
+            const int k0 = bl * kQK + 64 * g + 16 * h;
 #pragma unroll
             for (int i = 0; i < M; ++i) {
-                const float2 t01 = __fadd2_rn(acc[i][0], acc[i][1]);
-                const float2 t23 = __fadd2_rn(acc[i][2], acc[i][3]);
-                const float2 t = __fadd2_rn(t01, t23);
-                part_sum[i][u] = use ? (t.x + t.y) : 0.f;
-            }
-        }
-        float* rbuf = red + static_cast<size_t>(slot) * red_stride;
+                const float4* xl =
+                    reinterpret_cast<const float4*>(p.x + static_cast<size_t>(i) * p.k + k0);
+                const float4* xh = xl + 8;
 #pragma unroll
-        for (int i = 0; i < M; ++i) {
-            const float r = transpose_reduce4(part_sum[i][0], part_sum[i][1], part_sum[i][2],
-                                              part_sum[i][3], lane);
-            if ((lane & 7) == 0) {
-                const int u = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-                rbuf[(wit * M + i) * kSeg + u] = r;
+                for (int v = 0; v < 4; ++v) {
+                    const float4 a = __ldg(xl + v), b = __ldg(xh + v);
+                    xlo[i][2 * v] = make_float2(a.x, a.y);
+                    xlo[i][2 * v + 1] = make_float2(a.z, a.w);
+                    xhi[i][2 * v] = make_float2(b.x, b.y);
+                    xhi[i][2 * v + 1] = make_float2(b.z, b.w);
+                }
             }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&done[slot]);
 
-        if (lead_warp && s >= 1) finish_stage(s - 1, prev_slot, prev_phase, prev_rb);
+        // Decode lanes: lane -> (segment du, superblock position dpos of this
+        // warp's four, half of the sub-blocks).
+        const int du = lane >> 3, dpos = (lane >> 1) & 3, dhalf = lane & 1;
+        const int dbl = 4 * wit + dpos;
+        const int span = kSeg * nsb;
+        const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c);
+        const float4* lane_coef = reinterpret_cast<const float4*>(wcoef) + (lane >> 3) * 8 + 2 * g;
+        float4* dec_out = reinterpret_cast<float4*>(wcoef) + (du * 4 + dpos) * 8 + 4 * dhalf;
+        const int red_slot = p.team_warps * kSeg * M;
 
-        prev_slot = slot;
-        prev_phase = phase;
-        prev_rb = rb;
-        if (++slot == p.depth) {
-            slot = 0;
-            phase ^= 1u;
+        int slot = 0;
+        uint32_t phase = 0;
+        int rb = -T.head0;   // team-relative index of stage s's first row start
+        for (int s = 0; s < T.tr.nstages; ++s, rb += span) {
+            const uint8_t* st = T.ring + static_cast<size_t>(slot) * p.stage_bytes;
+            const int b_rel = rb > 0 ? rb : 0;
+            const int e_rel = (rb + span) < T.team_len ? (rb + span) : T.team_len;
+            const int nsb_stage = e_rel - b_rel;
+            const int head = b_rel - rb;   // row-relative index of the stage's first superblock
+
+            if (!abort_flag && !mbar_wait_bounded(&T.full[slot], phase, &g_fault_flags))
+                abort_flag = 1;
+
+            // Decode this warp's superblock headers of the stage.
+            {
+                const int idx = du * nsb + dbl - head;
+                if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage))
+                    decode4(st + static_cast<size_t>(idx) * kBlockBytes, dhalf, dec_out);
+            }
+            __syncwarp();
+
+            // The stage's (up to) kSeg row segments, branch-free: a lane whose
+            // superblock is not in a segment computes on superblock 0 and the
+            // result is discarded by a select.
+            float part_sum[M][kSeg];
+#pragma unroll
+            for (int u = 0; u < kSeg; ++u) {
+                const int idx = u * nsb - head + bl;
+                const bool use = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
+                const int off = use ? (u * nsb - head) * kBlockBytes : -bl * kBlockBytes;
+                const uint4 q = *reinterpret_cast<const uint4*>(st + lane_qoff + off);
+                const float4 clo = lane_coef[u * 32], chi = lane_coef[u * 32 + 1];
+                float2 acc[M][4];
+                dot_item<M>(q, clo, chi, xlo, xhi, acc);
+#pragma unroll
+                for (int i = 0; i < M; ++i) {
+                    const float2 t = __fadd2_rn(__fadd2_rn(acc[i][0], acc[i][1]),
+                                                __fadd2_rn(acc[i][2], acc[i][3]));
+                    part_sum[i][u] = use ? (t.x + t.y) : 0.f;
+                }
+            }
+            float* rbuf = T.red + static_cast<size_t>(slot) * red_slot;
+#pragma unroll
+            for (int i = 0; i < M; ++i) {
+                const float r = transpose_reduce4(part_sum[i][0], part_sum[i][1], part_sum[i][2],
+                                                  part_sum[i][3], lane);
+                if ((lane & 7) == 0) {
+                    const int u = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+                    rbuf[(wit * M + i) * kSeg + u] = r;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&T.done[slot]);
+            if (++slot == p.depth) {
+                slot = 0;
+                phase ^= 1u;
+            }
         }
-    }
-    if (lead_warp && tr.nstages > 0) finish_stage(tr.nstages - 1, prev_slot, prev_phase, prev_rb);
-
-    // After a lost copy, give the copies still in flight a bounded chance to
-    // land before the CTA's shared memory is released.
-    if (lead_warp && lane == 0 && abort_flag) {
-        for (int s = consumed; s < issued; ++s)
-            mbar_wait_bounded(&full[s % p.depth], static_cast<uint32_t>((s / p.depth) & 1),
-                              &g_fault_flags);
     }
     __syncthreads();
 
     // Rows cut between teams: the team holding a row's first superblock adds the
     // partial sums of the following teams that touch the row, in team order.
-    if (lead_warp && lane == 0 && tr.nseg > 0) {
-        const long long last = tr.row0 + tr.nseg - 1;
-        const long long lb = seg_begin(tr, tr.nseg - 1, nsb) - last * nsb;
-        const long long le = seg_end(tr, tr.nseg - 1, nsb) - last * nsb;
-        if (lb == 0 && le < nsb) {
-            float tot[M];
+    if (warp == compute_warps && lane < p.teams) {
+        const TeamRange tr = team_range(p, lane);
+        if (tr.nseg > 0) {
+            const long long last = tr.row0 + tr.nseg - 1;
+            const long long lb = seg_begin(tr, tr.nseg - 1, nsb) - last * nsb;
+            const long long le = seg_end(tr, tr.nseg - 1, nsb) - last * nsb;
+            if (lb == 0 && le < nsb) {
+                float tot[M];
 #pragma unroll
-            for (int i = 0; i < M; ++i) tot[i] = part[(team * 2 + 1) * M + i];
-            for (int t2 = team + 1; t2 < p.teams; ++t2) {
-                const TeamRange o = team_range(p, t2);
-                if (o.s0 >= (last + 1) * nsb) break;
-                if (o.s1 <= o.s0) continue;   // a team with an empty range
+                for (int i = 0; i < M; ++i) tot[i] = part[(lane * 2 + 1) * M + i];
+                for (int t2 = lane + 1; t2 < p.teams; ++t2) {
+                    const TeamRange o = team_range(p, t2);
+                    if (o.s0 >= (last + 1) * nsb) break;
+                    if (o.s1 <= o.s0) continue;   // a team with an empty range
 #pragma unroll
-                for (int i = 0; i < M; ++i) tot[i] += part[(t2 * 2 + 0) * M + i];
+                    for (int i = 0; i < M; ++i) tot[i] += part[(t2 * 2 + 0) * M + i];
+                }
+#pragma unroll
+                for (int i = 0; i < M; ++i) p.y[static_cast<size_t>(i) * p.n + last] = tot[i];
             }
-#pragma unroll
-            for (int i = 0; i < M; ++i) p.y[static_cast<size_t>(i) * p.n + last] = tot[i];
         }
     }
 }
@@ -496,7 +536,7 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
     off += static_cast<size_t>(teams) * 2 * depth * 8;
     *sp = q;
     *grid = ctas;
-    *block = teams * team_warps * 32;
+    *block = teams * team_warps * 32 + 32;   // + the producer warp
     *smem_bytes = static_cast<int>(off);
     return 1;
 }

@@ -46,8 +46,8 @@ def check_plan(m, n, k):
     nsb = k // 256
     ctas, teams, depth = p["grid"], p["teams"], p["depth"]
     team_warps = (nsb + 3) // 4
-    assert p["block"] == teams * team_warps * 32
-    assert p["block"] <= (640 if m == 1 else 512)
+    assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
+    assert p["block"] <= (640 if m == 1 else 512) + 32
     assert 2 <= depth <= 8 and 1 <= teams <= 15
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     coef_per_warp = SEG * 4 * 8 * 4 * 4          # [seg][4 positions][8 sub-blocks][A A B B]
