@@ -390,16 +390,22 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const int du = lane >> 3, dpos = (lane >> 1) & 3, dhalf = lane & 1;
         const int dbl = 4 * wit + dpos;
         const int span = kSeg * nsb;
+        // Shared-memory byte offsets (32-bit) of this team's ring, this lane's
+        // quant slice within a superblock row position, and this warp's
+        // coefficient buffer.
+        const uint32_t ring_off = static_cast<uint32_t>(T.ring - smem);
         const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c);
-        const float4* lane_coef = reinterpret_cast<const float4*>(wcoef) + (lane >> 3) * 8 + 2 * g;
-        float4* dec_out = reinterpret_cast<float4*>(wcoef) + (du * 4 + dpos) * 8 + 4 * dhalf;
+        const uint32_t coef_off = static_cast<uint32_t>(p.off_coef) +
+                                  static_cast<uint32_t>(warp) * kCoefFloatsPerWarp * 4u;
+        const uint32_t lane_coef_off = coef_off + static_cast<uint32_t>(((lane >> 3) * 8 + 2 * g) * 16);
+        const uint32_t dec_off = coef_off + static_cast<uint32_t>(((du * 4 + dpos) * 8 + 4 * dhalf) * 16);
         const int red_slot = p.team_warps * kSeg * M;
 
         int slot = 0;
         uint32_t phase = 0;
         int rb = -T.head0;   // team-relative index of stage s's first row start
         for (int s = 0; s < T.tr.nstages; ++s, rb += span) {
-            const uint8_t* st = T.ring + static_cast<size_t>(slot) * p.stage_bytes;
+            const uint32_t st_off = ring_off + static_cast<uint32_t>(slot) * p.stage_bytes;
             const int b_rel = rb > 0 ? rb : 0;
             const int e_rel = (rb + span) < T.team_len ? (rb + span) : T.team_len;
             const int nsb_stage = e_rel - b_rel;
@@ -412,28 +418,44 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             {
                 const int idx = du * nsb + dbl - head;
                 if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage))
-                    decode4(st + static_cast<size_t>(idx) * kBlockBytes, dhalf, dec_out);
+                    decode4(smem + st_off + static_cast<uint32_t>(idx) * kBlockBytes, dhalf,
+                            reinterpret_cast<float4*>(smem + dec_off));
             }
             __syncwarp();
 
             // The stage's (up to) kSeg row segments, branch-free: a lane whose
             // superblock is not in a segment computes on superblock 0 and the
-            // result is discarded by a select.
-            float part_sum[M][kSeg];
+            // result is discarded by a select. Item u + 1's operands are loaded
+            // while item u computes.
+            bool use[kSeg];
+            uint32_t qaddr[kSeg];
 #pragma unroll
             for (int u = 0; u < kSeg; ++u) {
                 const int idx = u * nsb - head + bl;
-                const bool use = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
-                const int off = use ? (u * nsb - head) * kBlockBytes : -bl * kBlockBytes;
-                const uint4 q = *reinterpret_cast<const uint4*>(st + lane_qoff + off);
-                const float4 clo = lane_coef[u * 32], chi = lane_coef[u * 32 + 1];
+                use[u] = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
+                qaddr[u] = st_off + (use[u] ? lane_qoff + static_cast<uint32_t>((u * nsb - head) * kBlockBytes)
+                                            : static_cast<uint32_t>(kQsOffset + 16 * c));
+            }
+            float part_sum[M][kSeg];
+            uint4 qn = *reinterpret_cast<const uint4*>(smem + qaddr[0]);
+            float4 clon = *reinterpret_cast<const float4*>(smem + lane_coef_off);
+            float4 chin = *reinterpret_cast<const float4*>(smem + lane_coef_off + 16);
+#pragma unroll
+            for (int u = 0; u < kSeg; ++u) {
+                const uint4 q = qn;
+                const float4 clo = clon, chi = chin;
+                if (u + 1 < kSeg) {
+                    qn = *reinterpret_cast<const uint4*>(smem + qaddr[u + 1]);
+                    clon = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * 512);
+                    chin = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * 512 + 16);
+                }
                 float2 acc[M][4];
                 dot_item<M>(q, clo, chi, xlo, xhi, acc);
 #pragma unroll
                 for (int i = 0; i < M; ++i) {
                     const float2 t = __fadd2_rn(__fadd2_rn(acc[i][0], acc[i][1]),
                                                 __fadd2_rn(acc[i][2], acc[i][3]));
-                    part_sum[i][u] = use ? (t.x + t.y) : 0.f;
+                    part_sum[i][u] = use[u] ? (t.x + t.y) : 0.f;
                 }
             }
             float* rbuf = T.red + static_cast<size_t>(slot) * red_slot;
