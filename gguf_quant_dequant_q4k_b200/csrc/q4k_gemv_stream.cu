@@ -9,12 +9,12 @@
 // B200 instead:
 //
 // * Work split. One persistent CTA per SM owns a balanced, contiguous range of
-//   whole rows (counts differ by at most one). The CTA's warps form T "teams";
-//   the CTA's superblocks (rows x K/256, contiguous in memory) are cut into T
-//   equal contiguous pieces at superblock granularity, one per team, so every
-//   team streams the same number of bytes. A row cut between two teams is
-//   finished from the teams' partial sums in shared memory, in team order
-//   (deterministic; no atomics, no global workspace).
+//   whole rows (counts differ by at most one). The CTA's compute warps form T
+//   "teams"; the CTA's superblocks (rows x K/256, contiguous in memory) are
+//   cut into T equal contiguous pieces at superblock granularity, one per
+//   team, so every team streams the same number of bytes. A row cut between
+//   two teams is finished from the teams' partial sums in shared memory, in
+//   team order (deterministic; no atomics, no global workspace).
 // * x-stationary. A team has ceil(K/1024) warps: team lane l owns the 16-byte
 //   quant slice c = l%8 of superblock position b = l/8 of every row, i.e. 32
 //   fixed weights of K (16 low nibbles of sub-block 2g and 16 high nibbles of
@@ -23,24 +23,27 @@
 //   is no K*4-byte shared-memory ceiling.
 // * Streaming. Each team streams its byte range through a ring of `depth`
 //   shared-memory stages with 1-D bulk async copies (cp.async.bulk, completing
-//   on an mbarrier; no multicast). A stage is up to 4 consecutive row segments
-//   (one contiguous copy). Every weight byte is read from HBM once. The first
-//   `depth` copies are issued before griddepcontrol.wait, so under
+//   on a "full" mbarrier; no multicast). A stage is up to 4 consecutive row
+//   segments (one contiguous copy). Every weight byte is read from HBM once.
+//   One producer warp per CTA (lane t serves team t) issues the copies, polls
+//   each team's "done" mbarrier (one arrival per warp per stage), adds the
+//   warps' partials of a drained stage into y and refills its slot at once.
+//   The first `depth` copies are issued before griddepcontrol.wait, so under
 //   programmatic dependent launch they overlap the previous kernel's tail.
-// * Decode. Once per stage the team decodes each superblock header (d, dmin,
-//   12 scale bytes; GGUF get_scale_min_k4 packing) into eight (A_j, B_j)
-//   pairs with A_j = 128*d*sc_j (exact) and B_j = -(A_j + dmin*m_j). A weight
-//   with quant q is then A_j*f + B_j where f = 1 + q/128 is built by one byte
-//   permute into the mantissa of 1.0 (exact): d*sc_j*q - dmin*m_j rounded
-//   once (B_j's own rounding, at most half an ulp of 128*d*sc_j + dmin*m_j, is
-//   the only other error). Weights and dot products use packed f32x2 FMAs.
+// * Decode. Once per stage each warp decodes the headers of its superblocks
+//   (d, dmin, 12 scale bytes; GGUF get_scale_min_k4 packing) into (A_j, B_j)
+//   pairs with A_j = 256*d*sc_j (exact) and B_j = -(128*d*sc_j + dmin*m_j).
+//   A weight with quant q is then A_j*f + B_j where f = 1/2 + q/256 is built by
+//   one byte permute of the masked nibble into the mantissa of 1/2 (exact):
+//   d*sc_j*q - dmin*m_j rounded once (B_j's own rounding, at most half an ulp
+//   of 128*d*sc_j + dmin*m_j, is the only other error). Weights and dot
+//   products use packed f32x2 FMAs.
 // * Reduction. Per stage each lane holds one partial per row segment; a
 //   4-segment transpose-reduce across the warp (5 shuffles) leaves one value
-//   per segment, and the team's warps are summed in shared memory.
+//   per segment, published to shared memory for the producer lane to add.
 //
-// Synchronisation per stage: wait on the stage's mbarrier (bounded), decode,
-// one named barrier per team; the team leader then refills the stage consumed
-// in the previous iteration and finishes the previous stage's row sums.
+// All waits are bounded: a wait that gives up raises a device fault flag
+// (q4k_device_fault_flags) and the kernel skips its remaining work.
 #include <cstdint>
 #include <cuda_fp16.h>
 
@@ -58,12 +61,12 @@ namespace {
 __device__ unsigned int g_fault_flags = 0;
 
 constexpr int kSeg = kStreamSegRows;         // row segments per stage
-constexpr uint32_t kMagicOne = 0x3F000000u;  // bytes 0,1 = 0x00, byte 3 = 0x3F
+constexpr uint32_t kMagicOne = 0x3F000000u;  // 1/2: bytes 0..2 = 0x00, byte 3 = 0x3F
 constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
 constexpr int kCoefFloatsPerWarp = kSeg * 4 * 8 * 4;  // [seg][4 positions][8 sub-blocks][A A B B]
 
-// f = 1 + q/128 for the nibble held in byte SEL of `masked` (bytes 0x80 | q):
-// the byte becomes bits 16..23 of 0x3F800000 + q * 2^16.
+// f = 1/2 + q/256 for the nibble q held in byte SEL of `masked` (bytes 0..15):
+// the byte becomes bits 16..23 of 0x3F000000 (1/2), i.e. mantissa bits 16..19.
 template <int SEL>
 __device__ __forceinline__ float nib_to_f(uint32_t masked) {
     return __uint_as_float(__byte_perm(masked, kMagicOne, 0x7054 | (SEL << 8)));
@@ -123,7 +126,9 @@ __device__ __forceinline__ void stage_span(const TeamRange& r, int t, int nsb, l
 }
 
 // Sub-blocks 4*half .. 4*half+3 of one superblock header -> four (A, A, B, B)
-// float4s: A_j = 128*d*sc_j (exact), B_j = -(A_j + dmin*m_j).
+// float4s with A_j = 256*d*sc_j and B_j = -(128*d*sc_j + dmin*m_j), so that
+// A_j*(1/2 + q/256) + B_j = d*sc_j*q - dmin*m_j. A_j and the two products are
+// exact; B_j is rounded once.
 __device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out) {
     const uint4 h = *reinterpret_cast<const uint4*>(sb);
     const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu)));
@@ -135,16 +140,18 @@ __device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out
                              : (h.z & 0x3F3F3F3Fu);
     const float d128 = d * 128.0f;
     // (2^23 + v) * s - 2^23 * s == v * s exactly for the 6-bit v and these s.
-    const float2 sa = make_float2(d128, d128), sb2 = make_float2(-8388608.0f * d128, -8388608.0f * d128);
-    const float2 ma = make_float2(dmin, dmin), mb = make_float2(-8388608.0f * dmin, -8388608.0f * dmin);
-    const float2 a01 = ffma2(sa, make_float2(byte_2p23<0>(sc), byte_2p23<1>(sc)), sb2);
+    const float2 sa = make_float2(d128, d128);
+    const float2 sb2 = make_float2(-8388608.0f * d128, -8388608.0f * d128);
+    const float2 ma = make_float2(dmin, dmin);
+    const float2 mb = make_float2(-8388608.0f * dmin, -8388608.0f * dmin);
+    const float2 a01 = ffma2(sa, make_float2(byte_2p23<0>(sc), byte_2p23<1>(sc)), sb2);  // 128 d sc
     const float2 a23 = ffma2(sa, make_float2(byte_2p23<2>(sc), byte_2p23<3>(sc)), sb2);
-    const float2 m01 = ffma2(ma, make_float2(byte_2p23<0>(mm), byte_2p23<1>(mm)), mb);
+    const float2 m01 = ffma2(ma, make_float2(byte_2p23<0>(mm), byte_2p23<1>(mm)), mb);  // dmin m
     const float2 m23 = ffma2(ma, make_float2(byte_2p23<2>(mm), byte_2p23<3>(mm)), mb);
-    out[0] = make_float4(a01.x, a01.x, -a01.x - m01.x, -a01.x - m01.x);
-    out[1] = make_float4(a01.y, a01.y, -a01.y - m01.y, -a01.y - m01.y);
-    out[2] = make_float4(a23.x, a23.x, -a23.x - m23.x, -a23.x - m23.x);
-    out[3] = make_float4(a23.y, a23.y, -a23.y - m23.y, -a23.y - m23.y);
+    out[0] = make_float4(2.f * a01.x, 2.f * a01.x, -a01.x - m01.x, -a01.x - m01.x);
+    out[1] = make_float4(2.f * a01.y, 2.f * a01.y, -a01.y - m01.y, -a01.y - m01.y);
+    out[2] = make_float4(2.f * a23.x, 2.f * a23.x, -a23.x - m23.x, -a23.x - m23.x);
+    out[3] = make_float4(2.f * a23.y, 2.f * a23.y, -a23.y - m23.y, -a23.y - m23.y);
 }
 
 // This lane's 32 weights of one row against its x registers, in four
@@ -159,8 +166,8 @@ __device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const 
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
         const uint32_t w = words[wi];
-        const uint32_t lo = (w & 0x0F0F0F0Fu) | 0x80808080u;
-        const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) | 0x80808080u;
+        const uint32_t lo = w & 0x0F0F0F0Fu;
+        const uint32_t hi = __umulhi(w, 1u << 28) & 0x0F0F0F0Fu;   // (w >> 4) on the FMA pipe
         const float2 wlo0 = ffma2(alo, make_float2(nib_to_f<0>(lo), nib_to_f<1>(lo)), blo);
         const float2 wlo1 = ffma2(alo, make_float2(nib_to_f<2>(lo), nib_to_f<3>(lo)), blo);
         const float2 whi0 = ffma2(ahi, make_float2(nib_to_f<0>(hi), nib_to_f<1>(hi)), bhi);
