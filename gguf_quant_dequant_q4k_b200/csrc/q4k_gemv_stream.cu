@@ -63,7 +63,7 @@ __device__ unsigned int g_fault_flags = 0;
 constexpr int kSeg = kStreamSegRows;         // row segments per stage
 constexpr uint32_t kMagicOne = 0x3F000000u;  // 1/2: bytes 0..2 = 0x00, byte 3 = 0x3F
 constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
-constexpr int kCoefFloatsPerWarp = kSeg * 4 * 8 * 4;  // [seg][4 positions][8 sub-blocks][A A B B]
+constexpr int kCoefFloatsPerWarp = kSeg * 4 * 4 * 4;  // [seg][4 positions][4 groups][A A' B B']
 
 // f = 1/2 + q/256 for the nibble q held in byte SEL of `masked` (bytes 0..15):
 // the byte becomes bits 16..23 of 0x3F000000 (1/2), i.e. mantissa bits 16..19.
@@ -116,20 +116,13 @@ __device__ __forceinline__ long long seg_end(const TeamRange& r, int i, int nsb)
     return e < r.s1 ? e : r.s1;
 }
 
-// Stage t of a team: flat superblock range [b, e) covering its segments.
-__device__ __forceinline__ void stage_span(const TeamRange& r, int t, int nsb, long long& b,
-                                           long long& e) {
-    const int i0 = t * kSeg;
-    const int i1 = (i0 + kSeg < r.nseg ? i0 + kSeg : r.nseg) - 1;
-    b = seg_begin(r, i0, nsb);
-    e = seg_end(r, i1, nsb);
-}
 
-// Sub-blocks 4*half .. 4*half+3 of one superblock header -> four (A, A, B, B)
-// float4s with A_j = 256*d*sc_j and B_j = -(128*d*sc_j + dmin*m_j), so that
+// Sub-blocks 4*half .. 4*half+3 of one superblock header, i.e. 64-weight groups
+// g = 2*half and 2*half+1, -> two float4s (A_2g, A_2g+1, B_2g, B_2g+1) with
+// A_j = 256*d*sc_j and B_j = -(128*d*sc_j + dmin*m_j), so that
 // A_j*(1/2 + q/256) + B_j = d*sc_j*q - dmin*m_j. A_j and the two products are
-// exact; B_j is rounded once.
-__device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out) {
+// exact; B_j is rounded once. out0/out1 receive groups 2*half and 2*half+1.
+__device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out0, float4* out1) {
     const uint4 h = *reinterpret_cast<const uint4*>(sb);
     const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu)));
     const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x >> 16)));
@@ -148,42 +141,44 @@ __device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out
     const float2 a23 = ffma2(sa, make_float2(byte_2p23<2>(sc), byte_2p23<3>(sc)), sb2);
     const float2 m01 = ffma2(ma, make_float2(byte_2p23<0>(mm), byte_2p23<1>(mm)), mb);  // dmin m
     const float2 m23 = ffma2(ma, make_float2(byte_2p23<2>(mm), byte_2p23<3>(mm)), mb);
-    out[0] = make_float4(2.f * a01.x, 2.f * a01.x, -a01.x - m01.x, -a01.x - m01.x);
-    out[1] = make_float4(2.f * a01.y, 2.f * a01.y, -a01.y - m01.y, -a01.y - m01.y);
-    out[2] = make_float4(2.f * a23.x, 2.f * a23.x, -a23.x - m23.x, -a23.x - m23.x);
-    out[3] = make_float4(2.f * a23.y, 2.f * a23.y, -a23.y - m23.y, -a23.y - m23.y);
+    const float2 A01 = __fadd2_rn(a01, a01), A23 = __fadd2_rn(a23, a23);
+    const float2 s01 = __fadd2_rn(a01, m01), s23 = __fadd2_rn(a23, m23);
+    *out0 = make_float4(A01.x, A01.y, -s01.x, -s01.y);
+    *out1 = make_float4(A23.x, A23.y, -s23.x, -s23.y);
 }
 
-// This lane's 32 weights of one row against its x registers, in four
-// independent f32x2 chains per vector (acc[i][0..3]); the first product
-// initialises each chain.
+// This lane's 32 weights of one row against its x registers. Byte e of the
+// 16-byte quant slice holds the low nibble (weight of sub-block 2g) and the
+// high nibble (sub-block 2g+1); the two form one f32x2 lane pair with
+// coefficients (A_2g, A_2g+1), (B_2g, B_2g+1) and x pair xp[i][e]. Four
+// independent accumulator chains per vector; the first product initialises
+// each chain.
 template <int M>
-__device__ __forceinline__ void dot_item(uint4 q, float4 clo, float4 chi, const float2 (&xlo)[M][8],
-                                         const float2 (&xhi)[M][8], float2 (&acc)[M][4]) {
-    const float2 alo = make_float2(clo.x, clo.y), blo = make_float2(clo.z, clo.w);
-    const float2 ahi = make_float2(chi.x, chi.y), bhi = make_float2(chi.z, chi.w);
+__device__ __forceinline__ void dot_item(uint4 q, float4 cf, const float2 (&xp)[M][16],
+                                         float2 (&acc)[M][4]) {
+    const float2 a = make_float2(cf.x, cf.y), b = make_float2(cf.z, cf.w);
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi) {
         const uint32_t w = words[wi];
         const uint32_t lo = w & 0x0F0F0F0Fu;
         const uint32_t hi = __umulhi(w, 1u << 28) & 0x0F0F0F0Fu;   // (w >> 4) on the FMA pipe
-        const float2 wlo0 = ffma2(alo, make_float2(nib_to_f<0>(lo), nib_to_f<1>(lo)), blo);
-        const float2 wlo1 = ffma2(alo, make_float2(nib_to_f<2>(lo), nib_to_f<3>(lo)), blo);
-        const float2 whi0 = ffma2(ahi, make_float2(nib_to_f<0>(hi), nib_to_f<1>(hi)), bhi);
-        const float2 whi1 = ffma2(ahi, make_float2(nib_to_f<2>(hi), nib_to_f<3>(hi)), bhi);
+        const float2 w0 = ffma2(a, make_float2(nib_to_f<0>(lo), nib_to_f<0>(hi)), b);
+        const float2 w1 = ffma2(a, make_float2(nib_to_f<1>(lo), nib_to_f<1>(hi)), b);
+        const float2 w2 = ffma2(a, make_float2(nib_to_f<2>(lo), nib_to_f<2>(hi)), b);
+        const float2 w3 = ffma2(a, make_float2(nib_to_f<3>(lo), nib_to_f<3>(hi)), b);
 #pragma unroll
         for (int i = 0; i < M; ++i) {
             if (wi == 0) {
-                acc[i][0] = __fmul2_rn(wlo0, xlo[i][0]);
-                acc[i][1] = __fmul2_rn(whi0, xhi[i][0]);
-                acc[i][2] = __fmul2_rn(wlo1, xlo[i][1]);
-                acc[i][3] = __fmul2_rn(whi1, xhi[i][1]);
+                acc[i][0] = __fmul2_rn(w0, xp[i][0]);
+                acc[i][1] = __fmul2_rn(w1, xp[i][1]);
+                acc[i][2] = __fmul2_rn(w2, xp[i][2]);
+                acc[i][3] = __fmul2_rn(w3, xp[i][3]);
             } else {
-                acc[i][0] = ffma2(wlo0, xlo[i][2 * wi], acc[i][0]);
-                acc[i][1] = ffma2(whi0, xhi[i][2 * wi], acc[i][1]);
-                acc[i][2] = ffma2(wlo1, xlo[i][2 * wi + 1], acc[i][2]);
-                acc[i][3] = ffma2(whi1, xhi[i][2 * wi + 1], acc[i][3]);
+                acc[i][0] = ffma2(w0, xp[i][4 * wi + 0], acc[i][0]);
+                acc[i][1] = ffma2(w1, xp[i][4 * wi + 1], acc[i][1]);
+                acc[i][2] = ffma2(w2, xp[i][4 * wi + 2], acc[i][2]);
+                acc[i][3] = ffma2(w3, xp[i][4 * wi + 3], acc[i][3]);
             }
         }
     }
@@ -360,19 +355,19 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const int wit = warp % p.team_warps;
         const int tl = wit * 32 + lane;
         const Team T = make_team<M>(p, smem, team);
-        float* wcoef = reinterpret_cast<float*>(smem + p.off_coef) +
-                       static_cast<size_t>(warp) * kCoefFloatsPerWarp;
         pdl_launch_dependents();
         pdl_wait();   // x and y belong to the dependency chain
 
         // This lane's fixed slice of K and its x values.
         const bool valid = tl < 8 * nsb;
         const int bl = tl >> 3, c = tl & 7, g = c >> 1, h = c & 1;
-        float2 xlo[M][8], xhi[M][8];
+        // xp[i][e] = (x of the low nibble of byte e, x of its high nibble):
+        // weights 64g + 16h + e and 64g + 32 + 16h + e of superblock position bl.
+        float2 xp[M][16];
 #pragma unroll
         for (int i = 0; i < M; ++i) {
 #pragma unroll
-            for (int v = 0; v < 8; ++v) xlo[i][v] = xhi[i][v] = make_float2(0.f, 0.f);
+            for (int e = 0; e < 16; ++e) xp[i][e] = make_float2(0.f, 0.f);
         }
         if (valid) {
             const int k0 = bl * kQK + 64 * g + 16 * h;
@@ -380,14 +375,14 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             for (int i = 0; i < M; ++i) {
                 const float4* xl =
                     reinterpret_cast<const float4*>(p.x + static_cast<size_t>(i) * p.k + k0);
-                const float4* xh = xl + 8;
+                const float4* xh = xl + 8;   // + 32 weights
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     const float4 a = __ldg(xl + v), b = __ldg(xh + v);
-                    xlo[i][2 * v] = make_float2(a.x, a.y);
-                    xlo[i][2 * v + 1] = make_float2(a.z, a.w);
-                    xhi[i][2 * v] = make_float2(b.x, b.y);
-                    xhi[i][2 * v + 1] = make_float2(b.z, b.w);
+                    xp[i][4 * v + 0] = make_float2(a.x, b.x);
+                    xp[i][4 * v + 1] = make_float2(a.y, b.y);
+                    xp[i][4 * v + 2] = make_float2(a.z, b.z);
+                    xp[i][4 * v + 3] = make_float2(a.w, b.w);
                 }
             }
         }
@@ -404,8 +399,13 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c);
         const uint32_t coef_off = static_cast<uint32_t>(p.off_coef) +
                                   static_cast<uint32_t>(warp) * kCoefFloatsPerWarp * 4u;
-        const uint32_t lane_coef_off = coef_off + static_cast<uint32_t>(((lane >> 3) * 8 + 2 * g) * 16);
-        const uint32_t dec_off = coef_off + static_cast<uint32_t>(((du * 4 + dpos) * 8 + 4 * dhalf) * 16);
+        // Coefficient float4 of (segment u, position pos, group g) sits at
+        // index (u*4 + pos)*4 + (g ^ (pos >> 1)): conflict-free for both the
+        // decode stores and the item loads.
+        const int lpos = lane >> 3;
+        const uint32_t lane_coef_off = coef_off + static_cast<uint32_t>((lpos * 4 + (g ^ (lpos >> 1))) * 16);
+        const uint32_t dec_off0 = coef_off + static_cast<uint32_t>(((du * 4 + dpos) * 4 + ((2 * dhalf) ^ (dpos >> 1))) * 16);
+        const uint32_t dec_off1 = coef_off + static_cast<uint32_t>(((du * 4 + dpos) * 4 + ((2 * dhalf + 1) ^ (dpos >> 1))) * 16);
         const int red_slot = p.team_warps * kSeg * M;
 
         int slot = 0;
@@ -426,7 +426,8 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 const int idx = du * nsb + dbl - head;
                 if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage))
                     decode4(smem + st_off + static_cast<uint32_t>(idx) * kBlockBytes, dhalf,
-                            reinterpret_cast<float4*>(smem + dec_off));
+                            reinterpret_cast<float4*>(smem + dec_off0),
+                            reinterpret_cast<float4*>(smem + dec_off1));
             }
             __syncwarp();
 
@@ -445,19 +446,17 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             }
             float part_sum[M][kSeg];
             uint4 qn = *reinterpret_cast<const uint4*>(smem + qaddr[0]);
-            float4 clon = *reinterpret_cast<const float4*>(smem + lane_coef_off);
-            float4 chin = *reinterpret_cast<const float4*>(smem + lane_coef_off + 16);
+            float4 cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off);
 #pragma unroll
             for (int u = 0; u < kSeg; ++u) {
                 const uint4 q = qn;
-                const float4 clo = clon, chi = chin;
+                const float4 cf = cfn;
                 if (u + 1 < kSeg) {
                     qn = *reinterpret_cast<const uint4*>(smem + qaddr[u + 1]);
-                    clon = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * 512);
-                    chin = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * 512 + 16);
+                    cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * 256);
                 }
                 float2 acc[M][4];
-                dot_item<M>(q, clo, chi, xlo, xhi, acc);
+                dot_item<M>(q, cf, xp, acc);
 #pragma unroll
                 for (int i = 0; i < M; ++i) {
                     const float2 t = __fadd2_rn(__fadd2_rn(acc[i][0], acc[i][1]),

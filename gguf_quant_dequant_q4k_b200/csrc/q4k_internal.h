@@ -4,7 +4,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/q4k.h"
+#include "q4k.h"  // include/ (on the include path)
 
 namespace q4k {
 

@@ -50,7 +50,7 @@ def check_plan(m, n, k):
     assert p["block"] <= (640 if m == 1 else 512) + 32
     assert 2 <= depth <= 8 and 1 <= teams <= 15
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
-    coef_per_warp = SEG * 4 * 8 * 4 * 4          # [seg][4 positions][8 sub-blocks][A A B B]
+    coef_per_warp = SEG * 4 * 4 * 4 * 4          # [seg][4 positions][4 groups][A A' B B']
     need = (teams * depth * stage_bytes + teams * team_warps * coef_per_warp
             + teams * depth * team_warps * SEG * m * 4 + teams * 2 * m * 4)
     need = -(-need // 16) * 16 + teams * 2 * depth * 8
