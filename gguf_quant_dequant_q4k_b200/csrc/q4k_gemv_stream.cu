@@ -63,7 +63,8 @@ __device__ unsigned int g_fault_flags = 0;
 constexpr int kSeg = kStreamSegRows;         // row segments per stage
 constexpr uint32_t kMagicOne = 0x3F000000u;  // 1/2: bytes 0..2 = 0x00, byte 3 = 0x3F
 constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
-constexpr int kCoefFloatsPerWarp = kSeg * 4 * 4 * 4;  // [seg][4 positions][4 groups][A A' B B']
+// Coefficient buffer per warp: [segment][position][4 groups] float4s.
+constexpr int coef_bytes_per_warp(int m) { return kSeg * (4 * stream_slices(m)) * 4 * 16; }
 
 // f = 1/2 + q/256 for the nibble q held in byte SEL of `masked` (bytes 0..15):
 // the byte becomes bits 16..23 of 0x3F000000 (1/2), i.e. mantissa bits 16..19.
@@ -117,15 +118,12 @@ __device__ __forceinline__ long long seg_end(const TeamRange& r, int i, int nsb)
 }
 
 
-// Sub-blocks 4*half .. 4*half+3 of one superblock header, i.e. 64-weight groups
-// g = 2*half and 2*half+1, -> two float4s (A_2g, A_2g+1, B_2g, B_2g+1) with
-// A_j = 256*d*sc_j and B_j = -(128*d*sc_j + dmin*m_j), so that
-// A_j*(1/2 + q/256) + B_j = d*sc_j*q - dmin*m_j. A_j and the two products are
-// exact; B_j is rounded once. out0/out1 receive groups 2*half and 2*half+1.
-__device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out0, float4* out1) {
-    const uint4 h = *reinterpret_cast<const uint4*>(sb);
-    const float d = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu)));
-    const float dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x >> 16)));
+// (A_2g, A_2g+1, B_2g, B_2g+1) for the two 64-weight groups g = 2*half and
+// 2*half+1 of one superblock header h (bytes 0..15), with A_j = 256*d*sc_j and
+// B_j = -(128*d*sc_j + dmin*m_j), so that A_j*(1/2 + q/256) + B_j =
+// d*sc_j*q - dmin*m_j. A_j and the two products are exact; B_j is rounded once.
+__device__ __forceinline__ void decode_half(uint4 h, float d, float dmin, int half, float4& out0,
+                                            float4& out1) {
     // six-bit fields of sub-blocks 4*half .. +3 (GGUF get_scale_min_k4 packing)
     const uint32_t sc = half ? ((h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u))
                              : (h.y & 0x3F3F3F3Fu);
@@ -143,43 +141,41 @@ __device__ __forceinline__ void decode4(const uint8_t* sb, int half, float4* out
     const float2 m23 = ffma2(ma, make_float2(byte_2p23<2>(mm), byte_2p23<3>(mm)), mb);
     const float2 A01 = __fadd2_rn(a01, a01), A23 = __fadd2_rn(a23, a23);
     const float2 s01 = __fadd2_rn(a01, m01), s23 = __fadd2_rn(a23, m23);
-    *out0 = make_float4(A01.x, A01.y, -s01.x, -s01.y);
-    *out1 = make_float4(A23.x, A23.y, -s23.x, -s23.y);
+    out0 = make_float4(A01.x, A01.y, -s01.x, -s01.y);
+    out1 = make_float4(A23.x, A23.y, -s23.x, -s23.y);
 }
 
-// This lane's 32 weights of one row against its x registers. Byte e of the
-// 16-byte quant slice holds the low nibble (weight of sub-block 2g) and the
-// high nibble (sub-block 2g+1); the two form one f32x2 lane pair with
-// coefficients (A_2g, A_2g+1), (B_2g, B_2g+1) and x pair xp[i][e]. Four
-// independent accumulator chains per vector; the first product initialises
-// each chain.
-template <int M>
-__device__ __forceinline__ void dot_item(uint4 q, float4 cf, const float2 (&xp)[M][16],
-                                         float2 (&acc)[M][4]) {
-    const float2 a = make_float2(cf.x, cf.y), b = make_float2(cf.z, cf.w);
-    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+__device__ __forceinline__ void header_scales(uint4 h, float& d, float& dmin) {
+    d = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu)));
+    dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x >> 16)));
+}
+
+// One 32-bit word of quants (bytes e = 0..3; low nibble = weight of sub-block
+// 2g, high nibble = weight of sub-block 2g+1) against x pairs xp[i][e0 + e]:
+// the two nibbles of a byte form one f32x2 lane pair with coefficients
+// a = (A_2g, A_2g+1), b = (B_2g, B_2g+1). Accumulates into acc[i][e]; `first`
+// initialises the chains.
+template <int M, int NX>
+__device__ __forceinline__ void dot_word(uint32_t w, float2 a, float2 b, const float2 (&xp)[M][NX],
+                                         int e0, bool first, float2 (&acc)[M][4]) {
+    const uint32_t lo = w & 0x0F0F0F0Fu;
+    const uint32_t hi = __umulhi(w, 1u << 28) & 0x0F0F0F0Fu;   // (w >> 4) on the FMA pipe
+    const float2 w0 = ffma2(a, make_float2(nib_to_f<0>(lo), nib_to_f<0>(hi)), b);
+    const float2 w1 = ffma2(a, make_float2(nib_to_f<1>(lo), nib_to_f<1>(hi)), b);
+    const float2 w2 = ffma2(a, make_float2(nib_to_f<2>(lo), nib_to_f<2>(hi)), b);
+    const float2 w3 = ffma2(a, make_float2(nib_to_f<3>(lo), nib_to_f<3>(hi)), b);
 #pragma unroll
-    for (int wi = 0; wi < 4; ++wi) {
-        const uint32_t w = words[wi];
-        const uint32_t lo = w & 0x0F0F0F0Fu;
-        const uint32_t hi = __umulhi(w, 1u << 28) & 0x0F0F0F0Fu;   // (w >> 4) on the FMA pipe
-        const float2 w0 = ffma2(a, make_float2(nib_to_f<0>(lo), nib_to_f<0>(hi)), b);
-        const float2 w1 = ffma2(a, make_float2(nib_to_f<1>(lo), nib_to_f<1>(hi)), b);
-        const float2 w2 = ffma2(a, make_float2(nib_to_f<2>(lo), nib_to_f<2>(hi)), b);
-        const float2 w3 = ffma2(a, make_float2(nib_to_f<3>(lo), nib_to_f<3>(hi)), b);
-#pragma unroll
-        for (int i = 0; i < M; ++i) {
-            if (wi == 0) {
-                acc[i][0] = __fmul2_rn(w0, xp[i][0]);
-                acc[i][1] = __fmul2_rn(w1, xp[i][1]);
-                acc[i][2] = __fmul2_rn(w2, xp[i][2]);
-                acc[i][3] = __fmul2_rn(w3, xp[i][3]);
-            } else {
-                acc[i][0] = ffma2(w0, xp[i][4 * wi + 0], acc[i][0]);
-                acc[i][1] = ffma2(w1, xp[i][4 * wi + 1], acc[i][1]);
-                acc[i][2] = ffma2(w2, xp[i][4 * wi + 2], acc[i][2]);
-                acc[i][3] = ffma2(w3, xp[i][4 * wi + 3], acc[i][3]);
-            }
+    for (int i = 0; i < M; ++i) {
+        if (first) {
+            acc[i][0] = __fmul2_rn(w0, xp[i][e0 + 0]);
+            acc[i][1] = __fmul2_rn(w1, xp[i][e0 + 1]);
+            acc[i][2] = __fmul2_rn(w2, xp[i][e0 + 2]);
+            acc[i][3] = __fmul2_rn(w3, xp[i][e0 + 3]);
+        } else {
+            acc[i][0] = ffma2(w0, xp[i][e0 + 0], acc[i][0]);
+            acc[i][1] = ffma2(w1, xp[i][e0 + 1], acc[i][1]);
+            acc[i][2] = ffma2(w2, xp[i][e0 + 2], acc[i][2]);
+            acc[i][3] = ffma2(w3, xp[i][e0 + 3], acc[i][3]);
         }
     }
 }
@@ -246,7 +242,7 @@ __device__ __forceinline__ Team make_team(const StreamParams& p, uint8_t* smem, 
     return t;
 }
 
-// Stage `st` (first row start rb team-relative) -> one bulk copy into `slot`.
+// Stage with first row start rb (team-relative) -> one bulk copy into `slot`.
 __device__ __forceinline__ void issue_stage(const Team& T, const StreamParams& p, int rb, int slot) {
     const int span = kSeg * p.nsb;
     const int b_rel = rb > 0 ? rb : 0;
@@ -257,11 +253,15 @@ __device__ __forceinline__ void issue_stage(const Team& T, const StreamParams& p
                   T.w + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &T.full[slot]);
 }
 
-template <int M>
-__global__ void __launch_bounds__(stream_max_threads(M) + 32, 1)
+// M vectors, S 16-byte quant slices (S*32 weights) per lane per row.
+template <int M, int S>
+__global__ void __maxnreg__(stream_max_regs(M))
 q4k_gemv_stream_kernel(const StreamParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ volatile int abort_flag;
+    constexpr int kLanesPerSb = 8 / S;        // lanes covering one superblock of a row
+    constexpr int kPos = 32 / kLanesPerSb;    // superblock positions per warp
+    constexpr int kNX = 16 * S;               // x pairs per lane per vector
     const int nsb = p.nsb;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -339,7 +339,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 atomicOr(&g_fault_flags, kFaultCopyTimeout);
                 abort_flag = 1;
             }
-            if (!__any_sync(0xFFFFFFFFu, progressed)) __nanosleep(32);
+            if (!__any_sync(0xFFFFFFFFu, progressed)) __nanosleep(64);
         }
         // After a lost copy, give the copies still in flight a bounded chance
         // to land before the CTA's shared memory is released.
@@ -353,31 +353,34 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         // ------------------------------------------------------------ compute
         const int team = warp / p.team_warps;
         const int wit = warp % p.team_warps;
-        const int tl = wit * 32 + lane;
         const Team T = make_team<M>(p, smem, team);
         pdl_launch_dependents();
         pdl_wait();   // x and y belong to the dependency chain
 
-        // This lane's fixed slice of K and its x values.
-        const bool valid = tl < 8 * nsb;
-        const int bl = tl >> 3, c = tl & 7, g = c >> 1, h = c & 1;
-        // xp[i][e] = (x of the low nibble of byte e, x of its high nibble):
-        // weights 64g + 16h + e and 64g + 32 + 16h + e of superblock position bl.
-        float2 xp[M][16];
+        // This lane's superblock position bl and its slices c0 .. c0+S-1 of the
+        // 8 16-byte quant slices: group g = c0/2 (sub-blocks 2g, 2g+1).
+        const int lpos = lane / kLanesPerSb;
+        const int c0 = (lane % kLanesPerSb) * S;
+        const int g = c0 >> 1;
+        const int bl = wit * kPos + lpos;
+        const bool valid = bl < nsb;
+        // xp[i][e] = (x of the low nibble of byte e of the lane's quant bytes, x
+        // of its high nibble): weights k0 + e and k0 + 32 + e.
+        float2 xp[M][kNX];
 #pragma unroll
         for (int i = 0; i < M; ++i) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) xp[i][e] = make_float2(0.f, 0.f);
+            for (int e = 0; e < kNX; ++e) xp[i][e] = make_float2(0.f, 0.f);
         }
         if (valid) {
-            const int k0 = bl * kQK + 64 * g + 16 * h;
+            const int k0 = bl * kQK + 64 * g + 16 * (c0 & 1);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
                 const float4* xl =
                     reinterpret_cast<const float4*>(p.x + static_cast<size_t>(i) * p.k + k0);
                 const float4* xh = xl + 8;   // + 32 weights
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
+                for (int v = 0; v < kNX / 4; ++v) {
                     const float4 a = __ldg(xl + v), b = __ldg(xh + v);
                     xp[i][4 * v + 0] = make_float2(a.x, b.x);
                     xp[i][4 * v + 1] = make_float2(a.y, b.y);
@@ -387,25 +390,24 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             }
         }
 
-        // Decode lanes: lane -> (segment du, superblock position dpos of this
-        // warp's four, half of the sub-blocks).
-        const int du = lane >> 3, dpos = (lane >> 1) & 3, dhalf = lane & 1;
-        const int dbl = 4 * wit + dpos;
+        // Shared-memory byte offsets (32-bit). The coefficient float4 of
+        // (segment u, position pos, group g) sits at (u*kPos + pos)*4 +
+        // (g ^ ((pos >> 1) & 3)): conflict-free for decode stores and item loads.
         const int span = kSeg * nsb;
-        // Shared-memory byte offsets (32-bit) of this team's ring, this lane's
-        // quant slice within a superblock row position, and this warp's
-        // coefficient buffer.
         const uint32_t ring_off = static_cast<uint32_t>(T.ring - smem);
-        const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c);
+        const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c0);
         const uint32_t coef_off = static_cast<uint32_t>(p.off_coef) +
-                                  static_cast<uint32_t>(warp) * kCoefFloatsPerWarp * 4u;
-        // Coefficient float4 of (segment u, position pos, group g) sits at
-        // index (u*4 + pos)*4 + (g ^ (pos >> 1)): conflict-free for both the
-        // decode stores and the item loads.
-        const int lpos = lane >> 3;
-        const uint32_t lane_coef_off = coef_off + static_cast<uint32_t>((lpos * 4 + (g ^ (lpos >> 1))) * 16);
-        const uint32_t dec_off0 = coef_off + static_cast<uint32_t>(((du * 4 + dpos) * 4 + ((2 * dhalf) ^ (dpos >> 1))) * 16);
-        const uint32_t dec_off1 = coef_off + static_cast<uint32_t>(((du * 4 + dpos) * 4 + ((2 * dhalf + 1) ^ (dpos >> 1))) * 16);
+                                  static_cast<uint32_t>(warp) * (kSeg * kPos * 4 * 16);
+        const uint32_t lane_coef_off =
+            coef_off + static_cast<uint32_t>((lpos * 4 + (g ^ ((lpos >> 1) & 3))) * 16);
+        // Decode lanes: S = 2: lane -> (segment du, position dpos), whole header;
+        // S = 1: lane -> (segment du, position dpos, half dhalf).
+        const int du = lane >> 3;
+        const int dpos = S == 2 ? (lane & 7) : ((lane >> 1) & 3);
+        const int dhalf = S == 2 ? 0 : (lane & 1);
+        const int dbl = wit * kPos + dpos;
+        const uint32_t dec_base = coef_off + static_cast<uint32_t>((du * kPos + dpos) * 4 * 16);
+        const int dswz = (dpos >> 1) & 3;
         const int red_slot = p.team_warps * kSeg * M;
 
         int slot = 0;
@@ -424,10 +426,20 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             // Decode this warp's superblock headers of the stage.
             {
                 const int idx = du * nsb + dbl - head;
-                if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage))
-                    decode4(smem + st_off + static_cast<uint32_t>(idx) * kBlockBytes, dhalf,
-                            reinterpret_cast<float4*>(smem + dec_off0),
-                            reinterpret_cast<float4*>(smem + dec_off1));
+                if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage)) {
+                    const uint4 hdr = *reinterpret_cast<const uint4*>(
+                        smem + st_off + static_cast<uint32_t>(idx) * kBlockBytes);
+                    float d, dmin;
+                    header_scales(hdr, d, dmin);
+#pragma unroll
+                    for (int hh = 0; hh < S; ++hh) {
+                        const int half = S == 2 ? hh : dhalf;
+                        float4 c_a, c_b;
+                        decode_half(hdr, d, dmin, half, c_a, c_b);
+                        *reinterpret_cast<float4*>(smem + dec_base + ((2 * half) ^ dswz) * 16) = c_a;
+                        *reinterpret_cast<float4*>(smem + dec_base + ((2 * half + 1) ^ dswz) * 16) = c_b;
+                    }
+                }
             }
             __syncwarp();
 
@@ -442,21 +454,34 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 const int idx = u * nsb - head + bl;
                 use[u] = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
                 qaddr[u] = st_off + (use[u] ? lane_qoff + static_cast<uint32_t>((u * nsb - head) * kBlockBytes)
-                                            : static_cast<uint32_t>(kQsOffset + 16 * c));
+                                            : static_cast<uint32_t>(kQsOffset + 16 * c0));
             }
             float part_sum[M][kSeg];
-            uint4 qn = *reinterpret_cast<const uint4*>(smem + qaddr[0]);
+            uint4 qn[S];
+#pragma unroll
+            for (int j = 0; j < S; ++j) qn[j] = *reinterpret_cast<const uint4*>(smem + qaddr[0] + 16 * j);
             float4 cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off);
 #pragma unroll
             for (int u = 0; u < kSeg; ++u) {
-                const uint4 q = qn;
+                uint4 q[S];
+#pragma unroll
+                for (int j = 0; j < S; ++j) q[j] = qn[j];
                 const float4 cf = cfn;
                 if (u + 1 < kSeg) {
-                    qn = *reinterpret_cast<const uint4*>(smem + qaddr[u + 1]);
-                    cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * 256);
+#pragma unroll
+                    for (int j = 0; j < S; ++j)
+                        qn[j] = *reinterpret_cast<const uint4*>(smem + qaddr[u + 1] + 16 * j);
+                    cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * kPos * 64);
                 }
+                const float2 a = make_float2(cf.x, cf.y), b = make_float2(cf.z, cf.w);
                 float2 acc[M][4];
-                dot_item<M>(q, cf, xp, acc);
+#pragma unroll
+                for (int j = 0; j < S; ++j) {
+                    dot_word<M, kNX>(q[j].x, a, b, xp, 16 * j + 0, j == 0, acc);
+                    dot_word<M, kNX>(q[j].y, a, b, xp, 16 * j + 4, false, acc);
+                    dot_word<M, kNX>(q[j].z, a, b, xp, 16 * j + 8, false, acc);
+                    dot_word<M, kNX>(q[j].w, a, b, xp, 16 * j + 12, false, acc);
+                }
 #pragma unroll
                 for (int i = 0; i < M; ++i) {
                     const float2 t = __fadd2_rn(__fadd2_rn(acc[i][0], acc[i][1]),
@@ -516,7 +541,8 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
                 int* block, int* smem_bytes) {
     const int nsb = k / kQK;
     if (m < 1 || m > kStreamMaxM || nsb > kStreamMaxNsb || n < 1) return 0;
-    const int team_warps = (nsb + 3) / 4;               // 8*nsb slices / 32 lanes
+    const int sl = stream_slices(m);                     // quant slices per lane
+    const int team_warps = (nsb * 8 / sl + 31) / 32;   // 8*nsb slices / (32 lanes * sl)
     const int max_warps = stream_max_threads(m) / 32;
     if (team_warps > max_warps) return 0;
     int teams = max_warps / team_warps;
@@ -527,7 +553,7 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
     // bytes per team besides its ring: coefficient buffers of its warps, the
     // per-slot partial sums, its cut-row partials and two barriers per slot
     auto fixed_team = [&](int depth) {
-        return team_warps * kCoefFloatsPerWarp * 4 + depth * team_warps * kSeg * m * 4 +
+        return team_warps * coef_bytes_per_warp(m) + depth * team_warps * kSeg * m * 4 +
                2 * m * 4 + 2 * depth * 8 + 16;
     };
     int depth = kStreamMaxDepth;
@@ -554,7 +580,7 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
     q.stage_bytes = stage_bytes;
     size_t off = static_cast<size_t>(teams) * depth * stage_bytes;
     q.off_coef = static_cast<int>(off);
-    off += static_cast<size_t>(teams) * team_warps * kCoefFloatsPerWarp * 4;
+    off += static_cast<size_t>(teams) * team_warps * coef_bytes_per_warp(m);
     q.off_red = static_cast<int>(off);
     off += static_cast<size_t>(teams) * depth * team_warps * kSeg * m * 4;
     q.off_part = static_cast<int>(off);
@@ -587,19 +613,19 @@ int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, 
     cfg.numAttrs = 1;
     cudaError_t e;
     if (m == 1) {
-        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1>, sp);
+        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, stream_slices(1)>, sp);
     } else {
-        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2>, sp);
+        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, stream_slices(2)>, sp);
     }
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
 
 int stream_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1>,
+    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, stream_slices(1)>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kStreamSmemBudget);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2>,
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, stream_slices(2)>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }

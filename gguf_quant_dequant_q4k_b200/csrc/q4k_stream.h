@@ -8,13 +8,18 @@ namespace q4k {
 
 constexpr int kStreamSegRows = 4;       // row segments per ring stage
 constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kernel
-// Threads per CTA (launch bound): 20 warps for one vector (x: 32 registers per
-// lane), 16 warps for two (x: 64 registers per lane).
-constexpr int stream_max_threads(int m) { return m == 1 ? 640 : 512; }
-constexpr int kStreamMaxNsb = 80;       // K <= 20480 (m = 1) / 16384 (m = 2): one team covers K
+// Quant slices (16 bytes = 32 weights) per lane and row: two for one vector,
+// one for two vectors (either way 64 x registers per lane).
+constexpr int stream_slices(int m) { return m == 1 ? 2 : 1; }
+// Compute threads per CTA (launch bound, plus one producer warp).
+constexpr int stream_max_threads(int m) { return m == 1 ? 512 : 512; }
+// Registers per thread so that stream_max_threads(m) + 32 threads fit the
+// 64K-register file: 120 for 17 warps.
+constexpr int stream_max_regs(int m) { return 65536 / (stream_max_threads(m) + 32) / 8 * 8; }
+constexpr int kStreamMaxNsb = 128;      // K <= 32768 (m = 1) / 16384 (m = 2): one team covers K
 constexpr int kStreamMaxTeams = 15;     // named barriers 1..15
 constexpr int kStreamMaxDepth = 8;
-constexpr int kStreamSmemBudget = 200 * 1024;
+constexpr int kStreamSmemBudget = 220 * 1024;
 
 struct StreamParams {
     const uint8_t* w;
