@@ -11,12 +11,15 @@ constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kern
 // Quant slices (16 bytes = 32 weights) per lane and row: two for one vector,
 // one for two vectors (either way 64 x registers per lane).
 constexpr int stream_slices(int m) { return m == 1 ? 2 : 1; }
-// Compute threads per CTA (launch bound, plus one producer warp).
-constexpr int stream_max_threads(int m) { return m == 1 ? 512 : 512; }
-// Registers per thread so that stream_max_threads(m) + 32 threads fit the
-// 64K-register file: 120 for 17 warps.
-constexpr int stream_max_regs(int m) { return 65536 / (stream_max_threads(m) + 32) / 8 * 8; }
-constexpr int kStreamMaxNsb = 128;      // K <= 32768 (m = 1) / 16384 (m = 2): one team covers K
+// Compute threads per CTA (plus one producer warp): 15 + 1 warps, i.e. four
+// warps on each of the SM's four sub-partitions.
+constexpr int stream_max_threads(int m) { return m == 1 ? 480 : 480; }
+// Registers per thread: each sub-partition has 16384 registers for its share
+// of the CTA's warps (allocated in multiples of 8 per thread).
+constexpr int stream_max_regs(int m) {
+    return 16384 / (((stream_max_threads(m) / 32 + 1 + 3) / 4) * 32) / 8 * 8;
+}
+constexpr int kStreamMaxNsb = 120;      // K <= 30720 (m = 1) / 15360 (m = 2): one team of <= 15 warps covers K
 constexpr int kStreamMaxTeams = 15;     // named barriers 1..15
 constexpr int kStreamMaxDepth = 8;
 constexpr int kStreamSmemBudget = 220 * 1024;
