@@ -86,18 +86,24 @@ struct TeamRange {
     int nstages;
 };
 
+// Team `team`'s superblock range in the calling CTA. Team boundaries are
+// computed CTA-relative in 32 bits (a CTA's rows*nsb is far below 2^31 for any
+// matrix whose N*K/256 fits the int arguments); only the CTA origin is 64-bit.
 __device__ __forceinline__ TeamRange team_range(const StreamParams& p, int team) {
-    const long long cta = blockIdx.x;
-    const long long rows = p.rows_base + (cta < p.rows_extra ? 1 : 0);
-    const long long row_begin = cta * p.rows_base + (cta < p.rows_extra ? cta : p.rows_extra);
-    const long long S0 = row_begin * p.nsb;
-    const long long L = rows * p.nsb;
+    const int cta = static_cast<int>(blockIdx.x);
+    const int rows = p.rows_base + (cta < p.rows_extra ? 1 : 0);
+    const long long row_begin =
+        static_cast<long long>(cta) * p.rows_base + (cta < p.rows_extra ? cta : p.rows_extra);
+    const int L = rows * p.nsb;
+    const int b = static_cast<int>((static_cast<unsigned long long>(L) * team) / p.teams);
+    const int e = static_cast<int>((static_cast<unsigned long long>(L) * (team + 1)) / p.teams);
     TeamRange r;
-    r.s0 = S0 + (L * team) / p.teams;
-    r.s1 = S0 + (L * (team + 1)) / p.teams;
-    if (r.s1 > r.s0) {
-        r.row0 = r.s0 / p.nsb;
-        r.nseg = static_cast<int>((r.s1 - 1) / p.nsb - r.row0 + 1);
+    r.s0 = row_begin * p.nsb + b;
+    r.s1 = row_begin * p.nsb + e;
+    if (e > b) {
+        const int rb = b / p.nsb;                 // CTA-relative first row
+        r.row0 = row_begin + rb;
+        r.nseg = (e - 1) / p.nsb - rb + 1;
         r.nstages = (r.nseg + kSeg - 1) / kSeg;
     } else {
         r.row0 = 0;

@@ -8,18 +8,19 @@ namespace q4k {
 
 constexpr int kStreamSegRows = 4;       // row segments per ring stage
 constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kernel
-// Quant slices (16 bytes = 32 weights) per lane and row: two for one vector,
-// one for two vectors (either way 64 x registers per lane).
-constexpr int stream_slices(int m) { return m == 1 ? 2 : 1; }
-// Compute threads per CTA (plus one producer warp): 15 + 1 warps, i.e. four
-// warps on each of the SM's four sub-partitions.
-constexpr int stream_max_threads(int m) { return m == 1 ? 480 : 480; }
-// Registers per thread: each sub-partition has 16384 registers for its share
-// of the CTA's warps (allocated in multiples of 8 per thread).
+// Quant slices (16 bytes = 32 weights) per lane and row. Measured on B200: one
+// slice per lane with more warps beats two slices with fewer warps on every
+// decode shape but the largest (within 2% there).
+constexpr int stream_slices(int m) { return m == 1 ? 1 : 1; }
+// Compute threads per CTA (plus one producer warp): 20 + 1 warps for one vector
+// (x: 32 registers per lane), 15 + 1 for two (x: 64 registers per lane).
+constexpr int stream_max_threads(int m) { return m == 1 ? 640 : 480; }
+// Registers per thread: each of the SM's four sub-partitions has 16384
+// registers for its share of the CTA's warps (allocated in multiples of 8).
 constexpr int stream_max_regs(int m) {
     return 16384 / (((stream_max_threads(m) / 32 + 1 + 3) / 4) * 32) / 8 * 8;
 }
-constexpr int kStreamMaxNsb = 120;      // K <= 30720 (m = 1) / 15360 (m = 2): one team of <= 15 warps covers K
+constexpr int kStreamMaxNsb = 80;       // K <= 20480 (m = 1) / 15360 (m = 2): one team covers K
 constexpr int kStreamMaxTeams = 15;     // named barriers 1..15
 constexpr int kStreamMaxDepth = 8;
 constexpr int kStreamSmemBudget = 220 * 1024;

@@ -45,10 +45,10 @@ def check_plan(m, n, k):
         return p
     nsb = k // 256
     ctas, teams, depth = p["grid"], p["teams"], p["depth"]
-    slices = 2 if m == 1 else 1                          # 16-byte quant slices per lane
+    slices = 1                                           # 16-byte quant slices per lane
     team_warps = -(-nsb * 8 // slices // 32)
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
-    assert p["block"] <= 480 + 32
+    assert p["block"] <= (640 if m == 1 else 480) + 32
     assert 2 <= depth <= 8 and 1 <= teams <= 15
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     coef_per_warp = SEG * (4 * slices) * 4 * 16    # [seg][positions][4 groups] float4s
@@ -111,7 +111,7 @@ SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
           + [(4096, 14336), (1024, 4096), (14336, 4096)]
           + [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280), (33, 2304), (37, 8960),
              (129, 256), (1, 14336), (3, 11008), (97, 4352), (300, 3840), (149, 1024),
-             (147, 20480), (1000, 20480), (77, 1536), (40, 4096), (200, 1792), (3, 30720),
+             (147, 20480), (1000, 20480), (77, 1536), (40, 4096), (200, 1792), (3, 20480),
              (150, 15360)])
 
 
@@ -132,7 +132,7 @@ def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(2, 4096, 14336, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     # outside the streaming kernel's range: the general kernel
     assert q4k.q4k_gemv_plan_for(3, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
-    assert q4k.q4k_gemv_plan_for(1, 64, 30720, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
-    assert q4k.q4k_gemv_plan_for(1, 64, 30976, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    assert q4k.q4k_gemv_plan_for(1, 64, 20480, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
+    assert q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
     assert q4k.q4k_gemv_plan_for(2, 64, 15360, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_plan_for(2, 64, 15616, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
