@@ -42,7 +42,8 @@ class Q4KError(RuntimeError):
 
 class q4k_gemv_plan(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_int), ("grid", ctypes.c_int), ("block", ctypes.c_int),
-                ("smem_bytes", ctypes.c_int), ("teams", ctypes.c_int), ("depth", ctypes.c_int),
+                ("smem_bytes", ctypes.c_int), ("cluster", ctypes.c_int), ("teams", ctypes.c_int),
+                ("depth", ctypes.c_int),
                 ("launches", ctypes.c_int), ("units", ctypes.c_longlong),
                 ("units_per_cta_max", ctypes.c_longlong)]
 

@@ -67,6 +67,10 @@ int current_device_info(DeviceInfo* info) {
                                                 : static_cast<int>(e2);
         if (g_dev_status[dev] == 0 && stream_set_attributes() != Q4K_OK)
             g_dev_status[dev] = q4k_last_cuda_error_value();
+        if (g_dev_status[dev] == 0) {
+            stream_cluster_occupancy(1, g_dev[dev].max_clusters[0]);
+            stream_cluster_occupancy(2, g_dev[dev].max_clusters[1]);
+        }
     });
     if (g_dev_status[dev] != 0) return cuda_failure(static_cast<cudaError_t>(g_dev_status[dev]));
     *info = g_dev[dev];

@@ -91,11 +91,11 @@ void launch_rows(const q4k_gemv_plan& plan, const void* w, const float* x, float
 
 }  // namespace
 
-int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, q4k_gemv_plan* plan,
-                     StreamParams* sp) {
+int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
+                     q4k_gemv_plan* plan, StreamParams* sp) {
     StreamParams q{};
     int grid = 0, block = 0, smem = 0;
-    if (plan_stream(m, n, k, num_sms, max_smem, &q, &grid, &block, &smem)) {
+    if (plan_stream(m, n, k, num_sms, max_smem, max_clusters, &q, &grid, &block, &smem)) {
         plan->kernel = Q4K_KERNEL_STREAM;
         plan->grid = grid;
         plan->block = block;
@@ -103,6 +103,7 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, q4k_gemv_pl
         plan->teams = q.teams;
         plan->depth = q.depth;
         plan->launches = 1;
+        plan->cluster = q.cluster;
         plan->units = n;
         plan->units_per_cta_max = q.rows_base + (q.rows_extra > 0 ? 1 : 0);
         if (sp) *sp = q;
@@ -114,6 +115,7 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, q4k_gemv_pl
     if (ctas > cap) ctas = cap;
     const long long warps = ctas * warps_per_cta;
     plan->kernel = Q4K_KERNEL_WARP_ROWS;
+    plan->cluster = 1;
     plan->grid = static_cast<int>(ctas);
     plan->block = kRowsThreads;
     plan->smem_bytes = 0;
@@ -126,14 +128,15 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, q4k_gemv_pl
 }
 
 int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
-    return plan_gemv_device(m, n, k, num_sms, kB200SmemOptin, plan, nullptr);
+    return plan_gemv_device(m, n, k, num_sms, kB200SmemOptin, nullptr, plan, nullptr);
 }
 
 int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n,
                 int k, cudaStream_t stream) {
     q4k_gemv_plan plan;
     StreamParams sp;
-    int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin, &plan, &sp);
+    const int* clusters = (m >= 1 && m <= 2) ? dev.max_clusters[m - 1] : nullptr;
+    int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin, clusters, &plan, &sp);
     if (st != Q4K_OK) return st;
     if (plan.kernel == Q4K_KERNEL_STREAM)
         return launch_stream(sp, plan.grid, plan.block, plan.smem_bytes, w, x, y, m, stream);

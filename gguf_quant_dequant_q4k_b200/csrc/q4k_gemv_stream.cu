@@ -86,22 +86,26 @@ struct TeamRange {
     int nstages;
 };
 
-// Team `team`'s superblock range in the calling CTA. Team boundaries are
-// computed CTA-relative in 32 bits (a CTA's rows*nsb is far below 2^31 for any
-// matrix whose N*K/256 fits the int arguments); only the CTA origin is 64-bit.
-__device__ __forceinline__ TeamRange team_range(const StreamParams& p, int team) {
-    const int cta = static_cast<int>(blockIdx.x);
-    const int rows = p.rows_base + (cta < p.rows_extra ? 1 : 0);
+// Superblock range of cluster-global team `gteam` (= cta_rank * teams + team)
+// of the calling CTA's cluster. The cluster owns a contiguous range of whole
+// rows; its C * teams teams cut it into equal contiguous pieces. Boundaries are
+// computed cluster-relative in 32 bits (a cluster's rows*nsb is far below
+// 2^31 for any matrix whose N*K/256 fits the int arguments); only the cluster
+// origin is 64-bit.
+__device__ __forceinline__ TeamRange team_range(const StreamParams& p, int gteam) {
+    const int q = static_cast<int>(blockIdx.x) / p.cluster;
+    const int rows = p.rows_base + (q < p.rows_extra ? 1 : 0);
     const long long row_begin =
-        static_cast<long long>(cta) * p.rows_base + (cta < p.rows_extra ? cta : p.rows_extra);
+        static_cast<long long>(q) * p.rows_base + (q < p.rows_extra ? q : p.rows_extra);
     const int L = rows * p.nsb;
-    const int b = static_cast<int>((static_cast<unsigned long long>(L) * team) / p.teams);
-    const int e = static_cast<int>((static_cast<unsigned long long>(L) * (team + 1)) / p.teams);
+    const unsigned nt = static_cast<unsigned>(p.cluster * p.teams);
+    const int b = static_cast<int>((static_cast<unsigned long long>(L) * gteam) / nt);
+    const int e = static_cast<int>((static_cast<unsigned long long>(L) * (gteam + 1)) / nt);
     TeamRange r;
     r.s0 = row_begin * p.nsb + b;
     r.s1 = row_begin * p.nsb + e;
     if (e > b) {
-        const int rb = b / p.nsb;                 // CTA-relative first row
+        const int rb = b / p.nsb;                 // cluster-relative first row
         r.row0 = row_begin + rb;
         r.nseg = (e - 1) / p.nsb - rb + 1;
         r.nstages = (r.nseg + kSeg - 1) / kSeg;
@@ -221,6 +225,27 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ int cta_rank(const StreamParams& p) {
+    return static_cast<int>(blockIdx.x) % p.cluster;
+}
+
+// Cluster-wide barrier with release/acquire semantics for shared memory.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// A float at the same shared-memory address in CTA `rank` of the cluster.
+__device__ __forceinline__ float ld_dsmem(const float* local, int rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                 : "=r"(remote)
+                 : "r"(smem_addr(local)), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
+
 // Per-team view of the kernel's shared memory and work range.
 struct Team {
     TeamRange tr;
@@ -236,7 +261,7 @@ struct Team {
 template <int M>
 __device__ __forceinline__ Team make_team(const StreamParams& p, uint8_t* smem, int team) {
     Team t;
-    t.tr = team_range(p, team);
+    t.tr = team_range(p, cta_rank(p) * p.teams + team);
     t.head0 = static_cast<int>(t.tr.s0 - t.tr.row0 * p.nsb);
     t.team_len = static_cast<int>(t.tr.s1 - t.tr.s0);
     t.w = p.w + t.tr.s0 * kBlockBytes;
@@ -274,17 +299,17 @@ q4k_gemv_stream_kernel(const StreamParams p) {
     const int compute_warps = p.teams * p.team_warps;
     float* part = reinterpret_cast<float*>(smem + p.off_part);   // [teams][2][M]
 
-    if (threadIdx.x == 0) {
-        abort_flag = 0;
-        uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
-        for (int t = 0; t < p.teams; ++t) {
-            for (int s = 0; s < p.depth; ++s) {
-                mbar_init(&bars[(2 * t) * p.depth + s], 1);
-                mbar_init(&bars[(2 * t + 1) * p.depth + s], p.team_warps);
-            }
+    if (threadIdx.x == 0) abort_flag = 0;
+    {
+        // barriers [team][full, done][depth]: one per thread
+        const int nbar = 2 * p.teams * p.depth;
+        const int i = static_cast<int>(threadIdx.x);
+        if (i < nbar) {
+            uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+            mbar_init(&bars[i], ((i / p.depth) & 1) ? p.team_warps : 1);
+            fence_mbar_init();
         }
-        fence_mbar_init();
-        for (int i = 0; i < p.teams * 2 * M; ++i) part[i] = 0.f;
+        if (i < p.teams * 2 * M) part[i] = 0.f;
     }
     __syncthreads();
 
@@ -513,12 +538,22 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             }
         }
     }
-    __syncthreads();
+    // All teams' cut-row partials must be in shared memory before any team of
+    // the cluster reads them.
+    if (p.cluster > 1)
+        cluster_sync();
+    else
+        __syncthreads();
 
-    // Rows cut between teams: the team holding a row's first superblock adds the
-    // partial sums of the following teams that touch the row, in team order.
+    // Rows cut between teams (of this CTA or of other CTAs of the cluster): the
+    // team holding a row's first superblock adds the partial sums of the
+    // following teams that touch the row, in team order; a partial held by
+    // another CTA of the cluster is read through distributed shared memory.
     if (warp == compute_warps && lane < p.teams) {
-        const TeamRange tr = team_range(p, lane);
+        const int rank = cta_rank(p);
+        const int gteam = rank * p.teams + lane;
+        const int nteams = p.cluster * p.teams;
+        const TeamRange tr = team_range(p, gteam);
         if (tr.nseg > 0) {
             const long long last = tr.row0 + tr.nseg - 1;
             const long long lb = seg_begin(tr, tr.nseg - 1, nsb) - last * nsb;
@@ -527,24 +562,40 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 float tot[M];
 #pragma unroll
                 for (int i = 0; i < M; ++i) tot[i] = part[(lane * 2 + 1) * M + i];
-                for (int t2 = lane + 1; t2 < p.teams; ++t2) {
-                    const TeamRange o = team_range(p, t2);
+                for (int g2 = gteam + 1; g2 < nteams; ++g2) {
+                    const TeamRange o = team_range(p, g2);
                     if (o.s0 >= (last + 1) * nsb) break;
                     if (o.s1 <= o.s0) continue;   // a team with an empty range
+                    const int r2 = g2 / p.teams, t2 = g2 % p.teams;
 #pragma unroll
-                    for (int i = 0; i < M; ++i) tot[i] += part[(t2 * 2 + 0) * M + i];
+                    for (int i = 0; i < M; ++i) {
+                        const float* src = part + (t2 * 2 + 0) * M + i;
+                        tot[i] += (r2 == rank) ? *src : ld_dsmem(src, r2);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < M; ++i) p.y[static_cast<size_t>(i) * p.n + last] = tot[i];
             }
         }
     }
+    // Keep this CTA's shared memory alive until the cluster has read it.
+    if (p.cluster > 1) cluster_sync();
 }
 
 }  // namespace
 
-int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp, int* grid,
-                int* block, int* smem_bytes) {
+namespace {
+
+// Clusters of c CTAs that can be resident at once.
+int resident_clusters(int c, int num_sms, const int* max_clusters) {
+    if (max_clusters != nullptr && max_clusters[c] > 0) return max_clusters[c];
+    return num_sms / c;
+}
+
+}  // namespace
+
+int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
+                StreamParams* sp, int* grid, int* block, int* smem_bytes) {
     const int nsb = k / kQK;
     if (m < 1 || m > kStreamMaxM || nsb > kStreamMaxNsb || n < 1) return 0;
     const int sl = stream_slices(m);                     // quant slices per lane
@@ -553,7 +604,27 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
     if (team_warps > max_warps) return 0;
     int teams = max_warps / team_warps;
     if (teams > kStreamMaxTeams) teams = kStreamMaxTeams;
-    const int ctas = n < num_sms ? n : num_sms;
+    // Cluster size: the smallest C (1, 2, 4, 8) whose most loaded CTA streams
+    // clearly (> 5%) fewer superblocks than with the next smaller size. A
+    // cluster owns whole rows; C > 1 splits rows across CTAs (split-K), which
+    // pays off when N is small against the number of SMs.
+    int cluster = 1, clusters = n < resident_clusters(1, num_sms, max_clusters)
+                                    ? n : resident_clusters(1, num_sms, max_clusters);
+    // superblocks of the most loaded CTA (a superblock is never split)
+    double best = static_cast<double>((n + clusters - 1) / clusters) * nsb;
+    for (int c = 2; c <= kStreamMaxCluster; c *= 2) {
+        int q = resident_clusters(c, num_sms, max_clusters);
+        if (q < 1) continue;
+        if (q > n) q = n;
+        const long long rows = (n + q - 1) / q;
+        const double work = static_cast<double>((rows * nsb + c - 1) / c);
+        if (work < 0.95 * best) {
+            best = work;
+            cluster = c;
+            clusters = q;
+        }
+    }
+    const int ctas = clusters * cluster;
     const int stage_bytes = ((kSeg * nsb * kBlockBytes) + 127) / 128 * 128;
     const int budget = (max_smem < kStreamSmemBudget ? max_smem : kStreamSmemBudget) - 1024;
     // bytes per team besides its ring: coefficient buffers of its warps, the
@@ -578,8 +649,9 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp
     q.n = n;
     q.k = k;
     q.nsb = nsb;
-    q.rows_base = n / ctas;
-    q.rows_extra = n % ctas;
+    q.cluster = cluster;
+    q.rows_base = n / clusters;
+    q.rows_extra = n % clusters;
     q.teams = teams;
     q.team_warps = team_warps;
     q.depth = depth;
@@ -612,11 +684,15 @@ int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, 
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(sp.cluster);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = sp.cluster > 1 ? 2 : 1;
     cudaError_t e;
     if (m == 1) {
         e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, stream_slices(1)>, sp);
@@ -639,6 +715,33 @@ int stream_set_attributes() {
 }  // namespace q4k
 
 namespace q4k {
+
+int stream_cluster_occupancy(int m, int* max_clusters) {
+    for (int c = 0; c <= kStreamMaxCluster; ++c) max_clusters[c] = 0;
+    for (int c = 1; c <= kStreamMaxCluster; c *= 2) {
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(c);
+        cfg.blockDim = dim3(stream_max_threads(m) + 32);
+        cfg.dynamicSmemBytes = kStreamSmemBudget;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(c);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int count = 0;
+        const cudaError_t e = (m == 1)
+            ? cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<1, stream_slices(1)>, &cfg)
+            : cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<2, stream_slices(2)>, &cfg);
+        if (e != cudaSuccess) {
+            cudaGetLastError();   // the query is advisory; clear the error
+            count = 0;
+        }
+        max_clusters[c] = count;
+    }
+    return Q4K_OK;
+}
 
 int read_fault_flags(unsigned* flags) {
     unsigned v = 0;

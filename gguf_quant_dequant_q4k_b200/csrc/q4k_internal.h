@@ -11,7 +11,8 @@ namespace q4k {
 // Per-device facts the launch planner needs, read once per device.
 struct DeviceInfo {
     int sm_count;
-    int max_smem_optin;  // largest dynamic shared memory a CTA may opt in to
+    int max_smem_optin;        // largest dynamic shared memory a CTA may opt in to
+    int max_clusters[2][9];    // resident clusters of c CTAs, streaming kernel, m = 1 / 2
 };
 
 // Returns Q4K_OK and fills *info for the current device, or Q4K_ERR_CUDA.

@@ -30,16 +30,25 @@ struct StreamParams {
     const float* x;
     float* y;
     int n, k, nsb;
-    int rows_base, rows_extra;  // CTA c owns rows_base (+1 if c < rows_extra) rows
+    int cluster;                // CTAs per thread-block cluster (1 = no cluster)
+    int rows_base, rows_extra;  // cluster q owns rows_base (+1 if q < rows_extra) rows
     int teams, team_warps, depth;
     int stage_bytes;            // bytes per ring slot
     int off_coef, off_red, off_part, off_bar;  // shared-memory offsets (bytes)
 };
 
+constexpr int kStreamMaxCluster = 8;    // portable cluster size limit
+
 // Fills the launch configuration; returns 0 if the streaming kernel does not
 // handle (m, k) or the shared-memory budget cannot hold two stages.
-int plan_stream(int m, int n, int k, int num_sms, int max_smem, StreamParams* sp, int* grid,
-                int* block, int* smem_bytes);
+// max_clusters[c] (c = 1..8, may be null) is how many clusters of c CTAs can
+// be resident at once; without it the planner assumes num_sms / c.
+int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
+                StreamParams* sp, int* grid, int* block, int* smem_bytes);
+
+// Resident clusters of c CTAs (c = 1..8) for the streaming kernel on the
+// current device, into max_clusters[c]; 0 where the query is not possible.
+int stream_cluster_occupancy(int m, int* max_clusters);
 
 int launch_stream(const StreamParams& sp, int grid, int block, int smem_bytes, const void* w,
                   const float* x, float* y, int m, cudaStream_t stream);

@@ -139,17 +139,22 @@ typedef struct q4k_gemv_plan {
     int grid;            /* CTAs                                                */
     int block;           /* threads per CTA                                     */
     int smem_bytes;      /* dynamic shared memory per CTA                       */
+    int cluster;         /* CTAs per thread-block cluster; > 1 splits rows (split-K) */
     int teams;           /* warp teams per CTA (streaming kernel; else 0)       */
     int depth;           /* bulk-copy ring stages per team (streaming; else 0)  */
     int launches;        /* kernels one call enqueues                           */
     long long units;     /* output rows shared out among the CTAs               */
-    long long units_per_cta_max; /* most rows any CTA owns                      */
+    long long units_per_cta_max; /* most rows any cluster (CTA if cluster = 1) owns */
 } q4k_gemv_plan;
 
 enum q4k_kernel {
     Q4K_KERNEL_WARP_ROWS = 1,   /* any K, m <= 8: one warp per row, loads via L1  */
-    Q4K_KERNEL_STREAM = 2       /* m <= 2, K <= 20480: bulk-copy streamed rows,
-                                   x held in registers, balanced per-SM ranges    */
+    Q4K_KERNEL_STREAM = 2       /* m <= 2, K <= 20480 (m = 1) / 15360 (m = 2):
+                                   bulk-copy streamed rows, x held in registers,
+                                   balanced per-SM ranges; small N splits rows
+                                   across the CTAs of a cluster (split-K) and
+                                   finishes them through distributed shared
+                                   memory                                         */
 };
 
 Q4K_API int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan *plan);

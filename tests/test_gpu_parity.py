@@ -252,6 +252,19 @@ def test_gemv_two_vectors_team_split(q4k, n, k):
     assert_gemv_close(y, yref, a, f"{n}x{k} m=2")
 
 
+@pytest.mark.parametrize("m", [1, 2])
+@pytest.mark.parametrize("n,k", [(1, 14336), (1, 4096), (2, 1536), (8, 14336), (16, 8960),
+                                 (40, 4096), (63, 11008), (100, 2048)])
+def test_gemv_small_n_cluster_split(q4k, n, k, m):
+    """Small N: rows are split across the CTAs of a thread-block cluster (split-K)
+    and finished through distributed shared memory."""
+    plan = q4k.q4k_gemv_plan_for(m, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
+    w, x = q4k_synth.q4k_problem(n, k, m, 50 + n + m)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(y, yref, a, f"{n}x{k} m={m} cluster={plan['cluster']}")
+
+
 def test_no_kernel_fault_flags(q4k):
     """No bounded wait on a bulk copy gave up during any of the runs above."""
     assert q4k.q4k_device_fault_flags() == 0

@@ -20,13 +20,15 @@ SM_COUNT = 148
 SMEM_OPTIN = 232448
 
 
-def team_range(cta, team, n, nsb, ctas, teams):
-    base, extra = n // ctas, n % ctas
-    rows = base + (1 if cta < extra else 0)
-    row_begin = cta * base + min(cta, extra)
+def team_range(cluster_id, gteam, n, nsb, clusters, cluster, teams):
+    """Superblock range of cluster-global team gteam (= cta_rank*teams + team)."""
+    base, extra = n // clusters, n % clusters
+    rows = base + (1 if cluster_id < extra else 0)
+    row_begin = cluster_id * base + min(cluster_id, extra)
     S0, L = row_begin * nsb, rows * nsb
-    s0 = S0 + (L * team) // teams
-    s1 = S0 + (L * (team + 1)) // teams
+    nt = cluster * teams
+    s0 = S0 + (L * gteam) // nt
+    s1 = S0 + (L * (gteam + 1)) // nt
     if s1 > s0:
         row0 = s0 // nsb
         nseg = (s1 - 1) // nsb - row0 + 1
@@ -44,7 +46,10 @@ def check_plan(m, n, k):
     if p["kernel"] != q4k.Q4K_KERNEL_STREAM:
         return p
     nsb = k // 256
-    ctas, teams, depth = p["grid"], p["teams"], p["depth"]
+    ctas, teams, depth, cluster = p["grid"], p["teams"], p["depth"], p["cluster"]
+    assert cluster in (1, 2, 4, 8) and ctas % cluster == 0
+    clusters = ctas // cluster
+    assert clusters <= n
     slices = 1                                           # 16-byte quant slices per lane
     team_warps = -(-nsb * 8 // slices // 32)
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
@@ -58,8 +63,10 @@ def check_plan(m, n, k):
     assert p["smem_bytes"] == need and need <= 220 * 1024 - 1024
     covered = [0] * (n * nsb)
     writes = [0] * n
-    for cta in range(ctas):
-        ranges = [team_range(cta, t, n, nsb, ctas, teams) for t in range(teams)]
+    for q in range(clusters):
+        # every team of the cluster, in cluster-global order (rank-major)
+        ranges = [team_range(q, g, n, nsb, clusters, cluster, teams)
+                  for g in range(cluster * teams)]
         for t, (s0, s1, row0, nseg) in enumerate(ranges):
             for sb in range(s0, s1):
                 covered[sb] += 1
@@ -92,7 +99,7 @@ def check_plan(m, n, k):
                 lb, le = lb - last * nsb, le - last * nsb
                 if lb == 0 and le < nsb:
                     got = le
-                    for t2 in range(t + 1, teams):
+                    for t2 in range(t + 1, cluster * teams):
                         o0, o1, _, _ = ranges[t2]
                         if o0 >= (last + 1) * nsb:
                             break
@@ -112,7 +119,7 @@ SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
           + [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280), (33, 2304), (37, 8960),
              (129, 256), (1, 14336), (3, 11008), (97, 4352), (300, 3840), (149, 1024),
              (147, 20480), (1000, 20480), (77, 1536), (40, 4096), (200, 1792), (3, 20480),
-             (150, 15360)])
+             (150, 15360), (1, 4096), (8, 14336), (16, 8960), (63, 11008), (2, 1536)])
 
 
 @pytest.mark.parametrize("n,k", SHAPES)
@@ -125,6 +132,15 @@ def test_lm_head_partition():
     p = check_plan(1, 128256, 4096)
     assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["grid"] == SM_COUNT
     assert p["units_per_cta_max"] == -(-128256 // SM_COUNT)
+
+
+@pytest.mark.parametrize("n,k,cluster", [(1, 14336, 8), (1, 256, 1), (40, 4096, 8),
+                                         (16, 8960, 8), (1536, 8960, 1), (4096, 4096, 1),
+                                         (128256, 4096, 1)])
+def test_cluster_choice(n, k, cluster):
+    """Small N splits rows across the CTAs of a cluster (split-K); large N does not."""
+    p = check_plan(1, n, k)
+    assert p["cluster"] == cluster, p
 
 
 def test_kernel_choice():
