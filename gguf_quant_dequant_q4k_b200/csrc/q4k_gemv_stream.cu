@@ -604,25 +604,19 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     if (team_warps > max_warps) return 0;
     int teams = max_warps / team_warps;
     if (teams > kStreamMaxTeams) teams = kStreamMaxTeams;
-    // Cluster size: the smallest C (1, 2, 4, 8) whose most loaded CTA streams
-    // clearly (> 5%) fewer superblocks than with the next smaller size. A
-    // cluster owns whole rows; C > 1 splits rows across CTAs (split-K), which
-    // pays off when N is small against the number of SMs.
-    int cluster = 1, clusters = n < resident_clusters(1, num_sms, max_clusters)
-                                    ? n : resident_clusters(1, num_sms, max_clusters);
-    // superblocks of the most loaded CTA (a superblock is never split)
-    double best = static_cast<double>((n + clusters - 1) / clusters) * nsb;
-    for (int c = 2; c <= kStreamMaxCluster; c *= 2) {
-        int q = resident_clusters(c, num_sms, max_clusters);
-        if (q < 1) continue;
-        if (q > n) q = n;
-        const long long rows = (n + q - 1) / q;
-        const double work = static_cast<double>((rows * nsb + c - 1) / c);
-        if (work < 0.95 * best) {
-            best = work;
-            cluster = c;
-            clusters = q;
-        }
+    // Cluster size. Within a CTA the warps of a team already split K, so a
+    // row of any supported K is processed by up to 20 warps at once; splitting
+    // rows across the CTAs of a cluster (split-K) adds a cluster launch and two
+    // cluster barriers (measured 2-6 us on B200 for clusters of 4-8) and paid
+    // off only for a handful of very long rows (N = 1, K = 14336: 7.2 -> 6.7
+    // us with clusters of 2). So: clusters of two CTAs for N < 8 and K >= 8192.
+    int cluster = 1;
+    int clusters = n < resident_clusters(1, num_sms, max_clusters)
+                       ? n : resident_clusters(1, num_sms, max_clusters);
+    if (n < kClusterMaxRows && nsb >= kClusterMinNsb &&
+        resident_clusters(2, num_sms, max_clusters) >= n) {
+        cluster = 2;
+        clusters = n;
     }
     const int ctas = clusters * cluster;
     const int stage_bytes = ((kSeg * nsb * kBlockBytes) + 127) / 128 * 128;

@@ -37,7 +37,9 @@ struct StreamParams {
     int off_coef, off_red, off_part, off_bar;  // shared-memory offsets (bytes)
 };
 
-constexpr int kStreamMaxCluster = 8;    // portable cluster size limit
+constexpr int kStreamMaxCluster = 8;    // cluster sizes the kernel supports (portable limit)
+constexpr int kClusterMaxRows = 8;      // split rows across a cluster only for N < 8 ...
+constexpr int kClusterMinNsb = 32;      // ... and K >= 8192
 
 // Fills the launch configuration; returns 0 if the streaming kernel does not
 // handle (m, k) or the shared-memory budget cannot hold two stages.

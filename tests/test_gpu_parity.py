@@ -253,11 +253,12 @@ def test_gemv_two_vectors_team_split(q4k, n, k):
 
 
 @pytest.mark.parametrize("m", [1, 2])
-@pytest.mark.parametrize("n,k", [(1, 14336), (1, 4096), (2, 1536), (8, 14336), (16, 8960),
-                                 (40, 4096), (63, 11008), (100, 2048)])
+@pytest.mark.parametrize("n,k", [(1, 14336), (3, 8960), (7, 11008), (5, 8192), (1, 4096),
+                                 (2, 1536), (8, 14336), (16, 8960), (40, 4096), (100, 2048)])
 def test_gemv_small_n_cluster_split(q4k, n, k, m):
-    """Small N: rows are split across the CTAs of a thread-block cluster (split-K)
-    and finished through distributed shared memory."""
+    """Small N: for N < 8 and K >= 8192 rows are split across the two CTAs of a
+    thread-block cluster (split-K) and finished through distributed shared
+    memory; the other shapes run one CTA per row."""
     plan = q4k.q4k_gemv_plan_for(m, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
     w, x = q4k_synth.q4k_problem(n, k, m, 50 + n + m)
     y = gpu_gemv(q4k, w, x, n, k)

@@ -47,7 +47,7 @@ def check_plan(m, n, k):
         return p
     nsb = k // 256
     ctas, teams, depth, cluster = p["grid"], p["teams"], p["depth"], p["cluster"]
-    assert cluster in (1, 2, 4, 8) and ctas % cluster == 0
+    assert cluster in (1, 2) and ctas % cluster == 0
     clusters = ctas // cluster
     assert clusters <= n
     slices = 1                                           # 16-byte quant slices per lane
@@ -134,11 +134,11 @@ def test_lm_head_partition():
     assert p["units_per_cta_max"] == -(-128256 // SM_COUNT)
 
 
-@pytest.mark.parametrize("n,k,cluster", [(1, 14336, 8), (1, 256, 1), (40, 4096, 8),
-                                         (16, 8960, 8), (1536, 8960, 1), (4096, 4096, 1),
-                                         (128256, 4096, 1)])
+@pytest.mark.parametrize("n,k,cluster", [(1, 14336, 2), (7, 8192, 2), (1, 256, 1), (40, 4096, 1),
+                                         (16, 8960, 1), (8, 14336, 1), (1, 7936, 1),
+                                         (1536, 8960, 1), (4096, 4096, 1), (128256, 4096, 1)])
 def test_cluster_choice(n, k, cluster):
-    """Small N splits rows across the CTAs of a cluster (split-K); large N does not."""
+    """N < 8 with K >= 8192 splits rows across the two CTAs of a cluster (split-K)."""
     p = check_plan(1, n, k)
     assert p["cluster"] == cluster, p
 
