@@ -206,6 +206,76 @@ def cpu_baseline() -> dict:
                       f"over {threads} threads, {dt:.2f} s"}
 
 
+# --------------------------------------------------------------------------- extra workloads
+
+def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
+    """The other decode workloads of the sweep's configuration list, on this GPU:
+    multi-vector shapes (m = 1, 2, 4, 8) and the 32-layer 8B-class decode sweep.
+    Each figure is bytes counted / device time (CUDA events)."""
+    out = {"multivector": [], "layer_sweep_32": None}
+    for n, k in q4k_synth.SHAPES_MULTIVEC:
+        w, _ = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEED_MULTIVEC[(n, k)])
+        wd = torch.from_numpy(w).to(dev)
+        ws = [wd] + [wd.clone() for _ in range(max(2, -(-2 * l2 // w.nbytes) + 1) - 1)]
+        for m in (1, 2, 4, 8):
+            x = torch.from_numpy(q4k_synth.x_vectors(k, m, 77 + m)).to(dev)
+            y = torch.empty((m, n), dtype=torch.float32, device=dev)
+            with torch.cuda.stream(stream):
+                for i in range(10):
+                    q4k.q4k_gemv(ws[i % len(ws)], x, y, m, n, k, stream=stream)
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            reps = 100
+            a0.record(stream)
+            for i in range(reps):
+                q4k.q4k_gemv(ws[i % len(ws)], x, y, m, n, k, stream=stream)
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            us = a0.elapsed_time(a1) * 1e3 / reps
+            b = bytes_counted(n, k, m)
+            out["multivector"].append({"n": n, "k": k, "m": m, "us_per_call": round(us, 3),
+                                       "gbs": round(b / us / 1e3, 1)})
+        del ws, wd
+    # 32 layers x (q, k, v, o, gate, up, down), each layer's weights seeded
+    # independently; one pass = 224 launches captured in one CUDA graph.
+    layers = []
+    total = 0
+    for layer in range(32):
+        for proj, (n, k) in enumerate(q4k_synth.LAYER_8B):
+            w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.layer_seed(layer, proj))
+            layers.append((torch.from_numpy(w).to(dev), torch.from_numpy(x).to(dev),
+                           torch.empty((1, n), dtype=torch.float32, device=dev), n, k))
+            total += bytes_counted(n, k)
+    def one_pass():
+        for w, x, y, n, k in layers:
+            q4k.q4k_gemv(w, x, y, 1, n, k, stream=stream)
+    with torch.cuda.stream(stream):
+        one_pass()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_pass()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    reps = 20
+    a0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g.replay()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = a0.elapsed_time(a1) * 1e3 / reps
+    out["layer_sweep_32"] = {"launches": len(layers), "bytes": total, "us_per_pass": round(us, 1),
+                             "gbs": round(total / us / 1e3, 1),
+                             "how": "one CUDA graph of the 224 projection GEMVs, replayed"}
+    del g, layers
+    torch.cuda.empty_cache()
+    return out
+
+
 # --------------------------------------------------------------------------- our arm
 
 def run_ours(args) -> None:
@@ -403,6 +473,8 @@ def run_ours(args) -> None:
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_extras and not args.skip_extras:
+        line["extra"] = extra_workloads(q4k, torch, dev, stream, l2)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
@@ -416,6 +488,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-graph", action="store_true", help="eager launches (for profilers)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the multi-vector and 32-layer sweep measurements")
     ap.add_argument("--shapes", default=None,
                     help="comma-separated NxK subset of the sweep (profiling runs only)")
     ap.add_argument("--skip-extras", action="store_true",
