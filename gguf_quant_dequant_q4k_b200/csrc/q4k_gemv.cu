@@ -95,14 +95,18 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
                      q4k_gemv_plan* plan, StreamParams* sp) {
     StreamParams q{};
     int grid = 0, block = 0, smem = 0;
-    if (plan_stream(m, n, k, num_sms, max_smem, max_clusters, &q, &grid, &block, &smem)) {
+    // m > 2: ceil(m/2) launches of the two-vector streaming kernel on vector
+    // pairs (each decoded weight reused for two vectors per pass).
+    const int m_launch = m <= kStreamMaxM ? m : kStreamMaxM;
+    const int* cl = max_clusters;
+    if (plan_stream(m_launch, n, k, num_sms, max_smem, cl, &q, &grid, &block, &smem)) {
         plan->kernel = Q4K_KERNEL_STREAM;
         plan->grid = grid;
         plan->block = block;
         plan->smem_bytes = smem;
         plan->teams = q.teams;
         plan->depth = q.depth;
-        plan->launches = 1;
+        plan->launches = (m + m_launch - 1) / m_launch;
         plan->cluster = q.cluster;
         plan->units = n;
         plan->units_per_cta_max = q.rows_base + (q.rows_extra > 0 ? 1 : 0);
@@ -135,11 +139,29 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, 
                 int k, cudaStream_t stream) {
     q4k_gemv_plan plan;
     StreamParams sp;
-    const int* clusters = (m >= 1 && m <= 2) ? dev.max_clusters[m - 1] : nullptr;
+    const int m_launch = m <= kStreamMaxM ? m : kStreamMaxM;
+    const int* clusters = dev.max_clusters[m_launch - 1];
     int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin, clusters, &plan, &sp);
     if (st != Q4K_OK) return st;
-    if (plan.kernel == Q4K_KERNEL_STREAM)
-        return launch_stream(sp, plan.grid, plan.block, plan.smem_bytes, w, x, y, m, stream);
+    if (plan.kernel == Q4K_KERNEL_STREAM) {
+        for (int i0 = 0; i0 < m; i0 += m_launch) {
+            const int mi = (m - i0) < m_launch ? (m - i0) : m_launch;
+            StreamParams spi = sp;
+            if (mi != m_launch) {   // the odd last vector runs the one-vector kernel
+                int g = 0, b = 0, sm = 0;
+                plan_stream(mi, n, k, dev.sm_count, dev.max_smem_optin, dev.max_clusters[mi - 1],
+                            &spi, &g, &b, &sm);
+                st = launch_stream(spi, g, b, sm, w, x + static_cast<size_t>(i0) * k,
+                                   y + static_cast<size_t>(i0) * n, mi, stream);
+            } else {
+                st = launch_stream(spi, plan.grid, plan.block, plan.smem_bytes, w,
+                                   x + static_cast<size_t>(i0) * k, y + static_cast<size_t>(i0) * n,
+                                   mi, stream);
+            }
+            if (st != Q4K_OK) return st;
+        }
+        return Q4K_OK;
+    }
     switch (m) {
         case 1: launch_rows<1>(plan, w, x, y, n, k, stream); break;
         case 2: launch_rows<2>(plan, w, x, y, n, k, stream); break;

@@ -149,7 +149,8 @@ typedef struct q4k_gemv_plan {
 
 enum q4k_kernel {
     Q4K_KERNEL_WARP_ROWS = 1,   /* any K, m <= 8: one warp per row, loads via L1  */
-    Q4K_KERNEL_STREAM = 2       /* m <= 2, K <= 20480 (m = 1) / 15360 (m = 2):
+    Q4K_KERNEL_STREAM = 2       /* K <= 20480 (m = 1) / 15360 (m >= 2); m > 2 runs
+                                   as ceil(m/2) launches on vector pairs;
                                    bulk-copy streamed rows, x held in registers,
                                    balanced per-SM ranges; small N splits rows
                                    across the CTAs of a cluster (split-K) and

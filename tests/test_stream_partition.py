@@ -147,7 +147,10 @@ def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(1, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_plan_for(2, 4096, 14336, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     # outside the streaming kernel's range: the general kernel
-    assert q4k.q4k_gemv_plan_for(3, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    p3 = q4k.q4k_gemv_plan_for(3, 4096, 4096, SM_COUNT)
+    assert p3["kernel"] == q4k.Q4K_KERNEL_STREAM and p3["launches"] == 2
+    assert q4k.q4k_gemv_plan_for(8, 4096, 14336, SM_COUNT)["launches"] == 4
+    assert q4k.q4k_gemv_plan_for(3, 64, 15616, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
     assert q4k.q4k_gemv_plan_for(1, 64, 20480, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
     assert q4k.q4k_gemv_plan_for(2, 64, 15360, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
