@@ -12,10 +12,11 @@ constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kern
 // slice per lane with more warps beats two slices with fewer warps on every
 // decode shape but the largest (within 2% there).
 constexpr int stream_slices(int m) { return m == 1 ? 1 : 1; }
-// Compute threads per CTA (plus one producer warp): 23 + 1 warps for one vector
-// (x: 32 registers per lane; six warps per sub-partition at 80 registers),
-// 15 + 1 for two (x: 64 registers per lane; four warps at 128 registers).
-constexpr int stream_max_threads(int m) { return m == 1 ? 736 : 480; }
+// Compute threads per CTA (plus one producer warp): 20 + 1 warps for one vector
+// (x: 32 registers per lane; up to six warps per sub-partition at 80
+// registers; 23 compute warps measured no faster), 15 + 1 for two (x: 64
+// registers per lane; four warps per sub-partition at 128 registers).
+constexpr int stream_max_threads(int m) { return m == 1 ? 640 : 480; }
 // Registers per thread: each of the SM's four sub-partitions has 16384
 // registers for its share of the CTA's warps (allocated in multiples of 8).
 constexpr int stream_max_regs(int m) {

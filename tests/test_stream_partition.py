@@ -53,7 +53,7 @@ def check_plan(m, n, k):
     slices = 1                                           # 16-byte quant slices per lane
     team_warps = -(-nsb * 8 // slices // 32)
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
-    assert p["block"] <= (736 if m == 1 else 480) + 32
+    assert p["block"] <= (640 if m == 1 else 480) + 32
     assert 2 <= depth <= 8 and 1 <= teams <= 15
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     coef_per_warp = SEG * (4 * slices) * 4 * 16    # [seg][positions][4 groups] float4s
