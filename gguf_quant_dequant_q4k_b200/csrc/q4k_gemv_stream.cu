@@ -1,4 +1,4 @@
-// q4k_gemv_stream.cu -- the streaming Q4_K GEMV for m = 1, 2 and K <= 32768.
+// q4k_gemv_stream.cu -- the streaming Q4_K GEMV for m = 1, 2 and K <= 20480 (m = 1) or 15360 (m = 2).
 //
 // What it computes: y[i][r] = sum_k W[r][k] x[i][k] with W in Q4_K, as the
 // pages' `Q4KGemv` / `TiledQ4KGemv` / `ChunkedTiledQ4KGemv` / `MwvQ4KGemv`
