@@ -26,10 +26,12 @@
 //   on a "full" mbarrier; no multicast). A stage is up to 4 consecutive row
 //   segments (one contiguous copy). Every weight byte is read from HBM once.
 //   One producer warp per CTA (lane t serves team t) issues the copies, polls
-//   each team's "done" mbarrier (one arrival per warp per stage), adds the
-//   warps' partials of a drained stage into y and refills its slot at once.
-//   The first `depth` copies are issued before griddepcontrol.wait, so under
-//   programmatic dependent launch they overlap the previous kernel's tail.
+//   each team's "done" mbarrier (one arrival per warp per stage), refills a
+//   drained slot at once and then adds the warps' partials into y. Each team's
+//   first stage is requested before griddepcontrol.wait, so under
+//   programmatic dependent launch it overlaps the previous kernel's tail; the
+//   rest of the ring follows once every compute warp has issued its x loads
+//   (x is the dependent input, so it must not queue behind the ring).
 // * Decode. Once per stage each warp decodes the headers of its superblocks
 //   (d, dmin, 12 scale bytes; GGUF get_scale_min_k4 packing) into (A_j, B_j)
 //   pairs with A_j = 256*d*sc_j (exact) and B_j = -(128*d*sc_j + dmin*m_j).
@@ -61,6 +63,7 @@ namespace {
 __device__ unsigned int g_fault_flags = 0;
 
 constexpr int kSeg = kStreamSegRows;         // row segments per stage
+constexpr unsigned kXIssuedBarrier = 1;      // named barrier: compute warps issued x loads
 constexpr uint32_t kMagicOne = 0x3F000000u;  // 1/2: bytes 0..2 = 0x00, byte 3 = 0x3F
 constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
 // Coefficient buffer per warp: [segment][position][4 groups] float4s.
@@ -85,6 +88,7 @@ struct TeamRange {
     int nseg;           // rows touched
     int nstages;
 };
+static_assert(sizeof(TeamRange) == kTeamRangeBytes, "team range table entry");
 
 // Superblock range of cluster-global team `gteam` (= cta_rank * teams + team)
 // of the calling CTA's cluster. The cluster owns a contiguous range of whole
@@ -99,8 +103,14 @@ __device__ __forceinline__ TeamRange team_range(const StreamParams& p, int gteam
         static_cast<long long>(q) * p.rows_base + (q < p.rows_extra ? q : p.rows_extra);
     const int L = rows * p.nsb;
     const unsigned nt = static_cast<unsigned>(p.cluster * p.teams);
-    const int b = static_cast<int>((static_cast<unsigned long long>(L) * gteam) / nt);
-    const int e = static_cast<int>((static_cast<unsigned long long>(L) * (gteam + 1)) / nt);
+    int b, e;
+    if (static_cast<unsigned>(L) <= 0xFFFFFFFFu / nt) {   // products fit 32 bits
+        b = static_cast<int>(static_cast<unsigned>(L) * gteam / nt);
+        e = static_cast<int>(static_cast<unsigned>(L) * (gteam + 1) / nt);
+    } else {
+        b = static_cast<int>((static_cast<unsigned long long>(L) * gteam) / nt);
+        e = static_cast<int>((static_cast<unsigned long long>(L) * (gteam + 1)) / nt);
+    }
     TeamRange r;
     r.s0 = row_begin * p.nsb + b;
     r.s1 = row_begin * p.nsb + e;
@@ -253,7 +263,7 @@ struct Team {
     int team_len;       // superblocks in the team's range
     const uint8_t* w;   // W at the team's first superblock
     uint8_t* ring;      // depth slots of stage_bytes
-    float* red;         // [depth][team_warps][M][kSeg] warp partials
+    float* red;         // [depth][2 phases][team_warps][M][kSeg] warp partials
     uint64_t* full;     // [depth] stage landed (1 arrival + bytes)
     uint64_t* done;     // [depth] stage consumed (team_warps arrivals)
 };
@@ -261,13 +271,13 @@ struct Team {
 template <int M>
 __device__ __forceinline__ Team make_team(const StreamParams& p, uint8_t* smem, int team) {
     Team t;
-    t.tr = team_range(p, cta_rank(p) * p.teams + team);
+    t.tr = reinterpret_cast<const TeamRange*>(smem + p.off_tr)[cta_rank(p) * p.teams + team];
     t.head0 = static_cast<int>(t.tr.s0 - t.tr.row0 * p.nsb);
     t.team_len = static_cast<int>(t.tr.s1 - t.tr.s0);
     t.w = p.w + t.tr.s0 * kBlockBytes;
     t.ring = smem + static_cast<size_t>(team) * p.depth * p.stage_bytes;
     t.red = reinterpret_cast<float*>(smem + p.off_red) +
-            static_cast<size_t>(team) * p.depth * p.team_warps * kSeg * M;
+            static_cast<size_t>(team) * p.depth * 2 * p.team_warps * kSeg * M;
     t.full = reinterpret_cast<uint64_t*>(smem + p.off_bar) + static_cast<size_t>(team) * 2 * p.depth;
     t.done = t.full + p.depth;
     return t;
@@ -310,6 +320,9 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             fence_mbar_init();
         }
         if (i < p.teams * 2 * M) part[i] = 0.f;
+        // superblock ranges of every team of the cluster (64-bit divisions once)
+        if (i < p.cluster * p.teams)
+            reinterpret_cast<TeamRange*>(smem + p.off_tr)[i] = team_range(p, i);
     }
     __syncthreads();
 
@@ -324,21 +337,34 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         if (own) {
             T = make_team<M>(p, smem, lane);
             nst = T.tr.nstages;
-            const int pre = nst < p.depth ? nst : p.depth;
+            const int all = nst < p.depth ? nst : p.depth;
+            const int pre = all < kStreamPreStages ? all : kStreamPreStages;
             for (int s = 0; s < pre; ++s) issue_stage(T, p, s * kSeg * nsb - T.head0, s);
         }
         pdl_launch_dependents();
         pdl_wait();
+        // x first: wait until every compute warp has issued its x loads.
+        named_barrier_sync(kXIssuedBarrier, blockDim.x);
+        if (own) {
+            const int all = nst < p.depth ? nst : p.depth;
+            const int pre = all < kStreamPreStages ? all : kStreamPreStages;
+            for (int s = pre; s < all; ++s) issue_stage(T, p, s * kSeg * nsb - T.head0, s);
+        }
         int tf = 0, fslot = 0;
         uint32_t fphase = 0;
         int rbf = own ? -T.head0 : 0;
         unsigned idle = 0;
+        const int red_slot = p.team_warps * kSeg * M;
         for (;;) {
             const bool active = own && tf < nst && !abort_flag;
             if (!__any_sync(0xFFFFFFFFu, active)) break;
             bool progressed = false;
             if (active && mbar_test_wait(&T.done[fslot], fphase)) {
-                const float* rbuf = T.red + static_cast<size_t>(fslot) * p.team_warps * kSeg * M;
+                // Refill the drained slot at once: its quant bytes are consumed,
+                // and its partial sums sit in the (slot, phase) half of the
+                // team's buffer, which the refilled stage does not write.
+                if (tf + p.depth < nst) issue_stage(T, p, rbf + p.depth * kSeg * nsb, fslot);
+                const float* rbuf = T.red + static_cast<size_t>(fslot * 2 + fphase) * red_slot;
 #pragma unroll
                 for (int u = 0; u < kSeg; ++u) {
                     if (tf * kSeg + u >= T.tr.nseg) break;
@@ -357,7 +383,6 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                             part[(lane * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
                     }
                 }
-                if (tf + p.depth < nst) issue_stage(T, p, rbf + p.depth * kSeg * nsb, fslot);
                 ++tf;
                 rbf += kSeg * nsb;
                 if (++fslot == p.depth) {
@@ -398,13 +423,11 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         // xp[i][e] = (x of the low nibble of byte e of the lane's quant bytes, x
         // of its high nibble): weights k0 + e and k0 + 32 + e.
         float2 xp[M][kNX];
-#pragma unroll
-        for (int i = 0; i < M; ++i) {
-#pragma unroll
-            for (int e = 0; e < kNX; ++e) xp[i][e] = make_float2(0.f, 0.f);
-        }
-        if (valid) {
-            const int k0 = bl * kQK + 64 * g + 16 * (c0 & 1);
+        {
+            // A lane past the last superblock position loads position 0's x
+            // (its products are discarded), so the loads need no branch and
+            // their latency overlaps the first stage's wait and decode.
+            const int k0 = (valid ? bl : 0) * kQK + 64 * g + 16 * (c0 & 1);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
                 const float4* xl =
@@ -420,6 +443,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 }
             }
         }
+        named_barrier_arrive(kXIssuedBarrier, blockDim.x);
 
         // Shared-memory byte offsets (32-bit). The coefficient float4 of
         // (segment u, position pos, group g) sits at (u*kPos + pos)*4 +
@@ -474,10 +498,11 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             }
             __syncwarp();
 
-            // The stage's (up to) kSeg row segments, branch-free: a lane whose
-            // superblock is not in a segment computes on superblock 0 and the
-            // result is discarded by a select. Item u + 1's operands are loaded
-            // while item u computes.
+            // The stage's (up to) kSeg row segments. Segments past the team's
+            // last row are skipped (a warp-uniform branch); inside a segment a
+            // lane whose superblock is not in it computes on superblock 0 and
+            // the result is discarded by a select. Item u + 1's operands are
+            // loaded while item u computes.
             bool use[kSeg];
             uint32_t qaddr[kSeg];
 #pragma unroll
@@ -487,18 +512,20 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 qaddr[u] = st_off + (use[u] ? lane_qoff + static_cast<uint32_t>((u * nsb - head) * kBlockBytes)
                                             : static_cast<uint32_t>(kQsOffset + 16 * c0));
             }
+            const int nseg_s = T.tr.nseg - s * kSeg < kSeg ? T.tr.nseg - s * kSeg : kSeg;
             float part_sum[M][kSeg];
             uint4 qn[S];
 #pragma unroll
             for (int j = 0; j < S; ++j) qn[j] = *reinterpret_cast<const uint4*>(smem + qaddr[0] + 16 * j);
             float4 cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off);
-#pragma unroll
-            for (int u = 0; u < kSeg; ++u) {
+            // Item u: the lane's slice of segment u; loads item u + 1's operands
+            // first if `next`.
+            auto item = [&](const int u, const bool next) {
                 uint4 q[S];
 #pragma unroll
                 for (int j = 0; j < S; ++j) q[j] = qn[j];
                 const float4 cf = cfn;
-                if (u + 1 < kSeg) {
+                if (next) {
 #pragma unroll
                     for (int j = 0; j < S; ++j)
                         qn[j] = *reinterpret_cast<const uint4*>(smem + qaddr[u + 1] + 16 * j);
@@ -519,8 +546,22 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                                                 __fadd2_rn(acc[i][2], acc[i][3]));
                     part_sum[i][u] = use[u] ? (t.x + t.y) : 0.f;
                 }
+            };
+            if (nseg_s == kSeg) {
+#pragma unroll
+                for (int u = 0; u < kSeg; ++u) item(u, u + 1 < kSeg);
+            } else {
+#pragma unroll
+                for (int u = 0; u < kSeg; ++u) {
+                    if (u < nseg_s) {
+                        item(u, u + 1 < nseg_s);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < M; ++i) part_sum[i][u] = 0.f;
+                    }
+                }
             }
-            float* rbuf = T.red + static_cast<size_t>(slot) * red_slot;
+            float* rbuf = T.red + static_cast<size_t>(slot * 2 + phase) * red_slot;
 #pragma unroll
             for (int i = 0; i < M; ++i) {
                 const float r = transpose_reduce4(part_sum[i][0], part_sum[i][1], part_sum[i][2],
@@ -553,7 +594,8 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const int rank = cta_rank(p);
         const int gteam = rank * p.teams + lane;
         const int nteams = p.cluster * p.teams;
-        const TeamRange tr = team_range(p, gteam);
+        const TeamRange* table = reinterpret_cast<const TeamRange*>(smem + p.off_tr);
+        const TeamRange tr = table[gteam];
         if (tr.nseg > 0) {
             const long long last = tr.row0 + tr.nseg - 1;
             const long long lb = seg_begin(tr, tr.nseg - 1, nsb) - last * nsb;
@@ -563,7 +605,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
 #pragma unroll
                 for (int i = 0; i < M; ++i) tot[i] = part[(lane * 2 + 1) * M + i];
                 for (int g2 = gteam + 1; g2 < nteams; ++g2) {
-                    const TeamRange o = team_range(p, g2);
+                    const TeamRange o = table[g2];
                     if (o.s0 >= (last + 1) * nsb) break;
                     if (o.s1 <= o.s0) continue;   // a team with an empty range
                     const int r2 = g2 / p.teams, t2 = g2 % p.teams;
@@ -622,10 +664,11 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     const int stage_bytes = ((kSeg * nsb * kBlockBytes) + 127) / 128 * 128;
     const int budget = (max_smem < kStreamSmemBudget ? max_smem : kStreamSmemBudget) - 1024;
     // bytes per team besides its ring: coefficient buffers of its warps, the
-    // per-slot partial sums, its cut-row partials and two barriers per slot
+    // partial sums per slot and ring phase, its cut-row partials, its entries of the cluster's
+    // team-range table and two barriers per slot
     auto fixed_team = [&](int depth) {
-        return team_warps * coef_bytes_per_warp(m) + depth * team_warps * kSeg * m * 4 +
-               2 * m * 4 + 2 * depth * 8 + 16;
+        return team_warps * coef_bytes_per_warp(m) + depth * 2 * team_warps * kSeg * m * 4 +
+               2 * m * 4 + cluster * kTeamRangeBytes + 2 * depth * 8 + 16;
     };
     int depth = kStreamMaxDepth;
     while (depth >= 2 && teams * (depth * stage_bytes + fixed_team(depth)) > budget) {
@@ -654,10 +697,12 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     q.off_coef = static_cast<int>(off);
     off += static_cast<size_t>(teams) * team_warps * coef_bytes_per_warp(m);
     q.off_red = static_cast<int>(off);
-    off += static_cast<size_t>(teams) * depth * team_warps * kSeg * m * 4;
+    off += static_cast<size_t>(teams) * depth * 2 * team_warps * kSeg * m * 4;
     q.off_part = static_cast<int>(off);
     off += static_cast<size_t>(teams) * 2 * m * 4;
     off = (off + 15) / 16 * 16;
+    q.off_tr = static_cast<int>(off);
+    off += static_cast<size_t>(cluster) * teams * kTeamRangeBytes;
     q.off_bar = static_cast<int>(off);
     off += static_cast<size_t>(teams) * 2 * depth * 8;
     *sp = q;

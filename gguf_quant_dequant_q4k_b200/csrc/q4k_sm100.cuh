@@ -71,6 +71,11 @@ __device__ __forceinline__ void named_barrier_sync(unsigned id, unsigned threads
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Arrives on named barrier `id` (of `threads` threads) without waiting.
+__device__ __forceinline__ void named_barrier_arrive(unsigned id, unsigned threads) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Programmatic dependent launch: wait until the preceding grid on the stream
 // has completed and its memory is visible / let the next grid start launching.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

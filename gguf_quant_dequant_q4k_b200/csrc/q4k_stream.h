@@ -23,9 +23,15 @@ constexpr int stream_max_regs(int m) {
     return 16384 / (((stream_max_threads(m) / 32 + 1 + 3) / 4) * 32) / 8 * 8;
 }
 constexpr int kStreamMaxNsb = 80;       // K <= 20480 (m = 1) / 15360 (m = 2): one team covers K
-constexpr int kStreamMaxTeams = 15;     // named barriers 1..15
+constexpr int kStreamMaxTeams = 20;     // one producer lane per team
 constexpr int kStreamMaxDepth = 8;
 constexpr int kStreamSmemBudget = 220 * 1024;
+// Ring stages each team requests before waiting on the preceding kernel (at
+// most the ring depth); the rest follow once every compute warp has issued its
+// x loads, so x is not queued behind them.
+constexpr int kStreamPreStages = 1;
+// Bytes of one entry of the kernel's table of team ranges.
+constexpr int kTeamRangeBytes = 32;
 
 struct StreamParams {
     const uint8_t* w;
@@ -36,7 +42,7 @@ struct StreamParams {
     int rows_base, rows_extra;  // cluster q owns rows_base (+1 if q < rows_extra) rows
     int teams, team_warps, depth;
     int stage_bytes;            // bytes per ring slot
-    int off_coef, off_red, off_part, off_bar;  // shared-memory offsets (bytes)
+    int off_coef, off_red, off_part, off_tr, off_bar;  // shared-memory offsets (bytes)
 };
 
 constexpr int kStreamMaxCluster = 8;    // cluster sizes the kernel supports (portable limit)

@@ -54,12 +54,12 @@ def check_plan(m, n, k):
     team_warps = -(-nsb * 8 // slices // 32)
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
     assert p["block"] <= (640 if m == 1 else 480) + 32
-    assert 2 <= depth <= 8 and 1 <= teams <= 15
+    assert 2 <= depth <= 8 and 1 <= teams <= 20
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     coef_per_warp = SEG * (4 * slices) * 4 * 16    # [seg][positions][4 groups] float4s
     need = (teams * depth * stage_bytes + teams * team_warps * coef_per_warp
-            + teams * depth * team_warps * SEG * m * 4 + teams * 2 * m * 4)
-    need = -(-need // 16) * 16 + teams * 2 * depth * 8
+            + teams * depth * 2 * team_warps * SEG * m * 4 + teams * 2 * m * 4)
+    need = -(-need // 16) * 16 + cluster * teams * 32 + teams * 2 * depth * 8
     assert p["smem_bytes"] == need and need <= 220 * 1024 - 1024
     covered = [0] * (n * nsb)
     writes = [0] * n
