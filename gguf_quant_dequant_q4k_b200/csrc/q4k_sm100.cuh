@@ -10,9 +10,11 @@ namespace q4k {
 
 // Fault flag bit raised by a kernel whose bounded wait on a bulk copy gave up.
 constexpr unsigned kFaultCopyTimeout = 1u;
-// try_wait iterations before a wait on a bulk copy is declared lost (each
-// iteration may suspend the thread for a hardware-chosen interval).
-constexpr unsigned kSpinLimit = 1u << 22;
+// try_wait iterations before a wait is declared lost (each iteration may
+// suspend the thread for up to kWaitHintNs, waking early when the phase
+// completes), so a lost copy is reported after about a second at most.
+constexpr unsigned kSpinLimit = 1u << 20;
+constexpr unsigned kWaitHintNs = 1000u;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -48,10 +50,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(kWaitHintNs)
         : "memory");
     return ok != 0;
 }
