@@ -84,6 +84,11 @@ class Oracle:
         L.q4k_oracle_gemv_rows.argtypes = [_u8p, _f32p, ctypes.c_int32, ctypes.c_int64, _i64p,
                                            ctypes.c_int64, _f64p, _f64p]
         L.q4k_oracle_gemv_rows.restype = None
+        L.q4k_oracle_embed_validate.argtypes = [ctypes.c_uint64] * 5
+        L.q4k_oracle_embed_validate.restype = ctypes.c_int
+        L.q4k_oracle_embed_lookup.argtypes = [_u8p] + [ctypes.c_uint64] * 5 + [ctypes.c_float,
+                                                                              _f32p]
+        L.q4k_oracle_embed_lookup.restype = ctypes.c_int
         self.L = L
         self.path = path
 
@@ -159,6 +164,25 @@ class Oracle:
                                     rows.size, _p(y, _f64p), _p(a, _f64p))
         return y, a
 
+    def embed_validate(self, table_bytes: int, rows: int, cols: int, hidden: int,
+                       token: int) -> int:
+        """Which of the embedding-table rules fails (EMBED_* codes; EMBED_OK = 0)."""
+        return self.L.q4k_oracle_embed_validate(table_bytes, rows, cols, hidden, token)
+
+    def embed_lookup(self, table: np.ndarray, rows: int, cols: int, hidden: int, token: int,
+                     embed_scale: float, table_bytes: int | None = None):
+        """(status, out): out = row `token` dequantised, times embed_scale (float32,
+        `hidden` values), or None when a rule fails."""
+        table = np.ascontiguousarray(table, dtype=np.uint8).reshape(-1)
+        nbytes = table.size if table_bytes is None else int(table_bytes)
+        out = np.zeros(max(int(hidden), 1), np.float32)
+        st = self.L.q4k_oracle_embed_lookup(_p(table, _u8p), nbytes, rows, cols, hidden, token,
+                                            float(embed_scale), _p(out, _f32p))
+        return st, (out[:hidden] if st == EMBED_OK else None)
+
+
+# q4k_oracle_embed_validate results
+EMBED_OK, EMBED_SHAPE, EMBED_TOKEN, EMBED_WIDTH, EMBED_OVERFLOW, EMBED_SIZE = range(6)
 
 _default: Oracle | None = None
 
@@ -197,6 +221,14 @@ def gemv(w, x, n, k, nthreads=1):
 
 def gemv_rows(w, x, n, k, rows):
     return default().gemv_rows(w, x, n, k, rows)
+
+
+def embed_validate(table_bytes, rows, cols, hidden, token):
+    return default().embed_validate(table_bytes, rows, cols, hidden, token)
+
+
+def embed_lookup(table, rows, cols, hidden, token, embed_scale, table_bytes=None):
+    return default().embed_lookup(table, rows, cols, hidden, token, embed_scale, table_bytes)
 
 
 def tolerance(a: np.ndarray) -> np.ndarray:

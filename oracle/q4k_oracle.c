@@ -248,3 +248,80 @@ void q4k_oracle_gemv_rows(const uint8_t *w, const float *x, int32_t m, int64_t k
     for (int64_t s = 0; s < nrows; ++s)
         gemv_row(w, x, m, k, rows[s], y + s, a + s, nrows);
 }
+
+/*
+ * Embedding lookup from a Q4_K table ("turbospark-runtime 0.1.0,
+ * src/real_forward_dispatch.rs": `validate_block_quant_embedding` with the
+ * Q4_K block constants, called by `validate_q4_k_embedding` before
+ * `encode_embed_lookup_q4_k(..., token, hidden, embed_scale)`).
+ *
+ * Validation, in the page's order; the return value says which rule failed:
+ *   Q4K_ORACLE_EMBED_SHAPE     the table is not [rows, hidden] (cols != hidden)
+ *   Q4K_ORACLE_EMBED_TOKEN     token >= rows
+ *   Q4K_ORACLE_EMBED_WIDTH     hidden == 0 or hidden not a whole number of 256-weight blocks
+ *   Q4K_ORACLE_EMBED_OVERFLOW  row size, table size or end of the selected row overflows 64 bits
+ *   Q4K_ORACLE_EMBED_SIZE      table_bytes != rows * row_bytes, or the selected row
+ *                              does not end inside the table
+ * with row_bytes = hidden / 256 * 144.
+ *
+ * Value (a reading: the page names the call but does not print the kernel):
+ * out[j] = fl32(w[j] * embed_scale), where w[j] is the dequantised f32 weight
+ * (above) of row `token`; the product of two floats is exact in double, so the
+ * double product rounded to float is that single f32 rounding.
+ */
+enum {
+    Q4K_ORACLE_EMBED_OK = 0,
+    Q4K_ORACLE_EMBED_SHAPE = 1,
+    Q4K_ORACLE_EMBED_TOKEN = 2,
+    Q4K_ORACLE_EMBED_WIDTH = 3,
+    Q4K_ORACLE_EMBED_OVERFLOW = 4,
+    Q4K_ORACLE_EMBED_SIZE = 5,
+};
+
+static int mul_overflows(uint64_t a, uint64_t b, uint64_t *out)
+{
+    if (a != 0 && b > UINT64_MAX / a)
+        return 1;
+    *out = a * b;
+    return 0;
+}
+
+int q4k_oracle_embed_validate(uint64_t table_bytes, uint64_t rows, uint64_t cols,
+                              uint64_t hidden, uint64_t token)
+{
+    if (cols != hidden)
+        return Q4K_ORACLE_EMBED_SHAPE;
+    if (token >= rows)
+        return Q4K_ORACLE_EMBED_TOKEN;
+    if (hidden == 0 || hidden % QK != 0)
+        return Q4K_ORACLE_EMBED_WIDTH;
+    uint64_t row_bytes, expected, selected_end;
+    if (mul_overflows(hidden / QK, SB_BYTES, &row_bytes))
+        return Q4K_ORACLE_EMBED_OVERFLOW;
+    if (mul_overflows(rows, row_bytes, &expected))
+        return Q4K_ORACLE_EMBED_OVERFLOW;
+    if (token == UINT64_MAX || mul_overflows(token + 1, row_bytes, &selected_end))
+        return Q4K_ORACLE_EMBED_OVERFLOW;
+    if (table_bytes != expected || selected_end > table_bytes)
+        return Q4K_ORACLE_EMBED_SIZE;
+    return Q4K_ORACLE_EMBED_OK;
+}
+
+/* out[0..hidden) = row `token` of the table times embed_scale; returns the
+ * validation result and writes nothing unless it is Q4K_ORACLE_EMBED_OK. */
+int q4k_oracle_embed_lookup(const uint8_t *table, uint64_t table_bytes, uint64_t rows,
+                            uint64_t cols, uint64_t hidden, uint64_t token, float embed_scale,
+                            float *out)
+{
+    int st = q4k_oracle_embed_validate(table_bytes, rows, cols, hidden, token);
+    if (st != Q4K_ORACLE_EMBED_OK)
+        return st;
+    uint64_t nsb = hidden / QK;
+    float wv[QK];
+    for (uint64_t b = 0; b < nsb; ++b) {
+        dequant_block(table + (token * nsb + b) * SB_BYTES, wv);
+        for (int t = 0; t < QK; ++t)
+            out[b * QK + t] = (float)((double)wv[t] * (double)embed_scale);
+    }
+    return Q4K_ORACLE_EMBED_OK;
+}

@@ -285,9 +285,80 @@ def check_golden(o):
     assert np.array_equal(deq[:, 255].astype(np.float64), ref[:, 3])
 
 
+def check_embed_page_cases(o):
+    """The page's own validation test (tests/golden/embed_validation_cases.txt)."""
+    path = os.path.join(GOLDEN, "embed_validation_cases.txt")
+    n = 0
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            *nums, expect = line.split()
+            st = o.embed_validate(*[int(v) for v in nums])
+            assert (st == 0) == (expect == "ok"), line
+            n += 1
+    assert n == 4
+
+
+def check_embed_rules(o):
+    """Each validation rule alone, in the page's order (codes: 1 shape, 2 token,
+    3 width, 4 overflow, 5 size)."""
+    row = 144
+    ok = (10 * row, 10, 256, 256, 9)
+    assert o.embed_validate(*ok) == 0
+    assert o.embed_validate(10 * row, 10, 512, 256, 9) == 1          # cols != hidden
+    assert o.embed_validate(10 * row, 10, 256, 256, 10) == 2         # token == rows
+    assert o.embed_validate(0, 0, 256, 256, 0) == 2                  # empty table
+    assert o.embed_validate(10 * row, 10, 300, 300, 0) == 3          # not whole blocks
+    assert o.embed_validate(0, 10, 0, 0, 0) == 3                     # zero width
+    assert o.embed_validate(10 * row + 1, 10, 256, 256, 0) == 5      # one byte too many
+    assert o.embed_validate(10 * row - 1, 10, 256, 256, 0) == 5      # one byte short
+    assert o.embed_validate(20 * 2 * row, 20, 512, 512, 19) == 0     # two blocks per row
+    assert o.embed_validate(20 * 2 * row, 20, 512, 512, 20) == 2
+    # shape is checked before the token, the token before the width
+    assert o.embed_validate(0, 1, 512, 256, 5) == 1
+    assert o.embed_validate(0, 1, 300, 300, 5) == 2
+    big = 1 << 63
+    assert o.embed_validate(0, big, 256, 256, 0) == 4                # rows * row_bytes overflows
+    assert o.embed_validate(0, big, 1 << 62, 1 << 62, 0) == 4        # wide rows: table size overflows
+
+
+def check_embed_values(o, seed=18):
+    """Rows 0, mid and last of small tables, several scales, against exact
+    arithmetic from the unpacked fields: w = d*sc*q - dmin*m rounded to f32, then
+    w * scale rounded to f32."""
+    rng = np.random.default_rng(seed)
+    for rows, hidden in [(3, 256), (5, 512), (2, 768)]:
+        nsb = hidden // 256
+        fields, blocks = [], []
+        for _ in range(rows * nsb):
+            d = int(np.float16(rng.uniform(1e-3, 2e-2)).view(np.uint16))
+            dm = int(np.float16(rng.uniform(1e-3, 2e-2)).view(np.uint16))
+            sc, mn, q = rng.integers(0, 64, 8), rng.integers(0, 64, 8), rng.integers(0, 16, 256)
+            fields.append((d, dm, sc, mn, q))
+            blocks.append(o.pack(d, dm, sc, mn, q))
+        table = np.concatenate(blocks)
+        for token in sorted({0, rows // 2, rows - 1}):
+            for scale in (1.0, 2.0, -0.5, 0.0, float(np.float32(0.1234567)), 3.0e-3):
+                st, out = o.embed_lookup(table, rows, hidden, hidden, token, scale)
+                assert st == 0
+                for b in range(nsb):
+                    d, dm, sc, mn, q = fields[token * nsb + b]
+                    for t in range(0, 256, 7):
+                        w = _exact_weight(d, dm, sc[t // 32], mn[t // 32], q[t])
+                        ref = np.float32(float(w * Fraction(float(np.float32(scale)))))
+                        got = out[b * 256 + t]
+                        assert got == ref or (np.isnan(got) and np.isnan(ref)), \
+                            (rows, hidden, token, scale, b, t, got, ref)
+    # a failed rule writes nothing and returns no row
+    st, out = o.embed_lookup(np.zeros(144 * 4, np.uint8), 4, 256, 256, 4, 1.0)
+    assert st == 2 and out is None
+
+
 ALL_CHECKS = [
     check_half_all_patterns, check_half_known, check_scale_bit_map, check_nibble_map,
     check_closed_forms, check_pack_roundtrip, check_unpack_pack_bytes, check_bruteforce_gemv,
     check_gemv_vs_matmul, check_unit_and_zero_vectors, check_vectors_independent,
-    check_threads_and_rows, check_golden,
+    check_threads_and_rows, check_golden, check_embed_page_cases, check_embed_rules,
+    check_embed_values,
 ]

@@ -27,6 +27,12 @@ MUTANTS = {
     "d_dmin_fields_swapped": ("*d_bits = u16le(sb + 0);", "*d_bits = u16le(sb + 2);"),
     "x_block_stride_dropped": ("x + (int64_t)i * k + b * QK", "x + (int64_t)i * k"),
     "abs_sum_signed": ("sa += fabs(p);", "sa += p;"),
+    "embed_token_off_by_one": ("if (token >= rows)", "if (token > rows)"),
+    "embed_size_check_relaxed": ("if (table_bytes != expected ||", "if (table_bytes < expected ||"),
+    "embed_width_rule_dropped": ("if (hidden == 0 || hidden % QK != 0)", "if (hidden == 0)"),
+    "embed_shape_rule_dropped": ("if (cols != hidden)\n        return Q4K_ORACLE_EMBED_SHAPE;", ""),
+    "embed_scale_not_applied": ("(float)((double)wv[t] * (double)embed_scale)", "wv[t]"),
+    "embed_wrong_row_stride": ("table + (token * nsb + b) * SB_BYTES", "table + (token + b) * SB_BYTES"),
 }
 
 
