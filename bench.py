@@ -273,7 +273,51 @@ def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
                              "how": "one CUDA graph of the 224 projection GEMVs, replayed"}
     del g, layers
     torch.cuda.empty_cache()
+    out["embedding"] = embedding_workloads(q4k, torch, dev, stream)
     return out
+
+
+def embedding_workloads(q4k, torch, dev, stream) -> list:
+    """Q4_K embedding lookups from a 128256 x 4096 table (an 8B model's token
+    embedding): one token (q4k_embed_lookup_f32) and gathers of 8 and 512
+    device-resident tokens (q4k_embed_gather_f32). Bytes counted per call =
+    rows read (hidden/256*144 each) + f32 rows written (4*hidden each)."""
+    rows, hidden = 128256, 4096
+    w, _ = q4k_synth.q4k_problem(rows, hidden, 1, q4k_synth.SEEDS[(rows, hidden)])
+    table = torch.from_numpy(w).to(dev)
+    rng = np.random.default_rng(3)
+    res = []
+    for n_tok in (1, 8, 512):
+        toks = torch.from_numpy(rng.integers(0, rows, n_tok).astype(np.int32)).to(dev)
+        out = torch.empty((n_tok, hidden), dtype=torch.float32, device=dev)
+
+        def call():
+            if n_tok == 1:
+                q4k.q4k_embed_lookup_f32(table, rows, hidden, hidden, 12345, 1.0, out,
+                                         stream=stream)
+            else:
+                q4k.q4k_embed_gather_f32(table, rows, hidden, toks, n_tok, 1.0, out,
+                                         stream=stream)
+        with torch.cuda.stream(stream):
+            for _ in range(10):
+                call()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        reps = 200
+        a0.record(stream)
+        for _ in range(reps):
+            call()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        us = a0.elapsed_time(a1) * 1e3 / reps
+        b = n_tok * (hidden // 256 * 144 + 4 * hidden)
+        res.append({"rows": rows, "hidden": hidden, "tokens": n_tok,
+                    "call": "q4k_embed_lookup_f32" if n_tok == 1 else "q4k_embed_gather_f32",
+                    "us_per_call": round(us, 3), "gbs": round(b / us / 1e3, 1)})
+    assert q4k.q4k_device_fault_flags() == 0
+    del table
+    torch.cuda.empty_cache()
+    return res
 
 
 # --------------------------------------------------------------------------- our arm

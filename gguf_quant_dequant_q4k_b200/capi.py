@@ -20,6 +20,9 @@ Q4K_ERR_ALIGN = 3
 Q4K_ERR_UNSUPPORTED_M = 4
 Q4K_ERR_CUDA = 5
 Q4K_ERR_OVERLAP = 6
+Q4K_ERR_RANGE = 7
+Q4K_FAULT_COPY_TIMEOUT = 1
+Q4K_FAULT_TOKEN_RANGE = 2
 Q4K_QK = 256
 Q4K_BLOCK_BYTES = 144
 Q4K_MAX_M = 8
@@ -28,7 +31,8 @@ Q4K_KERNEL_STREAM = 2
 
 # Every function include/q4k.h declares.
 EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
-           "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags")
+           "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags",
+           "q4k_embed_lookup_f32", "q4k_embed_gather_f32")
 
 
 class Q4KError(RuntimeError):
@@ -72,6 +76,12 @@ _lib.q4k_gemv_plan_for.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, cty
 _lib.q4k_gemv_plan_for.restype = ctypes.c_int
 _lib.q4k_device_fault_flags.argtypes = [ctypes.POINTER(ctypes.c_uint)]
 _lib.q4k_device_fault_flags.restype = ctypes.c_int
+_lib.q4k_embed_lookup_f32.argtypes = [_vp, ctypes.c_ulonglong, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_uint, ctypes.c_float, _vp, _vp]
+_lib.q4k_embed_lookup_f32.restype = ctypes.c_int
+_lib.q4k_embed_gather_f32.argtypes = [_vp, ctypes.c_ulonglong, ctypes.c_int, ctypes.c_int, _vp,
+                                      ctypes.c_int, ctypes.c_float, _vp, _vp]
+_lib.q4k_embed_gather_f32.restype = ctypes.c_int
 
 
 def library() -> ctypes.CDLL:
@@ -145,3 +155,48 @@ def q4k_dequant_f32(w, out, n: int, k: int, stream=None) -> None:
     st = q4k_dequant_f32_status(w, out, n, k, stream)
     if st != Q4K_OK:
         raise Q4KError(st, "q4k_dequant_f32")
+
+
+def _nbytes(t, given) -> int:
+    if given is not None:
+        return int(given)
+    return t.numel() * t.element_size()
+
+
+def q4k_embed_lookup_f32_status(table, rows: int, cols: int, hidden: int, token: int,
+                                embed_scale: float, out, stream=None,
+                                table_bytes: int | None = None) -> int:
+    """Raw status of the C call (no exception). table_bytes defaults to the
+    tensor's size; pass it explicitly with a raw pointer."""
+    return _lib.q4k_embed_lookup_f32(_ptr(table), _nbytes(table, table_bytes), int(rows),
+                                     int(cols), int(hidden), int(token) & 0xFFFFFFFF,
+                                     float(embed_scale), _ptr(out), _stream(stream))
+
+
+def q4k_embed_lookup_f32(table, rows: int, cols: int, hidden: int, token: int,
+                         embed_scale: float, out, stream=None,
+                         table_bytes: int | None = None) -> None:
+    """out[hidden] = row `token` of the Q4_K table [rows, cols], dequantised, x embed_scale."""
+    st = q4k_embed_lookup_f32_status(table, rows, cols, hidden, token, embed_scale, out, stream,
+                                     table_bytes)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_embed_lookup_f32")
+
+
+def q4k_embed_gather_f32_status(table, rows: int, hidden: int, tokens, n_tokens: int,
+                                embed_scale: float, out, stream=None,
+                                table_bytes: int | None = None) -> int:
+    return _lib.q4k_embed_gather_f32(_ptr(table), _nbytes(table, table_bytes), int(rows),
+                                     int(hidden), _ptr(tokens), int(n_tokens),
+                                     float(embed_scale), _ptr(out), _stream(stream))
+
+
+def q4k_embed_gather_f32(table, rows: int, hidden: int, tokens, n_tokens: int,
+                         embed_scale: float, out, stream=None,
+                         table_bytes: int | None = None) -> None:
+    """out[n_tokens, hidden] = rows tokens[i] (int32, device) of the table, x embed_scale.
+    A token outside the table gives a zero row and raises Q4K_FAULT_TOKEN_RANGE."""
+    st = q4k_embed_gather_f32_status(table, rows, hidden, tokens, n_tokens, embed_scale, out,
+                                     stream, table_bytes)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_embed_gather_f32")

@@ -94,6 +94,7 @@ const char* q4k_status_string(int status) {
         case Q4K_ERR_UNSUPPORTED_M: return "unsupported number of vectors (need 1 <= m <= 8)";
         case Q4K_ERR_CUDA: return "CUDA runtime error (see q4k_last_cuda_error)";
         case Q4K_ERR_OVERLAP: return "output overlaps an input";
+        case Q4K_ERR_RANGE: return "embedding token outside the table's rows";
         default: return "unknown status";
     }
 }
@@ -102,7 +103,58 @@ int q4k_last_cuda_error(void) { return t_last_cuda_error; }
 
 int q4k_device_fault_flags(unsigned int* flags) {
     if (flags == nullptr) return Q4K_ERR_NULL;
-    return read_fault_flags(flags);
+    unsigned a = 0, b = 0;
+    int st = read_fault_flags(&a);
+    if (st != Q4K_OK) return st;
+    st = read_embed_fault_flags(&b);
+    if (st != Q4K_OK) return st;
+    *flags = a | b;
+    return Q4K_OK;
+}
+
+int q4k_embed_lookup_f32(const void* table, unsigned long long table_bytes, int rows, int cols,
+                         int hidden, unsigned int token, float embed_scale, float* out,
+                         q4k_stream_t stream) {
+    // The checks of `validate_block_quant_embedding`, in its order.
+    if (cols != hidden) return Q4K_ERR_SHAPE;
+    if (rows <= 0 || token >= static_cast<unsigned>(rows)) return Q4K_ERR_RANGE;
+    if (hidden <= 0 || hidden % Q4K_QK != 0) return Q4K_ERR_SHAPE;
+    const unsigned long long row_bytes =
+        static_cast<unsigned long long>(hidden / Q4K_QK) * Q4K_BLOCK_BYTES;
+    const unsigned long long expected = static_cast<unsigned long long>(rows) * row_bytes;
+    const unsigned long long selected_end = (static_cast<unsigned long long>(token) + 1) * row_bytes;
+    if (table_bytes != expected || selected_end > table_bytes) return Q4K_ERR_SHAPE;
+    if (table == nullptr || out == nullptr) return Q4K_ERR_NULL;
+    if (!aligned(table, 16) || !aligned(out, 16)) return Q4K_ERR_ALIGN;
+    const size_t obytes = static_cast<size_t>(hidden) * sizeof(float);
+    if (overlaps(out, obytes, table, static_cast<size_t>(table_bytes))) return Q4K_ERR_OVERLAP;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return launch_embed(table, rows, hidden, nullptr, token, 1, embed_scale, out, dev.sm_count,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4k_embed_gather_f32(const void* table, unsigned long long table_bytes, int rows, int hidden,
+                         const int* tokens, int n_tokens, float embed_scale, float* out,
+                         q4k_stream_t stream) {
+    if (table == nullptr || tokens == nullptr || out == nullptr) return Q4K_ERR_NULL;
+    if (rows <= 0 || hidden <= 0 || hidden % Q4K_QK != 0 || n_tokens < 0) return Q4K_ERR_SHAPE;
+    const unsigned long long row_bytes =
+        static_cast<unsigned long long>(hidden / Q4K_QK) * Q4K_BLOCK_BYTES;
+    if (table_bytes != static_cast<unsigned long long>(rows) * row_bytes) return Q4K_ERR_SHAPE;
+    if (!aligned(table, 16) || !aligned(tokens, 4) || !aligned(out, 16)) return Q4K_ERR_ALIGN;
+    const size_t obytes = static_cast<size_t>(n_tokens) * static_cast<size_t>(hidden) * sizeof(float);
+    const size_t tbytes = static_cast<size_t>(n_tokens) * sizeof(int);
+    if (overlaps(out, obytes, table, static_cast<size_t>(table_bytes)) ||
+        overlaps(out, obytes, tokens, tbytes))
+        return Q4K_ERR_OVERLAP;
+    if (n_tokens == 0) return Q4K_OK;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return launch_embed(table, rows, hidden, tokens, 0u, n_tokens, embed_scale, out, dev.sm_count,
+                        reinterpret_cast<cudaStream_t>(stream));
 }
 
 int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {

@@ -35,4 +35,12 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, 
 
 int launch_dequant(const void* w, float* out, int n, int k, int num_sms, cudaStream_t stream);
 
+// Embedding rows: row tokens[i] (device array) or, if tokens is null, row
+// `token` (n_tokens = 1), dequantised and scaled. Arguments are validated.
+int launch_embed(const void* table, long long rows, int hidden, const int* tokens, unsigned token,
+                 int n_tokens, float scale, float* out, int num_sms, cudaStream_t stream);
+
+// Reads and clears the embedding kernel's fault flags (synchronises).
+int read_embed_fault_flags(unsigned* flags);
+
 }  // namespace q4k

@@ -69,8 +69,13 @@ enum q4k_status {
     Q4K_ERR_ALIGN = 3,          /* w or x not 16-byte aligned, y/out not 4-byte    */
     Q4K_ERR_UNSUPPORTED_M = 4,  /* m outside 1..Q4K_MAX_M                          */
     Q4K_ERR_CUDA = 5,           /* a CUDA runtime call failed (see last_cuda_error) */
-    Q4K_ERR_OVERLAP = 6         /* an output range overlaps an input range         */
+    Q4K_ERR_OVERLAP = 6,        /* an output range overlaps an input range         */
+    Q4K_ERR_RANGE = 7           /* an embedding token outside the table's rows     */
 };
+
+/* Bits of q4k_device_fault_flags(). */
+#define Q4K_FAULT_COPY_TIMEOUT 1u  /* a bounded wait on a bulk copy gave up          */
+#define Q4K_FAULT_TOKEN_RANGE 2u   /* q4k_embed_gather_f32 met a token outside the table */
 
 #define Q4K_QK 256          /* weights per superblock */
 #define Q4K_BLOCK_BYTES 144 /* bytes per superblock   */
@@ -121,11 +126,49 @@ Q4K_API const char *q4k_status_string(int status);
 Q4K_API int q4k_last_cuda_error(void);
 
 /*
- * Reads and clears the calling device's fault flags: bit 0 is set if a bounded
- * wait inside a kernel on a bulk copy into shared memory gave up (the kernel
- * then skipped its remaining work and returned; its output is invalid). This
- * never happens in normal operation. Synchronises the device. Returns a
- * q4k_status; *flags receives the flags.
+ * Embedding lookup: out = row `token` of a Q4_K embedding table, dequantised,
+ * times embed_scale ("turbospark-runtime 0.1.0, src/real_forward_dispatch.rs":
+ * `validate_q4_k_embedding` then `encode_embed_lookup_q4_k(..., token, hidden,
+ * embed_scale)`).
+ *   table      : a [rows, cols] Q4_K matrix, table_bytes bytes, 16-byte aligned.
+ *   hidden     : the model width the caller expects; out has hidden floats,
+ *                16-byte aligned, and must not overlap the table.
+ *   out[j]     = fl32(w[j] * embed_scale), w[j] the f32 weight d*sc*q - dmin*m.
+ * Checked before launch, in the page's order: cols != hidden -> Q4K_ERR_SHAPE;
+ * token >= rows -> Q4K_ERR_RANGE; hidden not a positive multiple of 256 ->
+ * Q4K_ERR_SHAPE; table_bytes != rows * (hidden/256) * 144, or the selected row
+ * not ending inside the table -> Q4K_ERR_SHAPE. Then NULL, alignment and
+ * overlap. Nothing is launched unless every check passes.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_embed_lookup_f32(const void *table, unsigned long long table_bytes, int rows,
+                                 int cols, int hidden, unsigned int token, float embed_scale,
+                                 float *out, q4k_stream_t stream);
+
+/*
+ * Row gather for n_tokens tokens held in device memory (a batch of lookups
+ * whose tokens were produced on the device): out[i*hidden + j] = fl32(w[j] of
+ * row tokens[i] * embed_scale).
+ *   table, table_bytes, rows, hidden: as above (the table is [rows, hidden];
+ *                table_bytes must equal rows * (hidden/256) * 144).
+ *   tokens     : n_tokens int32 in device memory, 4-byte aligned.
+ *   out        : n_tokens x hidden float32, 16-byte aligned, no overlap.
+ * A token outside 0..rows-1 cannot be refused before launch: its output row is
+ * written as zeros and Q4K_FAULT_TOKEN_RANGE is raised in the device fault
+ * flags. n_tokens == 0 launches nothing.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_embed_gather_f32(const void *table, unsigned long long table_bytes, int rows,
+                                 int hidden, const int *tokens, int n_tokens, float embed_scale,
+                                 float *out, q4k_stream_t stream);
+
+/*
+ * Reads and clears the calling device's fault flags (Q4K_FAULT_* bits):
+ * Q4K_FAULT_COPY_TIMEOUT if a bounded wait inside a kernel on a bulk copy into
+ * shared memory gave up (the kernel then skipped its remaining work and
+ * returned; its output is invalid; never happens in normal operation);
+ * Q4K_FAULT_TOKEN_RANGE if q4k_embed_gather_f32 met a token outside its table.
+ * Synchronises the device. Returns a q4k_status; *flags receives the flags.
  */
 Q4K_API int q4k_device_fault_flags(unsigned int *flags);
 

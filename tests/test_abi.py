@@ -43,7 +43,7 @@ def test_weight_bytes_size_rule():
 
 
 def test_status_strings():
-    for st in range(7):
+    for st in range(8):
         assert q4k.q4k_status_string(st)
     assert q4k.q4k_status_string(99) == "unknown status"
     assert q4k.q4k_last_cuda_error() == 0
@@ -89,3 +89,90 @@ def test_gemv_raises_q4kerror():
     with pytest.raises(q4k.Q4KError) as e:
         q4k.q4k_gemv(A16, A16 * 2, A16 * 3, 1, 4, 100, stream=0)
     assert e.value.status == q4k.Q4K_ERR_SHAPE
+
+
+# Embedding validation: every call below is refused before any CUDA call.
+GOLDEN_EMBED = os.path.join(ROOT, "tests", "golden", "embed_validation_cases.txt")
+
+
+def embed_page_cases():
+    cases = []
+    with open(GOLDEN_EMBED) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            *nums, expect = line.split()
+            cases.append(([int(v) for v in nums], expect))
+    return cases
+
+
+def test_embed_page_cases_refused_like_the_oracle():
+    """The page's validation test: the failing cases are refused by the C ABI
+    with the status the oracle's verdict maps to (token -> Q4K_ERR_RANGE, the
+    other rules -> Q4K_ERR_SHAPE); the passing case passes validation (it is then
+    refused for its NULL output, before any CUDA call)."""
+    import oracle
+    cases = embed_page_cases()
+    assert len(cases) == 4
+    for (table_bytes, rows, cols, hidden, token), expect in cases:
+        verdict = oracle.embed_validate(table_bytes, rows, cols, hidden, token)
+        st = capi.q4k_embed_lookup_f32_status(A16, rows, cols, hidden, token, 1.0, None,
+                                              stream=0, table_bytes=table_bytes)
+        if expect == "ok":
+            assert verdict == oracle.EMBED_OK and st == q4k.Q4K_ERR_NULL
+        else:
+            want = q4k.Q4K_ERR_RANGE if verdict == oracle.EMBED_TOKEN else q4k.Q4K_ERR_SHAPE
+            assert verdict != oracle.EMBED_OK and st == want, (table_bytes, rows, cols, token)
+
+
+@pytest.mark.parametrize("table_bytes,rows,cols,hidden,token,expect", [
+    (10 * 144, 10, 512, 256, 9, q4k.Q4K_ERR_SHAPE),      # cols != hidden
+    (10 * 144, 10, 256, 256, 10, q4k.Q4K_ERR_RANGE),     # token == rows
+    (0, 0, 256, 256, 0, q4k.Q4K_ERR_RANGE),              # empty table
+    (10 * 144, 10, 300, 300, 0, q4k.Q4K_ERR_SHAPE),      # not whole blocks
+    (0, 10, 0, 0, 0, q4k.Q4K_ERR_SHAPE),                 # zero width
+    (10 * 144 + 1, 10, 256, 256, 0, q4k.Q4K_ERR_SHAPE),  # one byte too many
+    (10 * 144 - 1, 10, 256, 256, 0, q4k.Q4K_ERR_SHAPE),  # one byte short
+    (0, 1, 512, 256, 5, q4k.Q4K_ERR_SHAPE),              # shape before token
+    (0, 1, 300, 300, 5, q4k.Q4K_ERR_RANGE),              # token before width
+])
+def test_embed_lookup_rules(table_bytes, rows, cols, hidden, token, expect):
+    import oracle
+    verdict = oracle.embed_validate(table_bytes, rows, cols, hidden, token)
+    assert (verdict == oracle.EMBED_TOKEN) == (expect == q4k.Q4K_ERR_RANGE)
+    assert verdict != oracle.EMBED_OK
+    st = capi.q4k_embed_lookup_f32_status(A16, rows, cols, hidden, token, 1.0, A16 * 4,
+                                          stream=0, table_bytes=table_bytes)
+    assert st == expect
+
+
+def test_embed_lookup_pointer_checks():
+    ok = dict(rows=10, cols=256, hidden=256, token=3, embed_scale=1.0, stream=0,
+              table_bytes=10 * 144)
+    assert capi.q4k_embed_lookup_f32_status(0, out=A16 * 4, **ok) == q4k.Q4K_ERR_NULL
+    assert capi.q4k_embed_lookup_f32_status(A16, out=0, **ok) == q4k.Q4K_ERR_NULL
+    assert capi.q4k_embed_lookup_f32_status(A16 + 8, out=A16 * 4, **ok) == q4k.Q4K_ERR_ALIGN
+    assert capi.q4k_embed_lookup_f32_status(A16, out=A16 * 4 + 4, **ok) == q4k.Q4K_ERR_ALIGN
+    assert capi.q4k_embed_lookup_f32_status(A16, out=A16 + 16, **ok) == q4k.Q4K_ERR_OVERLAP
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(table=0), q4k.Q4K_ERR_NULL),
+    (dict(tokens=0), q4k.Q4K_ERR_NULL),
+    (dict(out=0), q4k.Q4K_ERR_NULL),
+    (dict(rows=0, table_bytes=0), q4k.Q4K_ERR_SHAPE),
+    (dict(hidden=300), q4k.Q4K_ERR_SHAPE),
+    (dict(hidden=0), q4k.Q4K_ERR_SHAPE),
+    (dict(n_tokens=-1), q4k.Q4K_ERR_SHAPE),
+    (dict(table_bytes=10 * 144 - 144), q4k.Q4K_ERR_SHAPE),
+    (dict(tokens=A16 * 2 + 2), q4k.Q4K_ERR_ALIGN),
+    (dict(out=A16 * 4 + 8), q4k.Q4K_ERR_ALIGN),
+    (dict(out=A16), q4k.Q4K_ERR_OVERLAP),
+    (dict(tokens=A16 * 4 + 16), q4k.Q4K_ERR_OVERLAP),
+    (dict(n_tokens=0), q4k.Q4K_OK),                        # nothing to do: no launch
+])
+def test_embed_gather_checks(kw, expect):
+    args = dict(table=A16, rows=10, hidden=256, tokens=A16 * 2, n_tokens=4, embed_scale=1.0,
+                out=A16 * 4, stream=0, table_bytes=10 * 144)
+    args.update(kw)
+    assert capi.q4k_embed_gather_f32_status(**args) == expect
