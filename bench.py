@@ -210,14 +210,15 @@ def cpu_baseline() -> dict:
 
 def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
     """The other decode workloads of the sweep's configuration list, on this GPU:
-    multi-vector shapes (m = 1, 2, 4, 8) and the 32-layer 8B-class decode sweep.
+    multi-vector shapes (m = 1, 2, 4, 8, and the batches 16 and 32), the
+    32-layer 8B-class decode sweep and embedding lookups.
     Each figure is bytes counted / device time (CUDA events)."""
     out = {"multivector": [], "layer_sweep_32": None}
     for n, k in q4k_synth.SHAPES_MULTIVEC:
         w, _ = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEED_MULTIVEC[(n, k)])
         wd = torch.from_numpy(w).to(dev)
         ws = [wd] + [wd.clone() for _ in range(max(2, -(-2 * l2 // w.nbytes) + 1) - 1)]
-        for m in (1, 2, 4, 8):
+        for m in (1, 2, 4, 8, 16, 32):
             x = torch.from_numpy(q4k_synth.x_vectors(k, m, 77 + m)).to(dev)
             y = torch.empty((m, n), dtype=torch.float32, device=dev)
             with torch.cuda.stream(stream):

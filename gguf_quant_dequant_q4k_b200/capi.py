@@ -25,7 +25,7 @@ Q4K_FAULT_COPY_TIMEOUT = 1
 Q4K_FAULT_TOKEN_RANGE = 2
 Q4K_QK = 256
 Q4K_BLOCK_BYTES = 144
-Q4K_MAX_M = 8
+Q4K_MAX_M = 64
 Q4K_KERNEL_WARP_ROWS = 1
 Q4K_KERNEL_STREAM = 2
 

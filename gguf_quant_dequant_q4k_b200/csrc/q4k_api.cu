@@ -91,7 +91,7 @@ const char* q4k_status_string(int status) {
         case Q4K_ERR_NULL: return "null pointer argument";
         case Q4K_ERR_SHAPE: return "invalid shape (need n > 0, k > 0, k % 256 == 0)";
         case Q4K_ERR_ALIGN: return "misaligned pointer (w, x, out: 16 bytes; y: 4 bytes)";
-        case Q4K_ERR_UNSUPPORTED_M: return "unsupported number of vectors (need 1 <= m <= 8)";
+        case Q4K_ERR_UNSUPPORTED_M: return "unsupported number of vectors (need 1 <= m <= 64)";
         case Q4K_ERR_CUDA: return "CUDA runtime error (see q4k_last_cuda_error)";
         case Q4K_ERR_OVERLAP: return "output overlaps an input";
         case Q4K_ERR_RANGE: return "embedding token outside the table's rows";

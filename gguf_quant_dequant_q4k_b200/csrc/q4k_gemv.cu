@@ -1,8 +1,9 @@
-// q4k_gemv.cu -- y = W x for Q4_K W and 1..8 f32 vectors (q4k_gemv).
+// q4k_gemv.cu -- y = W x for Q4_K W and 1..64 f32 vectors (q4k_gemv).
 //
-// General path (any K, m <= 8): one warp per output row (the row-per-warp mapping of
-// the pages' `Q4KGemv`, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs",
-// grid (n,1) x 32 threads), with each decoded weight applied to all m vectors
+// General path (any K, tiles of up to 8 vectors): one warp per output row
+// (the row-per-warp mapping of the pages' `Q4KGemv`, "realizar 0.8.5,
+// src/cuda/executor/q4k_gemv_cached.rs", grid (n,1) x 32 threads), with each
+// decoded weight applied to all m vectors
 // (`BatchedQ4KGemv`, "realizar 0.8.5, src/cuda/executor/uses.rs": dequantise
 // once, multiply by M input vectors).
 //
@@ -20,6 +21,7 @@ namespace q4k {
 namespace {
 
 constexpr int kRowsThreads = 256;
+constexpr int kRowsMaxM = 8;   // vectors per launch of the general kernel
 
 template <int M>
 __global__ void __launch_bounds__(kRowsThreads)
@@ -125,7 +127,7 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
     plan->smem_bytes = 0;
     plan->teams = 0;
     plan->depth = 0;
-    plan->launches = 1;
+    plan->launches = (m + kRowsMaxM - 1) / kRowsMaxM;   // tiles of up to 8 vectors
     plan->units = n;
     plan->units_per_cta_max = ((n + warps - 1) / warps) * warps_per_cta;
     return Q4K_OK;
@@ -162,19 +164,25 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, 
         }
         return Q4K_OK;
     }
-    switch (m) {
-        case 1: launch_rows<1>(plan, w, x, y, n, k, stream); break;
-        case 2: launch_rows<2>(plan, w, x, y, n, k, stream); break;
-        case 3: launch_rows<3>(plan, w, x, y, n, k, stream); break;
-        case 4: launch_rows<4>(plan, w, x, y, n, k, stream); break;
-        case 5: launch_rows<5>(plan, w, x, y, n, k, stream); break;
-        case 6: launch_rows<6>(plan, w, x, y, n, k, stream); break;
-        case 7: launch_rows<7>(plan, w, x, y, n, k, stream); break;
-        case 8: launch_rows<8>(plan, w, x, y, n, k, stream); break;
-        default: return Q4K_ERR_UNSUPPORTED_M;
+    // vector tiles of up to 8 (the tiling of `batched_q4k_gemv_into`)
+    for (int i0 = 0; i0 < m; i0 += kRowsMaxM) {
+        const int mi = (m - i0) < kRowsMaxM ? (m - i0) : kRowsMaxM;
+        const float* xi = x + static_cast<size_t>(i0) * k;
+        float* yi = y + static_cast<size_t>(i0) * n;
+        switch (mi) {
+            case 1: launch_rows<1>(plan, w, xi, yi, n, k, stream); break;
+            case 2: launch_rows<2>(plan, w, xi, yi, n, k, stream); break;
+            case 3: launch_rows<3>(plan, w, xi, yi, n, k, stream); break;
+            case 4: launch_rows<4>(plan, w, xi, yi, n, k, stream); break;
+            case 5: launch_rows<5>(plan, w, xi, yi, n, k, stream); break;
+            case 6: launch_rows<6>(plan, w, xi, yi, n, k, stream); break;
+            case 7: launch_rows<7>(plan, w, xi, yi, n, k, stream); break;
+            default: launch_rows<8>(plan, w, xi, yi, n, k, stream); break;
+        }
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_failure(e);
     }
-    const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+    return Q4K_OK;
 }
 
 }  // namespace q4k

@@ -6,8 +6,9 @@
  * is the one the realizar pages launch as `Q4KGemv`, `TiledQ4KGemv`,
  * `ChunkedTiledQ4KGemv`, `MwvQ4KGemv` ("realizar 0.8.5,
  * src/cuda/executor/q4k_gemv_cached.rs": `q4k_gemv_cached`,
- * `q4k_gemv_indexed_async`) and `BatchedQ4KGemv` for up to 8 vectors
- * ("realizar 0.8.5, src/cuda/executor/uses.rs": `batched_q4k_gemv_into`).
+ * `q4k_gemv_indexed_async`) and `BatchedQ4KGemv` for batches of vectors
+ * ("realizar 0.8.5, src/cuda/executor/uses.rs": `batched_q4k_gemv_into`, up
+ * to 8 vectors per kernel, larger batches in tiles).
  * The dequantisation is the one "memra-engine 0.83.1, src/f16_ffi.rs" declares
  * as `memra_q4_K_dequant_f16` (Q4_K 144-byte superblocks to a row-major
  * mirror), here with an f32 target.
@@ -79,7 +80,7 @@ enum q4k_status {
 
 #define Q4K_QK 256          /* weights per superblock */
 #define Q4K_BLOCK_BYTES 144 /* bytes per superblock   */
-#define Q4K_MAX_M 8         /* most vectors per q4k_gemv call */
+#define Q4K_MAX_M 64        /* most vectors per q4k_gemv call */
 
 /*
  * y = W x for m vectors.
@@ -89,9 +90,13 @@ enum q4k_status {
  *        ("input: M x K row-major", `batched_q4k_gemv_into`).
  *   y  : m x N float32, row-major (vector i at y + i*N); fully overwritten,
  *        never accumulated into ("output: M x N row-major").
- *   m  : 1..8 vectors. Larger m is refused, not looped (the turbospark page,
- *        "turbospark-runtime 0.1.0, src/real_forward_dispatch.rs",
- *        `encode_gemm_any`, refuses rather than silently looping).
+ *   m  : 1..64 vectors. Batches run as kernels over tiles of the vectors (the
+ *        realizar page tiles m > 8 in `batched_q4k_gemv_into`): pairs on the
+ *        streaming kernel, eights on the general one; q4k_gemv_plan_for
+ *        reports the launch count. Larger m is refused, not looped (the
+ *        turbospark page, "turbospark-runtime 0.1.0,
+ *        src/real_forward_dispatch.rs", `encode_gemm_any`, refuses rather than
+ *        silently looping): that is a GEMM's size.
  * Accuracy: per element |y - sum_k w_nk x_ik| <= 1e-4 * sum_k |w_nk x_ik| + 1e-6,
  * where w_nk is the f32 value d*sc*q - dmin*m; accumulation is in f32.
  * Weight reads may start before the previous kernel on `stream` has finished
@@ -191,7 +196,8 @@ typedef struct q4k_gemv_plan {
 } q4k_gemv_plan;
 
 enum q4k_kernel {
-    Q4K_KERNEL_WARP_ROWS = 1,   /* any K, m <= 8: one warp per row, loads via L1  */
+    Q4K_KERNEL_WARP_ROWS = 1,   /* any K: one warp per row, loads via L1; m > 8
+                                   runs as ceil(m/8) launches on vector tiles   */
     Q4K_KERNEL_STREAM = 2       /* K <= 20480 (m = 1) / 15360 (m >= 2); m > 2 runs
                                    as ceil(m/2) launches on vector pairs;
                                    bulk-copy streamed rows, x held in registers,

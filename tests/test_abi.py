@@ -61,7 +61,7 @@ A16 = 1 << 20  # a 16-byte-aligned fake address; never dereferenced
     ((A16, A16 * 2, A16 * 3, 1, 0, 256), q4k.Q4K_ERR_SHAPE),
     ((A16, A16 * 2, A16 * 3, 1, -3, 256), q4k.Q4K_ERR_SHAPE),
     ((A16, A16 * 2, A16 * 3, 0, 4, 256), q4k.Q4K_ERR_UNSUPPORTED_M),
-    ((A16, A16 * 2, A16 * 3, 9, 4, 256), q4k.Q4K_ERR_UNSUPPORTED_M),
+    ((A16, A16 * 2, A16 * 3, 65, 4, 256), q4k.Q4K_ERR_UNSUPPORTED_M),
     ((A16 + 8, A16 * 2, A16 * 3, 1, 4, 256), q4k.Q4K_ERR_ALIGN),
     ((A16, A16 * 2 + 4, A16 * 3, 1, 4, 256), q4k.Q4K_ERR_ALIGN),
     ((A16, A16 * 2, A16 * 3 + 2, 1, 4, 256), q4k.Q4K_ERR_ALIGN),

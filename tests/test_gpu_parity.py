@@ -139,6 +139,29 @@ def test_gemv_multivector_shapes(q4k, n, k, m):
     assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
 
 
+@pytest.mark.parametrize("m", [9, 12, 16, 17, 32, 64])
+@pytest.mark.parametrize("n,k", [(33, 512), (200, 1792), (40, 20736)])
+def test_gemv_batches_beyond_eight(q4k, n, k, m):
+    """m > 8: vector tiles (pairs on the streaming kernel; eights on the general
+    kernel for K = 20736)."""
+    w, x = q4k_synth.q4k_problem(n, k, m, 11 * m + n)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
+
+
+@pytest.mark.parametrize("m", [16, 32])
+@pytest.mark.parametrize("n,k", q4k_synth.SHAPES_MULTIVEC)
+def test_gemv_batched_multivector_shapes_sampled(q4k, n, k, m):
+    """m = 16 and 32 on the multi-vector shapes; the oracle checks 24 sampled rows."""
+    w, x = q4k_synth.q4k_problem(n, k, m, q4k_synth.SEED_MULTIVEC[(n, k)] + m)
+    y = gpu_gemv(q4k, w, x, n, k)
+    rng = np.random.default_rng(m)
+    rows = np.unique(np.concatenate([[0, n - 1], rng.integers(0, n, 22)]))
+    yref, a = oracle.gemv_rows(w, x, n, k, rows)
+    assert_gemv_close(y[:, rows], yref, a, f"{n}x{k} m={m}")
+
+
 def test_gemv_32_layer_sweep_sampled(q4k):
     """All 224 projections of the 32-layer 8B-class decode sweep, each layer's
     weights seeded independently; the oracle checks 8 sampled rows of each."""
@@ -237,7 +260,8 @@ def test_invalid_arguments_on_gpu_enqueue_nothing(q4k):
     wt = torch.zeros(q4k.q4k_weight_bytes(n, k), dtype=torch.uint8, device="cuda")
     xt = torch.zeros(k, dtype=torch.float32, device="cuda")
     y = torch.full((n,), 3.0, device="cuda")
-    assert q4k.q4k_gemv_status(wt, xt, y, 9, n, k) == q4k.Q4K_ERR_UNSUPPORTED_M
+    assert q4k.q4k_gemv_status(wt, xt, y, 65, n, k) == q4k.Q4K_ERR_UNSUPPORTED_M
+    assert q4k.q4k_gemv_status(wt, xt, y, 9, n, k) == q4k.Q4K_ERR_OVERLAP   # x, y hold one vector
     assert q4k.q4k_gemv_status(wt.data_ptr() + 8, xt, y, 1, n, k) == q4k.Q4K_ERR_ALIGN
     assert q4k.q4k_gemv_status(wt, xt, y, 1, n, 500) == q4k.Q4K_ERR_SHAPE
     torch.cuda.synchronize()

@@ -155,3 +155,15 @@ def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
     assert q4k.q4k_gemv_plan_for(2, 64, 15360, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_plan_for(2, 64, 15616, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+
+
+def test_batches_beyond_eight_vectors():
+    """m > 8 runs as vector tiles: pairs on the streaming kernel, eights on the
+    general one (the realizar page tiles batches over 8); m > 64 is refused."""
+    assert q4k.q4k_gemv_plan_for(16, 14336, 4096, SM_COUNT)["launches"] == 8
+    assert q4k.q4k_gemv_plan_for(33, 4096, 4096, SM_COUNT)["launches"] == 17
+    assert q4k.q4k_gemv_plan_for(64, 4096, 4096, SM_COUNT)["launches"] == 32
+    p = q4k.q4k_gemv_plan_for(20, 64, 20736, SM_COUNT)
+    assert p["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS and p["launches"] == 3
+    with pytest.raises(q4k.Q4KError):
+        q4k.q4k_gemv_plan_for(65, 4096, 4096, SM_COUNT)
