@@ -231,6 +231,32 @@ def embed_lookup(table, rows, cols, hidden, token, embed_scale, table_bytes=None
     return default().embed_lookup(table, rows, cols, hidden, token, embed_scale, table_bytes)
 
 
+def swiglu_gemv(w_gate, w_up, x, n, k, nthreads=1):
+    """Fused gate/up GEMV with SwiGLU ("realizar 0.8.5" kernel cache page,
+    `FusedGateUpSwigluHwDp4aQ4KGemv { k: hidden_dim, n: intermediate_dim }`):
+    g = W_gate x and u = W_up x by the oracle GEMV (double), then
+    out = silu(g) * u = g / (1 + exp(-g)) * u in double.
+    Returns (out, g, u, a_g, a_u), all (m, n) float64 (a_*: sums of |w x|)."""
+    g, a_g = gemv(w_gate, x, n, k, nthreads)
+    u, a_u = gemv(w_up, x, n, k, nthreads)
+    with np.errstate(over="ignore"):
+        silu = g / (1.0 + np.exp(-g))
+    return silu * u, g, u, a_g, a_u
+
+
+def swiglu_tolerance(g, u, a_g, a_u, out):
+    """Per-element bound for a GPU SwiGLU GEMV against `swiglu_gemv`. The GPU's
+    g and u each carry the GEMV bound t = 1e-4 * sum|w x| + 1e-6; silu' lies in
+    [-0.1, 1.1], so silu(g) moves by at most 1.1 t_g; the f32 epilogue (exp,
+    divide, multiply) adds a few ulps of the result:
+      1.1 t_g (|u| + t_u) + (|silu(g)| + 1.1 t_g) t_u + 1e-6 |out| + 1e-30."""
+    tg = tolerance(a_g)
+    tu = tolerance(a_u)
+    with np.errstate(over="ignore"):
+        silu = np.abs(g / (1.0 + np.exp(-g)))
+    return 1.1 * tg * (np.abs(u) + tu) + (silu + 1.1 * tg) * tu + 1e-6 * np.abs(out) + 1e-30
+
+
 def tolerance(a: np.ndarray) -> np.ndarray:
     """Per-element GEMV bound |y_gpu - y_ref| <= 1e-4 * sum|w x| + 1e-6."""
     return 1e-4 * np.asarray(a) + 1e-6

@@ -355,10 +355,36 @@ def check_embed_values(o, seed=18):
     assert st == 2 and out is None
 
 
+def check_swiglu_composition(o, seed=19):
+    """SwiGLU GEMV: out = g * expit(g) * u with scipy's logistic function (a
+    library routine), g and u the GEMVs of the two matrices; special cases
+    silu(0) = 0, a zero up-projection gives 0, and silu(g) -> g for large g."""
+    import oracle as oracle_mod
+    from scipy.special import expit
+    saved = oracle_mod._default
+    oracle_mod._default = o
+    try:
+        n, k, m = 21, 768, 3
+        wg, x = q4k_synth.q4k_problem(n, k, m, seed)
+        wu, _ = q4k_synth.q4k_problem(n, k, 1, seed + 1)
+        out, g, u, a_g, a_u = oracle_mod.swiglu_gemv(wg, wu, x, n, k)
+        g2, _ = o.gemv(wg, x, n, k)
+        u2, _ = o.gemv(wu, x, n, k)
+        assert np.array_equal(g, g2) and np.array_equal(u, u2)
+        assert np.allclose(out, g * expit(g) * u, rtol=1e-14, atol=0)
+        zero, *_ = oracle_mod.swiglu_gemv(wg, wu, np.zeros((1, k), np.float32), n, k)
+        assert not zero.any()
+        same, gg, uu, *_ = oracle_mod.swiglu_gemv(wg, wg, 50.0 * x[:1], n, k)
+        big = gg[0] > 40
+        assert big.any() and np.allclose(same[0][big], gg[0][big] ** 2, rtol=1e-15)
+    finally:
+        oracle_mod._default = saved
+
+
 ALL_CHECKS = [
     check_half_all_patterns, check_half_known, check_scale_bit_map, check_nibble_map,
     check_closed_forms, check_pack_roundtrip, check_unpack_pack_bytes, check_bruteforce_gemv,
     check_gemv_vs_matmul, check_unit_and_zero_vectors, check_vectors_independent,
     check_threads_and_rows, check_golden, check_embed_page_cases, check_embed_rules,
-    check_embed_values,
+    check_embed_values, check_swiglu_composition,
 ]
