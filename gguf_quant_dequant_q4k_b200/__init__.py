@@ -1,4 +1,5 @@
-"""GGUF Q4_K GEMV, dequantisation and embedding lookup on one NVIDIA B200 (sm_100a).
+"""GGUF Q4_K GEMV (plain and fused gate/up SwiGLU), dequantisation and embedding
+lookup on one NVIDIA B200 (sm_100a).
 
 The computation runs in libq4k_b200.so (hand-written CUDA, C ABI in
 include/q4k.h); this package is its ctypes binding (`capi`), which takes torch
@@ -12,5 +13,6 @@ from .capi import (  # noqa: F401
     LIB_PATH, Q4KError, q4k_dequant_f32, q4k_dequant_f32_status, q4k_device_fault_flags,
     q4k_embed_gather_f32, q4k_embed_gather_f32_status, q4k_embed_lookup_f32,
     q4k_embed_lookup_f32_status, q4k_gemv, q4k_gemv_plan_for, q4k_gemv_status,
+    q4k_gemv_swiglu, q4k_gemv_swiglu_plan_for, q4k_gemv_swiglu_status,
     q4k_last_cuda_error, q4k_status_string, q4k_weight_bytes,
 )

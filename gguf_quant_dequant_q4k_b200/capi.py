@@ -32,7 +32,8 @@ Q4K_KERNEL_STREAM = 2
 # Every function include/q4k.h declares.
 EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
            "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags",
-           "q4k_embed_lookup_f32", "q4k_embed_gather_f32")
+           "q4k_embed_lookup_f32", "q4k_embed_gather_f32", "q4k_gemv_swiglu",
+           "q4k_gemv_swiglu_plan_for")
 
 
 class Q4KError(RuntimeError):
@@ -76,6 +77,12 @@ _lib.q4k_gemv_plan_for.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, cty
 _lib.q4k_gemv_plan_for.restype = ctypes.c_int
 _lib.q4k_device_fault_flags.argtypes = [ctypes.POINTER(ctypes.c_uint)]
 _lib.q4k_device_fault_flags.restype = ctypes.c_int
+_lib.q4k_gemv_swiglu.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                 _vp]
+_lib.q4k_gemv_swiglu.restype = ctypes.c_int
+_lib.q4k_gemv_swiglu_plan_for.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.POINTER(q4k_gemv_plan)]
+_lib.q4k_gemv_swiglu_plan_for.restype = ctypes.c_int
 _lib.q4k_embed_lookup_f32.argtypes = [_vp, ctypes.c_ulonglong, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_uint, ctypes.c_float, _vp, _vp]
 _lib.q4k_embed_lookup_f32.restype = ctypes.c_int
@@ -125,6 +132,14 @@ def q4k_gemv_plan_for(m: int, n: int, k: int, num_sms: int) -> dict:
     return plan.as_dict()
 
 
+def q4k_gemv_swiglu_plan_for(m: int, n: int, k: int, num_sms: int) -> dict:
+    plan = q4k_gemv_plan()
+    st = _lib.q4k_gemv_swiglu_plan_for(int(m), int(n), int(k), int(num_sms), ctypes.byref(plan))
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_gemv_swiglu_plan_for")
+    return plan.as_dict()
+
+
 def q4k_device_fault_flags() -> int:
     """Reads and clears the current device's kernel fault flags (synchronises)."""
     v = ctypes.c_uint(0)
@@ -144,6 +159,18 @@ def q4k_gemv(w, x, y, m: int, n: int, k: int, stream=None) -> None:
     st = q4k_gemv_status(w, x, y, m, n, k, stream)
     if st != Q4K_OK:
         raise Q4KError(st, "q4k_gemv")
+
+
+def q4k_gemv_swiglu_status(w_gate, w_up, x, y, m: int, n: int, k: int, stream=None) -> int:
+    return _lib.q4k_gemv_swiglu(_ptr(w_gate), _ptr(w_up), _ptr(x), _ptr(y), int(m), int(n),
+                                int(k), _stream(stream))
+
+
+def q4k_gemv_swiglu(w_gate, w_up, x, y, m: int, n: int, k: int, stream=None) -> None:
+    """y[m, n] = silu(W_gate x) * (W_up x) on `stream` (default: torch's current stream)."""
+    st = q4k_gemv_swiglu_status(w_gate, w_up, x, y, m, n, k, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_gemv_swiglu")
 
 
 def q4k_dequant_f32_status(w, out, n: int, k: int, stream=None) -> int:

@@ -161,7 +161,7 @@ int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
     if (plan == nullptr) return Q4K_ERR_NULL;
     if (weight_bytes_checked(n, k) == 0 || num_sms <= 0) return Q4K_ERR_SHAPE;
     if (m < 1 || m > Q4K_MAX_M) return Q4K_ERR_UNSUPPORTED_M;
-    return plan_gemv(m, n, k, num_sms, plan);
+    return plan_gemv(m, n, k, num_sms, false, plan);
 }
 
 int q4k_gemv(const void* w, const float* x, float* y, int m, int n, int k,
@@ -177,7 +177,33 @@ int q4k_gemv(const void* w, const float* x, float* y, int m, int n, int k,
     DeviceInfo dev;
     int st = current_device_info(&dev);
     if (st != Q4K_OK) return st;
-    return launch_gemv(dev, w, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
+    return launch_gemv(dev, w, nullptr, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4k_gemv_swiglu_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
+    if (plan == nullptr) return Q4K_ERR_NULL;
+    if (weight_bytes_checked(n, k) == 0 || num_sms <= 0) return Q4K_ERR_SHAPE;
+    if (m < 1 || m > Q4K_MAX_M) return Q4K_ERR_UNSUPPORTED_M;
+    return plan_gemv(m, n, k, num_sms, true, plan);
+}
+
+int q4k_gemv_swiglu(const void* w_gate, const void* w_up, const float* x, float* y, int m, int n,
+                    int k, q4k_stream_t stream) {
+    if (w_gate == nullptr || w_up == nullptr || x == nullptr || y == nullptr) return Q4K_ERR_NULL;
+    const size_t wbytes = weight_bytes_checked(n, k);
+    if (wbytes == 0) return Q4K_ERR_SHAPE;
+    if (m < 1 || m > Q4K_MAX_M) return Q4K_ERR_UNSUPPORTED_M;
+    if (!aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(x, 16) || !aligned(y, 4))
+        return Q4K_ERR_ALIGN;
+    const size_t xbytes = static_cast<size_t>(m) * static_cast<size_t>(k) * sizeof(float);
+    const size_t ybytes = static_cast<size_t>(m) * static_cast<size_t>(n) * sizeof(float);
+    if (overlaps(y, ybytes, w_gate, wbytes) || overlaps(y, ybytes, w_up, wbytes) ||
+        overlaps(y, ybytes, x, xbytes))
+        return Q4K_ERR_OVERLAP;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return launch_gemv(dev, w_gate, w_up, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int q4k_dequant_f32(const void* w, float* out, int n, int k, q4k_stream_t stream) {

@@ -15,6 +15,7 @@
 #include "q4k_internal.h"
 #include "q4k_stream.h"
 #include "q4k_superblock.cuh"
+#include "q4k_swiglu.cuh"
 
 namespace q4k {
 
@@ -23,85 +24,101 @@ namespace {
 constexpr int kRowsThreads = 256;
 constexpr int kRowsMaxM = 8;   // vectors per launch of the general kernel
 
+// Adds row `wr`'s products with the M vectors into acc[i] (lane's share: the
+// superblocks b = sub, sub + 4, ... and quant slice c of each).
 template <int M>
+__device__ __forceinline__ void rows_dot(const uint8_t* __restrict__ wr, const float* __restrict__ x,
+                                         int nsb, int k, int lane, float (&acc)[M]) {
+    const int c = lane & 7, sub = lane >> 3, g = c >> 1, h = c & 1;
+    for (int b = sub; b < nsb; b += 4) {
+        const uint8_t* sb = wr + static_cast<size_t>(b) * kBlockBytes;
+        const Header hd = decode_header(ldg_nc_v4(sb));
+        const uint4 qv = ldg_nc_v4(sb + kQsOffset + 16 * c);
+        float dsc0, dm0, dsc1, dm1;
+        subblock_coeffs(hd, 2 * g, dsc0, dm0);
+        subblock_coeffs(hd, 2 * g + 1, dsc1, dm1);
+        const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
+        float wl[16], wh[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const uint32_t byte = (words[e >> 2] >> (8 * (e & 3))) & 0xFFu;
+            wl[e] = weight_value(dsc0, dm0, byte & 15u);
+            wh[e] = weight_value(dsc1, dm1, byte >> 4);
+        }
+        const int k0 = b * kQK + 64 * g + 16 * h;
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const float4* xl = reinterpret_cast<const float4*>(x + static_cast<size_t>(i) * k + k0);
+            const float4* xh = xl + 8;  // +32 floats
+            float s = acc[i];
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const float4 a = __ldg(xl + v);
+                const float4 bq = __ldg(xh + v);
+                s = fmaf(wl[4 * v + 0], a.x, s);
+                s = fmaf(wl[4 * v + 1], a.y, s);
+                s = fmaf(wl[4 * v + 2], a.z, s);
+                s = fmaf(wl[4 * v + 3], a.w, s);
+                s = fmaf(wh[4 * v + 0], bq.x, s);
+                s = fmaf(wh[4 * v + 1], bq.y, s);
+                s = fmaf(wh[4 * v + 2], bq.z, s);
+                s = fmaf(wh[4 * v + 3], bq.w, s);
+            }
+            acc[i] = s;
+        }
+    }
+}
+
+// FUSED: y = silu(W x) * (W2 x) (the SwiGLU of a gate and an up projection).
+template <int M, bool FUSED>
 __global__ void __launch_bounds__(kRowsThreads)
-q4k_gemv_rows_kernel(const uint8_t* __restrict__ w, const float* __restrict__ x,
-                     float* __restrict__ y, int n, int k) {
+q4k_gemv_rows_kernel(const uint8_t* __restrict__ w, const uint8_t* __restrict__ w2,
+                     const float* __restrict__ x, float* __restrict__ y, int n, int k) {
     const int nsb = k / kQK;
     const int lane = threadIdx.x & 31;
-    const int c = lane & 7, sub = lane >> 3, g = c >> 1, h = c & 1;
     const int warp = (blockIdx.x * kRowsThreads + threadIdx.x) >> 5;
     const int nwarps = gridDim.x * (kRowsThreads / 32);
     for (int row = warp; row < n; row += nwarps) {
-        float acc[M];
+        float acc[M], acc2[M];
 #pragma unroll
-        for (int i = 0; i < M; ++i) acc[i] = 0.f;
-        const uint8_t* wr = w + static_cast<size_t>(row) * nsb * kBlockBytes;
-        for (int b = sub; b < nsb; b += 4) {
-            const uint8_t* sb = wr + static_cast<size_t>(b) * kBlockBytes;
-            const Header hd = decode_header(ldg_nc_v4(sb));
-            const uint4 qv = ldg_nc_v4(sb + kQsOffset + 16 * c);
-            float dsc0, dm0, dsc1, dm1;
-            subblock_coeffs(hd, 2 * g, dsc0, dm0);
-            subblock_coeffs(hd, 2 * g + 1, dsc1, dm1);
-            const uint32_t words[4] = {qv.x, qv.y, qv.z, qv.w};
-            float wl[16], wh[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const uint32_t byte = (words[e >> 2] >> (8 * (e & 3))) & 0xFFu;
-                wl[e] = weight_value(dsc0, dm0, byte & 15u);
-                wh[e] = weight_value(dsc1, dm1, byte >> 4);
-            }
-            const int k0 = b * kQK + 64 * g + 16 * h;
-#pragma unroll
-            for (int i = 0; i < M; ++i) {
-                const float4* xl = reinterpret_cast<const float4*>(x + static_cast<size_t>(i) * k + k0);
-                const float4* xh = xl + 8;  // +32 floats
-                float s = acc[i];
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float4 a = __ldg(xl + v);
-                    const float4 bq = __ldg(xh + v);
-                    s = fmaf(wl[4 * v + 0], a.x, s);
-                    s = fmaf(wl[4 * v + 1], a.y, s);
-                    s = fmaf(wl[4 * v + 2], a.z, s);
-                    s = fmaf(wl[4 * v + 3], a.w, s);
-                    s = fmaf(wh[4 * v + 0], bq.x, s);
-                    s = fmaf(wh[4 * v + 1], bq.y, s);
-                    s = fmaf(wh[4 * v + 2], bq.z, s);
-                    s = fmaf(wh[4 * v + 3], bq.w, s);
-                }
-                acc[i] = s;
-            }
-        }
+        for (int i = 0; i < M; ++i) acc[i] = acc2[i] = 0.f;
+        rows_dot<M>(w + static_cast<size_t>(row) * nsb * kBlockBytes, x, nsb, k, lane, acc);
+        if (FUSED) rows_dot<M>(w2 + static_cast<size_t>(row) * nsb * kBlockBytes, x, nsb, k, lane, acc2);
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            float s = acc[i];
+            float s = acc[i], s2 = acc2[i];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
-            if (lane == 0) y[static_cast<size_t>(i) * n + row] = s;
+            for (int off = 16; off > 0; off >>= 1) {
+                s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
+                if (FUSED) s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, off);
+            }
+            if (lane == 0) y[static_cast<size_t>(i) * n + row] = FUSED ? silu_mul(s, s2) : s;
         }
     }
 }
 
 template <int M>
-void launch_rows(const q4k_gemv_plan& plan, const void* w, const float* x, float* y, int n,
-                 int k, cudaStream_t stream) {
-    q4k_gemv_rows_kernel<M><<<plan.grid, plan.block, 0, stream>>>(
-        static_cast<const uint8_t*>(w), x, y, n, k);
+void launch_rows(const q4k_gemv_plan& plan, const void* w, const void* w2, const float* x,
+                 float* y, int n, int k, cudaStream_t stream) {
+    if (w2 != nullptr)
+        q4k_gemv_rows_kernel<M, true><<<plan.grid, plan.block, 0, stream>>>(
+            static_cast<const uint8_t*>(w), static_cast<const uint8_t*>(w2), x, y, n, k);
+    else
+        q4k_gemv_rows_kernel<M, false><<<plan.grid, plan.block, 0, stream>>>(
+            static_cast<const uint8_t*>(w), nullptr, x, y, n, k);
 }
 
 }  // namespace
 
 int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
-                     q4k_gemv_plan* plan, StreamParams* sp) {
+                     bool fused, q4k_gemv_plan* plan, StreamParams* sp) {
     StreamParams q{};
     int grid = 0, block = 0, smem = 0;
     // m > 2: ceil(m/2) launches of the two-vector streaming kernel on vector
     // pairs (each decoded weight reused for two vectors per pass).
     const int m_launch = m <= kStreamMaxM ? m : kStreamMaxM;
     const int* cl = max_clusters;
-    if (plan_stream(m_launch, n, k, num_sms, max_smem, cl, &q, &grid, &block, &smem)) {
+    if (plan_stream(m_launch, n, k, num_sms, max_smem, cl, fused, &q, &grid, &block, &smem)) {
         plan->kernel = Q4K_KERNEL_STREAM;
         plan->grid = grid;
         plan->block = block;
@@ -133,17 +150,19 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
     return Q4K_OK;
 }
 
-int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
-    return plan_gemv_device(m, n, k, num_sms, kB200SmemOptin, nullptr, plan, nullptr);
+int plan_gemv(int m, int n, int k, int num_sms, bool fused, q4k_gemv_plan* plan) {
+    return plan_gemv_device(m, n, k, num_sms, kB200SmemOptin, nullptr, fused, plan, nullptr);
 }
 
-int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n,
-                int k, cudaStream_t stream) {
+int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const float* x, float* y,
+                int m, int n, int k, cudaStream_t stream) {
     q4k_gemv_plan plan;
     StreamParams sp;
+    const bool fused = w2 != nullptr;
     const int m_launch = m <= kStreamMaxM ? m : kStreamMaxM;
     const int* clusters = dev.max_clusters[m_launch - 1];
-    int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin, clusters, &plan, &sp);
+    int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin, clusters, fused, &plan,
+                              &sp);
     if (st != Q4K_OK) return st;
     if (plan.kernel == Q4K_KERNEL_STREAM) {
         for (int i0 = 0; i0 < m; i0 += m_launch) {
@@ -151,12 +170,13 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, 
             StreamParams spi = sp;
             if (mi != m_launch) {   // the odd last vector runs the one-vector kernel
                 int g = 0, b = 0, sm = 0;
-                plan_stream(mi, n, k, dev.sm_count, dev.max_smem_optin, dev.max_clusters[mi - 1],
-                            &spi, &g, &b, &sm);
-                st = launch_stream(spi, g, b, sm, w, x + static_cast<size_t>(i0) * k,
+                if (!plan_stream(mi, n, k, dev.sm_count, dev.max_smem_optin,
+                                 dev.max_clusters[mi - 1], fused, &spi, &g, &b, &sm))
+                    return Q4K_ERR_SHAPE;   // not reached: fewer vectors never need more
+                st = launch_stream(spi, g, b, sm, w, w2, x + static_cast<size_t>(i0) * k,
                                    y + static_cast<size_t>(i0) * n, mi, stream);
             } else {
-                st = launch_stream(spi, plan.grid, plan.block, plan.smem_bytes, w,
+                st = launch_stream(spi, plan.grid, plan.block, plan.smem_bytes, w, w2,
                                    x + static_cast<size_t>(i0) * k, y + static_cast<size_t>(i0) * n,
                                    mi, stream);
             }
@@ -170,14 +190,14 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, 
         const float* xi = x + static_cast<size_t>(i0) * k;
         float* yi = y + static_cast<size_t>(i0) * n;
         switch (mi) {
-            case 1: launch_rows<1>(plan, w, xi, yi, n, k, stream); break;
-            case 2: launch_rows<2>(plan, w, xi, yi, n, k, stream); break;
-            case 3: launch_rows<3>(plan, w, xi, yi, n, k, stream); break;
-            case 4: launch_rows<4>(plan, w, xi, yi, n, k, stream); break;
-            case 5: launch_rows<5>(plan, w, xi, yi, n, k, stream); break;
-            case 6: launch_rows<6>(plan, w, xi, yi, n, k, stream); break;
-            case 7: launch_rows<7>(plan, w, xi, yi, n, k, stream); break;
-            default: launch_rows<8>(plan, w, xi, yi, n, k, stream); break;
+            case 1: launch_rows<1>(plan, w, w2, xi, yi, n, k, stream); break;
+            case 2: launch_rows<2>(plan, w, w2, xi, yi, n, k, stream); break;
+            case 3: launch_rows<3>(plan, w, w2, xi, yi, n, k, stream); break;
+            case 4: launch_rows<4>(plan, w, w2, xi, yi, n, k, stream); break;
+            case 5: launch_rows<5>(plan, w, w2, xi, yi, n, k, stream); break;
+            case 6: launch_rows<6>(plan, w, w2, xi, yi, n, k, stream); break;
+            case 7: launch_rows<7>(plan, w, w2, xi, yi, n, k, stream); break;
+            default: launch_rows<8>(plan, w, w2, xi, yi, n, k, stream); break;
         }
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_failure(e);

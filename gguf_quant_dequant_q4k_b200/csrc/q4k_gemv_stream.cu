@@ -53,6 +53,7 @@
 #include "q4k_sm100.cuh"
 #include "q4k_stream.h"
 #include "q4k_superblock.cuh"
+#include "q4k_swiglu.cuh"
 
 namespace q4k {
 
@@ -96,10 +97,15 @@ static_assert(sizeof(TeamRange) == kTeamRangeBytes, "team range table entry");
 // computed cluster-relative in 32 bits (a cluster's rows*nsb is far below
 // 2^31 for any matrix whose N*K/256 fits the int arguments); only the cluster
 // origin is 64-bit.
+// FUSED (fused gate/up SwiGLU, cluster = 1): the CTA's rows of the gate
+// matrix followed by the same rows of the up matrix form one virtual range of
+// 2 * rows rows, indexed from 0 (CTA-relative); its teams cut that range.
+template <bool FUSED>
 __device__ __forceinline__ TeamRange team_range(const StreamParams& p, int gteam) {
     const int q = static_cast<int>(blockIdx.x) / p.cluster;
-    const int rows = p.rows_base + (q < p.rows_extra ? 1 : 0);
-    const long long row_begin =
+    const int crows = p.rows_base + (q < p.rows_extra ? 1 : 0);
+    const int rows = FUSED ? 2 * crows : crows;
+    const long long row_begin = FUSED ? 0 :
         static_cast<long long>(q) * p.rows_base + (q < p.rows_extra ? q : p.rows_extra);
     const int L = rows * p.nsb;
     const unsigned nt = static_cast<unsigned>(p.cluster * p.teams);
@@ -125,6 +131,13 @@ __device__ __forceinline__ TeamRange team_range(const StreamParams& p, int gteam
         r.nstages = 0;
     }
     return r;
+}
+
+// First row and row count of the calling CTA's share (cluster = 1).
+__device__ __forceinline__ void cta_rows(const StreamParams& p, long long& row0, int& rows) {
+    const int q = static_cast<int>(blockIdx.x);
+    rows = p.rows_base + (q < p.rows_extra ? 1 : 0);
+    row0 = static_cast<long long>(q) * p.rows_base + (q < p.rows_extra ? q : p.rows_extra);
 }
 
 __device__ __forceinline__ long long seg_begin(const TeamRange& r, int i, int nsb) {
@@ -261,15 +274,23 @@ struct Team {
     float* red;         // [depth][2 phases][team_warps][M][kSeg] warp partials
     uint64_t* full;     // [depth] stage landed (1 arrival + bytes)
     uint64_t* done;     // [depth] stage consumed (team_warps arrivals)
+    long long cta_row0; // fused: the CTA's first row and row count
+    int cta_rows;
 };
 
-template <int M>
+template <int M, bool FUSED>
 __device__ __forceinline__ Team make_team(const StreamParams& p, uint8_t* smem, int team) {
     Team t;
+    if (FUSED) {
+        cta_rows(p, t.cta_row0, t.cta_rows);
+    } else {
+        t.cta_row0 = 0;
+        t.cta_rows = 0;
+    }
     t.tr = reinterpret_cast<const TeamRange*>(smem + p.off_tr)[cta_rank(p) * p.teams + team];
     t.head0 = static_cast<int>(t.tr.s0 - t.tr.row0 * p.nsb);
     t.team_len = static_cast<int>(t.tr.s1 - t.tr.s0);
-    t.w = p.w + t.tr.s0 * kBlockBytes;
+    t.w = FUSED ? p.w : p.w + t.tr.s0 * kBlockBytes;
     t.ring = smem + static_cast<size_t>(team) * p.depth * p.stage_bytes;
     t.red = reinterpret_cast<float*>(smem + p.off_red) +
             static_cast<size_t>(team) * p.depth * 2 * p.team_warps * kSeg * M;
@@ -278,19 +299,48 @@ __device__ __forceinline__ Team make_team(const StreamParams& p, uint8_t* smem, 
     return t;
 }
 
-// Stage with first row start rb (team-relative) -> one bulk copy into `slot`.
+// Stage with first row start rb (team-relative) -> one bulk copy into `slot`;
+// FUSED: two copies where the stage crosses from gate rows into up rows.
+template <bool FUSED>
 __device__ __forceinline__ void issue_stage(const Team& T, const StreamParams& p, int rb, int slot) {
     const int span = kSeg * p.nsb;
     const int b_rel = rb > 0 ? rb : 0;
     const int e_rel = (rb + span) < T.team_len ? (rb + span) : T.team_len;
     const uint32_t bytes = static_cast<uint32_t>(e_rel - b_rel) * kBlockBytes;
     mbar_arrive_expect_tx(&T.full[slot], bytes);
-    bulk_copy_g2s(T.ring + static_cast<size_t>(slot) * p.stage_bytes,
-                  T.w + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &T.full[slot]);
+    uint8_t* dst = T.ring + static_cast<size_t>(slot) * p.stage_bytes;
+    if (!FUSED) {
+        bulk_copy_g2s(dst, T.w + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &T.full[slot]);
+        return;
+    }
+    long long vs = T.tr.s0 + b_rel;                               // virtual, CTA-relative
+    const long long ve = T.tr.s0 + e_rel;
+    const long long bound = static_cast<long long>(T.cta_rows) * p.nsb;   // gate | up
+    const long long base = T.cta_row0 * p.nsb;
+    if (vs < bound) {
+        const long long e1 = ve < bound ? ve : bound;
+        const uint32_t nb = static_cast<uint32_t>(e1 - vs) * kBlockBytes;
+        bulk_copy_g2s(dst, p.w + static_cast<size_t>(base + vs) * kBlockBytes, nb, &T.full[slot]);
+        dst += nb;
+        vs = e1;
+    }
+    if (vs < ve)
+        bulk_copy_g2s(dst, p.w_up + static_cast<size_t>(base + vs - bound) * kBlockBytes,
+                      static_cast<uint32_t>(ve - vs) * kBlockBytes, &T.full[slot]);
+}
+
+// Where a finished row total goes: y, or (FUSED) the CTA's row-total buffer,
+// gate rows at 0..rows-1 and up rows at rows..2*rows-1 (virtual row index).
+template <bool FUSED>
+__device__ __forceinline__ float& row_out_ref(const StreamParams& p, uint8_t* smem, int i,
+                                              long long row) {
+    if (FUSED)
+        return reinterpret_cast<float*>(smem + p.off_rows)[static_cast<size_t>(i) * 2 * p.rows_cap + row];
+    return p.y[static_cast<size_t>(i) * p.n + row];
 }
 
 // M vectors, S 16-byte quant slices (S*32 weights) per lane per row.
-template <int M, int S>
+template <int M, int S, bool FUSED>
 __global__ void __maxnreg__(stream_max_regs(M))
 q4k_gemv_stream_kernel(const StreamParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -317,7 +367,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         if (i < p.teams * 2 * M) part[i] = 0.f;
         // superblock ranges of every team of the cluster (64-bit divisions once)
         if (i < p.cluster * p.teams)
-            reinterpret_cast<TeamRange*>(smem + p.off_tr)[i] = team_range(p, i);
+            reinterpret_cast<TeamRange*>(smem + p.off_tr)[i] = team_range<FUSED>(p, i);
     }
     __syncthreads();
 
@@ -330,11 +380,11 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         Team T;
         int nst = 0;
         if (own) {
-            T = make_team<M>(p, smem, lane);
+            T = make_team<M, FUSED>(p, smem, lane);
             nst = T.tr.nstages;
             const int all = nst < p.depth ? nst : p.depth;
             const int pre = all < kStreamPreStages ? all : kStreamPreStages;
-            for (int s = 0; s < pre; ++s) issue_stage(T, p, s * kSeg * nsb - T.head0, s);
+            for (int s = 0; s < pre; ++s) issue_stage<FUSED>(T, p, s * kSeg * nsb - T.head0, s);
         }
         pdl_launch_dependents();
         pdl_wait();
@@ -343,7 +393,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         if (own) {
             const int all = nst < p.depth ? nst : p.depth;
             const int pre = all < kStreamPreStages ? all : kStreamPreStages;
-            for (int s = pre; s < all; ++s) issue_stage(T, p, s * kSeg * nsb - T.head0, s);
+            for (int s = pre; s < all; ++s) issue_stage<FUSED>(T, p, s * kSeg * nsb - T.head0, s);
         }
         int tf = 0, fslot = 0;
         uint32_t fphase = 0;
@@ -358,7 +408,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 // Refill the drained slot at once: its quant bytes are consumed,
                 // and its partial sums sit in the (slot, phase) half of the
                 // team's buffer, which the refilled stage does not write.
-                if (tf + p.depth < nst) issue_stage(T, p, rbf + p.depth * kSeg * nsb, fslot);
+                if (tf + p.depth < nst) issue_stage<FUSED>(T, p, rbf + p.depth * kSeg * nsb, fslot);
                 const float* rbuf = T.red + static_cast<size_t>(fslot * 2 + fphase) * red_slot;
 #pragma unroll
                 for (int u = 0; u < kSeg; ++u) {
@@ -373,7 +423,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                         for (int wi = 0; wi < p.team_warps; ++wi)
                             tot += rbuf[(wi * M + i) * kSeg + u];
                         if (b == 0 && e == nsb)
-                            p.y[static_cast<size_t>(i) * p.n + row] = tot;
+                            row_out_ref<FUSED>(p, smem, i, row) = tot;
                         else
                             part[(lane * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
                     }
@@ -404,7 +454,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         // ------------------------------------------------------------ compute
         const int team = warp / p.team_warps;
         const int wit = warp % p.team_warps;
-        const Team T = make_team<M>(p, smem, team);
+        const Team T = make_team<M, FUSED>(p, smem, team);
         pdl_launch_dependents();
         pdl_wait();   // x and y belong to the dependency chain
 
@@ -609,12 +659,25 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < M; ++i) p.y[static_cast<size_t>(i) * p.n + last] = tot[i];
+                for (int i = 0; i < M; ++i) row_out_ref<FUSED>(p, smem, i, last) = tot[i];
             }
         }
     }
     // Keep this CTA's shared memory alive until the cluster has read it.
     if (p.cluster > 1) cluster_sync();
+    if (FUSED) {
+        // SwiGLU epilogue: y = silu(gate row total) * (up row total).
+        __syncthreads();
+        long long row0;
+        int rows;
+        cta_rows(p, row0, rows);
+        const float* tot = reinterpret_cast<const float*>(smem + p.off_rows);
+        for (int v = static_cast<int>(threadIdx.x); v < rows * M; v += static_cast<int>(blockDim.x)) {
+            const int i = v / rows, r = v - i * rows;
+            const float* ti = tot + static_cast<size_t>(i) * 2 * p.rows_cap;
+            p.y[static_cast<size_t>(i) * p.n + row0 + r] = silu_mul(ti[r], ti[rows + r]);
+        }
+    }
 }
 
 }  // namespace
@@ -630,7 +693,7 @@ int resident_clusters(int c, int num_sms, const int* max_clusters) {
 }  // namespace
 
 int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
-                StreamParams* sp, int* grid, int* block, int* smem_bytes) {
+                bool fused, StreamParams* sp, int* grid, int* block, int* smem_bytes) {
     const int nsb = k / kQK;
     if (m < 1 || m > kStreamMaxM || nsb > kStreamMaxNsb || n < 1) return 0;
     const int sl = stream_slices(m);                     // quant slices per lane
@@ -648,14 +711,19 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     int cluster = 1;
     int clusters = n < resident_clusters(1, num_sms, max_clusters)
                        ? n : resident_clusters(1, num_sms, max_clusters);
-    if (n < kClusterMaxRows && nsb >= kClusterMinNsb &&
+    if (!fused && n < kClusterMaxRows && nsb >= kClusterMinNsb &&
         resident_clusters(2, num_sms, max_clusters) >= n) {
         cluster = 2;
         clusters = n;
     }
     const int ctas = clusters * cluster;
     const int stage_bytes = ((kSeg * nsb * kBlockBytes) + 127) / 128 * 128;
-    const int budget = (max_smem < kStreamSmemBudget ? max_smem : kStreamSmemBudget) - 1024;
+    // fused: gate and up row totals of the CTA's rows, [m][2 * rows_cap] floats
+    const int rows_cap = (n + clusters - 1) / clusters;
+    const long long rows_bytes = fused ? (static_cast<long long>(m) * 2 * rows_cap * 4 + 15) / 16 * 16 : 0;
+    if (rows_bytes > kStreamMaxRowsBytes) return 0;
+    const int budget = (max_smem < kStreamSmemBudget ? max_smem : kStreamSmemBudget) - 1024 -
+                       static_cast<int>(rows_bytes);
     // bytes per team besides its ring: coefficient buffers of its warps, the
     // partial sums per slot and ring phase, its cut-row partials, its entries of the cluster's
     // team-range table and two barriers per slot
@@ -698,6 +766,9 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     off += static_cast<size_t>(cluster) * teams * kTeamRangeBytes;
     q.off_bar = static_cast<int>(off);
     off += static_cast<size_t>(teams) * 2 * depth * 8;
+    q.off_rows = static_cast<int>(off);
+    q.rows_cap = fused ? rows_cap : 0;
+    off += static_cast<size_t>(rows_bytes);
     *sp = q;
     *grid = ctas;
     *block = teams * team_warps * 32 + 32;   // + the producer warp
@@ -706,9 +777,10 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
 }
 
 int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, const void* w,
-                  const float* x, float* y, int m, cudaStream_t stream) {
+                  const void* w_up, const float* x, float* y, int m, cudaStream_t stream) {
     StreamParams sp = sp0;
     sp.w = static_cast<const uint8_t*>(w);
+    sp.w_up = static_cast<const uint8_t*>(w_up);
     sp.x = x;
     sp.y = y;
     cudaLaunchConfig_t cfg{};
@@ -726,20 +798,28 @@ int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, 
     cfg.attrs = attr;
     cfg.numAttrs = sp.cluster > 1 ? 2 : 1;
     cudaError_t e;
-    if (m == 1) {
-        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, stream_slices(1)>, sp);
+    if (w_up != nullptr) {
+        e = (m == 1) ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, stream_slices(1), true>, sp)
+                     : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, stream_slices(2), true>, sp);
     } else {
-        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, stream_slices(2)>, sp);
+        e = (m == 1) ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, stream_slices(1), false>, sp)
+                     : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, stream_slices(2), false>, sp);
     }
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
 
 int stream_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, stream_slices(1)>,
+    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, stream_slices(1), false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kStreamSmemBudget);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, stream_slices(2)>,
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, stream_slices(2), false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, stream_slices(1), true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, stream_slices(2), true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
@@ -764,8 +844,8 @@ int stream_cluster_occupancy(int m, int* max_clusters) {
         cfg.numAttrs = 1;
         int count = 0;
         const cudaError_t e = (m == 1)
-            ? cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<1, stream_slices(1)>, &cfg)
-            : cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<2, stream_slices(2)>, &cfg);
+            ? cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<1, stream_slices(1), false>, &cfg)
+            : cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<2, stream_slices(2), false>, &cfg);
         if (e != cudaSuccess) {
             cudaGetLastError();   // the query is advisory; clear the error
             count = 0;

@@ -26,12 +26,13 @@ int q4k_last_cuda_error_value();
 // host-only planner when no device is queried.
 constexpr int kB200SmemOptin = 232448;
 
-// Host-only launch planning (no CUDA calls).
-int plan_gemv(int m, int n, int k, int num_sms, q4k_gemv_plan* plan);
+// Host-only launch planning (no CUDA calls); fused: gate/up SwiGLU.
+int plan_gemv(int m, int n, int k, int num_sms, bool fused, q4k_gemv_plan* plan);
 
-// Enqueue the planned kernels on the current device. Arguments are already validated.
-int launch_gemv(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n,
-                int k, cudaStream_t stream);
+// Enqueue the planned kernels on the current device. Arguments are already
+// validated. w2 != null: y = silu(W x) * (W2 x) (fused gate/up SwiGLU).
+int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const float* x, float* y,
+                int m, int n, int k, cudaStream_t stream);
 
 int launch_dequant(const void* w, float* out, int n, int k, int num_sms, cudaStream_t stream);
 

@@ -26,6 +26,8 @@ constexpr int kStreamMaxNsb = 80;       // K <= 20480 (m = 1) / 15360 (m = 2): o
 constexpr int kStreamMaxTeams = 20;     // one producer lane per team
 constexpr int kStreamMaxDepth = 8;
 constexpr int kStreamSmemBudget = 220 * 1024;
+// Fused SwiGLU: most shared memory for the CTA's gate/up row totals.
+constexpr int kStreamMaxRowsBytes = 32 * 1024;
 // Ring stages each team requests before waiting on the preceding kernel (at
 // most the ring depth); the rest follow once every compute warp has issued its
 // x loads, so x is not queued behind them.
@@ -35,6 +37,7 @@ constexpr int kTeamRangeBytes = 32;
 
 struct StreamParams {
     const uint8_t* w;
+    const uint8_t* w_up;        // fused SwiGLU: the up projection (w is the gate)
     const float* x;
     float* y;
     int n, k, nsb;
@@ -43,6 +46,7 @@ struct StreamParams {
     int teams, team_warps, depth;
     int stage_bytes;            // bytes per ring slot
     int off_coef, off_red, off_part, off_tr, off_bar;  // shared-memory offsets (bytes)
+    int off_rows, rows_cap;     // fused: row totals [M][2 * rows_cap] (gate rows, up rows)
 };
 
 constexpr int kStreamMaxCluster = 8;    // cluster sizes the kernel supports (portable limit)
@@ -50,18 +54,20 @@ constexpr int kClusterMaxRows = 8;      // split rows across a cluster only for 
 constexpr int kClusterMinNsb = 32;      // ... and K >= 8192
 
 // Fills the launch configuration; returns 0 if the streaming kernel does not
-// handle (m, k) or the shared-memory budget cannot hold two stages.
+// handle (m, k) or the shared-memory budget cannot hold two stages. fused:
+// gate and up rows of a CTA share its teams (no cluster split).
 // max_clusters[c] (c = 1..8, may be null) is how many clusters of c CTAs can
 // be resident at once; without it the planner assumes num_sms / c.
 int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
-                StreamParams* sp, int* grid, int* block, int* smem_bytes);
+                bool fused, StreamParams* sp, int* grid, int* block, int* smem_bytes);
 
 // Resident clusters of c CTAs (c = 1..8) for the streaming kernel on the
 // current device, into max_clusters[c]; 0 where the query is not possible.
 int stream_cluster_occupancy(int m, int* max_clusters);
 
+// w_up != null: fused gate/up SwiGLU (w is the gate projection).
 int launch_stream(const StreamParams& sp, int grid, int block, int smem_bytes, const void* w,
-                  const float* x, float* y, int m, cudaStream_t stream);
+                  const void* w_up, const float* x, float* y, int m, cudaStream_t stream);
 
 // Per-device kernel attributes (dynamic shared memory opt-in).
 int stream_set_attributes();

@@ -109,6 +109,27 @@ Q4K_API int q4k_gemv(const void *w, const float *x, float *y, int m, int n, int 
              q4k_stream_t stream);
 
 /*
+ * Fused gate/up projection with SwiGLU: y = silu(W_gate x) * (W_up x), where
+ * silu(g) = g / (1 + exp(-g)), for m vectors ("realizar 0.8.5" kernel cache
+ * page: `FusedGateUpSwigluHwDp4aQ4KGemv { k: hidden_dim, n: intermediate_dim }`;
+ * here with f32 x and the exact per-weight dequantisation of q4k_gemv).
+ *   w_gate, w_up: two N x K Q4_K matrices laid out as w of q4k_gemv, each
+ *        16-byte aligned (they may be the same matrix).
+ *   x, y, m, n, k: as for q4k_gemv (y is m x N, fully overwritten).
+ * One pass streams both matrices and shares each x load between them; g and u
+ * are never written to memory.
+ * Accuracy: with t_g, t_u the q4k_gemv bounds of the two projections (t =
+ * 1e-4 * sum|w x| + 1e-6), per element
+ *   |y - silu(g) u| <= 1.1 t_g (|u| + t_u) + (|silu(g)| + 1.1 t_g) t_u + 1e-6 |y|
+ * (silu' lies in [-0.1, 1.1]; the last term is the f32 epilogue: expf, one
+ * divide, one multiply).
+ * Validation as q4k_gemv; y must not overlap either matrix or x.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_gemv_swiglu(const void *w_gate, const void *w_up, const float *x, float *y,
+                            int m, int n, int k, q4k_stream_t stream);
+
+/*
  * out = W dequantised to float32, row-major n x k (out[r*k + t] is weight t of
  * row r). Each value is d*sc*q - dmin*m rounded once to f32 (the products are
  * exact in f32), so results are bit-reproducible.
@@ -194,6 +215,10 @@ typedef struct q4k_gemv_plan {
     long long units;     /* output rows shared out among the CTAs               */
     long long units_per_cta_max; /* most rows any cluster (CTA if cluster = 1) owns */
 } q4k_gemv_plan;
+
+/* As q4k_gemv_plan_for, for q4k_gemv_swiglu (both matrices share one pass;
+ * `units` counts output rows, each the pair of a gate and an up row). */
+Q4K_API int q4k_gemv_swiglu_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan *plan);
 
 enum q4k_kernel {
     Q4K_KERNEL_WARP_ROWS = 1,   /* any K: one warp per row, loads via L1; m > 8

@@ -167,3 +167,82 @@ def test_batches_beyond_eight_vectors():
     assert p["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS and p["launches"] == 3
     with pytest.raises(q4k.Q4KError):
         q4k.q4k_gemv_plan_for(65, 4096, 4096, SM_COUNT)
+
+
+def check_fused_plan(m, n, k):
+    """Fused gate/up SwiGLU: each CTA's gate rows followed by the same up rows
+    form a virtual range of 2*rows rows that its teams cut; a stage crossing
+    from gate into up rows is two copies. Checks: every virtual superblock is
+    streamed once, every copy stays inside the CTA's rows of its matrix and is
+    a multiple of 16 bytes, every virtual row is finished exactly once, and
+    shared memory (with the row-total buffer) fits."""
+    p = q4k.q4k_gemv_swiglu_plan_for(m, n, k, SM_COUNT)
+    if p["kernel"] != q4k.Q4K_KERNEL_STREAM:
+        return p
+    nsb = k // 256
+    ctas, teams, depth = p["grid"], p["teams"], p["depth"]
+    assert p["cluster"] == 1 and ctas == min(n, SM_COUNT)
+    team_warps = -(-nsb * 8 // 32)
+    assert p["block"] == teams * team_warps * 32 + 32
+    stage_bytes = -(-SEG * nsb * 144 // 128) * 128
+    rows_cap = -(-n // ctas)
+    mi = min(m, 2)
+    need = (teams * depth * stage_bytes + teams * team_warps * SEG * 4 * 4 * 16
+            + teams * depth * 2 * team_warps * SEG * mi * 4 + teams * 2 * mi * 4)
+    need = -(-need // 16) * 16 + teams * 32 + teams * 2 * depth * 8
+    need += -(-(mi * 2 * rows_cap * 4) // 16) * 16
+    assert p["smem_bytes"] == need and need <= 220 * 1024 - 1024
+    base, extra = n // ctas, n % ctas
+    gate_seen = [0] * (n * nsb)
+    up_seen = [0] * (n * nsb)
+    for q in range(ctas):
+        rows = base + (1 if q < extra else 0)
+        row0 = q * base + min(q, extra)
+        L = 2 * rows * nsb
+        bound = rows * nsb
+        writes = [0] * (2 * rows)
+        ranges = []
+        for t in range(teams):
+            s0, s1 = L * t // teams, L * (t + 1) // teams
+            ranges.append((s0, s1))
+        for t, (s0, s1) in enumerate(ranges):
+            if s1 <= s0:
+                continue
+            rbase = s0 // nsb
+            nseg = (s1 - 1) // nsb - rbase + 1
+            for st in range(-(-nseg // SEG)):
+                vs = max(s0, (rbase + st * SEG) * nsb)
+                ve = min(s1, (rbase + st * SEG + SEG) * nsb)
+                assert 0 < (ve - vs) * 144 <= stage_bytes
+                pieces = []
+                if vs < bound:
+                    pieces.append(("gate", vs, min(ve, bound)))
+                if ve > bound:
+                    pieces.append(("up", max(vs, bound) - bound, ve - bound))
+                for which, a, b in pieces:
+                    assert 0 <= a < b <= rows * nsb and ((b - a) * 144) % 16 == 0
+                    seen = gate_seen if which == "gate" else up_seen
+                    for sb in range(a, b):
+                        seen[row0 * nsb + sb] += 1
+            for i in range(nseg):
+                v = rbase + i
+                b_, e_ = max(s0, v * nsb) - v * nsb, min(s1, (v + 1) * nsb) - v * nsb
+                if b_ == 0 and e_ == nsb:
+                    writes[v] += 1
+                elif b_ == 0:          # this team holds the row's first superblock
+                    writes[v] += 1
+        assert all(w == 1 for w in writes), (q, writes)
+    assert all(c == 1 for c in gate_seen) and all(c == 1 for c in up_seen)
+    return p
+
+
+@pytest.mark.parametrize("n,k", [(14336, 4096), (11008, 4096), (8960, 1536), (1, 256), (3, 4096),
+                                 (149, 1024), (300, 3840), (1000, 20480), (7, 14336)])
+@pytest.mark.parametrize("m", [1, 2, 3])
+def test_fused_partition(m, n, k):
+    check_fused_plan(m, n, k)
+
+
+def test_fused_falls_back_beyond_the_stream_range():
+    assert q4k.q4k_gemv_swiglu_plan_for(1, 64, 20736, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    assert q4k.q4k_gemv_swiglu_plan_for(1, 7, 14336, SM_COUNT)["cluster"] == 1
