@@ -275,7 +275,55 @@ def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
     del g, layers
     torch.cuda.empty_cache()
     out["embedding"] = embedding_workloads(q4k, torch, dev, stream)
+    out["swiglu"] = swiglu_workloads(q4k, torch, dev, stream, l2)
     return out
+
+
+def swiglu_workloads(q4k, torch, dev, stream, l2: int) -> list:
+    """Fused gate/up SwiGLU (q4k_gemv_swiglu) on the 7B and 8B FFN shapes, m = 1
+    and 2, against the same work as two q4k_gemv calls (the fused call also does
+    the SwiGLU, which the separate pair leaves undone). Bytes counted per call =
+    both matrices + x once + y once."""
+    res = []
+    for n, k in ((11008, 4096), (14336, 4096)):
+        wg, _ = q4k_synth.q4k_problem(n, k, 1, 400 + n)
+        wu, _ = q4k_synth.q4k_problem(n, k, 1, 401 + n)
+        copies = max(2, -(-2 * l2 // (2 * wg.nbytes)) + 1)
+        gs = [torch.from_numpy(wg).to(dev) for _ in range(copies)]
+        us = [torch.from_numpy(wu).to(dev) for _ in range(copies)]
+        for m in (1, 2):
+            x = torch.from_numpy(q4k_synth.x_vectors(k, m, 90 + m)).to(dev)
+            y = torch.empty((m, n), dtype=torch.float32, device=dev)
+            y2 = torch.empty((m, n), dtype=torch.float32, device=dev)
+
+            def timed(fn):
+                with torch.cuda.stream(stream):
+                    for i in range(10):
+                        fn(i)
+                a0 = torch.cuda.Event(enable_timing=True)
+                a1 = torch.cuda.Event(enable_timing=True)
+                reps = 100
+                a0.record(stream)
+                for i in range(reps):
+                    fn(i)
+                a1.record(stream)
+                torch.cuda.synchronize(dev)
+                return a0.elapsed_time(a1) * 1e3 / reps
+
+            fused = timed(lambda i: q4k.q4k_gemv_swiglu(gs[i % copies], us[i % copies], x, y, m,
+                                                        n, k, stream=stream))
+
+            def pair(i):
+                q4k.q4k_gemv(gs[i % copies], x, y, m, n, k, stream=stream)
+                q4k.q4k_gemv(us[i % copies], x, y2, m, n, k, stream=stream)
+            separate = timed(pair)
+            b = 2 * n * (k // 256) * 144 + 4 * m * (k + n)
+            res.append({"n": n, "k": k, "m": m, "us_per_call": round(fused, 3),
+                        "gbs": round(b / fused / 1e3, 1),
+                        "two_gemv_calls_us": round(separate, 3)})
+        del gs, us
+    torch.cuda.empty_cache()
+    return res
 
 
 def embedding_workloads(q4k, torch, dev, stream) -> list:
