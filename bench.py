@@ -272,6 +272,40 @@ def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
     out["layer_sweep_32"] = {"launches": len(layers), "bytes": total, "us_per_pass": round(us, 1),
                              "gbs": round(total / us / 1e3, 1),
                              "how": "one CUDA graph of the 224 projection GEMVs, replayed"}
+    del g
+    # The same weights with each layer's gate and up projections as one fused
+    # SwiGLU call (q4k_gemv_swiglu): 6 launches per layer, same bytes.
+    gate_i, up_i = 4, 5
+    assert q4k_synth.LAYER_8B[gate_i] == q4k_synth.LAYER_8B[up_i]
+    def fused_pass():
+        for layer in range(32):
+            base = layer * len(q4k_synth.LAYER_8B)
+            for proj in range(len(q4k_synth.LAYER_8B)):
+                w, x, y, n, k = layers[base + proj]
+                if proj == gate_i:
+                    q4k.q4k_gemv_swiglu(w, layers[base + up_i][0], x, y, 1, n, k, stream=stream)
+                elif proj != up_i:
+                    q4k.q4k_gemv(w, x, y, 1, n, k, stream=stream)
+    with torch.cuda.stream(stream):
+        fused_pass()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fused_pass()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    a0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g.replay()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = a0.elapsed_time(a1) * 1e3 / reps
+    out["layer_sweep_32_fused_gate_up"] = {
+        "launches": 32 * (len(q4k_synth.LAYER_8B) - 1), "bytes": total,
+        "us_per_pass": round(us, 1), "gbs": round(total / us / 1e3, 1),
+        "how": "the same 32 layers, gate and up of each layer as one q4k_gemv_swiglu call"}
     del g, layers
     torch.cuda.empty_cache()
     out["embedding"] = embedding_workloads(q4k, torch, dev, stream)
