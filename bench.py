@@ -405,6 +405,25 @@ def embedding_workloads(q4k, torch, dev, stream) -> list:
 
 # --------------------------------------------------------------------------- our arm
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's figure (max over ranks): a multi-GPU time is the job's
+    time, set by its slowest rank. `device` holds the reduction tensor (the
+    process group's device: a GPU under NCCL, the CPU under gloo)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: int, steps: int, ms: float) -> float:
+    """Bytes all ranks processed / the slowest rank's time, in GB/s (replicas:
+    every rank streams the same step)."""
+    return world * bytes_per_step * steps / (ms * 1e-3) / 1e9
+
+
 def run_ours(args) -> None:
     import torch
     import torch.distributed as dist
@@ -493,13 +512,9 @@ def run_ours(args) -> None:
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler is not None else None
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_per_step = ms / args.steps
-    value = world * BYTES_PER_STEP * args.steps / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(world, BYTES_PER_STEP, args.steps, ms)
 
     # per-projection us/call: R back-to-back calls over rotating copies
     per_shape = []
@@ -552,13 +567,8 @@ def run_ours(args) -> None:
         e2e_step(i)
     b1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = b0.elapsed_time(b1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = (world * BYTES_PER_STEP * e2e_steps / (e2e_ms * 1e-3) / 1e9
-                 if e2e_steps else None)
+    e2e_ms = max_over_ranks(b0.elapsed_time(b1), world, dev)
+    e2e_value = whole_job_gbs(world, BYTES_PER_STEP, e2e_steps, e2e_ms) if e2e_steps else None
 
     if world > 1:
         dist.barrier()
