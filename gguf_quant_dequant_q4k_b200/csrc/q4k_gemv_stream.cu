@@ -1,4 +1,5 @@
-// q4k_gemv_stream.cu -- the streaming Q4_K GEMV for m = 1, 2 and K <= 20480 (m = 1) or 15360 (m = 2).
+// q4k_gemv_stream.cu -- the streaming Q4_K GEMV (plain, or fused gate/up
+// SwiGLU) for m = 1, 2 and K <= 20480 (m = 1) or 15360 (m = 2).
 //
 // What it computes: y[i][r] = sum_k W[r][k] x[i][k] with W in Q4_K, as the
 // pages' `Q4KGemv` / `TiledQ4KGemv` / `ChunkedTiledQ4KGemv` / `MwvQ4KGemv`
@@ -43,6 +44,12 @@
 // * Reduction. Per stage each lane holds one partial per row segment; a
 //   4-segment transpose-reduce across the warp (5 shuffles) leaves one value
 //   per segment, published to shared memory for the producer lane to add.
+// * Fused gate/up SwiGLU (FUSED = true, q4k_gemv_swiglu): a CTA's rows of the
+//   gate matrix followed by the same rows of the up matrix form one virtual
+//   range that its teams cut as above (a stage crossing from gate into up rows
+//   is two copies); row totals go to shared memory, and the CTA finishes with
+//   y = silu(gate total) * (up total) for its rows ("realizar 0.8.5" kernel
+//   cache page: `FusedGateUpSwigluHwDp4aQ4KGemv`).
 //
 // All waits are bounded: a wait that gives up raises a device fault flag
 // (q4k_device_fault_flags) and the kernel skips its remaining work.
