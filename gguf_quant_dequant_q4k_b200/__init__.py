@@ -14,5 +14,5 @@ from .capi import (  # noqa: F401
     q4k_embed_gather_f32, q4k_embed_gather_f32_status, q4k_embed_lookup_f32,
     q4k_embed_lookup_f32_status, q4k_gemv, q4k_gemv_plan_for, q4k_gemv_status,
     q4k_gemv_swiglu, q4k_gemv_swiglu_plan_for, q4k_gemv_swiglu_status,
-    q4k_last_cuda_error, q4k_status_string, q4k_weight_bytes,
+    q4k_last_cuda_error, q4k_selftest_wait_timeout, q4k_status_string, q4k_weight_bytes,
 )

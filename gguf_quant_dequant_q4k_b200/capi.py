@@ -33,7 +33,7 @@ Q4K_KERNEL_STREAM = 2
 EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
            "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags",
            "q4k_embed_lookup_f32", "q4k_embed_gather_f32", "q4k_gemv_swiglu",
-           "q4k_gemv_swiglu_plan_for")
+           "q4k_gemv_swiglu_plan_for", "q4k_selftest_wait_timeout")
 
 
 class Q4KError(RuntimeError):
@@ -83,6 +83,8 @@ _lib.q4k_gemv_swiglu.restype = ctypes.c_int
 _lib.q4k_gemv_swiglu_plan_for.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           ctypes.POINTER(q4k_gemv_plan)]
 _lib.q4k_gemv_swiglu_plan_for.restype = ctypes.c_int
+_lib.q4k_selftest_wait_timeout.argtypes = [_vp]
+_lib.q4k_selftest_wait_timeout.restype = ctypes.c_int
 _lib.q4k_embed_lookup_f32.argtypes = [_vp, ctypes.c_ulonglong, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ctypes.c_uint, ctypes.c_float, _vp, _vp]
 _lib.q4k_embed_lookup_f32.restype = ctypes.c_int
@@ -138,6 +140,13 @@ def q4k_gemv_swiglu_plan_for(m: int, n: int, k: int, num_sms: int) -> dict:
     if st != Q4K_OK:
         raise Q4KError(st, "q4k_gemv_swiglu_plan_for")
     return plan.as_dict()
+
+
+def q4k_selftest_wait_timeout(stream=None) -> None:
+    """Enqueues the bounded-wait self-test kernel (raises Q4K_FAULT_COPY_TIMEOUT)."""
+    st = _lib.q4k_selftest_wait_timeout(_stream(stream))
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_selftest_wait_timeout")
 
 
 def q4k_device_fault_flags() -> int:

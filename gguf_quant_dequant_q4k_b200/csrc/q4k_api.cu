@@ -112,6 +112,13 @@ int q4k_device_fault_flags(unsigned int* flags) {
     return Q4K_OK;
 }
 
+int q4k_selftest_wait_timeout(q4k_stream_t stream) {
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return selftest_wait_timeout(reinterpret_cast<cudaStream_t>(stream));
+}
+
 int q4k_embed_lookup_f32(const void* table, unsigned long long table_bytes, int rows, int cols,
                          int hidden, unsigned int token, float embed_scale, float* out,
                          q4k_stream_t stream) {

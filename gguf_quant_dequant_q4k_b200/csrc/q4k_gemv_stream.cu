@@ -862,6 +862,26 @@ int stream_cluster_occupancy(int m, int* max_clusters) {
     return Q4K_OK;
 }
 
+namespace {
+
+// One thread waits, bounded, on an mbarrier phase that nothing completes: the
+// wait gives up after kSpinLimit tries and raises kFaultCopyTimeout, exactly as
+// a kernel's wait on a lost bulk copy would, then the kernel returns.
+__global__ void q4k_wait_timeout_selftest_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_bounded(&bar, 0u, &g_fault_flags);
+}
+
+}  // namespace
+
+int selftest_wait_timeout(cudaStream_t stream) {
+    q4k_wait_timeout_selftest_kernel<<<1, 1, 0, stream>>>();
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+}
+
 int read_fault_flags(unsigned* flags) {
     unsigned v = 0;
     cudaError_t e = cudaMemcpyFromSymbol(&v, g_fault_flags, sizeof(v));

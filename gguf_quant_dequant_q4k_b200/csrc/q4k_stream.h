@@ -75,4 +75,8 @@ int stream_set_attributes();
 // Reads and clears the device fault flags (synchronises the device).
 int read_fault_flags(unsigned* flags);
 
+// Enqueues a one-thread kernel whose bounded mbarrier wait runs out (nothing
+// completes the phase), raising the copy-timeout fault flag.
+int selftest_wait_timeout(cudaStream_t stream);
+
 }  // namespace q4k

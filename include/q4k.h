@@ -199,6 +199,17 @@ Q4K_API int q4k_embed_gather_f32(const void *table, unsigned long long table_byt
 Q4K_API int q4k_device_fault_flags(unsigned int *flags);
 
 /*
+ * Self-test of the bounded waits: enqueues on `stream` a one-thread kernel
+ * that waits on a shared-memory mbarrier phase nothing completes. The wait
+ * gives up after its bounded number of tries (each try may sleep up to 1 us;
+ * about a second in all), raises Q4K_FAULT_COPY_TIMEOUT and the kernel
+ * returns: the same path a kernel takes when a bulk copy is lost, with the
+ * CUDA context left usable. Read the flag with q4k_device_fault_flags().
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_selftest_wait_timeout(q4k_stream_t stream);
+
+/*
  * How q4k_gemv would run a problem on a B200 with `num_sms` SMs (host-only,
  * no CUDA call). Fills *plan and returns Q4K_OK, or the status q4k_gemv would
  * return for these sizes.
