@@ -50,7 +50,7 @@ class q4k_gemv_plan(ctypes.Structure):
                 ("smem_bytes", ctypes.c_int), ("cluster", ctypes.c_int), ("teams", ctypes.c_int),
                 ("depth", ctypes.c_int),
                 ("launches", ctypes.c_int), ("units", ctypes.c_longlong),
-                ("units_per_cta_max", ctypes.c_longlong)]
+                ("units_per_cta_max", ctypes.c_longlong), ("slices", ctypes.c_int)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}

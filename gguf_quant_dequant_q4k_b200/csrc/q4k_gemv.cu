@@ -129,6 +129,7 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
         plan->cluster = q.cluster;
         plan->units = n;
         plan->units_per_cta_max = q.rows_base + (q.rows_extra > 0 ? 1 : 0);
+        plan->slices = q.slices;
         if (sp) *sp = q;
         return Q4K_OK;
     }
@@ -147,6 +148,7 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
     plan->launches = (m + kRowsMaxM - 1) / kRowsMaxM;   // tiles of up to 8 vectors
     plan->units = n;
     plan->units_per_cta_max = ((n + warps - 1) / warps) * warps_per_cta;
+    plan->slices = 0;
     return Q4K_OK;
 }
 

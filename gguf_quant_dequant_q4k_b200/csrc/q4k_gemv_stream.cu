@@ -75,7 +75,7 @@ constexpr unsigned kXIssuedBarrier = 1;      // named barrier: compute warps iss
 constexpr uint32_t kMagicOne = 0x3F000000u;  // 1/2: bytes 0..2 = 0x00, byte 3 = 0x3F
 constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
 // Coefficient buffer per warp: [segment][position][4 groups] float4s.
-constexpr int coef_bytes_per_warp(int m) { return kSeg * (4 * stream_slices(m)) * 4 * 16; }
+constexpr int coef_bytes_per_warp(int slices) { return kSeg * (4 * slices) * 4 * 16; }
 
 // f = 1/2 + q/256 for the nibble q held in byte SEL of `masked` (bytes 0..15):
 // the byte becomes bits 16..23 of 0x3F000000 (1/2), i.e. mantissa bits 16..19.
@@ -348,7 +348,7 @@ __device__ __forceinline__ float& row_out_ref(const StreamParams& p, uint8_t* sm
 
 // M vectors, S 16-byte quant slices (S*32 weights) per lane per row.
 template <int M, int S, bool FUSED>
-__global__ void __maxnreg__(stream_max_regs(M))
+__global__ void __maxnreg__(stream_max_regs(M, S))
 q4k_gemv_stream_kernel(const StreamParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ volatile int abort_flag;
@@ -703,9 +703,10 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
                 bool fused, StreamParams* sp, int* grid, int* block, int* smem_bytes) {
     const int nsb = k / kQK;
     if (m < 1 || m > kStreamMaxM || nsb > kStreamMaxNsb || n < 1) return 0;
-    const int sl = stream_slices(m);                     // quant slices per lane
+    // quant slices per lane: two for one vector on very tall matrices
+    const int sl = (m == 1 && !fused && (n + num_sms - 1) / num_sms >= kWideMinRows) ? 2 : 1;
     const int team_warps = (nsb * 8 / sl + 31) / 32;   // 8*nsb slices / (32 lanes * sl)
-    const int max_warps = stream_max_threads(m) / 32;
+    const int max_warps = stream_max_threads(m, sl) / 32;
     if (team_warps > max_warps) return 0;
     int teams = max_warps / team_warps;
     if (teams > kStreamMaxTeams) teams = kStreamMaxTeams;
@@ -735,7 +736,7 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     // partial sums per slot and ring phase, its cut-row partials, its entries of the cluster's
     // team-range table and two barriers per slot
     auto fixed_team = [&](int depth) {
-        return team_warps * coef_bytes_per_warp(m) + depth * 2 * team_warps * kSeg * m * 4 +
+        return team_warps * coef_bytes_per_warp(sl) + depth * 2 * team_warps * kSeg * m * 4 +
                2 * m * 4 + cluster * kTeamRangeBytes + 2 * depth * 8 + 16;
     };
     int depth = kStreamMaxDepth;
@@ -761,9 +762,10 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     q.team_warps = team_warps;
     q.depth = depth;
     q.stage_bytes = stage_bytes;
+    q.slices = sl;
     size_t off = static_cast<size_t>(teams) * depth * stage_bytes;
     q.off_coef = static_cast<int>(off);
-    off += static_cast<size_t>(teams) * team_warps * coef_bytes_per_warp(m);
+    off += static_cast<size_t>(teams) * team_warps * coef_bytes_per_warp(sl);
     q.off_red = static_cast<int>(off);
     off += static_cast<size_t>(teams) * depth * 2 * team_warps * kSeg * m * 4;
     q.off_part = static_cast<int>(off);
@@ -806,27 +808,32 @@ int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, 
     cfg.numAttrs = sp.cluster > 1 ? 2 : 1;
     cudaError_t e;
     if (w_up != nullptr) {
-        e = (m == 1) ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, stream_slices(1), true>, sp)
-                     : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, stream_slices(2), true>, sp);
+        e = (m == 1) ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, 1, true>, sp)
+                     : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, 1, true>, sp);
+    } else if (m == 1) {
+        e = sp.slices == 2 ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, 2, false>, sp)
+                           : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, 1, false>, sp);
     } else {
-        e = (m == 1) ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, stream_slices(1), false>, sp)
-                     : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, stream_slices(2), false>, sp);
+        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, 1, false>, sp);
     }
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
 
 int stream_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, stream_slices(1), false>,
+    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, 1, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kStreamSmemBudget);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, stream_slices(2), false>,
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, 2, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, stream_slices(1), true>,
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, 1, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, stream_slices(2), true>,
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<1, 1, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, 1, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
@@ -840,7 +847,7 @@ int stream_cluster_occupancy(int m, int* max_clusters) {
     for (int c = 1; c <= kStreamMaxCluster; c *= 2) {
         cudaLaunchConfig_t cfg{};
         cfg.gridDim = dim3(c);
-        cfg.blockDim = dim3(stream_max_threads(m) + 32);
+        cfg.blockDim = dim3(stream_max_threads(m, 1) + 32);
         cfg.dynamicSmemBytes = kStreamSmemBudget;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -851,8 +858,8 @@ int stream_cluster_occupancy(int m, int* max_clusters) {
         cfg.numAttrs = 1;
         int count = 0;
         const cudaError_t e = (m == 1)
-            ? cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<1, stream_slices(1), false>, &cfg)
-            : cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<2, stream_slices(2), false>, &cfg);
+            ? cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<1, 1, false>, &cfg)
+            : cudaOccupancyMaxActiveClusters(&count, q4k_gemv_stream_kernel<2, 1, false>, &cfg);
         if (e != cudaSuccess) {
             cudaGetLastError();   // the query is advisory; clear the error
             count = 0;

@@ -8,19 +8,22 @@ namespace q4k {
 
 constexpr int kStreamSegRows = 4;       // row segments per ring stage
 constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kernel
-// Quant slices (16 bytes = 32 weights) per lane and row. Measured on B200: one
-// slice per lane with more warps beats two slices with fewer warps on every
-// decode shape but the largest (within 2% there).
-constexpr int stream_slices(int m) { return m == 1 ? 1 : 1; }
-// Compute threads per CTA (plus one producer warp): 20 + 1 warps for one vector
-// (x: 32 registers per lane; up to six warps per sub-partition at 80
-// registers; 23 compute warps measured no faster), 15 + 1 for two (x: 64
-// registers per lane; four warps per sub-partition at 128 registers).
-constexpr int stream_max_threads(int m) { return m == 1 ? 640 : 480; }
+// Quant slices (16 bytes = 32 weights) per lane and row: 1, or 2 for one
+// vector on very tall matrices (kWideMinRows rows or more per CTA: an LM
+// head). Two slices halve the per-item overheads but double the x registers
+// (64 per lane), so fewer warps fit; measured on B200 they win only where a
+// CTA has hundreds of rows to stream (LM head 128256x4096: 96.7 vs 98.7 us)
+// and lose 10-50 % on every decode projection below that.
+constexpr int kWideMinRows = 512;
+// Compute threads per CTA (plus one producer warp): one slice, one vector: 20
+// warps (x: 32 registers per lane; five or six warps per sub-partition at 80
+// registers; 23 measured no faster); two vectors, or two slices: 15 warps (x:
+// 64 registers per lane; four warps per sub-partition at 128 registers).
+constexpr int stream_max_threads(int m, int slices) { return (m == 1 && slices == 1) ? 640 : 480; }
 // Registers per thread: each of the SM's four sub-partitions has 16384
 // registers for its share of the CTA's warps (allocated in multiples of 8).
-constexpr int stream_max_regs(int m) {
-    return 16384 / (((stream_max_threads(m) / 32 + 1 + 3) / 4) * 32) / 8 * 8;
+constexpr int stream_max_regs(int m, int slices) {
+    return 16384 / (((stream_max_threads(m, slices) / 32 + 1 + 3) / 4) * 32) / 8 * 8;
 }
 constexpr int kStreamMaxNsb = 80;       // K <= 20480 (m = 1) / 15360 (m = 2): one team covers K
 constexpr int kStreamMaxTeams = 20;     // one producer lane per team
@@ -47,6 +50,7 @@ struct StreamParams {
     int stage_bytes;            // bytes per ring slot
     int off_coef, off_red, off_part, off_tr, off_bar;  // shared-memory offsets (bytes)
     int off_rows, rows_cap;     // fused: row totals [M][2 * rows_cap] (gate rows, up rows)
+    int slices;                 // 16-byte quant slices per lane (1 or 2)
 };
 
 constexpr int kStreamMaxCluster = 8;    // cluster sizes the kernel supports (portable limit)

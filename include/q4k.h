@@ -225,6 +225,7 @@ typedef struct q4k_gemv_plan {
     int launches;        /* kernels one call enqueues                           */
     long long units;     /* output rows shared out among the CTAs               */
     long long units_per_cta_max; /* most rows any cluster (CTA if cluster = 1) owns */
+    int slices;          /* streaming kernel: 16-byte quant slices per lane (1 or 2) */
 } q4k_gemv_plan;
 
 /* As q4k_gemv_plan_for, for q4k_gemv_swiglu (both matrices share one pass;

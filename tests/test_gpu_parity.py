@@ -139,6 +139,23 @@ def test_gemv_multivector_shapes(q4k, n, k, m):
     assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
 
 
+@pytest.mark.parametrize("n,k", [(75776, 4096), (100000, 20480), (151936, 1536)])
+def test_gemv_tall_two_slices_sampled(q4k, n, k):
+    """Very tall matrices (512 or more rows per CTA) run two quant slices per
+    lane; the oracle checks sampled rows, including every CTA boundary region."""
+    plan = q4k.q4k_gemv_plan_for(1, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert plan["slices"] == 2
+    w, x = q4k_synth.q4k_problem(n, k, 1, 60 + n % 97)
+    y = gpu_gemv(q4k, w, x, n, k)
+    assert np.isfinite(y).all()
+    rng = np.random.default_rng(n)
+    per = -(-n // plan["grid"])
+    edges = np.clip(np.arange(0, n, per)[:, None] + np.array([-1, 0, 1])[None, :], 0, n - 1)
+    rows = np.unique(np.concatenate([edges.reshape(-1)[::7], rng.integers(0, n, 40), [0, n - 1]]))
+    yref, a = oracle.gemv_rows(w, x, n, k, rows)
+    assert_gemv_close(y[:, rows], yref, a, f"{n}x{k}")
+
+
 @pytest.mark.parametrize("m", [9, 12, 16, 17, 32, 64])
 @pytest.mark.parametrize("n,k", [(33, 512), (200, 1792), (40, 20736)])
 def test_gemv_batches_beyond_eight(q4k, n, k, m):

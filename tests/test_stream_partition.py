@@ -50,10 +50,12 @@ def check_plan(m, n, k):
     assert cluster in (1, 2) and ctas % cluster == 0
     clusters = ctas // cluster
     assert clusters <= n
-    slices = 1                                           # 16-byte quant slices per lane
+    slices = p["slices"]                                 # 16-byte quant slices per lane
+    wide = m == 1 and -(-n // SM_COUNT) >= 512           # very tall: two slices
+    assert slices == (2 if wide else 1)
     team_warps = -(-nsb * 8 // slices // 32)
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
-    assert p["block"] <= (640 if m == 1 else 480) + 32
+    assert p["block"] <= (640 if (m == 1 and slices == 1) else 480) + 32
     assert 2 <= depth <= 8 and 1 <= teams <= 20
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     coef_per_warp = SEG * (4 * slices) * 4 * 16    # [seg][positions][4 groups] float4s
@@ -115,7 +117,8 @@ def check_plan(m, n, k):
 
 
 SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
-          + [(4096, 14336), (1024, 4096), (14336, 4096)]
+          + [(4096, 14336), (1024, 4096), (14336, 4096), (128256, 4096), (75776, 4096),
+             (75628, 4096), (151936, 1536), (100000, 20480)]
           + [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280), (33, 2304), (37, 8960),
              (129, 256), (1, 14336), (3, 11008), (97, 4352), (300, 3840), (149, 1024),
              (147, 20480), (1000, 20480), (77, 1536), (40, 4096), (200, 1792), (3, 20480),
