@@ -478,7 +478,9 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         {
             // A lane past the last superblock position loads position 0's x
             // (its products are discarded), so the loads need no branch and
-            // their latency overlaps the first stage's wait and decode.
+            // their latency overlaps the first stage's wait and decode. Plain
+            // (coherent, L1-allocating) loads: measured on B200 the
+            // non-coherent path made the K = 14336 call 10 % slower.
             const int k0 = (valid ? bl : 0) * kQK + 64 * g + 16 * (c0 & 1);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
@@ -487,7 +489,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 const float4* xh = xl + 8;   // + 32 weights
 #pragma unroll
                 for (int v = 0; v < kNX / 4; ++v) {
-                    const float4 a = __ldg(xl + v), b = __ldg(xh + v);
+                    const float4 a = xl[v], b = xh[v];
                     xp[i][4 * v + 0] = make_float2(a.x, b.x);
                     xp[i][4 * v + 1] = make_float2(a.y, b.y);
                     xp[i][4 * v + 2] = make_float2(a.z, b.z);
