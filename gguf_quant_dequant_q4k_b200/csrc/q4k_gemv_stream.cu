@@ -704,9 +704,14 @@ int resident_clusters(int c, int num_sms, const int* max_clusters) {
 int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
                 bool fused, StreamParams* sp, int* grid, int* block, int* smem_bytes) {
     const int nsb = k / kQK;
-    if (m < 1 || m > kStreamMaxM || nsb > kStreamMaxNsb || n < 1) return 0;
-    // quant slices per lane: two for one vector on very tall matrices
-    const int sl = (m == 1 && !fused && (n + num_sms - 1) / num_sms >= kWideMinRows) ? 2 : 1;
+    if (m < 1 || m > kStreamMaxM || n < 1) return 0;
+    // quant slices per lane: two for one vector on very tall matrices, and for
+    // one vector when K is too long for one-slice teams (K > 20480: a team of
+    // two-slice lanes covers K <= 30720 with 15 warps)
+    const bool wide = m == 1 && !fused &&
+                      ((n + num_sms - 1) / num_sms >= kWideMinRows || nsb > kStreamMaxNsb);
+    const int sl = wide ? 2 : 1;
+    if (nsb > kStreamMaxNsb * sl) return 0;
     const int team_warps = (nsb * 8 / sl + 31) / 32;   // 8*nsb slices / (32 lanes * sl)
     const int max_warps = stream_max_threads(m, sl) / 32;
     if (team_warps > max_warps) return 0;

@@ -25,7 +25,10 @@ constexpr int stream_max_threads(int m, int slices) { return (m == 1 && slices =
 constexpr int stream_max_regs(int m, int slices) {
     return 16384 / (((stream_max_threads(m, slices) / 32 + 1 + 3) / 4) * 32) / 8 * 8;
 }
-constexpr int kStreamMaxNsb = 80;       // K <= 20480 (m = 1) / 15360 (m = 2): one team covers K
+// Superblocks per row one team of one-slice lanes covers (K <= 20480 for one
+// vector, 15360 for two: the warps one team may have); two-slice lanes cover
+// twice as many (K <= 30720, one vector).
+constexpr int kStreamMaxNsb = 80;
 constexpr int kStreamMaxTeams = 20;     // one producer lane per team
 constexpr int kStreamMaxDepth = 8;
 constexpr int kStreamSmemBudget = 220 * 1024;

@@ -235,7 +235,7 @@ Q4K_API int q4k_gemv_swiglu_plan_for(int m, int n, int k, int num_sms, q4k_gemv_
 enum q4k_kernel {
     Q4K_KERNEL_WARP_ROWS = 1,   /* any K: one warp per row, loads via L1; m > 8
                                    runs as ceil(m/8) launches on vector tiles   */
-    Q4K_KERNEL_STREAM = 2       /* K <= 20480 (m = 1) / 15360 (m >= 2); m > 2 runs
+    Q4K_KERNEL_STREAM = 2       /* K <= 30720 (m = 1) / 15360 (m >= 2); m > 2 runs
                                    as ceil(m/2) launches on vector pairs;
                                    bulk-copy streamed rows, x held in registers,
                                    balanced per-SM ranges; small N splits rows

@@ -111,7 +111,8 @@ def test_gemv_config_shapes(q4k, n, k):
 @pytest.mark.parametrize("n,k", [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280),
                                  (33, 2304), (37, 8960), (129, 256), (1, 14336), (3, 11008),
                                  (97, 4352), (300, 3840), (149, 1024), (77, 1536), (40, 4096),
-                                 (147, 20480), (1000, 20480), (64, 20736), (2, 30720), (5, 30976), (2, 32768)])
+                                 (147, 20480), (1000, 20480), (64, 20736), (2, 30720), (5, 30976), (2, 32768),
+                                 (1000, 28672), (150, 23040), (7, 20736)])
 def test_gemv_ragged_shapes(q4k, n, k):
     w, x = q4k_synth.q4k_problem(n, k, 1, 1000 + n + k)
     y = gpu_gemv(q4k, w, x, n, k)
@@ -139,10 +140,11 @@ def test_gemv_multivector_shapes(q4k, n, k, m):
     assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
 
 
-@pytest.mark.parametrize("n,k", [(75776, 4096), (100000, 20480), (151936, 1536)])
+@pytest.mark.parametrize("n,k", [(75776, 4096), (100000, 20480), (151936, 1536), (8192, 28672)])
 def test_gemv_tall_two_slices_sampled(q4k, n, k):
-    """Very tall matrices (512 or more rows per CTA) run two quant slices per
-    lane; the oracle checks sampled rows, including every CTA boundary region."""
+    """Very tall matrices (512 or more rows per CTA) and K beyond 20480 (one
+    vector) run two quant slices per lane; the oracle checks sampled rows,
+    including every CTA boundary region."""
     plan = q4k.q4k_gemv_plan_for(1, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
     assert plan["slices"] == 2
     w, x = q4k_synth.q4k_problem(n, k, 1, 60 + n % 97)

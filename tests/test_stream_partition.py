@@ -51,7 +51,7 @@ def check_plan(m, n, k):
     clusters = ctas // cluster
     assert clusters <= n
     slices = p["slices"]                                 # 16-byte quant slices per lane
-    wide = m == 1 and -(-n // SM_COUNT) >= 512           # very tall: two slices
+    wide = m == 1 and (-(-n // SM_COUNT) >= 512 or nsb > 80)   # very tall or long K: two slices
     assert slices == (2 if wide else 1)
     team_warps = -(-nsb * 8 // slices // 32)
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
@@ -118,7 +118,8 @@ def check_plan(m, n, k):
 
 SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
           + [(4096, 14336), (1024, 4096), (14336, 4096), (128256, 4096), (75776, 4096),
-             (75628, 4096), (151936, 1536), (100000, 20480)]
+             (75628, 4096), (151936, 1536), (100000, 20480), (1000, 28672), (64, 30720),
+             (8192, 28672), (2, 30720), (7, 20736), (150, 23040)]
           + [(1, 256), (2, 256), (5, 512), (7, 768), (31, 1280), (33, 2304), (37, 8960),
              (129, 256), (1, 14336), (3, 11008), (97, 4352), (300, 3840), (149, 1024),
              (147, 20480), (1000, 20480), (77, 1536), (40, 4096), (200, 1792), (3, 20480),
@@ -155,7 +156,11 @@ def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(8, 4096, 14336, SM_COUNT)["launches"] == 4
     assert q4k.q4k_gemv_plan_for(3, 64, 15616, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
     assert q4k.q4k_gemv_plan_for(1, 64, 20480, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
-    assert q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    # one vector, K beyond one-slice teams: two-slice teams up to K = 30720
+    p = q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)
+    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2
+    assert q4k.q4k_gemv_plan_for(1, 64, 30720, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
+    assert q4k.q4k_gemv_plan_for(1, 64, 30976, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
     assert q4k.q4k_gemv_plan_for(2, 64, 15360, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_plan_for(2, 64, 15616, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
 
@@ -166,7 +171,7 @@ def test_batches_beyond_eight_vectors():
     assert q4k.q4k_gemv_plan_for(16, 14336, 4096, SM_COUNT)["launches"] == 8
     assert q4k.q4k_gemv_plan_for(33, 4096, 4096, SM_COUNT)["launches"] == 17
     assert q4k.q4k_gemv_plan_for(64, 4096, 4096, SM_COUNT)["launches"] == 32
-    p = q4k.q4k_gemv_plan_for(20, 64, 20736, SM_COUNT)
+    p = q4k.q4k_gemv_plan_for(20, 64, 30976, SM_COUNT)
     assert p["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS and p["launches"] == 3
     with pytest.raises(q4k.Q4KError):
         q4k.q4k_gemv_plan_for(65, 4096, 4096, SM_COUNT)
@@ -248,4 +253,5 @@ def test_fused_partition(m, n, k):
 
 def test_fused_falls_back_beyond_the_stream_range():
     assert q4k.q4k_gemv_swiglu_plan_for(1, 64, 20736, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    assert q4k.q4k_gemv_swiglu_plan_for(1, 64, 20480, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_swiglu_plan_for(1, 7, 14336, SM_COUNT)["cluster"] == 1
