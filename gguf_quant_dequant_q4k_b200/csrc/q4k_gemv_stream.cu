@@ -1,5 +1,5 @@
 // q4k_gemv_stream.cu -- the streaming Q4_K GEMV (plain, or fused gate/up
-// SwiGLU) for m = 1, 2 and K <= 20480 (m = 1) or 15360 (m = 2).
+// SwiGLU) for m = 1, 2 and K <= 30720 (m = 1) or 15360 (m = 2).
 //
 // What it computes: y[i][r] = sum_k W[r][k] x[i][k] with W in Q4_K, as the
 // pages' `Q4KGemv` / `TiledQ4KGemv` / `ChunkedTiledQ4KGemv` / `MwvQ4KGemv`
