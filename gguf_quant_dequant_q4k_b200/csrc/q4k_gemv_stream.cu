@@ -21,7 +21,9 @@
 //   fixed weights of K (16 low nibbles of sub-block 2g and 16 high nibbles of
 //   sub-block 2g+1, g = c/2). Its 32 x values per vector live in registers for
 //   the whole kernel, so x costs no shared-memory bandwidth per row and there
-//   is no K*4-byte shared-memory ceiling.
+//   is no K*4-byte shared-memory ceiling. For one vector on very tall
+//   matrices, or K > 20480, a lane owns two adjacent slices (S = 2: 64
+//   weights, ceil(K/2048) warps per team).
 // * Streaming. Each team streams its byte range through a ring of `depth`
 //   shared-memory stages with 1-D bulk async copies (cp.async.bulk, completing
 //   on a "full" mbarrier; no multicast). A stage is up to 4 consecutive row
