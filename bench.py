@@ -11,7 +11,11 @@ bytes = N*K/256*144 + 4*m*(K+N) per call.
 Under torchrun (N > 1) every rank runs the same sweep on its own GPU (replicas:
 the GEMV needs no exchange); value sums the bytes of all ranks over the slowest
 rank's time. `--impl reference` times the CPU oracle instead (rank 0 only).
-Prints one JSON line on rank 0.
+Prints one JSON line on rank 0. Besides the contract keys it carries
+`per_shape` (µs per call of each projection: 200 back-to-back calls over
+rotating weight copies, median of 5 repeats, and the same with one copy,
+`l2_hot_us_per_call`, where W fits in L2) and `extra` (multi-vector,
+32-layer, fused SwiGLU and embedding figures).
 """
 from __future__ import annotations
 
@@ -523,30 +527,35 @@ def run_ours(args) -> None:
     ms_per_step = ms / args.steps
     value = whole_job_gbs(world, BYTES_PER_STEP, args.steps, ms)
 
-    # per-projection us/call: R back-to-back calls over rotating copies
+    # per-projection us/call: R = 200 back-to-back calls over rotating copies
+    # (each copy re-read only after more than 2 x L2 of other traffic), median
+    # of 5 repeats; and the same with one copy (L2-hot where W fits in L2)
     per_shape = []
     peak, peak_kind = measured_peak()
-    for s, p in zip([] if args.skip_extras else shapes, plans):
-        reps = 200
+
+    def timed_calls(s, copies, reps=200):
         with torch.cuda.stream(stream):
             for i in range(10):
-                q4k.q4k_gemv(s["ws"][i % len(s["ws"])], s["x"], s["y"], 1, s["n"], s["k"],
-                             stream=stream)
+                q4k.q4k_gemv(s["ws"][i % copies], s["x"], s["y"], 1, s["n"], s["k"], stream=stream)
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         for i in range(reps):
-            q4k.q4k_gemv(s["ws"][i % len(s["ws"])], s["x"], s["y"], 1, s["n"], s["k"],
-                         stream=stream)
+            q4k.q4k_gemv(s["ws"][i % copies], s["x"], s["y"], 1, s["n"], s["k"], stream=stream)
         a1.record(stream)
         torch.cuda.synchronize(dev)
-        us = a0.elapsed_time(a1) * 1e3 / reps
+        return a0.elapsed_time(a1) * 1e3 / reps
+
+    for s, p in zip([] if args.skip_extras else shapes, plans):
+        us = statistics.median(timed_calls(s, len(s["ws"])) for _ in range(5))
+        hot = statistics.median(timed_calls(s, 1) for _ in range(5))
         b = bytes_counted(s["n"], s["k"])
         per_shape.append({"n": s["n"], "k": s["k"], "us_per_call": round(us, 3),
                           "gbs": round(b / us / 1e3, 1), "frac_of_measured": round(b / us / 1e3 / peak, 4),
                           "frac_of_nominal": round(b / us / 1e3 / NOMINAL_HBM_GBS, 4),
+                          "l2_hot_us_per_call": round(hot, 3),
                           "w_copies": len(s["ws"]), "kernel": p["kernel"], "grid": p["grid"],
-                          "teams": p["teams"], "depth": p["depth"]})
+                          "teams": p["teams"], "depth": p["depth"], "slices": p["slices"]})
 
     # end to end through the public API: pinned x -> device, gemv, y -> pinned host
     e2e_steps = 0 if args.skip_extras else min(args.steps, 500)
