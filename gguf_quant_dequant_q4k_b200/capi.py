@@ -97,11 +97,16 @@ def library() -> ctypes.CDLL:
     return _lib
 
 
-def _ptr(t) -> int | None:
+def _ptr(t, dtype: str | None = None, name: str = "") -> int | None:
+    """Device address of a tensor (or a raw integer address, passed through).
+    With `dtype` ("float32", "int32", "uint8"), a tensor of another element type
+    is refused: the library reads raw bytes and could not tell."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if dtype is not None and str(t.dtype).replace("torch.", "") != dtype:
+        raise TypeError(f"{name} must be a {dtype} tensor, got {t.dtype}")
     return t.data_ptr()
 
 
@@ -160,7 +165,8 @@ def q4k_device_fault_flags() -> int:
 
 def q4k_gemv_status(w, x, y, m: int, n: int, k: int, stream=None) -> int:
     """Raw status of the C call (no exception)."""
-    return _lib.q4k_gemv(_ptr(w), _ptr(x), _ptr(y), int(m), int(n), int(k), _stream(stream))
+    return _lib.q4k_gemv(_ptr(w), _ptr(x, "float32", "x"), _ptr(y, "float32", "y"), int(m), int(n),
+                         int(k), _stream(stream))
 
 
 def q4k_gemv(w, x, y, m: int, n: int, k: int, stream=None) -> None:
@@ -171,7 +177,8 @@ def q4k_gemv(w, x, y, m: int, n: int, k: int, stream=None) -> None:
 
 
 def q4k_gemv_swiglu_status(w_gate, w_up, x, y, m: int, n: int, k: int, stream=None) -> int:
-    return _lib.q4k_gemv_swiglu(_ptr(w_gate), _ptr(w_up), _ptr(x), _ptr(y), int(m), int(n),
+    return _lib.q4k_gemv_swiglu(_ptr(w_gate), _ptr(w_up), _ptr(x, "float32", "x"),
+                                _ptr(y, "float32", "y"), int(m), int(n),
                                 int(k), _stream(stream))
 
 
@@ -183,7 +190,8 @@ def q4k_gemv_swiglu(w_gate, w_up, x, y, m: int, n: int, k: int, stream=None) -> 
 
 
 def q4k_dequant_f32_status(w, out, n: int, k: int, stream=None) -> int:
-    return _lib.q4k_dequant_f32(_ptr(w), _ptr(out), int(n), int(k), _stream(stream))
+    return _lib.q4k_dequant_f32(_ptr(w), _ptr(out, "float32", "out"), int(n), int(k),
+                                _stream(stream))
 
 
 def q4k_dequant_f32(w, out, n: int, k: int, stream=None) -> None:
@@ -196,6 +204,8 @@ def q4k_dequant_f32(w, out, n: int, k: int, stream=None) -> None:
 def _nbytes(t, given) -> int:
     if given is not None:
         return int(given)
+    if t is None or isinstance(t, int):
+        raise ValueError("table_bytes is required with a raw address")
     return t.numel() * t.element_size()
 
 
@@ -206,7 +216,8 @@ def q4k_embed_lookup_f32_status(table, rows: int, cols: int, hidden: int, token:
     tensor's size; pass it explicitly with a raw pointer."""
     return _lib.q4k_embed_lookup_f32(_ptr(table), _nbytes(table, table_bytes), int(rows),
                                      int(cols), int(hidden), int(token) & 0xFFFFFFFF,
-                                     float(embed_scale), _ptr(out), _stream(stream))
+                                     float(embed_scale), _ptr(out, "float32", "out"),
+                                     _stream(stream))
 
 
 def q4k_embed_lookup_f32(table, rows: int, cols: int, hidden: int, token: int,
@@ -223,8 +234,9 @@ def q4k_embed_gather_f32_status(table, rows: int, hidden: int, tokens, n_tokens:
                                 embed_scale: float, out, stream=None,
                                 table_bytes: int | None = None) -> int:
     return _lib.q4k_embed_gather_f32(_ptr(table), _nbytes(table, table_bytes), int(rows),
-                                     int(hidden), _ptr(tokens), int(n_tokens),
-                                     float(embed_scale), _ptr(out), _stream(stream))
+                                     int(hidden), _ptr(tokens, "int32", "tokens"), int(n_tokens),
+                                     float(embed_scale), _ptr(out, "float32", "out"),
+                                     _stream(stream))
 
 
 def q4k_embed_gather_f32(table, rows: int, hidden: int, tokens, n_tokens: int,

@@ -176,3 +176,22 @@ def test_embed_gather_checks(kw, expect):
                 out=A16 * 4, stream=0, table_bytes=10 * 144)
     args.update(kw)
     assert capi.q4k_embed_gather_f32_status(**args) == expect
+
+
+def test_binding_refuses_wrong_element_types():
+    """The library reads raw bytes; the binding refuses tensors of another
+    element type before any call (CPU tensors here, never dereferenced)."""
+    torch = pytest.importorskip("torch")
+    half = torch.zeros(256, dtype=torch.float16)
+    f32 = torch.zeros(256, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        capi.q4k_gemv_status(A16, half, f32, 1, 1, 256, stream=0)
+    with pytest.raises(TypeError):
+        capi.q4k_gemv_status(A16, f32, half, 1, 1, 256, stream=0)
+    with pytest.raises(TypeError):
+        capi.q4k_dequant_f32_status(A16, half, 1, 256, stream=0)
+    with pytest.raises(TypeError):
+        capi.q4k_embed_gather_f32_status(A16, 10, 256, torch.zeros(4, dtype=torch.int64), 4,
+                                         1.0, A16 * 4, stream=0, table_bytes=10 * 144)
+    with pytest.raises(ValueError):
+        capi.q4k_embed_lookup_f32_status(A16, 10, 256, 256, 0, 1.0, A16 * 4, stream=0)
