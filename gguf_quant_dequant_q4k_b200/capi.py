@@ -97,17 +97,43 @@ def library() -> ctypes.CDLL:
     return _lib
 
 
-def _ptr(t, dtype: str | None = None, name: str = "") -> int | None:
-    """Device address of a tensor (or a raw integer address, passed through).
-    With `dtype` ("float32", "int32", "uint8"), a tensor of another element type
-    is refused: the library reads raw bytes and could not tell."""
+def _ptr(t, dtype: str | None = None, name: str = "", min_bytes: int = 0) -> int | None:
+    """Device address of a tensor (or a raw integer address, passed through
+    unchecked: the caller vouches for it).
+
+    A tensor must be a contiguous CUDA tensor on the current CUDA device (the
+    library launches there and cannot tell a host or foreign pointer from a
+    raw address) holding at least `min_bytes` bytes; with `dtype` ("float32",
+    "int32", "uint8") its element type must match, since the library reads raw
+    bytes. Anything else raises before the C call."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
     if dtype is not None and str(t.dtype).replace("torch.", "") != dtype:
         raise TypeError(f"{name} must be a {dtype} tensor, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name or 'tensor'} must be a CUDA tensor, got device {t.device}")
+    import torch
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name or 'tensor'} is on {t.device}, but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name or 'tensor'} must be contiguous")
+    have = t.numel() * t.element_size()
+    if have < min_bytes:
+        raise ValueError(f"{name or 'tensor'} holds {have} bytes, the call needs {min_bytes}")
     return t.data_ptr()
+
+
+def _need(count: int, item: int, valid: bool) -> int:
+    """Bytes a buffer must hold, or 0 where the C library will refuse the
+    call's sizes anyway (its status is then the answer)."""
+    return count * item if valid and count > 0 else 0
+
+
+def _gemv_sizes_valid(m: int, n: int, k: int) -> bool:
+    return 1 <= m <= Q4K_MAX_M and q4k_weight_bytes(n, k) > 0
 
 
 def _stream(stream) -> int | None:
@@ -164,8 +190,11 @@ def q4k_device_fault_flags() -> int:
 
 
 def q4k_gemv_status(w, x, y, m: int, n: int, k: int, stream=None) -> int:
-    """Raw status of the C call (no exception)."""
-    return _lib.q4k_gemv(_ptr(w), _ptr(x, "float32", "x"), _ptr(y, "float32", "y"), int(m), int(n),
+    """Raw status of the C call (no exception; tensor checks still raise)."""
+    ok = _gemv_sizes_valid(m, n, k)
+    return _lib.q4k_gemv(_ptr(w, None, "w", _need(q4k_weight_bytes(n, k), 1, ok)),
+                         _ptr(x, "float32", "x", _need(m * k, 4, ok)),
+                         _ptr(y, "float32", "y", _need(m * n, 4, ok)), int(m), int(n),
                          int(k), _stream(stream))
 
 
@@ -177,8 +206,11 @@ def q4k_gemv(w, x, y, m: int, n: int, k: int, stream=None) -> None:
 
 
 def q4k_gemv_swiglu_status(w_gate, w_up, x, y, m: int, n: int, k: int, stream=None) -> int:
-    return _lib.q4k_gemv_swiglu(_ptr(w_gate), _ptr(w_up), _ptr(x, "float32", "x"),
-                                _ptr(y, "float32", "y"), int(m), int(n),
+    ok = _gemv_sizes_valid(m, n, k)
+    wb = _need(q4k_weight_bytes(n, k), 1, ok)
+    return _lib.q4k_gemv_swiglu(_ptr(w_gate, None, "w_gate", wb), _ptr(w_up, None, "w_up", wb),
+                                _ptr(x, "float32", "x", _need(m * k, 4, ok)),
+                                _ptr(y, "float32", "y", _need(m * n, 4, ok)), int(m), int(n),
                                 int(k), _stream(stream))
 
 
@@ -190,7 +222,9 @@ def q4k_gemv_swiglu(w_gate, w_up, x, y, m: int, n: int, k: int, stream=None) -> 
 
 
 def q4k_dequant_f32_status(w, out, n: int, k: int, stream=None) -> int:
-    return _lib.q4k_dequant_f32(_ptr(w), _ptr(out, "float32", "out"), int(n), int(k),
+    ok = q4k_weight_bytes(n, k) > 0
+    return _lib.q4k_dequant_f32(_ptr(w, None, "w", _need(q4k_weight_bytes(n, k), 1, ok)),
+                                _ptr(out, "float32", "out", _need(n * k, 4, ok)), int(n), int(k),
                                 _stream(stream))
 
 
@@ -214,9 +248,11 @@ def q4k_embed_lookup_f32_status(table, rows: int, cols: int, hidden: int, token:
                                 table_bytes: int | None = None) -> int:
     """Raw status of the C call (no exception). table_bytes defaults to the
     tensor's size; pass it explicitly with a raw pointer."""
-    return _lib.q4k_embed_lookup_f32(_ptr(table), _nbytes(table, table_bytes), int(rows),
-                                     int(cols), int(hidden), int(token) & 0xFFFFFFFF,
-                                     float(embed_scale), _ptr(out, "float32", "out"),
+    ok = hidden > 0 and hidden % Q4K_QK == 0
+    return _lib.q4k_embed_lookup_f32(_ptr(table, None, "table"), _nbytes(table, table_bytes),
+                                     int(rows), int(cols), int(hidden), int(token) & 0xFFFFFFFF,
+                                     float(embed_scale),
+                                     _ptr(out, "float32", "out", _need(hidden, 4, ok)),
                                      _stream(stream))
 
 
@@ -233,9 +269,12 @@ def q4k_embed_lookup_f32(table, rows: int, cols: int, hidden: int, token: int,
 def q4k_embed_gather_f32_status(table, rows: int, hidden: int, tokens, n_tokens: int,
                                 embed_scale: float, out, stream=None,
                                 table_bytes: int | None = None) -> int:
-    return _lib.q4k_embed_gather_f32(_ptr(table), _nbytes(table, table_bytes), int(rows),
-                                     int(hidden), _ptr(tokens, "int32", "tokens"), int(n_tokens),
-                                     float(embed_scale), _ptr(out, "float32", "out"),
+    ok = hidden > 0 and hidden % Q4K_QK == 0 and n_tokens > 0
+    return _lib.q4k_embed_gather_f32(_ptr(table, None, "table"), _nbytes(table, table_bytes),
+                                     int(rows), int(hidden),
+                                     _ptr(tokens, "int32", "tokens", _need(n_tokens, 4, ok)),
+                                     int(n_tokens), float(embed_scale),
+                                     _ptr(out, "float32", "out", _need(n_tokens * hidden, 4, ok)),
                                      _stream(stream))
 
 

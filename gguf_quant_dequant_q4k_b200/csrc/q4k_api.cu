@@ -7,10 +7,11 @@
 // (`batched_q4k_gemv_into`, "realizar 0.8.5, src/cuda/executor/uses.rs") and is
 // refused rather than padded; the byte size N*(K/256)*144 is computed with
 // overflow checks (`validate_block_quant_embedding`, "turbospark-runtime
-// 0.1.0, src/real_forward_dispatch.rs"); more than 8 vectors is refused rather
-// than looped (`encode_gemm_any`, same page); a failed launch returns an error
-// code to the caller (the rc convention of "memra-engine 0.83.1,
-// src/f16_ffi.rs").
+// 0.1.0, src/real_forward_dispatch.rs"); more than Q4K_MAX_M (64) vectors is
+// refused rather than looped (`encode_gemm_any`, same page); a failed launch
+// returns an error code to the caller (the rc convention of "memra-engine
+// 0.83.1, src/f16_ffi.rs", `qmatvec_gemm_f16_raw`: a nonzero rc from
+// `memra_f16_pp_gemm` names its class, a CUDA error among them).
 #include <atomic>
 #include <cstdint>
 #include <cstring>

@@ -36,13 +36,16 @@
 //   rest of the ring follows once every compute warp has issued its x loads
 //   (x is the dependent input, so it must not queue behind the ring).
 // * Decode. Once per stage each warp decodes the headers of its superblocks
-//   (d, dmin, 12 scale bytes; GGUF get_scale_min_k4 packing) into (A_j, B_j)
-//   pairs with A_j = 256*d*sc_j (exact) and B_j = -(128*d*sc_j + dmin*m_j).
-//   A weight with quant q is then A_j*f + B_j where f = 1/2 + q/256 is built by
-//   one byte permute of the masked nibble into the mantissa of 1/2 (exact):
-//   d*sc_j*q - dmin*m_j rounded once (B_j's own rounding, at most half an ulp
-//   of 128*d*sc_j + dmin*m_j, is the only other error). Weights and dot
-//   products use packed f32x2 FMAs.
+//   (d, dmin, 12 scale bytes; GGUF get_scale_min_k4 packing) into (A_j, B_j,
+//   e_j) with A_j = 256*d*sc_j (exact), B_j = -fl(128*d*sc_j + dmin*m_j) and
+//   e_j the exact rounding error of that sum (TwoSum). A weight with quant q is
+//   formed as fma(A_j, f, B_j), f = 1/2 + q/256 built by one byte permute of
+//   the masked nibble into the mantissa of 1/2 (exact): that is w + e_j
+//   rounded once, w = d*sc_j*q - dmin*m_j. Each item then adds -e_j times the
+//   sum of the lane's x over sub-block j (a per-lane constant, since x stays
+//   in registers), so the error left per weight is the one rounding of w +
+//   e_j, relative to |w| up to |e_j| <= 2^-24 (128*d*sc_j + dmin*m_j). Weights
+//   and dot products use packed f32x2 FMAs.
 // * Reduction. Per stage each lane holds one partial per row segment; a
 //   4-segment transpose-reduce across the warp (5 shuffles) leaves one value
 //   per segment, published to shared memory for the producer lane to add.
@@ -76,8 +79,11 @@ constexpr int kSeg = kStreamSegRows;         // row segments per stage
 constexpr unsigned kXIssuedBarrier = 1;      // named barrier: compute warps issued x loads
 constexpr uint32_t kMagicOne = 0x3F000000u;  // 1/2: bytes 0..2 = 0x00, byte 3 = 0x3F
 constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
-// Coefficient buffer per warp: [segment][position][4 groups] float4s.
-constexpr int coef_bytes_per_warp(int slices) { return kSeg * (4 * slices) * 4 * 16; }
+// Coefficient buffer per warp: [segment][position][4 groups] float4s
+// (A_2g, A_2g+1, B_2g, B_2g+1), then [segment][position][4 groups] float2s
+// (-e_2g, -e_2g+1): B's rounding errors.
+__host__ __device__ constexpr int coef_main_bytes_per_warp(int slices) { return kSeg * (4 * slices) * 4 * 16; }
+__host__ __device__ constexpr int coef_bytes_per_warp(int slices) { return kSeg * (4 * slices) * 4 * (16 + 8); }
 
 // f = 1/2 + q/256 for the nibble q held in byte SEL of `masked` (bytes 0..15):
 // the byte becomes bits 16..23 of 0x3F000000 (1/2), i.e. mantissa bits 16..19.
@@ -160,12 +166,22 @@ __device__ __forceinline__ long long seg_end(const TeamRange& r, int i, int nsb)
 }
 
 
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    return __fadd2_rn(a, make_float2(-b.x, -b.y));
+}
+
 // (A_2g, A_2g+1, B_2g, B_2g+1) for the two 64-weight groups g = 2*half and
 // 2*half+1 of one superblock header h (bytes 0..15), with A_j = 256*d*sc_j and
-// B_j = -(128*d*sc_j + dmin*m_j), so that A_j*(1/2 + q/256) + B_j =
-// d*sc_j*q - dmin*m_j. A_j and the two products are exact; B_j is rounded once.
+// B_j = -fl(128*d*sc_j + dmin*m_j), so that A_j*(1/2 + q/256) + B_j =
+// d*sc_j*q - dmin*m_j + e_j, where e_j = 128*d*sc_j + dmin*m_j - fl(...) is
+// the rounding error of B_j. A_j and both products are exact, and e_j is
+// recovered exactly (TwoSum); `err` receives (-e_4h, -e_4h+1, -e_4h+2,
+// -e_4h+3). The weight the fma rounds is then w + e_j, rounded once; the
+// caller removes e_j's contribution as -e_j * (sum of the lane's x over
+// sub-block j), so the error left per weight is that one rounding of
+// w + e_j (|e_j| is at most half an ulp of 128*d*sc_j + dmin*m_j).
 __device__ __forceinline__ void decode_half(uint4 h, float d, float dmin, int half, float4& out0,
-                                            float4& out1) {
+                                            float4& out1, float4& err) {
     // six-bit fields of sub-blocks 4*half .. +3 (GGUF get_scale_min_k4 packing)
     const uint32_t sc = half ? ((h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u))
                              : (h.y & 0x3F3F3F3Fu);
@@ -183,8 +199,13 @@ __device__ __forceinline__ void decode_half(uint4 h, float d, float dmin, int ha
     const float2 m23 = ffma2(ma, make_float2(byte_2p23<2>(mm), byte_2p23<3>(mm)), mb);
     const float2 A01 = __fadd2_rn(a01, a01), A23 = __fadd2_rn(a23, a23);
     const float2 s01 = __fadd2_rn(a01, m01), s23 = __fadd2_rn(a23, m23);
+    // TwoSum: e = (a + m) - s exactly, without assuming |a| >= |m|.
+    const float2 v01 = fsub2(s01, a01), v23 = fsub2(s23, a23);
+    const float2 e01 = __fadd2_rn(fsub2(a01, fsub2(s01, v01)), fsub2(m01, v01));
+    const float2 e23 = __fadd2_rn(fsub2(a23, fsub2(s23, v23)), fsub2(m23, v23));
     out0 = make_float4(A01.x, A01.y, -s01.x, -s01.y);
     out1 = make_float4(A23.x, A23.y, -s23.x, -s23.y);
+    err = make_float4(-e01.x, -e01.y, -e23.x, -e23.y);
 }
 
 __device__ __forceinline__ void header_scales(uint4 h, float& d, float& dmin) {
@@ -452,10 +473,12 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             if (!__any_sync(0xFFFFFFFFu, progressed)) __nanosleep(64);
         }
         // After a lost copy, give the copies still in flight a bounded chance
-        // to land before the CTA's shared memory is released.
+        // to land before the CTA's shared memory is released. Stages [0, tf)
+        // were consumed; the ring holds the issued stages [tf, min(tf + depth,
+        // nst)), stage s completing phase (s / depth) & 1 of full[s % depth].
         if (own && abort_flag) {
-            const int first = nst - p.depth > 0 ? nst - p.depth : 0;
-            for (int s = first; s < nst; ++s)
+            const int last = tf + p.depth < nst ? tf + p.depth : nst;
+            for (int s = tf; s < last; ++s)
                 mbar_wait_bounded(&T.full[s % p.depth], static_cast<uint32_t>((s / p.depth) & 1),
                                   &g_fault_flags);
         }
@@ -500,6 +523,15 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             }
         }
         named_barrier_arrive(kXIssuedBarrier, blockDim.x);
+        // Per vector, the sums of the lane's low-nibble x values (sub-block
+        // 2g) and high-nibble x values (sub-block 2g+1).
+        float2 sx[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            sx[i] = xp[i][0];
+#pragma unroll
+            for (int e = 1; e < kNX; ++e) sx[i] = __fadd2_rn(sx[i], xp[i][e]);
+        }
 
         // Shared-memory byte offsets (32-bit). The coefficient float4 of
         // (segment u, position pos, group g) sits at (u*kPos + pos)*4 +
@@ -508,7 +540,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const uint32_t ring_off = static_cast<uint32_t>(T.ring - smem);
         const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c0);
         const uint32_t coef_off = static_cast<uint32_t>(p.off_coef) +
-                                  static_cast<uint32_t>(warp) * (kSeg * kPos * 4 * 16);
+                                  static_cast<uint32_t>(warp) * static_cast<uint32_t>(coef_bytes_per_warp(S));
         const uint32_t lane_coef_off =
             coef_off + static_cast<uint32_t>((lpos * 4 + (g ^ ((lpos >> 1) & 3))) * 16);
         // Decode lanes: S = 2: lane -> (segment du, position dpos), whole header;
@@ -519,6 +551,12 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const int dbl = wit * kPos + dpos;
         const uint32_t dec_base = coef_off + static_cast<uint32_t>((du * kPos + dpos) * 4 * 16);
         const int dswz = (dpos >> 1) & 3;
+        // B's rounding errors: float2 (-e_2g, -e_2g+1) of (segment, position,
+        // group) at err_off + ((u*kPos + pos)*4 + g)*8 (unswizzled: the item
+        // loads of a warp read 16 consecutive float2s, decode stores 16-byte runs).
+        const uint32_t err_off = coef_off + static_cast<uint32_t>(coef_main_bytes_per_warp(S));
+        const uint32_t dec_err = err_off + static_cast<uint32_t>((du * kPos + dpos) * 4 * 8);
+        const uint32_t lane_err_off = err_off + static_cast<uint32_t>((lpos * 4 + g) * 8);
         const int red_slot = p.team_warps * kSeg * M;
 
         int slot = 0;
@@ -545,10 +583,11 @@ q4k_gemv_stream_kernel(const StreamParams p) {
 #pragma unroll
                     for (int hh = 0; hh < S; ++hh) {
                         const int half = S == 2 ? hh : dhalf;
-                        float4 c_a, c_b;
-                        decode_half(hdr, d, dmin, half, c_a, c_b);
+                        float4 c_a, c_b, c_e;
+                        decode_half(hdr, d, dmin, half, c_a, c_b, c_e);
                         *reinterpret_cast<float4*>(smem + dec_base + ((2 * half) ^ dswz) * 16) = c_a;
                         *reinterpret_cast<float4*>(smem + dec_base + ((2 * half + 1) ^ dswz) * 16) = c_b;
+                        *reinterpret_cast<float4*>(smem + dec_err + half * 16) = c_e;
                     }
                 }
             }
@@ -581,6 +620,8 @@ q4k_gemv_stream_kernel(const StreamParams p) {
 #pragma unroll
                 for (int j = 0; j < S; ++j) q[j] = qn[j];
                 const float4 cf = cfn;
+                // used after the item's dot products: loaded here, not a step ahead
+                const float2 ne = *reinterpret_cast<const float2*>(smem + lane_err_off + u * kPos * 32);
                 if (next) {
 #pragma unroll
                     for (int j = 0; j < S; ++j)
@@ -598,6 +639,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 }
 #pragma unroll
                 for (int i = 0; i < M; ++i) {
+                    acc[i] = ffma2(ne, sx[i], acc[i]);   // remove B's rounding error
                     part_sum[i][u] = use[u] ? (acc[i].x + acc[i].y) : 0.f;
                 }
             };

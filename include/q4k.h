@@ -144,11 +144,17 @@ Q4K_API int q4k_dequant_f32(const void *w, float *out, int n, int k, q4k_stream_
  * `encode_gemv_any` pages check before every Q4_K launch). */
 Q4K_API size_t q4k_weight_bytes(int n, int k);
 
-/* A static, NUL-terminated description of a q4k_status value. */
+/* A static, NUL-terminated description of a q4k_status value. Status codes
+ * follow the return-code convention of the memra FFI ("memra-engine 0.83.1,
+ * src/f16_ffi.rs", `qmatvec_gemm_f16_raw`): every entry point returns an int,
+ * 0 on success, and a nonzero code names the class of failure (there: cudaError
+ * convert, no cuBLASLt algorithm, matmul status; here: the q4k_status values). */
 Q4K_API const char *q4k_status_string(int status);
 
 /* The cudaError_t behind the most recent Q4K_ERR_CUDA returned on the calling
- * thread (0 if none). */
+ * thread (0 if none): the CUDA error the memra rc convention folds into its
+ * "cudaError" class ("memra-engine 0.83.1, src/f16_ffi.rs",
+ * `qmatvec_gemm_f16_raw`), kept here as its own value. */
 Q4K_API int q4k_last_cuda_error(void);
 
 /*
@@ -189,7 +195,11 @@ Q4K_API int q4k_embed_gather_f32(const void *table, unsigned long long table_byt
                                  float *out, q4k_stream_t stream);
 
 /*
- * Reads and clears the calling device's fault flags (Q4K_FAULT_* bits):
+ * Reads and clears the calling device's fault flags (Q4K_FAULT_* bits). The
+ * pages report every failure to the caller as a return code (the rc classes of
+ * `memra_f16_pp_gemm`, "memra-engine 0.83.1, src/f16_ffi.rs",
+ * `qmatvec_gemm_f16_raw`); a failure found inside a running kernel cannot
+ * return one, so it is recorded here and read after the fact:
  * Q4K_FAULT_COPY_TIMEOUT if a bounded wait inside a kernel on a bulk copy into
  * shared memory gave up (the kernel then skipped its remaining work and
  * returned; its output is invalid; never happens in normal operation);

@@ -187,7 +187,7 @@ def test_binding_refuses_wrong_element_types():
     with pytest.raises(TypeError):
         capi.q4k_gemv_status(A16, half, f32, 1, 1, 256, stream=0)
     with pytest.raises(TypeError):
-        capi.q4k_gemv_status(A16, f32, half, 1, 1, 256, stream=0)
+        capi.q4k_gemv_status(A16, A16 * 2, half, 1, 1, 256, stream=0)
     with pytest.raises(TypeError):
         capi.q4k_dequant_f32_status(A16, half, 1, 256, stream=0)
     with pytest.raises(TypeError):
@@ -195,3 +195,19 @@ def test_binding_refuses_wrong_element_types():
                                          1.0, A16 * 4, stream=0, table_bytes=10 * 144)
     with pytest.raises(ValueError):
         capi.q4k_embed_lookup_f32_status(A16, 10, 256, 256, 0, 1.0, A16 * 4, stream=0)
+
+
+def test_binding_refuses_host_tensors():
+    """A CPU tensor would reach the kernel as a host pointer: refused before the
+    call (never dereferenced here)."""
+    torch = pytest.importorskip("torch")
+    f32 = torch.zeros(256, dtype=torch.float32)
+    w = torch.zeros(144, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        capi.q4k_gemv_status(A16, f32, A16 * 2, 1, 1, 256, stream=0)
+    with pytest.raises(ValueError):
+        capi.q4k_gemv_status(w, A16, A16 * 2, 1, 1, 256, stream=0)
+    with pytest.raises(ValueError):
+        capi.q4k_dequant_f32_status(A16, f32, 1, 256, stream=0)
+    with pytest.raises(ValueError):
+        capi.q4k_gemv_swiglu_status(A16, w, A16 * 2, A16 * 4, 1, 1, 256, stream=0)

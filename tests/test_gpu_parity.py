@@ -11,6 +11,7 @@ import pytest
 
 import oracle
 import q4k_synth
+import special_blocks
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -218,6 +219,90 @@ def test_gemv_unit_vectors_give_columns(q4k):
                           f"column {c}")
 
 
+def _gpu_columns(q4k, wt, n, k, cols, m):
+    """y for x = e_c, c in `cols`, as calls of m vectors each (the last call may
+    hold fewer). Returns (len(cols), n)."""
+    cols = np.asarray(cols)
+    eye = torch.zeros((len(cols), k), dtype=torch.float32, device="cuda")
+    eye[torch.arange(len(cols), device="cuda"), torch.from_numpy(cols).cuda()] = 1.0
+    y = torch.full((len(cols), n), float("nan"), dtype=torch.float32, device="cuda")
+    for i0 in range(0, len(cols), m):
+        mi = min(m, len(cols) - i0)
+        q4k.q4k_gemv(wt, eye[i0:i0 + mi], y[i0:i0 + mi], mi, n, k)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def _assert_columns(y, deq, cols, what):
+    ref = deq[:, cols].T.astype(np.float64)
+    assert_gemv_close(y, ref, np.abs(ref), what)
+
+
+@pytest.mark.parametrize("m", [1, 2, 64])
+def test_gemv_unit_vectors_every_column(q4k, m):
+    """x = e_c for every column c of a 257 x 2048 matrix: y must be column c of
+    the dequantised matrix within 1e-4 |w| + 1e-6 per element. m = 1 runs the
+    one-vector kernel, m = 2 and 64 the two-vector kernel (64 = 32 pairs)."""
+    n, k = 257, 2048
+    w, _ = q4k_synth.q4k_problem(n, k, 1, 32)
+    deq = oracle.dequant_f32(w, n, k)
+    cols = np.arange(k)
+    y = _gpu_columns(q4k, dev(w), n, k, cols, m)
+    _assert_columns(y, deq, cols, f"every column, m={m}")
+
+
+@pytest.mark.parametrize("n,k", [(33, 20736), (75776, 256)])
+def test_gemv_unit_vectors_every_column_two_slices(q4k, n, k):
+    """The two-slice one-vector kernel (K beyond 20480, or 512+ rows per CTA),
+    x = e_c for every column."""
+    plan = q4k.q4k_gemv_plan_for(1, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert plan["slices"] == 2
+    w, _ = q4k_synth.q4k_problem(n, k, 1, 36)
+    deq = oracle.dequant_f32(w, n, k)
+    cols = np.arange(k)
+    y = _gpu_columns(q4k, dev(w), n, k, cols, 1)
+    _assert_columns(y, deq, cols, f"every column, {n}x{k}")
+
+
+@pytest.mark.parametrize("m", [1, 2, 3])
+@pytest.mark.parametrize("n,k", [(40, 4096), (7, 14336), (300, 1536), (33, 20736)])
+def test_gemv_zero_quant_blocks(q4k, n, k, m):
+    """All-zero quants (weights exactly -dmin*m_j) with a large d*sc: y = W 1
+    and y = W x for x ~ N(0,1) within the per-element bound."""
+    w = special_blocks.zero_quant_matrix(n, k)
+    deq = oracle.dequant_f32(w, n, k)
+    assert (deq == np.float32(-float(np.uint16(0x1438).view(np.float16)))).all()
+    x = np.ones((m, k), np.float32)
+    x[1:] = q4k_synth.x_vectors(k, m - 1, 61 + m)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(y, yref, a, f"zero quants {n}x{k} m={m}")
+
+
+@pytest.mark.parametrize("m", [1, 2, 3])
+@pytest.mark.parametrize("n,k", [(40, 4096), (5, 14336), (149, 1024), (20, 20736)])
+def test_gemv_near_cancelling_blocks(q4k, n, k, m):
+    """Weights that nearly cancel with d != dmin (so B_j's rounding is not
+    exact), against all-ones and N(0,1) activations."""
+    w = special_blocks.near_cancelling_matrix(n, k, 62 + n)
+    x = np.ones((m, k), np.float32)
+    x[1:] = 10 * q4k_synth.x_vectors(k, m - 1, 63 + m)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(y, yref, a, f"near-cancelling {n}x{k} m={m}")
+
+
+def test_gemv_near_cancelling_every_column(q4k):
+    n, k = 65, 2048
+    w = special_blocks.near_cancelling_matrix(n, k, 64)
+    deq = oracle.dequant_f32(w, n, k)
+    wt = dev(w)
+    cols = np.arange(k)
+    for m in (1, 2):
+        _assert_columns(_gpu_columns(q4k, wt, n, k, cols, m), deq, cols,
+                        f"near-cancelling columns m={m}")
+
+
 def _cancelling_block():
     # sc_j = 4, m_j = 60, every q = 15, d = dmin  =>  every weight is exactly 0
     S = np.array([4, 4, 4, 4, 60 | 0xC0, 60 | 0xC0, 60 | 0xC0, 60 | 0xC0,
@@ -280,7 +365,18 @@ def test_invalid_arguments_on_gpu_enqueue_nothing(q4k):
     xt = torch.zeros(k, dtype=torch.float32, device="cuda")
     y = torch.full((n,), 3.0, device="cuda")
     assert q4k.q4k_gemv_status(wt, xt, y, 65, n, k) == q4k.Q4K_ERR_UNSUPPORTED_M
-    assert q4k.q4k_gemv_status(wt, xt, y, 9, n, k) == q4k.Q4K_ERR_OVERLAP   # x, y hold one vector
+    # x and y hold one vector: the binding refuses a tensor too small for 9;
+    # through raw addresses the library finds y overlapping x
+    with pytest.raises(ValueError):
+        q4k.q4k_gemv_status(wt, xt, y, 9, n, k)
+    assert (q4k.q4k_gemv_status(wt.data_ptr(), xt.data_ptr(), y.data_ptr(), 9, n, k)
+            == q4k.Q4K_ERR_OVERLAP)
+    with pytest.raises(ValueError):   # weights short of n*(k/256)*144 bytes
+        q4k.q4k_gemv_status(wt[:-16], xt, y, 1, n, k)
+    with pytest.raises(ValueError):   # a strided view is not a dense row-major buffer
+        q4k.q4k_gemv_status(wt, torch.zeros(2 * k, device="cuda")[::2], y, 1, n, k)
+    with pytest.raises(ValueError):   # dequant output too small
+        q4k.q4k_dequant_f32_status(wt, torch.zeros(n * k - 1, device="cuda"), n, k)
     assert q4k.q4k_gemv_status(wt.data_ptr() + 8, xt, y, 1, n, k) == q4k.Q4K_ERR_ALIGN
     assert q4k.q4k_gemv_status(wt, xt, y, 1, n, 500) == q4k.Q4K_ERR_SHAPE
     torch.cuda.synchronize()

@@ -8,6 +8,7 @@ import pytest
 
 import oracle
 import q4k_synth
+import special_blocks
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -116,3 +117,51 @@ def test_swiglu_matches_separate_gemvs(q4k):
     tol = oracle.swiglu_tolerance(go, uo, a_g, a_u, ref)
     assert np.all(np.abs(y - sep) <= 2 * tol)    # both within tol of the reference
     assert q4k.q4k_device_fault_flags() == 0
+
+
+def _swiglu_columns(q4k, wg, wu, n, k, m):
+    """y for x = e_c for every column c, m vectors per call."""
+    eye = torch.eye(k, dtype=torch.float32, device="cuda")
+    y = torch.full((k, n), float("nan"), dtype=torch.float32, device="cuda")
+    gt, ut = torch.from_numpy(wg).cuda(), torch.from_numpy(wu).cuda()
+    for i0 in range(0, k, m):
+        mi = min(m, k - i0)
+        q4k.q4k_gemv_swiglu(gt, ut, eye[i0:i0 + mi], y[i0:i0 + mi], mi, n, k)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+@pytest.mark.parametrize("m", [1, 2, 64])
+def test_swiglu_unit_vectors_every_column(q4k, m):
+    """x = e_c for every column of a 257 x 2048 gate (the seed-32 matrix) and
+    an up matrix: y = silu(gate column) * (up column) within the bound."""
+    n, k = 257, 2048
+    wg, _ = q4k_synth.q4k_problem(n, k, 1, 32)
+    wu, _ = q4k_synth.q4k_problem(n, k, 1, 37)
+    y = _swiglu_columns(q4k, wg, wu, n, k, m)
+    x = np.eye(k, dtype=np.float32)
+    assert_swiglu_close(y, wg, wu, x, n, k, f"every column m={m}")
+
+
+@pytest.mark.parametrize("m", [1, 2])
+@pytest.mark.parametrize("n,k", [(40, 4096), (300, 1536)])
+def test_swiglu_zero_quant_and_near_cancelling(q4k, n, k, m):
+    """Gate of all-zero-quant blocks (weights exactly -dmin*m_j) and up of
+    near-cancelling blocks, and the other way round, with x = 1 and N(0,1)."""
+    wz = special_blocks.zero_quant_matrix(n, k)
+    wc = special_blocks.near_cancelling_matrix(n, k, 70 + n)
+    x = np.ones((m, k), np.float32)
+    x[1:] = q4k_synth.x_vectors(k, m - 1, 71 + m)
+    for wg, wu, what in ((wz, wc, "zero/near"), (wc, wz, "near/zero")):
+        y = gpu_swiglu(q4k, wg, wu, x, n, k)
+        assert_swiglu_close(y, wg, wu, x, n, k, f"{what} {n}x{k} m={m}")
+
+
+def test_swiglu_near_cancelling_every_column(q4k):
+    n, k = 65, 2048
+    wg = special_blocks.near_cancelling_matrix(n, k, 72)
+    wu = special_blocks.zero_quant_matrix(n, k)
+    x = np.eye(k, dtype=np.float32)
+    for m in (1, 2):
+        y = _swiglu_columns(q4k, wg, wu, n, k, m)
+        assert_swiglu_close(y, wg, wu, x, n, k, f"near-cancelling columns m={m}")

@@ -58,7 +58,8 @@ def check_plan(m, n, k):
     assert p["block"] <= (640 if (m == 1 and slices == 1) else 480) + 32
     assert 2 <= depth <= 8 and 1 <= teams <= 20
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
-    coef_per_warp = SEG * (4 * slices) * 4 * 16    # [seg][positions][4 groups] float4s
+    # [seg][positions][4 groups] float4 coefficients + float2 rounding errors
+    coef_per_warp = SEG * (4 * slices) * 4 * (16 + 8)
     need = (teams * depth * stage_bytes + teams * team_warps * coef_per_warp
             + teams * depth * 2 * team_warps * SEG * m * 4 + teams * 2 * m * 4)
     need = -(-need // 16) * 16 + cluster * teams * 32 + teams * 2 * depth * 8
@@ -195,7 +196,7 @@ def check_fused_plan(m, n, k):
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     rows_cap = -(-n // ctas)
     mi = min(m, 2)
-    need = (teams * depth * stage_bytes + teams * team_warps * SEG * 4 * 4 * 16
+    need = (teams * depth * stage_bytes + teams * team_warps * SEG * 4 * 4 * (16 + 8)
             + teams * depth * 2 * team_warps * SEG * mi * 4 + teams * 2 * mi * 4)
     need = -(-need // 16) * 16 + teams * 32 + teams * 2 * depth * 8
     need += -(-(mi * 2 * rows_cap * 4) // 16) * 16
