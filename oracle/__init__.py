@@ -89,6 +89,12 @@ class Oracle:
         L.q4k_oracle_embed_lookup.argtypes = [_u8p] + [ctypes.c_uint64] * 5 + [ctypes.c_float,
                                                                               _f32p]
         L.q4k_oracle_embed_lookup.restype = ctypes.c_int
+        L.q4k_oracle_float_to_half.argtypes = [ctypes.c_float]
+        L.q4k_oracle_float_to_half.restype = ctypes.c_uint16
+        L.q4k_oracle_floats_to_half.argtypes = [_f32p, ctypes.c_int64, _u16p]
+        L.q4k_oracle_floats_to_half.restype = None
+        L.q4k_oracle_dequant_f16.argtypes = [_u8p, ctypes.c_int64, ctypes.c_int64, _u16p]
+        L.q4k_oracle_dequant_f16.restype = None
         self.L = L
         self.path = path
 
@@ -163,6 +169,42 @@ class Oracle:
         self.L.q4k_oracle_gemv_rows(_p(w, _u8p), _p(x, _f32p), m, k, _p(rows, _i64p),
                                     rows.size, _p(y, _f64p), _p(a, _f64p))
         return y, a
+
+    def floats_to_half(self, x: np.ndarray) -> np.ndarray:
+        """binary16 RNE bit patterns (uint16) of float32 values, same shape."""
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        out = np.empty(x.shape, np.uint16)
+        self.L.q4k_oracle_floats_to_half(_p(x.reshape(-1), _f32p), x.size,
+                                         _p(out.reshape(-1), _u16p))
+        return out
+
+    def dequant_f16(self, w: np.ndarray, n: int, k: int) -> np.ndarray:
+        """The fp16 mirror of W: (n, k) uint16 binary16 bit patterns."""
+        w = np.ascontiguousarray(w, dtype=np.uint8).reshape(-1)
+        _check_shape(w, n, k)
+        out = np.empty((n, k), np.uint16)
+        self.L.q4k_oracle_dequant_f16(_p(w, _u8p), n, k, _p(out, _u16p))
+        return out
+
+    def half_values(self, bits: np.ndarray) -> np.ndarray:
+        """float64 values of binary16 bit patterns (through half_to_double)."""
+        table = np.array([self.half_to_double(b) for b in range(65536)], np.float64) \
+            if not hasattr(self, "_half_table") else self._half_table
+        self._half_table = table
+        return table[np.asarray(bits, np.uint16).astype(np.int64)]
+
+    def gemm_f16(self, w16: np.ndarray, x16: np.ndarray, rows=None):
+        """Prefill GEMM reference on fp16 operands ("memra-engine 0.83.1,
+        src/f16_ffi.rs", `memra_f16_pp_gemm_pre`: y = x16 W16^T, fp16 inputs,
+        f32 output): y[i][r] = sum_k w16[r][k] * x16[i][k] and a[i][r] =
+        sum_k |w16[r][k] * x16[i][k]|, both in float64 from the exact binary16
+        values (a double matmul: every product is exact, the sums are
+        double-rounded only). w16 (n, k) and x16 (m, k) are uint16 bit
+        patterns; `rows` restricts the output columns to those rows of W.
+        Returns (y, a), each (m, len(rows) or n) float64."""
+        wv = self.half_values(w16 if rows is None else np.asarray(w16)[np.asarray(rows)])
+        xv = self.half_values(x16)
+        return xv @ wv.T, np.abs(xv) @ np.abs(wv).T
 
     def embed_validate(self, table_bytes: int, rows: int, cols: int, hidden: int,
                        token: int) -> int:
@@ -255,6 +297,32 @@ def swiglu_tolerance(g, u, a_g, a_u, out):
     with np.errstate(over="ignore"):
         silu = np.abs(g / (1.0 + np.exp(-g)))
     return 1.1 * tg * (np.abs(u) + tu) + (silu + 1.1 * tg) * tu + 1e-6 * np.abs(out) + 1e-30
+
+
+def floats_to_half(x):
+    return default().floats_to_half(x)
+
+
+def dequant_f16(w, n, k):
+    return default().dequant_f16(w, n, k)
+
+
+def half_values(bits):
+    return default().half_values(bits)
+
+
+def gemm_f16(w16, x16, rows=None):
+    return default().gemm_f16(w16, x16, rows)
+
+
+def gemm_f16_tolerance(a: np.ndarray, k: int) -> np.ndarray:
+    """Per-element bound for a GPU fp16 GEMM with f32 accumulation against
+    `gemm_f16`: the products of two binary16 values are exact in f32 (22
+    significant bits), so the only error is the accumulation of k products in
+    f32: at most k * u * sum|w x| for recursive summation with unit roundoff u,
+    taken here as 2^-23 (twice f32's 2^-24, allowing accumulation by
+    truncation rather than rounding), plus 1e-6 for the final store."""
+    return k * 2.0 ** -23 * np.asarray(a) + 1e-6
 
 
 def tolerance(a: np.ndarray) -> np.ndarray:

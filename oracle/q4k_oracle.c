@@ -38,6 +38,7 @@
  * so d*sc, d*sc*q and dmin*m are exact in f32 and the only rounding is the final
  * subtraction: the value is the correctly rounded f32 of d*sc*q - dmin*m.
  * GEMV terms are (double)w * (double)x, summed in double, in k order.
+ * The fp16 mirror (end of file) rounds those f32 values once more, to binary16.
  *
  * Build: gcc -O2 -fPIC -shared -ffp-contract=off -fno-fast-math -pthread
  */
@@ -324,4 +325,75 @@ int q4k_oracle_embed_lookup(const uint8_t *table, uint64_t table_bytes, uint64_t
             out[b * QK + t] = (float)((double)wv[t] * (double)embed_scale);
     }
     return Q4K_ORACLE_EMBED_OK;
+}
+
+/* ------------------------------------------------------------------------
+ * fp16 mirror for the prefill GEMM ("memra-engine 0.83.1, src/f16_ffi.rs":
+ * module doc -- a resident fp16 dequant mirror of the trunk weights feeds an
+ * fp16 GEMM with f32 accumulation; `memra_q4_K_dequant_f16` turns Q4_K
+ * superblocks into the row-major fp16 mirror, `memra_f16_cvt` turns f32
+ * activations into fp16). Reading taken where the page is silent: a mirror
+ * value is the binary16 round-to-nearest-even of the f32 dequantised value
+ * above, and an activation is the binary16 RNE of its f32 value.
+ * ------------------------------------------------------------------------ */
+
+/* binary32 -> binary16 by the definition of round-to-nearest, ties-to-even:
+ * the finite binary16 value nearest to f, and on a tie the one whose last
+ * fraction bit is 0; a magnitude of at least 65520 (the largest finite value
+ * 65504 plus half of its ulp 32) becomes infinity. NaN becomes the quiet NaN
+ * 0x7E00 with f's sign. The nearest values are found by bisection over the
+ * positive finite bit patterns 0x0000..0x7BFF, which increase with the value. */
+uint16_t q4k_oracle_float_to_half(float f)
+{
+    uint16_t sign = signbit(f) ? 0x8000 : 0;
+    if (isnan(f))
+        return (uint16_t)(sign | 0x7E00);
+    double v = fabs((double)f);
+    if (v >= 65520.0)
+        return (uint16_t)(sign | 0x7C00);
+    int lo = 0, hi = 0x7BFF;          /* invariant: value(lo) <= v */
+    if (q4k_oracle_half_to_double((uint16_t)hi) <= v) {
+        lo = hi;
+    } else {
+        while (hi - lo > 1) {         /* value(lo) <= v < value(hi) */
+            int mid = (lo + hi) / 2;
+            if (q4k_oracle_half_to_double((uint16_t)mid) <= v)
+                lo = mid;
+            else
+                hi = mid;
+        }
+    }
+    double below = q4k_oracle_half_to_double((uint16_t)lo);
+    if (below == v)
+        return (uint16_t)(sign | lo);
+    double above = (lo == 0x7BFF) ? 65536.0 : q4k_oracle_half_to_double((uint16_t)(lo + 1));
+    double dlo = v - below, dhi = above - v;   /* exact: all three are doubles of few bits */
+    int pick;
+    if (dlo < dhi)
+        pick = lo;
+    else if (dhi < dlo)
+        pick = lo + 1;
+    else
+        pick = (lo & 1) ? lo + 1 : lo;        /* tie: the even bit pattern */
+    return (uint16_t)(sign | pick);
+}
+
+/* out[i] = binary16 RNE of x[i] (the f32 -> fp16 activation convert). */
+void q4k_oracle_floats_to_half(const float *x, int64_t count, uint16_t *out)
+{
+    for (int64_t i = 0; i < count; ++i)
+        out[i] = q4k_oracle_float_to_half(x[i]);
+}
+
+/* out[n][k] (row-major binary16 bit patterns) = the fp16 mirror of W. */
+void q4k_oracle_dequant_f16(const uint8_t *w, int64_t n, int64_t k, uint16_t *out)
+{
+    int64_t nsb = k / QK;
+    float v[QK];
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t b = 0; b < nsb; ++b) {
+            dequant_block(w + (r * nsb + b) * SB_BYTES, v);
+            for (int t = 0; t < QK; ++t)
+                out[r * k + b * QK + t] = q4k_oracle_float_to_half(v[t]);
+        }
 }

@@ -381,10 +381,90 @@ def check_swiglu_composition(o, seed=19):
         oracle_mod._default = saved
 
 
+# --------------------------------------------------------------------------- fp16 mirror
+
+def check_float_to_half_vs_numpy(o, seed=20):
+    """binary32 -> binary16 RNE against numpy's float32 -> float16 conversion (a
+    library routine) on random bit patterns, on every binary16 value, on the
+    midpoints between neighbouring binary16 values and just either side of them."""
+    rng = np.random.default_rng(seed)
+    h = np.arange(0x7C00, dtype=np.uint32).astype(np.uint16)
+    hv = h.view(np.float16).astype(np.float64)
+    mids = (hv[:-1] + hv[1:]) / 2                      # exact in float32 below 2^16
+    mids32 = mids.astype(np.float32)
+    assert np.array_equal(mids32.astype(np.float64), mids)
+    near = np.concatenate([np.nextafter(mids32, np.float32(0)), mids32,
+                           np.nextafter(mids32, np.float32(np.inf))])
+    rand = rng.integers(0, 2 ** 32, 400_000, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    special = np.array([0.0, -0.0, 65504, 65519.996, 65520, 65536, 1e30, -1e30, np.inf, -np.inf,
+                        2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -25, 2.0 ** -26, 1e-45, -1e-45],
+                       np.float32)
+    for x in (hv.astype(np.float32), near, rand, special, -near):
+        got = o.floats_to_half(x)
+        with np.errstate(over="ignore"):
+            ref = x.astype(np.float16).view(np.uint16)
+        nan = np.isnan(x)
+        assert np.array_equal(got[~nan], ref[~nan]), \
+            f"{int((got[~nan] != ref[~nan]).sum())} conversions differ from numpy"
+        assert np.all(np.isnan(got[nan].view(np.float16)))
+
+
+def check_float_to_half_known(o):
+    """Hand-derived roundings: ties go to the even bit pattern, 65520 overflows."""
+    table = {1.0: 0x3C00, 65504.0: 0x7BFF, 65519.99: 0x7BFF, 65520.0: 0x7C00,
+             2.0 ** -24: 0x0001, 2.0 ** -25: 0x0000, 3 * 2.0 ** -25: 0x0002,
+             5 * 2.0 ** -25: 0x0002, 1 + 2.0 ** -11: 0x3C00, 1 + 3 * 2.0 ** -11: 0x3C02,
+             -2.0: 0xC000, 2.0 ** -14: 0x0400, 1023 * 2.0 ** -24: 0x03FF,
+             (2047 / 2) * 2.0 ** -24: 0x0400}
+    for v, bits in table.items():
+        assert int(o.floats_to_half(np.array([v], np.float32))[0]) == bits, (v, hex(bits))
+
+
+def check_dequant_f16(o, seed=21):
+    """The mirror is the binary16 rounding of the pinned f32 dequantisation:
+    against numpy's conversion of the oracle's f32 values, and a closed form."""
+    n, k = 6, 512
+    w, _ = q4k_synth.q4k_problem(n, k, 1, seed)
+    got = o.dequant_f16(w, n, k)
+    assert np.array_equal(got, o.dequant_f32(w, n, k).astype(np.float16).view(np.uint16))
+    ff = np.full(12, 0xFF, np.uint8)
+    blk = _block(H_ONE, H_HALF, ff, np.full(128, 0xFF, np.uint8))   # every weight 913.5
+    assert np.all(o.dequant_f16(blk, 1, 256) == np.float16(913.5).view(np.uint16))
+    blk = _block(H_ONE, H_HALF, ff, np.zeros(128, np.uint8))        # every weight -31.5
+    assert np.all(o.dequant_f16(blk, 1, 256) == np.float16(-31.5).view(np.uint16))
+
+
+def check_gemm_f16(o, seed=22):
+    """fp16 GEMM reference: exact rational sums of the binary16 products on a
+    tiny problem, unit vectors giving columns, and |.| sums."""
+    rng = np.random.default_rng(seed)
+    n, m, k = 3, 2, 16
+    w16 = rng.integers(0, 0x7C00, (n, k)).astype(np.uint16) | \
+        (rng.integers(0, 2, (n, k)).astype(np.uint16) << 15)
+    x16 = rng.integers(0x2000, 0x5000, (m, k)).astype(np.uint16)
+    y, a = o.gemm_f16(w16, x16)
+    for i in range(m):
+        for r in range(n):
+            ex = sum(Fraction(float(np.uint16(w16[r, t]).view(np.float16))) *
+                     Fraction(float(np.uint16(x16[i, t]).view(np.float16))) for t in range(k))
+            ab = sum(abs(Fraction(float(np.uint16(w16[r, t]).view(np.float16))) *
+                         Fraction(float(np.uint16(x16[i, t]).view(np.float16)))) for t in range(k))
+            assert abs(Fraction(y[i, r]) - ex) <= abs(ex) * Fraction(1, 2 ** 50), (i, r)
+            assert abs(Fraction(a[i, r]) - ab) <= ab * Fraction(1, 2 ** 50), (i, r)
+    eye = np.zeros((k, k), np.uint16)
+    eye[np.arange(k), np.arange(k)] = 0x3C00                        # binary16 1.0
+    cols, _ = o.gemm_f16(w16, eye)
+    assert np.array_equal(cols, np.array([[float(np.uint16(b).view(np.float16)) for b in row]
+                                          for row in w16]).T)
+    sub, _ = o.gemm_f16(w16, x16, rows=[2, 0])
+    assert np.array_equal(sub, y[:, [2, 0]])
+
+
 ALL_CHECKS = [
     check_half_all_patterns, check_half_known, check_scale_bit_map, check_nibble_map,
     check_closed_forms, check_pack_roundtrip, check_unpack_pack_bytes, check_bruteforce_gemv,
     check_gemv_vs_matmul, check_unit_and_zero_vectors, check_vectors_independent,
     check_threads_and_rows, check_golden, check_embed_page_cases, check_embed_rules,
-    check_embed_values, check_swiglu_composition,
+    check_embed_values, check_swiglu_composition, check_float_to_half_vs_numpy,
+    check_float_to_half_known, check_dequant_f16, check_gemm_f16,
 ]

@@ -33,6 +33,13 @@ MUTANTS = {
     "embed_shape_rule_dropped": ("if (cols != hidden)\n        return Q4K_ORACLE_EMBED_SHAPE;", ""),
     "embed_scale_not_applied": ("(float)((double)wv[t] * (double)embed_scale)", "wv[t]"),
     "embed_wrong_row_stride": ("table + (token * nsb + b) * SB_BYTES", "table + (token + b) * SB_BYTES"),
+    "half_ties_to_odd": ("pick = (lo & 1) ? lo + 1 : lo;", "pick = (lo & 1) ? lo : lo + 1;"),
+    "half_ties_away": ("pick = (lo & 1) ? lo + 1 : lo;", "pick = lo + 1;"),
+    "half_truncates": ("    else if (dhi < dlo)\n        pick = lo + 1;\n", ""),
+    "half_overflow_early": ("if (v >= 65520.0)", "if (v >= 65504.0)"),
+    "half_nan_to_inf": ("return (uint16_t)(sign | 0x7E00);", "return (uint16_t)(sign | 0x7C00);"),
+    "mirror_row_stride_dropped": ("out[r * k + b * QK + t] = q4k_oracle_float_to_half(v[t]);",
+                                  "out[b * QK + t] = q4k_oracle_float_to_half(v[t]);"),
 }
 
 
