@@ -13,8 +13,8 @@ the GEMV needs no exchange); value sums the bytes of all ranks over the slowest
 rank's time. `--impl reference` times the CPU oracle instead (rank 0 only).
 Prints one JSON line on rank 0. Besides the contract keys it carries
 `per_shape` (µs per call of each projection: 200 back-to-back calls over
-rotating weight copies, median of 5 repeats, and the same with one copy,
-`l2_hot_us_per_call`, where W fits in L2) and `extra` (multi-vector,
+rotating weight copies replayed from a CUDA graph, median of 5 repeats, and the
+same with one copy, `l2_hot_us_per_call`, where W fits in L2) and `extra` (multi-vector,
 32-layer, fused SwiGLU and embedding figures).
 """
 from __future__ import annotations
@@ -231,6 +231,31 @@ def cpu_baseline() -> dict:
 
 # --------------------------------------------------------------------------- extra workloads
 
+def device_us_per_call(torch, dev, stream, call, reps: int = 100, warm: int = 10) -> float:
+    """Device time per call of call(0), ..., call(reps - 1) back to back,
+    captured in one CUDA graph and replayed (after a warm-up replay), timed with
+    CUDA events on `stream`: the host's launch rate never enters."""
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            call(i)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(reps):
+            call(i)
+    with torch.cuda.stream(stream):
+        g.replay()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    del g
+    return a0.elapsed_time(a1) * 1e3 / reps
+
+
 def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
     """The other decode workloads of the sweep's configuration list, on this GPU:
     multi-vector shapes (m = 1, 2, 4, 8, and the batches 16 and 32), the
@@ -244,18 +269,9 @@ def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
         for m in (1, 2, 4, 8, 16, 32):
             x = torch.from_numpy(q4k_synth.x_vectors(k, m, 77 + m)).to(dev)
             y = torch.empty((m, n), dtype=torch.float32, device=dev)
-            with torch.cuda.stream(stream):
-                for i in range(10):
-                    q4k.q4k_gemv(ws[i % len(ws)], x, y, m, n, k, stream=stream)
-            a0 = torch.cuda.Event(enable_timing=True)
-            a1 = torch.cuda.Event(enable_timing=True)
-            reps = 100
-            a0.record(stream)
-            for i in range(reps):
-                q4k.q4k_gemv(ws[i % len(ws)], x, y, m, n, k, stream=stream)
-            a1.record(stream)
-            torch.cuda.synchronize(dev)
-            us = a0.elapsed_time(a1) * 1e3 / reps
+            us = device_us_per_call(
+                torch, dev, stream,
+                lambda i: q4k.q4k_gemv(ws[i % len(ws)], x, y, m, n, k, stream=stream))
             b = bytes_counted(n, k, m)
             out["multivector"].append({"n": n, "k": k, "m": m, "us_per_call": round(us, 3),
                                        "gbs": round(b / us / 1e3, 1)})
@@ -332,6 +348,7 @@ def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
     del g, layers
     torch.cuda.empty_cache()
     out["embedding"] = embedding_workloads(q4k, torch, dev, stream)
+    out["prefill_f16"] = prefill_workloads(q4k, torch, dev, stream)
     out["swiglu"] = swiglu_workloads(q4k, torch, dev, stream, l2)
     return out
 
@@ -354,18 +371,7 @@ def swiglu_workloads(q4k, torch, dev, stream, l2: int) -> list:
             y2 = torch.empty((m, n), dtype=torch.float32, device=dev)
 
             def timed(fn):
-                with torch.cuda.stream(stream):
-                    for i in range(10):
-                        fn(i)
-                a0 = torch.cuda.Event(enable_timing=True)
-                a1 = torch.cuda.Event(enable_timing=True)
-                reps = 100
-                a0.record(stream)
-                for i in range(reps):
-                    fn(i)
-                a1.record(stream)
-                torch.cuda.synchronize(dev)
-                return a0.elapsed_time(a1) * 1e3 / reps
+                return device_us_per_call(torch, dev, stream, fn)
 
             fused = timed(lambda i: q4k.q4k_gemv_swiglu(gs[i % copies], us[i % copies], x, y, m,
                                                         n, k, stream=stream))
@@ -383,6 +389,61 @@ def swiglu_workloads(q4k, torch, dev, stream, l2: int) -> list:
     return res
 
 
+PREFILL_TOKENS = 512
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor peak in TFLOP/s: the measured cuBLAS bf16 burst
+    figure (fp16 has the same nominal rate), else the recipe's fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured bf16 burst"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback bf16 burst"
+
+
+def prefill_workloads(q4k, torch, dev, stream) -> dict:
+    """The prefill route on the 8B-class projections at m = 512 tokens: the
+    fp16 mirror (q4k_dequant_f16, GB/s of Q4_K read + fp16 written), the GEMM on
+    pre-converted activations (q4k_gemm_f16) and the one-call route with the
+    convert into the caller's scratch (q4k_prefill_f16), in TFLOP/s (2 m n k per
+    call) against the dense tensor peak. Device time of 20 calls from a CUDA
+    graph after 5 eager ones."""
+    peak, peak_kind = measured_tensor_peak()
+    m = PREFILL_TOKENS
+    res = []
+
+    def timed(fn, reps=20):
+        return device_us_per_call(torch, dev, stream, lambda _i: fn(), reps=reps, warm=5)
+
+    for n, k in [(4096, 4096), (1024, 4096), (14336, 4096), (4096, 14336)]:
+        w, _ = q4k_synth.q4k_problem(n, k, 1, 530 + n + k)
+        wd = torch.from_numpy(w).to(dev)
+        w16 = torch.empty((n, k), dtype=torch.float16, device=dev)
+        x = torch.from_numpy(q4k_synth.x_vectors(k, m, 531)).to(dev)
+        x16 = torch.empty((m, k), dtype=torch.float16, device=dev)
+        scratch = torch.empty(m * k * 2, dtype=torch.uint8, device=dev)
+        y = torch.empty((m, n), dtype=torch.float32, device=dev)
+        mirror_us = timed(lambda: q4k.q4k_dequant_f16(wd, w16, n, k, stream=stream))
+        q4k.q4k_f32_to_f16(x, x16, m * k, stream=stream)
+        gemm_us = timed(lambda: q4k.q4k_gemm_f16(w16, x16, y, m, n, k, stream=stream))
+        one_us = timed(lambda: q4k.q4k_prefill_f16(w16, x, scratch, y, m, n, k, stream=stream))
+        flops = 2.0 * m * n * k
+        res.append({"m": m, "n": n, "k": k,
+                    "gemm_us": round(gemm_us, 2), "gemm_tflops": round(flops / gemm_us / 1e6, 1),
+                    "gemm_frac_of_peak": round(flops / gemm_us / 1e6 / peak, 3),
+                    "prefill_call_us": round(one_us, 2),
+                    "prefill_call_tflops": round(flops / one_us / 1e6, 1),
+                    "mirror_us": round(mirror_us, 2),
+                    "mirror_gbs": round((n * k // 256 * 144 + 2 * n * k) / mirror_us / 1e3, 1)})
+        del wd, w16, x, x16, scratch, y
+    torch.cuda.empty_cache()
+    assert q4k.q4k_device_fault_flags() == 0
+    return {"tokens": m, "peak_tflops": peak, "peak_kind": peak_kind, "shapes": res}
+
+
 def embedding_workloads(q4k, torch, dev, stream) -> list:
     """Q4_K embedding lookups from a 128256 x 4096 table (an 8B model's token
     embedding): one token (q4k_embed_lookup_f32) and gathers of 8 and 512
@@ -397,25 +458,14 @@ def embedding_workloads(q4k, torch, dev, stream) -> list:
         toks = torch.from_numpy(rng.integers(0, rows, n_tok).astype(np.int32)).to(dev)
         out = torch.empty((n_tok, hidden), dtype=torch.float32, device=dev)
 
-        def call():
+        def call(_i):
             if n_tok == 1:
                 q4k.q4k_embed_lookup_f32(table, rows, hidden, hidden, 12345, 1.0, out,
                                          stream=stream)
             else:
                 q4k.q4k_embed_gather_f32(table, rows, hidden, toks, n_tok, 1.0, out,
                                          stream=stream)
-        with torch.cuda.stream(stream):
-            for _ in range(10):
-                call()
-        a0 = torch.cuda.Event(enable_timing=True)
-        a1 = torch.cuda.Event(enable_timing=True)
-        reps = 200
-        a0.record(stream)
-        for _ in range(reps):
-            call()
-        a1.record(stream)
-        torch.cuda.synchronize(dev)
-        us = a0.elapsed_time(a1) * 1e3 / reps
+        us = device_us_per_call(torch, dev, stream, call, reps=200)
         b = n_tok * (hidden // 256 * 144 + 4 * hidden)
         res.append({"rows": rows, "hidden": hidden, "tokens": n_tok,
                     "call": "q4k_embed_lookup_f32" if n_tok == 1 else "q4k_embed_gather_f32",
@@ -560,17 +610,10 @@ def run_ours(args) -> None:
     peak, peak_kind = measured_peak()
 
     def timed_calls(s, copies, reps=200):
-        with torch.cuda.stream(stream):
-            for i in range(10):
-                q4k.q4k_gemv(s["ws"][i % copies], s["x"], s["y"], 1, s["n"], s["k"], stream=stream)
-        a0 = torch.cuda.Event(enable_timing=True)
-        a1 = torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for i in range(reps):
-            q4k.q4k_gemv(s["ws"][i % copies], s["x"], s["y"], 1, s["n"], s["k"], stream=stream)
-        a1.record(stream)
-        torch.cuda.synchronize(dev)
-        return a0.elapsed_time(a1) * 1e3 / reps
+        return device_us_per_call(
+            torch, dev, stream,
+            lambda i: q4k.q4k_gemv(s["ws"][i % copies], s["x"], s["y"], 1, s["n"], s["k"],
+                                   stream=stream), reps=reps)
 
     for s, p in zip([] if args.skip_extras else shapes, plans):
         us = statistics.median(timed_calls(s, len(s["ws"])) for _ in range(5))
@@ -677,6 +720,8 @@ def main():
                     help="comma-separated NxK subset of the sweep (profiling runs only)")
     ap.add_argument("--skip-extras", action="store_true",
                     help="skip the per-shape and end-to-end passes (profiling runs only)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="print only the prefill (fp16 mirror + tensor-core GEMM) figures")
     args = ap.parse_args()
     if args.steps < 1 or args.warmup < 0:
         raise SystemExit("--steps must be >= 1 and --warmup >= 0")
@@ -688,7 +733,14 @@ def main():
                 raise SystemExit(f"shape {sh} is not one of the sweep's")
         BYTES_PER_STEP = sum(bytes_counted(n, k) for n, k in SWEEP)
         WORKLOAD = "subset of the sweep: " + ", ".join(f"{n}x{k}" for n, k in SWEEP)
-    if args.impl == "reference":
+    if args.prefill_only:
+        import torch
+        import gguf_quant_dequant_q4k_b200 as q4k
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps(prefill_workloads(q4k, torch, dev, torch.cuda.Stream(device=dev))),
+              flush=True)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

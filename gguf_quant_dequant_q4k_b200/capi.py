@@ -26,6 +26,7 @@ Q4K_FAULT_TOKEN_RANGE = 2
 Q4K_QK = 256
 Q4K_BLOCK_BYTES = 144
 Q4K_MAX_M = 64
+Q4K_GEMM_K_MULTIPLE = 64
 Q4K_KERNEL_WARP_ROWS = 1
 Q4K_KERNEL_STREAM = 2
 
@@ -33,7 +34,8 @@ Q4K_KERNEL_STREAM = 2
 EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
            "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags",
            "q4k_embed_lookup_f32", "q4k_embed_gather_f32", "q4k_gemv_swiglu",
-           "q4k_gemv_swiglu_plan_for", "q4k_selftest_wait_timeout")
+           "q4k_gemv_swiglu_plan_for", "q4k_selftest_wait_timeout", "q4k_dequant_f16",
+           "q4k_f32_to_f16", "q4k_gemm_f16", "q4k_prefill_f16")
 
 
 class Q4KError(RuntimeError):
@@ -91,6 +93,17 @@ _lib.q4k_embed_lookup_f32.restype = ctypes.c_int
 _lib.q4k_embed_gather_f32.argtypes = [_vp, ctypes.c_ulonglong, ctypes.c_int, ctypes.c_int, _vp,
                                       ctypes.c_int, ctypes.c_float, _vp, _vp]
 _lib.q4k_embed_gather_f32.restype = ctypes.c_int
+
+
+_lib.q4k_dequant_f16.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp]
+_lib.q4k_dequant_f16.restype = ctypes.c_int
+_lib.q4k_f32_to_f16.argtypes = [_vp, _vp, ctypes.c_ulonglong, _vp]
+_lib.q4k_f32_to_f16.restype = ctypes.c_int
+_lib.q4k_gemm_f16.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp]
+_lib.q4k_gemm_f16.restype = ctypes.c_int
+_lib.q4k_prefill_f16.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                 _vp]
+_lib.q4k_prefill_f16.restype = ctypes.c_int
 
 
 def library() -> ctypes.CDLL:
@@ -287,3 +300,68 @@ def q4k_embed_gather_f32(table, rows: int, hidden: int, tokens, n_tokens: int,
                                      stream, table_bytes)
     if st != Q4K_OK:
         raise Q4KError(st, "q4k_embed_gather_f32")
+
+
+# --------------------------------------------------------------------------- prefill (fp16)
+
+def _gemm_sizes_valid(m: int, n: int, k: int) -> bool:
+    return m > 0 and n > 0 and k > 0 and k % Q4K_GEMM_K_MULTIPLE == 0
+
+
+def q4k_dequant_f16_status(w, out, n: int, k: int, stream=None) -> int:
+    ok = q4k_weight_bytes(n, k) > 0
+    return _lib.q4k_dequant_f16(_ptr(w, None, "w", _need(q4k_weight_bytes(n, k), 1, ok)),
+                                _ptr(out, "float16", "out", _need(n * k, 2, ok)), int(n), int(k),
+                                _stream(stream))
+
+
+def q4k_dequant_f16(w, out, n: int, k: int, stream=None) -> None:
+    """out[n, k] (float16) = the fp16 mirror of the Q4_K matrix W."""
+    st = q4k_dequant_f16_status(w, out, n, k, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_dequant_f16")
+
+
+def q4k_f32_to_f16_status(x, out, count: int, stream=None) -> int:
+    ok = count > 0
+    return _lib.q4k_f32_to_f16(_ptr(x, "float32", "x", _need(count, 4, ok)),
+                               _ptr(out, "float16", "out", _need(count, 2, ok)), int(count),
+                               _stream(stream))
+
+
+def q4k_f32_to_f16(x, out, count: int, stream=None) -> None:
+    """out[:count] (float16) = RNE binary16 of x[:count] (float32)."""
+    st = q4k_f32_to_f16_status(x, out, count, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_f32_to_f16")
+
+
+def q4k_gemm_f16_status(w16, x16, y, m: int, n: int, k: int, stream=None) -> int:
+    ok = _gemm_sizes_valid(m, n, k)
+    return _lib.q4k_gemm_f16(_ptr(w16, "float16", "w_f16", _need(n * k, 2, ok)),
+                             _ptr(x16, "float16", "x_f16", _need(m * k, 2, ok)),
+                             _ptr(y, "float32", "y", _need(m * n, 4, ok)), int(m), int(n), int(k),
+                             _stream(stream))
+
+
+def q4k_gemm_f16(w16, x16, y, m: int, n: int, k: int, stream=None) -> None:
+    """y[m, n] = x16[m, k] @ w16[n, k]^T (fp16 operands, f32 accumulation and output)."""
+    st = q4k_gemm_f16_status(w16, x16, y, m, n, k, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_gemm_f16")
+
+
+def q4k_prefill_f16_status(w16, x, scratch, y, m: int, n: int, k: int, stream=None) -> int:
+    ok = _gemm_sizes_valid(m, n, k)
+    return _lib.q4k_prefill_f16(_ptr(w16, "float16", "w_f16", _need(n * k, 2, ok)),
+                                _ptr(x, "float32", "x", _need(m * k, 4, ok)),
+                                _ptr(scratch, None, "x_f16_scratch", _need(m * k, 2, ok)),
+                                _ptr(y, "float32", "y", _need(m * n, 4, ok)), int(m), int(n),
+                                int(k), _stream(stream))
+
+
+def q4k_prefill_f16(w16, x, scratch, y, m: int, n: int, k: int, stream=None) -> None:
+    """y[m, n] = fp16(x[m, k]) @ w16[n, k]^T; `scratch` (m*k*2 bytes) receives fp16(x)."""
+    st = q4k_prefill_f16_status(w16, x, scratch, y, m, n, k, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_prefill_f16")

@@ -68,6 +68,8 @@ int current_device_info(DeviceInfo* info) {
                                                 : static_cast<int>(e2);
         if (g_dev_status[dev] == 0 && stream_set_attributes() != Q4K_OK)
             g_dev_status[dev] = q4k_last_cuda_error_value();
+        if (g_dev_status[dev] == 0 && gemm_set_attributes() != Q4K_OK)
+            g_dev_status[dev] = q4k_last_cuda_error_value();
         if (g_dev_status[dev] == 0) {
             stream_cluster_occupancy(1, g_dev[dev].max_clusters[0]);
             stream_cluster_occupancy(2, g_dev[dev].max_clusters[1]);
@@ -104,12 +106,14 @@ int q4k_last_cuda_error(void) { return t_last_cuda_error; }
 
 int q4k_device_fault_flags(unsigned int* flags) {
     if (flags == nullptr) return Q4K_ERR_NULL;
-    unsigned a = 0, b = 0;
+    unsigned a = 0, b = 0, c = 0;
     int st = read_fault_flags(&a);
     if (st != Q4K_OK) return st;
     st = read_embed_fault_flags(&b);
     if (st != Q4K_OK) return st;
-    *flags = a | b;
+    st = read_gemm_fault_flags(&c);
+    if (st != Q4K_OK) return st;
+    *flags = a | b | c;
     return Q4K_OK;
 }
 
@@ -225,6 +229,81 @@ int q4k_dequant_f32(const void* w, float* out, int n, int k, q4k_stream_t stream
     int st = current_device_info(&dev);
     if (st != Q4K_OK) return st;
     return launch_dequant(w, out, n, k, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4k_dequant_f16(const void* w, void* out, int n, int k, q4k_stream_t stream) {
+    if (w == nullptr || out == nullptr) return Q4K_ERR_NULL;
+    const size_t wbytes = weight_bytes_checked(n, k);
+    if (wbytes == 0) return Q4K_ERR_SHAPE;
+    if (!aligned(w, 16) || !aligned(out, 16)) return Q4K_ERR_ALIGN;
+    const size_t obytes = static_cast<size_t>(n) * static_cast<size_t>(k) * 2;
+    if (overlaps(out, obytes, w, wbytes)) return Q4K_ERR_OVERLAP;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return launch_dequant_f16(w, out, n, k, dev.sm_count, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4k_f32_to_f16(const float* x, void* out, unsigned long long count, q4k_stream_t stream) {
+    if (x == nullptr || out == nullptr) return Q4K_ERR_NULL;
+    if (count > (1ull << 62)) return Q4K_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(out, 16)) return Q4K_ERR_ALIGN;
+    if (overlaps(out, static_cast<size_t>(count) * 2, x, static_cast<size_t>(count) * 4))
+        return Q4K_ERR_OVERLAP;
+    if (count == 0) return Q4K_OK;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return launch_f32_to_f16(x, out, static_cast<long long>(count), dev.sm_count,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+// Shape and pointer checks shared by the two GEMM entry points.
+int check_gemm(const void* w16, const void* x16, const float* y, int m, int n, int k) {
+    if (w16 == nullptr || x16 == nullptr || y == nullptr) return Q4K_ERR_NULL;
+    if (m <= 0 || n <= 0 || k <= 0 || k % Q4K_GEMM_K_MULTIPLE != 0) return Q4K_ERR_SHAPE;
+    if (!aligned(w16, 16) || !aligned(x16, 16) || !aligned(y, 4)) return Q4K_ERR_ALIGN;
+    const size_t wbytes = static_cast<size_t>(n) * static_cast<size_t>(k) * 2;
+    const size_t xbytes = static_cast<size_t>(m) * static_cast<size_t>(k) * 2;
+    const size_t ybytes = static_cast<size_t>(m) * static_cast<size_t>(n) * 4;
+    if (overlaps(y, ybytes, w16, wbytes) || overlaps(y, ybytes, x16, xbytes)) return Q4K_ERR_OVERLAP;
+    return Q4K_OK;
+}
+
+}  // namespace
+
+int q4k_gemm_f16(const void* w_f16, const void* x_f16, float* y, int m, int n, int k,
+                 q4k_stream_t stream) {
+    int st = check_gemm(w_f16, x_f16, y, m, n, k);
+    if (st != Q4K_OK) return st;
+    DeviceInfo dev;
+    st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    return launch_gemm_f16(w_f16, x_f16, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int q4k_prefill_f16(const void* w_f16, const float* x, void* x_f16_scratch, float* y, int m, int n,
+                    int k, q4k_stream_t stream) {
+    if (x == nullptr) return Q4K_ERR_NULL;
+    int st = check_gemm(w_f16, x_f16_scratch, y, m, n, k);
+    if (st != Q4K_OK) return st;
+    if (!aligned(x, 16)) return Q4K_ERR_ALIGN;
+    const size_t xbytes = static_cast<size_t>(m) * static_cast<size_t>(k) * 4;
+    const size_t hbytes = static_cast<size_t>(m) * static_cast<size_t>(k) * 2;
+    const size_t wbytes = static_cast<size_t>(n) * static_cast<size_t>(k) * 2;
+    const size_t ybytes = static_cast<size_t>(m) * static_cast<size_t>(n) * 4;
+    if (overlaps(x_f16_scratch, hbytes, x, xbytes) || overlaps(x_f16_scratch, hbytes, w_f16, wbytes) ||
+        overlaps(y, ybytes, x, xbytes))
+        return Q4K_ERR_OVERLAP;
+    DeviceInfo dev;
+    st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = launch_f32_to_f16(x, x_f16_scratch, static_cast<long long>(m) * k, dev.sm_count, s);
+    if (st != Q4K_OK) return st;
+    return launch_gemm_f16(w_f16, x_f16_scratch, y, m, n, k, s);
 }
 
 }  // extern "C"

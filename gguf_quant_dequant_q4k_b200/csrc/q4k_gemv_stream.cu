@@ -749,18 +749,32 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
                 bool fused, StreamParams* sp, int* grid, int* block, int* smem_bytes) {
     const int nsb = k / kQK;
     if (m < 1 || m > kStreamMaxM || n < 1) return 0;
-    // quant slices per lane: two for one vector on very tall matrices, and for
-    // one vector when K is too long for one-slice teams (K > 20480: a team of
-    // two-slice lanes covers K <= 30720 with 15 warps)
+    // Compact CTAs: at most half of an SM's registers and shared memory, so
+    // that a CTA of the next kernel on the stream can be resident beside it
+    // (programmatic dependent launch then runs its prologue and first weight
+    // copies while this one finishes), with up to kCompactCtasPerSm per SM.
+    const bool compact_ok = kPlanMode != 0;
+    // quant slices per lane: two for one vector on very tall matrices, for one
+    // vector when K is too long for one-slice teams (K > 20480: a team of
+    // two-slice lanes covers K <= 30720 with 15 warps), and for a compact CTA
+    // whose one-slice team would not fit its warps
+    const int compact_warps1 = kCompactRegs / (stream_max_regs(m, 1) * 32) - 1;
+    const bool compact_s1 = compact_ok && (nsb * 8 + 31) / 32 <= compact_warps1;
+    const bool compact_s2 = compact_ok && m == 1 && !fused &&
+                            (nsb * 4 + 31) / 32 <= kCompactRegs / (stream_max_regs(1, 2) * 32) - 1;
+    const bool compact = compact_s1 || compact_s2;
     const bool wide = m == 1 && !fused &&
-                      ((n + num_sms - 1) / num_sms >= kWideMinRows || nsb > kStreamMaxNsb);
+                      ((n + num_sms - 1) / num_sms >= kWideMinRows || nsb > kStreamMaxNsb ||
+                       (compact && !compact_s1));
     const int sl = wide ? 2 : 1;
     if (nsb > kStreamMaxNsb * sl) return 0;
     const int team_warps = (nsb * 8 / sl + 31) / 32;   // 8*nsb slices / (32 lanes * sl)
-    const int max_warps = stream_max_threads(m, sl) / 32;
+    const int max_warps = compact ? kCompactRegs / (stream_max_regs(m, sl) * 32) - 1
+                                  : stream_max_threads(m, sl) / 32;
     if (team_warps > max_warps) return 0;
     int teams = max_warps / team_warps;
     if (teams > kStreamMaxTeams) teams = kStreamMaxTeams;
+    const int per_sm = compact ? kCompactCtasPerSm : 1;
     // Cluster size. Within a CTA the warps of a team already split K, so a
     // row of any supported K is processed by up to 20 warps at once; splitting
     // rows across the CTAs of a cluster (split-K) adds a cluster launch and two
@@ -768,8 +782,8 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     // off only for a handful of very long rows (N = 1, K = 14336: 7.2 -> 6.7
     // us with clusters of 2). So: clusters of two CTAs for N < 8 and K >= 8192.
     int cluster = 1;
-    int clusters = n < resident_clusters(1, num_sms, max_clusters)
-                       ? n : resident_clusters(1, num_sms, max_clusters);
+    const int resident1 = compact ? per_sm * num_sms : resident_clusters(1, num_sms, max_clusters);
+    int clusters = n < resident1 ? n : resident1;
     if (!fused && n < kClusterMaxRows && nsb >= kClusterMinNsb &&
         resident_clusters(2, num_sms, max_clusters) >= n) {
         cluster = 2;
@@ -781,8 +795,8 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     const int rows_cap = (n + clusters - 1) / clusters;
     const long long rows_bytes = fused ? (static_cast<long long>(m) * 2 * rows_cap * 4 + 15) / 16 * 16 : 0;
     if (rows_bytes > kStreamMaxRowsBytes) return 0;
-    const int budget = (max_smem < kStreamSmemBudget ? max_smem : kStreamSmemBudget) - 1024 -
-                       static_cast<int>(rows_bytes);
+    const int cap = compact ? kCompactSmem : kStreamSmemBudget;
+    const int budget = (max_smem < cap ? max_smem : cap) - 1024 - static_cast<int>(rows_bytes);
     // bytes per team besides its ring: coefficient buffers of its warps, the
     // partial sums per slot and ring phase, its cut-row partials, its entries of the cluster's
     // team-range table and two barriers per slot
@@ -790,13 +804,23 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
         return team_warps * coef_bytes_per_warp(sl) + depth * 2 * team_warps * kSeg * m * 4 +
                2 * m * 4 + cluster * kTeamRangeBytes + 2 * depth * 8 + 16;
     };
-    int depth = kStreamMaxDepth;
+    // A team never needs more slots than it has stages: a team's range is
+    // ceil(rows * nsb / teams) superblocks at most, touching at most
+    // ceil(that / nsb) + 1 row segments.
+    auto max_depth = [&](int t) {
+        const long long len = (static_cast<long long>(rows_cap) * (fused ? 2 : 1) * nsb +
+                               t * cluster - 1) / (t * cluster);
+        const long long segs = (len + nsb - 1) / nsb + 1;
+        const long long st = (segs + kSeg - 1) / kSeg;
+        return static_cast<int>(st < 2 ? 2 : (st > kStreamMaxDepth ? kStreamMaxDepth : st));
+    };
+    int depth = max_depth(teams);
     while (depth >= 2 && teams * (depth * stage_bytes + fixed_team(depth)) > budget) {
         if (depth > 2) {
             --depth;
         } else if (teams > 1) {
             --teams;
-            depth = kStreamMaxDepth;
+            depth = max_depth(teams);
         } else {
             break;
         }

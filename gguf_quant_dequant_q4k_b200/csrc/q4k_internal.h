@@ -44,4 +44,14 @@ int launch_embed(const void* table, long long rows, int hidden, const int* token
 // Reads and clears the embedding kernel's fault flags (synchronises).
 int read_embed_fault_flags(unsigned* flags);
 
+// Prefill path (fp16 mirror + tensor-core GEMM). Arguments are validated.
+int gemm_set_attributes();
+int gemm_tile_tokens(int m);     // tokens per CTA tile of the GEMM (128 or 256)
+int launch_gemm_f16(const void* w16, const void* x16, float* y, int m, int n, int k,
+                    cudaStream_t stream);
+int launch_f32_to_f16(const float* x, void* out, long long count, int num_sms,
+                      cudaStream_t stream);
+int launch_dequant_f16(const void* w, void* out, int n, int k, int num_sms, cudaStream_t stream);
+int read_gemm_fault_flags(unsigned* flags);
+
 }  // namespace q4k

@@ -56,6 +56,18 @@ struct StreamParams {
     int slices;                 // 16-byte quant slices per lane (1 or 2)
 };
 
+// Launch policy. 0: one CTA per SM with up to 20 compute warps and 220 KiB
+// of shared memory. 1 / 2: compact CTAs (at most kCompactRegs registers and
+// kCompactSmem bytes of shared memory, so that a CTA of the next kernel can be
+// resident beside each one) wherever a team fits, kCompactCtasPerSm per SM.
+#ifndef Q4K_PLAN_MODE
+#define Q4K_PLAN_MODE 0
+#endif
+constexpr int kPlanMode = Q4K_PLAN_MODE;
+constexpr int kCompactRegs = 32768;
+constexpr int kCompactSmem = 112 * 1024;
+constexpr int kCompactCtasPerSm = (Q4K_PLAN_MODE == 1) ? 2 : 1;
+
 constexpr int kStreamMaxCluster = 8;    // cluster sizes the kernel supports (portable limit)
 constexpr int kClusterMaxRows = 8;      // split rows across a cluster only for N < 8 ...
 constexpr int kClusterMinNsb = 32;      // ... and K >= 8192

@@ -1,0 +1,122 @@
+// q4k_tcgen05.cuh -- sm_100a tensor-core primitives for the fp16 prefill GEMM:
+// TMA tensor loads (cp.async.bulk.tensor, no multicast), tcgen05 MMA issued by
+// one thread with its accumulator in tensor memory (TMEM), commits to
+// mbarriers, TMEM allocation and loads, and the shared-memory / instruction
+// descriptors the MMA reads.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "q4k_sm100.cuh"
+
+namespace q4k {
+
+// --------------------------------------------------------------------- TMA
+
+// 2-D tiled tensor load of the box at element coordinates (x = innermost, y)
+// into shared memory, completing on `bar` (transaction bytes). x * element
+// size must be a multiple of 16 bytes; callers pass x as a multiple of 64
+// fp16 elements.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// --------------------------------------------------------------------- TMEM
+
+// Allocates `ncols` (a power of two >= 32) TMEM columns for the CTA; the
+// address lands in *slot (shared memory). Whole warp, converged.
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of the calling thread's lane (lane
+// quarter = warp % 4), starting at taddr = base + (lane0 << 16) + column.
+__device__ __forceinline__ void tmem_load_32cols(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// --------------------------------------------------------------------- MMA
+
+// Shared-memory matrix descriptor of a K-major operand tile stored with the
+// 128-byte swizzle that TMA's CU_TENSOR_MAP_SWIZZLE_128B writes: rows of 64
+// fp16 (128 bytes), groups of 8 rows 1024 bytes apart (stride byte offset),
+// tile base 1024-byte aligned (base offset 0). Fields: start address >> 4
+// (bits 0-13), leading byte offset >> 4 = 1 (bits 16-29; not used by the
+// swizzled K-major layout), stride byte offset >> 4 = 64 (bits 32-45),
+// descriptor version 1 (bits 46-47), swizzle mode 2 = 128 B (bits 61-63).
+// Stepping K by 16 elements inside the 128-byte row adds 32 bytes to the start
+// address: the hardware applies the swizzle to the absolute address bits.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_byte_addr) {
+    return static_cast<uint64_t>((smem_byte_addr & 0x3FFFFu) >> 4) | (1ull << 16) |
+           (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16 with fp16 A and B, f32
+// accumulator, both operands K-major, shape M x N: D format f32 (bits 4-5 =
+// 1), A and B format fp16 (bits 7-9, 10-12 = 0), N >> 3 (bits 17-22), M >> 4
+// (bits 24-28).
+__host__ __device__ constexpr uint32_t mma_f16_idesc(int m, int n) {
+    return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// D (TMEM) = A * B^T (+ D if accumulate): A M x 16 and B N x 16, K-major, fp16.
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// `bar` receives one arrival once every tcgen05.mma this thread issued before
+// has completed (its shared-memory operands are free again, its results are in
+// TMEM).
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+
+}  // namespace q4k

@@ -75,12 +75,14 @@ enum q4k_status {
 };
 
 /* Bits of q4k_device_fault_flags(). */
-#define Q4K_FAULT_COPY_TIMEOUT 1u  /* a bounded wait on a bulk copy gave up          */
+#define Q4K_FAULT_COPY_TIMEOUT 1u  /* a bounded wait on a bulk copy, a tensor copy or an
+                                      MMA commit gave up                               */
 #define Q4K_FAULT_TOKEN_RANGE 2u   /* q4k_embed_gather_f32 met a token outside the table */
 
 #define Q4K_QK 256          /* weights per superblock */
 #define Q4K_BLOCK_BYTES 144 /* bytes per superblock   */
 #define Q4K_MAX_M 64        /* most vectors per q4k_gemv call */
+#define Q4K_GEMM_K_MULTIPLE 64 /* q4k_gemm_f16 / q4k_prefill_f16: k % 64 == 0 */
 
 /*
  * y = W x for m vectors.
@@ -255,6 +257,66 @@ enum q4k_kernel {
 };
 
 Q4K_API int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan *plan);
+
+/*
+ * ---- Prefill path: fp16 mirror + tensor-core GEMM ----
+ * "memra-engine 0.83.1, src/f16_ffi.rs" (module doc): for prefill (m >= 512
+ * tokens) the weights are dequantised once into a resident fp16 mirror and
+ * each projection is an fp16 GEMM with f32 accumulation; activations are
+ * converted f32 -> fp16 first. The page calls cuBLASLt; here the GEMM is a
+ * hand-written tcgen05 kernel. Its accuracy contract differs from q4k_gemv's:
+ * the operands are rounded to binary16 (relative error up to 2^-11 each), and
+ * against the exact products of the fp16 operands the result satisfies, per
+ * element, |y - sum_k w16 x16| <= k * 2^-23 * sum_k |w16 x16| + 1e-6.
+ */
+
+/*
+ * out = the fp16 mirror of W: row-major n x k binary16, out[r*k + t] = the
+ * round-to-nearest-even binary16 of weight t of row r's f32 value
+ * d*sc*q - dmin*m (that value is itself rounded once), so results are
+ * bit-reproducible (`memra_q4_K_dequant_f16`, called from `build_q4k_f16_raw`
+ * with (w, dst, out_f, nsb_row, stream)).
+ *   w  : as for q4k_gemv (16-byte aligned).
+ *   out: n*k*2 bytes, 16-byte aligned, must not overlap w.
+ * Values beyond binary16's range become +-inf.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_dequant_f16(const void *w, void *out, int n, int k, q4k_stream_t stream);
+
+/*
+ * out[i] = binary16 round-to-nearest-even of x[i], i < count (`memra_f16_cvt`:
+ * the standalone f32 -> fp16 activation convert, one convert feeding several
+ * GEMMs). x and out 16-byte aligned, not overlapping. count == 0 launches
+ * nothing. Returns a q4k_status.
+ */
+Q4K_API int q4k_f32_to_f16(const float *x, void *out, unsigned long long count,
+                           q4k_stream_t stream);
+
+/*
+ * y = x16 * W16^T (`memra_f16_pp_gemm_pre`: the GEMM on pre-converted fp16
+ * activations, "TN": both operands K-major).
+ *   w_f16: n x k binary16, row-major (the mirror), 16-byte aligned.
+ *   x_f16: m x k binary16, row-major (token-major), 16-byte aligned.
+ *   y    : m x n float32, row-major, fully overwritten, must not overlap
+ *          either operand.
+ *   m, n >= 1; k >= 64 and a multiple of Q4K_GEMM_K_MULTIPLE (64).
+ * Accuracy: see the block comment above. Returns a q4k_status.
+ */
+Q4K_API int q4k_gemm_f16(const void *w_f16, const void *x_f16, float *y, int m, int n, int k,
+                         q4k_stream_t stream);
+
+/*
+ * y = fp16(x) * W16^T in one call (`memra_f16_pp_gemm`: f32 -> fp16 convert
+ * into a caller-provided scratch, then the GEMM, on one stream).
+ *   x            : m x k float32, row-major, 16-byte aligned.
+ *   x_f16_scratch: m*k*2 bytes of device memory the caller owns, 16-byte
+ *                  aligned; overwritten with fp16(x) (the GEMM's B operand);
+ *                  must not overlap x, w_f16 or y.
+ *   w_f16, y, m, n, k: as for q4k_gemm_f16.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_prefill_f16(const void *w_f16, const float *x, void *x_f16_scratch, float *y,
+                            int m, int n, int k, q4k_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -211,3 +211,41 @@ def test_binding_refuses_host_tensors():
         capi.q4k_dequant_f32_status(A16, f32, 1, 256, stream=0)
     with pytest.raises(ValueError):
         capi.q4k_gemv_swiglu_status(A16, w, A16 * 2, A16 * 4, 1, 1, 256, stream=0)
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((0, A16, A16 * 2, 4, 8, 64), q4k.Q4K_ERR_NULL),
+    ((A16, 0, A16 * 2, 4, 8, 64), q4k.Q4K_ERR_NULL),
+    ((A16, A16 * 2, 0, 4, 8, 64), q4k.Q4K_ERR_NULL),
+    ((A16, A16 * 2, A16 * 3, 0, 8, 64), q4k.Q4K_ERR_SHAPE),
+    ((A16, A16 * 2, A16 * 3, 4, 0, 64), q4k.Q4K_ERR_SHAPE),
+    ((A16, A16 * 2, A16 * 3, 4, 8, 32), q4k.Q4K_ERR_SHAPE),
+    ((A16, A16 * 2, A16 * 3, 4, 8, 0), q4k.Q4K_ERR_SHAPE),
+    ((A16 + 8, A16 * 2, A16 * 3, 4, 8, 64), q4k.Q4K_ERR_ALIGN),
+    ((A16, A16 * 2 + 8, A16 * 3, 4, 8, 64), q4k.Q4K_ERR_ALIGN),
+    ((A16, A16 * 2, A16 * 3 + 2, 4, 8, 64), q4k.Q4K_ERR_ALIGN),
+    ((A16, A16 * 2, A16 + 64, 4, 8, 64), q4k.Q4K_ERR_OVERLAP),        # y inside w16
+    ((A16, A16 * 2, A16 * 2 + 64, 4, 8, 64), q4k.Q4K_ERR_OVERLAP),    # y inside x16
+])
+def test_gemm_f16_validation(args, expect):
+    assert q4k.q4k_gemm_f16_status(*args, stream=0) == expect
+
+
+def test_prefill_and_convert_validation():
+    # scratch overlapping x, w16 or y; x misaligned; null x
+    assert q4k.q4k_prefill_f16_status(A16, A16 * 2, A16 * 2 + 16, A16 * 4, 4, 8, 64,
+                                      stream=0) == q4k.Q4K_ERR_OVERLAP
+    assert q4k.q4k_prefill_f16_status(A16, A16 * 2, A16 + 16, A16 * 4, 4, 8, 64,
+                                      stream=0) == q4k.Q4K_ERR_OVERLAP
+    assert q4k.q4k_prefill_f16_status(A16, A16 * 2 + 4, A16 * 3, A16 * 4, 4, 8, 64,
+                                      stream=0) == q4k.Q4K_ERR_ALIGN
+    assert q4k.q4k_prefill_f16_status(A16, 0, A16 * 3, A16 * 4, 4, 8, 64,
+                                      stream=0) == q4k.Q4K_ERR_NULL
+    assert q4k.q4k_prefill_f16_status(A16, A16 * 2, A16 * 3, A16 * 4, 4, 8, 100,
+                                      stream=0) == q4k.Q4K_ERR_SHAPE
+    assert q4k.q4k_f32_to_f16_status(A16, A16 + 8, 16, stream=0) == q4k.Q4K_ERR_ALIGN
+    assert q4k.q4k_f32_to_f16_status(A16, A16 + 16, 16, stream=0) == q4k.Q4K_ERR_OVERLAP
+    assert q4k.q4k_f32_to_f16_status(0, A16, 16, stream=0) == q4k.Q4K_ERR_NULL
+    assert q4k.q4k_dequant_f16_status(A16, A16 * 2, 4, 255, stream=0) == q4k.Q4K_ERR_SHAPE
+    assert q4k.q4k_dequant_f16_status(A16, A16 + 16, 4, 256, stream=0) == q4k.Q4K_ERR_OVERLAP
+    assert q4k.q4k_dequant_f16_status(A16, A16 * 2 + 8, 4, 256, stream=0) == q4k.Q4K_ERR_ALIGN
