@@ -75,7 +75,8 @@ namespace {
 // q4k_device_fault_flags(). Never set in normal operation.
 __device__ unsigned int g_fault_flags = 0;
 
-constexpr int kSeg = kStreamSegRows;         // row segments per stage
+constexpr int kSeg = kStreamSegRows;         // row segments per stage (a multiple of 4)
+static_assert(kSeg % 4 == 0, "stages hold groups of four row segments");
 constexpr unsigned kXIssuedBarrier = 1;      // named barrier: compute warps issued x loads
 constexpr uint32_t kMagicOne = 0x3F000000u;  // 1/2: bytes 0..2 = 0x00, byte 3 = 0x3F
 constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
@@ -572,22 +573,26 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             if (!abort_flag && !mbar_wait_bounded(&T.full[slot], phase, &g_fault_flags))
                 abort_flag = 1;
 
-            // Decode this warp's superblock headers of the stage.
-            {
-                const int idx = du * nsb + dbl - head;
+            // Decode this warp's superblock headers of the stage (segments
+            // du, du + 4, ...).
+#pragma unroll
+            for (int dg = 0; dg < kSeg / 4; ++dg) {
+                const int idx = (du + 4 * dg) * nsb + dbl - head;
                 if (dbl < nsb && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage)) {
                     const uint4 hdr = *reinterpret_cast<const uint4*>(
                         smem + st_off + static_cast<uint32_t>(idx) * kBlockBytes);
                     float d, dmin;
                     header_scales(hdr, d, dmin);
+                    const uint32_t cb = dec_base + static_cast<uint32_t>(dg * 4 * kPos * 4 * 16);
+                    const uint32_t eb = dec_err + static_cast<uint32_t>(dg * 4 * kPos * 4 * 8);
 #pragma unroll
                     for (int hh = 0; hh < S; ++hh) {
                         const int half = S == 2 ? hh : dhalf;
                         float4 c_a, c_b, c_e;
                         decode_half(hdr, d, dmin, half, c_a, c_b, c_e);
-                        *reinterpret_cast<float4*>(smem + dec_base + ((2 * half) ^ dswz) * 16) = c_a;
-                        *reinterpret_cast<float4*>(smem + dec_base + ((2 * half + 1) ^ dswz) * 16) = c_b;
-                        *reinterpret_cast<float4*>(smem + dec_err + half * 16) = c_e;
+                        *reinterpret_cast<float4*>(smem + cb + ((2 * half) ^ dswz) * 16) = c_a;
+                        *reinterpret_cast<float4*>(smem + cb + ((2 * half + 1) ^ dswz) * 16) = c_b;
+                        *reinterpret_cast<float4*>(smem + eb + half * 16) = c_e;
                     }
                 }
             }
@@ -660,11 +665,15 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             float* rbuf = T.red + static_cast<size_t>(slot * 2 + phase) * red_slot;
 #pragma unroll
             for (int i = 0; i < M; ++i) {
-                const float r = transpose_reduce4(part_sum[i][0], part_sum[i][1], part_sum[i][2],
-                                                  part_sum[i][3], lane);
-                if ((lane & 7) == 0) {
-                    const int u = ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
-                    rbuf[(wit * M + i) * kSeg + u] = r;
+#pragma unroll
+                for (int q = 0; q < kSeg / 4; ++q) {
+                    const float r = transpose_reduce4(part_sum[i][4 * q], part_sum[i][4 * q + 1],
+                                                      part_sum[i][4 * q + 2], part_sum[i][4 * q + 3],
+                                                      lane);
+                    if ((lane & 7) == 0) {
+                        const int u = 4 * q + ((lane >> 4) & 1) * 2 + ((lane >> 3) & 1);
+                        rbuf[(wit * M + i) * kSeg + u] = r;
+                    }
                 }
             }
             __syncwarp();

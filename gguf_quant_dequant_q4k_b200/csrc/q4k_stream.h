@@ -6,7 +6,10 @@
 
 namespace q4k {
 
-constexpr int kStreamSegRows = 4;       // row segments per ring stage
+// Row segments per ring stage (a multiple of 4). Measured on B200: 8 is
+// slower than 4 on every decode shape (register spills, LM head 101.7 ->
+// 110.3 us).
+constexpr int kStreamSegRows = 4;
 constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kernel
 // Quant slices (16 bytes = 32 weights) per lane and row: 1, or 2 for one
 // vector on very tall matrices (kWideMinRows rows or more per CTA: an LM
