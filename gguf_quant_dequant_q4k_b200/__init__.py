@@ -17,4 +17,6 @@ from .capi import (  # noqa: F401
     q4k_last_cuda_error, q4k_selftest_wait_timeout, q4k_status_string, q4k_weight_bytes,
     q4k_dequant_f16, q4k_dequant_f16_status, q4k_f32_to_f16, q4k_f32_to_f16_status,
     q4k_gemm_f16, q4k_gemm_f16_status, q4k_prefill_f16, q4k_prefill_f16_status,
+    q4k_prefill_f16_noalloc, q4k_prefill_f16_noalloc_status, Q4K_ERR_CAPACITY,
+    Q4K_PREFILL_NOALLOC_MAX_ELEMS,
 )

@@ -21,12 +21,14 @@ Q4K_ERR_UNSUPPORTED_M = 4
 Q4K_ERR_CUDA = 5
 Q4K_ERR_OVERLAP = 6
 Q4K_ERR_RANGE = 7
+Q4K_ERR_CAPACITY = 8
 Q4K_FAULT_COPY_TIMEOUT = 1
 Q4K_FAULT_TOKEN_RANGE = 2
 Q4K_QK = 256
 Q4K_BLOCK_BYTES = 144
 Q4K_MAX_M = 64
 Q4K_GEMM_K_MULTIPLE = 64
+Q4K_PREFILL_NOALLOC_MAX_ELEMS = 8388608
 Q4K_KERNEL_WARP_ROWS = 1
 Q4K_KERNEL_STREAM = 2
 
@@ -35,7 +37,7 @@ EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string
            "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags",
            "q4k_embed_lookup_f32", "q4k_embed_gather_f32", "q4k_gemv_swiglu",
            "q4k_gemv_swiglu_plan_for", "q4k_selftest_wait_timeout", "q4k_dequant_f16",
-           "q4k_f32_to_f16", "q4k_gemm_f16", "q4k_prefill_f16")
+           "q4k_f32_to_f16", "q4k_gemm_f16", "q4k_prefill_f16", "q4k_prefill_f16_noalloc")
 
 
 class Q4KError(RuntimeError):
@@ -104,6 +106,9 @@ _lib.q4k_gemm_f16.restype = ctypes.c_int
 _lib.q4k_prefill_f16.argtypes = [_vp, _vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                  _vp]
 _lib.q4k_prefill_f16.restype = ctypes.c_int
+_lib.q4k_prefill_f16_noalloc.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         _vp]
+_lib.q4k_prefill_f16_noalloc.restype = ctypes.c_int
 
 
 def library() -> ctypes.CDLL:
@@ -365,3 +370,21 @@ def q4k_prefill_f16(w16, x, scratch, y, m: int, n: int, k: int, stream=None) -> 
     st = q4k_prefill_f16_status(w16, x, scratch, y, m, n, k, stream)
     if st != Q4K_OK:
         raise Q4KError(st, "q4k_prefill_f16")
+
+
+def q4k_prefill_f16_noalloc_status(w16, x, y, m: int, n: int, k: int, stream=None) -> int:
+    """Raw status of the C call (no exception; tensor checks still raise)."""
+    ok = _gemm_sizes_valid(m, n, k) and m * k <= Q4K_PREFILL_NOALLOC_MAX_ELEMS
+    return _lib.q4k_prefill_f16_noalloc(_ptr(w16, "float16", "w_f16", _need(n * k, 2, ok)),
+                                        _ptr(x, "float32", "x", _need(m * k, 4, ok)),
+                                        _ptr(y, "float32", "y", _need(m * n, 4, ok)), int(m),
+                                        int(n), int(k), _stream(stream))
+
+
+def q4k_prefill_f16_noalloc(w16, x, y, m: int, n: int, k: int, stream=None) -> None:
+    """y[m, n] = fp16(x[m, k]) @ w16[n, k]^T using the library's fixed scratch
+    (for callers that cannot allocate device memory; m*k <=
+    Q4K_PREFILL_NOALLOC_MAX_ELEMS; calls that overlap on the GPU race)."""
+    st = q4k_prefill_f16_noalloc_status(w16, x, y, m, n, k, stream)
+    if st != Q4K_OK:
+        raise Q4KError(st, "q4k_prefill_f16_noalloc")

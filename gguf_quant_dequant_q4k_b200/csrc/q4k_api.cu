@@ -98,6 +98,9 @@ const char* q4k_status_string(int status) {
         case Q4K_ERR_CUDA: return "CUDA runtime error (see q4k_last_cuda_error)";
         case Q4K_ERR_OVERLAP: return "output overlaps an input";
         case Q4K_ERR_RANGE: return "embedding token outside the table's rows";
+        case Q4K_ERR_CAPACITY:
+            return "m * k exceeds the fixed scratch of q4k_prefill_f16_noalloc "
+                   "(Q4K_PREFILL_NOALLOC_MAX_ELEMS)";
         default: return "unknown status";
     }
 }
@@ -304,6 +307,26 @@ int q4k_prefill_f16(const void* w_f16, const float* x, void* x_f16_scratch, floa
     st = launch_f32_to_f16(x, x_f16_scratch, static_cast<long long>(m) * k, dev.sm_count, s);
     if (st != Q4K_OK) return st;
     return launch_gemm_f16(w_f16, x_f16_scratch, y, m, n, k, s);
+}
+
+int q4k_prefill_f16_noalloc(const void* w_f16, const float* x, float* y, int m, int n, int k,
+                            q4k_stream_t stream) {
+    if (w_f16 == nullptr || x == nullptr || y == nullptr) return Q4K_ERR_NULL;
+    if (m <= 0 || n <= 0 || k <= 0 || k % Q4K_GEMM_K_MULTIPLE != 0) return Q4K_ERR_SHAPE;
+    if (static_cast<long long>(m) * k > Q4K_PREFILL_NOALLOC_MAX_ELEMS) return Q4K_ERR_CAPACITY;
+    if (!aligned(w_f16, 16) || !aligned(x, 16) || !aligned(y, 4)) return Q4K_ERR_ALIGN;
+    const size_t xbytes = static_cast<size_t>(m) * static_cast<size_t>(k) * 4;
+    const size_t wbytes = static_cast<size_t>(n) * static_cast<size_t>(k) * 2;
+    const size_t ybytes = static_cast<size_t>(m) * static_cast<size_t>(n) * 4;
+    if (overlaps(y, ybytes, w_f16, wbytes) || overlaps(y, ybytes, x, xbytes)) return Q4K_ERR_OVERLAP;
+    DeviceInfo dev;
+    int st = current_device_info(&dev);
+    if (st != Q4K_OK) return st;
+    int device = 0;
+    const cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess) return cuda_failure(e);
+    return launch_prefill_noalloc(device, w_f16, x, y, m, n, k, dev.sm_count,
+                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -32,6 +32,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
+#include <mutex>
 
 #include "q4k_internal.h"
 #include "q4k_superblock.cuh"
@@ -312,6 +313,40 @@ int launch_dequant_f16(const void* w, void* out, int n, int k, int num_sms, cuda
         static_cast<const uint8_t*>(w), static_cast<__half*>(out), total_sb);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+}
+
+// ------------------------------------------------ fixed-scratch prefill variant
+//
+// q4k_prefill_f16_noalloc needs the same fp16 copy of x as q4k_prefill_f16,
+// but for callers that cannot allocate device memory it lives in this
+// file-scope array instead of a caller buffer. Host code cannot use the
+// array's name as a device address (on the host it names a stand-in object),
+// so the address is fetched once per device with cudaGetSymbolAddress while
+// that device is current, and passed to the kernels.
+namespace {
+
+static __device__ __align__(256) __half g_prefill_scratch[Q4K_PREFILL_NOALLOC_MAX_ELEMS];
+
+constexpr int kScratchDevices = 64;
+std::once_flag g_scratch_once[kScratchDevices];
+void* g_scratch_ptr[kScratchDevices];
+cudaError_t g_scratch_status[kScratchDevices];
+
+}  // namespace
+
+int launch_prefill_noalloc(int device, const void* w16, const float* x, float* y, int m, int n,
+                           int k, int num_sms, cudaStream_t stream) {
+    if (device < 0 || device >= kScratchDevices) return cuda_failure(cudaErrorInvalidDevice);
+    std::call_once(g_scratch_once[device], [device] {
+        void* ptr = nullptr;
+        g_scratch_status[device] = cudaGetSymbolAddress(&ptr, g_prefill_scratch);
+        g_scratch_ptr[device] = ptr;
+    });
+    if (g_scratch_status[device] != cudaSuccess) return cuda_failure(g_scratch_status[device]);
+    void* xh = g_scratch_ptr[device];
+    int st = launch_f32_to_f16(x, xh, static_cast<long long>(m) * k, num_sms, stream);
+    if (st != Q4K_OK) return st;
+    return launch_gemm_f16(w16, xh, y, m, n, k, stream);
 }
 
 int read_gemm_fault_flags(unsigned* flags) {

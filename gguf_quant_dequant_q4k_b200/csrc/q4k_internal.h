@@ -53,5 +53,10 @@ int launch_f32_to_f16(const float* x, void* out, long long count, int num_sms,
                       cudaStream_t stream);
 int launch_dequant_f16(const void* w, void* out, int n, int k, int num_sms, cudaStream_t stream);
 int read_gemm_fault_flags(unsigned* flags);
+// q4k_prefill_f16 with the file-scope scratch array of q4k_gemm_f16.cu
+// (m * k <= Q4K_PREFILL_NOALLOC_MAX_ELEMS, checked by the caller); `device` is
+// the current device.
+int launch_prefill_noalloc(int device, const void* w16, const float* x, float* y, int m, int n,
+                           int k, int num_sms, cudaStream_t stream);
 
 }  // namespace q4k

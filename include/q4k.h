@@ -71,7 +71,8 @@ enum q4k_status {
     Q4K_ERR_UNSUPPORTED_M = 4,  /* m outside 1..Q4K_MAX_M                          */
     Q4K_ERR_CUDA = 5,           /* a CUDA runtime call failed (see last_cuda_error) */
     Q4K_ERR_OVERLAP = 6,        /* an output range overlaps an input range         */
-    Q4K_ERR_RANGE = 7           /* an embedding token outside the table's rows     */
+    Q4K_ERR_RANGE = 7,          /* an embedding token outside the table's rows     */
+    Q4K_ERR_CAPACITY = 8        /* q4k_prefill_f16_noalloc: m*k above its fixed scratch */
 };
 
 /* Bits of q4k_device_fault_flags(). */
@@ -83,6 +84,7 @@ enum q4k_status {
 #define Q4K_BLOCK_BYTES 144 /* bytes per superblock   */
 #define Q4K_MAX_M 64        /* most vectors per q4k_gemv call */
 #define Q4K_GEMM_K_MULTIPLE 64 /* q4k_gemm_f16 / q4k_prefill_f16: k % 64 == 0 */
+#define Q4K_PREFILL_NOALLOC_MAX_ELEMS 8388608 /* q4k_prefill_f16_noalloc: m*k limit (16 MiB fp16) */
 
 /*
  * y = W x for m vectors.
@@ -317,6 +319,33 @@ Q4K_API int q4k_gemm_f16(const void *w_f16, const void *x_f16, float *y, int m, 
  */
 Q4K_API int q4k_prefill_f16(const void *w_f16, const float *x, void *x_f16_scratch, float *y,
                             int m, int n, int k, q4k_stream_t stream);
+
+/*
+ * q4k_prefill_f16 without a caller-provided scratch, for callers that cannot
+ * allocate device memory: for instance a plugin running inside a host
+ * application that owns all device memory through its own allocator and
+ * hands out no allocation hook, or a latency-critical loop where cudaMalloc
+ * (which may synchronise the device) is not allowed. The pages have no
+ * counterpart to this entry point (their GEMM always takes a scratch buffer).
+ *   w_f16, x, y, m, n, k: as for q4k_prefill_f16 (y fully overwritten).
+ * The fp16 copy of x goes to a fixed device array inside the library of
+ * Q4K_PREFILL_NOALLOC_MAX_ELEMS binary16 values (16 MiB), which every GPU that
+ * loads the library holds until the process exits. m*k above that limit is
+ * refused with Q4K_ERR_CAPACITY before anything is enqueued.
+ * Nothing is allocated or freed by the call: no cudaMalloc, no cudaFree, no
+ * allocating library routine. The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.
+ * Every call shares the one array, which keeps the last call's contents: each
+ * call overwrites the m*k values its GEMM then reads, so nothing needs to be
+ * cleared, but calls that overlap on the GPU (on different streams, or on
+ * different host threads without ordering) race on it and must be serialised
+ * by the caller.
+ * Accuracy and results: identical to q4k_prefill_f16 on the same inputs.
+ * Returns a q4k_status.
+ */
+Q4K_API int q4k_prefill_f16_noalloc(const void *w_f16, const float *x, float *y, int m, int n,
+                                    int k, q4k_stream_t stream);
 
 #ifdef __cplusplus
 }
