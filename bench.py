@@ -73,11 +73,16 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+GEMV_SOURCES = ("q4k_gemv_stream.cu", "q4k_stream.h", "q4k_gemv.cu", "q4k_sm100.cuh",
+                "q4k_superblock.cuh", "q4k_swiglu.cuh")
+
+
 def source_digest() -> str:
-    """Hash of the CUDA sources, to tell whether committed ncu counters still apply."""
+    """Hash of the GEMV kernel sources (the files the sweep's launches are built
+    from), to tell whether committed ncu counters still apply."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gguf_quant_dequant_q4k_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in GEMV_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]

@@ -284,7 +284,8 @@ int q4k_gemm_f16(const void* w_f16, const void* x_f16, float* y, int m, int n, i
     DeviceInfo dev;
     st = current_device_info(&dev);
     if (st != Q4K_OK) return st;
-    return launch_gemm_f16(w_f16, x_f16, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
+    return launch_gemm_f16(w_f16, x_f16, y, m, n, k, dev.sm_count,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int q4k_prefill_f16(const void* w_f16, const float* x, void* x_f16_scratch, float* y, int m, int n,
@@ -306,7 +307,7 @@ int q4k_prefill_f16(const void* w_f16, const float* x, void* x_f16_scratch, floa
     const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = launch_f32_to_f16(x, x_f16_scratch, static_cast<long long>(m) * k, dev.sm_count, s);
     if (st != Q4K_OK) return st;
-    return launch_gemm_f16(w_f16, x_f16_scratch, y, m, n, k, s);
+    return launch_gemm_f16(w_f16, x_f16_scratch, y, m, n, k, dev.sm_count, s);
 }
 
 int q4k_prefill_f16_noalloc(const void* w_f16, const float* x, float* y, int m, int n, int k,

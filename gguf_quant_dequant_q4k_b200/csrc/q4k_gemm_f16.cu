@@ -50,19 +50,27 @@ constexpr int kGemmThreads = 128;
 constexpr int kGemmBM = 128;          // W rows per tile (MMA M)
 constexpr int kGemmBK = 64;           // K elements per k-block (128 bytes of fp16)
 constexpr int kGemmMmaK = 16;         // K per tcgen05.mma of kind::f16
-constexpr int kGemmStages = 4;
+constexpr int kGemmRingBytes = 192 * 1024;
 
 __host__ __device__ constexpr int stage_a_bytes() { return kGemmBM * kGemmBK * 2; }
 __host__ __device__ constexpr int stage_b_bytes(int bn) { return bn * kGemmBK * 2; }
+// Ring stages: as many as 192 KiB holds, at most 8 (4 for 256-token tiles,
+// 6 for 128, 8 for 64).
+__host__ __device__ constexpr int gemm_stages(int bn) {
+    return kGemmRingBytes / (stage_a_bytes() + stage_b_bytes(bn)) < 8
+               ? kGemmRingBytes / (stage_a_bytes() + stage_b_bytes(bn))
+               : 8;
+}
 constexpr int gemm_smem_bytes(int bn) {
-    return 1024 /* alignment slack */ + kGemmStages * (stage_a_bytes() + stage_b_bytes(bn)) +
-           (2 * kGemmStages + 1) * 8 + 16;
+    return 1024 /* alignment slack */ + gemm_stages(bn) * (stage_a_bytes() + stage_b_bytes(bn)) +
+           (2 * gemm_stages(bn) + 1) * 8 + 16;
 }
 
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 q4k_gemm_f16_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
                     float* __restrict__ y, int m, int n, int k) {
+    constexpr int kGemmStages = gemm_stages(BN);
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned base: the swizzled operand tiles need it
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -278,21 +286,47 @@ int launch_gemm_bn(const void* w16, const void* x16, float* y, int m, int n, int
 }  // namespace
 
 int gemm_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(q4k_gemm_f16_kernel<128>,
+    cudaError_t e = cudaFuncSetAttribute(q4k_gemm_f16_kernel<64>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         gemm_smem_bytes(128));
+                                         gemm_smem_bytes(64));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemm_f16_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes(128));
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(q4k_gemm_f16_kernel<256>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, gemm_smem_bytes(256));
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
 
-int gemm_tile_tokens(int m) { return m > 128 ? 256 : 128; }
+// Tokens per CTA tile: the one that gives the fewest waves of tiles times the
+// tile's cost, a narrower MMA (N) streaming its operands less efficiently
+// through shared memory per flop (cost weights 1.5 / 1.1 / 1.0 for N = 64 /
+// 128 / 256).
+int gemm_tile_tokens(int m, int n, int num_sms) {
+    static const int kN[3] = {256, 128, 64};
+    static const double kCost[3] = {1.0, 1.1, 1.5};
+    int best = 256;
+    double best_t = 1e300;
+    for (int i = 0; i < 3; ++i) {
+        const long long tiles = static_cast<long long>((n + kGemmBM - 1) / kGemmBM) *
+                                ((m + kN[i] - 1) / kN[i]);
+        const long long waves = (tiles + num_sms - 1) / num_sms;
+        const double t = static_cast<double>(waves) * kN[i] * kCost[i];
+        if (t < best_t - 1e-9) {
+            best_t = t;
+            best = kN[i];
+        }
+    }
+    return best;
+}
 
-int launch_gemm_f16(const void* w16, const void* x16, float* y, int m, int n, int k,
+int launch_gemm_f16(const void* w16, const void* x16, float* y, int m, int n, int k, int num_sms,
                     cudaStream_t stream) {
-    return gemm_tile_tokens(m) == 256 ? launch_gemm_bn<256>(w16, x16, y, m, n, k, stream)
-                                      : launch_gemm_bn<128>(w16, x16, y, m, n, k, stream);
+    switch (gemm_tile_tokens(m, n, num_sms)) {
+        case 64: return launch_gemm_bn<64>(w16, x16, y, m, n, k, stream);
+        case 128: return launch_gemm_bn<128>(w16, x16, y, m, n, k, stream);
+        default: return launch_gemm_bn<256>(w16, x16, y, m, n, k, stream);
+    }
 }
 
 int launch_f32_to_f16(const float* x, void* out, long long count, int num_sms,
@@ -346,7 +380,7 @@ int launch_prefill_noalloc(int device, const void* w16, const float* x, float* y
     void* xh = g_scratch_ptr[device];
     int st = launch_f32_to_f16(x, xh, static_cast<long long>(m) * k, num_sms, stream);
     if (st != Q4K_OK) return st;
-    return launch_gemm_f16(w16, xh, y, m, n, k, stream);
+    return launch_gemm_f16(w16, xh, y, m, n, k, num_sms, stream);
 }
 
 int read_gemm_fault_flags(unsigned* flags) {

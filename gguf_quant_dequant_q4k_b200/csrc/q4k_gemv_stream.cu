@@ -762,7 +762,11 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     // that a CTA of the next kernel on the stream can be resident beside it
     // (programmatic dependent launch then runs its prologue and first weight
     // copies while this one finishes), with up to kCompactCtasPerSm per SM.
-    const bool compact_ok = kPlanMode != 0;
+    // (Not for very tall matrices: there the streaming rate decides, and the
+    // classic CTA's extra warps pay; measured on B200, LM head 128256 x 4096:
+    // 100.9 us classic, 118.6 us compact.)
+    const bool tall = (n + num_sms - 1) / num_sms >= kWideMinRows;
+    const bool compact_ok = kPlanMode != 0 && !(kPlanMode == 3 && tall);
     // quant slices per lane: two for one vector on very tall matrices, for one
     // vector when K is too long for one-slice teams (K > 20480: a team of
     // two-slice lanes covers K <= 30720 with 15 warps), and for a compact CTA

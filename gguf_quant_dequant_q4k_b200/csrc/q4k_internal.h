@@ -46,8 +46,8 @@ int read_embed_fault_flags(unsigned* flags);
 
 // Prefill path (fp16 mirror + tensor-core GEMM). Arguments are validated.
 int gemm_set_attributes();
-int gemm_tile_tokens(int m);     // tokens per CTA tile of the GEMM (128 or 256)
-int launch_gemm_f16(const void* w16, const void* x16, float* y, int m, int n, int k,
+int gemm_tile_tokens(int m, int n, int num_sms);   // tokens per CTA tile (64, 128 or 256)
+int launch_gemm_f16(const void* w16, const void* x16, float* y, int m, int n, int k, int num_sms,
                     cudaStream_t stream);
 int launch_f32_to_f16(const float* x, void* out, long long count, int num_sms,
                       cudaStream_t stream);

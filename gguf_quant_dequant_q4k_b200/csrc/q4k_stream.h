@@ -63,13 +63,15 @@ struct StreamParams {
 // of shared memory. 1 / 2: compact CTAs (at most kCompactRegs registers and
 // kCompactSmem bytes of shared memory, so that a CTA of the next kernel can be
 // resident beside each one) wherever a team fits, kCompactCtasPerSm per SM.
+// 3: as 1, except for very tall matrices (kWideMinRows rows per SM or more),
+// which keep the classic CTA.
 #ifndef Q4K_PLAN_MODE
-#define Q4K_PLAN_MODE 0
+#define Q4K_PLAN_MODE 3
 #endif
 constexpr int kPlanMode = Q4K_PLAN_MODE;
 constexpr int kCompactRegs = 32768;
 constexpr int kCompactSmem = 112 * 1024;
-constexpr int kCompactCtasPerSm = (Q4K_PLAN_MODE == 1) ? 2 : 1;
+constexpr int kCompactCtasPerSm = (Q4K_PLAN_MODE == 2) ? 1 : 2;
 
 constexpr int kStreamMaxCluster = 8;    // cluster sizes the kernel supports (portable limit)
 constexpr int kClusterMaxRows = 8;      // split rows across a cluster only for N < 8 ...

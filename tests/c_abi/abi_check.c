@@ -33,7 +33,7 @@ int main(void)
     q4k_gemv_plan plan;
     memset(&plan, 0, sizeof(plan));
     CHECK(q4k_gemv_plan_for(1, 4096, 4096, 148, &plan) == Q4K_OK);
-    CHECK(plan.kernel == Q4K_KERNEL_STREAM && plan.grid == 148 && plan.launches == 1);
+    CHECK(plan.kernel == Q4K_KERNEL_STREAM && plan.grid >= 148 && plan.launches == 1);
     CHECK(q4k_gemv_plan_for(1, 128256, 4096, 148, &plan) == Q4K_OK && plan.slices == 2);
     CHECK(q4k_gemv_plan_for(Q4K_MAX_M + 1, 4096, 4096, 148, &plan) == Q4K_ERR_UNSUPPORTED_M);
     CHECK(q4k_gemv_plan_for(1, 4096, 4000, 148, &plan) == Q4K_ERR_SHAPE);

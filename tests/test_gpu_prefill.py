@@ -108,7 +108,11 @@ def small_int_operands(m, n, k, seed):
 
 @pytest.mark.parametrize("m,n,k", [(1, 1, 64), (5, 7, 64), (128, 128, 256), (129, 130, 320),
                                    (256, 128, 1024), (300, 257, 512), (257, 384, 4096),
-                                   (512, 256, 14336)])
+                                   (512, 256, 14336),
+                                   # tile widths the launch picks on 148 SMs: 256, 128 and
+                                   # 64 tokens per CTA, and ragged edges of each
+                                   (512, 14336, 256), (512, 4096, 256), (512, 1024, 256),
+                                   (509, 14300, 192), (500, 4000, 320), (511, 1000, 128)])
 def test_gemm_f16_exact_on_integers(q4k, m, n, k):
     w16, x16 = small_int_operands(m, n, k, m * 7 + n)
     y = gpu_gemm(q4k, w16, x16, m, n, k)

@@ -37,6 +37,33 @@ def team_range(cluster_id, gteam, n, nsb, clusters, cluster, teams):
     return s0, s1, row0, nseg
 
 
+def stream_regs(m, slices):
+    """Registers per thread the kernel is compiled for (80 for one vector and
+    one slice, else 128)."""
+    threads = 640 if (m == 1 and slices == 1) else 480
+    return 16384 // (((threads // 32 + 1 + 3) // 4) * 32) // 8 * 8
+
+
+def expected_launch(m, n, k, fused):
+    """The launch policy the planner states: compact CTAs (at most 32768
+    registers and 112 KiB of shared memory, two per SM) unless the matrix is
+    very tall (512 or more rows per SM); two quant slices per lane for one
+    vector on very tall matrices, for K beyond one-slice teams, or where a
+    compact one-slice team would not fit. Returns (compact, slices, max compute
+    warps, CTAs per SM, shared-memory cap)."""
+    nsb = k // 256
+    mi = min(m, 2)
+    tall = -(-n // SM_COUNT) >= 512
+    cw = lambda regs: 32768 // (regs * 32) - 1
+    compact_s1 = (not tall) and -(-nsb * 8 // 32) <= cw(stream_regs(mi, 1))
+    compact_s2 = (not tall) and mi == 1 and not fused and -(-nsb * 4 // 32) <= cw(stream_regs(1, 2))
+    compact = compact_s1 or compact_s2
+    wide = mi == 1 and not fused and (tall or nsb > 80 or (compact and not compact_s1))
+    sl = 2 if wide else 1
+    maxw = cw(stream_regs(mi, sl)) if compact else (640 if (mi == 1 and sl == 1) else 480) // 32
+    return compact, sl, maxw, (2 if compact else 1), (112 if compact else 220) * 1024
+
+
 def seg_bounds(s0, s1, row0, i, nsb):
     return max(s0, (row0 + i) * nsb), min(s1, (row0 + i + 1) * nsb)
 
@@ -51,11 +78,14 @@ def check_plan(m, n, k):
     clusters = ctas // cluster
     assert clusters <= n
     slices = p["slices"]                                 # 16-byte quant slices per lane
-    wide = m == 1 and (-(-n // SM_COUNT) >= 512 or nsb > 80)   # very tall or long K: two slices
-    assert slices == (2 if wide else 1)
+    compact, exp_slices, maxw, per_sm, smem_cap = expected_launch(m, n, k, False)
+    assert slices == exp_slices
+    assert clusters <= per_sm * SM_COUNT
     team_warps = -(-nsb * 8 // slices // 32)
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
-    assert p["block"] <= (640 if (m == 1 and slices == 1) else 480) + 32
+    assert p["block"] <= maxw * 32 + 32
+    if compact:   # a compact CTA leaves room for one of the next kernel beside it
+        assert p["block"] * stream_regs(min(m, 2), slices) <= 32768
     assert 2 <= depth <= 8 and 1 <= teams <= 20
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     # [seg][positions][4 groups] float4 coefficients + float2 rounding errors
@@ -63,7 +93,7 @@ def check_plan(m, n, k):
     need = (teams * depth * stage_bytes + teams * team_warps * coef_per_warp
             + teams * depth * 2 * team_warps * SEG * m * 4 + teams * 2 * m * 4)
     need = -(-need // 16) * 16 + cluster * teams * 32 + teams * 2 * depth * 8
-    assert p["smem_bytes"] == need and need <= 220 * 1024 - 1024
+    assert p["smem_bytes"] == need and need <= smem_cap - 1024
     covered = [0] * (n * nsb)
     writes = [0] * n
     for q in range(clusters):
@@ -190,8 +220,10 @@ def check_fused_plan(m, n, k):
         return p
     nsb = k // 256
     ctas, teams, depth = p["grid"], p["teams"], p["depth"]
-    assert p["cluster"] == 1 and ctas == min(n, SM_COUNT)
+    compact, _, maxw, per_sm, smem_cap = expected_launch(m, n, k, True)
+    assert p["cluster"] == 1 and ctas == min(n, per_sm * SM_COUNT)
     team_warps = -(-nsb * 8 // 32)
+    assert teams * team_warps <= maxw
     assert p["block"] == teams * team_warps * 32 + 32
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     rows_cap = -(-n // ctas)
@@ -200,7 +232,7 @@ def check_fused_plan(m, n, k):
             + teams * depth * 2 * team_warps * SEG * mi * 4 + teams * 2 * mi * 4)
     need = -(-need // 16) * 16 + teams * 32 + teams * 2 * depth * 8
     need += -(-(mi * 2 * rows_cap * 4) // 16) * 16
-    assert p["smem_bytes"] == need and need <= 220 * 1024 - 1024
+    assert p["smem_bytes"] == need and need <= smem_cap - 1024
     base, extra = n // ctas, n % ctas
     gate_seen = [0] * (n * nsb)
     up_seen = [0] * (n * nsb)
