@@ -110,22 +110,70 @@ void launch_rows(const q4k_gemv_plan& plan, const void* w, const void* w2, const
 
 }  // namespace
 
+namespace {
+
+// Vectors per streaming launch: 1 or 2 for m <= 2. For m >= 3, groups of
+// four on half slices (each decoded superblock applied to the four vectors;
+// the last group padded up to four if it has three vectors, run on the one-
+// or two-vector kernel if it has one or two) where one launch of that kernel
+// covers K (K <= 7680); beyond that, pairs, which measured faster on B200 than
+// K-chunked groups of four (4096 x 14336, m = 4: 41.8 us as two pair launches,
+// 46.8 us as two K-chunks of the four-vector kernel; 14336 x 4096, m = 4:
+// 39.4 us as one four-vector launch, 40.2 us as two pairs). The fused SwiGLU
+// runs pairs.
+int group_size(int m, int nsb, bool fused) {
+    if (fused || m <= 2) return m <= 2 ? m : 2;
+    return nsb <= stream_max_nsb(4, 0) ? 4 : 2;
+}
+
+int kernel_vectors(int mi, bool fused) {
+    if (fused) return mi;
+    return mi >= 3 ? 4 : mi;
+}
+
+// K split into the fewest equal chunks (whole superblocks) one team covers:
+// each chunk is a launch over strided row segments, later chunks adding into y.
+struct KChunks {
+    int count, nsb;   // chunks, superblocks per chunk (the last one may be shorter)
+};
+
+KChunks k_chunks(int mk, int nsb) {
+    const int maxnsb = stream_max_nsb(mk, mk == 1 ? 2 : (mk == 2 ? 1 : 0));
+    KChunks c{1, nsb};
+    if (maxnsb <= 0 || nsb <= maxnsb) return c;
+    c.count = (nsb + maxnsb - 1) / maxnsb;
+    c.nsb = (nsb + c.count - 1) / c.count;
+    return c;
+}
+
+}  // namespace
+
 int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
                      bool fused, q4k_gemv_plan* plan, StreamParams* sp) {
     StreamParams q{};
     int grid = 0, block = 0, smem = 0;
-    // m > 2: ceil(m/2) launches of the two-vector streaming kernel on vector
-    // pairs (each decoded weight reused for two vectors per pass).
-    const int m_launch = m <= kStreamMaxM ? m : kStreamMaxM;
+    const int nsb = k / kQK;
+    const int gsz = group_size(m, nsb, fused);
+    const int mk = kernel_vectors(gsz, fused);
     const int* cl = max_clusters;
-    if (plan_stream(m_launch, n, k, num_sms, max_smem, cl, fused, &q, &grid, &block, &smem)) {
+    bool ok = plan_stream(mk, n, k, num_sms, max_smem, cl, fused, &q, &grid, &block, &smem) != 0;
+    int chunks = 1;
+    if (!ok && !fused) {
+        const KChunks c = k_chunks(mk, nsb);
+        if (c.count > 1) {
+            chunks = c.count;
+            ok = plan_stream(mk, n, c.nsb * kQK, num_sms, max_smem, cl, false, &q, &grid, &block,
+                             &smem) != 0;
+        }
+    }
+    if (ok) {
         plan->kernel = Q4K_KERNEL_STREAM;
         plan->grid = grid;
         plan->block = block;
         plan->smem_bytes = smem;
         plan->teams = q.teams;
         plan->depth = q.depth;
-        plan->launches = (m + m_launch - 1) / m_launch;
+        plan->launches = ((m + gsz - 1) / gsz) * chunks;
         plan->cluster = q.cluster;
         plan->units = n;
         plan->units_per_cta_max = q.rows_base + (q.rows_extra > 0 ? 1 : 0);
@@ -159,30 +207,40 @@ int plan_gemv(int m, int n, int k, int num_sms, bool fused, q4k_gemv_plan* plan)
 int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const float* x, float* y,
                 int m, int n, int k, cudaStream_t stream) {
     q4k_gemv_plan plan;
-    StreamParams sp;
     const bool fused = w2 != nullptr;
-    const int m_launch = m <= kStreamMaxM ? m : kStreamMaxM;
-    const int* clusters = dev.max_clusters[m_launch - 1];
-    int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin, clusters, fused, &plan,
-                              &sp);
+    const int gsz = group_size(m, k / kQK, fused);
+    int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin,
+                              dev.max_clusters[kernel_vectors(gsz, fused) == 1 ? 0 : 1], fused,
+                              &plan, nullptr);
     if (st != Q4K_OK) return st;
     if (plan.kernel == Q4K_KERNEL_STREAM) {
-        for (int i0 = 0; i0 < m; i0 += m_launch) {
-            const int mi = (m - i0) < m_launch ? (m - i0) : m_launch;
-            StreamParams spi = sp;
-            if (mi != m_launch) {   // the odd last vector runs the one-vector kernel
-                int g = 0, b = 0, sm = 0;
-                if (!plan_stream(mi, n, k, dev.sm_count, dev.max_smem_optin,
-                                 dev.max_clusters[mi - 1], fused, &spi, &g, &b, &sm))
-                    return Q4K_ERR_SHAPE;   // not reached: fewer vectors never need more
-                st = launch_stream(spi, g, b, sm, w, w2, x + static_cast<size_t>(i0) * k,
-                                   y + static_cast<size_t>(i0) * n, mi, stream);
-            } else {
-                st = launch_stream(spi, plan.grid, plan.block, plan.smem_bytes, w, w2,
-                                   x + static_cast<size_t>(i0) * k, y + static_cast<size_t>(i0) * n,
-                                   mi, stream);
+        const int nsb = k / kQK;
+        for (int i0 = 0; i0 < m; i0 += gsz) {
+            const int mi = (m - i0) < gsz ? (m - i0) : gsz;      // vectors of this group
+            const int mk = kernel_vectors(mi, fused);           // the kernel's M
+            const int* cl = dev.max_clusters[mk == 1 ? 0 : 1];
+            StreamParams sp;
+            int g = 0, b = 0, sm = 0;
+            KChunks c{1, nsb};
+            if (!plan_stream(mk, n, k, dev.sm_count, dev.max_smem_optin, cl, fused, &sp, &g, &b, &sm))
+                c = k_chunks(mk, nsb);
+            for (int ci = 0; ci < c.count; ++ci) {
+                const int sb0 = ci * c.nsb;
+                const int nsb_c = (nsb - sb0) < c.nsb ? (nsb - sb0) : c.nsb;
+                if (c.count > 1 &&
+                    !plan_stream(mk, n, nsb_c * kQK, dev.sm_count, dev.max_smem_optin, cl, fused, &sp,
+                                 &g, &b, &sm))
+                    return Q4K_ERR_SHAPE;   // not reached: a chunk never exceeds a team
+                sp.nsb_row = nsb;
+                sp.sb_off = sb0;
+                sp.x_stride = k;
+                sp.accumulate = ci > 0 ? 1 : 0;
+                sp.m_valid = mi;
+                st = launch_stream(sp, g, b, sm, w, w2,
+                                   x + static_cast<size_t>(i0) * k + static_cast<size_t>(sb0) * kQK,
+                                   y + static_cast<size_t>(i0) * n, mk, stream);
+                if (st != Q4K_OK) return st;
             }
-            if (st != Q4K_OK) return st;
         }
         return Q4K_OK;
     }

@@ -83,8 +83,12 @@ constexpr uint32_t kMagic2p23 = 0x4B000000u; // 2^23
 // Coefficient buffer per warp: [segment][position][4 groups] float4s
 // (A_2g, A_2g+1, B_2g, B_2g+1), then [segment][position][4 groups] float2s
 // (-e_2g, -e_2g+1): B's rounding errors.
-__host__ __device__ constexpr int coef_main_bytes_per_warp(int slices) { return kSeg * (4 * slices) * 4 * 16; }
-__host__ __device__ constexpr int coef_bytes_per_warp(int slices) { return kSeg * (4 * slices) * 4 * (16 + 8); }
+__host__ __device__ constexpr int coef_main_bytes_per_warp(int slices) {
+    return kSeg * pos_per_warp(slices) * 4 * 16;
+}
+__host__ __device__ constexpr int coef_bytes_per_warp(int slices) {
+    return kSeg * pos_per_warp(slices) * 4 * (16 + 8);
+}
 
 // f = 1/2 + q/256 for the nibble q held in byte SEL of `masked` (bytes 0..15):
 // the byte becomes bits 16..23 of 0x3F000000 (1/2), i.e. mantissa bits 16..19.
@@ -209,6 +213,62 @@ __device__ __forceinline__ void decode_half(uint4 h, float d, float dmin, int ha
     err = make_float4(-e01.x, -e01.y, -e23.x, -e23.y);
 }
 
+// As decode_half for the single 64-weight group g (sub-blocks 2g, 2g+1):
+// out = (A_2g, A_2g+1, B_2g, B_2g+1), err = (-e_2g, -e_2g+1).
+// exact: out = (A_2g, A_2g+1, -A_2g/2, -A_2g+1/2), err = (-dmin*m_2g, -dmin*m_2g+1)
+// instead (the weight formed as fma(A, f, -A/2) + (-dmin*m), rounded once).
+__device__ __forceinline__ void decode_group(uint4 h, float d, float dmin, int g, float4& out,
+                                             float2& err, bool exact = false) {
+    const int half = g >> 1;
+    const uint32_t sc = half ? ((h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u))
+                             : (h.y & 0x3F3F3F3Fu);
+    const uint32_t mm = half ? (((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u))
+                             : (h.z & 0x3F3F3F3Fu);
+    const uint32_t s0 = static_cast<uint32_t>((g & 1) * 2);   // bytes s0, s0 + 1 of the half
+    const float d128 = d * 128.0f;
+    const float2 sa = make_float2(d128, d128);
+    const float2 sb2 = make_float2(-8388608.0f * d128, -8388608.0f * d128);
+    const float2 ma = make_float2(dmin, dmin);
+    const float2 mb = make_float2(-8388608.0f * dmin, -8388608.0f * dmin);
+    const float2 scf = make_float2(__uint_as_float(__byte_perm(sc, kMagic2p23, 0x7650 | s0)),
+                                   __uint_as_float(__byte_perm(sc, kMagic2p23, 0x7650 | (s0 + 1))));
+    const float2 mmf = make_float2(__uint_as_float(__byte_perm(mm, kMagic2p23, 0x7650 | s0)),
+                                   __uint_as_float(__byte_perm(mm, kMagic2p23, 0x7650 | (s0 + 1))));
+    const float2 a = ffma2(sa, scf, sb2);   // 128 d sc (exact)
+    const float2 m = ffma2(ma, mmf, mb);    // dmin m (exact)
+    const float2 A = __fadd2_rn(a, a);
+    const float2 sm = __fadd2_rn(a, m);
+    const float2 v = fsub2(sm, a);
+    const float2 e = __fadd2_rn(fsub2(a, fsub2(sm, v)), fsub2(m, v));
+    if (exact) {
+        out = make_float4(A.x, A.y, -a.x, -a.y);
+        err = make_float2(-m.x, -m.y);
+        return;
+    }
+    out = make_float4(A.x, A.y, -sm.x, -sm.y);
+    err = make_float2(-e.x, -e.y);
+}
+
+// kWords consecutive 32-bit words of quant bytes from shared memory (one
+// 8- or 16-byte load per 16 bytes).
+template <int kWords>
+__device__ __forceinline__ void load_words(const uint8_t* smem, uint32_t addr, uint32_t (&w)[kWords]) {
+    if (kWords == 2) {
+        const uint2 v = *reinterpret_cast<const uint2*>(smem + addr);
+        w[0] = v.x;
+        w[1 % kWords] = v.y;
+    } else {
+#pragma unroll
+        for (int j = 0; j < kWords / 4; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + addr + 16 * j);
+            w[(4 * j + 0) % kWords] = v.x;
+            w[(4 * j + 1) % kWords] = v.y;
+            w[(4 * j + 2) % kWords] = v.z;
+            w[(4 * j + 3) % kWords] = v.w;
+        }
+    }
+}
+
 __device__ __forceinline__ void header_scales(uint4 h, float& d, float& dmin) {
     d = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x & 0xFFFFu)));
     dmin = __half2float(__ushort_as_half(static_cast<unsigned short>(h.x >> 16)));
@@ -221,15 +281,25 @@ __device__ __forceinline__ void header_scales(uint4 h, float& d, float& dmin) {
 // per vector (measured faster on B200 than four split chains: fewer
 // instructions, and the other warps hide the chain's latency); `first`
 // initialises the chain.
-template <int M, int NX>
+// EXACT: b = -A/2 (so A*f + b = d*sc*q exactly) and the weight is completed
+// as (d*sc*q) + mneg, mneg = (-dmin*m_2g, -dmin*m_2g+1): rounded once, with no
+// correction term (used where registers are too scarce for the per-lane x sums).
+template <int M, int NX, bool EXACT = false>
 __device__ __forceinline__ void dot_word(uint32_t w, float2 a, float2 b, const float2 (&xp)[M][NX],
-                                         int e0, bool first, float2 (&acc)[M]) {
+                                         int e0, bool first, float2 (&acc)[M],
+                                         float2 mneg = make_float2(0.f, 0.f)) {
     const uint32_t lo = w & 0x0F0F0F0Fu;
     const uint32_t hi = __umulhi(w, 1u << 28) & 0x0F0F0F0Fu;   // (w >> 4) on the FMA pipe
-    const float2 w0 = ffma2(a, make_float2(nib_to_f<0>(lo), nib_to_f<0>(hi)), b);
-    const float2 w1 = ffma2(a, make_float2(nib_to_f<1>(lo), nib_to_f<1>(hi)), b);
-    const float2 w2 = ffma2(a, make_float2(nib_to_f<2>(lo), nib_to_f<2>(hi)), b);
-    const float2 w3 = ffma2(a, make_float2(nib_to_f<3>(lo), nib_to_f<3>(hi)), b);
+    float2 w0 = ffma2(a, make_float2(nib_to_f<0>(lo), nib_to_f<0>(hi)), b);
+    float2 w1 = ffma2(a, make_float2(nib_to_f<1>(lo), nib_to_f<1>(hi)), b);
+    float2 w2 = ffma2(a, make_float2(nib_to_f<2>(lo), nib_to_f<2>(hi)), b);
+    float2 w3 = ffma2(a, make_float2(nib_to_f<3>(lo), nib_to_f<3>(hi)), b);
+    if (EXACT) {
+        w0 = __fadd2_rn(w0, mneg);
+        w1 = __fadd2_rn(w1, mneg);
+        w2 = __fadd2_rn(w2, mneg);
+        w3 = __fadd2_rn(w3, mneg);
+    }
 #pragma unroll
     for (int i = 0; i < M; ++i) {
         acc[i] = first ? __fmul2_rn(w0, xp[i][e0 + 0]) : ffma2(w0, xp[i][e0 + 0], acc[i]);
@@ -341,7 +411,24 @@ __device__ __forceinline__ void issue_stage(const Team& T, const StreamParams& p
     mbar_arrive_expect_tx(&T.full[slot], bytes);
     uint8_t* dst = T.ring + static_cast<size_t>(slot) * p.stage_bytes;
     if (!FUSED) {
-        bulk_copy_g2s(dst, T.w + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &T.full[slot]);
+        if (p.nsb_row == p.nsb && p.sb_off == 0) {   // contiguous rows: one copy
+            bulk_copy_g2s(dst, T.w + static_cast<size_t>(b_rel) * kBlockBytes, bytes, &T.full[slot]);
+            return;
+        }
+        // a K-chunk of longer rows: one copy per row segment, from row r's
+        // superblocks sb_off + col of its nsb_row
+        long long vs = T.tr.s0 + b_rel;
+        const long long ve = T.tr.s0 + e_rel;
+        while (vs < ve) {
+            const long long r = vs / p.nsb;
+            const long long c = vs - r * p.nsb;
+            const long long e = ve < (r + 1) * p.nsb ? ve : (r + 1) * p.nsb;
+            const uint32_t nb = static_cast<uint32_t>(e - vs) * kBlockBytes;
+            bulk_copy_g2s(dst, p.w + static_cast<size_t>(r * p.nsb_row + p.sb_off + c) * kBlockBytes,
+                          nb, &T.full[slot]);
+            dst += nb;
+            vs = e;
+        }
         return;
     }
     long long vs = T.tr.s0 + b_rel;                               // virtual, CTA-relative
@@ -370,15 +457,31 @@ __device__ __forceinline__ float& row_out_ref(const StreamParams& p, uint8_t* sm
     return p.y[static_cast<size_t>(i) * p.n + row];
 }
 
-// M vectors, S 16-byte quant slices (S*32 weights) per lane per row.
+// Finishes row `row` of vector i: y = tot, or y += tot for a later K-chunk;
+// vectors beyond m_valid (padding of a partial vector group) are not stored.
+template <bool FUSED>
+__device__ __forceinline__ void store_row(const StreamParams& p, uint8_t* smem, int i, long long row,
+                                          float tot) {
+    if (i >= p.m_valid) return;
+    float& r = row_out_ref<FUSED>(p, smem, i, row);
+    r = p.accumulate ? r + tot : tot;
+}
+
+// M vectors, S 16-byte quant slices (S*32 weights) per lane per row; S = 0:
+// one 8-byte half slice (16 weights).
 template <int M, int S, bool FUSED>
 __global__ void __maxnreg__(stream_max_regs(M, S))
 q4k_gemv_stream_kernel(const StreamParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ volatile int abort_flag;
-    constexpr int kLanesPerSb = 8 / S;        // lanes covering one superblock of a row
-    constexpr int kPos = 32 / kLanesPerSb;    // superblock positions per warp
-    constexpr int kNX = 16 * S;               // x pairs per lane per vector
+    constexpr int kLanesPerSb = lanes_per_sb(S);   // lanes covering one superblock of a row
+    constexpr int kPos = pos_per_warp(S);          // superblock positions per warp
+    constexpr int kNX = lane_bytes(S);             // x pairs per lane per vector
+    constexpr int kWords = kNX / 4;                // 32-bit quant words per lane and row
+    // Four vectors (half slices): weights formed exactly (one more packed add
+    // per weight pair) instead of the per-lane x sums of the correction term,
+    // which would not fit the registers beside four vectors' x.
+    constexpr bool kExactW = (M >= 4);
     const int nsb = p.nsb;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -441,6 +544,26 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 // team's buffer, which the refilled stage does not write.
                 if (tf + p.depth < nst) issue_stage<FUSED>(T, p, rbf + p.depth * kSeg * nsb, fslot);
                 const float* rbuf = T.red + static_cast<size_t>(fslot * 2 + fphase) * red_slot;
+                // Sum the team's warp partials: warp wi's M*kSeg values are
+                // consecutive ([wi][i][u]), so each warp's block is read as
+                // float4s, the loads of several warps in flight before their
+                // adds (warp order, as a serial sum would add them).
+                constexpr int kVals = M * kSeg;
+                float tot[kVals];
+#pragma unroll
+                for (int v = 0; v < kVals; ++v) tot[v] = 0.f;
+#pragma unroll 4
+                for (int wi = 0; wi < p.team_warps; ++wi) {
+                    const float4* src = reinterpret_cast<const float4*>(rbuf + wi * kVals);
+#pragma unroll
+                    for (int v4 = 0; v4 < kVals / 4; ++v4) {
+                        const float4 t = src[v4];
+                        tot[4 * v4 + 0] += t.x;
+                        tot[4 * v4 + 1] += t.y;
+                        tot[4 * v4 + 2] += t.z;
+                        tot[4 * v4 + 3] += t.w;
+                    }
+                }
 #pragma unroll
                 for (int u = 0; u < kSeg; ++u) {
                     if (tf * kSeg + u >= T.tr.nseg) break;
@@ -450,13 +573,10 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                     const long long row = T.tr.row0 + tf * kSeg + u;
 #pragma unroll
                     for (int i = 0; i < M; ++i) {
-                        float tot = 0.f;
-                        for (int wi = 0; wi < p.team_warps; ++wi)
-                            tot += rbuf[(wi * M + i) * kSeg + u];
                         if (b == 0 && e == nsb)
-                            row_out_ref<FUSED>(p, smem, i, row) = tot;
+                            store_row<FUSED>(p, smem, i, row, tot[i * kSeg + u]);
                         else
-                            part[(lane * 2 + (b > 0 ? 0 : 1)) * M + i] = tot;
+                            part[(lane * 2 + (b > 0 ? 0 : 1)) * M + i] = tot[i * kSeg + u];
                     }
                 }
                 ++tf;
@@ -491,11 +611,13 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         pdl_launch_dependents();
         pdl_wait();   // x and y belong to the dependency chain
 
-        // This lane's superblock position bl and its slices c0 .. c0+S-1 of the
-        // 8 16-byte quant slices: group g = c0/2 (sub-blocks 2g, 2g+1).
+        // This lane's superblock position bl and its kNX quant bytes, from
+        // byte qoff of the superblock's 128: group g = qoff / 32 (sub-blocks
+        // 2g, 2g+1), bytes b0 .. b0 + kNX - 1 of the group's 32.
         const int lpos = lane / kLanesPerSb;
-        const int c0 = (lane % kLanesPerSb) * S;
-        const int g = c0 >> 1;
+        const int qoff = (lane % kLanesPerSb) * kNX;
+        const int g = qoff >> 5;
+        const int b0 = qoff & 31;
         const int bl = wit * kPos + lpos;
         const bool valid = bl < nsb;
         // xp[i][e] = (x of the low nibble of byte e of the lane's quant bytes, x
@@ -507,15 +629,18 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             // their latency overlaps the first stage's wait and decode. Plain
             // (coherent, L1-allocating) loads: measured on B200 the
             // non-coherent path made the K = 14336 call 10 % slower.
-            const int k0 = (valid ? bl : 0) * kQK + 64 * g + 16 * (c0 & 1);
+            // A vector past m_valid (padding) reads vector 0's x and uses zeros.
+            const int k0 = (valid ? bl : 0) * kQK + 64 * g + b0;
+            const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
-                const float4* xl =
-                    reinterpret_cast<const float4*>(p.x + static_cast<size_t>(i) * p.k + k0);
+                const bool vi = i < p.m_valid;
+                const float4* xl = reinterpret_cast<const float4*>(
+                    p.x + static_cast<size_t>(vi ? i : 0) * p.x_stride + k0);
                 const float4* xh = xl + 8;   // + 32 weights
 #pragma unroll
                 for (int v = 0; v < kNX / 4; ++v) {
-                    const float4 a = xl[v], b = xh[v];
+                    const float4 a = vi ? xl[v] : zero4, b = vi ? xh[v] : zero4;
                     xp[i][4 * v + 0] = make_float2(a.x, b.x);
                     xp[i][4 * v + 1] = make_float2(a.y, b.y);
                     xp[i][4 * v + 2] = make_float2(a.z, b.z);
@@ -529,6 +654,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         float2 sx[M];
 #pragma unroll
         for (int i = 0; i < M; ++i) {
+            if (kExactW) continue;
             sx[i] = xp[i][0];
 #pragma unroll
             for (int e = 1; e < kNX; ++e) sx[i] = __fadd2_rn(sx[i], xp[i][e]);
@@ -539,16 +665,18 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         // (g ^ ((pos >> 1) & 3)): conflict-free for decode stores and item loads.
         const int span = kSeg * nsb;
         const uint32_t ring_off = static_cast<uint32_t>(T.ring - smem);
-        const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + 16 * c0);
+        const uint32_t lane_qoff = static_cast<uint32_t>(bl * kBlockBytes + kQsOffset + qoff);
         const uint32_t coef_off = static_cast<uint32_t>(p.off_coef) +
                                   static_cast<uint32_t>(warp) * static_cast<uint32_t>(coef_bytes_per_warp(S));
         const uint32_t lane_coef_off =
             coef_off + static_cast<uint32_t>((lpos * 4 + (g ^ ((lpos >> 1) & 3))) * 16);
         // Decode lanes: S = 2: lane -> (segment du, position dpos), whole header;
-        // S = 1: lane -> (segment du, position dpos, half dhalf).
+        // S = 1: lane -> (segment du, position dpos, half dhalf); S = 0: lane ->
+        // (segment du, position dpos, group dgrp).
         const int du = lane >> 3;
-        const int dpos = S == 2 ? (lane & 7) : ((lane >> 1) & 3);
-        const int dhalf = S == 2 ? 0 : (lane & 1);
+        const int dpos = S == 2 ? (lane & 7) : (S == 1 ? ((lane >> 1) & 3) : ((lane >> 2) & 1));
+        const int dhalf = S == 1 ? (lane & 1) : 0;
+        const int dgrp = lane & 3;
         const int dbl = wit * kPos + dpos;
         const uint32_t dec_base = coef_off + static_cast<uint32_t>((du * kPos + dpos) * 4 * 16);
         const int dswz = (dpos >> 1) & 3;
@@ -585,6 +713,13 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                     header_scales(hdr, d, dmin);
                     const uint32_t cb = dec_base + static_cast<uint32_t>(dg * 4 * kPos * 4 * 16);
                     const uint32_t eb = dec_err + static_cast<uint32_t>(dg * 4 * kPos * 4 * 8);
+                    if (S == 0) {
+                        float4 c_g;
+                        float2 e_g;
+                        decode_group(hdr, d, dmin, dgrp, c_g, e_g, kExactW);
+                        *reinterpret_cast<float4*>(smem + cb + (dgrp ^ dswz) * 16) = c_g;
+                        *reinterpret_cast<float2*>(smem + eb + dgrp * 8) = e_g;
+                    }
 #pragma unroll
                     for (int hh = 0; hh < S; ++hh) {
                         const int half = S == 2 ? hh : dhalf;
@@ -610,41 +745,34 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 const int idx = u * nsb - head + bl;
                 use[u] = valid && static_cast<unsigned>(idx) < static_cast<unsigned>(nsb_stage);
                 qaddr[u] = st_off + (use[u] ? lane_qoff + static_cast<uint32_t>((u * nsb - head) * kBlockBytes)
-                                            : static_cast<uint32_t>(kQsOffset + 16 * c0));
+                                            : static_cast<uint32_t>(kQsOffset + qoff));
             }
             const int nseg_s = T.tr.nseg - s * kSeg < kSeg ? T.tr.nseg - s * kSeg : kSeg;
             float part_sum[M][kSeg];
-            uint4 qn[S];
-#pragma unroll
-            for (int j = 0; j < S; ++j) qn[j] = *reinterpret_cast<const uint4*>(smem + qaddr[0] + 16 * j);
+            uint32_t qn[kWords];
+            load_words<kWords>(smem, qaddr[0], qn);
             float4 cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off);
             // Item u: the lane's slice of segment u; loads item u + 1's operands
             // first if `next`.
             auto item = [&](const int u, const bool next) {
-                uint4 q[S];
+                uint32_t q[kWords];
 #pragma unroll
-                for (int j = 0; j < S; ++j) q[j] = qn[j];
+                for (int j = 0; j < kWords; ++j) q[j] = qn[j];
                 const float4 cf = cfn;
                 // used after the item's dot products: loaded here, not a step ahead
                 const float2 ne = *reinterpret_cast<const float2*>(smem + lane_err_off + u * kPos * 32);
                 if (next) {
-#pragma unroll
-                    for (int j = 0; j < S; ++j)
-                        qn[j] = *reinterpret_cast<const uint4*>(smem + qaddr[u + 1] + 16 * j);
+                    load_words<kWords>(smem, qaddr[u + 1], qn);
                     cfn = *reinterpret_cast<const float4*>(smem + lane_coef_off + (u + 1) * kPos * 64);
                 }
                 const float2 a = make_float2(cf.x, cf.y), b = make_float2(cf.z, cf.w);
                 float2 acc[M];
 #pragma unroll
-                for (int j = 0; j < S; ++j) {
-                    dot_word<M, kNX>(q[j].x, a, b, xp, 16 * j + 0, j == 0, acc);
-                    dot_word<M, kNX>(q[j].y, a, b, xp, 16 * j + 4, false, acc);
-                    dot_word<M, kNX>(q[j].z, a, b, xp, 16 * j + 8, false, acc);
-                    dot_word<M, kNX>(q[j].w, a, b, xp, 16 * j + 12, false, acc);
-                }
+                for (int j = 0; j < kWords; ++j)
+                    dot_word<M, kNX, kExactW>(q[j], a, b, xp, 4 * j, j == 0, acc, ne);
 #pragma unroll
                 for (int i = 0; i < M; ++i) {
-                    acc[i] = ffma2(ne, sx[i], acc[i]);   // remove B's rounding error
+                    if (!kExactW) acc[i] = ffma2(ne, sx[i], acc[i]);   // remove B's rounding error
                     part_sum[i][u] = use[u] ? (acc[i].x + acc[i].y) : 0.f;
                 }
             };
@@ -721,7 +849,7 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < M; ++i) row_out_ref<FUSED>(p, smem, i, last) = tot[i];
+                for (int i = 0; i < M; ++i) store_row<FUSED>(p, smem, i, last, tot[i]);
             }
         }
     }
@@ -754,10 +882,19 @@ int resident_clusters(int c, int num_sms, const int* max_clusters) {
 
 }  // namespace
 
+int stream_max_nsb(int m, int slices) {
+    if ((m == 4) != (slices == 0)) return 0;   // four vectors on half slices, else whole slices
+    // the warps of one team (one CTA's compute warps) times positions per warp
+    const int by_warps = (stream_max_threads(m, slices) / 32) * pos_per_warp(slices);
+    const int cap = kStreamMaxNsb * (slices == 0 ? 1 : slices);
+    return by_warps < cap ? by_warps : cap;
+}
+
 int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
                 bool fused, StreamParams* sp, int* grid, int* block, int* smem_bytes) {
     const int nsb = k / kQK;
-    if (m < 1 || m > kStreamMaxM || n < 1) return 0;
+    if (m < 1 || m > kStreamMaxM || m == 3 || n < 1) return 0;
+    if (m == 4 && fused) return 0;
     // Compact CTAs: at most half of an SM's registers and shared memory, so
     // that a CTA of the next kernel on the stream can be resident beside it
     // (programmatic dependent launch then runs its prologue and first weight
@@ -766,11 +903,13 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     // classic CTA's extra warps pay; measured on B200, LM head 128256 x 4096:
     // 100.9 us classic, 118.6 us compact.)
     const bool tall = (n + num_sms - 1) / num_sms >= kWideMinRows;
-    const bool compact_ok = kPlanMode != 0 && !(kPlanMode == 3 && tall);
+    const bool compact_ok = kPlanMode != 0 && !(kPlanMode == 3 && tall) && m <= 2;
     // quant slices per lane: two for one vector on very tall matrices, for one
     // vector when K is too long for one-slice teams (K > 20480: a team of
     // two-slice lanes covers K <= 30720 with 15 warps), and for a compact CTA
-    // whose one-slice team would not fit its warps
+    // whose one-slice team would not fit its warps; four vectors run on 8-byte
+    // half slices (16 weights per lane: 64 registers of x, as for two vectors
+    // on one slice)
     const int compact_warps1 = kCompactRegs / (stream_max_regs(m, 1) * 32) - 1;
     const bool compact_s1 = compact_ok && (nsb * 8 + 31) / 32 <= compact_warps1;
     const bool compact_s2 = compact_ok && m == 1 && !fused &&
@@ -779,9 +918,9 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     const bool wide = m == 1 && !fused &&
                       ((n + num_sms - 1) / num_sms >= kWideMinRows || nsb > kStreamMaxNsb ||
                        (compact && !compact_s1));
-    const int sl = wide ? 2 : 1;
-    if (nsb > kStreamMaxNsb * sl) return 0;
-    const int team_warps = (nsb * 8 / sl + 31) / 32;   // 8*nsb slices / (32 lanes * sl)
+    const int sl = m == 4 ? 0 : (wide ? 2 : 1);
+    if (nsb > stream_max_nsb(m, sl)) return 0;
+    const int team_warps = (nsb * lanes_per_sb(sl) + 31) / 32;
     const int max_warps = compact ? kCompactRegs / (stream_max_regs(m, sl) * 32) - 1
                                   : stream_max_threads(m, sl) / 32;
     if (team_warps > max_warps) return 0;
@@ -851,6 +990,11 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     q.depth = depth;
     q.stage_bytes = stage_bytes;
     q.slices = sl;
+    q.nsb_row = nsb;
+    q.sb_off = 0;
+    q.x_stride = k;
+    q.accumulate = 0;
+    q.m_valid = m;
     size_t off = static_cast<size_t>(teams) * depth * stage_bytes;
     q.off_coef = static_cast<int>(off);
     off += static_cast<size_t>(teams) * team_warps * coef_bytes_per_warp(sl);
@@ -901,8 +1045,10 @@ int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, 
     } else if (m == 1) {
         e = sp.slices == 2 ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, 2, false>, sp)
                            : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, 1, false>, sp);
-    } else {
+    } else if (m == 2) {
         e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, 1, false>, sp);
+    } else {
+        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<4, 0, false>, sp);
     }
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
@@ -922,6 +1068,9 @@ int stream_set_attributes() {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, 1, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<4, 0, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }

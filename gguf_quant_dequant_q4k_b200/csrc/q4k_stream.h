@@ -10,7 +10,14 @@ namespace q4k {
 // slower than 4 on every decode shape (register spills, LM head 101.7 ->
 // 110.3 us).
 constexpr int kStreamSegRows = 4;
-constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kernel
+constexpr int kStreamMaxM = 4;          // vectors handled by one streaming launch (1, 2 or 4)
+
+// Lane geometry for S 16-byte quant slices per lane and row (S = 0: one
+// 8-byte half slice): quant bytes per lane and row, lanes per superblock,
+// superblock positions per warp.
+__host__ __device__ constexpr int lane_bytes(int s) { return s == 0 ? 8 : 16 * s; }
+__host__ __device__ constexpr int lanes_per_sb(int s) { return 128 / lane_bytes(s); }
+__host__ __device__ constexpr int pos_per_warp(int s) { return 32 / lanes_per_sb(s); }
 // Quant slices (16 bytes = 32 weights) per lane and row: 1, or 2 for one
 // vector on very tall matrices (kWideMinRows rows or more per CTA: an LM
 // head). Two slices halve the per-item overheads but double the x registers
@@ -20,12 +27,15 @@ constexpr int kStreamMaxM = 2;          // vectors handled by the streaming kern
 constexpr int kWideMinRows = 512;
 // Compute threads per CTA (plus one producer warp): one slice, one vector: 20
 // warps (x: 32 registers per lane; five or six warps per sub-partition at 80
-// registers; 23 measured no faster); two vectors, or two slices: 15 warps (x:
-// 64 registers per lane; four warps per sub-partition at 128 registers).
-constexpr int stream_max_threads(int m, int slices) { return (m == 1 && slices == 1) ? 640 : 480; }
+// registers; 23 measured no faster); two vectors, two slices, or four vectors
+// on half slices: 15 warps (x: 64 registers per lane; four warps per
+// sub-partition at 128 registers).
+__host__ __device__ constexpr int stream_max_threads(int m, int slices) {
+    return (m == 1 && slices == 1) ? 640 : 480;
+}
 // Registers per thread: each of the SM's four sub-partitions has 16384
 // registers for its share of the CTA's warps (allocated in multiples of 8).
-constexpr int stream_max_regs(int m, int slices) {
+__host__ __device__ constexpr int stream_max_regs(int m, int slices) {
     return 16384 / (((stream_max_threads(m, slices) / 32 + 1 + 3) / 4) * 32) / 8 * 8;
 }
 // Superblocks per row one team of one-slice lanes covers (K <= 20480 for one
@@ -56,7 +66,14 @@ struct StreamParams {
     int stage_bytes;            // bytes per ring slot
     int off_coef, off_red, off_part, off_tr, off_bar;  // shared-memory offsets (bytes)
     int off_rows, rows_cap;     // fused: row totals [M][2 * rows_cap] (gate rows, up rows)
-    int slices;                 // 16-byte quant slices per lane (1 or 2)
+    int slices;                 // 16-byte quant slices per lane (1 or 2; 0: one 8-byte half)
+    // A K-chunk of longer rows: the kernel's rows are nsb superblocks starting
+    // at superblock sb_off of rows nsb_row long (nsb_row == nsb, sb_off == 0
+    // for a whole matrix); x points at the chunk's first element of vector 0
+    // and vectors are x_stride floats apart.
+    int nsb_row, sb_off, x_stride;
+    int accumulate;             // 1: y += the chunk's sums (a later K-chunk); 0: y = sums
+    int m_valid;                // vectors present (<= the kernel's M; the rest are padding)
 };
 
 // Launch policy. 0: one CTA per SM with up to 20 compute warps and 220 KiB
@@ -88,6 +105,10 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
 // Resident clusters of c CTAs (c = 1..8) for the streaming kernel on the
 // current device, into max_clusters[c]; 0 where the query is not possible.
 int stream_cluster_occupancy(int m, int* max_clusters);
+
+// Most superblocks per row one team can cover for m vectors at `slices`
+// (0 if the streaming kernel has no such configuration).
+int stream_max_nsb(int m, int slices);
 
 // w_up != null: fused gate/up SwiGLU (w is the gate projection).
 int launch_stream(const StreamParams& sp, int grid, int block, int smem_bytes, const void* w,

@@ -159,6 +159,27 @@ def test_gemv_tall_two_slices_sampled(q4k, n, k):
     assert_gemv_close(y[:, rows], yref, a, f"{n}x{k}")
 
 
+@pytest.mark.parametrize("m,n,k", [(3, 40, 20736), (4, 33, 14336), (4, 300, 7680), (3, 300, 7936),
+                                   (5, 77, 15616), (1, 9, 40960), (2, 17, 33024), (1, 4096, 61440),
+                                   (7, 150, 11008), (4, 1, 14336), (3, 5, 8192)])
+def test_gemv_k_chunks_and_vector_groups(q4k, m, n, k):
+    """K beyond one team runs as K-chunks of strided row segments, later chunks
+    adding into y; three to eight vectors run in groups of four on half slices
+    (a group of three padded); y starts as NaN, so the first chunk must
+    overwrite it."""
+    plan = q4k.q4k_gemv_plan_for(m, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert plan["kernel"] == q4k.Q4K_KERNEL_STREAM
+    w, x = q4k_synth.q4k_problem(n, k, m, 70 + m + n)
+    y = gpu_gemv(q4k, w, x, n, k)
+    if n * k <= 4096 * 61440 // 8:
+        yref, a = oracle.gemv(w, x, n, k, nthreads=NTHREADS)
+        assert_gemv_close(y, yref, a, f"{m}x{n}x{k}")
+    else:
+        rows = np.unique(np.concatenate([[0, n - 1], np.random.default_rng(n).integers(0, n, 30)]))
+        yref, a = oracle.gemv_rows(w, x, n, k, rows)
+        assert_gemv_close(y[:, rows], yref, a, f"{m}x{n}x{k}")
+
+
 @pytest.mark.parametrize("m", [9, 12, 16, 17, 32, 64])
 @pytest.mark.parametrize("n,k", [(33, 512), (200, 1792), (40, 20736)])
 def test_gemv_batches_beyond_eight(q4k, n, k, m):

@@ -44,6 +44,40 @@ def stream_regs(m, slices):
     return 16384 // (((threads // 32 + 1 + 3) // 4) * 32) // 8 * 8
 
 
+def lane_geometry(slices):
+    """(quant bytes per lane and row, lanes per superblock, positions per
+    warp): slices 16-byte quant slices per lane, 0 meaning one 8-byte half."""
+    lb = 8 if slices == 0 else 16 * slices
+    return lb, 128 // lb, 32 // (128 // lb)
+
+
+def kernel_vectors(m, fused=False, k=None):
+    """Vectors one streaming launch carries: 1, 2, or 4 (groups of four for
+    m >= 3 where one four-vector launch covers K <= 7680, else pairs; the
+    fused SwiGLU runs pairs)."""
+    if fused or m <= 2:
+        return min(m, 2)
+    return 4 if k is None or k <= 7680 else 2
+
+
+def max_nsb(mk, slices):
+    threads = 640 if (mk == 1 and slices == 1) else 480
+    return min((threads // 32) * lane_geometry(slices)[2], 80 * max(slices, 1))
+
+
+def k_chunk_nsbs(m, k):
+    """Superblocks of each K-chunk the library launches for the first vector
+    group: the fewest equal chunks one team covers (the last may be shorter)."""
+    mk = kernel_vectors(m, k=k)
+    nsb = k // 256
+    top = max_nsb(mk, 2 if mk == 1 else (1 if mk == 2 else 0))
+    if nsb <= top:
+        return [nsb]
+    count = -(-nsb // top)
+    per = -(-nsb // count)
+    return [min(per, nsb - i * per) for i in range(count)]
+
+
 def expected_launch(m, n, k, fused):
     """The launch policy the planner states: compact CTAs (at most 32768
     registers and 112 KiB of shared memory, two per SM) unless the matrix is
@@ -52,7 +86,9 @@ def expected_launch(m, n, k, fused):
     compact one-slice team would not fit. Returns (compact, slices, max compute
     warps, CTAs per SM, shared-memory cap)."""
     nsb = k // 256
-    mi = min(m, 2)
+    mi = kernel_vectors(m, fused, k)
+    if mi == 4:    # four vectors: half slices, one CTA per SM, up to 15 compute warps
+        return False, 0, 15, 1, 220 * 1024
     tall = -(-n // SM_COUNT) >= 512
     cw = lambda regs: 32768 // (regs * 32) - 1
     compact_s1 = (not tall) and -(-nsb * 8 // 32) <= cw(stream_regs(mi, 1))
@@ -72,26 +108,41 @@ def check_plan(m, n, k):
     p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
     if p["kernel"] != q4k.Q4K_KERNEL_STREAM:
         return p
+    chunks = k_chunk_nsbs(m, k)
+    mk0 = kernel_vectors(m, k=k)
+    groups = -(-m // mk0)
+    assert p["launches"] == groups * len(chunks)
+    assert sum(chunks) == k // 256 and max(chunks) <= max_nsb(mk0, p["slices"])
+    m = mk0
+    if len(chunks) > 1:
+        # every K-chunk is a launch on rows of chunk length (the partition below
+        # is the first chunk's; the last chunk's is checked as its own plan)
+        if chunks[-1] != chunks[0]:
+            check_plan(m, n, chunks[-1] * 256)
+        k = chunks[0] * 256
     nsb = k // 256
     ctas, teams, depth, cluster = p["grid"], p["teams"], p["depth"], p["cluster"]
     assert cluster in (1, 2) and ctas % cluster == 0
     clusters = ctas // cluster
     assert clusters <= n
-    slices = p["slices"]                                 # 16-byte quant slices per lane
+    slices = p["slices"]                     # 16-byte quant slices per lane (0: one 8-byte half)
     compact, exp_slices, maxw, per_sm, smem_cap = expected_launch(m, n, k, False)
     assert slices == exp_slices
     assert clusters <= per_sm * SM_COUNT
-    team_warps = -(-nsb * 8 // slices // 32)
+    lb, lanes_sb, pos = lane_geometry(slices)
+    team_warps = -(-nsb * lanes_sb // 32)
+    assert team_warps * pos >= nsb            # a team's lanes cover every superblock position
     assert p["block"] == teams * team_warps * 32 + 32      # + one producer warp
     assert p["block"] <= maxw * 32 + 32
+    mk = m
     if compact:   # a compact CTA leaves room for one of the next kernel beside it
-        assert p["block"] * stream_regs(min(m, 2), slices) <= 32768
+        assert p["block"] * stream_regs(mk, slices) <= 32768
     assert 2 <= depth <= 8 and 1 <= teams <= 20
     stage_bytes = -(-SEG * nsb * 144 // 128) * 128
     # [seg][positions][4 groups] float4 coefficients + float2 rounding errors
-    coef_per_warp = SEG * (4 * slices) * 4 * (16 + 8)
+    coef_per_warp = SEG * pos * 4 * (16 + 8)
     need = (teams * depth * stage_bytes + teams * team_warps * coef_per_warp
-            + teams * depth * 2 * team_warps * SEG * m * 4 + teams * 2 * m * 4)
+            + teams * depth * 2 * team_warps * SEG * mk * 4 + teams * 2 * mk * 4)
     need = -(-need // 16) * 16 + cluster * teams * 32 + teams * 2 * depth * 8
     assert p["smem_bytes"] == need and need <= smem_cap - 1024
     covered = [0] * (n * nsb)
@@ -158,7 +209,7 @@ SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
 
 
 @pytest.mark.parametrize("n,k", SHAPES)
-@pytest.mark.parametrize("m", [1, 2])
+@pytest.mark.parametrize("m", [1, 2, 3, 4])
 def test_stream_partition(m, n, k):
     check_plan(m, n, k)
 
@@ -181,29 +232,38 @@ def test_cluster_choice(n, k, cluster):
 def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(1, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_plan_for(2, 4096, 14336, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
-    # outside the streaming kernel's range: the general kernel
+    # three or four vectors: one launch of the four-vector kernel (half slices)
     p3 = q4k.q4k_gemv_plan_for(3, 4096, 4096, SM_COUNT)
-    assert p3["kernel"] == q4k.Q4K_KERNEL_STREAM and p3["launches"] == 2
-    assert q4k.q4k_gemv_plan_for(8, 4096, 14336, SM_COUNT)["launches"] == 4
-    assert q4k.q4k_gemv_plan_for(3, 64, 15616, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    assert p3["kernel"] == q4k.Q4K_KERNEL_STREAM and p3["launches"] == 1 and p3["slices"] == 0
+    # eight vectors on K = 14336 (beyond one four-vector launch): four pairs
+    p8 = q4k.q4k_gemv_plan_for(8, 4096, 14336, SM_COUNT)
+    assert p8["launches"] == 4 and p8["slices"] == 1
+    assert q4k.q4k_gemv_plan_for(8, 14336, 4096, SM_COUNT)["launches"] == 2
+    assert q4k.q4k_gemv_plan_for(5, 4096, 4096, SM_COUNT)["launches"] == 2
     assert q4k.q4k_gemv_plan_for(1, 64, 20480, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     # one vector, K beyond one-slice teams: two-slice teams up to K = 30720
     p = q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)
-    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2
-    assert q4k.q4k_gemv_plan_for(1, 64, 30720, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
-    assert q4k.q4k_gemv_plan_for(1, 64, 30976, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
-    assert q4k.q4k_gemv_plan_for(2, 64, 15360, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
-    assert q4k.q4k_gemv_plan_for(2, 64, 15616, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS
+    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2 and p["launches"] == 1
+    assert q4k.q4k_gemv_plan_for(1, 64, 30720, SM_COUNT)["launches"] == 1
+    # beyond one team: K-chunks on the streaming kernel, never the general one
+    for m, k, launches in [(1, 30976, 2), (1, 61440, 2), (1, 61696, 3), (2, 15360, 1),
+                           (2, 15616, 2), (3, 7680, 1), (3, 7936, 2), (4, 15616, 4)]:
+        p = q4k.q4k_gemv_plan_for(m, 64, k, SM_COUNT)
+        assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["launches"] == launches, (m, k, p)
+    # the fused SwiGLU beyond the streaming range stays on the general kernel
+    assert (q4k.q4k_gemv_swiglu_plan_for(1, 64, 20736, SM_COUNT)["kernel"]
+            == q4k.Q4K_KERNEL_WARP_ROWS)
 
 
 def test_batches_beyond_eight_vectors():
-    """m > 8 runs as vector tiles: pairs on the streaming kernel, eights on the
-    general one (the realizar page tiles batches over 8); m > 64 is refused."""
-    assert q4k.q4k_gemv_plan_for(16, 14336, 4096, SM_COUNT)["launches"] == 8
-    assert q4k.q4k_gemv_plan_for(33, 4096, 4096, SM_COUNT)["launches"] == 17
-    assert q4k.q4k_gemv_plan_for(64, 4096, 4096, SM_COUNT)["launches"] == 32
+    """m > 8 runs as vector tiles (the realizar page tiles batches over 8):
+    groups of four on the streaming kernel, each K-chunked where K is beyond a
+    team; m > 64 is refused."""
+    assert q4k.q4k_gemv_plan_for(16, 14336, 4096, SM_COUNT)["launches"] == 4
+    assert q4k.q4k_gemv_plan_for(33, 4096, 4096, SM_COUNT)["launches"] == 9
+    assert q4k.q4k_gemv_plan_for(64, 4096, 4096, SM_COUNT)["launches"] == 16
     p = q4k.q4k_gemv_plan_for(20, 64, 30976, SM_COUNT)
-    assert p["kernel"] == q4k.Q4K_KERNEL_WARP_ROWS and p["launches"] == 3
+    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["launches"] == 10 * 3
     with pytest.raises(q4k.Q4KError):
         q4k.q4k_gemv_plan_for(65, 4096, 4096, SM_COUNT)
 
