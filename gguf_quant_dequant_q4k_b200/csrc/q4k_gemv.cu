@@ -12,6 +12,7 @@
 // carries weight 64g+16h+l (low nibble, sub-block 2g) and weight 64g+32+16h+l
 // (high nibble, sub-block 2g+1), with g = c/2, h = c%2. The warp's 32 quant
 // loads are 4 x 128 contiguous bytes.
+#include "q4k_gemv_tc.h"
 #include "q4k_internal.h"
 #include "q4k_stream.h"
 #include "q4k_superblock.cuh"
@@ -148,8 +149,31 @@ KChunks k_chunks(int mk, int nsb) {
 
 }  // namespace
 
+// m >= 3 vectors (plain projection): the tensor-core kernel, one pair of
+// launches (digits, GEMV) per group of up to 16 vectors.
+bool use_tc(int m, bool fused) { return !fused && m >= kTcMinM; }
+
 int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
                      bool fused, q4k_gemv_plan* plan, StreamParams* sp) {
+    if (use_tc(m, fused)) {
+        const int tiles = (n + kTcRows - 1) / kTcRows;
+        const int grid = tc_ctas(tiles, k / kQK, num_sms);
+        const long long items = static_cast<long long>(tiles) * (k / kQK);
+        const int groups = (m + kTcMaxM - 1) / kTcMaxM;
+        const int mp = tc_vectors_padded(m < kTcMaxM ? m : kTcMaxM);
+        plan->kernel = Q4K_KERNEL_TC;
+        plan->grid = grid;
+        plan->block = tc_threads();
+        plan->smem_bytes = tc_smem_bytes(mp);
+        plan->cluster = 1;
+        plan->teams = 0;
+        plan->depth = tc_stages(mp);
+        plan->launches = 2 * groups;
+        plan->units = items;   // (128-row tile, superblock column) items
+        plan->units_per_cta_max = (items + grid - 1) / grid;
+        plan->slices = 0;
+        return Q4K_OK;
+    }
     StreamParams q{};
     int grid = 0, block = 0, smem = 0;
     const int nsb = k / kQK;
@@ -208,6 +232,7 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const floa
                 int m, int n, int k, cudaStream_t stream) {
     q4k_gemv_plan plan;
     const bool fused = w2 != nullptr;
+    if (use_tc(m, fused)) return launch_gemv_tc(dev, w, x, y, m, n, k, stream);
     const int gsz = group_size(m, k / kQK, fused);
     int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin,
                               dev.max_clusters[kernel_vectors(gsz, fused) == 1 ? 0 : 1], fused,

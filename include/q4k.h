@@ -94,15 +94,29 @@ enum q4k_status {
  *        ("input: M x K row-major", `batched_q4k_gemv_into`).
  *   y  : m x N float32, row-major (vector i at y + i*N); fully overwritten,
  *        never accumulated into ("output: M x N row-major").
- *   m  : 1..64 vectors. Batches run as kernels over tiles of the vectors (the
- *        realizar page tiles m > 8 in `batched_q4k_gemv_into`): pairs on the
- *        streaming kernel, eights on the general one; q4k_gemv_plan_for
- *        reports the launch count. Larger m is refused, not looped (the
- *        turbospark page, "turbospark-runtime 0.1.0,
+ *   m  : 1..64 vectors. One or two vectors run on the streaming kernel (one
+ *        launch, or K-chunks of it for long K). Three or more run on the
+ *        tensor-core kernel in groups of up to 16 (the realizar page tiles
+ *        m > 8 in `batched_q4k_gemv_into` and has an m = 16 / 32 branch): each
+ *        group is a digits launch and a GEMV launch, the weights decoded once
+ *        per group. q4k_gemv_plan_for reports the launch count. Larger m is
+ *        refused, not looped (the turbospark page, "turbospark-runtime 0.1.0,
  *        src/real_forward_dispatch.rs", `encode_gemm_any`, refuses rather than
  *        silently looping): that is a GEMM's size.
+ * Workspace: for m >= 3 the call allocates a device workspace from the
+ * device's default memory pool, stream-ordered on `stream`
+ * (cudaMallocAsync / cudaFreeAsync; capturable in a CUDA graph), of
+ * (K/256) * (N_mma*512 + 80*mp) + 2048*mp*ctas + 4*ceil(N/128) bytes
+ * (mp = 8 or 16, N_mma = 48 or 80, ctas <= SM count): 2.7 MiB for
+ * N = 14336, K = 4096, m = 8. m <= 2 allocates nothing.
  * Accuracy: per element |y - sum_k w_nk x_ik| <= 1e-4 * sum_k |w_nk x_ik| + 1e-6,
- * where w_nk is the f32 value d*sc*q - dmin*m; accumulation is in f32.
+ * where w_nk is the f32 value d*sc*q - dmin*m; for m <= 2 accumulation is in
+ * f32. For m >= 3 the products are exact integers (x scaled per 256-element
+ * block by 2^(33 - E), E the exponent of the block's largest |x|, and
+ * rounded to an integer) combined in f64, so the bound holds with one more
+ * term, 2^-33 * sum_k |w_nk| * max_block(k) |x_i|, which is below 1e-6 unless
+ * that sum exceeds 8590 (e.g. K = 14336 and |x| up to ~1 with most of w x
+ * cancelling); an inf or NaN in x_i makes every element of y_i NaN.
  * Weight reads may start before the previous kernel on `stream` has finished
  * (programmatic dependent launch): x is read and y written only after it has.
  * W is treated as constant model data: it must not be written by work still
@@ -249,13 +263,21 @@ Q4K_API int q4k_gemv_swiglu_plan_for(int m, int n, int k, int num_sms, q4k_gemv_
 enum q4k_kernel {
     Q4K_KERNEL_WARP_ROWS = 1,   /* any K: one warp per row, loads via L1; m > 8
                                    runs as ceil(m/8) launches on vector tiles   */
-    Q4K_KERNEL_STREAM = 2       /* K <= 30720 (m = 1) / 15360 (m >= 2); m > 2 runs
+    Q4K_KERNEL_STREAM = 2,      /* K <= 30720 (m = 1) / 15360 (m >= 2); m > 2 runs
                                    as ceil(m/2) launches on vector pairs;
                                    bulk-copy streamed rows, x held in registers,
                                    balanced per-SM ranges; small N splits rows
                                    across the CTAs of a cluster (split-K) and
                                    finishes them through distributed shared
                                    memory                                         */
+    Q4K_KERNEL_TC = 3           /* m >= 3: tcgen05 tensor cores, each superblock
+                                   decoded once for up to 16 vectors (groups of
+                                   16 beyond), exact integer products of sc*q
+                                   and base-128 digits of the scaled x; two
+                                   launches per group (digits, GEMV); `units`
+                                   counts (128-row tile, superblock column)
+                                   items, shared out in equal contiguous ranges;
+                                   `depth` is the weight-ring depth             */
 };
 
 Q4K_API int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan *plan);

@@ -163,12 +163,12 @@ def test_gemv_tall_two_slices_sampled(q4k, n, k):
                                    (5, 77, 15616), (1, 9, 40960), (2, 17, 33024), (1, 4096, 61440),
                                    (7, 150, 11008), (4, 1, 14336), (3, 5, 8192)])
 def test_gemv_k_chunks_and_vector_groups(q4k, m, n, k):
-    """K beyond one team runs as K-chunks of strided row segments, later chunks
-    adding into y; three to eight vectors run in groups of four on half slices
-    (a group of three padded); y starts as NaN, so the first chunk must
-    overwrite it."""
+    """K beyond one team: one or two vectors run as K-chunks of strided row
+    segments on the streaming kernel, later chunks adding into y; three or more
+    run on the tensor-core kernel, which takes any K; y starts as NaN, so the
+    first launch must overwrite it."""
     plan = q4k.q4k_gemv_plan_for(m, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
-    assert plan["kernel"] == q4k.Q4K_KERNEL_STREAM
+    assert plan["kernel"] == (q4k.Q4K_KERNEL_STREAM if m <= 2 else q4k.Q4K_KERNEL_TC)
     w, x = q4k_synth.q4k_problem(n, k, m, 70 + m + n)
     y = gpu_gemv(q4k, w, x, n, k)
     if n * k <= 4096 * 61440 // 8:

@@ -209,9 +209,53 @@ SHAPES = (q4k_synth.SHAPES_TINY + q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B
 
 
 @pytest.mark.parametrize("n,k", SHAPES)
-@pytest.mark.parametrize("m", [1, 2, 3, 4])
+@pytest.mark.parametrize("m", [1, 2])
 def test_stream_partition(m, n, k):
     check_plan(m, n, k)
+
+
+def check_tc_plan(m, n, k):
+    """m >= 3: the tensor-core kernel. One persistent CTA per SM at most, over
+    128-row tiles; a digits launch and a GEMV launch per group of up to 16
+    vectors; the stage ring (digit image of N x 256 fp16, 128 x 144 bytes of
+    weights, 80 bytes of block metadata per vector) fits shared memory."""
+    p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
+    assert p["kernel"] == q4k.Q4K_KERNEL_TC
+    tiles, nsb = -(-n // 128), k // 256
+    items = tiles * nsb                          # (128-row tile, superblock column)
+    assert p["grid"] == min(items, SM_COUNT) and p["block"] == 480 and p["cluster"] == 1
+    assert p["launches"] == 2 * -(-m // 16)
+    mp = 8 if min(m, 16) <= 8 else 16
+    n_mma = -(-5 * mp // 16) * 16
+    wstages = 4 if mp == 8 else 3              # weight ring
+    bstages = min(6, (212 * 1024 - wstages * 128 * 144 - 16 * mp * 80) // (n_mma * 512))   # digit images
+    assert p["depth"] == wstages and bstages >= 3
+    assert p["smem_bytes"] == (1024 + bstages * n_mma * 512 + 16 * mp * 80 + wstages * 128 * 144
+                               + (2 * (bstages + 16 + wstages) + 11) * 8 + 16)
+    assert p["smem_bytes"] <= 232448
+    assert p["units"] == items and p["units_per_cta_max"] == -(-items // p["grid"])
+    # equal contiguous ranges: every item owned once, counts differ by at most one
+    ranges = [(items * c // p["grid"], items * (c + 1) // p["grid"]) for c in range(p["grid"])]
+    assert ranges[0][0] == 0 and ranges[-1][1] == items
+    assert all(r1 == s2 for (_, r1), (s2, _) in zip(ranges, ranges[1:]))
+    assert max(b - a for a, b in ranges) - min(b - a for a, b in ranges) <= 1
+    return p
+
+
+def test_tc_balanced_items():
+    """The tile x superblock items are shared out evenly over up to 148 CTAs:
+    14336 x 4096 (1792 items) gives 12 or 13 per CTA, 1536 x 1536 (72 items)
+    one per CTA."""
+    p = q4k.q4k_gemv_plan_for(8, 14336, 4096, SM_COUNT)
+    assert p["grid"] == SM_COUNT and p["units_per_cta_max"] == 13
+    p = q4k.q4k_gemv_plan_for(8, 1536, 1536, SM_COUNT)
+    assert p["grid"] == 72 and p["units_per_cta_max"] == 1
+
+
+@pytest.mark.parametrize("n,k", SHAPES)
+@pytest.mark.parametrize("m", [3, 4, 8, 9, 16, 17, 64])
+def test_tc_plan(m, n, k):
+    check_tc_plan(m, n, k)
 
 
 def test_lm_head_partition():
@@ -232,14 +276,11 @@ def test_cluster_choice(n, k, cluster):
 def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(1, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     assert q4k.q4k_gemv_plan_for(2, 4096, 14336, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
-    # three or four vectors: one launch of the four-vector kernel (half slices)
-    p3 = q4k.q4k_gemv_plan_for(3, 4096, 4096, SM_COUNT)
-    assert p3["kernel"] == q4k.Q4K_KERNEL_STREAM and p3["launches"] == 1 and p3["slices"] == 0
-    # eight vectors on K = 14336 (beyond one four-vector launch): four pairs
-    p8 = q4k.q4k_gemv_plan_for(8, 4096, 14336, SM_COUNT)
-    assert p8["launches"] == 4 and p8["slices"] == 1
-    assert q4k.q4k_gemv_plan_for(8, 14336, 4096, SM_COUNT)["launches"] == 2
-    assert q4k.q4k_gemv_plan_for(5, 4096, 4096, SM_COUNT)["launches"] == 2
+    # three or more vectors: the tensor-core kernel (digits + GEMV per 16 vectors)
+    for m, n, k in [(3, 4096, 4096), (8, 4096, 14336), (8, 14336, 4096), (5, 4096, 4096),
+                    (16, 128256, 4096), (3, 64, 61696)]:
+        p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
+        assert p["kernel"] == q4k.Q4K_KERNEL_TC and p["launches"] == 2, (m, n, k, p)
     assert q4k.q4k_gemv_plan_for(1, 64, 20480, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
     # one vector, K beyond one-slice teams: two-slice teams up to K = 30720
     p = q4k.q4k_gemv_plan_for(1, 64, 20736, SM_COUNT)
@@ -247,7 +288,7 @@ def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(1, 64, 30720, SM_COUNT)["launches"] == 1
     # beyond one team: K-chunks on the streaming kernel, never the general one
     for m, k, launches in [(1, 30976, 2), (1, 61440, 2), (1, 61696, 3), (2, 15360, 1),
-                           (2, 15616, 2), (3, 7680, 1), (3, 7936, 2), (4, 15616, 4)]:
+                           (2, 15616, 2)]:
         p = q4k.q4k_gemv_plan_for(m, 64, k, SM_COUNT)
         assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["launches"] == launches, (m, k, p)
     # the fused SwiGLU beyond the streaming range stays on the general kernel
@@ -256,14 +297,13 @@ def test_kernel_choice():
 
 
 def test_batches_beyond_eight_vectors():
-    """m > 8 runs as vector tiles (the realizar page tiles batches over 8):
-    groups of four on the streaming kernel, each K-chunked where K is beyond a
-    team; m > 64 is refused."""
-    assert q4k.q4k_gemv_plan_for(16, 14336, 4096, SM_COUNT)["launches"] == 4
-    assert q4k.q4k_gemv_plan_for(33, 4096, 4096, SM_COUNT)["launches"] == 9
-    assert q4k.q4k_gemv_plan_for(64, 4096, 4096, SM_COUNT)["launches"] == 16
+    """m > 16 runs as vector groups of 16 on the tensor-core kernel (the
+    realizar page tiles batches); m > 64 is refused."""
+    assert q4k.q4k_gemv_plan_for(16, 14336, 4096, SM_COUNT)["launches"] == 2
+    assert q4k.q4k_gemv_plan_for(33, 4096, 4096, SM_COUNT)["launches"] == 6
+    assert q4k.q4k_gemv_plan_for(64, 4096, 4096, SM_COUNT)["launches"] == 8
     p = q4k.q4k_gemv_plan_for(20, 64, 30976, SM_COUNT)
-    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["launches"] == 10 * 3
+    assert p["kernel"] == q4k.Q4K_KERNEL_TC and p["launches"] == 4
     with pytest.raises(q4k.Q4KError):
         q4k.q4k_gemv_plan_for(65, 4096, 4096, SM_COUNT)
 
