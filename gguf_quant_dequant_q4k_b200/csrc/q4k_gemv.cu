@@ -113,24 +113,9 @@ void launch_rows(const q4k_gemv_plan& plan, const void* w, const void* w2, const
 
 namespace {
 
-// Vectors per streaming launch: 1 or 2 for m <= 2. For m >= 3, groups of
-// four on half slices (each decoded superblock applied to the four vectors;
-// the last group padded up to four if it has three vectors, run on the one-
-// or two-vector kernel if it has one or two) where one launch of that kernel
-// covers K (K <= 7680); beyond that, pairs, which measured faster on B200 than
-// K-chunked groups of four (4096 x 14336, m = 4: 41.8 us as two pair launches,
-// 46.8 us as two K-chunks of the four-vector kernel; 14336 x 4096, m = 4:
-// 39.4 us as one four-vector launch, 40.2 us as two pairs). The fused SwiGLU
-// runs pairs.
-int group_size(int m, int nsb, bool fused) {
-    if (fused || m <= 2) return m <= 2 ? m : 2;
-    return nsb <= stream_max_nsb(4, 0) ? 4 : 2;
-}
-
-int kernel_vectors(int mi, bool fused) {
-    if (fused) return mi;
-    return mi >= 3 ? 4 : mi;
-}
+// Vectors per streaming launch: 1 or 2 (q4k_gemv runs m >= 3 on the
+// tensor-core kernel); the fused SwiGLU runs any m as pairs.
+int group_size(int m) { return m <= 2 ? m : 2; }
 
 // K split into the fewest equal chunks (whole superblocks) one team covers:
 // each chunk is a launch over strided row segments, later chunks adding into y.
@@ -139,7 +124,7 @@ struct KChunks {
 };
 
 KChunks k_chunks(int mk, int nsb) {
-    const int maxnsb = stream_max_nsb(mk, mk == 1 ? 2 : (mk == 2 ? 1 : 0));
+    const int maxnsb = stream_max_nsb(mk, mk == 1 ? 2 : 1);
     KChunks c{1, nsb};
     if (maxnsb <= 0 || nsb <= maxnsb) return c;
     c.count = (nsb + maxnsb - 1) / maxnsb;
@@ -177,8 +162,7 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
     StreamParams q{};
     int grid = 0, block = 0, smem = 0;
     const int nsb = k / kQK;
-    const int gsz = group_size(m, nsb, fused);
-    const int mk = kernel_vectors(gsz, fused);
+    const int mk = group_size(m);
     const int* cl = max_clusters;
     bool ok = plan_stream(mk, n, k, num_sms, max_smem, cl, fused, &q, &grid, &block, &smem) != 0;
     int chunks = 1;
@@ -197,7 +181,7 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
         plan->smem_bytes = smem;
         plan->teams = q.teams;
         plan->depth = q.depth;
-        plan->launches = ((m + gsz - 1) / gsz) * chunks;
+        plan->launches = ((m + mk - 1) / mk) * chunks;
         plan->cluster = q.cluster;
         plan->units = n;
         plan->units_per_cta_max = q.rows_base + (q.rows_extra > 0 ? 1 : 0);
@@ -233,16 +217,14 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const floa
     q4k_gemv_plan plan;
     const bool fused = w2 != nullptr;
     if (use_tc(m, fused)) return launch_gemv_tc(dev, w, x, y, m, n, k, stream);
-    const int gsz = group_size(m, k / kQK, fused);
+    const int gsz = group_size(m);
     int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin,
-                              dev.max_clusters[kernel_vectors(gsz, fused) == 1 ? 0 : 1], fused,
-                              &plan, nullptr);
+                              dev.max_clusters[gsz == 1 ? 0 : 1], fused, &plan, nullptr);
     if (st != Q4K_OK) return st;
     if (plan.kernel == Q4K_KERNEL_STREAM) {
         const int nsb = k / kQK;
         for (int i0 = 0; i0 < m; i0 += gsz) {
-            const int mi = (m - i0) < gsz ? (m - i0) : gsz;      // vectors of this group
-            const int mk = kernel_vectors(mi, fused);           // the kernel's M
+            const int mk = (m - i0) < gsz ? (m - i0) : gsz;     // vectors of this group
             const int* cl = dev.max_clusters[mk == 1 ? 0 : 1];
             StreamParams sp;
             int g = 0, b = 0, sm = 0;
@@ -260,7 +242,6 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const floa
                 sp.sb_off = sb0;
                 sp.x_stride = k;
                 sp.accumulate = ci > 0 ? 1 : 0;
-                sp.m_valid = mi;
                 st = launch_stream(sp, g, b, sm, w, w2,
                                    x + static_cast<size_t>(i0) * k + static_cast<size_t>(sb0) * kQK,
                                    y + static_cast<size_t>(i0) * n, mk, stream);

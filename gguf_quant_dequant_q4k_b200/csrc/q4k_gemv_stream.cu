@@ -213,42 +213,6 @@ __device__ __forceinline__ void decode_half(uint4 h, float d, float dmin, int ha
     err = make_float4(-e01.x, -e01.y, -e23.x, -e23.y);
 }
 
-// As decode_half for the single 64-weight group g (sub-blocks 2g, 2g+1):
-// out = (A_2g, A_2g+1, B_2g, B_2g+1), err = (-e_2g, -e_2g+1).
-// exact: out = (A_2g, A_2g+1, -A_2g/2, -A_2g+1/2), err = (-dmin*m_2g, -dmin*m_2g+1)
-// instead (the weight formed as fma(A, f, -A/2) + (-dmin*m), rounded once).
-__device__ __forceinline__ void decode_group(uint4 h, float d, float dmin, int g, float4& out,
-                                             float2& err, bool exact = false) {
-    const int half = g >> 1;
-    const uint32_t sc = half ? ((h.w & 0x0F0F0F0Fu) | ((h.y >> 2) & 0x30303030u))
-                             : (h.y & 0x3F3F3F3Fu);
-    const uint32_t mm = half ? (((h.w >> 4) & 0x0F0F0F0Fu) | ((h.z >> 2) & 0x30303030u))
-                             : (h.z & 0x3F3F3F3Fu);
-    const uint32_t s0 = static_cast<uint32_t>((g & 1) * 2);   // bytes s0, s0 + 1 of the half
-    const float d128 = d * 128.0f;
-    const float2 sa = make_float2(d128, d128);
-    const float2 sb2 = make_float2(-8388608.0f * d128, -8388608.0f * d128);
-    const float2 ma = make_float2(dmin, dmin);
-    const float2 mb = make_float2(-8388608.0f * dmin, -8388608.0f * dmin);
-    const float2 scf = make_float2(__uint_as_float(__byte_perm(sc, kMagic2p23, 0x7650 | s0)),
-                                   __uint_as_float(__byte_perm(sc, kMagic2p23, 0x7650 | (s0 + 1))));
-    const float2 mmf = make_float2(__uint_as_float(__byte_perm(mm, kMagic2p23, 0x7650 | s0)),
-                                   __uint_as_float(__byte_perm(mm, kMagic2p23, 0x7650 | (s0 + 1))));
-    const float2 a = ffma2(sa, scf, sb2);   // 128 d sc (exact)
-    const float2 m = ffma2(ma, mmf, mb);    // dmin m (exact)
-    const float2 A = __fadd2_rn(a, a);
-    const float2 sm = __fadd2_rn(a, m);
-    const float2 v = fsub2(sm, a);
-    const float2 e = __fadd2_rn(fsub2(a, fsub2(sm, v)), fsub2(m, v));
-    if (exact) {
-        out = make_float4(A.x, A.y, -a.x, -a.y);
-        err = make_float2(-m.x, -m.y);
-        return;
-    }
-    out = make_float4(A.x, A.y, -sm.x, -sm.y);
-    err = make_float2(-e.x, -e.y);
-}
-
 // kWords consecutive 32-bit words of quant bytes from shared memory (one
 // 8- or 16-byte load per 16 bytes).
 template <int kWords>
@@ -281,25 +245,15 @@ __device__ __forceinline__ void header_scales(uint4 h, float& d, float& dmin) {
 // per vector (measured faster on B200 than four split chains: fewer
 // instructions, and the other warps hide the chain's latency); `first`
 // initialises the chain.
-// EXACT: b = -A/2 (so A*f + b = d*sc*q exactly) and the weight is completed
-// as (d*sc*q) + mneg, mneg = (-dmin*m_2g, -dmin*m_2g+1): rounded once, with no
-// correction term (used where registers are too scarce for the per-lane x sums).
-template <int M, int NX, bool EXACT = false>
+template <int M, int NX>
 __device__ __forceinline__ void dot_word(uint32_t w, float2 a, float2 b, const float2 (&xp)[M][NX],
-                                         int e0, bool first, float2 (&acc)[M],
-                                         float2 mneg = make_float2(0.f, 0.f)) {
+                                         int e0, bool first, float2 (&acc)[M]) {
     const uint32_t lo = w & 0x0F0F0F0Fu;
     const uint32_t hi = __umulhi(w, 1u << 28) & 0x0F0F0F0Fu;   // (w >> 4) on the FMA pipe
     float2 w0 = ffma2(a, make_float2(nib_to_f<0>(lo), nib_to_f<0>(hi)), b);
     float2 w1 = ffma2(a, make_float2(nib_to_f<1>(lo), nib_to_f<1>(hi)), b);
     float2 w2 = ffma2(a, make_float2(nib_to_f<2>(lo), nib_to_f<2>(hi)), b);
     float2 w3 = ffma2(a, make_float2(nib_to_f<3>(lo), nib_to_f<3>(hi)), b);
-    if (EXACT) {
-        w0 = __fadd2_rn(w0, mneg);
-        w1 = __fadd2_rn(w1, mneg);
-        w2 = __fadd2_rn(w2, mneg);
-        w3 = __fadd2_rn(w3, mneg);
-    }
 #pragma unroll
     for (int i = 0; i < M; ++i) {
         acc[i] = first ? __fmul2_rn(w0, xp[i][e0 + 0]) : ffma2(w0, xp[i][e0 + 0], acc[i]);
@@ -454,18 +408,15 @@ __device__ __forceinline__ float& row_out_ref(const StreamParams& p, uint8_t* sm
     return p.y[static_cast<size_t>(i) * p.n + row];
 }
 
-// Finishes row `row` of vector i: y = tot, or y += tot for a later K-chunk;
-// vectors beyond m_valid (padding of a partial vector group) are not stored.
+// Finishes row `row` of vector i: y = tot, or y += tot for a later K-chunk.
 template <bool FUSED>
 __device__ __forceinline__ void store_row(const StreamParams& p, uint8_t* smem, int i, long long row,
                                           float tot) {
-    if (i >= p.m_valid) return;
     float& r = row_out_ref<FUSED>(p, smem, i, row);
     r = p.accumulate ? r + tot : tot;
 }
 
-// M vectors, S 16-byte quant slices (S*32 weights) per lane per row; S = 0:
-// one 8-byte half slice (16 weights).
+// M vectors, S 16-byte quant slices (S*32 weights) per lane per row.
 template <int M, int S, bool FUSED>
 __global__ void __maxnreg__(stream_max_regs(M, S))
 q4k_gemv_stream_kernel(const StreamParams p) {
@@ -475,10 +426,6 @@ q4k_gemv_stream_kernel(const StreamParams p) {
     constexpr int kPos = pos_per_warp(S);          // superblock positions per warp
     constexpr int kNX = lane_bytes(S);             // x pairs per lane per vector
     constexpr int kWords = kNX / 4;                // 32-bit quant words per lane and row
-    // Four vectors (half slices): weights formed exactly (one more packed add
-    // per weight pair) instead of the per-lane x sums of the correction term,
-    // which would not fit the registers beside four vectors' x.
-    constexpr bool kExactW = (M >= 4);
     const int nsb = p.nsb;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -626,18 +573,15 @@ q4k_gemv_stream_kernel(const StreamParams p) {
             // their latency overlaps the first stage's wait and decode. Plain
             // (coherent, L1-allocating) loads: measured on B200 the
             // non-coherent path made the K = 14336 call 10 % slower.
-            // A vector past m_valid (padding) reads vector 0's x and uses zeros.
             const int k0 = (valid ? bl : 0) * kQK + 64 * g + b0;
-            const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < M; ++i) {
-                const bool vi = i < p.m_valid;
                 const float4* xl = reinterpret_cast<const float4*>(
-                    p.x + static_cast<size_t>(vi ? i : 0) * p.x_stride + k0);
+                    p.x + static_cast<size_t>(i) * p.x_stride + k0);
                 const float4* xh = xl + 8;   // + 32 weights
 #pragma unroll
                 for (int v = 0; v < kNX / 4; ++v) {
-                    const float4 a = vi ? xl[v] : zero4, b = vi ? xh[v] : zero4;
+                    const float4 a = xl[v], b = xh[v];
                     xp[i][4 * v + 0] = make_float2(a.x, b.x);
                     xp[i][4 * v + 1] = make_float2(a.y, b.y);
                     xp[i][4 * v + 2] = make_float2(a.z, b.z);
@@ -651,7 +595,6 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         float2 sx[M];
 #pragma unroll
         for (int i = 0; i < M; ++i) {
-            if (kExactW) continue;
             sx[i] = xp[i][0];
 #pragma unroll
             for (int e = 1; e < kNX; ++e) sx[i] = __fadd2_rn(sx[i], xp[i][e]);
@@ -668,12 +611,10 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const uint32_t lane_coef_off =
             coef_off + static_cast<uint32_t>((lpos * 4 + (g ^ ((lpos >> 1) & 3))) * 16);
         // Decode lanes: S = 2: lane -> (segment du, position dpos), whole header;
-        // S = 1: lane -> (segment du, position dpos, half dhalf); S = 0: lane ->
-        // (segment du, position dpos, group dgrp).
+        // S = 1: lane -> (segment du, position dpos, half dhalf).
         const int du = lane >> 3;
-        const int dpos = S == 2 ? (lane & 7) : (S == 1 ? ((lane >> 1) & 3) : ((lane >> 2) & 1));
+        const int dpos = S == 2 ? (lane & 7) : ((lane >> 1) & 3);
         const int dhalf = S == 1 ? (lane & 1) : 0;
-        const int dgrp = lane & 3;
         const int dbl = wit * kPos + dpos;
         const uint32_t dec_base = coef_off + static_cast<uint32_t>((du * kPos + dpos) * 4 * 16);
         const int dswz = (dpos >> 1) & 3;
@@ -710,13 +651,6 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                     header_scales(hdr, d, dmin);
                     const uint32_t cb = dec_base + static_cast<uint32_t>(dg * 4 * kPos * 4 * 16);
                     const uint32_t eb = dec_err + static_cast<uint32_t>(dg * 4 * kPos * 4 * 8);
-                    if (S == 0) {
-                        float4 c_g;
-                        float2 e_g;
-                        decode_group(hdr, d, dmin, dgrp, c_g, e_g, kExactW);
-                        *reinterpret_cast<float4*>(smem + cb + (dgrp ^ dswz) * 16) = c_g;
-                        *reinterpret_cast<float2*>(smem + eb + dgrp * 8) = e_g;
-                    }
 #pragma unroll
                     for (int hh = 0; hh < S; ++hh) {
                         const int half = S == 2 ? hh : dhalf;
@@ -766,10 +700,10 @@ q4k_gemv_stream_kernel(const StreamParams p) {
                 float2 acc[M];
 #pragma unroll
                 for (int j = 0; j < kWords; ++j)
-                    dot_word<M, kNX, kExactW>(q[j], a, b, xp, 4 * j, j == 0, acc, ne);
+                    dot_word<M, kNX>(q[j], a, b, xp, 4 * j, j == 0, acc);
 #pragma unroll
                 for (int i = 0; i < M; ++i) {
-                    if (!kExactW) acc[i] = ffma2(ne, sx[i], acc[i]);   // remove B's rounding error
+                    acc[i] = ffma2(ne, sx[i], acc[i]);   // remove B's rounding error
                     part_sum[i][u] = use[u] ? (acc[i].x + acc[i].y) : 0.f;
                 }
             };
@@ -880,18 +814,17 @@ int resident_clusters(int c, int num_sms, const int* max_clusters) {
 }  // namespace
 
 int stream_max_nsb(int m, int slices) {
-    if ((m == 4) != (slices == 0)) return 0;   // four vectors on half slices, else whole slices
+    if (m < 1 || m > kStreamMaxM || slices < 1 || slices > 2) return 0;
     // the warps of one team (one CTA's compute warps) times positions per warp
     const int by_warps = (stream_max_threads(m, slices) / 32) * pos_per_warp(slices);
-    const int cap = kStreamMaxNsb * (slices == 0 ? 1 : slices);
+    const int cap = kStreamMaxNsb * slices;
     return by_warps < cap ? by_warps : cap;
 }
 
 int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
                 bool fused, StreamParams* sp, int* grid, int* block, int* smem_bytes) {
     const int nsb = k / kQK;
-    if (m < 1 || m > kStreamMaxM || m == 3 || n < 1) return 0;
-    if (m == 4 && fused) return 0;
+    if (m < 1 || m > kStreamMaxM || n < 1) return 0;
     // Compact CTAs: at most half of an SM's registers and shared memory, so
     // that a CTA of the next kernel on the stream can be resident beside it
     // (programmatic dependent launch then runs its prologue and first weight
@@ -900,13 +833,11 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     // classic CTA's extra warps pay; measured on B200, LM head 128256 x 4096:
     // 100.9 us classic, 118.6 us compact.)
     const bool tall = (n + num_sms - 1) / num_sms >= kWideMinRows;
-    const bool compact_ok = kPlanMode != 0 && !(kPlanMode == 3 && tall) && m <= 2;
+    const bool compact_ok = kPlanMode != 0 && !(kPlanMode == 3 && tall);
     // quant slices per lane: two for one vector on very tall matrices, for one
     // vector when K is too long for one-slice teams (K > 20480: a team of
     // two-slice lanes covers K <= 30720 with 15 warps), and for a compact CTA
-    // whose one-slice team would not fit its warps; four vectors run on 8-byte
-    // half slices (16 weights per lane: 64 registers of x, as for two vectors
-    // on one slice)
+    // whose one-slice team would not fit its warps
     const int compact_warps1 = kCompactRegs / (stream_max_regs(m, 1) * 32) - 1;
     const bool compact_s1 = compact_ok && (nsb * 8 + 31) / 32 <= compact_warps1;
     const bool compact_s2 = compact_ok && m == 1 && !fused &&
@@ -915,7 +846,7 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     const bool wide = m == 1 && !fused &&
                       ((n + num_sms - 1) / num_sms >= kWideMinRows || nsb > kStreamMaxNsb ||
                        (compact && !compact_s1));
-    const int sl = m == 4 ? 0 : (wide ? 2 : 1);
+    const int sl = wide ? 2 : 1;
     if (nsb > stream_max_nsb(m, sl)) return 0;
     const int team_warps = (nsb * lanes_per_sb(sl) + 31) / 32;
     const int max_warps = compact ? kCompactRegs / (stream_max_regs(m, sl) * 32) - 1
@@ -991,7 +922,6 @@ int plan_stream(int m, int n, int k, int num_sms, int max_smem, const int* max_c
     q.sb_off = 0;
     q.x_stride = k;
     q.accumulate = 0;
-    q.m_valid = m;
     size_t off = static_cast<size_t>(teams) * depth * stage_bytes;
     q.off_coef = static_cast<int>(off);
     off += static_cast<size_t>(teams) * team_warps * coef_bytes_per_warp(sl);
@@ -1042,10 +972,8 @@ int launch_stream(const StreamParams& sp0, int grid, int block, int smem_bytes, 
     } else if (m == 1) {
         e = sp.slices == 2 ? cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, 2, false>, sp)
                            : cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<1, 1, false>, sp);
-    } else if (m == 2) {
-        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, 1, false>, sp);
     } else {
-        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<4, 0, false>, sp);
+        e = cudaLaunchKernelEx(&cfg, q4k_gemv_stream_kernel<2, 1, false>, sp);
     }
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
@@ -1065,9 +993,6 @@ int stream_set_attributes() {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<2, 1, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_stream_kernel<4, 0, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmemBudget);
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }

@@ -10,12 +10,12 @@ namespace q4k {
 // slower than 4 on every decode shape (register spills, LM head 101.7 ->
 // 110.3 us).
 constexpr int kStreamSegRows = 4;
-constexpr int kStreamMaxM = 4;          // vectors handled by one streaming launch (1, 2 or 4)
+constexpr int kStreamMaxM = 2;          // vectors handled by one streaming launch (1 or 2)
 
-// Lane geometry for S 16-byte quant slices per lane and row (S = 0: one
-// 8-byte half slice): quant bytes per lane and row, lanes per superblock,
-// superblock positions per warp.
-__host__ __device__ constexpr int lane_bytes(int s) { return s == 0 ? 8 : 16 * s; }
+// Lane geometry for S 16-byte quant slices per lane and row (S = 1 or 2):
+// quant bytes per lane and row, lanes per superblock, superblock positions
+// per warp.
+__host__ __device__ constexpr int lane_bytes(int s) { return 16 * s; }
 __host__ __device__ constexpr int lanes_per_sb(int s) { return 128 / lane_bytes(s); }
 __host__ __device__ constexpr int pos_per_warp(int s) { return 32 / lanes_per_sb(s); }
 // Quant slices (16 bytes = 32 weights) per lane and row: 1, or 2 for one
@@ -27,8 +27,8 @@ __host__ __device__ constexpr int pos_per_warp(int s) { return 32 / lanes_per_sb
 constexpr int kWideMinRows = 512;
 // Compute threads per CTA (plus one producer warp): one slice, one vector: 20
 // warps (x: 32 registers per lane; five or six warps per sub-partition at 80
-// registers; 23 measured no faster); two vectors, two slices, or four vectors
-// on half slices: 15 warps (x: 64 registers per lane; four warps per
+// registers; 23 measured no faster); two vectors or two slices: 15 warps (x:
+// 64 registers per lane; four warps per
 // sub-partition at 128 registers).
 __host__ __device__ constexpr int stream_max_threads(int m, int slices) {
     return (m == 1 && slices == 1) ? 640 : 480;
@@ -73,7 +73,6 @@ struct StreamParams {
     // and vectors are x_stride floats apart.
     int nsb_row, sb_off, x_stride;
     int accumulate;             // 1: y += the chunk's sums (a later K-chunk); 0: y = sums
-    int m_valid;                // vectors present (<= the kernel's M; the rest are padding)
 };
 
 // Launch policy. 0: one CTA per SM with up to 20 compute warps and 220 KiB

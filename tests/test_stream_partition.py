@@ -46,31 +46,28 @@ def stream_regs(m, slices):
 
 def lane_geometry(slices):
     """(quant bytes per lane and row, lanes per superblock, positions per
-    warp): slices 16-byte quant slices per lane, 0 meaning one 8-byte half."""
-    lb = 8 if slices == 0 else 16 * slices
+    warp): slices (1 or 2) 16-byte quant slices per lane."""
+    lb = 16 * slices
     return lb, 128 // lb, 32 // (128 // lb)
 
 
-def kernel_vectors(m, fused=False, k=None):
-    """Vectors one streaming launch carries: 1, 2, or 4 (groups of four for
-    m >= 3 where one four-vector launch covers K <= 7680, else pairs; the
-    fused SwiGLU runs pairs)."""
-    if fused or m <= 2:
-        return min(m, 2)
-    return 4 if k is None or k <= 7680 else 2
+def kernel_vectors(m):
+    """Vectors one streaming launch carries: 1 or 2 (the streaming kernel runs
+    m <= 2 for q4k_gemv, and pairs for the fused SwiGLU)."""
+    return min(m, 2)
 
 
 def max_nsb(mk, slices):
     threads = 640 if (mk == 1 and slices == 1) else 480
-    return min((threads // 32) * lane_geometry(slices)[2], 80 * max(slices, 1))
+    return min((threads // 32) * lane_geometry(slices)[2], 80 * slices)
 
 
 def k_chunk_nsbs(m, k):
     """Superblocks of each K-chunk the library launches for the first vector
     group: the fewest equal chunks one team covers (the last may be shorter)."""
-    mk = kernel_vectors(m, k=k)
+    mk = kernel_vectors(m)
     nsb = k // 256
-    top = max_nsb(mk, 2 if mk == 1 else (1 if mk == 2 else 0))
+    top = max_nsb(mk, 2 if mk == 1 else 1)
     if nsb <= top:
         return [nsb]
     count = -(-nsb // top)
@@ -86,9 +83,7 @@ def expected_launch(m, n, k, fused):
     compact one-slice team would not fit. Returns (compact, slices, max compute
     warps, CTAs per SM, shared-memory cap)."""
     nsb = k // 256
-    mi = kernel_vectors(m, fused, k)
-    if mi == 4:    # four vectors: half slices, one CTA per SM, up to 15 compute warps
-        return False, 0, 15, 1, 220 * 1024
+    mi = kernel_vectors(m)
     tall = -(-n // SM_COUNT) >= 512
     cw = lambda regs: 32768 // (regs * 32) - 1
     compact_s1 = (not tall) and -(-nsb * 8 // 32) <= cw(stream_regs(mi, 1))
@@ -109,7 +104,7 @@ def check_plan(m, n, k):
     if p["kernel"] != q4k.Q4K_KERNEL_STREAM:
         return p
     chunks = k_chunk_nsbs(m, k)
-    mk0 = kernel_vectors(m, k=k)
+    mk0 = kernel_vectors(m)
     groups = -(-m // mk0)
     assert p["launches"] == groups * len(chunks)
     assert sum(chunks) == k // 256 and max(chunks) <= max_nsb(mk0, p["slices"])
