@@ -37,7 +37,8 @@ import q4k_synth  # noqa: E402
 
 METRIC = ("Q4_K GEMV µs/call & achieved HBM GB/s (% of B200 peak), m=1, "
           "N×K sweep")
-SWEEP = q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B + q4k_synth.SHAPES_8B
+FULL_SWEEP = q4k_synth.SHAPES_1P5B + q4k_synth.SHAPES_7B + q4k_synth.SHAPES_8B
+SWEEP = FULL_SWEEP
 WORKLOAD = ("Q4_K GEMV m=1 decode sweep, one call per projection: "
             + ", ".join(f"{n}x{k}" for n, k in SWEEP))
 NOMINAL_HBM_GBS = 8000.0
@@ -50,12 +51,13 @@ def bytes_counted(n: int, k: int, m: int = 1) -> int:
 
 
 BYTES_PER_STEP = sum(bytes_counted(n, k) for n, k in SWEEP)
+VECTORS = 1   # vectors per call of the timed sweep (--vectors, profiling runs only)
 
 
 def workload_config(world: int) -> dict:
     """The `config` of the JSON line: the same for the GPU arm and the oracle arm."""
     return {
-        "workload": WORKLOAD, "m": 1, "bytes_per_step": BYTES_PER_STEP,
+        "workload": WORKLOAD, "m": VECTORS, "bytes_per_step": BYTES_PER_STEP,
         "bytes_rule": "N*K/256*144 + 4*m*(K+N) per call",
         "l2": (f"inputs larger than L2: {BYTES_PER_STEP / 1e6:.0f} MB of Q4_K per step and two "
                f"rotating copies of every W, so a copy is re-read only after "
@@ -527,22 +529,23 @@ def run_ours(args) -> None:
     # after more than 2 x L2 of other traffic
     shapes = []
     for n, k in SWEEP:
-        w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS[(n, k)])
+        seed = q4k_synth.SEEDS.get((n, k), q4k_synth.SEED_MULTIVEC.get((n, k)))
+        w, x = q4k_synth.q4k_problem(n, k, VECTORS, seed)
         wdev = torch.from_numpy(w).to(dev)
         copies = max(2, -(-2 * l2 // w.nbytes) + 1)
         ws = [wdev] + [wdev.clone() for _ in range(copies - 1)]
         xdev = torch.from_numpy(x).to(dev)
-        ydev = torch.empty((1, n), dtype=torch.float32, device=dev)
+        ydev = torch.empty((VECTORS, n), dtype=torch.float32, device=dev)
         shapes.append({"n": n, "k": k, "ws": ws, "x": xdev, "y": ydev, "x_host": x})
     torch.cuda.synchronize(dev)
-    plans = [q4k.q4k_gemv_plan_for(1, s["n"], s["k"], props.multi_processor_count)
+    plans = [q4k.q4k_gemv_plan_for(VECTORS, s["n"], s["k"], props.multi_processor_count)
              for s in shapes]
     launches_per_step = sum(p["launches"] for p in plans)
 
     def sweep(step_index: int):
         for s in shapes:
             w = s["ws"][step_index % 2]
-            q4k.q4k_gemv(w, s["x"], s["y"], 1, s["n"], s["k"], stream=stream)
+            q4k.q4k_gemv(w, s["x"], s["y"], VECTORS, s["n"], s["k"], stream=stream)
 
     # CUDA graphs of GRAPH_STEPS steps and of one step (copies alternate step
     # to step; an even GRAPH_STEPS keeps the alternation across replays)
@@ -676,6 +679,7 @@ def run_ours(args) -> None:
         return
 
     achieved = BYTES_PER_STEP / (ms_per_step * 1e-3) / 1e9   # per GPU, all launches of a step
+    full_sweep = VECTORS == 1 and SWEEP == FULL_SWEEP
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": (warm_replays * GRAPH_STEPS + 1) if use_graph else warm_steps,
@@ -692,8 +696,10 @@ def run_ours(args) -> None:
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_kind": f"{peak_kind} copy bandwidth",
             "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
-            "traffic": committed_traffic(), "algorithmic_bytes": BYTES_PER_STEP,
-            "per": "one step = the 8 q4k_gemv launches of the sweep",
+            "traffic": committed_traffic() if full_sweep else None,
+            "algorithmic_bytes": BYTES_PER_STEP,
+            "per": (f"one step = the {len(shapes)} q4k_gemv calls ({launches_per_step} "
+                    f"launches) of the {'sweep' if full_sweep else 'subset'}"),
             "kernel": "q4k_gemv",
         },
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -725,19 +731,27 @@ def main():
                     help="comma-separated NxK subset of the sweep (profiling runs only)")
     ap.add_argument("--skip-extras", action="store_true",
                     help="skip the per-shape and end-to-end passes (profiling runs only)")
+    ap.add_argument("--vectors", type=int, default=1,
+                    help="vectors per call of the timed sweep (profiling runs only: needs "
+                         "--shapes and --skip-extras; the multi-vector shapes are allowed)")
     ap.add_argument("--prefill-only", action="store_true",
                     help="print only the prefill (fp16 mirror + tensor-core GEMM) figures")
     args = ap.parse_args()
     if args.steps < 1 or args.warmup < 0:
         raise SystemExit("--steps must be >= 1 and --warmup >= 0")
+    if args.vectors != 1 and not (args.shapes and args.skip_extras):
+        raise SystemExit("--vectors needs --shapes and --skip-extras")
     if args.shapes:
-        global SWEEP, BYTES_PER_STEP, WORKLOAD
+        global SWEEP, BYTES_PER_STEP, WORKLOAD, VECTORS
+        VECTORS = args.vectors
         SWEEP = [tuple(int(v) for v in s.lower().split("x")) for s in args.shapes.split(",")]
         for sh in SWEEP:
-            if sh not in q4k_synth.SEEDS:
+            if sh not in q4k_synth.SEEDS and not (VECTORS > 1 and sh in q4k_synth.SEED_MULTIVEC):
                 raise SystemExit(f"shape {sh} is not one of the sweep's")
-        BYTES_PER_STEP = sum(bytes_counted(n, k) for n, k in SWEEP)
+        BYTES_PER_STEP = sum(bytes_counted(n, k, VECTORS) for n, k in SWEEP)
         WORKLOAD = "subset of the sweep: " + ", ".join(f"{n}x{k}" for n, k in SWEEP)
+        if VECTORS > 1:
+            WORKLOAD += f", {VECTORS} vectors per call"
     if args.prefill_only:
         import torch
         import gguf_quant_dequant_q4k_b200 as q4k

@@ -147,5 +147,59 @@ def test_tc_deterministic_and_rows_only(q4k):
     assert_gemv_close(y.cpu().numpy().reshape(m, n), yref, a, "rows")
 
 
+def test_tc_lm_head_sampled(q4k):
+    """m = 4 on the 128256 x 4096 LM head: 16032 items over the CTAs, several
+    tiles per CTA and a cut tile at most CTA boundaries; 40 sampled rows."""
+    n, k, m = 128256, 4096, 4
+    w, x = q4k_synth.q4k_problem(n, k, m, 8)
+    y = gpu_gemv(q4k, w, x, n, k)
+    rows = np.unique(np.concatenate([[0, 127, 128, n - 1], np.random.default_rng(3).integers(0, n, 36)]))
+    yref, a = oracle.gemv_rows(w, x, n, k, rows)
+    assert_gemv_close(y[:, rows], yref, a, "LM head m=4")
+
+
+def test_tc_graph_capture_and_two_streams(q4k):
+    """Calls captured in a CUDA graph (the call's stream-ordered workspace
+    becomes graph memory nodes) replay to the eager result; calls on two
+    streams at once (one workspace each) both match it."""
+    n, k, m = 1000, 2048, 6
+    w, x = q4k_synth.q4k_problem(n, k, m, 17)
+    wt, xt = dev(w), dev(x.reshape(m, k))
+    eager = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    q4k.q4k_gemv(wt, xt, eager, m, n, k)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    ys = [torch.full((m, n), float("nan"), device="cuda") for _ in range(3)]
+    with torch.cuda.stream(s):   # warm-up outside capture
+        q4k.q4k_gemv(wt, xt, ys[0], m, n, k, stream=s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for y in ys:
+            q4k.q4k_gemv(wt, xt, y, m, n, k, stream=s)
+    for y in ys:
+        y.fill_(float("nan"))
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        g.replay()
+        g.replay()
+    s.synchronize()
+    for y in ys:
+        assert torch.equal(y.view(torch.int32), eager.view(torch.int32))
+    del g
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    y1 = torch.full((m, n), float("nan"), device="cuda")
+    y2 = torch.full((m, n), float("nan"), device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(5):
+        q4k.q4k_gemv(wt, xt, y1, m, n, k, stream=s1)
+        q4k.q4k_gemv(wt, xt, y2, m, n, k, stream=s2)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int32), eager.view(torch.int32))
+    assert torch.equal(y2.view(torch.int32), eager.view(torch.int32))
+    yref, a = oracle.gemv(w, x, n, k)
+    assert_gemv_close(eager.cpu().numpy(), yref, a, "eager")
+
+
 def test_tc_no_fault_flags(q4k):
     assert q4k.q4k_device_fault_flags() == 0
