@@ -32,6 +32,7 @@ Q4K_PREFILL_NOALLOC_MAX_ELEMS = 8388608
 Q4K_KERNEL_WARP_ROWS = 1
 Q4K_KERNEL_STREAM = 2
 Q4K_KERNEL_TC = 3
+Q4K_KERNEL_I8 = 4
 
 # Every function include/q4k.h declares.
 EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",

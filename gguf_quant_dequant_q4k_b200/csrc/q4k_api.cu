@@ -17,6 +17,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "q4k_gemv_i8.h"
 #include "q4k_gemv_tc.h"
 #include "q4k_internal.h"
 #include "q4k_stream.h"
@@ -73,6 +74,8 @@ int current_device_info(DeviceInfo* info) {
             g_dev_status[dev] = q4k_last_cuda_error_value();
         if (g_dev_status[dev] == 0 && tc_set_attributes() != Q4K_OK)
             g_dev_status[dev] = q4k_last_cuda_error_value();
+        if (g_dev_status[dev] == 0 && i8_set_attributes() != Q4K_OK)
+            g_dev_status[dev] = q4k_last_cuda_error_value();
         if (g_dev_status[dev] == 0) {
             stream_cluster_occupancy(1, g_dev[dev].max_clusters[0]);
             stream_cluster_occupancy(2, g_dev[dev].max_clusters[1]);
@@ -112,7 +115,7 @@ int q4k_last_cuda_error(void) { return t_last_cuda_error; }
 
 int q4k_device_fault_flags(unsigned int* flags) {
     if (flags == nullptr) return Q4K_ERR_NULL;
-    unsigned a = 0, b = 0, c = 0, t = 0;
+    unsigned a = 0, b = 0, c = 0, t = 0, i = 0;
     int st = read_fault_flags(&a);
     if (st != Q4K_OK) return st;
     st = read_embed_fault_flags(&b);
@@ -121,7 +124,9 @@ int q4k_device_fault_flags(unsigned int* flags) {
     if (st != Q4K_OK) return st;
     st = read_tc_fault_flags(&t);
     if (st != Q4K_OK) return st;
-    *flags = a | b | c | t;
+    st = read_i8_fault_flags(&i);
+    if (st != Q4K_OK) return st;
+    *flags = a | b | c | t | i;
     return Q4K_OK;
 }
 

@@ -12,6 +12,7 @@
 // carries weight 64g+16h+l (low nibble, sub-block 2g) and weight 64g+32+16h+l
 // (high nibble, sub-block 2g+1), with g = c/2, h = c%2. The warp's 32 quant
 // loads are 4 x 128 contiguous bytes.
+#include "q4k_gemv_i8.h"
 #include "q4k_gemv_tc.h"
 #include "q4k_internal.h"
 #include "q4k_stream.h"
@@ -138,8 +139,30 @@ KChunks k_chunks(int mk, int nsb) {
 // launches (digits, GEMV) per group of up to 16 vectors.
 bool use_tc(int m, bool fused) { return !fused && m >= kTcMinM; }
 
+// One vector on a tall matrix (whole 128-row tiles for every SM): the
+// integer tensor-core kernel, one launch.
+bool use_i8(int m, int n, int k, int num_sms, int max_smem, bool fused) {
+    return !fused && i8_applies(m, n, k, num_sms, max_smem);
+}
+
 int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
                      bool fused, q4k_gemv_plan* plan, StreamParams* sp) {
+    if (use_i8(m, n, k, num_sms, max_smem, fused)) {
+        const int tiles = (n + kI8Rows - 1) / kI8Rows;
+        const int grid = i8_ctas(tiles, num_sms);
+        plan->kernel = Q4K_KERNEL_I8;
+        plan->grid = grid;
+        plan->block = i8_threads();
+        plan->smem_bytes = i8_smem_bytes(k / kQK);
+        plan->cluster = 1;
+        plan->teams = 0;
+        plan->depth = i8_wstages(k / kQK);
+        plan->launches = 1;
+        plan->units = tiles;   // whole 128-row tiles
+        plan->units_per_cta_max = (tiles + grid - 1) / grid;
+        plan->slices = 0;
+        return Q4K_OK;
+    }
     if (use_tc(m, fused)) {
         const int tiles = (n + kTcRows - 1) / kTcRows;
         const int grid = tc_ctas(tiles, k / kQK, num_sms);
@@ -216,6 +239,7 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const floa
                 int m, int n, int k, cudaStream_t stream) {
     q4k_gemv_plan plan;
     const bool fused = w2 != nullptr;
+    if (use_i8(m, n, k, dev.sm_count, dev.max_smem_optin, fused)) return launch_gemv_i8(dev, w, x, y, n, k, stream);
     if (use_tc(m, fused)) return launch_gemv_tc(dev, w, x, y, m, n, k, stream);
     const int gsz = group_size(m);
     int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin,

@@ -1,0 +1,550 @@
+// q4k_gemv_i8.cu -- y = W x for Q4_K W and one f32 vector on tall matrices
+// (the LM head of a decode step: the pages' `Q4KGemv` over a vocabulary-sized
+// W, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs"), on the tcgen05
+// tensor cores with 8-bit integer operands. Every product is formed exactly
+// in integers; only the final combination and the output rounding are inexact.
+//
+// * Weights. Weight t of superblock b of a row is d*sc_j*q_t - dmin*m_j
+//   (sub-block j = t/32). The MMA's A operand is the quant nibble itself as an
+//   unsigned byte: the low nibbles of a quant word (w & 0x0F0F0F0F) are four
+//   consecutive weights of sub-block 2g, its high nibbles (w & 0xF0F0F0F0,
+//   i.e. 16 q) four of sub-block 2g+1, so one bit operation decodes four
+//   weights. The decoded superblock column of a tile (128 rows x 256 bytes)
+//   goes to tensor memory with tcgen05.st.
+// * Vector. Each CTA scales every 256-element block b of x to
+//   X = round(x * 2^(33 - E_b)), E_b the exponent of the block's largest |x|
+//   (|X| < 2^33; exact where |x| >= 2^(E_b - 10), else off by at most
+//   2^(E_b - 34)), and splits X into five balanced base-128 digits
+//   X = sum_l 128^l X_l, X_l in [-64, 63], the rows l of the MMA's B operand
+//   (signed bytes; rows 5..7 of the N = 8 operand are not read back).
+// * Products. One MMA (K = 32) per sub-block j, each into its own accumulator
+//   columns: D_j[row][l] = sum over the sub-block of A * X_l, an integer of at
+//   most 32 * 15 * 64 (sixteen times that for odd j). The epilogue forms
+//   S = sum_j sc_j * sum_l 128^l D_j[l] (/16 for odd j) exactly in 64-bit
+//   integers (|S| < 2^52), M = sum_j m_j * S0_j (S0_j: the sum of X over
+//   sub-block j; exact in f64), and adds 2^(E_b - 33) * (d*S - dmin*M) to the
+//   row's f64 total; y is that total rounded to f32 once. So
+//   |y - sum w x| <= 2^-24 (|y| + sum |w x|) + sum_t |w_t| 2^(E_t - 34), the
+//   bound of the batched tensor-core path; non-finite x makes y NaN.
+// * Pipeline. A persistent CTA owns whole 128-row tiles and walks their
+//   superblock columns in order. A producer thread streams each column of a
+//   tile (128 rows x 144 bytes, one 2-D TMA box) through up to eight stages;
+//   two sets of four decode warps (one per TMEM lane quarter), alternate
+//   items each, write A into one of four TMEM buffers and hand each row's
+//   superblock header on through a shared-memory ring; one elected lane of the MMA warp issues the column's 8 MMAs into
+//   one of four accumulators; eight epilogue warps (two per lane quarter,
+//   four sub-blocks each) read the accumulator (tcgen05.ld) and combine it. The digit image of the whole vector stays in
+//   shared memory for the kernel.
+//
+// All waits are bounded: one that gives up raises Q4K_FAULT_COPY_TIMEOUT and
+// the CTA lets its copies and MMAs complete (bounded) before it releases shared
+// and tensor memory.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "q4k_gemv_i8.h"
+#include "q4k_gemv_tc.h"
+#include "q4k_internal.h"
+#include "q4k_sm100.cuh"
+#include "q4k_superblock.cuh"
+#include "q4k_tcgen05.cuh"
+
+namespace q4k {
+
+// Raised (Q4K_FAULT_COPY_TIMEOUT) by a CTA whose bounded wait gave up; read
+// and cleared by q4k_device_fault_flags(). Never set in normal operation.
+__device__ unsigned int g_i8_fault_flags = 0;
+
+namespace {
+
+// Two sets of four decode warps (one warp per TMEM lane quarter each) take
+// alternate items: a warp waits for its tensor-memory stores before it
+// signals the item, and the two sets keep two items' stores in flight.
+constexpr int kI8Quarters = 4;
+constexpr int kI8DecodeSets = 2;
+constexpr int kI8DecodeWarps = kI8Quarters * kI8DecodeSets;   // warps 0-7: decode into TMEM
+constexpr int kI8EpiWarps = 2 * kI8Quarters;                   // warps 8-15: epilogue
+constexpr int kI8ProducerWarp = 16;    // weight copies
+constexpr int kI8MmaWarp = 17;
+constexpr int kI8Warps = 18;
+constexpr int kI8Threads = 32 * kI8Warps;
+constexpr int kI8Limbs = 5;
+constexpr int kI8N = 8;                      // MMA N: digit rows 0..4
+constexpr int kI8ImageBytes = kI8N * kQK;    // one block's digit image (K-major, swizzled)
+constexpr int kI8MetaDoubles = 10;           // 2^(E-33), S0_0..7, pad
+constexpr int kI8RawBytes = kI8Rows * kBlockBytes;
+constexpr int kI8Acols = 64;                 // TMEM columns of one decoded superblock (256 bytes)
+constexpr int kI8ABufs = 4;
+constexpr int kI8Dcols = 8 * kI8N;           // one accumulator: 8 sub-blocks x N columns
+constexpr int kI8DBufs = 4;
+constexpr int kI8Dcol0 = kI8ABufs * kI8Acols;
+constexpr int kI8TmemCols = 512;
+constexpr int kI8HSlots = kI8ABufs + kI8DBufs;   // header ring (see the decode)
+constexpr int kI8HeaderBytes = kI8Rows * 16;      // one column's row headers
+constexpr int kI8Barriers = 2 * kI8MaxWStages + kI8ABufs + 2 * kI8DBufs + 2 * kI8HSlots + 1;
+static_assert(kI8Dcol0 + kI8DBufs * kI8Dcols <= kI8TmemCols, "TMEM buffers");
+// Item it uses A buffer and accumulator it % 4: one commit per item tells the
+// decode that the A buffer is free and the epilogue that the accumulator is
+// complete.
+static_assert(kI8ABufs == kI8DBufs, "A buffers and accumulators share the MMA-done barriers");
+
+// Shared memory: [digit images][metadata][row headers] (1024-aligned),
+// [weight stages], [barriers], TMEM slot. The weight ring gets as many stages
+// as the budget leaves, at most kI8MaxWStages.
+__host__ __device__ constexpr int i8_wring_offset(int nsb) {
+    return (nsb * (kI8ImageBytes + kI8MetaDoubles * 8) + kI8HSlots * kI8HeaderBytes + 1023) / 1024 * 1024;
+}
+__host__ __device__ constexpr int i8_fit_stages(int nsb) {
+    return (kI8SmemBudget - 1024 - i8_wring_offset(nsb) - kI8Barriers * 8 - 16) / kI8RawBytes;
+}
+// 8, 6 or 4 (the kernel's instantiations), or fewer if even 4 do not fit
+__host__ __device__ constexpr int i8_wstages_nsb(int nsb) {
+    return i8_fit_stages(nsb) >= 8 ? 8 : i8_fit_stages(nsb) >= 6 ? 6 : i8_fit_stages(nsb) >= 4 ? 4 : i8_fit_stages(nsb);
+}
+__host__ __device__ constexpr int i8_smem_bytes_nsb(int nsb) {
+    return 1024 + i8_wring_offset(nsb) + i8_wstages_nsb(nsb) * kI8RawBytes + kI8Barriers * 8 + 16;
+}
+
+// Byte offset of (row n, K position kk) in one block's digit image: two
+// 128-element atoms along K, each N rows x 128 bytes in the 128-byte swizzled
+// K-major layout (8-row groups 1024 bytes apart; 16-byte chunk c of row n
+// stored at chunk c ^ (n % 8)).
+__host__ __device__ constexpr int i8_image_offset(int n, int kk) {
+    return (kk >> 7) * (kI8N * 128) + (n >> 3) * 1024 + (n & 7) * 128 +
+           ((((kk & 127) >> 4) ^ (n & 7)) << 4) + (kk & 15);
+}
+
+__device__ __forceinline__ bool i8_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_bounded(bar, parity, &g_i8_fault_flags);
+}
+
+// Small non-negative integer (< 2^31) to f64 exactly, on the FP64 pipe.
+__device__ __forceinline__ double u32_to_f64(uint32_t v) {
+    return __longlong_as_double(0x4330000000000000LL | v) - 4503599627370496.0;
+}
+
+// Low bytes of four ints packed into one word (byte i from v[i]).
+__device__ __forceinline__ uint32_t pack_bytes(int a, int b, int c, int d) {
+    const uint32_t ab = __byte_perm(static_cast<uint32_t>(a), static_cast<uint32_t>(b), 0x0040u);
+    const uint32_t cd = __byte_perm(static_cast<uint32_t>(c), static_cast<uint32_t>(d), 0x0040u);
+    return __byte_perm(ab, cd, 0x5410u);
+}
+
+// Digit image and metadata of x's 256-element blocks b = first, first +
+// stride, ... (one warp per block; lane holds K positions 8*lane .. + 7).
+__device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, uint8_t* image,
+                                          double* meta, int first, int stride, int lane) {
+    for (int b = first; b < nsb; b += stride) {
+        const float4* src = reinterpret_cast<const float4*>(x + static_cast<size_t>(b) * kQK + 8 * lane);
+        const float4 a = src[0], c = src[1];
+        const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        bool finite = true;
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            finite = finite && isfinite(v[e]);
+            amax = fmaxf(amax, fabsf(v[e]));
+        }
+        finite = __all_sync(0xFFFFFFFFu, finite);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        int ex = 0;
+        if (finite && amax > 0.f) frexpf(amax, &ex);   // amax in [2^(ex-1), 2^ex)
+        const bool scaled = finite && amax > 0.f;
+        // 2^(33 - ex) from its exponent field (ex >= -148)
+        const double up = scaled ? __longlong_as_double(static_cast<long long>(1023 + 33 - ex) << 52) : 0.0;
+        long long sum = 0;
+        int r[8];       // X >> 7 after the first digit (|.| < 2^27)
+        int dig[8];     // current digit
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            // exact scaling, one rounding (a non-finite block has X = 0)
+            const long long X = scaled ? __double2ll_rn(static_cast<double>(v[e]) * up) : 0;
+            sum += X;
+            dig[e] = ((static_cast<int>(X) + 64) & 127) - 64;
+            r[e] = static_cast<int>((X - dig[e]) >> 7);
+        }
+        // S0 of sub-block j = lanes 4j .. 4j+3
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+        double* md = meta + static_cast<size_t>(b) * kI8MetaDoubles;
+        if ((lane & 3) == 0) md[1 + (lane >> 2)] = static_cast<double>(sum);
+        if (lane == 0) {
+            md[0] = finite ? (scaled ? __longlong_as_double(static_cast<long long>(1023 + ex - 33) << 52) : 0.0)
+                           : __longlong_as_double(0x7FF8000000000000LL);
+            md[9] = 0.0;
+        }
+        uint8_t* img = image + static_cast<size_t>(b) * kI8ImageBytes;
+#pragma unroll
+        for (int l = 0; l < kI8Limbs; ++l) {
+            if (l > 0) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    dig[e] = ((r[e] + 64) & 127) - 64;
+                    r[e] = (r[e] - dig[e]) >> 7;
+                }
+            }
+            *reinterpret_cast<uint2*>(img + i8_image_offset(l, 8 * lane)) =
+                make_uint2(pack_bytes(dig[0], dig[1], dig[2], dig[3]),
+                           pack_bytes(dig[4], dig[5], dig[6], dig[7]));
+        }
+    }
+}
+
+struct I8Params {
+    const float* x;      // [k]
+    float* y;            // [n]
+    int n, nsb, tiles;
+};
+
+template <int WS>
+__global__ void __launch_bounds__(kI8Threads, 1)
+q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) {
+    constexpr uint32_t kIdesc = mma_i8_idesc(kI8Rows, kI8N);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned (the swizzled digit images need it), as an offset from
+    // smem_raw so that accesses stay shared-memory accesses
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    const int nsb = p.nsb;
+    uint8_t* image = smem;                                        // [nsb][kI8ImageBytes]
+    double* meta = reinterpret_cast<double*>(smem + nsb * kI8ImageBytes);   // [nsb][10]
+    uint4* hring = reinterpret_cast<uint4*>(meta + nsb * kI8MetaDoubles);    // [kI8HSlots][128]
+    uint8_t* wring = smem + i8_wring_offset(nsb);                 // [WS][128 rows][144]
+    uint64_t* wfull = reinterpret_cast<uint64_t*>(wring + WS * kI8RawBytes);
+    uint64_t* wempty = wfull + kI8MaxWStages;
+    uint64_t* afull = wempty + kI8MaxWStages;  // decoded A in TMEM buffer
+    uint64_t* dfull = afull + kI8ABufs;        // MMAs done: A buffer free, accumulator complete
+    uint64_t* dfree = dfull + kI8DBufs;        // accumulator read
+    uint64_t* hfull = dfree + kI8DBufs;        // row headers of an item written
+    uint64_t* hfree = hfull + kI8HSlots;       // row headers read
+    uint64_t* mma_done = hfree + kI8HSlots;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    __shared__ volatile int abort_flag;
+    __shared__ double xchange[2 * kI8Rows];   // epilogue: half 1's row totals, by tile parity
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // whole tiles [t0, t1) of this CTA, every superblock column of each
+    const int t0 = static_cast<int>(static_cast<long long>(p.tiles) * blockIdx.x / gridDim.x);
+    const int t1 = static_cast<int>(static_cast<long long>(p.tiles) * (blockIdx.x + 1) / gridDim.x);
+    const int count = (t1 - t0) * nsb;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < WS; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], kI8Quarters);
+        }
+        for (int j = 0; j < kI8ABufs; ++j) mbar_init(&afull[j], kI8Quarters);
+        for (int j = 0; j < kI8DBufs; ++j) {
+            mbar_init(&dfull[j], 1);
+            mbar_init(&dfree[j], kI8EpiWarps);
+        }
+        for (int j = 0; j < kI8HSlots; ++j) {
+            mbar_init(&hfull[j], kI8Quarters);
+            mbar_init(&hfree[j], kI8EpiWarps);
+        }
+        mbar_init(mma_done, 1);
+        fence_mbar_init();
+        tma_prefetch_map(&map_w);
+    }
+    if (warp == kI8MmaWarp) tmem_alloc(tmem_slot, kI8TmemCols);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    pdl_launch_dependents();
+
+    // Weight copies, item it = superblock column it % nsb of tile t0 + it / nsb.
+    // The first kI8PreStages are constant data: issued before the preceding
+    // kernels finish; the rest of the ring follows the vector's loads (behind
+    // a full ring of copies those wait microseconds).
+    int p_it = 0, p_tile = t0, p_b = 0;
+    auto produce = [&](int upto) {
+        for (; p_it < upto && !abort_flag; ++p_it) {
+            const int s = p_it % WS;
+            if (p_it >= WS && !i8_wait(&wempty[s], static_cast<uint32_t>(((p_it / WS) - 1) & 1))) {
+                abort_flag = 1;
+                break;
+            }
+            mbar_arrive_expect_tx(&wfull[s], kI8RawBytes);
+            tma_load_2d(wring + s * kI8RawBytes, &map_w, p_b * kBlockBytes, p_tile * kI8Rows, &wfull[s]);
+            if (++p_b == nsb) {
+                p_b = 0;
+                ++p_tile;
+            }
+        }
+    };
+    if (warp == kI8ProducerWarp && lane == 0) produce(count < kI8PreStages ? count : kI8PreStages);
+    __syncwarp();
+
+    pdl_wait();   // x is produced, and y may be read, by the preceding work on the stream
+    i8_digits(p.x, nsb, image, meta, warp, kI8Warps, lane);
+    fence_proxy_async_smem();   // the image is read by the MMAs
+    __syncthreads();
+
+    if (warp == kI8ProducerWarp) {
+        if (lane == 0) {
+            produce(count);
+            if (abort_flag) {
+                // let the copies still in flight land before shared memory goes
+                const int issued = p_it;
+                for (int i = issued > WS ? issued - WS : 0; i < issued; ++i)
+                    i8_wait(&wfull[i % WS], static_cast<uint32_t>((i / WS) & 1));
+            }
+        }
+    } else if (warp == kI8MmaWarp) {
+        // ------------------------------------------------------------ MMA
+        // The warp runs converged and one elected lane issues the MMAs and
+        // commits: sub-block j of the column is MMA j, A from TMEM columns
+        // 8j..8j+7 of the buffer, B = the block's digit rows at K 32j, the
+        // accumulator columns j*N .. j*N + N - 1 (no accumulation across MMAs).
+        int b = 0;
+        for (int it = 0; it < count; ++it, b = (b + 1 == nsb) ? 0 : b + 1) {
+            const int a = it % kI8ABufs, d = it % kI8DBufs;
+            const bool ok = !abort_flag && i8_wait(&afull[a], static_cast<uint32_t>((it / kI8ABufs) & 1)) &&
+                            (it < kI8DBufs ||
+                             i8_wait(&dfree[d], static_cast<uint32_t>(((it / kI8DBufs) - 1) & 1)));
+            if (!__all_sync(0xFFFFFFFFu, ok)) {
+                abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t img = smem_addr(image + static_cast<size_t>(b) * kI8ImageBytes);
+            const uint32_t dcol = tmem + static_cast<uint32_t>(kI8Dcol0 + d * kI8Dcols);
+            const uint32_t acol = tmem + static_cast<uint32_t>(a * kI8Acols);
+            if (elect_one()) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    // K position 32j: atom j / 4 (N * 128 bytes each), 32 bytes per
+                    // MMA inside it
+                    const uint64_t bdesc = sw128_kmajor_desc(img + (j >> 2) * (kI8N * 128) + (j & 3) * 32);
+                    mma_i8_tmem_a(dcol + static_cast<uint32_t>(j * kI8N), acol + static_cast<uint32_t>(8 * j),
+                                  bdesc, kIdesc, 0u);
+                }
+                mma_commit(&dfull[d]);
+            }
+            __syncwarp();
+        }
+        if (elect_one()) {
+            mma_commit(mma_done);   // every MMA issued above has completed
+            i8_wait(mma_done, 0u);
+        }
+        __syncwarp();
+    } else if (warp < kI8DecodeWarps) {
+        // ------------------------------------------------------------ decode
+        // Lane = row of the tile; its quant word u of group g = u / 8 gives
+        // columns 16g + u % 8 (low nibbles: sub-block 2g) and 16g + 8 + u % 8
+        // (high nibbles: sub-block 2g+1) of the buffer. The row's 16-byte
+        // superblock header goes to the header ring for the epilogue.
+        const int quarter = warp % kI8Quarters;
+        const int row = 32 * quarter + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
+        for (int it = warp / kI8Quarters; it < count; it += kI8DecodeSets) {
+            const int s = it % WS, a = it % kI8ABufs, hs = it % kI8HSlots;
+            // The weight stage is read into registers and released before the
+            // waits for the item's A buffer and header slot, so that the copy
+            // ring keeps streaming while the later stages catch up.
+            bool ok = !abort_flag && i8_wait(&wfull[s], static_cast<uint32_t>((it / WS) & 1));
+            if (!__all_sync(0xFFFFFFFFu, ok)) {
+                abort_flag = 1;
+                break;
+            }
+            const uint4* rq = reinterpret_cast<const uint4*>(wring + s * kI8RawBytes + row * kBlockBytes);
+            const uint4 hdr = rq[0];
+            uint4 q[8];   // the row's 128 quant bytes
+#pragma unroll
+            for (int v = 0; v < 8; ++v) q[v] = rq[1 + v];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wempty[s]);   // the stage is free once read
+            ok = (it < kI8ABufs || i8_wait(&dfull[a], static_cast<uint32_t>(((it / kI8ABufs) - 1) & 1))) &&
+                 (it < kI8HSlots || i8_wait(&hfree[hs], static_cast<uint32_t>(((it / kI8HSlots) - 1) & 1)));
+            if (!__all_sync(0xFFFFFFFFu, ok)) {
+                abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            hring[hs * kI8Rows + row] = hdr;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&hfull[hs]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {   // groups 2h, 2h+1: 32 columns
+                uint32_t cols[32];
+#pragma unroll
+                for (int gg = 0; gg < 2; ++gg) {
+                    const uint4 q0 = q[2 * (2 * h + gg)], q1 = q[2 * (2 * h + gg) + 1];
+                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        cols[16 * gg + c] = words[c] & 0x0F0F0F0Fu;
+                        cols[16 * gg + 8 + c] = words[c] & 0xF0F0F0F0u;
+                    }
+                }
+                tmem_store_32cols(lane_base + static_cast<uint32_t>(a * kI8Acols + 32 * h), cols);
+            }
+            tmem_wait_st();
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[a]);
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        // Two warps per lane quarter share each item: half h takes sub-blocks
+        // 4h .. 4h+3 (accumulator columns 32h .. 32h+31). Each keeps its own
+        // f64 row total; at the end of a tile half 1 hands its total to half
+        // 0 (shared memory, a named barrier per quarter), which adds the two
+        // in that order and stores y.
+        const int quarter = warp % kI8Quarters;
+        const int half = (warp - kI8DecodeWarps) / kI8Quarters;
+        const int row = 32 * quarter + lane;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
+        double ytot = 0.0;
+        int tile = t0, b = 0;
+        for (int it = 0; it < count; ++it) {
+            const int grow = tile * kI8Rows + row;
+            const int d = it % kI8DBufs, hs = it % kI8HSlots;
+            const bool ok = !abort_flag && i8_wait(&dfull[d], static_cast<uint32_t>((it / kI8DBufs) & 1)) &&
+                            i8_wait(&hfull[hs], static_cast<uint32_t>((it / kI8HSlots) & 1));
+            if (__all_sync(0xFFFFFFFFu, ok)) {
+                // this row's superblock header (d, dmin, sc_j, m_j)
+                const uint4 hraw = hring[hs * kI8Rows + row];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&hfree[hs]);
+                tc_fence_after_sync();
+                uint32_t r[32];   // D_j[l] at column (j - 4h)*N + l
+                tmem_load_32cols_async(lane_base + static_cast<uint32_t>(kI8Dcol0 + d * kI8Dcols + 32 * half), r);
+                tmem_wait_ld();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dfree[d]);
+                const Header hd = decode_header(hraw);
+                const uint32_t scw = half ? hd.sc_hi : hd.sc_lo, mw = half ? hd.m_hi : hd.m_lo;
+                // S = sum_j sc_j * T_j over the half's sub-blocks, T_j = sum_l
+                // 128^l D_j[l] (D / 16 for odd j) = lo_j + 2^21 hi_j with
+                // lo_j = D0 + 128 D1 + 2^14 D2 (|lo| < 2^29) and hi_j = D3 + 128
+                // D4 (|hi| < 2^22): sum sc*lo in 64 bits, sum sc*hi in 32
+                // (4 * 63 * 3962880 < 2^31).
+                long long s_lo = 0;
+                int s_hi = 0;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t* rj = r + jj * kI8N;
+                    const int D0 = static_cast<int>(rj[0]), D1 = static_cast<int>(rj[1]);
+                    const int D2 = static_cast<int>(rj[2]), D3 = static_cast<int>(rj[3]);
+                    const int D4 = static_cast<int>(rj[4]);
+                    int lo, hi;
+                    if (jj & 1) {   // odd j: A = 16 q, every D is a multiple of 16
+                        lo = (D0 >> 4) + 8 * D1 + 1024 * D2;
+                        hi = (D3 >> 4) + 8 * D4;
+                    } else {
+                        lo = D0 + 128 * D1 + 16384 * D2;
+                        hi = D3 + 128 * D4;
+                    }
+                    const int sc = static_cast<int>(byte_of(scw, jj));
+                    s_lo += static_cast<long long>(sc) * lo;
+                    s_hi += sc * hi;
+                }
+                const long long S = s_lo + (static_cast<long long>(s_hi) << 21);   // |S| < 2^51
+                const double* mb = meta + static_cast<size_t>(b) * kI8MetaDoubles + 1 + 4 * half;
+                // M = sum_j m_j * S0_j over the half's sub-blocks, two chains
+                // (exact: integers below 2^53)
+                double ma = u32_to_f64(byte_of(mw, 0)) * mb[0];
+                double mc = u32_to_f64(byte_of(mw, 1)) * mb[1];
+                ma = fma(u32_to_f64(byte_of(mw, 2)), mb[2], ma);
+                mc = fma(u32_to_f64(byte_of(mw, 3)), mb[3], mc);
+                const double dd = hd.d, dm = hd.dmin;
+                const double scale = meta[static_cast<size_t>(b) * kI8MetaDoubles];
+                ytot = fma(scale, fma(dd, static_cast<double>(S), -(dm * (ma + mc))), ytot);
+            } else {
+                abort_flag = 1;
+            }
+            if (++b == nsb) {
+                double* xc = xchange + (tile & 1) * kI8Rows;   // alternate tiles: one barrier per tile
+                if (half == 1) xc[row] = ytot;
+                named_barrier_sync(1 + quarter, 64);
+                if (half == 0 && !abort_flag && grow < p.n) p.y[grow] = static_cast<float>(ytot + xc[row]);
+                ytot = 0.0;
+                b = 0;
+                ++tile;
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kI8MmaWarp) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kI8TmemCols);
+    }
+}
+
+}  // namespace
+
+int i8_max_nsb(int max_smem) {
+    int nsb = 0;
+    while (i8_wstages_nsb(nsb + 1) >= kI8MinWStages && i8_smem_bytes_nsb(nsb + 1) <= max_smem) ++nsb;
+    return nsb;
+}
+
+int i8_smem_bytes(int nsb) { return i8_smem_bytes_nsb(nsb); }
+int i8_wstages(int nsb) { return i8_wstages_nsb(nsb); }
+int i8_threads() { return kI8Threads; }
+int i8_ctas(int tiles, int num_sms) { return tiles < num_sms ? tiles : num_sms; }
+
+bool i8_applies(int m, int n, int k, int num_sms, int max_smem) {
+    if (m != 1 || n < 1 || k < kQK || k % kQK != 0 || num_sms < 1) return false;
+    const long long tiles = (static_cast<long long>(n) + kI8Rows - 1) / kI8Rows;
+    if (tiles < num_sms) return false;
+    // busiest CTA: ceil(tiles / SMs) tiles; at most 1/kI8MaxImbalance above the mean
+    const long long busiest = (tiles + num_sms - 1) / num_sms;
+    if (busiest * num_sms * kI8MaxImbalance > tiles * (kI8MaxImbalance + 1)) return false;
+    return k / kQK <= i8_max_nsb(max_smem);
+}
+
+int i8_set_attributes() {
+    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kI8SmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
+    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+}
+
+int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int n, int k,
+                   cudaStream_t stream) {
+    const int nsb = k / kQK;
+    const int tiles = (n + kI8Rows - 1) / kI8Rows;
+    CUtensorMap map;
+    if (!make_weight_map(&map, w, n, nsb)) return cuda_failure(cudaErrorInvalidValue);
+    const I8Params ip{x, y, n, nsb, tiles};
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(i8_ctas(tiles, dev.sm_count)));
+    cfg.blockDim = dim3(kI8Threads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(i8_smem_bytes_nsb(nsb));
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int ws = i8_wstages_nsb(nsb);
+    const cudaError_t e = ws >= 8   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8>, map, ip)
+                          : ws >= 6 ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6>, map, ip)
+                                    : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4>, map, ip);
+    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+}
+
+int read_i8_fault_flags(unsigned* flags) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_i8_fault_flags, sizeof(v));
+    if (e != cudaSuccess) return cuda_failure(e);
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_i8_fault_flags, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_failure(e);
+    *flags = v;
+    return Q4K_OK;
+}
+
+}  // namespace q4k

@@ -690,33 +690,6 @@ q4k_gemv_tc_kernel(const __grid_constant__ CUtensorMap map_w, const TcParams p) 
     }
 }
 
-// 2-D map of the Q4_K matrix as bytes: rows of nsb*144 bytes, boxes of one
-// superblock column (144 bytes) by 128 rows; rows past n read as zeros.
-bool make_weight_map(CUtensorMap* map, const void* w, int n, int nsb) {
-    using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                       const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                       const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                       CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-    static EncodeTiledFn fn = [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            ptr = nullptr;
-        return reinterpret_cast<EncodeTiledFn>(ptr);
-    }();
-    if (fn == nullptr) return false;
-    const cuuint64_t row_bytes = static_cast<cuuint64_t>(nsb) * kBlockBytes;
-    const cuuint64_t dims[2] = {row_bytes, static_cast<cuuint64_t>(n)};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(kTcRows)};
-    const cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(w), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MP>
 cudaError_t launch_tc_group(const CUtensorMap& map, const TcParams& tp, int grid, cudaStream_t stream) {
     cudaLaunchConfig_t cfg{};
@@ -778,6 +751,33 @@ TcLayout tc_layout(int m, int n, int k, int num_sms) {
 }
 
 }  // namespace
+
+// 2-D map of the Q4_K matrix as bytes: rows of nsb*144 bytes, boxes of one
+// superblock column (144 bytes) by 128 rows; rows past n read as zeros.
+bool make_weight_map(CUtensorMap* map, const void* w, int n, int nsb) {
+    using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                       const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                       const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                       CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeTiledFn fn = [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            ptr = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    if (fn == nullptr) return false;
+    const cuuint64_t row_bytes = static_cast<cuuint64_t>(nsb) * kBlockBytes;
+    const cuuint64_t dims[2] = {row_bytes, static_cast<cuuint64_t>(n)};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(kTcRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(w), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 int tc_smem_bytes(int mp) { return tc_smem_bytes_mp(mp); }
 int tc_stages(int mp) { return tc_wstages_mp(mp); }

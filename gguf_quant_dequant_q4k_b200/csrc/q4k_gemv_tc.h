@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstddef>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace q4k {
@@ -32,6 +33,11 @@ int tc_ctas(int tiles, int nsb, int num_sms);
 // for the vectors' digit images, block metadata and the partial totals of
 // tiles cut between CTAs.
 size_t tc_workspace_bytes(int m, int n, int k, int num_sms);
+
+// 2-D tensor map of a Q4_K matrix as bytes (rows of nsb*144 bytes, boxes of
+// one superblock column by kTcRows rows, rows past n read as zeros); false if
+// the driver's encoder is unavailable or rejects the map.
+bool make_weight_map(CUtensorMap* map, const void* w, int n, int nsb);
 
 int tc_set_attributes();
 int launch_gemv_tc(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n,

@@ -90,6 +90,23 @@ __device__ __forceinline__ void tmem_store_32cols(uint32_t taddr, const uint32_t
         : "memory");
 }
 
+// As tmem_load_32cols, without the wait: the registers are valid after
+// tmem_wait_ld().
+__device__ __forceinline__ void tmem_load_32cols_async(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -173,6 +190,37 @@ __device__ __forceinline__ void mma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a,
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
         "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Instruction descriptor of tcgen05.mma kind::i8 with unsigned 8-bit A, signed
+// 8-bit B, s32 accumulator, both operands K-major, shape M x N: D format s32
+// (bits 4-5 = 2), A format u8 (bits 7-9 = 0), B format s8 (bits 10-12 = 1), no
+// saturation (bit 3), N >> 3 (bits 17-22), M >> 4 (bits 24-28). For M = 128, N
+// is 8 or a multiple of 16 up to 256.
+__host__ __device__ constexpr uint32_t mma_i8_idesc(int m, int n) {
+    return (2u << 4) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+// D (TMEM, s32) = A * B^T (+ D if accumulate), kind::i8, with A read from
+// tensor memory: A is M x 32 bytes in TMEM lanes 0..M-1 (row i in lane i),
+// four K elements per 32-bit column (element 4c + t in byte t of column c)
+// starting at column address tmem_a (8 columns); B N x 32 bytes, K-major, as
+// for mma_f16 (a K step of 32 elements is 32 bytes, as for fp16's 16).
+__device__ __forceinline__ void mma_i8_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (an MMA operand written with st.shared).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // `bar` receives one arrival once every tcgen05.mma this thread issued before

@@ -270,7 +270,7 @@ enum q4k_kernel {
                                    across the CTAs of a cluster (split-K) and
                                    finishes them through distributed shared
                                    memory                                         */
-    Q4K_KERNEL_TC = 3           /* m >= 3: tcgen05 tensor cores, each superblock
+    Q4K_KERNEL_TC = 3,          /* m >= 3: tcgen05 tensor cores, each superblock
                                    decoded once for up to 16 vectors (groups of
                                    16 beyond), exact integer products of sc*q
                                    and base-128 digits of the scaled x; two
@@ -278,6 +278,14 @@ enum q4k_kernel {
                                    counts (128-row tile, superblock column)
                                    items, shared out in equal contiguous ranges;
                                    `depth` is the weight-ring depth             */
+    Q4K_KERNEL_I8 = 4           /* m = 1 on tall matrices (at least one 128-row
+                                   tile per SM, the busiest SM at most 1/8 above
+                                   the mean, K <= 256 * 62): tcgen05 kind::i8,
+                                   the quant nibbles times base-128 digits of
+                                   the scaled x, exact integer products; one
+                                   launch; `units` counts 128-row tiles, whole
+                                   tiles per CTA; `depth` is the weight-ring
+                                   depth                                        */
 };
 
 Q4K_API int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan *plan);

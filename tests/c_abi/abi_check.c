@@ -34,7 +34,10 @@ int main(void)
     memset(&plan, 0, sizeof(plan));
     CHECK(q4k_gemv_plan_for(1, 4096, 4096, 148, &plan) == Q4K_OK);
     CHECK(plan.kernel == Q4K_KERNEL_STREAM && plan.grid >= 148 && plan.launches == 1);
-    CHECK(q4k_gemv_plan_for(1, 128256, 4096, 148, &plan) == Q4K_OK && plan.slices == 2);
+    CHECK(q4k_gemv_plan_for(1, 128256, 4096, 148, &plan) == Q4K_OK && plan.kernel == Q4K_KERNEL_I8 &&
+          plan.grid == 148 && plan.units == 1002 && plan.units_per_cta_max == 7 && plan.launches == 1);
+    CHECK(q4k_gemv_plan_for(1, 128256, 20480, 148, &plan) == Q4K_OK && plan.kernel == Q4K_KERNEL_STREAM &&
+          plan.slices == 2);
     CHECK(q4k_gemv_plan_for(Q4K_MAX_M + 1, 4096, 4096, 148, &plan) == Q4K_ERR_UNSUPPORTED_M);
     CHECK(q4k_gemv_plan_for(1, 4096, 4000, 148, &plan) == Q4K_ERR_SHAPE);
     CHECK(q4k_gemv_swiglu_plan_for(1, 14336, 4096, 148, &plan) == Q4K_OK && plan.cluster == 1);

@@ -253,15 +253,67 @@ def test_tc_plan(m, n, k):
     check_tc_plan(m, n, k)
 
 
+def i8_expected(m, n, k):
+    """Whether q4k_gemv runs this shape on the integer tensor-core kernel: one
+    vector, at least one 128-row tile per SM, the busiest CTA (whole tiles) at
+    most 1/8 above the mean, and the digit image plus four weight stages in
+    the shared-memory budget (K <= 256 * 62)."""
+    tiles, nsb = -(-n // 128), k // 256
+    if m != 1 or tiles < SM_COUNT:
+        return False
+    busiest = -(-tiles // SM_COUNT)
+    return busiest * SM_COUNT * 8 <= tiles * 9 and nsb <= 62
+
+
+def check_i8_plan(n, k):
+    """One persistent CTA per SM owning whole 128-row tiles (equal contiguous
+    ranges); 18 warps; the vector's digit image (2 KB per superblock column),
+    its block metadata (80 B per column), an 8-slot header ring (2 KB each)
+    and 8, 6 or 4 weight stages of 128 x 144 bytes in 220 KB."""
+    p = q4k.q4k_gemv_plan_for(1, n, k, SM_COUNT)
+    assert p["kernel"] == q4k.Q4K_KERNEL_I8, p
+    tiles, nsb = -(-n // 128), k // 256
+    assert p["grid"] == SM_COUNT and p["block"] == 18 * 32 and p["cluster"] == 1
+    assert p["launches"] == 1 and p["units"] == tiles
+    assert p["units_per_cta_max"] == -(-tiles // SM_COUNT)
+    off = -(-(nsb * (2048 + 80) + 8 * 2048) // 1024) * 1024
+    barriers = 2 * 8 + 4 + 2 * 4 + 2 * 8 + 1
+    fit = (220 * 1024 - 1024 - off - barriers * 8 - 16) // (128 * 144)
+    ws = 8 if fit >= 8 else 6 if fit >= 6 else 4
+    assert fit >= 4 and p["depth"] == ws
+    assert p["smem_bytes"] == 1024 + off + ws * 128 * 144 + barriers * 8 + 16 <= 220 * 1024
+    ranges = [(tiles * c // p["grid"], tiles * (c + 1) // p["grid"]) for c in range(p["grid"])]
+    assert ranges[0][0] == 0 and ranges[-1][1] == tiles
+    assert all(r1 == s2 for (_, r1), (s2, _) in zip(ranges, ranges[1:]))
+    assert max(b - a for a, b in ranges) * SM_COUNT * 8 <= tiles * 9
+    return p
+
+
+@pytest.mark.parametrize("n,k", SHAPES + [(148 * 128, 256), (296 * 128 - 51, 512), (1184 * 128 + 1, 4096),
+                                          (160 * 128, 4096), (128256, 15872), (128256, 16128)])
+@pytest.mark.parametrize("m", [1, 2])
+def test_i8_choice(m, n, k):
+    """One vector on tall matrices runs on the integer tensor-core kernel; any
+    other shape keeps its streaming / batched plan."""
+    p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
+    if i8_expected(m, n, k):
+        check_i8_plan(n, k)
+    else:
+        assert p["kernel"] != q4k.Q4K_KERNEL_I8, (m, n, k, p)
+
+
 def test_lm_head_partition():
-    p = check_plan(1, 128256, 4096)
-    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["grid"] == SM_COUNT
-    assert p["units_per_cta_max"] == -(-128256 // SM_COUNT)
+    """The LM head (1002 tiles): 7 tiles on 114 CTAs, 6 on the other 34."""
+    p = check_i8_plan(128256, 4096)
+    assert p["units_per_cta_max"] == 7 and p["depth"] == 8
+    # beyond the digit image's K the tall matrix streams with two-slice lanes
+    p = check_plan(1, 128256, 20480)
+    assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2
 
 
 @pytest.mark.parametrize("n,k,cluster", [(1, 14336, 2), (7, 8192, 2), (1, 256, 1), (40, 4096, 1),
                                          (16, 8960, 1), (8, 14336, 1), (1, 7936, 1),
-                                         (1536, 8960, 1), (4096, 4096, 1), (128256, 4096, 1)])
+                                         (1536, 8960, 1), (4096, 4096, 1), (128256, 20480, 1)])
 def test_cluster_choice(n, k, cluster):
     """N < 8 with K >= 8192 splits rows across the two CTAs of a cluster (split-K)."""
     p = check_plan(1, n, k)
