@@ -139,8 +139,8 @@ KChunks k_chunks(int mk, int nsb) {
 // launches (digits, GEMV) per group of up to 16 vectors.
 bool use_tc(int m, bool fused) { return !fused && m >= kTcMinM; }
 
-// One vector on a tall matrix (whole 128-row tiles for every SM): the
-// integer tensor-core kernel, one launch.
+// One vector (plain projection, K within the digit image): the integer
+// tensor-core kernel, one launch.
 bool use_i8(int m, int n, int k, int num_sms, int max_smem, bool fused) {
     return !fused && i8_applies(m, n, k, num_sms, max_smem);
 }
@@ -149,7 +149,8 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
                      bool fused, q4k_gemv_plan* plan, StreamParams* sp) {
     if (use_i8(m, n, k, num_sms, max_smem, fused)) {
         const int tiles = (n + kI8Rows - 1) / kI8Rows;
-        const int grid = i8_ctas(tiles, num_sms);
+        const int grid = i8_ctas(tiles, k / kQK, num_sms);
+        const long long items = static_cast<long long>(tiles) * (k / kQK);
         plan->kernel = Q4K_KERNEL_I8;
         plan->grid = grid;
         plan->block = i8_threads();
@@ -158,8 +159,10 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
         plan->teams = 0;
         plan->depth = i8_wstages(k / kQK);
         plan->launches = 1;
-        plan->units = tiles;   // whole 128-row tiles
-        plan->units_per_cta_max = (tiles + grid - 1) / grid;
+        plan->units = items;   // (128-row tile, superblock column) items
+        plan->units_per_cta_max = i8_whole_tiles(tiles, num_sms)
+                                      ? static_cast<long long>((tiles + grid - 1) / grid) * (k / kQK)
+                                      : (items + grid - 1) / grid;
         plan->slices = 0;
         return Q4K_OK;
     }

@@ -42,6 +42,9 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_fp16.h>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "q4k_gemv_i8.h"
 #include "q4k_gemv_tc.h"
@@ -68,6 +71,7 @@ constexpr int kI8EpiWarps = 2 * kI8Quarters;                   // warps 8-15: ep
 constexpr int kI8ProducerWarp = 16;    // weight copies
 constexpr int kI8MmaWarp = 17;
 constexpr int kI8Warps = 18;
+constexpr unsigned kI8PieceBarrier = 5;   // named barrier of the epilogue's first half (1-4: quarter pairs)
 constexpr int kI8Threads = 32 * kI8Warps;
 constexpr int kI8Limbs = 5;
 constexpr int kI8N = 8;                      // MMA N: digit rows 0..4
@@ -131,11 +135,14 @@ __device__ __forceinline__ uint32_t pack_bytes(int a, int b, int c, int d) {
     return __byte_perm(ab, cd, 0x5410u);
 }
 
-// Digit image and metadata of x's 256-element blocks b = first, first +
-// stride, ... (one warp per block; lane holds K positions 8*lane .. + 7).
-__device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, uint8_t* image,
-                                          double* meta, int first, int stride, int lane) {
-    for (int b = first; b < nsb; b += stride) {
+// Digit image and metadata of x's 256-element blocks b0, b0 + 1, ... (ncols
+// of them, modulo nsb): block j of those for j = first, first + stride, ...
+// (one warp per block; lane holds K positions 8*lane .. + 7).
+__device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, int b0, int ncols,
+                                          uint8_t* image, double* meta, int first, int stride,
+                                          int lane) {
+    for (int j = first; j < ncols; j += stride) {
+        const int b = (b0 + j) % nsb;
         const float4* src = reinterpret_cast<const float4*>(x + static_cast<size_t>(b) * kQK + 8 * lane);
         const float4 a = src[0], c = src[1];
         const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
@@ -195,8 +202,76 @@ __device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, 
 struct I8Params {
     const float* x;      // [k]
     float* y;            // [n]
+    double* part;        // tiles cut between CTAs: [CTA][2][128] partial row totals
+    unsigned* done;      // tiles cut between CTAs: [tiles] pieces published (zero between launches)
     int n, nsb, tiles;
+    int whole;           // 1: CTAs own whole tiles (no tile is cut)
 };
+
+// The work is the flat sequence of items f = tile * nsb + b (superblock
+// column b of 128-row tile `tile`), cut into gridDim.x equal contiguous
+// ranges: CTA c owns [i8_item_begin(c), i8_item_begin(c + 1)). A tile cut
+// between CTAs is finished by the last of them to publish its piece.
+__device__ __forceinline__ long long i8_item_begin(long long items, int c, int ctas) {
+    return items * c / ctas;
+}
+
+// The CTA whose range holds item f.
+__device__ __forceinline__ int i8_item_owner(long long items, long long f, int ctas) {
+    return static_cast<int>(((f + 1) * ctas - 1) / items);
+}
+
+// After the CTA's last item, the 128 threads of the epilogue's first half
+// (thread = row) make the CTA's cut pieces (slot 0: the tile its range starts
+// in, slot 1: the tile it ends in) visible, count them in per tile, and
+// finish each tile whose last piece this CTA published: add the pieces of
+// the CTAs holding part of the tile, in CTA order, and store y.
+__device__ __forceinline__ void i8_finish_pieces(const I8Params& p, long long items, bool has0, int t0,
+                                                 bool has1, int t1, int row, int* last_flags,
+                                                 bool aborted) {
+    __threadfence();
+    named_barrier_sync(kI8PieceBarrier, kI8Rows);
+    if (row < 2) {
+        const bool has = row == 0 ? has0 : has1;
+        const int t = row == 0 ? t0 : t1;
+        bool last = false;
+        if (has && !aborted) {
+            const long long tf0 = static_cast<long long>(t) * p.nsb;
+            const int pieces = i8_item_owner(items, tf0 + p.nsb - 1, gridDim.x) - i8_item_owner(items, tf0, gridDim.x);
+            last = atomicAdd(&p.done[t], 1u) == static_cast<unsigned>(pieces);
+            if (last) p.done[t] = 0u;   // every other piece is in: the counter is free for the next launch
+        }
+        last_flags[row] = last ? 1 : 0;
+    }
+    named_barrier_sync(kI8PieceBarrier, kI8Rows);
+#pragma unroll 1
+    for (int q = 0; q < 2; ++q) {
+        if (!last_flags[q]) continue;
+        __threadfence();
+        const int t = q == 0 ? t0 : t1;
+        const long long tf0 = static_cast<long long>(t) * p.nsb;
+        const int c_first = i8_item_owner(items, tf0, gridDim.x);
+        const int c_last = i8_item_owner(items, tf0 + p.nsb - 1, gridDim.x);
+        // Every CTA after c_first starts inside tile t (its piece is slot 0);
+        // c_first's piece is slot 0 only if its range starts at the tile.
+        const int first_slot = i8_item_begin(items, c_first, gridDim.x) < tf0 ? 1 : 0;
+        double tot = 0.0;
+        // four pieces per round: their loads are independent and in flight together
+        for (int c0 = c_first; c0 <= c_last; c0 += 4) {
+            double val[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = c0 + j;
+                const int cs = c == c_first ? first_slot : 0;
+                val[j] = c <= c_last ? __ldcg(p.part + (static_cast<size_t>(c) * 2 + cs) * kI8Rows + row) : 0.0;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tot += val[j];   // pieces added in CTA order
+        }
+        const int grow = t * kI8Rows + row;
+        if (grow < p.n) p.y[grow] = static_cast<float>(tot);
+    }
+}
 
 template <int WS>
 __global__ void __launch_bounds__(kI8Threads, 1)
@@ -221,14 +296,21 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     uint64_t* mma_done = hfree + kI8HSlots;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     __shared__ volatile int abort_flag;
-    __shared__ double xchange[2 * kI8Rows];   // epilogue: half 1's row totals, by tile parity
+    __shared__ double xchange[2 * kI8Rows];   // epilogue: half 1's row totals, by piece parity
+    __shared__ int last_piece[2];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // whole tiles [t0, t1) of this CTA, every superblock column of each
-    const int t0 = static_cast<int>(static_cast<long long>(p.tiles) * blockIdx.x / gridDim.x);
-    const int t1 = static_cast<int>(static_cast<long long>(p.tiles) * (blockIdx.x + 1) / gridDim.x);
-    const int count = (t1 - t0) * nsb;
+    // items [f0, f1) of this CTA, from superblock column b00 of tile tile0:
+    // equal contiguous item ranges, or (whole) equal contiguous tile ranges
+    const long long items = static_cast<long long>(p.tiles) * nsb;
+    const long long f0 = p.whole ? i8_item_begin(p.tiles, blockIdx.x, gridDim.x) * nsb
+                                 : i8_item_begin(items, blockIdx.x, gridDim.x);
+    const long long f1 = p.whole ? i8_item_begin(p.tiles, blockIdx.x + 1, gridDim.x) * nsb
+                                 : i8_item_begin(items, blockIdx.x + 1, gridDim.x);
+    const int count = static_cast<int>(f1 - f0);
+    const int tile0 = static_cast<int>(f0 / nsb);
+    const int b00 = static_cast<int>(f0 % nsb);
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
@@ -256,11 +338,11 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     const uint32_t tmem = *tmem_slot;
     pdl_launch_dependents();
 
-    // Weight copies, item it = superblock column it % nsb of tile t0 + it / nsb.
+    // Weight copies of items f0 + it.
     // The first kI8PreStages are constant data: issued before the preceding
     // kernels finish; the rest of the ring follows the vector's loads (behind
     // a full ring of copies those wait microseconds).
-    int p_it = 0, p_tile = t0, p_b = 0;
+    int p_it = 0, p_tile = tile0, p_b = b00;
     auto produce = [&](int upto) {
         for (; p_it < upto && !abort_flag; ++p_it) {
             const int s = p_it % WS;
@@ -280,7 +362,7 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     __syncwarp();
 
     pdl_wait();   // x is produced, and y may be read, by the preceding work on the stream
-    i8_digits(p.x, nsb, image, meta, warp, kI8Warps, lane);
+    i8_digits(p.x, nsb, b00, count < nsb ? count : nsb, image, meta, warp, kI8Warps, lane);
     fence_proxy_async_smem();   // the image is read by the MMAs
     __syncthreads();
 
@@ -300,7 +382,7 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         // commits: sub-block j of the column is MMA j, A from TMEM columns
         // 8j..8j+7 of the buffer, B = the block's digit rows at K 32j, the
         // accumulator columns j*N .. j*N + N - 1 (no accumulation across MMAs).
-        int b = 0;
+        int b = b00;
         for (int it = 0; it < count; ++it, b = (b + 1 == nsb) ? 0 : b + 1) {
             const int a = it % kI8ABufs, d = it % kI8DBufs;
             const bool ok = !abort_flag && i8_wait(&afull[a], static_cast<uint32_t>((it / kI8ABufs) & 1)) &&
@@ -400,7 +482,11 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
         double ytot = 0.0;
-        int tile = t0, b = 0;
+        int tile = tile0, b = b00;
+        int bstart = b;                    // first superblock column of the current piece
+        bool has0 = false, has1 = false;   // cut pieces written (slot 0 / 1)
+        int tile1 = 0;                     // tile of the slot-1 piece
+        int parity = 0;                    // alternates per piece: one barrier per piece
         for (int it = 0; it < count; ++it) {
             const int grow = tile * kI8Rows + row;
             const int d = it % kI8DBufs, hs = it % kI8HSlots;
@@ -459,16 +545,37 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
             } else {
                 abort_flag = 1;
             }
-            if (++b == nsb) {
-                double* xc = xchange + (tile & 1) * kI8Rows;   // alternate tiles: one barrier per tile
+            if (b == nsb - 1 || it == count - 1) {
+                // end of this CTA's piece of `tile`: the halves' totals, added
+                double* xc = xchange + parity * kI8Rows;
                 if (half == 1) xc[row] = ytot;
                 named_barrier_sync(1 + quarter, 64);
-                if (half == 0 && !abort_flag && grow < p.n) p.y[grow] = static_cast<float>(ytot + xc[row]);
+                if (half == 0) {
+                    const double tot = ytot + xc[row];
+                    if (bstart == 0 && b == nsb - 1) {   // the whole tile
+                        if (!abort_flag && grow < p.n) p.y[grow] = static_cast<float>(tot);
+                    } else if (tile == tile0) {
+                        p.part[(static_cast<size_t>(blockIdx.x) * 2 + 0) * kI8Rows + row] = tot;
+                        has0 = true;
+                    } else {
+                        p.part[(static_cast<size_t>(blockIdx.x) * 2 + 1) * kI8Rows + row] = tot;
+                        has1 = true;
+                        tile1 = tile;
+                    }
+                }
                 ytot = 0.0;
+                bstart = 0;
+                parity ^= 1;
+            }
+            if (++b == nsb) {
                 b = 0;
                 ++tile;
             }
         }
+        // every thread of the first half takes this branch or none (the
+        // pieces depend only on the CTA's range)
+        if (half == 0 && (has0 || has1))
+            i8_finish_pieces(p, items, has0, tile0, has1, tile1, row, last_piece, abort_flag != 0);
     }
 
     tc_fence_before_sync();
@@ -490,17 +597,91 @@ int i8_max_nsb(int max_smem) {
 int i8_smem_bytes(int nsb) { return i8_smem_bytes_nsb(nsb); }
 int i8_wstages(int nsb) { return i8_wstages_nsb(nsb); }
 int i8_threads() { return kI8Threads; }
-int i8_ctas(int tiles, int num_sms) { return tiles < num_sms ? tiles : num_sms; }
+int i8_ctas(int tiles, int nsb, int num_sms) {
+    if (i8_whole_tiles(tiles, num_sms)) return num_sms;
+    const long long items = static_cast<long long>(tiles) * nsb;
+    return items < num_sms ? static_cast<int>(items) : num_sms;
+}
+
+bool i8_whole_tiles(int tiles, int num_sms) {
+    if (tiles < num_sms) return false;
+    const long long busiest = (static_cast<long long>(tiles) + num_sms - 1) / num_sms;
+    return busiest * num_sms * kI8MaxImbalance <= static_cast<long long>(tiles) * (kI8MaxImbalance + 1);
+}
+
+bool i8_cuts_tiles(int tiles, int nsb, int num_sms) {
+    if (i8_whole_tiles(tiles, num_sms)) return false;
+    const long long items = static_cast<long long>(tiles) * nsb;
+    const int ctas = i8_ctas(tiles, nsb, num_sms);
+    for (int c = 1; c < ctas; ++c)
+        if ((items * c / ctas) % nsb != 0) return true;
+    return false;
+}
 
 bool i8_applies(int m, int n, int k, int num_sms, int max_smem) {
     if (m != 1 || n < 1 || k < kQK || k % kQK != 0 || num_sms < 1) return false;
+    const int nsb = k / kQK;
+    if (nsb > i8_max_nsb(max_smem)) return false;
     const long long tiles = (static_cast<long long>(n) + kI8Rows - 1) / kI8Rows;
-    if (tiles < num_sms) return false;
-    // busiest CTA: ceil(tiles / SMs) tiles; at most 1/kI8MaxImbalance above the mean
-    const long long busiest = (tiles + num_sms - 1) / num_sms;
-    if (busiest * num_sms * kI8MaxImbalance > tiles * (kI8MaxImbalance + 1)) return false;
-    return k / kQK <= i8_max_nsb(max_smem);
+    if (tiles * nsb >= (1LL << 31) / num_sms) return false;   // item counts in 32 bits
+    // whole tiles per CTA, or enough (tile, column) items per CTA that the
+    // kernel's fixed cost (digit image, pipeline fill, cut tiles) pays off
+    return i8_whole_tiles(static_cast<int>(tiles), num_sms) ||
+           tiles * nsb >= static_cast<long long>(kI8MinItemsPerCta) * num_sms;
 }
+
+namespace {
+
+// Scratch for tiles cut between CTAs, one per (device, stream): the per-tile
+// counters (zeroed once; every launch leaves them zero, the last publisher of a
+// tile resetting its counter) and the pieces, [SMs][2][128] f64. Calls on one
+// stream run in order, so a stream's calls never share it concurrently.
+struct I8Scratch {
+    void* ptr = nullptr;
+    int tiles_cap = 0;
+    int ctas_cap = 0;
+};
+std::mutex g_i8_mu;
+std::map<std::pair<int, uintptr_t>, I8Scratch> g_i8_scratch;
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// Counters then pieces: the pieces' offset for a region of `tiles` counters.
+size_t scratch_part_offset(int tiles) { return align256(static_cast<size_t>(tiles) * sizeof(unsigned)); }
+
+// The stream's scratch for `tiles` tiles and `ctas` CTAs, (re)allocated in
+// stream order if missing or too small; *done stays null if the stream is
+// capturing a graph and has none large enough yet (the caller then allocates
+// per call).
+cudaError_t stream_scratch(int device, cudaStream_t stream, int tiles, int ctas, unsigned** done,
+                           double** part) {
+    *done = nullptr;
+    *part = nullptr;
+    std::lock_guard<std::mutex> lock(g_i8_mu);
+    I8Scratch& sc = g_i8_scratch[{device, reinterpret_cast<uintptr_t>(stream)}];
+    if (sc.ptr == nullptr || sc.tiles_cap < tiles || sc.ctas_cap < ctas) {
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        cudaError_t e = cudaStreamIsCapturing(stream, &cap);
+        if (e != cudaSuccess || cap != cudaStreamCaptureStatusNone) return e;
+        const int tcap = tiles > 4096 ? tiles : 4096;
+        const int ccap = ctas > 256 ? ctas : 256;
+        void* p = nullptr;
+        e = cudaMallocAsync(&p, scratch_part_offset(tcap) + static_cast<size_t>(ccap) * 2 * kI8Rows * sizeof(double),
+                            stream);
+        if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(p, 0, static_cast<size_t>(tcap) * sizeof(unsigned), stream);
+        if (e != cudaSuccess) return e;
+        if (sc.ptr != nullptr) cudaFreeAsync(sc.ptr, stream);
+        sc.ptr = p;
+        sc.tiles_cap = tcap;
+        sc.ctas_cap = ccap;
+    }
+    *done = static_cast<unsigned*>(sc.ptr);
+    *part = reinterpret_cast<double*>(static_cast<uint8_t*>(sc.ptr) + scratch_part_offset(sc.tiles_cap));
+    return cudaSuccess;
+}
+
+}  // namespace
 
 int i8_set_attributes() {
     cudaError_t e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -516,11 +697,33 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
                    cudaStream_t stream) {
     const int nsb = k / kQK;
     const int tiles = (n + kI8Rows - 1) / kI8Rows;
+    const int ctas = i8_ctas(tiles, nsb, dev.sm_count);
+    const bool whole = i8_whole_tiles(tiles, dev.sm_count);
     CUtensorMap map;
     if (!make_weight_map(&map, w, n, nsb)) return cuda_failure(cudaErrorInvalidValue);
-    const I8Params ip{x, y, n, nsb, tiles};
+    // Tiles cut between CTAs: the stream's scratch, or (a graph being
+    // captured on a stream without one) a stream-ordered allocation of this
+    // call, counters zeroed on the stream.
+    unsigned* done = nullptr;
+    double* part = nullptr;
+    void* own = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (i8_cuts_tiles(tiles, nsb, dev.sm_count)) {
+        int device = 0;
+        e = cudaGetDevice(&device);
+        if (e == cudaSuccess) e = stream_scratch(device, stream, tiles, ctas, &done, &part);
+        if (e == cudaSuccess && done == nullptr) {
+            e = cudaMallocAsync(&own, scratch_part_offset(tiles) + static_cast<size_t>(ctas) * 2 * kI8Rows * sizeof(double),
+                                stream);
+            if (e == cudaSuccess) e = cudaMemsetAsync(own, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream);
+            done = static_cast<unsigned*>(own);
+            part = reinterpret_cast<double*>(static_cast<uint8_t*>(own) + scratch_part_offset(tiles));
+        }
+        if (e != cudaSuccess) return cuda_failure(e);
+    }
+    const I8Params ip{x, y, part, done, n, nsb, tiles, whole ? 1 : 0};
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(i8_ctas(tiles, dev.sm_count)));
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
     cfg.blockDim = dim3(kI8Threads);
     cfg.dynamicSmemBytes = static_cast<size_t>(i8_smem_bytes_nsb(nsb));
     cfg.stream = stream;
@@ -529,10 +732,14 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int ws = i8_wstages_nsb(nsb);
-    const cudaError_t e = ws >= 8   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8>, map, ip)
-                          : ws >= 6 ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6>, map, ip)
-                                    : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4>, map, ip);
+    const int wstages = i8_wstages_nsb(nsb);
+    e = wstages >= 8   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8>, map, ip)
+        : wstages >= 6 ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6>, map, ip)
+                       : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4>, map, ip);
+    if (own != nullptr) {
+        const cudaError_t ef = cudaFreeAsync(own, stream);
+        if (e == cudaSuccess) e = ef;
+    }
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
 
@@ -540,6 +747,19 @@ int read_i8_fault_flags(unsigned* flags) {
     unsigned v = 0;
     cudaError_t e = cudaMemcpyFromSymbol(&v, g_i8_fault_flags, sizeof(v));
     if (e != cudaSuccess) return cuda_failure(e);
+    if (v != 0) {
+        // A launch that gave up may have left cut-tile counters of this
+        // device's stream scratches non-zero: clear them.
+        int device = 0;
+        e = cudaGetDevice(&device);
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        std::lock_guard<std::mutex> lock(g_i8_mu);
+        for (auto& kv : g_i8_scratch)
+            if (e == cudaSuccess && kv.first.first == device && kv.second.ptr != nullptr)
+                e = cudaMemset(kv.second.ptr, 0, static_cast<size_t>(kv.second.tiles_cap) * sizeof(unsigned));
+        if (e == cudaSuccess) e = cudaDeviceSynchronize();
+        if (e != cudaSuccess) return cuda_failure(e);
+    }
     const unsigned zero = 0;
     e = cudaMemcpyToSymbol(g_i8_fault_flags, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_failure(e);

@@ -12,8 +12,9 @@ constexpr int kI8Rows = 128;      // rows per tile: the MMA's M
 constexpr int kI8MaxWStages = 8;  // weight stages (one superblock column of a tile each) ...
 constexpr int kI8MinWStages = 4;  // ... 8, 6 or 4, as many as fit beside the digit image
 constexpr int kI8PreStages = 2;   // weight stages requested before the dependency wait
-constexpr int kI8MaxImbalance = 8;   // whole tiles per CTA: at most 1/8 of the CTAs' time idle
 constexpr int kI8SmemBudget = 220 * 1024;   // dynamic shared memory a CTA may use
+constexpr int kI8MaxImbalance = 8;   // whole tiles per CTA: the busiest CTA at most 1/8 above the mean
+constexpr int kI8MinItemsPerCta = 5; // cut tiles: at least this many items per CTA on average
 
 // Superblocks per row the kernel keeps the vector's digit image for (shared
 // memory): K up to 256 times this.
@@ -21,11 +22,18 @@ int i8_max_nsb(int max_smem);
 int i8_smem_bytes(int nsb);
 int i8_wstages(int nsb);
 int i8_threads();
-// CTAs: one per SM at most, each owning whole 128-row tiles.
-int i8_ctas(int tiles, int num_sms);
-// True if q4k_gemv runs one vector of this shape on the kernel: every SM gets
-// whole tiles with the busiest CTA at most 1/kI8MaxImbalance above the mean,
-// and the digit image fits beside the weight stages.
+// Whole 128-row tiles per CTA: at least one tile per SM and the busiest CTA
+// at most 1/kI8MaxImbalance above the mean.
+bool i8_whole_tiles(int tiles, int num_sms);
+// CTAs: one per SM at most, owning whole tiles (i8_whole_tiles) or equal
+// contiguous ranges of the tiles x nsb (tile, superblock column) items.
+int i8_ctas(int tiles, int nsb, int num_sms);
+// True if some CTA range starts inside a tile (the tile is then finished from
+// pieces in the stream's scratch).
+bool i8_cuts_tiles(int tiles, int nsb, int num_sms);
+// True if q4k_gemv runs one vector of this shape on the kernel: the vector's
+// digit image fits beside four weight stages, and the CTAs own whole tiles or
+// at least kI8MinItemsPerCta items each on average.
 bool i8_applies(int m, int n, int k, int num_sms, int max_smem);
 
 int i8_set_attributes();

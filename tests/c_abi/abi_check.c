@@ -35,7 +35,8 @@ int main(void)
     CHECK(q4k_gemv_plan_for(1, 4096, 4096, 148, &plan) == Q4K_OK);
     CHECK(plan.kernel == Q4K_KERNEL_STREAM && plan.grid >= 148 && plan.launches == 1);
     CHECK(q4k_gemv_plan_for(1, 128256, 4096, 148, &plan) == Q4K_OK && plan.kernel == Q4K_KERNEL_I8 &&
-          plan.grid == 148 && plan.units == 1002 && plan.units_per_cta_max == 7 && plan.launches == 1);
+          plan.grid == 148 && plan.units == 1002 * 16 && plan.units_per_cta_max == 7 * 16 &&
+          plan.launches == 1);
     CHECK(q4k_gemv_plan_for(1, 128256, 20480, 148, &plan) == Q4K_OK && plan.kernel == Q4K_KERNEL_STREAM &&
           plan.slices == 2);
     CHECK(q4k_gemv_plan_for(Q4K_MAX_M + 1, 4096, 4096, 148, &plan) == Q4K_ERR_UNSUPPORTED_M);

@@ -64,6 +64,20 @@ def test_i8_ragged_tiles(q4k, n, k):
     assert_gemv_close(y, yref, a, f"{n}x{k}")
 
 
+@pytest.mark.parametrize("n,k", [(11008, 4096), (4096, 14336), (3000, 15872), (4096 + 77, 8192)])
+def test_i8_cut_tiles(q4k, n, k):
+    """Fewer tiles than a whole-tile split needs: equal item ranges, tiles cut
+    between CTAs and finished from their pieces (in CTA order) by the last CTA
+    to publish one; a ragged last tile; identical bits on a second call (the
+    stream's scratch counters are left zero by each launch)."""
+    w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS.get((n, k), n + k))
+    y = gpu_gemv(q4k, w, x, n, k)
+    y2 = gpu_gemv(q4k, w, x, n, k)
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))
+    yref, a = oracle.gemv(w, x, n, k, nthreads=8)
+    assert_gemv_close(y, yref, a, f"{n}x{k}")
+
+
 def test_i8_one_column_tiles(q4k):
     """K = 256: every item ends a tile (1185 tiles, 8 or 9 per CTA)."""
     n, k = 1184 * 128 + 1, 256

@@ -141,13 +141,13 @@ def test_gemv_multivector_shapes(q4k, n, k, m):
     assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
 
 
-@pytest.mark.parametrize("n,k", [(75904, 4096), (100000, 20480), (75904, 1536), (8192, 28672)])
+@pytest.mark.parametrize("n,k", [(75904, 256), (100000, 20480), (151936, 20480), (8192, 28672)])
 def test_gemv_tall_two_slices_sampled(q4k, n, k):
     """Very tall matrices (512 or more rows per CTA) that the integer
-    tensor-core kernel does not take (593 tiles: whole tiles per CTA would
-    leave the busiest CTA 25 % above the mean; K beyond its digit image) and K
-    beyond 20480 (one vector) run two quant slices per lane on the streaming
-    kernel; the oracle checks sampled rows, including every CTA boundary region."""
+    tensor-core kernel does not take (K beyond its digit image, or too few
+    superblock columns per CTA with whole tiles uneven) and K beyond 20480
+    (one vector) run two quant slices per lane on the streaming kernel; the
+    oracle checks sampled rows, including every CTA boundary region."""
     plan = q4k.q4k_gemv_plan_for(1, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
     assert plan["slices"] == 2
     w, x = q4k_synth.q4k_problem(n, k, 1, 60 + n % 97)

@@ -253,47 +253,66 @@ def test_tc_plan(m, n, k):
     check_tc_plan(m, n, k)
 
 
+def i8_whole(tiles):
+    busiest = -(-tiles // SM_COUNT)
+    return tiles >= SM_COUNT and busiest * SM_COUNT * 8 <= tiles * 9
+
+
 def i8_expected(m, n, k):
     """Whether q4k_gemv runs this shape on the integer tensor-core kernel: one
-    vector, at least one 128-row tile per SM, the busiest CTA (whole tiles) at
-    most 1/8 above the mean, and the digit image plus four weight stages in
-    the shared-memory budget (K <= 256 * 62)."""
+    vector, the digit image plus four weight stages in the shared-memory
+    budget (K <= 256 * 62), and whole tiles per CTA (at least one 128-row tile
+    per SM, the busiest CTA at most 1/8 above the mean) or at least 5 (tile,
+    superblock column) items per CTA on average."""
     tiles, nsb = -(-n // 128), k // 256
-    if m != 1 or tiles < SM_COUNT:
+    if m != 1 or nsb > 62:
         return False
-    busiest = -(-tiles // SM_COUNT)
-    return busiest * SM_COUNT * 8 <= tiles * 9 and nsb <= 62
+    return i8_whole(tiles) or tiles * nsb >= 5 * SM_COUNT
 
 
 def check_i8_plan(n, k):
-    """One persistent CTA per SM owning whole 128-row tiles (equal contiguous
-    ranges); 18 warps; the vector's digit image (2 KB per superblock column),
+    """One persistent CTA per SM at most: whole 128-row tiles in equal
+    contiguous tile ranges, or equal contiguous ranges of the tiles x nsb
+    items; 18 warps; the vector's digit image (2 KB per superblock column),
     its block metadata (80 B per column), an 8-slot header ring (2 KB each)
     and 8, 6 or 4 weight stages of 128 x 144 bytes in 220 KB."""
     p = q4k.q4k_gemv_plan_for(1, n, k, SM_COUNT)
     assert p["kernel"] == q4k.Q4K_KERNEL_I8, p
     tiles, nsb = -(-n // 128), k // 256
-    assert p["grid"] == SM_COUNT and p["block"] == 18 * 32 and p["cluster"] == 1
-    assert p["launches"] == 1 and p["units"] == tiles
-    assert p["units_per_cta_max"] == -(-tiles // SM_COUNT)
+    items = tiles * nsb
+    whole = i8_whole(tiles)
+    assert p["grid"] == (SM_COUNT if whole else min(items, SM_COUNT))
+    assert p["block"] == 18 * 32 and p["cluster"] == 1 and p["launches"] == 1 and p["units"] == items
     off = -(-(nsb * (2048 + 80) + 8 * 2048) // 1024) * 1024
     barriers = 2 * 8 + 4 + 2 * 4 + 2 * 8 + 1
     fit = (220 * 1024 - 1024 - off - barriers * 8 - 16) // (128 * 144)
     ws = 8 if fit >= 8 else 6 if fit >= 6 else 4
     assert fit >= 4 and p["depth"] == ws
     assert p["smem_bytes"] == 1024 + off + ws * 128 * 144 + barriers * 8 + 16 <= 220 * 1024
-    ranges = [(tiles * c // p["grid"], tiles * (c + 1) // p["grid"]) for c in range(p["grid"])]
-    assert ranges[0][0] == 0 and ranges[-1][1] == tiles
+    if whole:
+        ranges = [(tiles * c // p["grid"] * nsb, tiles * (c + 1) // p["grid"] * nsb) for c in range(p["grid"])]
+        assert all(a % nsb == 0 and b % nsb == 0 for a, b in ranges)   # no tile is cut
+        assert p["units_per_cta_max"] == -(-tiles // p["grid"]) * nsb
+    else:
+        ranges = [(items * c // p["grid"], items * (c + 1) // p["grid"]) for c in range(p["grid"])]
+        assert p["units_per_cta_max"] == -(-items // p["grid"])
+        assert max(b - a for a, b in ranges) - min(b - a for a, b in ranges) <= 1
+    assert ranges[0][0] == 0 and ranges[-1][1] == items
     assert all(r1 == s2 for (_, r1), (s2, _) in zip(ranges, ranges[1:]))
-    assert max(b - a for a, b in ranges) * SM_COUNT * 8 <= tiles * 9
+    # a tile cut between CTAs: its pieces come from consecutive CTAs, at most
+    # two per CTA (the tile its range starts in and the one it ends in)
+    for a, b in ranges:
+        if b > a:
+            assert (b - 1) // nsb - a // nsb + 1 >= 1
     return p
 
 
 @pytest.mark.parametrize("n,k", SHAPES + [(148 * 128, 256), (296 * 128 - 51, 512), (1184 * 128 + 1, 4096),
-                                          (160 * 128, 4096), (128256, 15872), (128256, 16128)])
+                                          (160 * 128, 4096), (128256, 15872), (128256, 16128),
+                                          (3000, 15872), (4096 + 77, 8192), (2048, 8192)])
 @pytest.mark.parametrize("m", [1, 2])
 def test_i8_choice(m, n, k):
-    """One vector on tall matrices runs on the integer tensor-core kernel; any
+    """One vector runs on the integer tensor-core kernel where it pays; any
     other shape keeps its streaming / batched plan."""
     p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
     if i8_expected(m, n, k):
@@ -302,10 +321,20 @@ def test_i8_choice(m, n, k):
         assert p["kernel"] != q4k.Q4K_KERNEL_I8, (m, n, k, p)
 
 
+def test_i8_sweep_choice():
+    """The decode sweep: the LM head (whole tiles) and the 7B/8B FFN
+    projections (cut tiles) on the integer kernel, the smaller projections on
+    the streaming kernel."""
+    want = {(8960, 1536): 2, (1536, 8960): 2, (1536, 1536): 2, (11008, 4096): 4, (4096, 11008): 4,
+            (4096, 4096): 2, (4096, 14336): 4, (128256, 4096): 4}
+    for (n, k), kern in want.items():
+        assert q4k.q4k_gemv_plan_for(1, n, k, SM_COUNT)["kernel"] == kern, (n, k)
+
+
 def test_lm_head_partition():
     """The LM head (1002 tiles): 7 tiles on 114 CTAs, 6 on the other 34."""
     p = check_i8_plan(128256, 4096)
-    assert p["units_per_cta_max"] == 7 and p["depth"] == 8
+    assert p["units_per_cta_max"] == 7 * 16 and p["depth"] == 8
     # beyond the digit image's K the tall matrix streams with two-slice lanes
     p = check_plan(1, 128256, 20480)
     assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2
