@@ -149,8 +149,9 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
                      bool fused, q4k_gemv_plan* plan, StreamParams* sp) {
     if (use_i8(m, n, k, num_sms, max_smem, fused)) {
         const int tiles = (n + kI8Rows - 1) / kI8Rows;
-        const int grid = i8_ctas(tiles, k / kQK, num_sms);
-        const long long items = static_cast<long long>(tiles) * (k / kQK);
+        const int nsb = k / kQK, cpi = i8_cpi(nsb);
+        const int grid = i8_ctas(tiles, nsb, num_sms);
+        const long long items = static_cast<long long>(tiles) * nsb;   // superblock columns of tiles
         plan->kernel = Q4K_KERNEL_I8;
         plan->grid = grid;
         plan->block = i8_threads();
@@ -159,10 +160,11 @@ int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* 
         plan->teams = 0;
         plan->depth = i8_wstages(k / kQK);
         plan->launches = 1;
-        plan->units = items;   // (128-row tile, superblock column) items
-        plan->units_per_cta_max = i8_whole_tiles(tiles, num_sms)
-                                      ? static_cast<long long>((tiles + grid - 1) / grid) * (k / kQK)
-                                      : (items + grid - 1) / grid;
+        plan->units = items;   // (128-row tile, superblock column) units, cpi per item
+        plan->units_per_cta_max =
+            i8_whole_tiles(tiles, num_sms)
+                ? static_cast<long long>((tiles + grid - 1) / grid) * nsb
+                : (static_cast<long long>(tiles) * (nsb / cpi) + grid - 1) / grid * cpi;
         plan->slices = 0;
         return Q4K_OK;
     }

@@ -1,6 +1,6 @@
-// q4k_gemv_i8.cu -- y = W x for Q4_K W and one f32 vector on tall matrices
-// (the LM head of a decode step: the pages' `Q4KGemv` over a vocabulary-sized
-// W, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs"), on the tcgen05
+// q4k_gemv_i8.cu -- y = W x for Q4_K W and one f32 vector (the pages'
+// `Q4KGemv`, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs": the LM
+// head and the larger projections of a decode step), on the tcgen05
 // tensor cores with 8-bit integer operands. Every product is formed exactly
 // in integers; only the final combination and the output rounding are inexact.
 //
@@ -26,15 +26,20 @@
 //   row's f64 total; y is that total rounded to f32 once. So
 //   |y - sum w x| <= 2^-24 (|y| + sum |w x|) + sum_t |w_t| 2^(E_t - 34), the
 //   bound of the batched tensor-core path; non-finite x makes y NaN.
-// * Pipeline. A persistent CTA owns whole 128-row tiles and walks their
-//   superblock columns in order. A producer thread streams each column of a
-//   tile (128 rows x 144 bytes, one 2-D TMA box) through up to eight stages;
-//   two sets of four decode warps (one per TMEM lane quarter), alternate
-//   items each, write A into one of four TMEM buffers and hand each row's
-//   superblock header on through a shared-memory ring; one elected lane of the MMA warp issues the column's 8 MMAs into
-//   one of four accumulators; eight epilogue warps (two per lane quarter,
-//   four sub-blocks each) read the accumulator (tcgen05.ld) and combine it. The digit image of the whole vector stays in
-//   shared memory for the kernel.
+// * Pipeline. A persistent CTA owns whole 128-row tiles, or an equal range of
+//   (tile, superblock column) items with tiles cut between CTAs finished from
+//   pieces, and walks its items in order; an item is one superblock column, or
+//   two where K/256 is even and four two-column stages fit (the per-item
+//   waits, polls and hand-offs then cost half as much per column). A producer
+//   thread streams each item (128 rows x 144 bytes per column, one 3-D TMA
+//   box) through the weight stages; two sets of four decode warps (one per
+//   TMEM lane quarter), alternate items each, write A into one of the TMEM
+//   buffers and hand each row's superblock headers on through a shared-memory
+//   ring; one elected lane of the MMA warp issues the item's 8 MMAs per column
+//   into one of the accumulators; eight epilogue warps (two per lane quarter:
+//   a column each, or four sub-blocks each with one column per item) read the
+//   accumulator (tcgen05.ld) and combine it. The digit image of the vector's
+//   blocks the CTA needs stays in shared memory for the kernel.
 //
 // All waits are bounded: one that gives up raises Q4K_FAULT_COPY_TIMEOUT and
 // the CTA lets its copies and MMAs complete (bounded) before it releases shared
@@ -77,37 +82,45 @@ constexpr int kI8Limbs = 5;
 constexpr int kI8N = 8;                      // MMA N: digit rows 0..4
 constexpr int kI8ImageBytes = kI8N * kQK;    // one block's digit image (K-major, swizzled)
 constexpr int kI8MetaDoubles = 10;           // 2^(E-33), S0_0..7, pad
-constexpr int kI8RawBytes = kI8Rows * kBlockBytes;
-constexpr int kI8Acols = 64;                 // TMEM columns of one decoded superblock (256 bytes)
-constexpr int kI8ABufs = 4;
-constexpr int kI8Dcols = 8 * kI8N;           // one accumulator: 8 sub-blocks x N columns
-constexpr int kI8DBufs = 4;
-constexpr int kI8Dcol0 = kI8ABufs * kI8Acols;
+constexpr int kI8RawBytes = kI8Rows * kBlockBytes;   // one superblock column of a tile
+constexpr int kI8ColTmem = 64;               // TMEM columns of one decoded superblock column (256 bytes)
+constexpr int kI8ColAcc = 8 * kI8N;          // accumulator columns of one superblock column
 constexpr int kI8TmemCols = 512;
-constexpr int kI8HSlots = kI8ABufs + kI8DBufs;   // header ring (see the decode)
+constexpr int kI8Dcol0 = 256;                // A buffers in TMEM columns 0..255, accumulators after them
+// An item is CPI (1 or 2) superblock columns of a tile: A buffers and
+// accumulators of CPI * 64 columns, 4 / CPI of each.
+__host__ __device__ constexpr int i8_bufs(int cpi) { return 4 / cpi; }
+constexpr int kI8HSlotCols = 8;              // header ring: 8 superblock columns' row headers
 constexpr int kI8HeaderBytes = kI8Rows * 16;      // one column's row headers
-constexpr int kI8Barriers = 2 * kI8MaxWStages + kI8ABufs + 2 * kI8DBufs + 2 * kI8HSlots + 1;
-static_assert(kI8Dcol0 + kI8DBufs * kI8Dcols <= kI8TmemCols, "TMEM buffers");
-// Item it uses A buffer and accumulator it % 4: one commit per item tells the
-// decode that the A buffer is free and the epilogue that the accumulator is
-// complete.
-static_assert(kI8ABufs == kI8DBufs, "A buffers and accumulators share the MMA-done barriers");
+// barriers sized for one column per item (the most buffers)
+constexpr int kI8Barriers = 2 * kI8MaxWStages + 4 + 2 * 4 + 2 * kI8HSlotCols + 1;
+static_assert(kI8Dcol0 + 4 * kI8ColAcc <= kI8TmemCols && 4 * kI8ColTmem <= kI8Dcol0, "TMEM buffers");
 
 // Shared memory: [digit images][metadata][row headers] (1024-aligned),
-// [weight stages], [barriers], TMEM slot. The weight ring gets as many stages
-// as the budget leaves, at most kI8MaxWStages.
+// [weight stages of CPI columns], [barriers], TMEM slot. The weight ring gets
+// as many stages as the budget leaves, at most kI8MaxWStages (one column per
+// item) or 4 (two).
 __host__ __device__ constexpr int i8_wring_offset(int nsb) {
-    return (nsb * (kI8ImageBytes + kI8MetaDoubles * 8) + kI8HSlots * kI8HeaderBytes + 1023) / 1024 * 1024;
+    return (nsb * (kI8ImageBytes + kI8MetaDoubles * 8) + kI8HSlotCols * kI8HeaderBytes + 1023) / 1024 * 1024;
 }
-__host__ __device__ constexpr int i8_fit_stages(int nsb) {
-    return (kI8SmemBudget - 1024 - i8_wring_offset(nsb) - kI8Barriers * 8 - 16) / kI8RawBytes;
+__host__ __device__ constexpr int i8_fit_stages(int nsb, int cpi) {
+    return (kI8SmemBudget - 1024 - i8_wring_offset(nsb) - kI8Barriers * 8 - 16) / (cpi * kI8RawBytes);
 }
-// 8, 6 or 4 (the kernel's instantiations), or fewer if even 4 do not fit
+// Two columns per item where K/256 is even and four two-column stages fit.
+__host__ __device__ constexpr int i8_cpi_nsb(int nsb) {
+    return (nsb % 2 == 0 && i8_fit_stages(nsb, 2) >= 4) ? 2 : 1;
+}
+// the kernel's instantiations: 8, 6 or 4 one-column stages, 4 two-column
+// stages (fewer if even those do not fit)
 __host__ __device__ constexpr int i8_wstages_nsb(int nsb) {
-    return i8_fit_stages(nsb) >= 8 ? 8 : i8_fit_stages(nsb) >= 6 ? 6 : i8_fit_stages(nsb) >= 4 ? 4 : i8_fit_stages(nsb);
+    return i8_cpi_nsb(nsb) == 2 ? 4
+           : i8_fit_stages(nsb, 1) >= 8 ? 8
+           : i8_fit_stages(nsb, 1) >= 6 ? 6
+           : i8_fit_stages(nsb, 1) >= 4 ? 4
+                                        : i8_fit_stages(nsb, 1);
 }
 __host__ __device__ constexpr int i8_smem_bytes_nsb(int nsb) {
-    return 1024 + i8_wring_offset(nsb) + i8_wstages_nsb(nsb) * kI8RawBytes + kI8Barriers * 8 + 16;
+    return 1024 + i8_wring_offset(nsb) + i8_wstages_nsb(nsb) * i8_cpi_nsb(nsb) * kI8RawBytes + kI8Barriers * 8 + 16;
 }
 
 // Byte offset of (row n, K position kk) in one block's digit image: two
@@ -205,11 +218,13 @@ struct I8Params {
     double* part;        // tiles cut between CTAs: [CTA][2][128] partial row totals
     unsigned* done;      // tiles cut between CTAs: [tiles] pieces published (zero between launches)
     int n, nsb, tiles;
+    int npi;             // items per tile: nsb / CPI
     int whole;           // 1: CTAs own whole tiles (no tile is cut)
 };
 
-// The work is the flat sequence of items f = tile * nsb + b (superblock
-// column b of 128-row tile `tile`), cut into gridDim.x equal contiguous
+// The work is the flat sequence of items f = tile * npi + i (superblock
+// columns CPI*i .. CPI*i + CPI - 1 of 128-row tile `tile`), cut into gridDim.x
+// equal contiguous
 // ranges: CTA c owns [i8_item_begin(c), i8_item_begin(c + 1)). A tile cut
 // between CTAs is finished by the last of them to publish its piece.
 __device__ __forceinline__ long long i8_item_begin(long long items, int c, int ctas) {
@@ -236,8 +251,8 @@ __device__ __forceinline__ void i8_finish_pieces(const I8Params& p, long long it
         const int t = row == 0 ? t0 : t1;
         bool last = false;
         if (has && !aborted) {
-            const long long tf0 = static_cast<long long>(t) * p.nsb;
-            const int pieces = i8_item_owner(items, tf0 + p.nsb - 1, gridDim.x) - i8_item_owner(items, tf0, gridDim.x);
+            const long long tf0 = static_cast<long long>(t) * p.npi;
+            const int pieces = i8_item_owner(items, tf0 + p.npi - 1, gridDim.x) - i8_item_owner(items, tf0, gridDim.x);
             last = atomicAdd(&p.done[t], 1u) == static_cast<unsigned>(pieces);
             if (last) p.done[t] = 0u;   // every other piece is in: the counter is free for the next launch
         }
@@ -249,9 +264,9 @@ __device__ __forceinline__ void i8_finish_pieces(const I8Params& p, long long it
         if (!last_flags[q]) continue;
         __threadfence();
         const int t = q == 0 ? t0 : t1;
-        const long long tf0 = static_cast<long long>(t) * p.nsb;
+        const long long tf0 = static_cast<long long>(t) * p.npi;
         const int c_first = i8_item_owner(items, tf0, gridDim.x);
-        const int c_last = i8_item_owner(items, tf0 + p.nsb - 1, gridDim.x);
+        const int c_last = i8_item_owner(items, tf0 + p.npi - 1, gridDim.x);
         // Every CTA after c_first starts inside tile t (its piece is slot 0);
         // c_first's piece is slot 0 only if its range starts at the tile.
         const int first_slot = i8_item_begin(items, c_first, gridDim.x) < tf0 ? 1 : 0;
@@ -273,27 +288,72 @@ __device__ __forceinline__ void i8_finish_pieces(const I8Params& p, long long it
     }
 }
 
-template <int WS>
+// The epilogue's sum for one row and one superblock column over sub-blocks
+// j0 .. j0 + NJ - 1: r holds D_j[l] at r[(j - j0) * N + l]. Returns
+// d * S - dmin * M with S = sum_j sc_j * T_j, T_j = sum_l 128^l D_j[l] (D / 16
+// for odd j) = lo_j + 2^21 hi_j, lo_j = D0 + 128 D1 + 2^14 D2 (|lo| < 2^29),
+// hi_j = D3 + 128 D4 (|hi| < 2^22): sum sc*lo in 64 bits, sum sc*hi in 32
+// (8 * 63 * 3962880 < 2^31); M = sum_j m_j * S0_j (mb[1 + j] = S0_j, exact in
+// f64, two chains).
+template <int NJ>
+__device__ __forceinline__ double i8_column_sum(const uint32_t* r, const Header& hd, const double* mb, int j0) {
+    long long s_lo = 0;
+    int s_hi = 0;
+    double ma = 0.0, mc = 0.0;
+#pragma unroll
+    for (int jj = 0; jj < NJ; ++jj) {
+        const int j = j0 + jj;
+        const uint32_t* rj = r + jj * kI8N;
+        const int D0 = static_cast<int>(rj[0]), D1 = static_cast<int>(rj[1]);
+        const int D2 = static_cast<int>(rj[2]), D3 = static_cast<int>(rj[3]);
+        const int D4 = static_cast<int>(rj[4]);
+        int lo, hi;
+        if (jj & 1) {   // odd j (j0 is even): A = 16 q, every D is a multiple of 16
+            lo = (D0 >> 4) + 8 * D1 + 1024 * D2;
+            hi = (D3 >> 4) + 8 * D4;
+        } else {
+            lo = D0 + 128 * D1 + 16384 * D2;
+            hi = D3 + 128 * D4;
+        }
+        const uint32_t scw = j < 4 ? hd.sc_lo : hd.sc_hi, mw = j < 4 ? hd.m_lo : hd.m_hi;
+        const int sc = static_cast<int>(byte_of(scw, j & 3));
+        s_lo += static_cast<long long>(sc) * lo;
+        s_hi += sc * hi;
+        const double mj = u32_to_f64(byte_of(mw, j & 3)) * mb[1 + j];
+        if (jj & 1) mc += mj; else ma += mj;
+    }
+    const long long S = s_lo + (static_cast<long long>(s_hi) << 21);   // |S| < 2^52
+    const double dd = hd.d, dm = hd.dmin;
+    return fma(dd, static_cast<double>(S), -(dm * (ma + mc)));
+}
+
+template <int WS, int CPI>
 __global__ void __launch_bounds__(kI8Threads, 1)
 q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) {
     constexpr uint32_t kIdesc = mma_i8_idesc(kI8Rows, kI8N);
+    constexpr int kBufs = i8_bufs(CPI);               // A buffers = accumulators
+    constexpr int kHSlots = kI8HSlotCols / CPI;       // header ring slots (items)
+    constexpr int kStage = CPI * kI8RawBytes;         // one weight stage
+    // Item it uses A buffer and accumulator it % kBufs: one commit per item
+    // tells the decode that the A buffer is free and the epilogue that the
+    // accumulator is complete.
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned (the swizzled digit images need it), as an offset from
     // smem_raw so that accesses stay shared-memory accesses
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-    const int nsb = p.nsb;
+    const int nsb = p.nsb, npi = p.npi;
     uint8_t* image = smem;                                        // [nsb][kI8ImageBytes]
     double* meta = reinterpret_cast<double*>(smem + nsb * kI8ImageBytes);   // [nsb][10]
-    uint4* hring = reinterpret_cast<uint4*>(meta + nsb * kI8MetaDoubles);    // [kI8HSlots][128]
-    uint8_t* wring = smem + i8_wring_offset(nsb);                 // [WS][128 rows][144]
-    uint64_t* wfull = reinterpret_cast<uint64_t*>(wring + WS * kI8RawBytes);
+    uint4* hring = reinterpret_cast<uint4*>(meta + nsb * kI8MetaDoubles);    // [slot][CPI][128]
+    uint8_t* wring = smem + i8_wring_offset(nsb);                 // [WS][128 rows][CPI][144]
+    uint64_t* wfull = reinterpret_cast<uint64_t*>(wring + WS * kStage);
     uint64_t* wempty = wfull + kI8MaxWStages;
     uint64_t* afull = wempty + kI8MaxWStages;  // decoded A in TMEM buffer
-    uint64_t* dfull = afull + kI8ABufs;        // MMAs done: A buffer free, accumulator complete
-    uint64_t* dfree = dfull + kI8DBufs;        // accumulator read
-    uint64_t* hfull = dfree + kI8DBufs;        // row headers of an item written
-    uint64_t* hfree = hfull + kI8HSlots;       // row headers read
-    uint64_t* mma_done = hfree + kI8HSlots;
+    uint64_t* dfull = afull + 4;               // MMAs done: A buffer free, accumulator complete
+    uint64_t* dfree = dfull + 4;               // accumulator read
+    uint64_t* hfull = dfree + 4;               // row headers of an item written
+    uint64_t* hfree = hfull + kI8HSlotCols;    // row headers read
+    uint64_t* mma_done = hfree + kI8HSlotCols;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     __shared__ volatile int abort_flag;
     __shared__ double xchange[2 * kI8Rows];   // epilogue: half 1's row totals, by piece parity
@@ -301,16 +361,16 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // items [f0, f1) of this CTA, from superblock column b00 of tile tile0:
-    // equal contiguous item ranges, or (whole) equal contiguous tile ranges
-    const long long items = static_cast<long long>(p.tiles) * nsb;
-    const long long f0 = p.whole ? i8_item_begin(p.tiles, blockIdx.x, gridDim.x) * nsb
+    // items [f0, f1) of this CTA, from item i00 of tile tile0: equal
+    // contiguous item ranges, or (whole) equal contiguous tile ranges
+    const long long items = static_cast<long long>(p.tiles) * npi;
+    const long long f0 = p.whole ? i8_item_begin(p.tiles, blockIdx.x, gridDim.x) * npi
                                  : i8_item_begin(items, blockIdx.x, gridDim.x);
-    const long long f1 = p.whole ? i8_item_begin(p.tiles, blockIdx.x + 1, gridDim.x) * nsb
+    const long long f1 = p.whole ? i8_item_begin(p.tiles, blockIdx.x + 1, gridDim.x) * npi
                                  : i8_item_begin(items, blockIdx.x + 1, gridDim.x);
     const int count = static_cast<int>(f1 - f0);
-    const int tile0 = static_cast<int>(f0 / nsb);
-    const int b00 = static_cast<int>(f0 % nsb);
+    const int tile0 = static_cast<int>(f0 / npi);
+    const int i00 = static_cast<int>(f0 % npi);
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
@@ -318,12 +378,12 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
             mbar_init(&wfull[s], 1);
             mbar_init(&wempty[s], kI8Quarters);
         }
-        for (int j = 0; j < kI8ABufs; ++j) mbar_init(&afull[j], kI8Quarters);
-        for (int j = 0; j < kI8DBufs; ++j) {
+        for (int j = 0; j < kBufs; ++j) {
+            mbar_init(&afull[j], kI8Quarters);
             mbar_init(&dfull[j], 1);
             mbar_init(&dfree[j], kI8EpiWarps);
         }
-        for (int j = 0; j < kI8HSlots; ++j) {
+        for (int j = 0; j < kHSlots; ++j) {
             mbar_init(&hfull[j], kI8Quarters);
             mbar_init(&hfree[j], kI8EpiWarps);
         }
@@ -338,11 +398,11 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     const uint32_t tmem = *tmem_slot;
     pdl_launch_dependents();
 
-    // Weight copies of items f0 + it.
+    // Weight copies of items f0 + it: one 3-D box of CPI columns x 128 rows.
     // The first kI8PreStages are constant data: issued before the preceding
     // kernels finish; the rest of the ring follows the vector's loads (behind
     // a full ring of copies those wait microseconds).
-    int p_it = 0, p_tile = tile0, p_b = b00;
+    int p_it = 0, p_tile = tile0, p_i = i00;
     auto produce = [&](int upto) {
         for (; p_it < upto && !abort_flag; ++p_it) {
             const int s = p_it % WS;
@@ -350,10 +410,10 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                 abort_flag = 1;
                 break;
             }
-            mbar_arrive_expect_tx(&wfull[s], kI8RawBytes);
-            tma_load_2d(wring + s * kI8RawBytes, &map_w, p_b * kBlockBytes, p_tile * kI8Rows, &wfull[s]);
-            if (++p_b == nsb) {
-                p_b = 0;
+            mbar_arrive_expect_tx(&wfull[s], kStage);
+            tma_load_3d(wring + s * kStage, &map_w, 0, p_i * CPI, p_tile * kI8Rows, &wfull[s]);
+            if (++p_i == npi) {
+                p_i = 0;
                 ++p_tile;
             }
         }
@@ -362,7 +422,7 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     __syncwarp();
 
     pdl_wait();   // x is produced, and y may be read, by the preceding work on the stream
-    i8_digits(p.x, nsb, b00, count < nsb ? count : nsb, image, meta, warp, kI8Warps, lane);
+    i8_digits(p.x, nsb, i00 * CPI, count * CPI < nsb ? count * CPI : nsb, image, meta, warp, kI8Warps, lane);
     fence_proxy_async_smem();   // the image is read by the MMAs
     __syncthreads();
 
@@ -379,33 +439,36 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     } else if (warp == kI8MmaWarp) {
         // ------------------------------------------------------------ MMA
         // The warp runs converged and one elected lane issues the MMAs and
-        // commits: sub-block j of the column is MMA j, A from TMEM columns
-        // 8j..8j+7 of the buffer, B = the block's digit rows at K 32j, the
-        // accumulator columns j*N .. j*N + N - 1 (no accumulation across MMAs).
-        int b = b00;
-        for (int it = 0; it < count; ++it, b = (b + 1 == nsb) ? 0 : b + 1) {
-            const int a = it % kI8ABufs, d = it % kI8DBufs;
-            const bool ok = !abort_flag && i8_wait(&afull[a], static_cast<uint32_t>((it / kI8ABufs) & 1)) &&
-                            (it < kI8DBufs ||
-                             i8_wait(&dfree[d], static_cast<uint32_t>(((it / kI8DBufs) - 1) & 1)));
+        // commits: sub-block j of column c of the item is one MMA, A from TMEM
+        // columns 64c + 8j .. +7 of the buffer, B = the column's digit rows at
+        // K 32j, the accumulator columns 64c + 8j .. +7 (no accumulation
+        // across MMAs).
+        int i = i00;
+        for (int it = 0; it < count; ++it, i = (i + 1 == npi) ? 0 : i + 1) {
+            const int a = it % kBufs;
+            const bool ok = !abort_flag && i8_wait(&afull[a], static_cast<uint32_t>((it / kBufs) & 1)) &&
+                            (it < kBufs || i8_wait(&dfree[a], static_cast<uint32_t>(((it / kBufs) - 1) & 1)));
             if (!__all_sync(0xFFFFFFFFu, ok)) {
                 abort_flag = 1;
                 break;
             }
             tc_fence_after_sync();
-            const uint32_t img = smem_addr(image + static_cast<size_t>(b) * kI8ImageBytes);
-            const uint32_t dcol = tmem + static_cast<uint32_t>(kI8Dcol0 + d * kI8Dcols);
-            const uint32_t acol = tmem + static_cast<uint32_t>(a * kI8Acols);
+            const uint32_t dcol = tmem + static_cast<uint32_t>(kI8Dcol0 + a * CPI * kI8ColAcc);
+            const uint32_t acol = tmem + static_cast<uint32_t>(a * CPI * kI8ColTmem);
             if (elect_one()) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    // K position 32j: atom j / 4 (N * 128 bytes each), 32 bytes per
-                    // MMA inside it
-                    const uint64_t bdesc = sw128_kmajor_desc(img + (j >> 2) * (kI8N * 128) + (j & 3) * 32);
-                    mma_i8_tmem_a(dcol + static_cast<uint32_t>(j * kI8N), acol + static_cast<uint32_t>(8 * j),
-                                  bdesc, kIdesc, 0u);
+                for (int c = 0; c < CPI; ++c) {
+                    const uint32_t img = smem_addr(image + static_cast<size_t>(i * CPI + c) * kI8ImageBytes);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        // K position 32j: atom j / 4 (N * 128 bytes each), 32 bytes
+                        // per MMA inside it
+                        const uint64_t bdesc = sw128_kmajor_desc(img + (j >> 2) * (kI8N * 128) + (j & 3) * 32);
+                        mma_i8_tmem_a(dcol + static_cast<uint32_t>(c * kI8ColAcc + j * kI8N),
+                                      acol + static_cast<uint32_t>(c * kI8ColTmem + 8 * j), bdesc, kIdesc, 0u);
+                    }
                 }
-                mma_commit(&dfull[d]);
+                mma_commit(&dfull[a]);
             }
             __syncwarp();
         }
@@ -416,55 +479,55 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         __syncwarp();
     } else if (warp < kI8DecodeWarps) {
         // ------------------------------------------------------------ decode
-        // Lane = row of the tile; its quant word u of group g = u / 8 gives
-        // columns 16g + u % 8 (low nibbles: sub-block 2g) and 16g + 8 + u % 8
-        // (high nibbles: sub-block 2g+1) of the buffer. The row's 16-byte
-        // superblock header goes to the header ring for the epilogue.
+        // Lane = row of the tile; for column c of the item its quant word u of
+        // group g = u / 8 gives buffer columns 64c + 16g + u % 8 (low nibbles:
+        // sub-block 2g) and 64c + 16g + 8 + u % 8 (high nibbles: sub-block
+        // 2g+1). The row's 16-byte superblock headers go to the header ring for
+        // the epilogue.
         const int quarter = warp % kI8Quarters;
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
         for (int it = warp / kI8Quarters; it < count; it += kI8DecodeSets) {
-            const int s = it % WS, a = it % kI8ABufs, hs = it % kI8HSlots;
-            // The weight stage is read into registers and released before the
-            // waits for the item's A buffer and header slot, so that the copy
-            // ring keeps streaming while the later stages catch up.
-            bool ok = !abort_flag && i8_wait(&wfull[s], static_cast<uint32_t>((it / WS) & 1));
-            if (!__all_sync(0xFFFFFFFFu, ok)) {
-                abort_flag = 1;
-                break;
-            }
-            const uint4* rq = reinterpret_cast<const uint4*>(wring + s * kI8RawBytes + row * kBlockBytes);
-            const uint4 hdr = rq[0];
-            uint4 q[8];   // the row's 128 quant bytes
-#pragma unroll
-            for (int v = 0; v < 8; ++v) q[v] = rq[1 + v];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&wempty[s]);   // the stage is free once read
-            ok = (it < kI8ABufs || i8_wait(&dfull[a], static_cast<uint32_t>(((it / kI8ABufs) - 1) & 1))) &&
-                 (it < kI8HSlots || i8_wait(&hfree[hs], static_cast<uint32_t>(((it / kI8HSlots) - 1) & 1)));
+            const int s = it % WS, a = it % kBufs, hs = it % kHSlots;
+            const bool ok = !abort_flag && i8_wait(&wfull[s], static_cast<uint32_t>((it / WS) & 1)) &&
+                            (it < kBufs || i8_wait(&dfull[a], static_cast<uint32_t>(((it / kBufs) - 1) & 1))) &&
+                            (it < kHSlots || i8_wait(&hfree[hs], static_cast<uint32_t>(((it / kHSlots) - 1) & 1)));
             if (!__all_sync(0xFFFFFFFFu, ok)) {
                 abort_flag = 1;
                 break;
             }
             tc_fence_after_sync();
-            hring[hs * kI8Rows + row] = hdr;
+#pragma unroll
+            for (int c = 0; c < CPI; ++c) {
+                const uint4* rq = reinterpret_cast<const uint4*>(wring + s * kStage + (row * CPI + c) * kBlockBytes);
+                const uint4 hdr = rq[0];
+                uint4 q[8];   // the row's 128 quant bytes of column c
+#pragma unroll
+                for (int v = 0; v < 8; ++v) q[v] = rq[1 + v];
+                if (c == CPI - 1) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&wempty[s]);   // the stage is read
+                }
+                hring[(hs * CPI + c) * kI8Rows + row] = hdr;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {   // groups 2h, 2h+1: 32 columns
+                    uint32_t cols[32];
+#pragma unroll
+                    for (int gg = 0; gg < 2; ++gg) {
+                        const uint4 q0 = q[2 * (2 * h + gg)], q1 = q[2 * (2 * h + gg) + 1];
+                        const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            cols[16 * gg + k] = words[k] & 0x0F0F0F0Fu;
+                            cols[16 * gg + 8 + k] = words[k] & 0xF0F0F0F0u;
+                        }
+                    }
+                    tmem_store_32cols(lane_base + static_cast<uint32_t>(a * CPI * kI8ColTmem + c * kI8ColTmem + 32 * h),
+                                      cols);
+                }
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&hfull[hs]);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {   // groups 2h, 2h+1: 32 columns
-                uint32_t cols[32];
-#pragma unroll
-                for (int gg = 0; gg < 2; ++gg) {
-                    const uint4 q0 = q[2 * (2 * h + gg)], q1 = q[2 * (2 * h + gg) + 1];
-                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        cols[16 * gg + c] = words[c] & 0x0F0F0F0Fu;
-                        cols[16 * gg + 8 + c] = words[c] & 0xF0F0F0F0u;
-                    }
-                }
-                tmem_store_32cols(lane_base + static_cast<uint32_t>(a * kI8Acols + 32 * h), cols);
-            }
             tmem_wait_st();
             tc_fence_before_sync();
             __syncwarp();
@@ -472,87 +535,62 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        // Two warps per lane quarter share each item: half h takes sub-blocks
-        // 4h .. 4h+3 (accumulator columns 32h .. 32h+31). Each keeps its own
-        // f64 row total; at the end of a tile half 1 hands its total to half
-        // 0 (shared memory, a named barrier per quarter), which adds the two
-        // in that order and stores y.
+        // Two warps per lane quarter share each item: with two columns per
+        // item half h takes column h, with one half h takes sub-blocks 4h ..
+        // 4h+3. Each keeps its own f64 row total; at the end of a piece (the
+        // CTA's part of a tile) half 1 hands its total to half 0 (shared
+        // memory, a named barrier per quarter), which adds the two in that
+        // order and stores y or the piece.
         const int quarter = warp % kI8Quarters;
         const int half = (warp - kI8DecodeWarps) / kI8Quarters;
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
+        constexpr int kCols = CPI == 2 ? 64 : 32;   // accumulator columns a half reads
         double ytot = 0.0;
-        int tile = tile0, b = b00;
-        int bstart = b;                    // first superblock column of the current piece
+        int tile = tile0, i = i00;
+        int istart = i;                    // first item of the current piece
         bool has0 = false, has1 = false;   // cut pieces written (slot 0 / 1)
         int tile1 = 0;                     // tile of the slot-1 piece
         int parity = 0;                    // alternates per piece: one barrier per piece
         for (int it = 0; it < count; ++it) {
             const int grow = tile * kI8Rows + row;
-            const int d = it % kI8DBufs, hs = it % kI8HSlots;
-            const bool ok = !abort_flag && i8_wait(&dfull[d], static_cast<uint32_t>((it / kI8DBufs) & 1)) &&
-                            i8_wait(&hfull[hs], static_cast<uint32_t>((it / kI8HSlots) & 1));
+            const int a = it % kBufs, hs = it % kHSlots;
+            const bool ok = !abort_flag && i8_wait(&dfull[a], static_cast<uint32_t>((it / kBufs) & 1)) &&
+                            i8_wait(&hfull[hs], static_cast<uint32_t>((it / kHSlots) & 1));
             if (__all_sync(0xFFFFFFFFu, ok)) {
+                const int c = CPI == 2 ? half : 0;   // the item's column this half reads
                 // this row's superblock header (d, dmin, sc_j, m_j)
-                const uint4 hraw = hring[hs * kI8Rows + row];
+                const uint4 hraw = hring[(hs * CPI + c) * kI8Rows + row];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&hfree[hs]);
                 tc_fence_after_sync();
-                uint32_t r[32];   // D_j[l] at column (j - 4h)*N + l
-                tmem_load_32cols_async(lane_base + static_cast<uint32_t>(kI8Dcol0 + d * kI8Dcols + 32 * half), r);
+                uint32_t r[kCols];   // D_j[l] of the half's sub-blocks at (j - j0) * N + l
+                const uint32_t dcol = lane_base + static_cast<uint32_t>(kI8Dcol0 + a * CPI * kI8ColAcc +
+                                                                        (CPI == 2 ? c * kI8ColAcc : 32 * half));
+                tmem_load_32cols_async(dcol, *reinterpret_cast<uint32_t(*)[32]>(r));
+                if constexpr (CPI == 2) tmem_load_32cols_async(dcol + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
                 tmem_wait_ld();
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&dfree[d]);
+                if (lane == 0) mbar_arrive(&dfree[a]);
                 const Header hd = decode_header(hraw);
-                const uint32_t scw = half ? hd.sc_hi : hd.sc_lo, mw = half ? hd.m_hi : hd.m_lo;
-                // S = sum_j sc_j * T_j over the half's sub-blocks, T_j = sum_l
-                // 128^l D_j[l] (D / 16 for odd j) = lo_j + 2^21 hi_j with
-                // lo_j = D0 + 128 D1 + 2^14 D2 (|lo| < 2^29) and hi_j = D3 + 128
-                // D4 (|hi| < 2^22): sum sc*lo in 64 bits, sum sc*hi in 32
-                // (4 * 63 * 3962880 < 2^31).
-                long long s_lo = 0;
-                int s_hi = 0;
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t* rj = r + jj * kI8N;
-                    const int D0 = static_cast<int>(rj[0]), D1 = static_cast<int>(rj[1]);
-                    const int D2 = static_cast<int>(rj[2]), D3 = static_cast<int>(rj[3]);
-                    const int D4 = static_cast<int>(rj[4]);
-                    int lo, hi;
-                    if (jj & 1) {   // odd j: A = 16 q, every D is a multiple of 16
-                        lo = (D0 >> 4) + 8 * D1 + 1024 * D2;
-                        hi = (D3 >> 4) + 8 * D4;
-                    } else {
-                        lo = D0 + 128 * D1 + 16384 * D2;
-                        hi = D3 + 128 * D4;
-                    }
-                    const int sc = static_cast<int>(byte_of(scw, jj));
-                    s_lo += static_cast<long long>(sc) * lo;
-                    s_hi += sc * hi;
-                }
-                const long long S = s_lo + (static_cast<long long>(s_hi) << 21);   // |S| < 2^51
-                const double* mb = meta + static_cast<size_t>(b) * kI8MetaDoubles + 1 + 4 * half;
-                // M = sum_j m_j * S0_j over the half's sub-blocks, two chains
-                // (exact: integers below 2^53)
-                double ma = u32_to_f64(byte_of(mw, 0)) * mb[0];
-                double mc = u32_to_f64(byte_of(mw, 1)) * mb[1];
-                ma = fma(u32_to_f64(byte_of(mw, 2)), mb[2], ma);
-                mc = fma(u32_to_f64(byte_of(mw, 3)), mb[3], mc);
-                const double dd = hd.d, dm = hd.dmin;
-                const double scale = meta[static_cast<size_t>(b) * kI8MetaDoubles];
-                ytot = fma(scale, fma(dd, static_cast<double>(S), -(dm * (ma + mc))), ytot);
+                const int b = i * CPI + c;
+                const double* mb = meta + static_cast<size_t>(b) * kI8MetaDoubles;
+                double part;
+                if constexpr (CPI == 2) part = i8_column_sum<8>(r, hd, mb, 0);
+                else part = i8_column_sum<4>(r, hd, mb, 4 * half);
+                ytot = fma(mb[0], part, ytot);
             } else {
                 abort_flag = 1;
             }
-            if (b == nsb - 1 || it == count - 1) {
+            if (i == npi - 1 || it == count - 1) {
                 // end of this CTA's piece of `tile`: the halves' totals, added
                 double* xc = xchange + parity * kI8Rows;
                 if (half == 1) xc[row] = ytot;
                 named_barrier_sync(1 + quarter, 64);
                 if (half == 0) {
                     const double tot = ytot + xc[row];
-                    if (bstart == 0 && b == nsb - 1) {   // the whole tile
+                    if (istart == 0 && i == npi - 1) {   // the whole tile
                         if (!abort_flag && grow < p.n) p.y[grow] = static_cast<float>(tot);
                     } else if (tile == tile0) {
                         p.part[(static_cast<size_t>(blockIdx.x) * 2 + 0) * kI8Rows + row] = tot;
@@ -564,11 +602,11 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                     }
                 }
                 ytot = 0.0;
-                bstart = 0;
+                istart = 0;
                 parity ^= 1;
             }
-            if (++b == nsb) {
-                b = 0;
+            if (++i == npi) {
+                i = 0;
                 ++tile;
             }
         }
@@ -597,9 +635,11 @@ int i8_max_nsb(int max_smem) {
 int i8_smem_bytes(int nsb) { return i8_smem_bytes_nsb(nsb); }
 int i8_wstages(int nsb) { return i8_wstages_nsb(nsb); }
 int i8_threads() { return kI8Threads; }
+int i8_cpi(int nsb) { return i8_cpi_nsb(nsb); }
+
 int i8_ctas(int tiles, int nsb, int num_sms) {
     if (i8_whole_tiles(tiles, num_sms)) return num_sms;
-    const long long items = static_cast<long long>(tiles) * nsb;
+    const long long items = static_cast<long long>(tiles) * (nsb / i8_cpi_nsb(nsb));
     return items < num_sms ? static_cast<int>(items) : num_sms;
 }
 
@@ -611,10 +651,11 @@ bool i8_whole_tiles(int tiles, int num_sms) {
 
 bool i8_cuts_tiles(int tiles, int nsb, int num_sms) {
     if (i8_whole_tiles(tiles, num_sms)) return false;
-    const long long items = static_cast<long long>(tiles) * nsb;
+    const int npi = nsb / i8_cpi_nsb(nsb);
+    const long long items = static_cast<long long>(tiles) * npi;
     const int ctas = i8_ctas(tiles, nsb, num_sms);
     for (int c = 1; c < ctas; ++c)
-        if ((items * c / ctas) % nsb != 0) return true;
+        if ((items * c / ctas) % npi != 0) return true;
     return false;
 }
 
@@ -684,23 +725,59 @@ cudaError_t stream_scratch(int device, cudaStream_t stream, int tiles, int ctas,
 }  // namespace
 
 int i8_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<8, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kI8SmemBudget);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<6>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
+        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<6, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
+        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
     return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
 }
+
+namespace {
+
+// 3-D map of the Q4_K matrix as bytes: (byte of a superblock, superblock
+// column, row) with strides 144 and nsb*144; boxes of cpi superblock columns
+// by 128 rows (one item); rows past n read as zeros.
+bool make_weight_map3(CUtensorMap* map, const void* w, int n, int nsb, int cpi) {
+    using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                       const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                       const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                       CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeTiledFn fn = [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            ptr = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBlockBytes), static_cast<cuuint64_t>(nsb),
+                                static_cast<cuuint64_t>(n)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(kBlockBytes),
+                                   static_cast<cuuint64_t>(nsb) * kBlockBytes};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBlockBytes), static_cast<cuuint32_t>(cpi),
+                               static_cast<cuuint32_t>(kI8Rows)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(w), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int n, int k,
                    cudaStream_t stream) {
     const int nsb = k / kQK;
+    const int cpi = i8_cpi_nsb(nsb);
     const int tiles = (n + kI8Rows - 1) / kI8Rows;
     const int ctas = i8_ctas(tiles, nsb, dev.sm_count);
     const bool whole = i8_whole_tiles(tiles, dev.sm_count);
     CUtensorMap map;
-    if (!make_weight_map(&map, w, n, nsb)) return cuda_failure(cudaErrorInvalidValue);
+    if (!make_weight_map3(&map, w, n, nsb, cpi)) return cuda_failure(cudaErrorInvalidValue);
     // Tiles cut between CTAs: the stream's scratch, or (a graph being
     // captured on a stream without one) a stream-ordered allocation of this
     // call, counters zeroed on the stream.
@@ -721,7 +798,7 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
         }
         if (e != cudaSuccess) return cuda_failure(e);
     }
-    const I8Params ip{x, y, part, done, n, nsb, tiles, whole ? 1 : 0};
+    const I8Params ip{x, y, part, done, n, nsb, tiles, nsb / cpi, whole ? 1 : 0};
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(ctas));
     cfg.blockDim = dim3(kI8Threads);
@@ -733,9 +810,10 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const int wstages = i8_wstages_nsb(nsb);
-    e = wstages >= 8   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8>, map, ip)
-        : wstages >= 6 ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6>, map, ip)
-                       : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4>, map, ip);
+    e = cpi == 2         ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 2>, map, ip)
+        : wstages >= 8   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8, 1>, map, ip)
+        : wstages >= 6   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6, 1>, map, ip)
+                         : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 1>, map, ip);
     if (own != nullptr) {
         const cudaError_t ef = cudaFreeAsync(own, stream);
         if (e == cudaSuccess) e = ef;

@@ -9,8 +9,8 @@ namespace q4k {
 struct DeviceInfo;
 
 constexpr int kI8Rows = 128;      // rows per tile: the MMA's M
-constexpr int kI8MaxWStages = 8;  // weight stages (one superblock column of a tile each) ...
-constexpr int kI8MinWStages = 4;  // ... 8, 6 or 4, as many as fit beside the digit image
+constexpr int kI8MaxWStages = 8;  // weight stages: 8, 6 or 4 of one superblock column of a tile,
+constexpr int kI8MinWStages = 4;  // or 4 of two, as many as fit beside the digit image
 constexpr int kI8PreStages = 2;   // weight stages requested before the dependency wait
 constexpr int kI8SmemBudget = 220 * 1024;   // dynamic shared memory a CTA may use
 constexpr int kI8MaxImbalance = 8;   // whole tiles per CTA: the busiest CTA at most 1/8 above the mean
@@ -20,6 +20,8 @@ constexpr int kI8MinItemsPerCta = 5; // cut tiles: at least this many items per 
 // memory): K up to 256 times this.
 int i8_max_nsb(int max_smem);
 int i8_smem_bytes(int nsb);
+// superblock columns per item (1 or 2) and weight stages (of that many columns)
+int i8_cpi(int nsb);
 int i8_wstages(int nsb);
 int i8_threads();
 // Whole 128-row tiles per CTA: at least one tile per SM and the busiest CTA

@@ -279,23 +279,25 @@ def check_i8_plan(n, k):
     p = q4k.q4k_gemv_plan_for(1, n, k, SM_COUNT)
     assert p["kernel"] == q4k.Q4K_KERNEL_I8, p
     tiles, nsb = -(-n // 128), k // 256
-    items = tiles * nsb
     whole = i8_whole(tiles)
-    assert p["grid"] == (SM_COUNT if whole else min(items, SM_COUNT))
-    assert p["block"] == 18 * 32 and p["cluster"] == 1 and p["launches"] == 1 and p["units"] == items
     off = -(-(nsb * (2048 + 80) + 8 * 2048) // 1024) * 1024
     barriers = 2 * 8 + 4 + 2 * 4 + 2 * 8 + 1
-    fit = (220 * 1024 - 1024 - off - barriers * 8 - 16) // (128 * 144)
-    ws = 8 if fit >= 8 else 6 if fit >= 6 else 4
-    assert fit >= 4 and p["depth"] == ws
-    assert p["smem_bytes"] == 1024 + off + ws * 128 * 144 + barriers * 8 + 16 <= 220 * 1024
+    fit = lambda cpi: (220 * 1024 - 1024 - off - barriers * 8 - 16) // (cpi * 128 * 144)
+    cpi = 2 if nsb % 2 == 0 and fit(2) >= 4 else 1     # superblock columns per item
+    ws = 4 if cpi == 2 else 8 if fit(1) >= 8 else 6 if fit(1) >= 6 else 4
+    assert fit(cpi) >= 4 and p["depth"] == ws
+    assert p["smem_bytes"] == 1024 + off + ws * cpi * 128 * 144 + barriers * 8 + 16 <= 220 * 1024
+    npi = nsb // cpi
+    items = tiles * npi
+    assert p["grid"] == (SM_COUNT if whole else min(items, SM_COUNT))
+    assert p["block"] == 18 * 32 and p["cluster"] == 1 and p["launches"] == 1 and p["units"] == tiles * nsb
     if whole:
-        ranges = [(tiles * c // p["grid"] * nsb, tiles * (c + 1) // p["grid"] * nsb) for c in range(p["grid"])]
-        assert all(a % nsb == 0 and b % nsb == 0 for a, b in ranges)   # no tile is cut
+        ranges = [(tiles * c // p["grid"] * npi, tiles * (c + 1) // p["grid"] * npi) for c in range(p["grid"])]
+        assert all(a % npi == 0 and b % npi == 0 for a, b in ranges)   # no tile is cut
         assert p["units_per_cta_max"] == -(-tiles // p["grid"]) * nsb
     else:
         ranges = [(items * c // p["grid"], items * (c + 1) // p["grid"]) for c in range(p["grid"])]
-        assert p["units_per_cta_max"] == -(-items // p["grid"])
+        assert p["units_per_cta_max"] == -(-items // p["grid"]) * cpi
         assert max(b - a for a, b in ranges) - min(b - a for a, b in ranges) <= 1
     assert ranges[0][0] == 0 and ranges[-1][1] == items
     assert all(r1 == s2 for (_, r1), (s2, _) in zip(ranges, ranges[1:]))
@@ -334,7 +336,7 @@ def test_i8_sweep_choice():
 def test_lm_head_partition():
     """The LM head (1002 tiles): 7 tiles on 114 CTAs, 6 on the other 34."""
     p = check_i8_plan(128256, 4096)
-    assert p["units_per_cta_max"] == 7 * 16 and p["depth"] == 8
+    assert p["units_per_cta_max"] == 7 * 16 and p["depth"] == 4   # four stages of two columns
     # beyond the digit image's K the tall matrix streams with two-slice lanes
     p = check_plan(1, 128256, 20480)
     assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2
