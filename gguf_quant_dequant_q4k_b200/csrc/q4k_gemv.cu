@@ -142,30 +142,26 @@ bool use_tc(int m, bool fused) { return !fused && m >= kTcMinM; }
 // One vector (plain projection, K within the digit image): the integer
 // tensor-core kernel, one launch.
 bool use_i8(int m, int n, int k, int num_sms, int max_smem, bool fused) {
-    return !fused && i8_applies(m, n, k, num_sms, max_smem);
+    I8Config c;
+    return !fused && i8_config(m, n, k, num_sms, max_smem, &c);
 }
 
 int plan_gemv_device(int m, int n, int k, int num_sms, int max_smem, const int* max_clusters,
                      bool fused, q4k_gemv_plan* plan, StreamParams* sp) {
-    if (use_i8(m, n, k, num_sms, max_smem, fused)) {
-        const int tiles = (n + kI8Rows - 1) / kI8Rows;
-        const int nsb = k / kQK, cpi = i8_cpi(nsb);
-        const int grid = i8_ctas(tiles, nsb, num_sms);
-        const long long items = static_cast<long long>(tiles) * nsb;   // superblock columns of tiles
+    I8Config ic;
+    if (!fused && i8_config(m, n, k, num_sms, max_smem, &ic)) {
+        const long long tiles = (static_cast<long long>(n) + kI8Rows - 1) / kI8Rows;
         plan->kernel = Q4K_KERNEL_I8;
-        plan->grid = grid;
+        plan->grid = ic.ctas;
         plan->block = i8_threads();
-        plan->smem_bytes = i8_smem_bytes(k / kQK);
+        plan->smem_bytes = ic.smem;
         plan->cluster = 1;
         plan->teams = 0;
-        plan->depth = i8_wstages(k / kQK);
+        plan->depth = ic.wstages;
         plan->launches = 1;
-        plan->units = items;   // (128-row tile, superblock column) units, cpi per item
-        plan->units_per_cta_max =
-            i8_whole_tiles(tiles, num_sms)
-                ? static_cast<long long>((tiles + grid - 1) / grid) * nsb
-                : (static_cast<long long>(tiles) * (nsb / cpi) + grid - 1) / grid * cpi;
-        plan->slices = 0;
+        plan->units = tiles * (k / kQK);   // (128-row tile, superblock column) units, cpi per item
+        plan->units_per_cta_max = ic.items_per_cta_max * ic.cpi;
+        plan->slices = ic.cpi;             // superblock columns per item
         return Q4K_OK;
     }
     if (use_tc(m, fused)) {

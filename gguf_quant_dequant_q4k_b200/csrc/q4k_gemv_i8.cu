@@ -96,31 +96,17 @@ constexpr int kI8HeaderBytes = kI8Rows * 16;      // one column's row headers
 constexpr int kI8Barriers = 2 * kI8MaxWStages + 4 + 2 * 4 + 2 * kI8HSlotCols + 1;
 static_assert(kI8Dcol0 + 4 * kI8ColAcc <= kI8TmemCols && 4 * kI8ColTmem <= kI8Dcol0, "TMEM buffers");
 
-// Shared memory: [digit images][metadata][row headers] (1024-aligned),
-// [weight stages of CPI columns], [barriers], TMEM slot. The weight ring gets
-// as many stages as the budget leaves, at most kI8MaxWStages (one column per
-// item) or 4 (two).
-__host__ __device__ constexpr int i8_wring_offset(int nsb) {
-    return (nsb * (kI8ImageBytes + kI8MetaDoubles * 8) + kI8HSlotCols * kI8HeaderBytes + 1023) / 1024 * 1024;
+// Shared memory: [digit images][metadata] of the CTA's `ncols` superblock
+// columns, [row headers] (1024-aligned), [weight stages of CPI columns],
+// [barriers], TMEM slot.
+__host__ __device__ constexpr int i8_wring_offset(int ncols) {
+    return (ncols * (kI8ImageBytes + kI8MetaDoubles * 8) + kI8HSlotCols * kI8HeaderBytes + 1023) / 1024 * 1024;
 }
-__host__ __device__ constexpr int i8_fit_stages(int nsb, int cpi) {
-    return (kI8SmemBudget - 1024 - i8_wring_offset(nsb) - kI8Barriers * 8 - 16) / (cpi * kI8RawBytes);
+__host__ __device__ constexpr int i8_fit_stages(int ncols, int cpi) {
+    return (kI8SmemBudget - 1024 - i8_wring_offset(ncols) - kI8Barriers * 8 - 16) / (cpi * kI8RawBytes);
 }
-// Two columns per item where K/256 is even and four two-column stages fit.
-__host__ __device__ constexpr int i8_cpi_nsb(int nsb) {
-    return (nsb % 2 == 0 && i8_fit_stages(nsb, 2) >= 4) ? 2 : 1;
-}
-// the kernel's instantiations: 8, 6 or 4 one-column stages, 4 two-column
-// stages (fewer if even those do not fit)
-__host__ __device__ constexpr int i8_wstages_nsb(int nsb) {
-    return i8_cpi_nsb(nsb) == 2 ? 4
-           : i8_fit_stages(nsb, 1) >= 8 ? 8
-           : i8_fit_stages(nsb, 1) >= 6 ? 6
-           : i8_fit_stages(nsb, 1) >= 4 ? 4
-                                        : i8_fit_stages(nsb, 1);
-}
-__host__ __device__ constexpr int i8_smem_bytes_nsb(int nsb) {
-    return 1024 + i8_wring_offset(nsb) + i8_wstages_nsb(nsb) * i8_cpi_nsb(nsb) * kI8RawBytes + kI8Barriers * 8 + 16;
+__host__ __device__ constexpr int i8_smem_bytes_cfg(int ncols, int cpi, int wstages) {
+    return 1024 + i8_wring_offset(ncols) + wstages * cpi * kI8RawBytes + kI8Barriers * 8 + 16;
 }
 
 // Byte offset of (row n, K position kk) in one block's digit image: two
@@ -148,14 +134,16 @@ __device__ __forceinline__ uint32_t pack_bytes(int a, int b, int c, int d) {
     return __byte_perm(ab, cd, 0x5410u);
 }
 
-// Digit image and metadata of x's 256-element blocks b0, b0 + 1, ... (ncols
-// of them, modulo nsb): block j of those for j = first, first + stride, ...
-// (one warp per block; lane holds K positions 8*lane .. + 7).
-__device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, int b0, int ncols,
+// Digit image and metadata of x's 256-element blocks: slot j (j = first,
+// first + stride, ... < ncols) holds padded column (b0 + j) mod pnsb, which is
+// block b of x if b < nsb (a padded column past the row gets nothing). One
+// warp per block; lane holds K positions 8*lane .. + 7.
+__device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, int pnsb, int b0, int ncols,
                                           uint8_t* image, double* meta, int first, int stride,
                                           int lane) {
     for (int j = first; j < ncols; j += stride) {
-        const int b = (b0 + j) % nsb;
+        const int b = (b0 + j) % pnsb;
+        if (b >= nsb) continue;
         const float4* src = reinterpret_cast<const float4*>(x + static_cast<size_t>(b) * kQK + 8 * lane);
         const float4 a = src[0], c = src[1];
         const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
@@ -188,14 +176,14 @@ __device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, 
         // S0 of sub-block j = lanes 4j .. 4j+3
         sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
         sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-        double* md = meta + static_cast<size_t>(b) * kI8MetaDoubles;
+        double* md = meta + static_cast<size_t>(j) * kI8MetaDoubles;
         if ((lane & 3) == 0) md[1 + (lane >> 2)] = static_cast<double>(sum);
         if (lane == 0) {
             md[0] = finite ? (scaled ? __longlong_as_double(static_cast<long long>(1023 + ex - 33) << 52) : 0.0)
                            : __longlong_as_double(0x7FF8000000000000LL);
             md[9] = 0.0;
         }
-        uint8_t* img = image + static_cast<size_t>(b) * kI8ImageBytes;
+        uint8_t* img = image + static_cast<size_t>(j) * kI8ImageBytes;
 #pragma unroll
         for (int l = 0; l < kI8Limbs; ++l) {
             if (l > 0) {
@@ -218,7 +206,9 @@ struct I8Params {
     double* part;        // tiles cut between CTAs: [CTA][2][128] partial row totals
     unsigned* done;      // tiles cut between CTAs: [tiles] pieces published (zero between launches)
     int n, nsb, tiles;
-    int npi;             // items per tile: nsb / CPI
+    int npi;             // items per tile: ceil(nsb / CPI); the last one of a tile may
+                         // hold a column past the row (zero-filled, skipped)
+    int ncols;           // digit-image slots: the CTA's columns, from its first one
     int whole;           // 1: CTAs own whole tiles (no tile is cut)
 };
 
@@ -342,10 +332,11 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     // smem_raw so that accesses stay shared-memory accesses
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int nsb = p.nsb, npi = p.npi;
-    uint8_t* image = smem;                                        // [nsb][kI8ImageBytes]
-    double* meta = reinterpret_cast<double*>(smem + nsb * kI8ImageBytes);   // [nsb][10]
-    uint4* hring = reinterpret_cast<uint4*>(meta + nsb * kI8MetaDoubles);    // [slot][CPI][128]
-    uint8_t* wring = smem + i8_wring_offset(nsb);                 // [WS][128 rows][CPI][144]
+    const int pnsb = npi * CPI;                                   // columns per tile, padded
+    uint8_t* image = smem;                                        // [ncols][kI8ImageBytes]
+    double* meta = reinterpret_cast<double*>(smem + p.ncols * kI8ImageBytes);   // [ncols][10]
+    uint4* hring = reinterpret_cast<uint4*>(meta + p.ncols * kI8MetaDoubles);    // [slot][CPI][128]
+    uint8_t* wring = smem + i8_wring_offset(p.ncols);             // [WS][128 rows][CPI][144]
     uint64_t* wfull = reinterpret_cast<uint64_t*>(wring + WS * kStage);
     uint64_t* wempty = wfull + kI8MaxWStages;
     uint64_t* afull = wempty + kI8MaxWStages;  // decoded A in TMEM buffer
@@ -371,6 +362,10 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     const int count = static_cast<int>(f1 - f0);
     const int tile0 = static_cast<int>(f0 / npi);
     const int i00 = static_cast<int>(f0 % npi);
+    // digit-image slot of (padded) column pb: its distance from the CTA's first
+    // column, modulo the padded row
+    const int pb_first = i00 * CPI;
+    auto slot_of = [&](int pb) { return pb >= pb_first ? pb - pb_first : pb - pb_first + pnsb; };
 
     if (threadIdx.x == 0) {
         abort_flag = 0;
@@ -422,7 +417,7 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     __syncwarp();
 
     pdl_wait();   // x is produced, and y may be read, by the preceding work on the stream
-    i8_digits(p.x, nsb, i00 * CPI, count * CPI < nsb ? count * CPI : nsb, image, meta, warp, kI8Warps, lane);
+    i8_digits(p.x, nsb, pnsb, pb_first, count * CPI < pnsb ? count * CPI : pnsb, image, meta, warp, kI8Warps, lane);
     fence_proxy_async_smem();   // the image is read by the MMAs
     __syncthreads();
 
@@ -458,7 +453,9 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
             if (elect_one()) {
 #pragma unroll
                 for (int c = 0; c < CPI; ++c) {
-                    const uint32_t img = smem_addr(image + static_cast<size_t>(i * CPI + c) * kI8ImageBytes);
+                    const int pb = i * CPI + c;
+                    if (pb >= nsb) continue;   // past the row: no MMA, the epilogue skips it
+                    const uint32_t img = smem_addr(image + static_cast<size_t>(slot_of(pb)) * kI8ImageBytes);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         // K position 32j: atom j / 4 (N * 128 bytes each), 32 bytes
@@ -573,13 +570,15 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&dfree[a]);
-                const Header hd = decode_header(hraw);
-                const int b = i * CPI + c;
-                const double* mb = meta + static_cast<size_t>(b) * kI8MetaDoubles;
-                double part;
-                if constexpr (CPI == 2) part = i8_column_sum<8>(r, hd, mb, 0);
-                else part = i8_column_sum<4>(r, hd, mb, 4 * half);
-                ytot = fma(mb[0], part, ytot);
+                const int pb = i * CPI + c;
+                if (pb < nsb) {   // a column past the row (odd K/256, two columns per item) adds nothing
+                    const Header hd = decode_header(hraw);
+                    const double* mb = meta + static_cast<size_t>(slot_of(pb)) * kI8MetaDoubles;
+                    double part;
+                    if constexpr (CPI == 2) part = i8_column_sum<8>(r, hd, mb, 0);
+                    else part = i8_column_sum<4>(r, hd, mb, 4 * half);
+                    ytot = fma(mb[0], part, ytot);
+                }
             } else {
                 abort_flag = 1;
             }
@@ -626,49 +625,50 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
 
 }  // namespace
 
-int i8_max_nsb(int max_smem) {
-    int nsb = 0;
-    while (i8_wstages_nsb(nsb + 1) >= kI8MinWStages && i8_smem_bytes_nsb(nsb + 1) <= max_smem) ++nsb;
-    return nsb;
-}
-
-int i8_smem_bytes(int nsb) { return i8_smem_bytes_nsb(nsb); }
-int i8_wstages(int nsb) { return i8_wstages_nsb(nsb); }
-int i8_threads() { return kI8Threads; }
-int i8_cpi(int nsb) { return i8_cpi_nsb(nsb); }
-
-int i8_ctas(int tiles, int nsb, int num_sms) {
-    if (i8_whole_tiles(tiles, num_sms)) return num_sms;
-    const long long items = static_cast<long long>(tiles) * (nsb / i8_cpi_nsb(nsb));
-    return items < num_sms ? static_cast<int>(items) : num_sms;
-}
-
 bool i8_whole_tiles(int tiles, int num_sms) {
     if (tiles < num_sms) return false;
     const long long busiest = (static_cast<long long>(tiles) + num_sms - 1) / num_sms;
     return busiest * num_sms * kI8MaxImbalance <= static_cast<long long>(tiles) * (kI8MaxImbalance + 1);
 }
 
-bool i8_cuts_tiles(int tiles, int nsb, int num_sms) {
-    if (i8_whole_tiles(tiles, num_sms)) return false;
-    const int npi = nsb / i8_cpi_nsb(nsb);
-    const long long items = static_cast<long long>(tiles) * npi;
-    const int ctas = i8_ctas(tiles, nsb, num_sms);
-    for (int c = 1; c < ctas; ++c)
-        if ((items * c / ctas) % npi != 0) return true;
-    return false;
-}
+int i8_threads() { return kI8Threads; }
 
-bool i8_applies(int m, int n, int k, int num_sms, int max_smem) {
+bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg) {
     if (m != 1 || n < 1 || k < kQK || k % kQK != 0 || num_sms < 1) return false;
     const int nsb = k / kQK;
-    if (nsb > i8_max_nsb(max_smem)) return false;
     const long long tiles = (static_cast<long long>(n) + kI8Rows - 1) / kI8Rows;
     if (tiles * nsb >= (1LL << 31) / num_sms) return false;   // item counts in 32 bits
-    // whole tiles per CTA, or enough (tile, column) items per CTA that the
+    const bool whole = i8_whole_tiles(static_cast<int>(tiles), num_sms);
+    // whole tiles per CTA, or enough (tile, column) units per CTA that the
     // kernel's fixed cost (digit image, pipeline fill, cut tiles) pays off
-    return i8_whole_tiles(static_cast<int>(tiles), num_sms) ||
-           tiles * nsb >= static_cast<long long>(kI8MinItemsPerCta) * num_sms;
+    if (!whole && tiles * nsb < static_cast<long long>(kI8MinItemsPerCta) * num_sms) return false;
+    const int budget = max_smem < kI8SmemBudget ? max_smem : kI8SmemBudget;
+    // two columns per item unless an odd K/256 is small (the padded column of
+    // each tile's last item would be a large share of the work)
+    for (int cpi = (nsb % 2 == 0 || nsb >= 9) ? 2 : 1; cpi >= 1; --cpi) {
+        I8Config c;
+        c.cpi = cpi;
+        c.npi = (nsb + cpi - 1) / cpi;
+        c.items = tiles * c.npi;
+        c.whole = whole ? 1 : 0;
+        c.ctas = whole ? num_sms : static_cast<int>(c.items < num_sms ? c.items : num_sms);
+        c.items_per_cta_max = whole ? (tiles + c.ctas - 1) / c.ctas * c.npi : (c.items + c.ctas - 1) / c.ctas;
+        const long long pnsb = static_cast<long long>(c.npi) * cpi;
+        c.ncols = static_cast<int>(c.items_per_cta_max * cpi < pnsb ? c.items_per_cta_max * cpi : pnsb);
+        const int fit = i8_fit_stages(c.ncols, cpi);
+        // the kernel's instantiations: 4 two-column stages; 8, 6 or 4 one-column
+        if (fit < kI8MinWStages) continue;
+        c.wstages = cpi == 2 ? 4 : fit >= 8 ? 8 : fit >= 6 ? 6 : 4;
+        c.smem = i8_smem_bytes_cfg(c.ncols, cpi, c.wstages);
+        if (c.smem > budget) continue;
+        c.cuts = 0;
+        if (!whole)
+            for (int q = 1; q < c.ctas && !c.cuts; ++q)
+                if ((c.items * q / c.ctas) % c.npi != 0) c.cuts = 1;
+        *cfg = c;
+        return true;
+    }
+    return false;
 }
 
 namespace {
@@ -771,13 +771,12 @@ bool make_weight_map3(CUtensorMap* map, const void* w, int n, int nsb, int cpi) 
 
 int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int n, int k,
                    cudaStream_t stream) {
+    I8Config c;
+    if (!i8_config(1, n, k, dev.sm_count, dev.max_smem_optin, &c)) return Q4K_ERR_SHAPE;   // not reached
     const int nsb = k / kQK;
-    const int cpi = i8_cpi_nsb(nsb);
     const int tiles = (n + kI8Rows - 1) / kI8Rows;
-    const int ctas = i8_ctas(tiles, nsb, dev.sm_count);
-    const bool whole = i8_whole_tiles(tiles, dev.sm_count);
     CUtensorMap map;
-    if (!make_weight_map3(&map, w, n, nsb, cpi)) return cuda_failure(cudaErrorInvalidValue);
+    if (!make_weight_map3(&map, w, n, nsb, c.cpi)) return cuda_failure(cudaErrorInvalidValue);
     // Tiles cut between CTAs: the stream's scratch, or (a graph being
     // captured on a stream without one) a stream-ordered allocation of this
     // call, counters zeroed on the stream.
@@ -785,12 +784,12 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
     double* part = nullptr;
     void* own = nullptr;
     cudaError_t e = cudaSuccess;
-    if (i8_cuts_tiles(tiles, nsb, dev.sm_count)) {
+    if (c.cuts) {
         int device = 0;
         e = cudaGetDevice(&device);
-        if (e == cudaSuccess) e = stream_scratch(device, stream, tiles, ctas, &done, &part);
+        if (e == cudaSuccess) e = stream_scratch(device, stream, tiles, c.ctas, &done, &part);
         if (e == cudaSuccess && done == nullptr) {
-            e = cudaMallocAsync(&own, scratch_part_offset(tiles) + static_cast<size_t>(ctas) * 2 * kI8Rows * sizeof(double),
+            e = cudaMallocAsync(&own, scratch_part_offset(tiles) + static_cast<size_t>(c.ctas) * 2 * kI8Rows * sizeof(double),
                                 stream);
             if (e == cudaSuccess) e = cudaMemsetAsync(own, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream);
             done = static_cast<unsigned*>(own);
@@ -798,22 +797,21 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
         }
         if (e != cudaSuccess) return cuda_failure(e);
     }
-    const I8Params ip{x, y, part, done, n, nsb, tiles, nsb / cpi, whole ? 1 : 0};
+    const I8Params ip{x, y, part, done, n, nsb, tiles, c.npi, c.ncols, c.whole};
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(static_cast<unsigned>(ctas));
+    cfg.gridDim = dim3(static_cast<unsigned>(c.ctas));
     cfg.blockDim = dim3(kI8Threads);
-    cfg.dynamicSmemBytes = static_cast<size_t>(i8_smem_bytes_nsb(nsb));
+    cfg.dynamicSmemBytes = static_cast<size_t>(c.smem);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int wstages = i8_wstages_nsb(nsb);
-    e = cpi == 2         ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 2>, map, ip)
-        : wstages >= 8   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8, 1>, map, ip)
-        : wstages >= 6   ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6, 1>, map, ip)
-                         : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 1>, map, ip);
+    e = c.cpi == 2          ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 2>, map, ip)
+        : c.wstages >= 8    ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8, 1>, map, ip)
+        : c.wstages >= 6    ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6, 1>, map, ip)
+                            : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 1>, map, ip);
     if (own != nullptr) {
         const cudaError_t ef = cudaFreeAsync(own, stream);
         if (e == cudaSuccess) e = ef;

@@ -16,27 +16,29 @@ constexpr int kI8SmemBudget = 220 * 1024;   // dynamic shared memory a CTA may u
 constexpr int kI8MaxImbalance = 8;   // whole tiles per CTA: the busiest CTA at most 1/8 above the mean
 constexpr int kI8MinItemsPerCta = 5; // cut tiles: at least this many items per CTA on average
 
-// Superblocks per row the kernel keeps the vector's digit image for (shared
-// memory): K up to 256 times this.
-int i8_max_nsb(int max_smem);
-int i8_smem_bytes(int nsb);
-// superblock columns per item (1 or 2) and weight stages (of that many columns)
-int i8_cpi(int nsb);
-int i8_wstages(int nsb);
-int i8_threads();
+// One call's launch shape on the kernel.
+struct I8Config {
+    int cpi;                      // superblock columns per item (1 or 2)
+    int npi;                      // items per tile: ceil(nsb / cpi)
+    int ncols;                    // digit-image slots a CTA keeps (its columns, padded)
+    int wstages;                  // weight stages of cpi columns
+    int ctas;                     // one per SM at most
+    int whole;                    // 1: equal ranges of whole tiles, else of items
+    int cuts;                     // 1: some tile is cut between CTAs (pieces in the scratch)
+    int smem;                     // dynamic shared memory per CTA
+    long long items;              // tiles * npi
+    long long items_per_cta_max;
+};
+
 // Whole 128-row tiles per CTA: at least one tile per SM and the busiest CTA
 // at most 1/kI8MaxImbalance above the mean.
 bool i8_whole_tiles(int tiles, int num_sms);
-// CTAs: one per SM at most, owning whole tiles (i8_whole_tiles) or equal
-// contiguous ranges of the tiles x nsb (tile, superblock column) items.
-int i8_ctas(int tiles, int nsb, int num_sms);
-// True if some CTA range starts inside a tile (the tile is then finished from
-// pieces in the stream's scratch).
-bool i8_cuts_tiles(int tiles, int nsb, int num_sms);
-// True if q4k_gemv runs one vector of this shape on the kernel: the vector's
-// digit image fits beside four weight stages, and the CTAs own whole tiles or
-// at least kI8MinItemsPerCta items each on average.
-bool i8_applies(int m, int n, int k, int num_sms, int max_smem);
+int i8_threads();
+// True (and *cfg filled) if q4k_gemv runs one vector of this shape on the
+// kernel: whole tiles per CTA or at least kI8MinItemsPerCta superblock columns
+// per CTA on average, and the CTA's digit image beside at least four weight
+// stages (two columns per item where that fits, else one).
+bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg);
 
 int i8_set_attributes();
 int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int n, int k,

@@ -141,7 +141,7 @@ def test_gemv_multivector_shapes(q4k, n, k, m):
     assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
 
 
-@pytest.mark.parametrize("n,k", [(75904, 256), (100000, 20480), (151936, 20480), (8192, 28672)])
+@pytest.mark.parametrize("n,k", [(75904, 256), (100000, 20480), (151936, 20480), (64, 28672)])
 def test_gemv_tall_two_slices_sampled(q4k, n, k):
     """Very tall matrices (512 or more rows per CTA) that the integer
     tensor-core kernel does not take (K beyond its digit image, or too few
@@ -166,11 +166,15 @@ def test_gemv_tall_two_slices_sampled(q4k, n, k):
                                    (7, 150, 11008), (4, 1, 14336), (3, 5, 8192)])
 def test_gemv_k_chunks_and_vector_groups(q4k, m, n, k):
     """K beyond one team: one or two vectors run as K-chunks of strided row
-    segments on the streaming kernel, later chunks adding into y; three or more
-    run on the tensor-core kernel, which takes any K; y starts as NaN, so the
-    first launch must overwrite it."""
+    segments on the streaming kernel, later chunks adding into y (one vector
+    on a matrix with enough superblock columns per SM, 4096 x 61440, runs on
+    the integer tensor-core kernel instead); three or more run on the
+    tensor-core kernel, which takes any K; y starts as NaN, so the first
+    launch must overwrite it."""
     plan = q4k.q4k_gemv_plan_for(m, n, k, torch.cuda.get_device_properties(0).multi_processor_count)
-    assert plan["kernel"] == (q4k.Q4K_KERNEL_STREAM if m <= 2 else q4k.Q4K_KERNEL_TC)
+    expected = (q4k.Q4K_KERNEL_I8 if (m, n, k) == (1, 4096, 61440) else q4k.Q4K_KERNEL_STREAM) if m <= 2 \
+        else q4k.Q4K_KERNEL_TC
+    assert plan["kernel"] == expected
     w, x = q4k_synth.q4k_problem(n, k, m, 70 + m + n)
     y = gpu_gemv(q4k, w, x, n, k)
     if n * k <= 4096 * 61440 // 8:

@@ -258,60 +258,69 @@ def i8_whole(tiles):
     return tiles >= SM_COUNT and busiest * SM_COUNT * 8 <= tiles * 9
 
 
-def i8_expected(m, n, k):
-    """Whether q4k_gemv runs this shape on the integer tensor-core kernel: one
-    vector, the digit image plus four weight stages in the shared-memory
-    budget (K <= 256 * 62), and whole tiles per CTA (at least one 128-row tile
-    per SM, the busiest CTA at most 1/8 above the mean) or at least 5 (tile,
-    superblock column) items per CTA on average."""
+def i8_config(n, k):
+    """The integer kernel's launch for one vector of an n x k matrix, or None:
+    whole tiles per CTA (at least one 128-row tile per SM, the busiest CTA at
+    most 1/8 above the mean) or at least 5 superblock columns per CTA on
+    average; items of two superblock columns (padded at the end of a tile for
+    an odd K/256 >= 9) where four two-column weight stages fit beside the
+    CTA's digit-image slots (2 KB image + 80 B metadata per column, 8 x 2 KB of
+    header ring), else one column with 8, 6 or 4 stages."""
     tiles, nsb = -(-n // 128), k // 256
-    if m != 1 or nsb > 62:
-        return False
-    return i8_whole(tiles) or tiles * nsb >= 5 * SM_COUNT
+    whole = i8_whole(tiles)
+    if not whole and tiles * nsb < 5 * SM_COUNT:
+        return None
+    barriers = 2 * 8 + 4 + 2 * 4 + 2 * 8 + 1
+    for cpi in ([2, 1] if nsb % 2 == 0 or nsb >= 9 else [1]):
+        npi = -(-nsb // cpi)
+        items = tiles * npi
+        ctas = SM_COUNT if whole else min(items, SM_COUNT)
+        per = -(-tiles // ctas) * npi if whole else -(-items // ctas)
+        ncols = min(per * cpi, npi * cpi)
+        off = -(-(ncols * (2048 + 80) + 8 * 2048) // 1024) * 1024
+        fit = (220 * 1024 - 1024 - off - barriers * 8 - 16) // (cpi * 128 * 144)
+        if fit < 4:
+            continue
+        ws = 4 if cpi == 2 else 8 if fit >= 8 else 6 if fit >= 6 else 4
+        smem = 1024 + off + ws * cpi * 128 * 144 + barriers * 8 + 16
+        return dict(cpi=cpi, npi=npi, items=items, ctas=ctas, per=per, ncols=ncols, ws=ws, smem=smem,
+                    whole=whole)
+    return None
+
+
+def i8_expected(m, n, k):
+    return m == 1 and i8_config(n, k) is not None
 
 
 def check_i8_plan(n, k):
-    """One persistent CTA per SM at most: whole 128-row tiles in equal
-    contiguous tile ranges, or equal contiguous ranges of the tiles x nsb
-    items; 18 warps; the vector's digit image (2 KB per superblock column),
-    its block metadata (80 B per column), an 8-slot header ring (2 KB each)
-    and 8, 6 or 4 weight stages of 128 x 144 bytes in 220 KB."""
+    """One persistent CTA per SM at most over equal contiguous ranges of whole
+    tiles or of items; 18 warps; the plan's smem, stages and per-CTA share as
+    the launch rule above gives them."""
     p = q4k.q4k_gemv_plan_for(1, n, k, SM_COUNT)
     assert p["kernel"] == q4k.Q4K_KERNEL_I8, p
+    c = i8_config(n, k)
     tiles, nsb = -(-n // 128), k // 256
-    whole = i8_whole(tiles)
-    off = -(-(nsb * (2048 + 80) + 8 * 2048) // 1024) * 1024
-    barriers = 2 * 8 + 4 + 2 * 4 + 2 * 8 + 1
-    fit = lambda cpi: (220 * 1024 - 1024 - off - barriers * 8 - 16) // (cpi * 128 * 144)
-    cpi = 2 if nsb % 2 == 0 and fit(2) >= 4 else 1     # superblock columns per item
-    ws = 4 if cpi == 2 else 8 if fit(1) >= 8 else 6 if fit(1) >= 6 else 4
-    assert fit(cpi) >= 4 and p["depth"] == ws
-    assert p["smem_bytes"] == 1024 + off + ws * cpi * 128 * 144 + barriers * 8 + 16 <= 220 * 1024
-    npi = nsb // cpi
-    items = tiles * npi
-    assert p["grid"] == (SM_COUNT if whole else min(items, SM_COUNT))
-    assert p["block"] == 18 * 32 and p["cluster"] == 1 and p["launches"] == 1 and p["units"] == tiles * nsb
-    if whole:
-        ranges = [(tiles * c // p["grid"] * npi, tiles * (c + 1) // p["grid"] * npi) for c in range(p["grid"])]
+    assert p["grid"] == c["ctas"] and p["block"] == 18 * 32 and p["cluster"] == 1 and p["launches"] == 1
+    assert p["slices"] == c["cpi"] and p["depth"] == c["ws"] and p["smem_bytes"] == c["smem"] <= 220 * 1024
+    assert p["units"] == tiles * nsb and p["units_per_cta_max"] == c["per"] * c["cpi"]
+    npi, items = c["npi"], c["items"]
+    if c["whole"]:
+        ranges = [(tiles * q // p["grid"] * npi, tiles * (q + 1) // p["grid"] * npi) for q in range(p["grid"])]
         assert all(a % npi == 0 and b % npi == 0 for a, b in ranges)   # no tile is cut
-        assert p["units_per_cta_max"] == -(-tiles // p["grid"]) * nsb
     else:
-        ranges = [(items * c // p["grid"], items * (c + 1) // p["grid"]) for c in range(p["grid"])]
-        assert p["units_per_cta_max"] == -(-items // p["grid"]) * cpi
+        ranges = [(items * q // p["grid"], items * (q + 1) // p["grid"]) for q in range(p["grid"])]
         assert max(b - a for a, b in ranges) - min(b - a for a, b in ranges) <= 1
     assert ranges[0][0] == 0 and ranges[-1][1] == items
     assert all(r1 == s2 for (_, r1), (s2, _) in zip(ranges, ranges[1:]))
-    # a tile cut between CTAs: its pieces come from consecutive CTAs, at most
-    # two per CTA (the tile its range starts in and the one it ends in)
-    for a, b in ranges:
-        if b > a:
-            assert (b - 1) // nsb - a // nsb + 1 >= 1
+    # a CTA's digit-image slots cover every (padded) column of its range
+    assert all(min((b - a) * c["cpi"], npi * c["cpi"]) <= c["ncols"] for a, b in ranges)
     return p
 
 
 @pytest.mark.parametrize("n,k", SHAPES + [(148 * 128, 256), (296 * 128 - 51, 512), (1184 * 128 + 1, 4096),
                                           (160 * 128, 4096), (128256, 15872), (128256, 16128),
-                                          (3000, 15872), (4096 + 77, 8192), (2048, 8192)])
+                                          (3000, 15872), (4096 + 77, 8192), (2048, 8192), (4096, 28672),
+                                          (5000, 11008), (151553, 256), (8192, 28672), (18944, 15872)])
 @pytest.mark.parametrize("m", [1, 2])
 def test_i8_choice(m, n, k):
     """One vector runs on the integer tensor-core kernel where it pays; any
@@ -336,7 +345,7 @@ def test_i8_sweep_choice():
 def test_lm_head_partition():
     """The LM head (1002 tiles): 7 tiles on 114 CTAs, 6 on the other 34."""
     p = check_i8_plan(128256, 4096)
-    assert p["units_per_cta_max"] == 7 * 16 and p["depth"] == 4   # four stages of two columns
+    assert p["units_per_cta_max"] == 7 * 16 and p["depth"] == 4 and p["slices"] == 2   # four stages of two columns
     # beyond the digit image's K the tall matrix streams with two-slice lanes
     p = check_plan(1, 128256, 20480)
     assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2
