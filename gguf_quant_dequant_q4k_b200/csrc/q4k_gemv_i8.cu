@@ -226,60 +226,60 @@ __device__ __forceinline__ int i8_item_owner(long long items, long long f, int c
     return static_cast<int>(((f + 1) * ctas - 1) / items);
 }
 
-// After the CTA's last item, the 128 threads of the epilogue's first half
-// (thread = row) make the CTA's cut pieces (slot 0: the tile its range starts
-// in, slot 1: the tile it ends in) visible, count them in per tile, and
-// finish each tile whose last piece this CTA published: add the pieces of
-// the CTAs holding part of the tile, in CTA order, and store y.
-__device__ __forceinline__ void i8_finish_pieces(const I8Params& p, long long items, bool has0, int t0,
-                                                 bool has1, int t1, int row, int* last_flags,
-                                                 bool aborted) {
-    __threadfence();
-    named_barrier_sync(kI8PieceBarrier, kI8Rows);
-    if (row < 2) {
-        const bool has = row == 0 ? has0 : has1;
-        const int t = row == 0 ? t0 : t1;
+// Counter add with acquire-release semantics at GPU scope: it publishes every
+// write the CTA ordered before it (a barrier) and sees every piece published
+// before it.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* ptr, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+    return old;
+}
+
+// The 128 threads of the epilogue's first half (thread = row) publish the
+// CTA's piece of tile t (slot 0: the tile its range starts in, slot 1: the
+// one it ends in; the totals are already stored) and, if it is the tile's
+// last piece, finish the tile: add the pieces of the CTAs holding part of it,
+// in CTA order, and store y.
+// (Out of line: it runs at most twice per CTA, and inlined its registers would
+// spill those of the epilogue loop.)
+__device__ __noinline__ void i8_publish_piece(const double* part, unsigned* done, float* y, int n, int npi,
+                                              long long items, int t, int row, int* last_flag, bool aborted) {
+    named_barrier_sync(kI8PieceBarrier, kI8Rows);   // every row's total is stored
+    const long long tf0 = static_cast<long long>(t) * npi;
+    const int c_first = i8_item_owner(items, tf0, gridDim.x);
+    const int c_last = i8_item_owner(items, tf0 + npi - 1, gridDim.x);
+    if (row == 0) {
         bool last = false;
-        if (has && !aborted) {
-            const long long tf0 = static_cast<long long>(t) * p.npi;
-            const int pieces = i8_item_owner(items, tf0 + p.npi - 1, gridDim.x) - i8_item_owner(items, tf0, gridDim.x);
-            last = atomicAdd(&p.done[t], 1u) == static_cast<unsigned>(pieces);
-            if (last) p.done[t] = 0u;   // every other piece is in: the counter is free for the next launch
+        if (!aborted) {
+            last = atom_add_acq_rel_gpu(&done[t], 1u) == static_cast<unsigned>(c_last - c_first);
+            if (last) done[t] = 0u;   // every other piece is in: the counter is free for the next launch
         }
-        last_flags[row] = last ? 1 : 0;
+        *last_flag = last ? 1 : 0;
     }
     named_barrier_sync(kI8PieceBarrier, kI8Rows);
-#pragma unroll 1
-    for (int q = 0; q < 2; ++q) {
-        if (!last_flags[q]) continue;
-        __threadfence();
-        const int t = q == 0 ? t0 : t1;
-        const long long tf0 = static_cast<long long>(t) * p.npi;
-        const int c_first = i8_item_owner(items, tf0, gridDim.x);
-        const int c_last = i8_item_owner(items, tf0 + p.npi - 1, gridDim.x);
-        // Every CTA after c_first starts inside tile t (its piece is slot 0);
-        // c_first's piece is slot 0 only if its range starts at the tile.
-        const int first_slot = i8_item_begin(items, c_first, gridDim.x) < tf0 ? 1 : 0;
-        double tot = 0.0;
-        // four pieces per round: their loads are independent and in flight together
-        for (int c0 = c_first; c0 <= c_last; c0 += 4) {
-            double val[4];
+    if (!*last_flag) return;
+    // Every CTA after c_first starts inside tile t (its piece is slot 0);
+    // c_first's piece is slot 0 only if its range starts at the tile.
+    const int first_slot = i8_item_begin(items, c_first, gridDim.x) < tf0 ? 1 : 0;
+    double tot = 0.0;
+    // four pieces per round: their loads are independent and in flight together
+    for (int c0 = c_first; c0 <= c_last; c0 += 4) {
+        double val[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int c = c0 + j;
-                const int cs = c == c_first ? first_slot : 0;
-                val[j] = c <= c_last ? __ldcg(p.part + (static_cast<size_t>(c) * 2 + cs) * kI8Rows + row) : 0.0;
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) tot += val[j];   // pieces added in CTA order
+        for (int j = 0; j < 4; ++j) {
+            const int c = c0 + j;
+            const int cs = c == c_first ? first_slot : 0;
+            val[j] = c <= c_last ? __ldcg(part + (static_cast<size_t>(c) * 2 + cs) * kI8Rows + row) : 0.0;
         }
-        const int grow = t * kI8Rows + row;
-        if (grow < p.n) p.y[grow] = static_cast<float>(tot);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tot += val[j];   // pieces added in CTA order
     }
+    const int grow = t * kI8Rows + row;
+    if (grow < n) y[grow] = static_cast<float>(tot);
 }
 
 // The epilogue's sum for one row and one superblock column over sub-blocks
-// j0 .. j0 + NJ - 1: r holds D_j[l] at r[(j - j0) * N + l]. Returns
+// j0 .. j0 + NJ - 1: r holds D_j[l] at r[(j - j0) * 5 + l]. Returns
 // d * S - dmin * M with S = sum_j sc_j * T_j, T_j = sum_l 128^l D_j[l] (D / 16
 // for odd j) = lo_j + 2^21 hi_j, lo_j = D0 + 128 D1 + 2^14 D2 (|lo| < 2^29),
 // hi_j = D3 + 128 D4 (|hi| < 2^22): sum sc*lo in 64 bits, sum sc*hi in 32
@@ -293,7 +293,7 @@ __device__ __forceinline__ double i8_column_sum(const uint32_t* r, const Header&
 #pragma unroll
     for (int jj = 0; jj < NJ; ++jj) {
         const int j = j0 + jj;
-        const uint32_t* rj = r + jj * kI8N;
+        const uint32_t* rj = r + jj * kI8Limbs;
         const int D0 = static_cast<int>(rj[0]), D1 = static_cast<int>(rj[1]);
         const int D2 = static_cast<int>(rj[2]), D3 = static_cast<int>(rj[3]);
         const int D4 = static_cast<int>(rj[4]);
@@ -542,12 +542,11 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         const int half = (warp - kI8DecodeWarps) / kI8Quarters;
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
-        constexpr int kCols = CPI == 2 ? 64 : 32;   // accumulator columns a half reads
         double ytot = 0.0;
         int tile = tile0, i = i00;
         int istart = i;                    // first item of the current piece
-        bool has0 = false, has1 = false;   // cut pieces written (slot 0 / 1)
-        int tile1 = 0;                     // tile of the slot-1 piece
+        bool has1 = false;                 // a cut piece left to publish after the last item
+        int tile1 = 0;                     // its tile
         int parity = 0;                    // alternates per piece: one barrier per piece
         for (int it = 0; it < count; ++it) {
             const int grow = tile * kI8Rows + row;
@@ -561,11 +560,12 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&hfree[hs]);
                 tc_fence_after_sync();
-                uint32_t r[kCols];   // D_j[l] of the half's sub-blocks at (j - j0) * N + l
+                constexpr int kNJ = CPI == 2 ? 8 : 4;   // sub-blocks this half sums
+                uint32_t r[kNJ * kI8Limbs];            // D_j[l] at (j - j0) * 5 + l: the digit columns only
                 const uint32_t dcol = lane_base + static_cast<uint32_t>(kI8Dcol0 + a * CPI * kI8ColAcc +
                                                                         (CPI == 2 ? c * kI8ColAcc : 32 * half));
-                tmem_load_32cols_async(dcol, *reinterpret_cast<uint32_t(*)[32]>(r));
-                if constexpr (CPI == 2) tmem_load_32cols_async(dcol + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+#pragma unroll
+                for (int jj = 0; jj < kNJ; ++jj) tmem_load_5cols(dcol + static_cast<uint32_t>(jj * kI8N), r + jj * kI8Limbs);
                 tmem_wait_ld();
                 tc_fence_before_sync();
                 __syncwarp();
@@ -591,13 +591,18 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                     const double tot = ytot + xc[row];
                     if (istart == 0 && i == npi - 1) {   // the whole tile
                         if (!abort_flag && grow < p.n) p.y[grow] = static_cast<float>(tot);
-                    } else if (tile == tile0) {
-                        p.part[(static_cast<size_t>(blockIdx.x) * 2 + 0) * kI8Rows + row] = tot;
-                        has0 = true;
                     } else {
-                        p.part[(static_cast<size_t>(blockIdx.x) * 2 + 1) * kI8Rows + row] = tot;
-                        has1 = true;
-                        tile1 = tile;
+                        // a piece: slot 0 is published at once (the rest of
+                        // the range follows), slot 1 after the last item
+                        const int slot = tile == tile0 ? 0 : 1;
+                        p.part[(static_cast<size_t>(blockIdx.x) * 2 + slot) * kI8Rows + row] = tot;
+                        if (slot == 0 && it < count - 1) {
+                            i8_publish_piece(p.part, p.done, p.y, p.n, npi, items, tile, row, &last_piece[0],
+                                             abort_flag != 0);
+                        } else {
+                            has1 = true;
+                            tile1 = tile;
+                        }
                     }
                 }
                 ytot = 0.0;
@@ -611,8 +616,8 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         }
         // every thread of the first half takes this branch or none (the
         // pieces depend only on the CTA's range)
-        if (half == 0 && (has0 || has1))
-            i8_finish_pieces(p, items, has0, tile0, has1, tile1, row, last_piece, abort_flag != 0);
+        if (half == 0 && has1)
+            i8_publish_piece(p.part, p.done, p.y, p.n, npi, items, tile1, row, &last_piece[1], abort_flag != 0);
     }
 
     tc_fence_before_sync();
