@@ -76,7 +76,8 @@ def measured_peak():
 
 
 GEMV_SOURCES = ("q4k_gemv_stream.cu", "q4k_stream.h", "q4k_gemv.cu", "q4k_sm100.cuh",
-                "q4k_superblock.cuh", "q4k_swiglu.cuh")
+                "q4k_superblock.cuh", "q4k_swiglu.cuh", "q4k_gemv_i8.cu", "q4k_gemv_i8.h",
+                "q4k_tcgen05.cuh")
 
 
 def source_digest() -> str:
