@@ -240,7 +240,7 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const floa
                 int m, int n, int k, cudaStream_t stream) {
     q4k_gemv_plan plan;
     const bool fused = w2 != nullptr;
-    if (use_i8(m, n, k, dev.sm_count, dev.max_smem_optin, fused)) return launch_gemv_i8(dev, w, x, y, n, k, stream);
+    if (use_i8(m, n, k, dev.sm_count, dev.max_smem_optin, fused)) return launch_gemv_i8(dev, w, x, y, m, n, k, stream);
     if (use_tc(m, fused)) return launch_gemv_tc(dev, w, x, y, m, n, k, stream);
     const int gsz = group_size(m);
     int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin,

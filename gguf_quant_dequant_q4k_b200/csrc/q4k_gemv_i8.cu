@@ -26,6 +26,16 @@
 //   row's f64 total; y is that total rounded to f32 once. So
 //   |y - sum w x| <= 2^-24 (|y| + sum |w x|) + sum_t |w_t| 2^(E_t - 34), the
 //   bound of the batched tensor-core path; non-finite x makes y NaN.
+// * Several vectors (m = 2..4: the pages' `BatchedQ4KGemv`, "realizar 0.8.5,
+//   src/cuda/executor/uses.rs", `batched_q4k_gemv_into`: W decoded once, every
+//   vector multiplied by it). Each decoded superblock column meets the digits
+//   of all MV = 2 or 4 vectors in the same 8 MMAs: vector v's block is scaled
+//   to X = round(x * 2^(30 - E_b)) (|X| <= 2^30; exact where |x| >= 2^(E_b -
+//   7), else off by at most 2^(E_b - 31)) and split into four balanced
+//   base-256 digits, B rows 4v .. 4v+3 (N = 4 MV). The epilogue forms
+//   P_l = sum_j sc_j D_j[l] in 32-bit integers (odd j: a separate sum, /16 at
+//   the end) and S = sum_l 256^l P_l in 64 bits (|S| < 2^50), then as above;
+//   the error bound's last term becomes sum_t |w_t| 2^(E_t - 31).
 // * Pipeline. A persistent CTA owns whole 128-row tiles, or an equal range of
 //   (tile, superblock column) items with tiles cut between CTAs finished from
 //   pieces, and walks its items in order; an item is one superblock column, or
@@ -69,52 +79,64 @@ namespace {
 // Two sets of four decode warps (one warp per TMEM lane quarter each) take
 // alternate items: a warp waits for its tensor-memory stores before it
 // signals the item, and the two sets keep two items' stores in flight.
+// Eight epilogue warps (two per lane quarter), the producer (weight copies)
+// and the MMA warp.
 constexpr int kI8Quarters = 4;
 constexpr int kI8DecodeSets = 2;
 constexpr int kI8DecodeWarps = kI8Quarters * kI8DecodeSets;   // warps 0-7: decode into TMEM
 constexpr int kI8EpiWarps = 2 * kI8Quarters;                   // warps 8-15: epilogue
-constexpr int kI8ProducerWarp = 16;    // weight copies
+constexpr int kI8ProducerWarp = 16;
 constexpr int kI8MmaWarp = 17;
 constexpr int kI8Warps = 18;
-constexpr unsigned kI8PieceBarrier = 5;   // named barrier of the epilogue's first half (1-4: quarter pairs)
 constexpr int kI8Threads = 32 * kI8Warps;
-constexpr int kI8Limbs = 5;
-constexpr int kI8N = 8;                      // MMA N: digit rows 0..4
-constexpr int kI8ImageBytes = kI8N * kQK;    // one block's digit image (K-major, swizzled)
-constexpr int kI8MetaDoubles = 10;           // 2^(E-33), S0_0..7, pad
+// named barrier of the threads publishing a piece (1-4: the quarter pairs of
+// the one-vector epilogue)
+constexpr unsigned kI8PieceBarrier = 5;
 constexpr int kI8RawBytes = kI8Rows * kBlockBytes;   // one superblock column of a tile
 constexpr int kI8ColTmem = 64;               // TMEM columns of one decoded superblock column (256 bytes)
-constexpr int kI8ColAcc = 8 * kI8N;          // accumulator columns of one superblock column
 constexpr int kI8TmemCols = 512;
-constexpr int kI8Dcol0 = 256;                // A buffers in TMEM columns 0..255, accumulators after them
-// An item is CPI (1 or 2) superblock columns of a tile: A buffers and
-// accumulators of CPI * 64 columns, 4 / CPI of each.
-__host__ __device__ constexpr int i8_bufs(int cpi) { return 4 / cpi; }
+constexpr int kI8VecMeta = 10;               // per vector and block: 2^(E-33) (2^(E-30)), S0_0..7, pad
+// MV vectors per launch (1, 2 or 4): digit rows of the B operand (MMA N;
+// rows 5..7 unused for one vector), digits per vector, one block's digit
+// image (K-major, swizzled), its metadata, accumulator columns of one
+// superblock column.
+__host__ __device__ constexpr int i8_n(int mv) { return mv == 1 ? 8 : 4 * mv; }
+__host__ __device__ constexpr int i8_limbs(int mv) { return mv == 1 ? 5 : 4; }
+__host__ __device__ constexpr int i8_image_bytes(int mv) { return i8_n(mv) * kQK; }
+__host__ __device__ constexpr int i8_meta_doubles(int mv) { return kI8VecMeta * mv; }
+__host__ __device__ constexpr int i8_col_acc(int mv) { return 8 * i8_n(mv); }
+// An item is CPI (1 or 2) superblock columns of a tile: A buffers of CPI * 64
+// TMEM columns and accumulators of CPI * 8N, 4 / CPI of each (2 for four
+// vectors), the A buffers first.
+__host__ __device__ constexpr int i8_bufs(int cpi, int mv) { return mv == 4 ? 2 : 4 / cpi; }
+__host__ __device__ constexpr int i8_dcol0(int cpi, int mv) { return i8_bufs(cpi, mv) * cpi * kI8ColTmem; }
 constexpr int kI8HSlotCols = 8;              // header ring: 8 superblock columns' row headers
 constexpr int kI8HeaderBytes = kI8Rows * 16;      // one column's row headers
 // barriers sized for one column per item (the most buffers)
 constexpr int kI8Barriers = 2 * kI8MaxWStages + 4 + 2 * 4 + 2 * kI8HSlotCols + 1;
-static_assert(kI8Dcol0 + 4 * kI8ColAcc <= kI8TmemCols && 4 * kI8ColTmem <= kI8Dcol0, "TMEM buffers");
+static_assert(i8_dcol0(1, 1) + 4 * i8_col_acc(1) <= kI8TmemCols &&
+              i8_dcol0(1, 4) + 2 * i8_col_acc(4) <= kI8TmemCols, "TMEM buffers");
 
 // Shared memory: [digit images][metadata] of the CTA's `ncols` superblock
 // columns, [row headers] (1024-aligned), [weight stages of CPI columns],
 // [barriers], TMEM slot.
-__host__ __device__ constexpr int i8_wring_offset(int ncols) {
-    return (ncols * (kI8ImageBytes + kI8MetaDoubles * 8) + kI8HSlotCols * kI8HeaderBytes + 1023) / 1024 * 1024;
+__host__ __device__ constexpr int i8_wring_offset(int ncols, int mv) {
+    return (ncols * (i8_image_bytes(mv) + i8_meta_doubles(mv) * 8) + kI8HSlotCols * kI8HeaderBytes + 1023) /
+           1024 * 1024;
 }
-__host__ __device__ constexpr int i8_fit_stages(int ncols, int cpi) {
-    return (kI8SmemBudget - 1024 - i8_wring_offset(ncols) - kI8Barriers * 8 - 16) / (cpi * kI8RawBytes);
+__host__ __device__ constexpr int i8_fit_stages(int ncols, int cpi, int mv) {
+    return (kI8SmemBudget - 1024 - i8_wring_offset(ncols, mv) - kI8Barriers * 8 - 16) / (cpi * kI8RawBytes);
 }
-__host__ __device__ constexpr int i8_smem_bytes_cfg(int ncols, int cpi, int wstages) {
-    return 1024 + i8_wring_offset(ncols) + wstages * cpi * kI8RawBytes + kI8Barriers * 8 + 16;
+__host__ __device__ constexpr int i8_smem_bytes_cfg(int ncols, int cpi, int wstages, int mv) {
+    return 1024 + i8_wring_offset(ncols, mv) + wstages * cpi * kI8RawBytes + kI8Barriers * 8 + 16;
 }
 
-// Byte offset of (row n, K position kk) in one block's digit image: two
-// 128-element atoms along K, each N rows x 128 bytes in the 128-byte swizzled
-// K-major layout (8-row groups 1024 bytes apart; 16-byte chunk c of row n
-// stored at chunk c ^ (n % 8)).
-__host__ __device__ constexpr int i8_image_offset(int n, int kk) {
-    return (kk >> 7) * (kI8N * 128) + (n >> 3) * 1024 + (n & 7) * 128 +
+// Byte offset of (row n, K position kk) in one block's digit image of N rows:
+// two 128-element atoms along K, each N rows x 128 bytes in the 128-byte
+// swizzled K-major layout (8-row groups 1024 bytes apart; 16-byte chunk c of
+// row n stored at chunk c ^ (n % 8)).
+__host__ __device__ constexpr int i8_image_offset(int n, int kk, int nrows) {
+    return (kk >> 7) * (nrows * 128) + (n >> 3) * 1024 + (n & 7) * 128 +
            ((((kk & 127) >> 4) ^ (n & 7)) << 4) + (kk & 15);
 }
 
@@ -176,16 +198,16 @@ __device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, 
         // S0 of sub-block j = lanes 4j .. 4j+3
         sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);
         sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
-        double* md = meta + static_cast<size_t>(j) * kI8MetaDoubles;
+        double* md = meta + static_cast<size_t>(j) * i8_meta_doubles(1);
         if ((lane & 3) == 0) md[1 + (lane >> 2)] = static_cast<double>(sum);
         if (lane == 0) {
             md[0] = finite ? (scaled ? __longlong_as_double(static_cast<long long>(1023 + ex - 33) << 52) : 0.0)
                            : __longlong_as_double(0x7FF8000000000000LL);
             md[9] = 0.0;
         }
-        uint8_t* img = image + static_cast<size_t>(j) * kI8ImageBytes;
+        uint8_t* img = image + static_cast<size_t>(j) * i8_image_bytes(1);
 #pragma unroll
-        for (int l = 0; l < kI8Limbs; ++l) {
+        for (int l = 0; l < i8_limbs(1); ++l) {
             if (l > 0) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -193,7 +215,76 @@ __device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, 
                     r[e] = (r[e] - dig[e]) >> 7;
                 }
             }
-            *reinterpret_cast<uint2*>(img + i8_image_offset(l, 8 * lane)) =
+            *reinterpret_cast<uint2*>(img + i8_image_offset(l, 8 * lane, i8_n(1))) =
+                make_uint2(pack_bytes(dig[0], dig[1], dig[2], dig[3]),
+                           pack_bytes(dig[4], dig[5], dig[6], dig[7]));
+        }
+    }
+}
+
+// The same for MV = 2 or 4 vectors (rows of x, `k` apart; vectors v >= m get
+// nothing, their accumulator columns are never read): one warp per (slot,
+// vector); X = round(x * 2^(30 - E_b)) split into four balanced base-256
+// digits X = sum_l 256^l X_l, X_l in [-128, 127] (|X| <= 2^30 leaves the last
+// one within [-64, 64]), B rows 4v + l; the vector's metadata at
+// meta[slot][10 v ..]: 2^(E_b - 30), pad, then S0_j (|S0_j| <= 2^35) as the
+// int pair (S0_j mod 2^18, floor(S0_j / 2^18)) for j = 0..7.
+template <int MV>
+__device__ __forceinline__ void i8_digits_mv(const float* __restrict__ x, int m, int k, int nsb, int pnsb, int b0,
+                                             int ncols, uint8_t* image, double* meta, int first, int stride,
+                                             int lane) {
+    for (int job = first; job < ncols * MV; job += stride) {
+        const int j = job / MV, vec = job % MV;
+        const int b = (b0 + j) % pnsb;
+        if (b >= nsb || vec >= m) continue;
+        const float4* src = reinterpret_cast<const float4*>(x + static_cast<size_t>(vec) * k +
+                                                            static_cast<size_t>(b) * kQK + 8 * lane);
+        const float4 a = src[0], c = src[1];
+        const float v[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        bool finite = true;
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            finite = finite && isfinite(v[e]);
+            amax = fmaxf(amax, fabsf(v[e]));
+        }
+        finite = __all_sync(0xFFFFFFFFu, finite);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        int ex = 0;
+        if (finite && amax > 0.f) frexpf(amax, &ex);   // amax in [2^(ex-1), 2^ex)
+        const bool scaled = finite && amax > 0.f;
+        // 2^(30 - ex) from its exponent field (ex >= -148)
+        const double up = scaled ? __longlong_as_double(static_cast<long long>(1023 + 30 - ex) << 52) : 0.0;
+        long long sum = 0;
+        int r[8];   // remainder after the digits so far
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            // exact scaling, one rounding (a non-finite block has X = 0)
+            r[e] = scaled ? __double2int_rn(static_cast<double>(v[e]) * up) : 0;
+            sum += r[e];
+        }
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 1);   // S0 of sub-block j = lanes 4j .. 4j+3
+        sum += __shfl_xor_sync(0xFFFFFFFFu, sum, 2);
+        double* md = meta + static_cast<size_t>(j) * i8_meta_doubles(MV) + kI8VecMeta * vec;
+        if ((lane & 3) == 0)   // S0_j = 2^18 h + l, l in [0, 2^18)
+            reinterpret_cast<int2*>(md + 2)[lane >> 2] =
+                make_int2(static_cast<int>(sum & 0x3FFFF), static_cast<int>(sum >> 18));
+        if (lane == 0) {
+            md[0] = finite ? (scaled ? __longlong_as_double(static_cast<long long>(1023 + ex - 30) << 52) : 0.0)
+                           : __longlong_as_double(0x7FF8000000000000LL);
+            md[1] = 0.0;
+        }
+        uint8_t* img = image + static_cast<size_t>(j) * i8_image_bytes(MV);
+#pragma unroll
+        for (int l = 0; l < i8_limbs(MV); ++l) {
+            int dig[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                dig[e] = ((r[e] + 128) & 255) - 128;
+                r[e] = (r[e] - dig[e]) >> 8;
+            }
+            *reinterpret_cast<uint2*>(img + i8_image_offset(4 * vec + l, 8 * lane, i8_n(MV))) =
                 make_uint2(pack_bytes(dig[0], dig[1], dig[2], dig[3]),
                            pack_bytes(dig[4], dig[5], dig[6], dig[7]));
         }
@@ -201,11 +292,11 @@ __device__ __forceinline__ void i8_digits(const float* __restrict__ x, int nsb, 
 }
 
 struct I8Params {
-    const float* x;      // [k]
-    float* y;            // [n]
-    double* part;        // tiles cut between CTAs: [CTA][2][128] partial row totals
+    const float* x;      // [m][k]
+    float* y;            // [m][n]
+    double* part;        // tiles cut between CTAs: [CTA][2][MV][128] partial row totals
     unsigned* done;      // tiles cut between CTAs: [tiles] pieces published (zero between launches)
-    int n, nsb, tiles;
+    int m, n, k, nsb, tiles;
     int npi;             // items per tile: ceil(nsb / CPI); the last one of a tile may
                          // hold a column past the row (zero-filled, skipped)
     int ncols;           // digit-image slots: the CTA's columns, from its first one
@@ -235,20 +326,24 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* ptr, unsigned
     return old;
 }
 
-// The 128 threads of the epilogue's first half (thread = row) publish the
-// CTA's piece of tile t (slot 0: the tile its range starts in, slot 1: the
-// one it ends in; the totals are already stored) and, if it is the tile's
-// last piece, finish the tile: add the pieces of the CTAs holding part of it,
-// in CTA order, and store y.
+// The `nthreads` publishing threads (the epilogue's first half for one
+// vector, thread = row; every epilogue warp for several, each with its row
+// and vector) publish the CTA's piece of tile t (slot 0: the tile its range
+// starts in, slot 1: the one it ends in; the totals of its mv vectors are
+// already stored) and, if it is the tile's last piece, finish the tile: add
+// the pieces of the CTAs holding part of it, in CTA order, and store y for
+// the thread's vectors v0, v0 + vstep, ... < v1. The leader thread takes the
+// counter.
 // (Out of line: it runs at most twice per CTA, and inlined its registers would
 // spill those of the epilogue loop.)
-__device__ __noinline__ void i8_publish_piece(const double* part, unsigned* done, float* y, int n, int npi,
-                                              long long items, int t, int row, int* last_flag, bool aborted) {
-    named_barrier_sync(kI8PieceBarrier, kI8Rows);   // every row's total is stored
+__device__ __noinline__ void i8_publish_piece(const double* part, unsigned* done, float* y, int n, int mv, int v0,
+                                              int v1, int vstep, int npi, long long items, int t, int row,
+                                              bool leader, int nthreads, int* last_flag, bool aborted) {
+    named_barrier_sync(kI8PieceBarrier, nthreads);   // every row's total is stored
     const long long tf0 = static_cast<long long>(t) * npi;
     const int c_first = i8_item_owner(items, tf0, gridDim.x);
     const int c_last = i8_item_owner(items, tf0 + npi - 1, gridDim.x);
-    if (row == 0) {
+    if (leader) {
         bool last = false;
         if (!aborted) {
             last = atom_add_acq_rel_gpu(&done[t], 1u) == static_cast<unsigned>(c_last - c_first);
@@ -256,26 +351,29 @@ __device__ __noinline__ void i8_publish_piece(const double* part, unsigned* done
         }
         *last_flag = last ? 1 : 0;
     }
-    named_barrier_sync(kI8PieceBarrier, kI8Rows);
+    named_barrier_sync(kI8PieceBarrier, nthreads);
     if (!*last_flag) return;
     // Every CTA after c_first starts inside tile t (its piece is slot 0);
     // c_first's piece is slot 0 only if its range starts at the tile.
     const int first_slot = i8_item_begin(items, c_first, gridDim.x) < tf0 ? 1 : 0;
-    double tot = 0.0;
-    // four pieces per round: their loads are independent and in flight together
-    for (int c0 = c_first; c0 <= c_last; c0 += 4) {
-        double val[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = c0 + j;
-            const int cs = c == c_first ? first_slot : 0;
-            val[j] = c <= c_last ? __ldcg(part + (static_cast<size_t>(c) * 2 + cs) * kI8Rows + row) : 0.0;
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) tot += val[j];   // pieces added in CTA order
-    }
     const int grow = t * kI8Rows + row;
-    if (grow < n) y[grow] = static_cast<float>(tot);
+    for (int v = v0; v < v1; v += vstep) {
+        double tot = 0.0;
+        // four pieces per round: their loads are independent and in flight together
+        for (int c0 = c_first; c0 <= c_last; c0 += 4) {
+            double val[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = c0 + j;
+                const int cs = c == c_first ? first_slot : 0;
+                val[j] = c <= c_last ? __ldcg(part + ((static_cast<size_t>(c) * 2 + cs) * mv + v) * kI8Rows + row)
+                                     : 0.0;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tot += val[j];   // pieces added in CTA order
+        }
+        if (grow < n) y[static_cast<size_t>(v) * n + grow] = static_cast<float>(tot);
+    }
 }
 
 // The epilogue's sum for one row and one superblock column over sub-blocks
@@ -293,7 +391,7 @@ __device__ __forceinline__ double i8_column_sum(const uint32_t* r, const Header&
 #pragma unroll
     for (int jj = 0; jj < NJ; ++jj) {
         const int j = j0 + jj;
-        const uint32_t* rj = r + jj * kI8Limbs;
+        const uint32_t* rj = r + jj * i8_limbs(1);
         const int D0 = static_cast<int>(rj[0]), D1 = static_cast<int>(rj[1]);
         const int D2 = static_cast<int>(rj[2]), D3 = static_cast<int>(rj[3]);
         const int D4 = static_cast<int>(rj[4]);
@@ -317,11 +415,59 @@ __device__ __forceinline__ double i8_column_sum(const uint32_t* r, const Header&
     return fma(dd, static_cast<double>(S), -(dm * (ma + mc)));
 }
 
-template <int WS, int CPI>
+// The same for one of MV >= 2 vectors and one superblock column, digits in
+// base 256, in two steps of four sub-blocks: i8_b256_add takes D_j[l] of
+// sub-blocks j0 .. j0+3 from r[4 (j - j0) + l] into P_l = sum_j sc_j D_j[l]
+// (even and odd sub-blocks summed apart: |even| <= 4 * 63 * 32 * 15 * 128 <
+// 2^24, |odd| sixteen times that, < 2^28, a multiple of 16) and M = 2^18
+// sum_j m_j h_j + sum_j m_j l_j (each sum within 32 bits: |h_j| < 2^17), with
+// mb the vector's metadata (mb[0] = 2^(E-30); from byte 16 S0_j = 2^18 h_j +
+// l_j as int pairs (l_j, h_j), l_j in [0, 2^18)); i8_b256_sum returns
+// d * S - dmin * M with S = sum_l 256^l P_l (|S| < 2^50).
+struct I8B256Acc {
+    int pe[4], po[4], ml, mh;
+};
+
+__device__ __forceinline__ void i8_b256_add(I8B256Acc& acc, const uint32_t* r, const Header& hd, const double* mb,
+                                            int j0) {
+    const int4* s0 = reinterpret_cast<const int4*>(mb + 2);   // (l_0, h_0, l_1, h_1), ...
+    const uint32_t scw = j0 == 0 ? hd.sc_lo : hd.sc_hi, mw = j0 == 0 ? hd.m_lo : hd.m_hi;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+        const int sc = static_cast<int>(byte_of(scw, jj));
+#pragma unroll
+        for (int l = 0; l < 4; ++l) {
+            if (jj & 1) acc.po[l] += sc * static_cast<int>(r[4 * jj + l]);
+            else acc.pe[l] += sc * static_cast<int>(r[4 * jj + l]);
+        }
+        const int4 q = s0[(j0 + jj) >> 1];
+        const int mj = static_cast<int>(byte_of(mw, jj));
+        acc.ml += mj * ((jj & 1) ? q.z : q.x);
+        acc.mh += mj * ((jj & 1) ? q.w : q.y);
+    }
+}
+
+__device__ __forceinline__ double i8_b256_sum(const I8B256Acc& acc, const Header& hd) {
+    long long S = 0;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) S += static_cast<long long>(acc.pe[l] + (acc.po[l] >> 4)) << (8 * l);
+    const long long M = (static_cast<long long>(acc.mh) << 18) + acc.ml;
+    const double dd = hd.d, dm = hd.dmin;
+    return fma(dd, static_cast<double>(S), -(dm * static_cast<double>(M)));
+}
+
+template <int WS, int CPI, int MV>
 __global__ void __launch_bounds__(kI8Threads, 1)
 q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) {
-    constexpr uint32_t kIdesc = mma_i8_idesc(kI8Rows, kI8N);
-    constexpr int kBufs = i8_bufs(CPI);               // A buffers = accumulators
+    constexpr int kN = i8_n(MV);                      // MMA N: digit rows
+    constexpr uint32_t kIdesc = mma_i8_idesc(kI8Rows, kN);
+    constexpr int kBufs = i8_bufs(CPI, MV);           // A buffers = accumulators
+    constexpr int kDcol0 = i8_dcol0(CPI, MV);         // first accumulator column
+    constexpr int kColAcc = i8_col_acc(MV);           // accumulator columns of one superblock column
+    constexpr int kImage = i8_image_bytes(MV);
+    constexpr int kMeta = i8_meta_doubles(MV);
+    static_assert((MV == 1 || MV == 2 || MV == 4) && (MV != 4 || CPI == 1), "vectors per launch");
+    static_assert(kDcol0 + kBufs * CPI * kColAcc <= kI8TmemCols && kBufs <= 4, "TMEM buffers");
     constexpr int kHSlots = kI8HSlotCols / CPI;       // header ring slots (items)
     constexpr int kStage = CPI * kI8RawBytes;         // one weight stage
     // Item it uses A buffer and accumulator it % kBufs: one commit per item
@@ -333,10 +479,10 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int nsb = p.nsb, npi = p.npi;
     const int pnsb = npi * CPI;                                   // columns per tile, padded
-    uint8_t* image = smem;                                        // [ncols][kI8ImageBytes]
-    double* meta = reinterpret_cast<double*>(smem + p.ncols * kI8ImageBytes);   // [ncols][10]
-    uint4* hring = reinterpret_cast<uint4*>(meta + p.ncols * kI8MetaDoubles);    // [slot][CPI][128]
-    uint8_t* wring = smem + i8_wring_offset(p.ncols);             // [WS][128 rows][CPI][144]
+    uint8_t* image = smem;                                        // [ncols][kImage]
+    double* meta = reinterpret_cast<double*>(smem + p.ncols * kImage);   // [ncols][MV][10]
+    uint4* hring = reinterpret_cast<uint4*>(meta + p.ncols * kMeta);      // [slot][CPI][128]
+    uint8_t* wring = smem + i8_wring_offset(p.ncols, MV);         // [WS][128 rows][CPI][144]
     uint64_t* wfull = reinterpret_cast<uint64_t*>(wring + WS * kStage);
     uint64_t* wempty = wfull + kI8MaxWStages;
     uint64_t* afull = wempty + kI8MaxWStages;  // decoded A in TMEM buffer
@@ -347,7 +493,7 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     uint64_t* mma_done = hfree + kI8HSlotCols;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     __shared__ volatile int abort_flag;
-    __shared__ double xchange[2 * kI8Rows];   // epilogue: half 1's row totals, by piece parity
+    __shared__ double xchange[MV == 1 ? 2 * kI8Rows : 1];   // one vector's epilogue: half 1's totals, by piece parity
     __shared__ int last_piece[2];
 
     const int warp = threadIdx.x >> 5;
@@ -417,7 +563,13 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     __syncwarp();
 
     pdl_wait();   // x is produced, and y may be read, by the preceding work on the stream
-    i8_digits(p.x, nsb, pnsb, pb_first, count * CPI < pnsb ? count * CPI : pnsb, image, meta, warp, kI8Warps, lane);
+    {
+        const int ncols_used = count * CPI < pnsb ? count * CPI : pnsb;
+        if constexpr (MV == 1)
+            i8_digits(p.x, nsb, pnsb, pb_first, ncols_used, image, meta, warp, kI8Warps, lane);
+        else
+            i8_digits_mv<MV>(p.x, p.m, p.k, nsb, pnsb, pb_first, ncols_used, image, meta, warp, kI8Warps, lane);
+    }
     fence_proxy_async_smem();   // the image is read by the MMAs
     __syncthreads();
 
@@ -436,7 +588,7 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         // The warp runs converged and one elected lane issues the MMAs and
         // commits: sub-block j of column c of the item is one MMA, A from TMEM
         // columns 64c + 8j .. +7 of the buffer, B = the column's digit rows at
-        // K 32j, the accumulator columns 64c + 8j .. +7 (no accumulation
+        // K 32j, the accumulator columns 8N c + N j .. +N-1 (no accumulation
         // across MMAs).
         int i = i00;
         for (int it = 0; it < count; ++it, i = (i + 1 == npi) ? 0 : i + 1) {
@@ -448,20 +600,20 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                 break;
             }
             tc_fence_after_sync();
-            const uint32_t dcol = tmem + static_cast<uint32_t>(kI8Dcol0 + a * CPI * kI8ColAcc);
+            const uint32_t dcol = tmem + static_cast<uint32_t>(kDcol0 + a * CPI * kColAcc);
             const uint32_t acol = tmem + static_cast<uint32_t>(a * CPI * kI8ColTmem);
             if (elect_one()) {
 #pragma unroll
                 for (int c = 0; c < CPI; ++c) {
                     const int pb = i * CPI + c;
                     if (pb >= nsb) continue;   // past the row: no MMA, the epilogue skips it
-                    const uint32_t img = smem_addr(image + static_cast<size_t>(slot_of(pb)) * kI8ImageBytes);
+                    const uint32_t img = smem_addr(image + static_cast<size_t>(slot_of(pb)) * kImage);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         // K position 32j: atom j / 4 (N * 128 bytes each), 32 bytes
                         // per MMA inside it
-                        const uint64_t bdesc = sw128_kmajor_desc(img + (j >> 2) * (kI8N * 128) + (j & 3) * 32);
-                        mma_i8_tmem_a(dcol + static_cast<uint32_t>(c * kI8ColAcc + j * kI8N),
+                        const uint64_t bdesc = sw128_kmajor_desc(img + (j >> 2) * (kN * 128) + (j & 3) * 32);
+                        mma_i8_tmem_a(dcol + static_cast<uint32_t>(c * kColAcc + j * kN),
                                       acol + static_cast<uint32_t>(c * kI8ColTmem + 8 * j), bdesc, kIdesc, 0u);
                     }
                 }
@@ -532,17 +684,34 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        // Two warps per lane quarter share each item: with two columns per
-        // item half h takes column h, with one half h takes sub-blocks 4h ..
-        // 4h+3. Each keeps its own f64 row total; at the end of a piece (the
-        // CTA's part of a tile) half 1 hands its total to half 0 (shared
-        // memory, a named barrier per quarter), which adds the two in that
-        // order and stores y or the piece.
+        // Two warps per lane quarter. One vector: they share each item (with
+        // two columns per item half h takes column h, with one half h takes
+        // sub-blocks 4h .. 4h+3), each keeping its own f64 row total; at the
+        // end of a piece (the CTA's part of a tile) half 1 hands its total to
+        // half 0 (shared memory, a named barrier per quarter), which adds the
+        // two in that order and stores y or the piece. MV >= 2 vectors: half h
+        // takes vectors h, h + 2 of its lane quarter in every column of the
+        // item, one group (column, vector) after the other, and keeps and
+        // stores those vectors' row totals.
         const int quarter = warp % kI8Quarters;
-        const int half = (warp - kI8DecodeWarps) / kI8Quarters;
+        const int eg = (warp - kI8DecodeWarps) / kI8Quarters;   // half (one vector) or first vector
+        constexpr int kVW = MV == 1 ? 1 : MV / 2;   // vectors this warp sums: eg + kVStep * vv
+        constexpr int kVStep = 2;
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
-        double ytot = 0.0;
+        // a piece of tile t is published by half 0 (one vector: every vector's
+        // row total is there) or by every epilogue warp (its vector)
+        auto publish = [&](int t, int* flag) {
+            if constexpr (MV == 1)
+                i8_publish_piece(p.part, p.done, p.y, p.n, 1, 0, p.m, 1, npi, items, t, row, row == 0, kI8Rows, flag,
+                                 abort_flag != 0);
+            else
+                i8_publish_piece(p.part, p.done, p.y, p.n, MV, eg, p.m, kVStep, npi, items, t, row,
+                                 row == 0 && eg == 0, 32 * kI8EpiWarps, flag, abort_flag != 0);
+        };
+        double ytot[kVW];
+#pragma unroll
+        for (int vv = 0; vv < kVW; ++vv) ytot[vv] = 0.0;
         int tile = tile0, i = i00;
         int istart = i;                    // first item of the current piece
         bool has1 = false;                 // a cut piece left to publish after the last item
@@ -553,19 +722,22 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
             const int a = it % kBufs, hs = it % kHSlots;
             const bool ok = !abort_flag && i8_wait(&dfull[a], static_cast<uint32_t>((it / kBufs) & 1)) &&
                             i8_wait(&hfull[hs], static_cast<uint32_t>((it / kHSlots) & 1));
-            if (__all_sync(0xFFFFFFFFu, ok)) {
-                const int c = CPI == 2 ? half : 0;   // the item's column this half reads
+            if (!__all_sync(0xFFFFFFFFu, ok)) {
+                abort_flag = 1;
+            } else if constexpr (MV == 1) {
+                const int c = CPI == 2 ? eg : 0;   // the item's column this half reads
                 // this row's superblock header (d, dmin, sc_j, m_j)
                 const uint4 hraw = hring[(hs * CPI + c) * kI8Rows + row];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&hfree[hs]);
                 tc_fence_after_sync();
                 constexpr int kNJ = CPI == 2 ? 8 : 4;   // sub-blocks this half sums
-                uint32_t r[kNJ * kI8Limbs];            // D_j[l] at (j - j0) * 5 + l: the digit columns only
-                const uint32_t dcol = lane_base + static_cast<uint32_t>(kI8Dcol0 + a * CPI * kI8ColAcc +
-                                                                        (CPI == 2 ? c * kI8ColAcc : 32 * half));
+                constexpr int kL = i8_limbs(1);
+                uint32_t r[kNJ * kL];                   // D_j[l] at (j - j0) * 5 + l: the digit columns only
+                const uint32_t dcol = lane_base + static_cast<uint32_t>(kDcol0 + a * CPI * kColAcc +
+                                                                        (CPI == 2 ? c * kColAcc : 32 * eg));
 #pragma unroll
-                for (int jj = 0; jj < kNJ; ++jj) tmem_load_5cols(dcol + static_cast<uint32_t>(jj * kI8N), r + jj * kI8Limbs);
+                for (int jj = 0; jj < kNJ; ++jj) tmem_load_5cols(dcol + static_cast<uint32_t>(jj * kN), r + jj * kL);
                 tmem_wait_ld();
                 tc_fence_before_sync();
                 __syncwarp();
@@ -573,39 +745,89 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                 const int pb = i * CPI + c;
                 if (pb < nsb) {   // a column past the row (odd K/256, two columns per item) adds nothing
                     const Header hd = decode_header(hraw);
-                    const double* mb = meta + static_cast<size_t>(slot_of(pb)) * kI8MetaDoubles;
+                    const double* mb = meta + static_cast<size_t>(slot_of(pb)) * kMeta;
                     double part;
                     if constexpr (CPI == 2) part = i8_column_sum<8>(r, hd, mb, 0);
-                    else part = i8_column_sum<4>(r, hd, mb, 4 * half);
-                    ytot = fma(mb[0], part, ytot);
+                    else part = i8_column_sum<4>(r, hd, mb, 4 * eg);
+                    ytot[0] = fma(mb[0], part, ytot[0]);
                 }
             } else {
-                abort_flag = 1;
+                uint4 hraw[CPI];   // this row's headers of the item's columns
+#pragma unroll
+                for (int c = 0; c < CPI; ++c) hraw[c] = hring[(hs * CPI + c) * kI8Rows + row];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&hfree[hs]);
+                tc_fence_after_sync();
+                // (column, vector) groups, one after the other
+#pragma unroll
+                for (int g = 0; g < CPI * kVW; ++g) {
+                    const int c = g / kVW, vv = g % kVW, vec = eg + kVStep * vv;
+                    const int pb = i * CPI + c;
+                    // warp-uniform: a column past the row or a vector past m adds nothing
+                    const bool use = pb < nsb && vec < p.m;
+                    uint32_t r[32];   // D_j[l] of this vector at 4 j + l
+                    if (use) {
+                        const uint32_t dcol = lane_base + static_cast<uint32_t>(kDcol0 + (a * CPI + c) * kColAcc +
+                                                                                4 * vec);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) tmem_load_4cols_at(dcol + static_cast<uint32_t>(j * kN), r + 4 * j);
+                    }
+                    tmem_wait_ld();
+                    if (g == CPI * kVW - 1) {   // the item's accumulator is read
+                        tc_fence_before_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&dfree[a]);
+                    }
+                    if (use) {
+                        const Header hd = decode_header(hraw[c]);
+                        const double* mb = meta + static_cast<size_t>(slot_of(pb)) * kMeta + kI8VecMeta * vec;
+                        I8B256Acc acc{{0, 0, 0, 0}, {0, 0, 0, 0}, 0, 0};
+                        i8_b256_add(acc, r, hd, mb, 0);
+                        i8_b256_add(acc, r + 16, hd, mb, 4);
+                        ytot[vv] = fma(mb[0], i8_b256_sum(acc, hd), ytot[vv]);
+                    }
+                }
             }
             if (i == npi - 1 || it == count - 1) {
-                // end of this CTA's piece of `tile`: the halves' totals, added
-                double* xc = xchange + parity * kI8Rows;
-                if (half == 1) xc[row] = ytot;
-                named_barrier_sync(1 + quarter, 64);
-                if (half == 0) {
-                    const double tot = ytot + xc[row];
+                // end of this CTA's piece of `tile`
+                bool store = true;   // this thread holds totals to store
+                double tot[kVW];
+#pragma unroll
+                for (int vv = 0; vv < kVW; ++vv) tot[vv] = ytot[vv];
+                if constexpr (MV == 1) {   // the halves' totals, added
+                    double* xc = xchange + parity * kI8Rows;
+                    if (eg == 1) xc[row] = ytot[0];
+                    named_barrier_sync(1 + quarter, 64);
+                    store = eg == 0;
+                    if (store) tot[0] = ytot[0] + xc[row];
+                }
+                if (store) {
                     if (istart == 0 && i == npi - 1) {   // the whole tile
-                        if (!abort_flag && grow < p.n) p.y[grow] = static_cast<float>(tot);
+#pragma unroll
+                        for (int vv = 0; vv < kVW; ++vv) {
+                            const int vec = MV == 1 ? 0 : eg + kVStep * vv;
+                            if (!abort_flag && grow < p.n && vec < p.m)
+                                p.y[static_cast<size_t>(vec) * p.n + grow] = static_cast<float>(tot[vv]);
+                        }
                     } else {
                         // a piece: slot 0 is published at once (the rest of
                         // the range follows), slot 1 after the last item
                         const int slot = tile == tile0 ? 0 : 1;
-                        p.part[(static_cast<size_t>(blockIdx.x) * 2 + slot) * kI8Rows + row] = tot;
+#pragma unroll
+                        for (int vv = 0; vv < kVW; ++vv) {
+                            const int vec = MV == 1 ? 0 : eg + kVStep * vv;
+                            p.part[((static_cast<size_t>(blockIdx.x) * 2 + slot) * MV + vec) * kI8Rows + row] = tot[vv];
+                        }
                         if (slot == 0 && it < count - 1) {
-                            i8_publish_piece(p.part, p.done, p.y, p.n, npi, items, tile, row, &last_piece[0],
-                                             abort_flag != 0);
+                            publish(tile, &last_piece[0]);
                         } else {
                             has1 = true;
                             tile1 = tile;
                         }
                     }
                 }
-                ytot = 0.0;
+#pragma unroll
+                for (int vv = 0; vv < kVW; ++vv) ytot[vv] = 0.0;
                 istart = 0;
                 parity ^= 1;
             }
@@ -614,10 +836,9 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
                 ++tile;
             }
         }
-        // every thread of the first half takes this branch or none (the
-        // pieces depend only on the CTA's range)
-        if (half == 0 && has1)
-            i8_publish_piece(p.part, p.done, p.y, p.n, npi, items, tile1, row, &last_piece[1], abort_flag != 0);
+        // every publishing thread takes this branch or none (the pieces
+        // depend only on the CTA's range)
+        if (has1) publish(tile1, &last_piece[1]);
     }
 
     tc_fence_before_sync();
@@ -639,7 +860,8 @@ bool i8_whole_tiles(int tiles, int num_sms) {
 int i8_threads() { return kI8Threads; }
 
 bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg) {
-    if (m != 1 || n < 1 || k < kQK || k % kQK != 0 || num_sms < 1) return false;
+    if (m < 1 || m > kI8MaxM || n < 1 || k < kQK || k % kQK != 0 || num_sms < 1) return false;
+    const int mv = m == 1 ? 1 : m == 2 ? 2 : 4;
     const int nsb = k / kQK;
     const long long tiles = (static_cast<long long>(n) + kI8Rows - 1) / kI8Rows;
     if (tiles * nsb >= (1LL << 31) / num_sms) return false;   // item counts in 32 bits
@@ -649,9 +871,11 @@ bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg) {
     if (!whole && tiles * nsb < static_cast<long long>(kI8MinItemsPerCta) * num_sms) return false;
     const int budget = max_smem < kI8SmemBudget ? max_smem : kI8SmemBudget;
     // two columns per item unless an odd K/256 is small (the padded column of
-    // each tile's last item would be a large share of the work)
-    for (int cpi = (nsb % 2 == 0 || nsb >= 9) ? 2 : 1; cpi >= 1; --cpi) {
+    // each tile's last item would be a large share of the work) or four
+    // vectors' accumulators leave tensor memory for one column only
+    for (int cpi = mv < 4 && (nsb % 2 == 0 || nsb >= 9) ? 2 : 1; cpi >= 1; --cpi) {
         I8Config c;
+        c.mv = mv;
         c.cpi = cpi;
         c.npi = (nsb + cpi - 1) / cpi;
         c.items = tiles * c.npi;
@@ -660,11 +884,11 @@ bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg) {
         c.items_per_cta_max = whole ? (tiles + c.ctas - 1) / c.ctas * c.npi : (c.items + c.ctas - 1) / c.ctas;
         const long long pnsb = static_cast<long long>(c.npi) * cpi;
         c.ncols = static_cast<int>(c.items_per_cta_max * cpi < pnsb ? c.items_per_cta_max * cpi : pnsb);
-        const int fit = i8_fit_stages(c.ncols, cpi);
+        const int fit = i8_fit_stages(c.ncols, cpi, mv);
         // the kernel's instantiations: 4 two-column stages; 8, 6 or 4 one-column
         if (fit < kI8MinWStages) continue;
         c.wstages = cpi == 2 ? 4 : fit >= 8 ? 8 : fit >= 6 ? 6 : 4;
-        c.smem = i8_smem_bytes_cfg(c.ncols, cpi, c.wstages);
+        c.smem = i8_smem_bytes_cfg(c.ncols, cpi, c.wstages, mv);
         if (c.smem > budget) continue;
         c.cuts = 0;
         if (!whole)
@@ -680,8 +904,9 @@ namespace {
 
 // Scratch for tiles cut between CTAs, one per (device, stream): the per-tile
 // counters (zeroed once; every launch leaves them zero, the last publisher of a
-// tile resetting its counter) and the pieces, [SMs][2][128] f64. Calls on one
-// stream run in order, so a stream's calls never share it concurrently.
+// tile resetting its counter) and the pieces, [SMs][2][up to 4 vectors][128]
+// f64. Calls on one stream run in order, so a stream's calls never share it
+// concurrently.
 struct I8Scratch {
     void* ptr = nullptr;
     int tiles_cap = 0;
@@ -692,8 +917,10 @@ std::map<std::pair<int, uintptr_t>, I8Scratch> g_i8_scratch;
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
-// Counters then pieces: the pieces' offset for a region of `tiles` counters.
+// Counters then pieces: the pieces' offset for a region of `tiles` counters,
+// the pieces' bytes for `ctas` CTAs.
 size_t scratch_part_offset(int tiles) { return align256(static_cast<size_t>(tiles) * sizeof(unsigned)); }
+size_t scratch_part_bytes(int ctas) { return static_cast<size_t>(ctas) * 2 * kI8MaxM * kI8Rows * sizeof(double); }
 
 // The stream's scratch for `tiles` tiles and `ctas` CTAs, (re)allocated in
 // stream order if missing or too small; *done stays null if the stream is
@@ -712,8 +939,7 @@ cudaError_t stream_scratch(int device, cudaStream_t stream, int tiles, int ctas,
         const int tcap = tiles > 4096 ? tiles : 4096;
         const int ccap = ctas > 256 ? ctas : 256;
         void* p = nullptr;
-        e = cudaMallocAsync(&p, scratch_part_offset(tcap) + static_cast<size_t>(ccap) * 2 * kI8Rows * sizeof(double),
-                            stream);
+        e = cudaMallocAsync(&p, scratch_part_offset(tcap) + scratch_part_bytes(ccap), stream);
         if (e != cudaSuccess) return e;
         e = cudaMemsetAsync(p, 0, static_cast<size_t>(tcap) * sizeof(unsigned), stream);
         if (e != cudaSuccess) return e;
@@ -729,16 +955,20 @@ cudaError_t stream_scratch(int device, cudaStream_t stream, int tiles, int ctas,
 
 }  // namespace
 
+template <int WS, int CPI, int MV>
+cudaError_t i8_set_attribute() {
+    return cudaFuncSetAttribute(q4k_gemv_i8_kernel<WS, CPI, MV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kI8SmemBudget);
+}
+
 int i8_set_attributes() {
-    cudaError_t e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<8, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kI8SmemBudget);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<6, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(q4k_gemv_i8_kernel<4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kI8SmemBudget);
-    return e == cudaSuccess ? Q4K_OK : cuda_failure(e);
+    const cudaError_t es[] = {i8_set_attribute<8, 1, 1>(), i8_set_attribute<6, 1, 1>(), i8_set_attribute<4, 1, 1>(),
+                              i8_set_attribute<4, 2, 1>(), i8_set_attribute<8, 1, 2>(), i8_set_attribute<6, 1, 2>(),
+                              i8_set_attribute<4, 1, 2>(), i8_set_attribute<4, 2, 2>(), i8_set_attribute<8, 1, 4>(),
+                              i8_set_attribute<6, 1, 4>(), i8_set_attribute<4, 1, 4>()};
+    for (const cudaError_t e : es)
+        if (e != cudaSuccess) return cuda_failure(e);
+    return Q4K_OK;
 }
 
 namespace {
@@ -774,10 +1004,26 @@ bool make_weight_map3(CUtensorMap* map, const void* w, int n, int nsb, int cpi) 
 
 }  // namespace
 
-int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int n, int k,
+namespace {
+
+// The kernel's instantiation for a launch shape (the ones i8_config picks).
+template <int MV>
+cudaError_t launch_i8_mv(const cudaLaunchConfig_t& cfg, const I8Config& c, const CUtensorMap& map,
+                         const I8Params& ip) {
+    if constexpr (MV < 4) {
+        if (c.cpi == 2) return cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 2, MV>, map, ip);
+    }
+    return c.wstages >= 8 ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8, 1, MV>, map, ip)
+         : c.wstages >= 6 ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6, 1, MV>, map, ip)
+                          : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 1, MV>, map, ip);
+}
+
+}  // namespace
+
+int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n, int k,
                    cudaStream_t stream) {
     I8Config c;
-    if (!i8_config(1, n, k, dev.sm_count, dev.max_smem_optin, &c)) return Q4K_ERR_SHAPE;   // not reached
+    if (!i8_config(m, n, k, dev.sm_count, dev.max_smem_optin, &c)) return Q4K_ERR_SHAPE;   // not reached
     const int nsb = k / kQK;
     const int tiles = (n + kI8Rows - 1) / kI8Rows;
     CUtensorMap map;
@@ -794,15 +1040,14 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
         e = cudaGetDevice(&device);
         if (e == cudaSuccess) e = stream_scratch(device, stream, tiles, c.ctas, &done, &part);
         if (e == cudaSuccess && done == nullptr) {
-            e = cudaMallocAsync(&own, scratch_part_offset(tiles) + static_cast<size_t>(c.ctas) * 2 * kI8Rows * sizeof(double),
-                                stream);
+            e = cudaMallocAsync(&own, scratch_part_offset(tiles) + scratch_part_bytes(c.ctas), stream);
             if (e == cudaSuccess) e = cudaMemsetAsync(own, 0, static_cast<size_t>(tiles) * sizeof(unsigned), stream);
             done = static_cast<unsigned*>(own);
             part = reinterpret_cast<double*>(static_cast<uint8_t*>(own) + scratch_part_offset(tiles));
         }
         if (e != cudaSuccess) return cuda_failure(e);
     }
-    const I8Params ip{x, y, part, done, n, nsb, tiles, c.npi, c.ncols, c.whole};
+    const I8Params ip{x, y, part, done, m, n, k, nsb, tiles, c.npi, c.ncols, c.whole};
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(c.ctas));
     cfg.blockDim = dim3(kI8Threads);
@@ -813,10 +1058,9 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = c.cpi == 2          ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 2>, map, ip)
-        : c.wstages >= 8    ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<8, 1>, map, ip)
-        : c.wstages >= 6    ? cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<6, 1>, map, ip)
-                            : cudaLaunchKernelEx(&cfg, q4k_gemv_i8_kernel<4, 1>, map, ip);
+    e = c.mv == 1 ? launch_i8_mv<1>(cfg, c, map, ip)
+      : c.mv == 2 ? launch_i8_mv<2>(cfg, c, map, ip)
+                  : launch_i8_mv<4>(cfg, c, map, ip);
     if (own != nullptr) {
         const cudaError_t ef = cudaFreeAsync(own, stream);
         if (e == cudaSuccess) e = ef;

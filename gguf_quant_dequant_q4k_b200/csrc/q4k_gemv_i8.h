@@ -1,5 +1,5 @@
-// q4k_gemv_i8.h -- host-side interface of the one-vector tensor-core GEMV for
-// tall matrices (q4k_gemv_i8.cu): when it applies, its launch sizes.
+// q4k_gemv_i8.h -- host-side interface of the integer tensor-core GEMV for
+// one to four vectors (q4k_gemv_i8.cu): when it applies, its launch sizes.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -9,6 +9,7 @@ namespace q4k {
 struct DeviceInfo;
 
 constexpr int kI8Rows = 128;      // rows per tile: the MMA's M
+constexpr int kI8MaxM = 4;        // vectors per launch (1, 2, or 3-4 as four)
 constexpr int kI8MaxWStages = 8;  // weight stages: 8, 6 or 4 of one superblock column of a tile,
 constexpr int kI8MinWStages = 4;  // or 4 of two, as many as fit beside the digit image
 constexpr int kI8PreStages = 2;   // weight stages requested before the dependency wait
@@ -18,7 +19,8 @@ constexpr int kI8MinItemsPerCta = 5; // cut tiles: at least this many items per 
 
 // One call's launch shape on the kernel.
 struct I8Config {
-    int cpi;                      // superblock columns per item (1 or 2)
+    int mv;                       // vectors the kernel is built for: 1, 2 or 4 (m = 3 as four)
+    int cpi;                      // superblock columns per item (1 or 2; 1 for four vectors)
     int npi;                      // items per tile: ceil(nsb / cpi)
     int ncols;                    // digit-image slots a CTA keeps (its columns, padded)
     int wstages;                  // weight stages of cpi columns
@@ -34,14 +36,14 @@ struct I8Config {
 // at most 1/kI8MaxImbalance above the mean.
 bool i8_whole_tiles(int tiles, int num_sms);
 int i8_threads();
-// True (and *cfg filled) if q4k_gemv runs one vector of this shape on the
-// kernel: whole tiles per CTA or at least kI8MinItemsPerCta superblock columns
-// per CTA on average, and the CTA's digit image beside at least four weight
-// stages (two columns per item where that fits, else one).
+// True (and *cfg filled) if q4k_gemv runs m <= kI8MaxM vectors of this shape
+// on the kernel: whole tiles per CTA or at least kI8MinItemsPerCta superblock
+// columns per CTA on average, and the CTA's digit image beside at least four
+// weight stages (two columns per item where that fits, else one).
 bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg);
 
 int i8_set_attributes();
-int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int n, int k,
+int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n, int k,
                    cudaStream_t stream);
 int read_i8_fault_flags(unsigned* flags);
 

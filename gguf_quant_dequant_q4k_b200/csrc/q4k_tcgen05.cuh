@@ -139,6 +139,14 @@ __device__ __forceinline__ void tmem_load_8cols(uint32_t taddr, uint32_t (&r)[8]
                  : "memory");
 }
 
+// 4 consecutive TMEM columns into r[0..3] (valid after tmem_wait_ld()).
+__device__ __forceinline__ void tmem_load_4cols_at(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+}
+
 // 5 consecutive TMEM columns of the calling thread's lane (an x4 and an x1
 // load); the registers are valid after tmem_wait_ld().
 __device__ __forceinline__ void tmem_load_5cols(uint32_t taddr, uint32_t* r) {

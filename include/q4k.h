@@ -94,28 +94,31 @@ enum q4k_status {
  *        ("input: M x K row-major", `batched_q4k_gemv_into`).
  *   y  : m x N float32, row-major (vector i at y + i*N); fully overwritten,
  *        never accumulated into ("output: M x N row-major").
- *   m  : 1..64 vectors. One vector runs on the integer tensor-core kernel
- *        (Q4K_KERNEL_I8, one launch) where K <= 256*62 and the matrix gives
- *        every SM whole 128-row tiles or at least 5 (tile, superblock column)
- *        items, else, like two vectors, on the streaming kernel (one launch,
- *        or K-chunks of it for long K). Three or more run on the
- *        tensor-core kernel in groups of up to 16 (the realizar page tiles
+ *   m  : 1..64 vectors. One to four vectors run on the integer tensor-core
+ *        kernel (Q4K_KERNEL_I8, one launch, the weights decoded once for all
+ *        of them; m = 3 as four) where the matrix gives every SM whole
+ *        128-row tiles or at least 5 (tile, superblock column) items and the
+ *        CTA's digit image fits beside four weight stages (one vector:
+ *        K <= 256*62); otherwise one or two vectors run on the streaming
+ *        kernel (one launch, or K-chunks of it for long K), and three or more
+ *        on the tensor-core kernel in groups of up to 16 (the realizar page tiles
  *        m > 8 in `batched_q4k_gemv_into` and has an m = 16 / 32 branch): each
  *        group is a digits launch and a GEMV launch, the weights decoded once
  *        per group. q4k_gemv_plan_for reports the launch count. Larger m is
  *        refused, not looped (the turbospark page, "turbospark-runtime 0.1.0,
  *        src/real_forward_dispatch.rs", `encode_gemm_any`, refuses rather than
  *        silently looping): that is a GEMM's size.
- * Workspace: for m >= 3 the call allocates a device workspace from the
+ * Workspace: for m >= 3 on the tensor-core kernel the call allocates a
+ * device workspace from the
  * device's default memory pool, stream-ordered on `stream`
  * (cudaMallocAsync / cudaFreeAsync; capturable in a CUDA graph), of
  * (K/256) * (N_mma*512 + 80*mp) + 2048*mp*ctas + 4*ceil(N/128) bytes
  * (mp = 8 or 16, N_mma = 48 or 80, ctas <= SM count): 2.7 MiB for
  * N = 14336, K = 4096, m = 8. m = 2, and m = 1 on the streaming kernel,
- * allocate nothing. m = 1 on the integer kernel with tiles cut between CTAs
+ * allocate nothing. The integer kernel with tiles cut between CTAs
  * (q4k_gemv_plan_for: kernel Q4K_KERNEL_I8, units not a multiple of the CTAs'
  * whole-tile ranges) uses a scratch the library keeps per (device, stream):
- * ceil(4*max(tiles, 4096), 256) + 2048*max(ctas, 256) bytes, allocated
+ * ceil(4*max(tiles, 4096), 256) + 8192*max(ctas, 256) bytes, allocated
  * stream-ordered on the first such call on `stream` outside graph capture
  * (inside a capture with none yet, the call allocates and frees its own,
  * capturable) and kept for the process; every launch leaves its counters
@@ -125,12 +128,13 @@ enum q4k_status {
  * q4k_gemv calls on that stream.
  * Accuracy: per element |y - sum_k w_nk x_ik| <= 1e-4 * sum_k |w_nk x_ik| + 1e-6,
  * where w_nk is the f32 value d*sc*q - dmin*m; for m <= 2 accumulation is in
- * f32. For m >= 3, and m = 1 on the integer kernel, the products are exact
- * integers (x scaled per 256-element
- * block by 2^(33 - E), E the exponent of the block's largest |x|, and
- * rounded to an integer) combined in f64, so the bound holds with one more
- * term, 2^-33 * sum_k |w_nk| * max_block(k) |x_i|, which is below 1e-6 unless
- * that sum exceeds 8590 (e.g. K = 14336 and |x| up to ~1 with most of w x
+ * f32 on the streaming kernel. On the tensor-core and integer kernels the
+ * products are exact integers (x scaled per 256-element block by 2^(33 - E)
+ * (2^(30 - E) for two to four vectors on the integer kernel), E the exponent
+ * of the block's largest |x|, and rounded to an integer) combined in f64, so
+ * the bound holds with one more term, 2^-33 * sum_k |w_nk| * max_block(k)
+ * |x_i| (2^-30 * ... for those), which is below 1e-6 unless that sum
+ * exceeds 8590 (1074) (e.g. K = 14336 and |x| up to ~1 with most of w x
  * cancelling); an inf or NaN in x_i makes every element of y_i NaN.
  * Weight reads may start before the previous kernel on `stream` has finished
  * (programmatic dependent launch): x is read and y written only after it has.
@@ -293,12 +297,15 @@ enum q4k_kernel {
                                    counts (128-row tile, superblock column)
                                    items, shared out in equal contiguous ranges;
                                    `depth` is the weight-ring depth             */
-    Q4K_KERNEL_I8 = 4           /* m = 1, K <= 256 * 62, and whole 128-row
-                                   tiles for every SM (the busiest SM at most
-                                   1/8 above the mean) or >= 5 items per SM:
-                                   tcgen05 kind::i8, the quant nibbles times
-                                   base-128 digits of the scaled x, exact
-                                   integer products; one launch; `units` counts
+    Q4K_KERNEL_I8 = 4           /* m <= 4, the digit image beside four weight
+                                   stages (m = 1: K <= 256 * 62), and whole
+                                   128-row tiles for every SM (the busiest SM
+                                   at most 1/8 above the mean) or >= 5 items
+                                   per SM: tcgen05 kind::i8, the quant nibbles
+                                   times base-128 (m = 1) or base-256 digits
+                                   of the scaled x, exact integer products;
+                                   one launch; `slices` is the superblock
+                                   columns per item; `units` counts
                                    (128-row tile, superblock column) items, in
                                    whole-tile or equal ranges (cut tiles are
                                    finished from pieces in the stream's

@@ -1,5 +1,5 @@
-"""Parity of the one-vector integer tensor-core GEMV (q4k_gemv with m = 1 on
-tall matrices, Q4K_KERNEL_I8) with the CPU oracle, on a B200.
+"""Parity of the integer tensor-core GEMV (q4k_gemv with m = 1..4 on tall
+matrices, Q4K_KERNEL_I8) with the CPU oracle, on a B200.
 
 Bound: |y_gpu - y_ref| <= 1e-4 * sum|w x| + 1e-6 per element (y_ref in double),
 as for every q4k_gemv path. The cases here are the ones its number format and
@@ -9,6 +9,9 @@ huge, subnormal and zero blocks, non-finite values); CTAs own whole 128-row
 tiles (a ragged last tile, one and several superblock columns per tile, an odd
 column count, the largest K whose digit image fits shared memory); each
 item's sums are split between two epilogue warps and added at the tile's end.
+Two to four vectors share each decoded superblock (base-256 digits of every
+vector in one MMA operand, vector 3 unused for m = 3); each epilogue warp sums
+its own vectors, and cut tiles publish a piece per vector.
 """
 import numpy as np
 import pytest
@@ -33,9 +36,11 @@ def dev(a):
 
 
 def gpu_gemv(q4k, w, x, n, k):
-    assert q4k.q4k_gemv_plan_for(1, n, k, 148)["kernel"] == q4k.Q4K_KERNEL_I8
-    y = torch.full((1, n), float("nan"), dtype=torch.float32, device="cuda")
-    q4k.q4k_gemv(dev(w), dev(np.asarray(x, np.float32).reshape(1, k)), y, 1, n, k)
+    x = np.asarray(x, np.float32).reshape(-1, k)
+    m = x.shape[0]
+    assert q4k.q4k_gemv_plan_for(m, n, k, 148)["kernel"] == q4k.Q4K_KERNEL_I8
+    y = torch.full((m, n), float("nan"), dtype=torch.float32, device="cuda")
+    q4k.q4k_gemv(dev(w), dev(x), y, m, n, k)
     torch.cuda.synchronize()
     return y.cpu().numpy()
 
@@ -225,6 +230,132 @@ def test_i8_graph_capture_and_two_streams(q4k):
     assert torch.equal(y2.view(torch.int32), eager.view(torch.int32))
     yref, a = oracle.gemv(w, x, n, k, nthreads=8)
     assert_gemv_close(eager.cpu().numpy(), yref, a, "eager")
+
+
+# ------------------------------------------------------------ 2 to 4 vectors
+
+@pytest.mark.parametrize("m", [2, 3, 4])
+@pytest.mark.parametrize("n,k", [(296 * 128 - 51, 512), (11008, 4096), (4096 + 77, 8192), (3000, 15872),
+                                 (20000, 2304)])
+def test_i8_vectors_ragged_and_cut_tiles(q4k, n, k, m):
+    """Whole tiles with a ragged last one; tiles cut between CTAs with a piece
+    per vector; 62 superblock columns; an odd 9 (two columns per item for two
+    vectors, the padded column skipped). Identical bits on a second call."""
+    w, x = q4k_synth.q4k_problem(n, k, m, n % 1000 + k + m)
+    y = gpu_gemv(q4k, w, x, n, k)
+    y2 = gpu_gemv(q4k, w, x, n, k)
+    assert np.array_equal(y.view(np.uint32), y2.view(np.uint32))
+    yref, a = oracle.gemv(w, x, n, k, nthreads=8)
+    assert_gemv_close(y, yref, a, f"{n}x{k} m={m}")
+
+
+@pytest.mark.parametrize("m", [3, 4])
+def test_i8_vectors_dynamic_range(q4k, m):
+    """Each vector its own scales: one at 1e-30, one at 1e30, one with a
+    subnormal block, a zero block and a 2^20 outlier; the last one unchanged."""
+    n, k = 296 * 128, 2048
+    w, x = q4k_synth.q4k_problem(n, k, m, 78)
+    x = x.reshape(m, k).copy()
+    x[0] *= np.float32(1e-30)
+    x[1] *= np.float32(1e30)
+    x[2, 512:768] = (np.arange(256, dtype=np.float32) - 128) * np.float32(1e-43)
+    x[2, 768:1024] = 0.0
+    x[2, 1024 + 17] = np.float32(2.0 ** 20)
+    y = gpu_gemv(q4k, w, x, n, k)
+    yref, a = oracle.gemv(w, x, n, k, nthreads=8)
+    assert_gemv_close(y, yref, a, f"dynamic range m={m}")
+
+
+@pytest.mark.parametrize("m", [2, 4])
+def test_i8_vectors_unit_columns(q4k, m):
+    """x_v = e_(t_v): every y_v is the f32 dequantised column t_v, bit for bit
+    (the unit scales to 2^29, one base-256 digit 32)."""
+    n, k = 296 * 128 - 3, 2048
+    w, _ = q4k_synth.q4k_problem(n, k, 1, 33)
+    ts = [0, 255, 256 + 100, 2047][:m]
+    x = np.zeros((m, k), np.float32)
+    for v, t in enumerate(ts):
+        x[v, t] = 1.0
+    y = gpu_gemv(q4k, w, x, n, k)
+    deq = oracle.dequant_f32(w, n, k).reshape(n, k)
+    for v, t in enumerate(ts):
+        assert np.array_equal(y[v].view(np.uint32), deq[:, t].copy().view(np.uint32)), (v, t)
+
+
+def test_i8_vectors_non_finite_stays_in_its_vector(q4k):
+    """A NaN in vector 1 makes all of y_1 NaN and leaves the others exact to
+    the bound."""
+    n, k, m = 11008, 4096, 4
+    w, x = q4k_synth.q4k_problem(n, k, m, 6)
+    x = x.reshape(m, k).copy()
+    x[1, 3000] = np.nan
+    y = gpu_gemv(q4k, w, x, n, k)
+    assert np.isnan(y[1]).all()
+    keep = [0, 2, 3]
+    yref, a = oracle.gemv(w, x[keep], n, k, nthreads=8)
+    assert_gemv_close(y[keep], yref, a, "other vectors")
+
+
+def test_i8_vectors_rows_only(q4k):
+    """Nothing outside y's m x n floats is written."""
+    n, k, m = 4096, 14336, 3
+    w, x = q4k_synth.q4k_problem(n, k, m, 10)
+    wt, xt = dev(w), dev(x.reshape(m, k))
+    guard = 64
+    buf = torch.full((m * n + 2 * guard,), 7.0, dtype=torch.float32, device="cuda")
+    y = buf[guard:guard + m * n].view(m, n)
+    q4k.q4k_gemv(wt, xt, y, m, n, k)
+    torch.cuda.synchronize()
+    assert (buf[:guard] == 7.0).all() and (buf[guard + m * n:] == 7.0).all()
+    rows = sampled(n, 60, 4)
+    yref, a = oracle.gemv_rows(w, x, n, k, rows)
+    assert_gemv_close(y.cpu().numpy()[:, rows], yref, a, "rows m=3")
+
+
+@pytest.mark.parametrize("m", [2, 4])
+def test_i8_vectors_lm_head_sampled(q4k, m):
+    """The 128256 x 4096 LM head with two and four vectors; 100 sampled rows."""
+    n, k = 128256, 4096
+    w, x = q4k_synth.q4k_problem(n, k, m, 12 + m)
+    y = gpu_gemv(q4k, w, x, n, k)
+    rows = sampled(n, 100, 7)
+    yref, a = oracle.gemv_rows(w, x, n, k, rows)
+    assert_gemv_close(y[:, rows], yref, a, f"LM head m={m}")
+
+
+def test_i8_vectors_graph_capture_and_two_streams(q4k):
+    """Four vectors on cut tiles: graph replays and two concurrent streams give
+    the eager bits (each stream's piece scratch holds four vectors)."""
+    n, k, m = 11008, 4096, 4
+    w, x = q4k_synth.q4k_problem(n, k, m, 18)
+    wt, xt = dev(w), dev(x.reshape(m, k))
+    eager = torch.empty((m, n), dtype=torch.float32, device="cuda")
+    q4k.q4k_gemv(wt, xt, eager, m, n, k)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    y = torch.full((m, n), float("nan"), device="cuda")
+    with torch.cuda.stream(s):
+        q4k.q4k_gemv(wt, xt, y, m, n, k, stream=s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        q4k.q4k_gemv(wt, xt, y, m, n, k, stream=s)
+    y.fill_(float("nan"))
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int32), eager.view(torch.int32))
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    y1 = torch.full((m, n), float("nan"), device="cuda")
+    y2 = torch.full((m, n), float("nan"), device="cuda")
+    with torch.cuda.stream(s1):
+        q4k.q4k_gemv(wt, xt, y1, m, n, k, stream=s1)
+    with torch.cuda.stream(s2):
+        q4k.q4k_gemv(wt, xt, y2, m, n, k, stream=s2)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int32), eager.view(torch.int32))
+    assert torch.equal(y2.view(torch.int32), eager.view(torch.int32))
+    del g
 
 
 def test_i8_no_fault_flags(q4k):

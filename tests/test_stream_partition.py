@@ -250,7 +250,12 @@ def test_tc_balanced_items():
 @pytest.mark.parametrize("n,k", SHAPES)
 @pytest.mark.parametrize("m", [3, 4, 8, 9, 16, 17, 64])
 def test_tc_plan(m, n, k):
-    check_tc_plan(m, n, k)
+    """Three or more vectors: the tensor-core kernel, except three or four on a
+    shape the integer kernel takes."""
+    if i8_expected(m, n, k):
+        check_i8_plan(n, k, m)
+    else:
+        check_tc_plan(m, n, k)
 
 
 def i8_whole(tiles):
@@ -258,26 +263,33 @@ def i8_whole(tiles):
     return tiles >= SM_COUNT and busiest * SM_COUNT * 8 <= tiles * 9
 
 
-def i8_config(n, k):
-    """The integer kernel's launch for one vector of an n x k matrix, or None:
-    whole tiles per CTA (at least one 128-row tile per SM, the busiest CTA at
-    most 1/8 above the mean) or at least 5 superblock columns per CTA on
-    average; items of two superblock columns (padded at the end of a tile for
-    an odd K/256 >= 9) where four two-column weight stages fit beside the
-    CTA's digit-image slots (2 KB image + 80 B metadata per column, 8 x 2 KB of
-    header ring), else one column with 8, 6 or 4 stages."""
+def i8_config(n, k, m=1):
+    """The integer kernel's launch for m <= 4 vectors of an n x k matrix (m = 3
+    as four), or None: whole tiles per CTA (at least one 128-row tile per SM,
+    the busiest CTA at most 1/8 above the mean) or at least 5 superblock
+    columns per CTA on average; items of two superblock columns (padded at the
+    end of a tile for an odd K/256 >= 9; never for four vectors, whose
+    accumulators leave tensor memory for one) where four two-column weight
+    stages fit beside the CTA's digit-image slots (an image of N x 256 bytes,
+    N = 8 for one vector and 4 per vector otherwise, + 80 B of metadata per
+    vector and column; 8 x 2 KB of header ring), else one column with 8, 6 or
+    4 stages."""
+    if not 1 <= m <= 4:
+        return None
+    mv = 1 if m == 1 else 2 if m == 2 else 4
+    image, meta = (8 if mv == 1 else 4 * mv) * 256, 80 * mv
     tiles, nsb = -(-n // 128), k // 256
     whole = i8_whole(tiles)
     if not whole and tiles * nsb < 5 * SM_COUNT:
         return None
     barriers = 2 * 8 + 4 + 2 * 4 + 2 * 8 + 1
-    for cpi in ([2, 1] if nsb % 2 == 0 or nsb >= 9 else [1]):
+    for cpi in ([2, 1] if mv < 4 and (nsb % 2 == 0 or nsb >= 9) else [1]):
         npi = -(-nsb // cpi)
         items = tiles * npi
         ctas = SM_COUNT if whole else min(items, SM_COUNT)
         per = -(-tiles // ctas) * npi if whole else -(-items // ctas)
         ncols = min(per * cpi, npi * cpi)
-        off = -(-(ncols * (2048 + 80) + 8 * 2048) // 1024) * 1024
+        off = -(-(ncols * (image + meta) + 8 * 2048) // 1024) * 1024
         fit = (220 * 1024 - 1024 - off - barriers * 8 - 16) // (cpi * 128 * 144)
         if fit < 4:
             continue
@@ -289,16 +301,16 @@ def i8_config(n, k):
 
 
 def i8_expected(m, n, k):
-    return m == 1 and i8_config(n, k) is not None
+    return i8_config(n, k, m) is not None
 
 
-def check_i8_plan(n, k):
+def check_i8_plan(n, k, m=1):
     """One persistent CTA per SM at most over equal contiguous ranges of whole
     tiles or of items; 18 warps; the plan's smem, stages and per-CTA share as
     the launch rule above gives them."""
-    p = q4k.q4k_gemv_plan_for(1, n, k, SM_COUNT)
+    p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
     assert p["kernel"] == q4k.Q4K_KERNEL_I8, p
-    c = i8_config(n, k)
+    c = i8_config(n, k, m)
     tiles, nsb = -(-n // 128), k // 256
     assert p["grid"] == c["ctas"] and p["block"] == 18 * 32 and p["cluster"] == 1 and p["launches"] == 1
     assert p["slices"] == c["cpi"] and p["depth"] == c["ws"] and p["smem_bytes"] == c["smem"] <= 220 * 1024
@@ -321,13 +333,13 @@ def check_i8_plan(n, k):
                                           (160 * 128, 4096), (128256, 15872), (128256, 16128),
                                           (3000, 15872), (4096 + 77, 8192), (2048, 8192), (4096, 28672),
                                           (5000, 11008), (151553, 256), (8192, 28672), (18944, 15872)])
-@pytest.mark.parametrize("m", [1, 2])
+@pytest.mark.parametrize("m", [1, 2, 3, 4, 5])
 def test_i8_choice(m, n, k):
-    """One vector runs on the integer tensor-core kernel where it pays; any
-    other shape keeps its streaming / batched plan."""
+    """Up to four vectors run on the integer tensor-core kernel where it pays;
+    any other shape (or m) keeps its streaming / batched plan."""
     p = q4k.q4k_gemv_plan_for(m, n, k, SM_COUNT)
     if i8_expected(m, n, k):
-        check_i8_plan(n, k)
+        check_i8_plan(n, k, m)
     else:
         assert p["kernel"] != q4k.Q4K_KERNEL_I8, (m, n, k, p)
 
@@ -346,6 +358,11 @@ def test_lm_head_partition():
     """The LM head (1002 tiles): 7 tiles on 114 CTAs, 6 on the other 34."""
     p = check_i8_plan(128256, 4096)
     assert p["units_per_cta_max"] == 7 * 16 and p["depth"] == 4 and p["slices"] == 2   # four stages of two columns
+    # two vectors: the same items; four: one column per item, six stages beside a 70 KB image
+    p = check_i8_plan(128256, 4096, 2)
+    assert p["depth"] == 4 and p["slices"] == 2
+    p = check_i8_plan(128256, 4096, 4)
+    assert p["units_per_cta_max"] == 7 * 16 and p["depth"] == 6 and p["slices"] == 1
     # beyond the digit image's K the tall matrix streams with two-slice lanes
     p = check_plan(1, 128256, 20480)
     assert p["kernel"] == q4k.Q4K_KERNEL_STREAM and p["slices"] == 2
@@ -362,7 +379,10 @@ def test_cluster_choice(n, k, cluster):
 
 def test_kernel_choice():
     assert q4k.q4k_gemv_plan_for(1, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
-    assert q4k.q4k_gemv_plan_for(2, 4096, 14336, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
+    assert q4k.q4k_gemv_plan_for(2, 4096, 4096, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_STREAM
+    # two to four vectors on the larger projections: the integer kernel (W read once)
+    for m in (2, 3, 4):
+        assert q4k.q4k_gemv_plan_for(m, 4096, 14336, SM_COUNT)["kernel"] == q4k.Q4K_KERNEL_I8, m
     # three or more vectors: the tensor-core kernel (digits + GEMV per 16 vectors)
     for m, n, k in [(3, 4096, 4096), (8, 4096, 14336), (8, 14336, 4096), (5, 4096, 4096),
                     (16, 128256, 4096), (3, 64, 61696)]:
