@@ -326,19 +326,26 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* ptr, unsigned
     return old;
 }
 
-// The `nthreads` publishing threads (the epilogue's first half for one
-// vector, thread = row; every epilogue warp for several, each with its row
-// and vector) publish the CTA's piece of tile t (slot 0: the tile its range
-// starts in, slot 1: the one it ends in; the totals of its mv vectors are
-// already stored) and, if it is the tile's last piece, finish the tile: add
-// the pieces of the CTAs holding part of it, in CTA order, and store y for
-// the thread's vectors v0, v0 + vstep, ... < v1. The leader thread takes the
-// counter.
+// The publishing threads (the epilogue's first half for one vector, thread =
+// row; every epilogue warp for several, each with its row and vectors) publish
+// the CTA's piece of tile t (slot 0: the tile its range starts in, slot 1: the
+// one it ends in; the totals of its MV vectors are already stored) and, if it
+// is the tile's last piece, finish the tile: add the pieces of the CTAs
+// holding part of it, in CTA order, and store y for the thread's vectors v0,
+// v0 + 2, ... < v1 (vector 0 for one). The leader thread takes the counter.
 // (Out of line: it runs at most twice per CTA, and inlined its registers would
 // spill those of the epilogue loop.)
-__device__ __noinline__ void i8_publish_piece(const double* part, unsigned* done, float* y, int n, int mv, int v0,
-                                              int v1, int vstep, int npi, long long items, int t, int row,
-                                              bool leader, int nthreads, int* last_flag, bool aborted) {
+template <int MV>
+__device__ __noinline__ void i8_publish_piece(const double* part, unsigned* done, float* y, int n, int v0, int v1,
+                                              int npi, long long items, int t, int row, bool leader, int* last_flag,
+                                              bool aborted) {
+    // one vector: the epilogue's first half; several: every epilogue warp
+    constexpr unsigned nthreads = MV == 1 ? kI8Rows : 32 * kI8EpiWarps;
+    constexpr int vstep = MV == 1 ? 1 : 2;
+    if constexpr (MV == 1) {
+        v0 = 0;
+        v1 = 1;
+    }
     named_barrier_sync(kI8PieceBarrier, nthreads);   // every row's total is stored
     const long long tf0 = static_cast<long long>(t) * npi;
     const int c_first = i8_item_owner(items, tf0, gridDim.x);
@@ -366,7 +373,7 @@ __device__ __noinline__ void i8_publish_piece(const double* part, unsigned* done
             for (int j = 0; j < 4; ++j) {
                 const int c = c0 + j;
                 const int cs = c == c_first ? first_slot : 0;
-                val[j] = c <= c_last ? __ldcg(part + ((static_cast<size_t>(c) * 2 + cs) * mv + v) * kI8Rows + row)
+                val[j] = c <= c_last ? __ldcg(part + ((static_cast<size_t>(c) * 2 + cs) * MV + v) * kI8Rows + row)
                                      : 0.0;
             }
 #pragma unroll
@@ -702,12 +709,8 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         // a piece of tile t is published by half 0 (one vector: every vector's
         // row total is there) or by every epilogue warp (its vector)
         auto publish = [&](int t, int* flag) {
-            if constexpr (MV == 1)
-                i8_publish_piece(p.part, p.done, p.y, p.n, 1, 0, p.m, 1, npi, items, t, row, row == 0, kI8Rows, flag,
+            i8_publish_piece<MV>(p.part, p.done, p.y, p.n, eg, p.m, npi, items, t, row, row == 0 && eg == 0, flag,
                                  abort_flag != 0);
-            else
-                i8_publish_piece(p.part, p.done, p.y, p.n, MV, eg, p.m, kVStep, npi, items, t, row,
-                                 row == 0 && eg == 0, 32 * kI8EpiWarps, flag, abort_flag != 0);
         };
         double ytot[kVW];
 #pragma unroll
