@@ -358,5 +358,22 @@ def test_i8_vectors_graph_capture_and_two_streams(q4k):
     del g
 
 
+@pytest.mark.parametrize("m,k,depth,cpi", [(2, 256, 8, 1), (2, 1792, 8, 1), (2, 6912, 6, 1), (2, 11264, 4, 1),
+                                           (1, 7168, 6, 1), (3, 5632, 4, 1), (4, 3584, 6, 1)])
+def test_i8_every_instantiation(q4k, m, k, depth, cpi):
+    """One whole 128-row tile per CTA (N = 148 * 128) with the digit image
+    growing with K: each ring depth / items-of-one-column variant of the
+    kernel the launch rule picks, checked on the first and last tiles and
+    sampled rows."""
+    n = 148 * 128
+    p = q4k.q4k_gemv_plan_for(m, n, k, 148)
+    assert p["kernel"] == q4k.Q4K_KERNEL_I8 and p["depth"] == depth and p["slices"] == cpi, p
+    w, x = q4k_synth.q4k_problem(n, k, m, k + m)
+    y = gpu_gemv(q4k, w, x, n, k)
+    rows = np.unique(np.concatenate([np.arange(128), np.arange(n - 128, n), sampled(n, 80, k)]))
+    yref, a = oracle.gemv_rows(w, x, n, k, rows)
+    assert_gemv_close(y[:, rows], yref, a, f"{n}x{k} m={m}")
+
+
 def test_i8_no_fault_flags(q4k):
     assert q4k.q4k_device_fault_flags() == 0
