@@ -1,7 +1,8 @@
-// q4k_gemv_i8.cu -- y = W x for Q4_K W and one f32 vector (the pages'
-// `Q4KGemv`, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs": the LM
-// head and the larger projections of a decode step), on the tcgen05
-// tensor cores with 8-bit integer operands. Every product is formed exactly
+// q4k_gemv_i8.cu -- y = W x for Q4_K W and one to four f32 vectors (the
+// pages' `Q4KGemv`, "realizar 0.8.5, src/cuda/executor/q4k_gemv_cached.rs",
+// and the small batches of `BatchedQ4KGemv`: the LM head and the larger
+// projections of a decode step), on the tcgen05 tensor cores with 8-bit
+// integer operands. Every product is formed exactly
 // in integers; only the final combination and the output rounding are inexact.
 //
 // * Weights. Weight t of superblock b of a row is d*sc_j*q_t - dmin*m_j
@@ -47,9 +48,10 @@
 //   buffers and hand each row's superblock headers on through a shared-memory
 //   ring; one elected lane of the MMA warp issues the item's 8 MMAs per column
 //   into one of the accumulators; eight epilogue warps (two per lane quarter:
-//   a column each, or four sub-blocks each with one column per item) read the
-//   accumulator (tcgen05.ld) and combine it. The digit image of the vector's
-//   blocks the CTA needs stays in shared memory for the kernel.
+//   for one vector a column each, or four sub-blocks each with one column per
+//   item; for several, vectors h and h + 2 each) read the accumulator
+//   (tcgen05.ld) and combine it. The digit image of the vectors' blocks the
+//   CTA needs stays in shared memory for the kernel.
 //
 // All waits are bounded: one that gives up raises Q4K_FAULT_COPY_TIMEOUT and
 // the CTA lets its copies and MMAs complete (bounded) before it releases shared
@@ -706,8 +708,8 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
         constexpr int kVStep = 2;
         const int row = 32 * quarter + lane;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * quarter) << 16);
-        // a piece of tile t is published by half 0 (one vector: every vector's
-        // row total is there) or by every epilogue warp (its vector)
+        // a piece of tile t is published by half 0 (one vector: the row's
+        // total is there) or by every epilogue warp (its vectors)
         auto publish = [&](int t, int* flag) {
             i8_publish_piece<MV>(p.part, p.done, p.y, p.n, eg, p.m, npi, items, t, row, row == 0 && eg == 0, flag,
                                  abort_flag != 0);
