@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -80,14 +81,23 @@ GEMV_SOURCES = ("q4k_gemv_stream.cu", "q4k_stream.h", "q4k_gemv.cu", "q4k_sm100.
                 "q4k_tcgen05.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and blank-line / trailing-space
+    differences (string literals in these files hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def source_digest() -> str:
-    """Hash of the GEMV kernel sources (the files the sweep's launches are built
-    from), to tell whether committed ncu counters still apply."""
+    """Hash of the code of the GEMV kernel sources (the files the sweep's
+    launches are built from; comments ignored), to tell whether committed ncu
+    counters still apply."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gguf_quant_dequant_q4k_b200", "csrc")
     for name in GEMV_SOURCES:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
