@@ -115,7 +115,7 @@ void launch_rows(const q4k_gemv_plan& plan, const void* w, const void* w2, const
 namespace {
 
 // Vectors per streaming launch: 1 or 2 (q4k_gemv runs m >= 3 on the
-// tensor-core kernel); the fused SwiGLU runs any m as pairs.
+// tensor-core kernels); the fused SwiGLU runs any m as pairs.
 int group_size(int m) { return m <= 2 ? m : 2; }
 
 // K split into the fewest equal chunks (whole superblocks) one team covers:
@@ -135,12 +135,14 @@ KChunks k_chunks(int mk, int nsb) {
 
 }  // namespace
 
-// m >= 3 vectors (plain projection): the tensor-core kernel, one pair of
-// launches (digits, GEMV) per group of up to 16 vectors.
+// m >= 3 vectors (plain projection) where the integer kernel does not take
+// them: the tensor-core batched kernel, one pair of launches (digits, GEMV)
+// per group of up to 16 vectors.
 bool use_tc(int m, bool fused) { return !fused && m >= kTcMinM; }
 
-// One vector (plain projection, K within the digit image): the integer
-// tensor-core kernel, one launch.
+// One to four vectors (plain projection) on a matrix whose tiles or items give
+// every SM enough work, the digit image beside four weight stages: the
+// integer tensor-core kernel, one launch (checked before use_tc).
 bool use_i8(int m, int n, int k, int num_sms, int max_smem, bool fused) {
     I8Config c;
     return !fused && i8_config(m, n, k, num_sms, max_smem, &c);
