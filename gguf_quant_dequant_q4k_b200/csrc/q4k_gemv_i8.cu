@@ -870,10 +870,16 @@ bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg) {
     const int nsb = k / kQK;
     const long long tiles = (static_cast<long long>(n) + kI8Rows - 1) / kI8Rows;
     if (tiles * nsb >= (1LL << 31) / num_sms) return false;   // item counts in 32 bits
-    const bool whole = i8_whole_tiles(static_cast<int>(tiles), num_sms);
+    bool whole = i8_whole_tiles(static_cast<int>(tiles), num_sms);
     // whole tiles per CTA, or enough (tile, column) units per CTA that the
     // kernel's fixed cost (digit image, pipeline fill, cut tiles) pays off
     if (!whole && tiles * nsb < static_cast<long long>(kI8MinItemsPerCta) * num_sms) return false;
+    // fewer tiles than SMs: one whole tile per CTA on `tiles` CTAs where the
+    // columns that adds to the busiest CTA (nsb * (1 - tiles / SMs) against
+    // an equal split) cost less than publishing and finishing cut tiles
+    if (!whole && tiles < num_sms &&
+        static_cast<long long>(nsb) * (num_sms - tiles) <= static_cast<long long>(i8_whole_extra_cols(mv)) * num_sms)
+        whole = true;
     const int budget = max_smem < kI8SmemBudget ? max_smem : kI8SmemBudget;
     // two columns per item unless an odd K/256 is small (the padded column of
     // each tile's last item would be a large share of the work) or four
@@ -885,7 +891,7 @@ bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg) {
         c.npi = (nsb + cpi - 1) / cpi;
         c.items = tiles * c.npi;
         c.whole = whole ? 1 : 0;
-        c.ctas = whole ? num_sms : static_cast<int>(c.items < num_sms ? c.items : num_sms);
+        c.ctas = static_cast<int>(whole ? (tiles < num_sms ? tiles : num_sms) : (c.items < num_sms ? c.items : num_sms));
         c.items_per_cta_max = whole ? (tiles + c.ctas - 1) / c.ctas * c.npi : (c.items + c.ctas - 1) / c.ctas;
         const long long pnsb = static_cast<long long>(c.npi) * cpi;
         c.ncols = static_cast<int>(c.items_per_cta_max * cpi < pnsb ? c.items_per_cta_max * cpi : pnsb);

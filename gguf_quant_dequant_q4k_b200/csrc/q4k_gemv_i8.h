@@ -16,6 +16,11 @@ constexpr int kI8PreStages = 2;   // weight stages requested before the dependen
 constexpr int kI8SmemBudget = 220 * 1024;   // dynamic shared memory a CTA may use
 constexpr int kI8MaxImbalance = 8;   // whole tiles per CTA: the busiest CTA at most 1/8 above the mean
 constexpr int kI8MinItemsPerCta = 5; // cut tiles: at least this many items per CTA on average
+// Fewer tiles than SMs: one whole tile per CTA if that adds at most this many
+// superblock columns to the busiest CTA (against equal item ranges), by
+// vectors per launch: measured, cut tiles' publication is worth ~3 us, i.e.
+// ~7 / 5 / 3 columns of one / two / four vectors.
+constexpr int i8_whole_extra_cols(int mv) { return mv == 1 ? 7 : mv == 2 ? 5 : 3; }
 
 // One call's launch shape on the kernel.
 struct I8Config {
@@ -33,13 +38,15 @@ struct I8Config {
 };
 
 // Whole 128-row tiles per CTA: at least one tile per SM and the busiest CTA
-// at most 1/kI8MaxImbalance above the mean.
+// at most 1/kI8MaxImbalance above the mean (i8_config also takes one tile per
+// CTA on fewer CTAs than SMs, per i8_whole_extra_cols).
 bool i8_whole_tiles(int tiles, int num_sms);
 int i8_threads();
 // True (and *cfg filled) if q4k_gemv runs m <= kI8MaxM vectors of this shape
 // on the kernel: whole tiles per CTA or at least kI8MinItemsPerCta superblock
 // columns per CTA on average, and the CTA's digit image beside at least four
-// weight stages (two columns per item where that fits, else one).
+// weight stages (two columns per item where that fits, else one). Whole tiles
+// run on min(tiles, SMs) CTAs.
 bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg);
 
 int i8_set_attributes();

@@ -282,11 +282,15 @@ def i8_config(n, k, m=1):
     whole = i8_whole(tiles)
     if not whole and tiles * nsb < 5 * SM_COUNT:
         return None
+    # fewer tiles than SMs: one whole tile per CTA where that adds at most
+    # 7 / 5 / 3 superblock columns (one / two / four vectors) to the busiest CTA
+    if not whole and tiles < SM_COUNT and nsb * (SM_COUNT - tiles) <= {1: 7, 2: 5, 4: 3}[mv] * SM_COUNT:
+        whole = True
     barriers = 2 * 8 + 4 + 2 * 4 + 2 * 8 + 1
     for cpi in ([2, 1] if mv < 4 and (nsb % 2 == 0 or nsb >= 9) else [1]):
         npi = -(-nsb // cpi)
         items = tiles * npi
-        ctas = SM_COUNT if whole else min(items, SM_COUNT)
+        ctas = min(tiles, SM_COUNT) if whole else min(items, SM_COUNT)
         per = -(-tiles // ctas) * npi if whole else -(-items // ctas)
         ncols = min(per * cpi, npi * cpi)
         off = -(-(ncols * (image + meta) + 8 * 2048) // 1024) * 1024
@@ -342,6 +346,19 @@ def test_i8_choice(m, n, k):
         check_i8_plan(n, k, m)
     else:
         assert p["kernel"] != q4k.Q4K_KERNEL_I8, (m, n, k, p)
+
+
+def test_i8_few_tiles_whole():
+    """The 8B/7B FFN up projections (112 / 86 tiles): one whole tile per CTA on
+    112 / 86 CTAs for one vector; two vectors keep it for 112 tiles only, four
+    for neither (their columns cost more than the cut tiles' publication)."""
+    for m, n, whole_ctas in [(1, 14336, 112), (1, 11008, 86), (2, 14336, 112), (2, 11008, None),
+                             (4, 14336, None), (4, 11008, None)]:
+        p = check_i8_plan(n, 4096, m)
+        if whole_ctas:
+            assert p["grid"] == whole_ctas and p["units_per_cta_max"] == 16, (m, n, p)
+        else:
+            assert p["grid"] == SM_COUNT, (m, n, p)
 
 
 def test_i8_sweep_choice():
