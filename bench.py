@@ -330,6 +330,55 @@ def extra_workloads(q4k, torch, dev, stream, l2: int) -> dict:
                              "gbs": round(total / us / 1e3, 1),
                              "how": "one CUDA graph of the 224 projection GEMVs, replayed"}
     del g
+    # The same weights as a decode step reads them: k and v take q's input and
+    # up takes gate's, and those three calls pass Q4K_GEMV_X_READY (their x
+    # is final before the preceding call starts), so their x loads overlap
+    # the preceding kernel's tail.
+    shared_from = {1: 0, 2: 0, 5: 4}   # projection -> projection whose x it reads
+    per_layer = len(q4k_synth.LAYER_8B)
+    def one_pass_x_ready():
+        for idx, (w, x, y, n, k) in enumerate(layers):
+            proj = idx % per_layer
+            if proj in shared_from:
+                x = layers[idx - proj + shared_from[proj]][1]
+            q4k.q4k_gemv(w, x, y, 1, n, k, stream=stream, x_ready=proj in shared_from)
+    with torch.cuda.stream(stream):
+        one_pass_x_ready()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        one_pass_x_ready()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    a0 = torch.cuda.Event(enable_timing=True)
+    a1 = torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g.replay()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = a0.elapsed_time(a1) * 1e3 / reps
+    out["layer_sweep_32_x_ready"] = {
+        "launches": len(layers), "bytes": total, "us_per_pass": round(us, 1), "gbs": round(total / us / 1e3, 1),
+        "how": "the same 224 GEMVs, k / v reading q's input and up reading gate's, those calls with "
+               "Q4K_GEMV_X_READY"}
+    del g
+    # Per call with Q4K_GEMV_X_READY (back-to-back calls of one projection on a
+    # constant x, rotating weight copies as in per_shape).
+    out["x_ready_per_call"] = []
+    for n, k in SWEEP:
+        w, x = q4k_synth.q4k_problem(n, k, 1, q4k_synth.SEEDS[(n, k)])
+        wd = torch.from_numpy(w).to(dev)
+        ws = [wd] + [wd.clone() for _ in range(max(2, -(-2 * l2 // w.nbytes) + 1) - 1)]
+        xd = torch.from_numpy(x).to(dev)
+        y = torch.empty((1, n), dtype=torch.float32, device=dev)
+        us = device_us_per_call(
+            torch, dev, stream,
+            lambda i: q4k.q4k_gemv(ws[i % len(ws)], xd, y, 1, n, k, stream=stream, x_ready=True))
+        out["x_ready_per_call"].append({"n": n, "k": k, "us_per_call": round(us, 3)})
+        del ws, wd
     # The same weights with each layer's gate and up projections as one fused
     # SwiGLU call (q4k_gemv_swiglu): 6 launches per layer, same bytes.
     gate_i, up_i = 4, 5

@@ -9,7 +9,8 @@ not built: there is no CPU path.
 from .capi import (  # noqa: F401
     EXPORTS, Q4K_BLOCK_BYTES, Q4K_GEMM_K_MULTIPLE, Q4K_ERR_ALIGN, Q4K_ERR_CUDA, Q4K_ERR_NULL, Q4K_ERR_OVERLAP,
     Q4K_ERR_RANGE, Q4K_ERR_SHAPE, Q4K_ERR_UNSUPPORTED_M, Q4K_FAULT_COPY_TIMEOUT,
-    Q4K_FAULT_TOKEN_RANGE, Q4K_KERNEL_I8, Q4K_KERNEL_STREAM, Q4K_KERNEL_TC, Q4K_KERNEL_WARP_ROWS, Q4K_MAX_M, Q4K_OK, Q4K_QK,
+    Q4K_FAULT_TOKEN_RANGE, Q4K_GEMV_X_READY, Q4K_KERNEL_I8, Q4K_KERNEL_STREAM, Q4K_KERNEL_TC, Q4K_KERNEL_WARP_ROWS,
+    Q4K_MAX_M, Q4K_OK, Q4K_QK,
     LIB_PATH, Q4KError, q4k_dequant_f32, q4k_dequant_f32_status, q4k_device_fault_flags,
     q4k_embed_gather_f32, q4k_embed_gather_f32_status, q4k_embed_lookup_f32,
     q4k_embed_lookup_f32_status, q4k_gemv, q4k_gemv_plan_for, q4k_gemv_status,

@@ -27,6 +27,7 @@ Q4K_FAULT_TOKEN_RANGE = 2
 Q4K_QK = 256
 Q4K_BLOCK_BYTES = 144
 Q4K_MAX_M = 64
+Q4K_GEMV_X_READY = 0x1   # q4k_gemv_ex flag: x not written by the pending work on the stream
 Q4K_GEMM_K_MULTIPLE = 64
 Q4K_PREFILL_NOALLOC_MAX_ELEMS = 8388608
 Q4K_KERNEL_WARP_ROWS = 1
@@ -35,7 +36,7 @@ Q4K_KERNEL_TC = 3
 Q4K_KERNEL_I8 = 4
 
 # Every function include/q4k.h declares.
-EXPORTS = ("q4k_gemv", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
+EXPORTS = ("q4k_gemv", "q4k_gemv_ex", "q4k_dequant_f32", "q4k_weight_bytes", "q4k_status_string",
            "q4k_last_cuda_error", "q4k_gemv_plan_for", "q4k_device_fault_flags",
            "q4k_embed_lookup_f32", "q4k_embed_gather_f32", "q4k_gemv_swiglu",
            "q4k_gemv_swiglu_plan_for", "q4k_selftest_wait_timeout", "q4k_dequant_f16",
@@ -70,6 +71,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 _vp = ctypes.c_void_p
 _lib.q4k_gemv.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, _vp]
 _lib.q4k_gemv.restype = ctypes.c_int
+_lib.q4k_gemv_ex.argtypes = [_vp, _vp, _vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_uint, _vp]
+_lib.q4k_gemv_ex.restype = ctypes.c_int
 _lib.q4k_dequant_f32.argtypes = [_vp, _vp, ctypes.c_int, ctypes.c_int, _vp]
 _lib.q4k_dequant_f32.restype = ctypes.c_int
 _lib.q4k_weight_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
@@ -209,18 +212,22 @@ def q4k_device_fault_flags() -> int:
     return v.value
 
 
-def q4k_gemv_status(w, x, y, m: int, n: int, k: int, stream=None) -> int:
+def q4k_gemv_status(w, x, y, m: int, n: int, k: int, stream=None, flags: int = 0) -> int:
     """Raw status of the C call (no exception; tensor checks still raise)."""
     ok = _gemv_sizes_valid(m, n, k)
-    return _lib.q4k_gemv(_ptr(w, None, "w", _need(q4k_weight_bytes(n, k), 1, ok)),
-                         _ptr(x, "float32", "x", _need(m * k, 4, ok)),
-                         _ptr(y, "float32", "y", _need(m * n, 4, ok)), int(m), int(n),
-                         int(k), _stream(stream))
+    args = (_ptr(w, None, "w", _need(q4k_weight_bytes(n, k), 1, ok)),
+            _ptr(x, "float32", "x", _need(m * k, 4, ok)),
+            _ptr(y, "float32", "y", _need(m * n, 4, ok)), int(m), int(n), int(k))
+    if flags == 0:
+        return _lib.q4k_gemv(*args, _stream(stream))
+    return _lib.q4k_gemv_ex(*args, int(flags), _stream(stream))
 
 
-def q4k_gemv(w, x, y, m: int, n: int, k: int, stream=None) -> None:
-    """y[m, n] = W[n, k] x[m, k] on `stream` (default: torch's current stream)."""
-    st = q4k_gemv_status(w, x, y, m, n, k, stream)
+def q4k_gemv(w, x, y, m: int, n: int, k: int, stream=None, x_ready: bool = False) -> None:
+    """y[m, n] = W[n, k] x[m, k] on `stream` (default: torch's current stream).
+    x_ready: x is not written by the work still pending on `stream`
+    (Q4K_GEMV_X_READY: it may be read before that work finishes)."""
+    st = q4k_gemv_status(w, x, y, m, n, k, stream, Q4K_GEMV_X_READY if x_ready else 0)
     if st != Q4K_OK:
         raise Q4KError(st, "q4k_gemv")
 

@@ -191,7 +191,13 @@ int q4k_gemv_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {
 
 int q4k_gemv(const void* w, const float* x, float* y, int m, int n, int k,
              q4k_stream_t stream) {
+    return q4k_gemv_ex(w, x, y, m, n, k, 0u, stream);
+}
+
+int q4k_gemv_ex(const void* w, const float* x, float* y, int m, int n, int k, unsigned flags,
+                q4k_stream_t stream) {
     if (w == nullptr || x == nullptr || y == nullptr) return Q4K_ERR_NULL;
+    if ((flags & ~Q4K_GEMV_X_READY) != 0u) return Q4K_ERR_SHAPE;
     const size_t wbytes = weight_bytes_checked(n, k);
     if (wbytes == 0) return Q4K_ERR_SHAPE;
     if (m < 1 || m > Q4K_MAX_M) return Q4K_ERR_UNSUPPORTED_M;
@@ -202,7 +208,8 @@ int q4k_gemv(const void* w, const float* x, float* y, int m, int n, int k,
     DeviceInfo dev;
     int st = current_device_info(&dev);
     if (st != Q4K_OK) return st;
-    return launch_gemv(dev, w, nullptr, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream));
+    return launch_gemv(dev, w, nullptr, x, y, m, n, k, reinterpret_cast<cudaStream_t>(stream),
+                       (flags & Q4K_GEMV_X_READY) != 0u);
 }
 
 int q4k_gemv_swiglu_plan_for(int m, int n, int k, int num_sms, q4k_gemv_plan* plan) {

@@ -239,10 +239,10 @@ int plan_gemv(int m, int n, int k, int num_sms, bool fused, q4k_gemv_plan* plan)
 }
 
 int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const float* x, float* y,
-                int m, int n, int k, cudaStream_t stream) {
+                int m, int n, int k, cudaStream_t stream, bool x_ready) {
     q4k_gemv_plan plan;
     const bool fused = w2 != nullptr;
-    if (use_i8(m, n, k, dev.sm_count, dev.max_smem_optin, fused)) return launch_gemv_i8(dev, w, x, y, m, n, k, stream);
+    if (use_i8(m, n, k, dev.sm_count, dev.max_smem_optin, fused)) return launch_gemv_i8(dev, w, x, y, m, n, k, stream, x_ready);
     if (use_tc(m, fused)) return launch_gemv_tc(dev, w, x, y, m, n, k, stream);
     const int gsz = group_size(m);
     int st = plan_gemv_device(m, n, k, dev.sm_count, dev.max_smem_optin,
@@ -269,6 +269,7 @@ int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const floa
                 sp.sb_off = sb0;
                 sp.x_stride = k;
                 sp.accumulate = ci > 0 ? 1 : 0;
+                sp.x_ready = x_ready && !fused ? 1 : 0;
                 st = launch_stream(sp, g, b, sm, w, w2,
                                    x + static_cast<size_t>(i0) * k + static_cast<size_t>(sb0) * kQK,
                                    y + static_cast<size_t>(i0) * n, mk, stream);

@@ -303,6 +303,9 @@ struct I8Params {
                          // hold a column past the row (zero-filled, skipped)
     int ncols;           // digit-image slots: the CTA's columns, from its first one
     int whole;           // 1: CTAs own whole tiles (no tile is cut)
+    int x_ready;         // 1: x is not written by the preceding work: the digit image
+                         // is formed before the grid dependency resolves, and only the
+                         // epilogue (the one role writing global memory) waits for it
 };
 
 // The work is the flat sequence of items f = tile * npi + i (superblock
@@ -571,7 +574,9 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
     if (warp == kI8ProducerWarp && lane == 0) produce(count < kI8PreStages ? count : kI8PreStages);
     __syncwarp();
 
-    pdl_wait();   // x is produced, and y may be read, by the preceding work on the stream
+    // x is produced, and y and the cut-tile counters may be used, by the
+    // preceding work on the stream (x excepted when the caller says so)
+    if (!p.x_ready) pdl_wait();
     {
         const int ncols_used = count * CPI < pnsb ? count * CPI : pnsb;
         if constexpr (MV == 1)
@@ -714,6 +719,7 @@ q4k_gemv_i8_kernel(const __grid_constant__ CUtensorMap map_w, const I8Params p) 
             i8_publish_piece<MV>(p.part, p.done, p.y, p.n, eg, p.m, npi, items, t, row, row == 0 && eg == 0, flag,
                                  abort_flag != 0);
         };
+        if (p.x_ready) pdl_wait();   // before this role's first global write
         double ytot[kVW];
 #pragma unroll
         for (int vv = 0; vv < kVW; ++vv) ytot[vv] = 0.0;
@@ -1032,7 +1038,7 @@ cudaError_t launch_i8_mv(const cudaLaunchConfig_t& cfg, const I8Config& c, const
 }  // namespace
 
 int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n, int k,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, bool x_ready) {
     I8Config c;
     if (!i8_config(m, n, k, dev.sm_count, dev.max_smem_optin, &c)) return Q4K_ERR_SHAPE;   // not reached
     const int nsb = k / kQK;
@@ -1058,7 +1064,7 @@ int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* 
         }
         if (e != cudaSuccess) return cuda_failure(e);
     }
-    const I8Params ip{x, y, part, done, m, n, k, nsb, tiles, c.npi, c.ncols, c.whole};
+    const I8Params ip{x, y, part, done, m, n, k, nsb, tiles, c.npi, c.ncols, c.whole, x_ready ? 1 : 0};
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(c.ctas));
     cfg.blockDim = dim3(kI8Threads);

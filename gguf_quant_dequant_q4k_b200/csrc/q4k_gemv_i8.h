@@ -51,7 +51,7 @@ bool i8_config(int m, int n, int k, int num_sms, int max_smem, I8Config* cfg);
 
 int i8_set_attributes();
 int launch_gemv_i8(const DeviceInfo& dev, const void* w, const float* x, float* y, int m, int n, int k,
-                   cudaStream_t stream);
+                   cudaStream_t stream, bool x_ready);
 int read_i8_fault_flags(unsigned* flags);
 
 }  // namespace q4k

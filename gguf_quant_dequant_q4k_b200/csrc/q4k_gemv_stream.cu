@@ -553,7 +553,10 @@ q4k_gemv_stream_kernel(const StreamParams p) {
         const int wit = warp % p.team_warps;
         const Team T = make_team<M, FUSED>(p, smem, team);
         pdl_launch_dependents();
-        pdl_wait();   // x and y belong to the dependency chain
+        // x belongs to the dependency chain unless the caller says otherwise;
+        // these warps write only shared memory (the producer, which stores
+        // y, waits in any case)
+        if (!p.x_ready) pdl_wait();
 
         // This lane's superblock position bl and its kNX quant bytes, from
         // byte qoff of the superblock's 128: group g = qoff / 32 (sub-blocks

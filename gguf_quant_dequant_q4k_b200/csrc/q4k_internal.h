@@ -31,8 +31,10 @@ int plan_gemv(int m, int n, int k, int num_sms, bool fused, q4k_gemv_plan* plan)
 
 // Enqueue the planned kernels on the current device. Arguments are already
 // validated. w2 != null: y = silu(W x) * (W2 x) (fused gate/up SwiGLU).
+// x_ready: x is not written by the preceding work on the stream (read before
+// the grid dependency resolves; y still written after it).
 int launch_gemv(const DeviceInfo& dev, const void* w, const void* w2, const float* x, float* y,
-                int m, int n, int k, cudaStream_t stream);
+                int m, int n, int k, cudaStream_t stream, bool x_ready = false);
 
 int launch_dequant(const void* w, float* out, int n, int k, int num_sms, cudaStream_t stream);
 

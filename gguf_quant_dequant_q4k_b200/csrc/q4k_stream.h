@@ -73,6 +73,8 @@ struct StreamParams {
     // and vectors are x_stride floats apart.
     int nsb_row, sb_off, x_stride;
     int accumulate;             // 1: y += the chunk's sums (a later K-chunk); 0: y = sums
+    int x_ready;                // 1: x is not written by the preceding work: the compute
+                                // warps read it without waiting for the grid dependency
 };
 
 // Launch policy. 0: one CTA per SM with up to 20 compute warps and 220 KiB

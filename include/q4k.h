@@ -146,6 +146,31 @@ Q4K_API int q4k_gemv(const void *w, const float *x, float *y, int m, int n, int 
              q4k_stream_t stream);
 
 /*
+ * As q4k_gemv, with flags:
+ *   Q4K_GEMV_X_READY: x is already final when the kernel enqueued on
+ *     `stream` just before this call begins executing: the call may read x
+ *     before that kernel has finished (programmatic dependent launch); y is
+ *     still written only after it has. The q4k kernels let their successors
+ *     start early, so a chain of q4k calls can run partly at once: x must not
+ *     be written by any of them still pending. The typical case: x written by
+ *     a kernel that does not trigger its dependents early (or by a copy),
+ *     read by one q4k_gemv without the flag and then by further ones with it
+ *     (the k and v projections after q, up after gate). Undefined results
+ *     otherwise. Applies on the streaming and integer kernels; the batched
+ *     tensor-core kernel (m >= 3 on the smaller matrices, m > 4) ignores it.
+ * Other bits of `flags` must be zero (Q4K_ERR_SHAPE otherwise). Several GEMVs
+ * reading one input are the pages' pattern: an input vector is uploaded once
+ * and then serves a series of GEMV launches (`q4k_upload_to_input_buffer`,
+ * `q4k_gemv_launch_to_ptr`, "realizar 0.8.5,
+ * src/cuda/executor/q4k_gemv_cached.rs"), and a layer normalises its input
+ * twice, for attention and for the FFN (`preload_batched_prefill_modules`,
+ * "realizar 0.8.5, src/cuda/executor/layers/modules_utilities.rs").
+ */
+#define Q4K_GEMV_X_READY 0x1u
+Q4K_API int q4k_gemv_ex(const void *w, const float *x, float *y, int m, int n, int k, unsigned flags,
+                        q4k_stream_t stream);
+
+/*
  * Fused gate/up projection with SwiGLU: y = silu(W_gate x) * (W_up x), where
  * silu(g) = g / (1 + exp(-g)), for m vectors ("realizar 0.8.5" kernel cache
  * page: `FusedGateUpSwigluHwDp4aQ4KGemv { k: hidden_dim, n: intermediate_dim }`;

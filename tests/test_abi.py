@@ -70,6 +70,14 @@ A16 = 1 << 20  # a 16-byte-aligned fake address; never dereferenced
 ])
 def test_gemv_validation_before_any_cuda_call(args, expect):
     assert q4k.q4k_gemv_status(*args, stream=0) == expect
+    # q4k_gemv_ex with the x-ready flag validates the same way
+    assert q4k.q4k_gemv_status(*args, stream=0, flags=q4k.Q4K_GEMV_X_READY) == expect
+
+
+@pytest.mark.parametrize("flags", [0x2, 0x80000000, 0xFFFFFFFF])
+def test_gemv_ex_rejects_unknown_flags(flags):
+    """Bits other than Q4K_GEMV_X_READY are refused before any CUDA call."""
+    assert q4k.q4k_gemv_status(A16, A16 * 2, A16 * 3, 1, 4, 256, stream=0, flags=flags) == q4k.Q4K_ERR_SHAPE
 
 
 @pytest.mark.parametrize("args,expect", [

@@ -432,6 +432,70 @@ def test_gemv_small_n_cluster_split(q4k, n, k, m):
     assert_gemv_close(y, yref, a, f"{n}x{k} m={m} cluster={plan['cluster']}")
 
 
+@pytest.mark.parametrize("m,n,k", [(1, 1536, 1536), (2, 4096, 4096), (1, 64, 61696), (1, 148 * 128, 512),
+                                   (1, 4096, 14336), (2, 11008, 4096), (4, 11008, 4096), (8, 300, 2048)])
+def test_gemv_x_ready_same_bits(q4k, m, n, k):
+    """Q4K_GEMV_X_READY (x read before the preceding kernel finishes) gives
+    the plain call's bits on every path: streaming (one and two vectors,
+    K-chunks), integer kernel (whole and cut tiles, two and four vectors),
+    and the batched kernel, which ignores it."""
+    w, x = q4k_synth.q4k_problem(n, k, m, 90 + m + n % 97)
+    wt, xt = dev(w), dev(np.asarray(x, np.float32).reshape(m, k))
+    y0 = torch.full((m, n), float("nan"), device="cuda")
+    y1 = torch.full((m, n), float("nan"), device="cuda")
+    q4k.q4k_gemv(wt, xt, y0, m, n, k)
+    q4k.q4k_gemv(wt, xt, y1, m, n, k, x_ready=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int32), y1.view(torch.int32))
+    rows = np.unique(np.concatenate([[0, n - 1], np.random.default_rng(n).integers(0, n, 40)]))
+    yref, a = oracle.gemv_rows(w, x, n, k, rows)
+    assert_gemv_close(y1.cpu().numpy()[:, rows], yref, a, f"x_ready {m}x{n}x{k}")
+
+
+def test_gemv_x_ready_chain(q4k):
+    """A chain on one stream, eager and in a CUDA graph: q = Wq x; k = Wk x
+    and v = Wv x flagged (x is not written by the pending work); h = Wo q
+    unflagged (q is). Every output matches the oracle."""
+    d = 2048
+    x = q4k_synth.x_vectors(d, 1, 5)
+    mats = [q4k_synth.q4k_problem(d, d, 1, 60 + i)[0] for i in range(4)]
+    wq, wk, wv, wo = (dev(w) for w in mats)
+    xt = dev(x.reshape(1, d))
+    outs = [torch.full((1, d), float("nan"), device="cuda") for _ in range(4)]
+    s = torch.cuda.Stream()
+
+    def chain():
+        q4k.q4k_gemv(wq, xt, outs[0], 1, d, d, stream=s)
+        q4k.q4k_gemv(wk, xt, outs[1], 1, d, d, stream=s, x_ready=True)
+        q4k.q4k_gemv(wv, xt, outs[2], 1, d, d, stream=s, x_ready=True)
+        q4k.q4k_gemv(wo, outs[0], outs[3], 1, d, d, stream=s)
+
+    def check():
+        torch.cuda.synchronize()
+        got = [o.cpu().numpy() for o in outs]
+        for i, w in enumerate(mats[:3]):
+            yref, a = oracle.gemv(w, x, d, d)
+            assert_gemv_close(got[i], yref, a, f"projection {i}")
+        yref, a = oracle.gemv(mats[3], got[0], d, d)
+        assert_gemv_close(got[3], yref, a, "dependent projection")
+
+    with torch.cuda.stream(s):
+        chain()
+    check()
+    for o in outs:
+        o.fill_(float("nan"))
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        chain()
+    for o in outs:
+        o.fill_(float("nan"))
+    torch.cuda.synchronize()
+    g.replay()
+    check()
+    del g
+
+
 def test_no_kernel_fault_flags(q4k):
     """No bounded wait on a bulk copy gave up during any of the runs above."""
     assert q4k.q4k_device_fault_flags() == 0
